@@ -1,0 +1,217 @@
+"""Pins for the oracle's pooling and block selection (CPU only).
+
+Each test checks the oracle against something other than itself: a library routine,
+brute-force enumeration, a closed form or an invariant the pages fix.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (scale * torch.randn(shape, generator=g)).to(torch.bfloat16)
+
+
+# --------------------------------------------------------------------------- pool
+
+def test_pool_constant_block_is_exact():
+    b, hkv, N, d, B = 1, 2, 64, 8, 16
+    vals = torch.tensor([0.5, -1.25, 3.0, 0.0078125], dtype=torch.float32)
+    k = torch.empty(b, hkv, N, d)
+    for j in range(N // B):
+        k[:, :, j * B:(j + 1) * B, :] = vals[j]
+    kbar = oracle.pool_keys(k.to(torch.bfloat16), B)
+    for j in range(N // B):
+        assert np.all(kbar[:, :, j, :] == float(vals[j]))
+
+
+@pytest.mark.parametrize("B", [1, 2, 8, 128])
+def test_pool_matches_numpy_mean(B):
+    k = _bf16((2, 3, 256, 16), seed=1)
+    kbar = oracle.pool_keys(k, B)
+    ref = oracle.bf16_to_f64(k).reshape(2, 3, 256 // B, B, 16).mean(axis=3)
+    np.testing.assert_allclose(kbar, ref, rtol=0, atol=1e-15)
+
+
+def test_pool_rejects_ragged_block():
+    with pytest.raises(ValueError):
+        oracle.pool_keys(_bf16((1, 1, 100, 8), 0), 64)
+
+
+# ---------------------------------------------------------------------- selection
+
+def _brute_force_sets(s_row, c, k):
+    """Own block plus the (k-1)-subset of past blocks with the largest score sum."""
+    past = list(range(c))
+    if c <= k - 1:
+        return set(past) | {c}
+    best, best_sum = None, -math.inf
+    for comb in itertools.combinations(past, k - 1):
+        tot = sum(s_row[j] for j in comb)
+        if tot > best_sum:
+            best, best_sum = comb, tot
+    return set(best) | {c}
+
+
+@pytest.mark.parametrize("B", [1, 2, 8, 128])
+def test_select_matches_brute_force(B):
+    n = 8 if B < 128 else 6
+    N = n * B
+    d = 8
+    q = _bf16((1, 2, N, d), seed=10 + B)
+    k = _bf16((1, 1, N, d), seed=20 + B)
+    kbar = oracle.pool_keys(k, B)
+    # Every row of every block, all k in 1..n.
+    rows = np.arange(N, dtype=np.int32)
+    s = oracle.gate_scores(q, kbar, B, rows)
+    # Independent check of the scores: numpy inner products with the pooled keys.
+    qd = oracle.bf16_to_f64(q)
+    for h in range(2):
+        full = qd[0, h] @ kbar[0, 0].T
+        for i in range(0, N, max(1, N // 37)):
+            c = i // B
+            np.testing.assert_allclose(s[0, h, i, :c], full[i, :c], rtol=1e-13, atol=1e-13)
+            assert np.all(np.isneginf(s[0, h, i, c:]))
+    for k_ in range(1, n + 1):
+        idx, gap = oracle.select_topk(s, N, B, k_, rows)
+        for h in range(2):
+            for i in rows:
+                c = i // B
+                got = [x for x in idx[0, h, i] if x >= 0]
+                assert got == sorted(got)
+                assert len(got) == min(k_, c + 1)
+                assert list(idx[0, h, i, len(got):]) == [-1] * (k_ - len(got))
+                assert set(got) == _brute_force_sets(s[0, h, i], c, k_), (B, k_, h, i)
+
+
+def test_select_token_level_when_block_is_one():
+    """B = 1: the gate score of block j is <q_i, k_j> itself; the row keeps its own
+    token and the k-1 past tokens with the largest raw inner products."""
+    N, d, k_ = 64, 16, 5
+    q = _bf16((1, 1, N, d), 3)
+    k = _bf16((1, 1, N, d), 4)
+    s = oracle.gate_scores(q, oracle.pool_keys(k, 1), 1)
+    idx, _ = oracle.select_topk(s, N, 1, k_)
+    qd, kd = oracle.bf16_to_f64(q)[0, 0], oracle.bf16_to_f64(k)[0, 0]
+    for i in range(N):
+        raw = qd[i] @ kd[:i].T
+        order = sorted(range(i), key=lambda j: (-raw[j], j))
+        want = sorted(order[:k_ - 1] + [i])
+        assert [x for x in idx[0, 0, i] if x >= 0] == want
+
+
+def test_future_blocks_never_chosen_and_own_block_forced():
+    """A future block with a huge pooled key is never selected; the own block is
+    kept even when its pooled key scores lowest (MoBA §인과성 보존)."""
+    N, B, d = 512, 64, 4
+    n = N // B
+    q = torch.ones(1, 1, N, d)
+    k = torch.zeros(1, 1, N, d)
+    for j in range(n):
+        k[0, 0, j * B:(j + 1) * B, :] = float(j % 3) - 1.0
+    k[0, 0, 7 * B:, :] = 50.0   # last block scores highest of all
+    k[0, 0, 3 * B:4 * B, :] = -50.0  # block 3 scores lowest
+    q, k = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    s = oracle.gate_scores(q, oracle.pool_keys(k, B), B)
+    idx, _ = oracle.select_topk(s, N, B, 2)
+    for i in range(N):
+        c = i // B
+        got = [x for x in idx[0, 0, i] if x >= 0]
+        assert c in got
+        assert all(x <= c for x in got)
+    rows_in_3 = range(3 * B, 4 * B)
+    for i in rows_in_3:
+        assert 3 in idx[0, 0, i]
+
+
+def test_ties_go_to_the_lower_block():
+    N, B, d = 256, 32, 4
+    q = torch.ones(1, 1, N, d, dtype=torch.bfloat16)
+    k = torch.ones(1, 1, N, d, dtype=torch.bfloat16)  # every pooled key identical
+    s = oracle.gate_scores(q, oracle.pool_keys(k, B), B)
+    idx, gap = oracle.select_topk(s, N, B, 3)
+    for i in range(2 * B, N):
+        c = i // B
+        assert list(idx[0, 0, i]) == [0, 1, c]
+        # With c <= k-1 every past block is kept and no choice is made.
+        assert gap[0, 0, i] == (0.0 if c > 2 else np.inf)
+
+
+def test_gap_is_kth_minus_k_plus_first_past_score():
+    N, B, d = 1024, 64, 16
+    q = _bf16((1, 1, N, d), 7)
+    k = _bf16((1, 1, N, d), 8)
+    s = oracle.gate_scores(q, oracle.pool_keys(k, B), B)
+    for k_ in (1, 2, 4):
+        _, gap = oracle.select_topk(s, N, B, k_)
+        for i in range(0, N, 13):
+            c = i // B
+            if c <= k_ - 1 or k_ == 1:
+                assert gap[0, 0, i] == math.inf
+            else:
+                desc = np.sort(s[0, 0, i, :c])[::-1]
+                assert gap[0, 0, i] == desc[k_ - 2] - desc[k_ - 1]
+
+
+def test_attended_key_count_closed_form():
+    """|J_i| = (i mod B) + 1 + min(k-1, c) * B (q = 0 makes lse = ln|J|)."""
+    N, B, d, k_ = 1024, 64, 8, 4
+    q = _bf16((1, 1, N, d), 11)
+    k = _bf16((1, 1, N, d), 12)
+    v = _bf16((1, 1, N, d), 13)
+    s = oracle.gate_scores(q, oracle.pool_keys(k, B), B)
+    idx, _ = oracle.select_topk(s, N, B, k_)
+    zero_q = torch.zeros_like(q)
+    _, lse = oracle.attention(zero_q, k, v, mode=oracle.MODE_MOBA, block=B, topk=k_, idx=idx)
+    i = np.arange(N)
+    want = (i % B) + 1 + np.minimum(k_ - 1, i // B) * B
+    np.testing.assert_allclose(lse[0, 0], np.log(want), rtol=0, atol=1e-12)
+
+
+def test_sparsity_matches_the_pages_arithmetic():
+    with open(os.path.join(GOLDEN, "sparsity.json")) as f:
+        cases = json.load(f)["cases"]
+    d = 2
+    for case in cases:
+        N, B, k_ = case["N"], case["B"], case["k"]
+        q = _bf16((1, 1, N, d), 5)
+        k = _bf16((1, 1, N, d), 6)
+        v = torch.zeros_like(k)
+        last = np.array([N - 1], dtype=np.int32)
+        s = oracle.gate_scores(q, oracle.pool_keys(k, B), B, last)
+        idx, _ = oracle.select_topk(s, N, B, k_, last)
+        _, lse = oracle.attention(torch.zeros_like(q), k, v, mode=oracle.MODE_MOBA, block=B,
+                                  topk=k_, idx=idx, rows=last)
+        nkeys = round(math.exp(lse[0, 0, 0]))
+        assert nkeys == k_ * B
+        assert 1.0 - nkeys / N == pytest.approx(case["sparsity"], abs=0)
+
+
+def test_selection_invariant_under_a_common_key_shift():
+    """Adding one vector u to every key shifts every gate score of a row by <q, u>:
+    the chosen blocks do not change.  Values on a coarse grid keep k + u exact in
+    bf16."""
+    N, B, d = 512, 32, 8
+    g = torch.Generator().manual_seed(9)
+    q = (torch.randint(-16, 17, (1, 2, N, d), generator=g) / 8.0).to(torch.bfloat16)
+    k = (torch.randint(-16, 17, (1, 1, N, d), generator=g) / 8.0).to(torch.bfloat16)
+    u = (torch.randint(-8, 9, (d,), generator=g) / 2.0)
+    k2 = (k.float() + u).to(torch.bfloat16)
+    assert torch.equal(k2.float(), k.float() + u)
+    s1 = oracle.gate_scores(q, oracle.pool_keys(k, B), B)
+    s2 = oracle.gate_scores(q, oracle.pool_keys(k2, B), B)
+    i1, g1 = oracle.select_topk(s1, N, B, 4)
+    i2, g2 = oracle.select_topk(s2, N, B, 4)
+    assert np.array_equal(i1, i2)
+    finite = np.isfinite(g1)
+    np.testing.assert_allclose(g1[finite], g2[finite], atol=1e-12)

@@ -1,0 +1,113 @@
+"""Seeded synthetic inputs and named workload shapes.
+
+This module holds no step of the method: it only draws q, k, v (and nothing else)
+from seeded generators.  Both the CUDA path and the CPU oracle take their inputs from
+here, so they see the same bf16 values.
+
+Recipe: with ``torch.Generator('cpu').manual_seed(seed)`` draw q, k, v in that order
+as float32 N(0, 1) of shapes [b, hq, N, d], [b, hkv, N, d], [b, hkv, N, d]; for the
+MoBA workloads draw one offset vector per (batch, kv-head, block), N(0, 0.5^2) of
+shape [b, hkv, N/B, d], add it to every key of its block (so that the pooled keys
+separate and the gate's choices are not near-ties); cast all three to bf16.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    batch: int
+    hq: int
+    hkv: int
+    seqlen: int
+    d: int
+    block: int = 0          # MoBA block size B (0 for pure sliding-window attention)
+    topk: int = 0           # blocks kept per query, the own block included
+    window: int = 0         # causal window (0 = none)
+    key_offset_std: float = 0.0
+    sampled_rows: bool = False   # the oracle checks sampled rows only
+    note: str = ""
+
+    @property
+    def kind(self) -> str:
+        return "moba" if self.block > 0 else "swa"
+
+    @property
+    def nblocks(self) -> int:
+        return self.seqlen // self.block if self.block else 0
+
+
+# The five workloads the method is measured and checked on.
+WORKLOADS = {
+    "tiny": Workload("tiny", 1, 1, 1, 1024, 64, block=128, topk=3,
+                     note="1 head, 8 blocks of 128, top-3"),
+    "gqa32k": Workload("gqa32k", 1, 32, 8, 32768, 128, block=512, topk=3, key_offset_std=0.5,
+                       note="GQA 32 q / 8 kv heads, 64 blocks of 512, top-3"),
+    "swa16k": Workload("swa16k", 1, 32, 32, 16384, 80, window=4096,
+                       note="sliding window 4096, 32 heads, d=80"),
+    "hybrid64k": Workload("hybrid64k", 2, 8, 4, 65536, 128, block=2048, topk=16, window=512,
+                          key_offset_std=0.5, sampled_rows=True,
+                          note="GQA 8/4, 32 blocks of 2048, top-16 unioned with window 512"),
+    "moba1m": Workload("moba1m", 1, 32, 8, 1 << 20, 128, block=4096, topk=12, key_offset_std=0.5,
+                       sampled_rows=True, note="1M tokens, 256 blocks of 4096, top-12"),
+}
+
+
+def make_inputs(w: Workload, seed: int = 0, device: str = "cpu"):
+    """q [b,hq,N,d], k, v [b,hkv,N,d] as bf16 tensors on ``device`` (drawn on the CPU)."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    b, N, d = w.batch, w.seqlen, w.d
+    q = _randn_bf16((b, w.hq, N, d), g)
+    k32 = torch.randn((b, w.hkv, N, d), generator=g, dtype=torch.float32)
+    v = _randn_bf16((b, w.hkv, N, d), g)
+    if w.key_offset_std > 0:
+        off = torch.randn((b, w.hkv, N // w.block, d), generator=g, dtype=torch.float32)
+        k32 += (w.key_offset_std * off).repeat_interleave(w.block, dim=2)
+    k = k32.to(torch.bfloat16)
+    del k32
+    return q.to(device), k.to(device), v.to(device)
+
+
+def _randn_bf16(shape, g, chunk: int = 1 << 26):
+    """N(0,1) float32 draws cast to bf16, drawn in row chunks to bound host memory."""
+    out = torch.empty(shape, dtype=torch.bfloat16)
+    flat = out.view(-1)
+    total = flat.numel()
+    for s in range(0, total, chunk):
+        e = min(total, s + chunk)
+        flat[s:e] = torch.randn(e - s, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    return out
+
+
+def small_moba(batch=1, hq=2, hkv=1, seqlen=1024, d=64, block=128, topk=3, window=0,
+               key_offset_std=0.5, name="small"):
+    """A MoBA workload of arbitrary (small) shape with the standard recipe."""
+    return Workload(name, batch, hq, hkv, seqlen, d, block=block, topk=topk, window=window,
+                    key_offset_std=key_offset_std)
+
+
+def small_swa(batch=1, hq=2, hkv=2, seqlen=1000, d=80, window=300, name="small_swa"):
+    return Workload(name, batch, hq, hkv, seqlen, d, window=window)
+
+
+def sampled_rows(w: Workload, seed: int = 0) -> np.ndarray:
+    """Query positions the oracle checks on the large workloads: the first and last
+    row of every 8th block, the first and last 64 rows of 4 random blocks (tile and
+    block edges), and 256 uniform rows; drawn with seed + 1000.  Sorted, unique."""
+    rng = np.random.default_rng(seed + 1000)
+    N = w.seqlen
+    B = w.block if w.block else 4096
+    n = N // B
+    rows = []
+    for j in range(0, n, 8):
+        rows += [j * B, j * B + B - 1]
+    for j in rng.choice(n, size=min(4, n), replace=False):
+        rows += list(range(j * B, j * B + min(64, B)))
+        rows += list(range(j * B + B - min(64, B), j * B + B))
+    rows += list(rng.integers(0, N, size=256))
+    return np.unique(np.asarray(rows, dtype=np.int32))
