@@ -1,0 +1,462 @@
+"""Benchmark: MoBA block-sparse attention prefill on B200, one JSON line.
+
+One step is the whole hot path over one batch of the workload: key pooling, gate
+scores + top-k + dispatch lists, and block-sparse attention with the merge
+(moba_pool_keys -> moba_select_topk -> moba_attn_fwd), inputs resident in HBM.
+`value` is attended TFLOP/s (4 d |J_i| summed over rows, heads and batch, divided by
+the device time of the step); tokens/s, per-stage times, the dense-causal comparators
+(torch SDPA and this library's own kernel with a window >= N) and the roofline of the
+attention stage ride along.  `e2e` measures the same through the C ABI with host
+buffers (host->device copies of q, k, v and device->host copies of out, lse inside the
+timed region).  `--impl reference` times the fp64 CPU oracle instead.
+
+Multi-GPU (torchrun): every rank runs its own copy of the workload (the method
+shards over batch / kv-head groups with no exchange): weak scaling, no collective on
+the data path; the timed region is bracketed by barriers and the max over ranks is
+reported.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "block-sparse attn prefill TFLOPS & tokens/s vs dense causal, % of roofline"
+UNIT = "TFLOP/s (attended)"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gqa32k", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-comparators", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ accounting
+
+def attended_pairs_moba(idx: torch.Tensor, w: workloads.Workload) -> int:
+    """Sum over rows, heads and batch of |J_i| for the blocks in idx (own block causal,
+    past blocks whole) unioned with the causal window."""
+    B, N = w.block, w.seqlen
+    i = torch.arange(N, device=idx.device)
+    c = i // B
+    own = (i % B) + 1
+    past = ((idx >= 0) & (idx < c[None, None, :, None])).sum(-1)  # [b, h, N]
+    total = own.sum().item() * w.batch * w.hq + int(past.sum().item()) * B
+    if w.window > 0:
+        # Window keys in blocks the row did not select.
+        extra = 0
+        for blk_off in range(1, (w.window + B - 1) // B + 1):
+            blk = c - blk_off
+            ok = blk >= 0
+            lo = torch.clamp(i - w.window + 1, min=0)
+            start = torch.maximum(blk * B, lo)
+            end = torch.minimum(blk * B + B - 1, i)
+            cnt = torch.clamp(end - start + 1, min=0) * ok
+            sel = (idx == blk[None, None, :, None]).any(-1)
+            extra += int((cnt[None, None, :] * (~sel)).sum().item())
+        total += extra
+    return int(total)
+
+
+def attended_pairs_swa(w: workloads.Workload) -> int:
+    i = np.arange(w.seqlen, dtype=np.int64)
+    return int(np.minimum(i + 1, w.window).sum()) * w.batch * w.hq
+
+
+def dense_pairs(w: workloads.Workload) -> int:
+    return w.seqlen * (w.seqlen + 1) // 2 * w.batch * w.hq
+
+
+# --------------------------------------------------------------------- clocks
+
+def physical_gpu(local: int) -> str:
+    """The nvidia-smi id (index or UUID) of CUDA device `local` of this process."""
+    vis = [x.strip() for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    return vis[local] if local < len(vis) else str(local)
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: str):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu,
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx = float(parts[1])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, device):
+    import block_sparse_long_prefill_b200 as moba
+    from block_sparse_long_prefill_b200 import MobaPrefill
+
+    w = workloads.WORKLOADS[args.workload]
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream()
+    q, k, v = workloads.make_inputs(w, seed=args.seed + rank)
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    qd, kd, vd = q.to(device), k.to(device), v.to(device)
+    del q, k, v
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
+
+    if w.kind == "moba":
+        runner = MobaPrefill(w.batch, w.hq, w.hkv, w.seqlen, w.d, w.block, w.topk, w.window,
+                             device=device)
+
+        def stages():
+            moba.moba_pool_keys(kd, w.block, runner.kbar, runner.kbar_split)
+            yield "pool"
+            moba.moba_select_topk(qd, runner.kbar_split, w.block, w.topk, runner.workspace,
+                                  runner.idx)
+            yield "select"
+            moba.moba_attn_fwd(qd, kd, vd, runner.idx, w.block, w.topk, runner.workspace,
+                               w.window, out=runner.out, lse=runner.lse)
+            yield "attention"
+        out_t, lse_t = runner.out, runner.lse
+        layout_chunks = 1
+        try:
+            per_row = (w.topk - 1) * (w.d * 2 + 4) * w.batch * w.hq
+            cap = 4 << 30
+            if per_row * w.seqlen > cap:
+                rows = max(128, (cap // per_row) // 128 * 128)
+                layout_chunks = math.ceil(w.seqlen / rows)
+        except ZeroDivisionError:
+            pass
+        launches_per_step = 2 + (2 if w.topk > 1 else 0) + layout_chunks * (2 if w.topk > 1 else 1)
+    else:
+        out_t = torch.empty_like(qd)
+        lse_t = torch.empty(w.batch, w.hq, w.seqlen, dtype=torch.float32, device=device)
+
+        def stages():
+            moba.swa_attn_fwd(qd, kd, vd, w.window, out=out_t, lse=lse_t)
+            yield "attention"
+        launches_per_step = 1
+
+    def step_timed():
+        evs = [torch.cuda.Event(enable_timing=True)]
+        evs[0].record(stream)
+        names = []
+        for name in stages():
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            evs.append(e)
+            names.append(name)
+        return evs, names
+
+    for _ in range(args.warmup):
+        for _ in stages():
+            pass
+    torch.cuda.synchronize()
+    assert moba.device_status() == 0
+
+    pairs = attended_pairs_moba(runner.idx, w) if w.kind == "moba" else attended_pairs_swa(w)
+    flops = 4.0 * w.d * pairs
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    per_stage = {}
+    total_ms = 0.0
+    with ClockSampler(physical_gpu(torch.cuda.current_device())) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            evs, names = step_timed()
+            torch.cuda.synchronize()
+            total_ms += evs[0].elapsed_time(evs[-1])
+            for a, b_, n in zip(evs[:-1], evs[1:], names):
+                per_stage.setdefault(n, []).append(a.elapsed_time(b_))
+    torch.cuda.synchronize()
+    if world > 1:
+        t = torch.tensor([total_ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+        torch.distributed.barrier()
+    assert moba.device_status() == 0
+    assert torch.isfinite(out_t.float()).all().item(), "non-finite output"
+    ms = total_ms / args.steps
+    tflops_total = flops * world / (ms * 1e-3) / 1e12
+    tokens = w.batch * w.seqlen * world / (ms * 1e-3)
+
+    hbm, tc_peak, tc_sus, peak_kind = peaks()
+    stage_ms = {n: sum(v) / len(v) for n, v in per_stage.items()}
+    attn_ms = stage_ms["attention"]
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4), "traffic": None,
+                "kernel": "moba_attn_fwd (past-block pass + own-block pass)" if w.kind == "moba"
+                else "swa_attn_fwd", "peak_kind": f"bf16 dense burst, {peak_kind}"}
+    extra = {}
+    if w.kind == "moba":
+        sel_ms = stage_ms["pool"] + stage_ms["select"]
+        n_entries = int(((runner.idx >= 0).sum().item()) - w.batch * w.hq * w.seqlen)
+        sel_bytes = (w.batch * w.hkv * w.seqlen * w.d * 2 + w.batch * w.hq * w.seqlen * w.d * 2
+                     + 2 * w.batch * w.hq * w.seqlen * w.topk * 4 + 2 * n_entries * 4)
+        extra["selection"] = {"ms": round(sel_ms, 4), "bytes": sel_bytes,
+                              "gbs": round(sel_bytes / (sel_ms * 1e-3) / 1e9, 1),
+                              "frac_hbm": round(sel_bytes / (sel_ms * 1e-3) / 1e9 / hbm, 4)}
+
+    # ---------------------------------------------------------------- e2e (host buffers)
+    out_h = torch.empty(out_t.shape, dtype=out_t.dtype, pin_memory=True)
+    lse_h = torch.empty(lse_t.shape, dtype=lse_t.dtype, pin_memory=True)
+    e2e_ms = 0.0
+    for it in range(args.warmup + args.steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        for _ in stages():
+            pass
+        out_h.copy_(out_t, non_blocking=True)
+        lse_h.copy_(lse_t, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            e2e_ms += e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_ms /= args.steps
+    h2d = (qh.numel() + kh.numel() + vh.numel()) * 2
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+    e2e = {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+           "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # ---------------------------------------------------------------- comparators
+    comps = {}
+    if not args.no_comparators and rank == 0:
+        dflops = 4.0 * w.d * dense_pairs(w)
+        G = w.hq // w.hkv
+        kr = kd.repeat_interleave(G, dim=1) if G > 1 else kd
+        vr = vd.repeat_interleave(G, dim=1) if G > 1 else vd
+        import torch.nn.functional as F
+
+        def timeit(fn, reps):
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize()
+            tot = 0.0
+            for _ in range(reps):
+                flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b_ = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b_.record(stream)
+                torch.cuda.synchronize()
+                tot += a.elapsed_time(b_)
+            return tot / reps
+
+        sd_ms = timeit(lambda: F.scaled_dot_product_attention(qd, kr, vr, is_causal=True),
+                       max(3, args.steps // 4))
+        own_out = torch.empty_like(qd)
+        own_lse = torch.empty(w.batch, w.hq, w.seqlen, dtype=torch.float32, device=device)
+        od_ms = timeit(lambda: moba.swa_attn_fwd(qd, kd, vd, w.seqlen, out=own_out, lse=own_lse),
+                       max(3, args.steps // 4))
+        comps = {"dense_causal_sdpa": {"ms": round(sd_ms, 4),
+                                       "tflops": round(dflops / (sd_ms * 1e-3) / 1e12, 2),
+                                       "speedup_of_moba": round(sd_ms / ms, 3)},
+                 "dense_causal_own_kernel": {"ms": round(od_ms, 4),
+                                             "tflops": round(dflops / (od_ms * 1e-3) / 1e12, 2),
+                                             "frac_of_peak": round(dflops / (od_ms * 1e-3) / 1e12
+                                                                   / tc_peak, 4)}}
+        del kr, vr
+
+    cpu = None
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
+        cpu = cpu_baseline(w, args.seed, target_s=12.0)
+
+    clocks = clk.summary()
+    line = {"metric": METRIC, "value": round(tflops_total, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) q,k,v; per-block key offsets; no dataset)",
+            "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv,
+                       "seq_len": w.seqlen, "d": w.d, "block": w.block, "topk": w.topk,
+                       "window": w.window, "parallelism": f"replicas x{world}" if world > 1 else "1 gpu",
+                       "l2": "flushed between timed steps (256 MB write)"},
+            "tokens_per_s": round(tokens, 1), "attended_flops_per_step": flops,
+            "stages_ms": {k_: round(v_, 4) for k_, v_ in stage_ms.items()},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
+    line.update(extra)
+    line.update(comps)
+    return line
+
+
+# ------------------------------------------------------------ oracle timing
+
+def cpu_baseline(w: workloads.Workload, seed: int, target_s: float):
+    """Times the fp64 oracle on this workload: the full key pooling plus selection and
+    attention for a seeded sample of query rows (all heads), sized to about target_s
+    seconds; reports the attended TFLOP/s extrapolated to the whole workload."""
+    import oracle
+
+    q, k, v = workloads.make_inputs(w, seed)
+    rng = np.random.default_rng(seed + 2000)
+    N = w.seqlen
+
+    def run(nrows):
+        rows = np.sort(rng.choice(N, size=nrows, replace=False)).astype(np.int32)
+        t0 = time.perf_counter()
+        if w.kind == "moba":
+            kbar = oracle.pool_keys(k, w.block)
+            t1 = time.perf_counter()
+            s = oracle.gate_scores(q, kbar, w.block, rows)
+            idx, _ = oracle.select_topk(s, N, w.block, w.topk, rows)
+            oracle.attention(q, k, v, mode=oracle.MODE_MOBA, block=w.block, topk=w.topk, idx=idx,
+                             window=w.window, rows=rows)
+            t2 = time.perf_counter()
+            i = rows.astype(np.int64)
+            c = i // w.block
+            pairs_rows = int(((i % w.block) + 1 + np.minimum(w.topk - 1, c) * w.block).sum()) * w.batch * w.hq
+            return t1 - t0, t2 - t1, pairs_rows
+        oracle.swa(q, k, v, window=w.window, rows=rows)
+        t2 = time.perf_counter()
+        pairs_rows = int(np.minimum(rows.astype(np.int64) + 1, w.window).sum()) * w.batch * w.hq
+        return 0.0, t2 - t0, pairs_rows
+
+    probe = min(N, 32)
+    tp, ta, _ = run(probe)
+    per_row = max(ta / probe, 1e-6)
+    nrows = int(min(N, max(probe, target_s / per_row)))
+    tp, ta, pairs_rows = run(nrows)
+    full_s = tp + ta * N / nrows
+    pairs = attended_pairs_swa(w) if w.kind == "swa" else None
+    if pairs is None:
+        i = np.arange(N, dtype=np.int64)
+        pairs = int(((i % w.block) + 1 + np.minimum(w.topk - 1, i // w.block) * w.block).sum()) * w.batch * w.hq
+    flops = 4.0 * w.d * pairs
+    return {"value": flops / full_s / 1e12, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"full key pooling + {nrows} of {N} query rows x {w.batch * w.hq} heads "
+                      f"(seeded); whole-workload time extrapolated by rows: {full_s:.1f} s",
+            "sample_seconds": round(tp + ta, 2)}
+
+
+def run_reference(args, rank, world):
+    """The oracle on the host cores as the reference arm (rank 0 only)."""
+    w = workloads.WORKLOADS[args.workload]
+    if rank != 0:
+        return None
+    per_step = []
+    last = None
+    for it in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        last = cpu_baseline(w, args.seed + it, target_s=3.0)
+        if it >= args.warmup:
+            per_step.append(last["value"])
+    value = statistics.median(per_step)
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv,
+                       "seq_len": w.seqlen, "d": w.d, "block": w.block, "topk": w.topk,
+                       "window": w.window},
+            "cpu_baseline": {**last, "value": value},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    line = run_ours(args, rank, world, torch.device("cuda", local))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

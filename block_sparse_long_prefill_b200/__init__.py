@@ -1,0 +1,197 @@
+"""MoBA block-sparse attention prefill and sliding-window attention prefill on B200.
+
+A thin ctypes binding over ``libmoba.so`` (declared in ``include/moba.h``).  The
+functions here only turn torch tensors into pointers, strides and a stream and pass
+them through the C ABI: every step of the computation runs in the library's sm_100a
+kernels.  There is no CPU fallback; importing fails loudly when the library is
+missing.
+
+Method sources (by page title and section):
+  [MoBA] "MoBA: 어텐션에 전문가 혼합을 적용해 긴 문맥을 효율적으로 처리하는 블록 어텐션
+         (feat. MoonshotAI)", PyTorch KR forum summary of the MoBA paper.
+  [SWA]  "SWA + MoE: 어텐션과 희소 전문가", Bit-Axon architecture page.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoba.so")
+
+MOBA_OK = 0
+_STATUS = {
+    -1: "MOBA_ERR_SHAPE", -2: "MOBA_ERR_DIM", -3: "MOBA_ERR_ALIGN", -4: "MOBA_ERR_ARG",
+    -5: "MOBA_ERR_WORKSPACE", -6: "MOBA_ERR_LAUNCH", -7: "MOBA_ERR_DEVICE", -8: "MOBA_ERR_NODEVICE",
+}
+
+# Entry points declared in include/moba.h.
+ABI_FUNCTIONS = ("moba_workspace_size", "moba_pool_keys", "moba_select_topk", "moba_attn_fwd",
+                 "swa_attn_fwd", "moba_device_status", "moba_status_string")
+
+
+class MobaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn}: {_STATUS.get(code, code)} ({status_string(code)})")
+
+
+class MobaTensor(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("sb", ctypes.c_int64), ("sh", ctypes.c_int64),
+                ("sn", ctypes.c_int64)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m block_sparse_long_prefill_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    I, P, S = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+    T = MobaTensor
+    lib.moba_workspace_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(S)]
+    lib.moba_pool_keys.argtypes = [T, I, I, I, I, I, P, P, P]
+    lib.moba_select_topk.argtypes = [T, P, I, I, I, I, I, I, I, P, P, S, P]
+    lib.moba_attn_fwd.argtypes = [T, T, T, P, I, I, I, I, I, I, I, I, ctypes.c_float, T, P, P, S, P]
+    lib.swa_attn_fwd.argtypes = [T, T, T, I, I, I, I, I, I, ctypes.c_float, T, P, P]
+    lib.moba_device_status.argtypes = []
+    lib.moba_status_string.argtypes = [I]
+    lib.moba_status_string.restype = ctypes.c_char_p
+    for name in ABI_FUNCTIONS[:-1]:
+        getattr(lib, name).restype = I
+    return lib
+
+
+_lib = _load()
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return _lib.moba_status_string(int(code)).decode()
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != MOBA_OK:
+        raise MobaError(fn, rc)
+
+
+def _t(x: torch.Tensor) -> MobaTensor:
+    """[b, h, n, d] tensor with a contiguous last dimension -> moba_tensor."""
+    if x.dim() != 4:
+        raise ValueError("expected a [batch, heads, N, d] tensor")
+    if x.stride(3) != 1:
+        raise ValueError("the head dimension must be contiguous")
+    return MobaTensor(x.data_ptr(), x.stride(0), x.stride(1), x.stride(2))
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def workspace_size(batch, hq, hkv, N, d, block, topk) -> int:
+    out = ctypes.c_size_t(0)
+    _check("moba_workspace_size",
+           _lib.moba_workspace_size(batch, hq, hkv, N, d, block, topk, ctypes.byref(out)))
+    return out.value
+
+
+def moba_pool_keys(k: torch.Tensor, block: int, kbar=None, kbar_split=None, stream=None):
+    """[MoBA] §블록 분할과 top-k 게이팅: block means of the keys.  Returns (kbar float32
+    [b, hkv, n, d], kbar_split bf16 [b, hkv, 2, n, d])."""
+    b, hkv, N, d = k.shape
+    n = N // block
+    if kbar is None:
+        kbar = torch.empty(b, hkv, n, d, dtype=torch.float32, device=k.device)
+    if kbar_split is None:
+        kbar_split = torch.empty(b, hkv, 2, n, d, dtype=torch.bfloat16, device=k.device)
+    _check("moba_pool_keys", _lib.moba_pool_keys(_t(k), b, hkv, N, d, block, kbar.data_ptr(),
+                                                 kbar_split.data_ptr(), _stream(stream)))
+    return kbar, kbar_split
+
+
+def moba_select_topk(q: torch.Tensor, kbar_split: torch.Tensor, block: int, topk: int,
+                     workspace: torch.Tensor, idx=None, stream=None):
+    """[MoBA] §블록 분할과 top-k 게이팅 + §인과성 보존: per-row block choices (int32
+    [b, hq, N, topk], ascending, -1 padded) and the dispatch lists in ``workspace``."""
+    b, hq, N, d = q.shape
+    hkv = kbar_split.shape[1]
+    if idx is None:
+        idx = torch.empty(b, hq, N, topk, dtype=torch.int32, device=q.device)
+    _check("moba_select_topk",
+           _lib.moba_select_topk(_t(q), kbar_split.data_ptr(), b, hq, hkv, N, d, block, topk,
+                                 idx.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                 _stream(stream)))
+    return idx
+
+
+def moba_attn_fwd(q, k, v, idx, block: int, topk: int, workspace: torch.Tensor, window: int = 0,
+                  scale: float = 0.0, out=None, lse=None, stream=None):
+    """[MoBA] §MoBA의 구현: attention over the selected blocks (unioned with the causal
+    window).  Returns (out bf16 [b, hq, N, d], lse float32 [b, hq, N])."""
+    b, hq, N, d = q.shape
+    hkv = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device)
+    _check("moba_attn_fwd",
+           _lib.moba_attn_fwd(_t(q), _t(k), _t(v), idx.data_ptr(), b, hq, hkv, N, d, block, topk,
+                              window, float(scale), _t(out), lse.data_ptr(), workspace.data_ptr(),
+                              workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def swa_attn_fwd(q, k, v, window: int, scale: float = 0.0, out=None, lse=None, stream=None):
+    """[SWA] §슬라이딩 윈도우 마스크: causal band attention (window >= N is dense causal)."""
+    b, hq, N, d = q.shape
+    hkv = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device)
+    _check("swa_attn_fwd",
+           _lib.swa_attn_fwd(_t(q), _t(k), _t(v), b, hq, hkv, N, d, window, float(scale), _t(out),
+                             lse.data_ptr(), _stream(stream)))
+    return out, lse
+
+
+def device_status() -> int:
+    """Reads and clears the device-side wait-timeout status (synchronises)."""
+    return int(_lib.moba_device_status())
+
+
+class MobaPrefill:
+    """The three MoBA calls with their buffers allocated once for a fixed shape."""
+
+    def __init__(self, batch, hq, hkv, N, d, block, topk, window=0, device="cuda"):
+        self.shape = (batch, hq, hkv, N, d)
+        self.block, self.topk, self.window = block, topk, window
+        n = N // block
+        self.workspace = torch.empty(workspace_size(batch, hq, hkv, N, d, block, topk),
+                                     dtype=torch.uint8, device=device)
+        self.kbar = torch.empty(batch, hkv, n, d, dtype=torch.float32, device=device)
+        self.kbar_split = torch.empty(batch, hkv, 2, n, d, dtype=torch.bfloat16, device=device)
+        self.idx = torch.empty(batch, hq, N, topk, dtype=torch.int32, device=device)
+        self.out = torch.empty(batch, hq, N, d, dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(batch, hq, N, dtype=torch.float32, device=device)
+
+    def __call__(self, q, k, v, stream=None):
+        moba_pool_keys(k, self.block, self.kbar, self.kbar_split, stream)
+        moba_select_topk(q, self.kbar_split, self.block, self.topk, self.workspace, self.idx, stream)
+        moba_attn_fwd(q, k, v, self.idx, self.block, self.topk, self.workspace, self.window,
+                      out=self.out, lse=self.lse, stream=stream)
+        return self.out, self.lse
+
+
+def moba_prefill(q, k, v, block: int, topk: int, window: int = 0, stream=None):
+    """Pool, select and attend in one call; returns (out, lse, idx)."""
+    b, hq, N, d = q.shape
+    runner = MobaPrefill(b, hq, k.shape[1], N, d, block, topk, window, device=q.device)
+    out, lse = runner(q, k, v, stream)
+    return out, lse, runner.idx

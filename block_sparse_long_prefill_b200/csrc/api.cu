@@ -1,0 +1,319 @@
+// api.cu -- the C ABI of libmoba (declared in include/moba.h): argument checks,
+// workspace carving, TMA descriptors and kernel launches.  Every step of the
+// computation runs in the kernels of select.cu and attn.cu.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "moba.h"
+#include "params.h"
+
+namespace moba {
+
+__device__ int g_device_status[2] = {MOBA_OK, 0};
+
+cudaError_t launch_pool(const uint16_t *k, int64_t sb, int64_t sh, int64_t sn, int batch, int hkv,
+                        int N, int d, int block, float *kbar, uint16_t *split, cudaStream_t st);
+cudaError_t launch_gate(const SelectParams &p, cudaStream_t st);
+cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileoff, int nlists,
+                        cudaStream_t st);
+cudaError_t launch_scatter(const ScatterParams &p, cudaStream_t st);
+cudaError_t launch_attn(const CUtensorMap *maps, const AttnParams &p, int mode, int grid,
+                        cudaStream_t st);
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_tensor(const moba_tensor &t) {
+  if (!t.ptr) return MOBA_ERR_ARG;
+  if (!aligned16(t.ptr)) return MOBA_ERR_ALIGN;
+  // bf16 strides in elements: 16-byte multiples.
+  if ((t.sb % 8) || (t.sh % 8) || (t.sn % 8) || t.sb < 0 || t.sh < 0 || t.sn < 0)
+    return MOBA_ERR_ALIGN;
+  return MOBA_OK;
+}
+
+int check_device(int *num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOBA_ERR_NODEVICE;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return MOBA_ERR_NODEVICE;
+  if (major != 10) return MOBA_ERR_NODEVICE;
+  if (num_sms && cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOBA_ERR_NODEVICE;
+  return MOBA_OK;
+}
+
+int check_attn_dim(int d) { return (d == 64 || d == 80 || d == 128) ? MOBA_OK : MOBA_ERR_DIM; }
+
+int check_moba_shape(int batch, int hq, int hkv, int N, int d, int block, int topk) {
+  if (batch < 1 || hq < 1 || hkv < 1 || N < 1 || block < 1) return MOBA_ERR_SHAPE;
+  if (hq % hkv) return MOBA_ERR_SHAPE;
+  if (block % kTileRows || N % block) return MOBA_ERR_SHAPE;
+  if (topk < 1 || topk > 32) return MOBA_ERR_ARG;
+  const long long G = hq / hkv;
+  if ((long long)N * G * (topk - 1) >= (1ll << 31)) return MOBA_ERR_SHAPE;
+  if ((long long)batch * hq * N * (topk - 1) >= (1ll << 31)) return MOBA_ERR_SHAPE;
+  if ((long long)batch * hq * N * topk >= (1ll << 40)) return MOBA_ERR_SHAPE;
+  if (check_attn_dim(d) != MOBA_OK) return MOBA_ERR_DIM;
+  return MOBA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 4-D map over a bf16 [batch, heads, N, d] tensor (dims innermost first: d, N, heads,
+// batch) whose box is `cols` columns x 128 rows, with the given swizzle.
+int make_map(CUtensorMap *map, const moba_tensor &t, int batch, int heads, int N, int d, int cols,
+             CUtensorMapSwizzle swz) {
+  auto enc = get_encode();
+  if (!enc) return MOBA_ERR_LAUNCH;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)heads, (cuuint64_t)batch};
+  cuuint64_t strides[3] = {(cuuint64_t)t.sn * 2, (cuuint64_t)t.sh * 2, (cuuint64_t)t.sb * 2};
+  // A size-1 dimension may carry any stride; give TMA a legal one.
+  if (heads == 1) strides[1] = strides[0] * (cuuint64_t)N;
+  if (batch == 1) strides[2] = strides[1] * (cuuint64_t)heads;
+  cuuint32_t box[4] = {(cuuint32_t)cols, 128u, 1u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.ptr, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOBA_OK : MOBA_ERR_LAUNCH;
+}
+
+// Q, Q tail, K, K tail, V, V tail.
+int make_attn_maps(CUtensorMap *maps, const moba_tensor &q, const moba_tensor &k,
+                   const moba_tensor &v, int batch, int hq, int hkv, int N, int d) {
+  const moba_tensor *ts[3] = {&q, &k, &v};
+  const int heads[3] = {hq, hkv, hkv};
+  for (int a = 0; a < 3; ++a) {
+    int rc = make_map(&maps[2 * a], *ts[a], batch, heads[a], N, d, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+    if (d == 80)
+      rc = make_map(&maps[2 * a + 1], *ts[a], batch, heads[a], N, d, 16, CU_TENSOR_MAP_SWIZZLE_32B);
+    else
+      maps[2 * a + 1] = maps[2 * a];
+    if (rc) return rc;
+  }
+  return MOBA_OK;
+}
+
+int launch_status(cudaError_t e) { return e == cudaSuccess ? MOBA_OK : MOBA_ERR_LAUNCH; }
+
+// Device address of the status words on the current device.
+int status_words(int **ptr) {
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return MOBA_ERR_LAUNCH;
+  *ptr = static_cast<int *>(p);
+  return MOBA_OK;
+}
+
+}  // namespace
+}  // namespace moba
+
+using namespace moba;
+
+extern "C" {
+
+int moba_workspace_size(int batch, int hq, int hkv, int N, int d, int block, int topk,
+                        size_t *bytes) {
+  if (!bytes) return MOBA_ERR_ARG;
+  const int rc = check_moba_shape(batch, hq, hkv, N, d, block, topk);
+  if (rc) return rc;
+  *bytes = make_layout(batch, hq, hkv, N, d, block, topk).total;
+  return MOBA_OK;
+}
+
+int moba_pool_keys(moba_tensor k, int batch, int hkv, int N, int d, int block, float *kbar,
+                   void *kbar_split, void *stream) {
+  if (batch < 1 || hkv < 1 || N < 1 || block < 1 || N % block) return MOBA_ERR_SHAPE;
+  if (d < 8 || d > 256 || d % 8) return MOBA_ERR_DIM;
+  int rc = check_tensor(k);
+  if (rc) return rc;
+  if (!kbar || !kbar_split) return MOBA_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(kbar) & 3u) || (reinterpret_cast<uintptr_t>(kbar_split) & 1u))
+    return MOBA_ERR_ALIGN;
+  if ((rc = check_device(nullptr))) return rc;
+  return launch_status(launch_pool(static_cast<const uint16_t *>(k.ptr), k.sb, k.sh, k.sn, batch,
+                                   hkv, N, d, block, kbar, static_cast<uint16_t *>(kbar_split),
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, int hkv, int N,
+                     int d, int block, int topk, int32_t *idx, void *workspace,
+                     size_t workspace_bytes, void *stream) {
+  int rc = check_moba_shape(batch, hq, hkv, N, d, block, topk);
+  if (rc) return rc;
+  if ((rc = check_tensor(q))) return rc;
+  if (!kbar_split || !idx) return MOBA_ERR_ARG;
+  if (!aligned16(kbar_split) || (reinterpret_cast<uintptr_t>(idx) & 3u)) return MOBA_ERR_ALIGN;
+  const WorkspaceLayout w = make_layout(batch, hq, hkv, N, d, block, topk);
+  if (!workspace || workspace_bytes < w.total) return MOBA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MOBA_ERR_ALIGN;
+  if ((rc = check_device(nullptr))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char *ws = static_cast<char *>(workspace);
+  int *counts = reinterpret_cast<int *>(ws + w.off_counts);
+  if (cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)w.nlists, st) != cudaSuccess)
+    return MOBA_ERR_LAUNCH;
+  SelectParams sp{};
+  sp.q = static_cast<const uint16_t *>(q.ptr);
+  sp.q_sb = q.sb; sp.q_sh = q.sh; sp.q_sn = q.sn;
+  sp.kbar_split = static_cast<const uint16_t *>(kbar_split);
+  sp.idx = idx;
+  sp.counts = counts;
+  sp.batch = batch; sp.hq = hq; sp.hkv = hkv; sp.N = N; sp.d = d; sp.block = block;
+  sp.topk = topk; sp.nblk = w.nblk; sp.G = w.G; sp.chunk_rows = w.chunk_rows;
+  if ((rc = launch_status(launch_gate(sp, st)))) return rc;
+  if (w.npast == 0) return MOBA_OK;
+  int *cursor = reinterpret_cast<int *>(ws + w.off_cursor);
+  int *listoff = reinterpret_cast<int *>(ws + w.off_listoff);
+  int *tileoff = reinterpret_cast<int *>(ws + w.off_tileoff);
+  if ((rc = launch_status(launch_scan(counts, cursor, listoff, tileoff, w.nlists, st)))) return rc;
+  ScatterParams cp{};
+  cp.idx = idx;
+  cp.cursor = cursor;
+  cp.entries = reinterpret_cast<uint32_t *>(ws + w.off_entries);
+  cp.batch = batch; cp.hq = hq; cp.hkv = hkv; cp.N = N; cp.block = block; cp.topk = topk;
+  cp.nblk = w.nblk; cp.G = w.G; cp.chunk_rows = w.chunk_rows;
+  return launch_status(launch_scatter(cp, st));
+}
+
+int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *idx, int batch,
+                  int hq, int hkv, int N, int d, int block, int topk, int window, float scale,
+                  moba_tensor out, float *lse, void *workspace, size_t workspace_bytes,
+                  void *stream) {
+  int rc = check_moba_shape(batch, hq, hkv, N, d, block, topk);
+  if (rc) return rc;
+  if (window < 0) return MOBA_ERR_ARG;
+  if ((rc = check_tensor(q)) || (rc = check_tensor(k)) || (rc = check_tensor(v)) ||
+      (rc = check_tensor(out)))
+    return rc;
+  if (!idx || !lse) return MOBA_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return MOBA_ERR_ALIGN;
+  const WorkspaceLayout w = make_layout(batch, hq, hkv, N, d, block, topk);
+  if (!workspace || workspace_bytes < w.total) return MOBA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MOBA_ERR_ALIGN;
+  int nsm = 0;
+  if ((rc = check_device(&nsm))) return rc;
+  CUtensorMap maps[6];
+  if ((rc = make_attn_maps(maps, q, k, v, batch, hq, hkv, N, d))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char *ws = static_cast<char *>(workspace);
+  AttnParams p{};
+  if ((rc = status_words(&p.status))) return rc;
+  p.q = static_cast<const uint16_t *>(q.ptr);
+  p.q_sb = q.sb; p.q_sh = q.sh; p.q_sn = q.sn;
+  p.out = static_cast<uint16_t *>(out.ptr);
+  p.o_sb = out.sb; p.o_sh = out.sh; p.o_sn = out.sn;
+  p.lse = lse;
+  p.idx = idx;
+  p.batch = batch; p.hq = hq; p.hkv = hkv; p.N = N; p.d = d; p.block = block; p.topk = topk;
+  p.window = window; p.G = w.G;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.is_moba = 1;
+  p.listoff = reinterpret_cast<const int *>(ws + w.off_listoff);
+  p.tileoff = reinterpret_cast<const int *>(ws + w.off_tileoff);
+  p.entries = reinterpret_cast<const uint32_t *>(ws + w.off_entries);
+  p.opart = reinterpret_cast<uint16_t *>(ws + w.off_opart);
+  p.lpart = reinterpret_cast<float *>(ws + w.off_lpart);
+  p.chunk_rows = w.chunk_rows;
+  p.npast = w.npast;
+  p.nblk = w.nblk;
+  p.lists_per_chunk = batch * hkv * w.nblk;
+  for (int c = 0; c < w.nchunks; ++c) {
+    p.chunk = c;
+    p.row_begin = c * w.chunk_rows;
+    p.row_end = (c + 1) * w.chunk_rows < N ? (c + 1) * w.chunk_rows : N;
+    if (w.npast > 0) {
+      p.ntiles = 0;  // read from the workspace by the kernel
+      if ((rc = launch_status(launch_attn(maps, p, kGathered, nsm, st)))) return rc;
+    }
+    const int nq = (p.row_end - p.row_begin + kTileRows - 1) / kTileRows;
+    p.ntiles = nq * hq * batch;
+    const int grid = p.ntiles < nsm ? p.ntiles : nsm;
+    if ((rc = launch_status(launch_attn(maps, p, kQueryMajor, grid, st)))) return rc;
+  }
+  return MOBA_OK;
+}
+
+int swa_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq, int hkv, int N,
+                 int d, int window, float scale, moba_tensor out, float *lse, void *stream) {
+  if (batch < 1 || hq < 1 || hkv < 1 || N < 1 || hq % hkv) return MOBA_ERR_SHAPE;
+  if (window < 1) return MOBA_ERR_ARG;
+  int rc = check_attn_dim(d);
+  if (rc) return rc;
+  if ((rc = check_tensor(q)) || (rc = check_tensor(k)) || (rc = check_tensor(v)) ||
+      (rc = check_tensor(out)))
+    return rc;
+  if (!lse) return MOBA_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return MOBA_ERR_ALIGN;
+  int nsm = 0;
+  if ((rc = check_device(&nsm))) return rc;
+  CUtensorMap maps[6];
+  if ((rc = make_attn_maps(maps, q, k, v, batch, hq, hkv, N, d))) return rc;
+  AttnParams p{};
+  if ((rc = status_words(&p.status))) return rc;
+  p.q = static_cast<const uint16_t *>(q.ptr);
+  p.q_sb = q.sb; p.q_sh = q.sh; p.q_sn = q.sn;
+  p.out = static_cast<uint16_t *>(out.ptr);
+  p.o_sb = out.sb; p.o_sh = out.sh; p.o_sn = out.sn;
+  p.lse = lse;
+  p.idx = nullptr;
+  p.batch = batch; p.hq = hq; p.hkv = hkv; p.N = N; p.d = d; p.block = 0; p.topk = 0;
+  p.window = window < N ? window : N;
+  p.G = hq / hkv;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.is_moba = 0;
+  p.row_begin = 0;
+  p.row_end = N;
+  const int nq = (N + kTileRows - 1) / kTileRows;
+  p.ntiles = nq * hq * batch;
+  p.npast = 0;
+  const int grid = p.ntiles < nsm ? p.ntiles : nsm;
+  return launch_status(launch_attn(maps, p, kQueryMajor, grid, static_cast<cudaStream_t>(stream)));
+}
+
+int moba_device_status(void) {
+  int v[2] = {MOBA_OK, 0};
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOBA_ERR_LAUNCH;
+  if (cudaMemcpyFromSymbol(v, g_device_status, sizeof(v)) != cudaSuccess) return MOBA_ERR_LAUNCH;
+  const int zero[2] = {MOBA_OK, 0};
+  if (cudaMemcpyToSymbol(g_device_status, zero, sizeof(zero)) != cudaSuccess) return MOBA_ERR_LAUNCH;
+  return v[0];
+}
+
+const char *moba_status_string(int status) {
+  switch (status) {
+    case MOBA_OK: return "ok";
+    case MOBA_ERR_SHAPE: return "unsupported shape (N % block, hq % hkv, block % 128, size limits)";
+    case MOBA_ERR_DIM: return "unsupported head dimension";
+    case MOBA_ERR_ALIGN: return "pointer or stride not 16-byte aligned";
+    case MOBA_ERR_ARG: return "invalid argument";
+    case MOBA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOBA_ERR_LAUNCH: return "CUDA launch or driver call failed";
+    case MOBA_ERR_DEVICE: return "a kernel wait timed out on the device";
+    case MOBA_ERR_NODEVICE: return "no sm_100 device is current";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,629 @@
+// attn.cu -- block-sparse / sliding-window attention forward on sm_100a tensor cores.
+//
+// [MoBA] = "MoBA: 어텐션에 전문가 혼합을 적용해 긴 문맥을 효율적으로 처리하는 블록 어텐션
+//          (feat. MoonshotAI)", PyTorch KR forum summary of the MoBA paper.
+// [SWA]  = "SWA + MoE: 어텐션과 희소 전문가", Bit-Axon architecture page.
+//
+// One persistent kernel, two tile kinds:
+//   kQueryMajor  128 contiguous query rows of one (batch, q-head).  MoBA: the causal own
+//                block (§"MoBA의 구현": current block with causal=True), the window
+//                tail into earlier unselected blocks, and the merge of the past-block
+//                partials by log-sum-exp (step 5).  SWA: the causal band of [SWA]
+//                §"슬라이딩 윈도우 마스크".
+//   kGathered    up to 128 (row, q-head) pairs of one block-major list against the
+//                whole past block they picked (steps 3-4, causal=False); writes a
+//                normalised partial output and its log-sum-exp per (row, slot).
+//
+// Per CTA (256 threads, one CTA per SM, 512 TMEM columns):
+//   warp 0      TMA producer: K/V chunks of 128 keys (and the query tile, query-major)
+//   warp 1      tcgen05 MMA issuer (one thread) and TMEM owner
+//   warps 2-3   query-row gather with cp.async (gathered tiles)
+//   warps 4-7   softmax, O correction and epilogue; thread r owns row r (TMEM lane r)
+// TMEM: S/P double buffer at columns [0,128) and [128,256); O at [256, 256+D).
+// S = Q K^T is an SS MMA; P (bf16) overwrites its own S columns and is the A operand
+// (from TMEM) of O += P V.  Softmax uses exp2 with a lazily raised running maximum:
+// O and l are rescaled only when the row maximum grows by more than 2^8.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "params.h"
+
+namespace moba {
+
+constexpr int kAttnThreads = 256;
+constexpr int kRescaleThreshold = 8;  // log2 units
+
+template <int D>
+struct AttnCfg {
+  static constexpr int ST = (D == 128) ? 2 : 3;            // K/V pipeline stages
+  static constexpr int R0 = 128 * 128;                     // bytes of the 64-column region
+  static constexpr int R1 = (D == 128) ? 128 * 128 : (D == 80 ? 128 * 32 : 0);
+  static constexpr int TILE = R0 + ((R1 + 1023) / 1024) * 1024;  // one 128 x D operand tile
+  static constexpr int Q_OFF = 0;                          // 2 query buffers
+  static constexpr int K_OFF = 2 * TILE;                   // ST key stages
+  static constexpr int V_OFF = K_OFF + ST * TILE;          // ST value stages
+  static constexpr int BAR_OFF = V_OFF + ST * TILE;
+  static constexpr int SMEM = BAR_OFF + 1024 + 1024;       // + barriers + alignment slack
+  static constexpr uint32_t BYTES = 128u * D * 2u;         // bytes one full tile load moves
+};
+
+struct Bars {
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[3], v_full[3], kv_empty[3];
+  uint64_t s_full[2];
+  uint64_t p_full, o_done, o_free, mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// What one tile covers.  All roles derive it independently from the tile index.
+struct TileInfo {
+  int b, h, hk;
+  int i0;          // query-major: first row
+  int rows;        // valid rows
+  int nc;          // key chunks
+  int key0;        // query-major MoBA: first key of the tail (window) range
+  int ntail;       // query-major MoBA: chunks before the own block
+  int cB;          // query-major MoBA: first key of the own block
+  // gathered
+  int list;        // list id
+  int ent0;        // first entry of this tile in the entry array
+  int j;           // past block
+};
+
+__device__ __forceinline__ void query_major_tile(const AttnParams &p, int t, TileInfo &ti) {
+  const int HB = p.hq * p.batch;
+  const int nq = (p.row_end - p.row_begin + kTileRows - 1) / kTileRows;
+  const int qt = nq - 1 - t / HB;  // later (heavier) tiles first
+  const int hb = t % HB;
+  ti.h = hb % p.hq;
+  ti.b = hb / p.hq;
+  ti.hk = ti.h / p.G;
+  ti.i0 = p.row_begin + qt * kTileRows;
+  ti.rows = min(kTileRows, p.row_end - ti.i0);
+  const int ilast = ti.i0 + ti.rows - 1;
+  if (p.is_moba) {
+    ti.cB = (ti.i0 / p.block) * p.block;
+    int tl = ti.cB;
+    if (p.window > 0) {
+      const int lo = max(0, ti.i0 - p.window + 1);
+      tl = min(ti.cB, (lo / kTileKeys) * kTileKeys);
+    }
+    ti.key0 = tl;
+    ti.ntail = (ti.cB - tl) / kTileKeys;
+    ti.nc = ti.ntail + (ti.i0 - ti.cB) / kTileKeys + 1;
+  } else {
+    const int lo = max(0, ti.i0 - p.window + 1);
+    ti.key0 = (lo / kTileKeys) * kTileKeys;
+    ti.ntail = 0;
+    ti.cB = 0;
+    ti.nc = (ilast - ti.key0) / kTileKeys + 1;
+  }
+}
+
+__device__ __forceinline__ void gathered_tile(const AttnParams &p, int t, TileInfo &ti) {
+  // Binary search the list whose tile range holds t (lists of this chunk only).
+  int lo = p.chunk * p.lists_per_chunk, hi = lo + p.lists_per_chunk;  // tileoff[lo] <= t < tileoff[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(p.tileoff + mid) <= t) lo = mid; else hi = mid;
+  }
+  const int L = lo;
+  const int first = __ldg(p.listoff + L);
+  const int count = __ldg(p.listoff + L + 1) - first;
+  const int start = (t - __ldg(p.tileoff + L)) * kTileRows;
+  ti.list = L;
+  ti.ent0 = first + start;
+  ti.rows = min(kTileRows, count - start);
+  ti.j = L % p.nblk;
+  ti.hk = (L / p.nblk) % p.hkv;
+  ti.b = (L / (p.nblk * p.hkv)) % p.batch;
+  ti.h = -1;
+  ti.nc = p.block / kTileKeys;
+}
+
+// Key of chunk m of a tile.
+template <int MODE>
+__device__ __forceinline__ int chunk_key(const AttnParams &p, const TileInfo &ti, int m) {
+  if (MODE == kGathered) return ti.j * p.block + m * kTileKeys;
+  return ti.key0 + m * kTileKeys;
+}
+
+// Operand descriptors.  Region 0 holds columns [0, 64) of a 128-row tile (128-byte
+// rows, 128-byte swizzle); region 1 holds columns [64, 128) the same way (D = 128) or
+// columns [64, 80) with 32-byte rows and 32-byte swizzle (D = 80).
+template <int D>
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int ks) {
+  if (ks < 4) return smem_desc(tile + ks * 32, 16, 1024, kSwizzle128);
+  if (D == 128) return smem_desc(tile + AttnCfg<D>::R0 + (ks - 4) * 32, 16, 1024, kSwizzle128);
+  return smem_desc(tile + AttnCfg<D>::R0, 16, 256, kSwizzle32);
+}
+
+// V as the MN-major B operand of O += P V: keys [16 kk, 16 kk + 16), columns of region
+// `rg` (64 columns with 128-byte swizzle, or 16 columns with 32-byte swizzle).
+template <int D>
+__device__ __forceinline__ uint64_t v_desc(uint32_t tile, int kk, int rg) {
+  if (rg == 0) return smem_desc(tile + kk * 2048, 16, 1024, kSwizzle128);
+  if (D == 128) return smem_desc(tile + AttnCfg<D>::R0 + kk * 2048, 16, 1024, kSwizzle128);
+  return smem_desc(tile + AttnCfg<D>::R0 + kk * 512, 16, 256, kSwizzle32);
+}
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ1,
+                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK1,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmV1,
+                const AttnParams p) {
+  using C = AttnCfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char *sbase = smem_raw + (base - raw);
+  Bars &bar = *reinterpret_cast<Bars *>(sbase + C::BAR_OFF);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int site0 = (MODE * 16 + (D == 64 ? 0 : (D == 80 ? 1 : 2))) * 256;
+
+  // Tile range.
+  int t_begin = 0, t_end = p.ntiles;
+  if (MODE == kGathered) {
+    t_begin = __ldg(p.tileoff + p.chunk * p.lists_per_chunk);
+    t_end = __ldg(p.tileoff + (p.chunk + 1) * p.lists_per_chunk);
+  }
+
+  if (tid == 0) {
+    mbar_init(&bar.q_full[0], MODE == kGathered ? 64 : 1);
+    mbar_init(&bar.q_full[1], MODE == kGathered ? 64 : 1);
+    mbar_init(&bar.q_empty[0], 1);
+    mbar_init(&bar.q_empty[1], 1);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(&bar.k_full[s], 1);
+      mbar_init(&bar.v_full[s], 1);
+      mbar_init(&bar.kv_empty[s], 1);
+    }
+    mbar_init(&bar.s_full[0], 1);
+    mbar_init(&bar.s_full[1], 1);
+    mbar_init(&bar.p_full, 128);
+    mbar_init(&bar.o_done, 1);
+    mbar_init(&bar.o_free, 128);
+    mbar_init(&bar.mma_done, 1);
+    bar.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    if (MODE == kQueryMajor) tma_prefetch_desc(&tmQ);
+  }
+  if (warp == 1) {
+    tmem_alloc(&bar.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+  volatile int *abort = &bar.abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t kvc = 0;
+      int lt = 0;
+      bool ok = true;
+      for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x, ++lt) {
+        TileInfo ti;
+        if (MODE == kGathered) gathered_tile(p, t, ti); else query_major_tile(p, t, ti);
+        if (MODE == kQueryMajor) {
+          const int qb = lt & 1;
+          if (!(ok = mbar_wait(&bar.q_empty[qb], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 1))) break;
+          const uint32_t qt = base + C::Q_OFF + qb * C::TILE;
+          mbar_arrive_expect_tx(&bar.q_full[qb], C::BYTES);
+          tma_load_4d(sbase + (qt - base), &tmQ, &bar.q_full[qb], 0, ti.i0, ti.h, ti.b);
+          if (D == 128) tma_load_4d(sbase + (qt - base) + C::R0, &tmQ1, &bar.q_full[qb], 64, ti.i0, ti.h, ti.b);
+          if (D == 80) tma_load_4d(sbase + (qt - base) + C::R0, &tmQ1, &bar.q_full[qb], 64, ti.i0, ti.h, ti.b);
+        }
+        for (int m = 0; m < ti.nc; ++m, ++kvc) {
+          const int st = kvc % C::ST;
+          if (!(ok = mbar_wait(&bar.kv_empty[st], ((kvc / C::ST) & 1) ^ 1, abort, p.status, site0 + 2))) break;
+          const int key = chunk_key<MODE>(p, ti, m);
+          unsigned char *kd = sbase + C::K_OFF + st * C::TILE;
+          unsigned char *vd = sbase + C::V_OFF + st * C::TILE;
+          mbar_arrive_expect_tx(&bar.k_full[st], C::BYTES);
+          tma_load_4d(kd, &tmK, &bar.k_full[st], 0, key, ti.hk, ti.b);
+          if (D != 64) tma_load_4d(kd + C::R0, &tmK1, &bar.k_full[st], 64, key, ti.hk, ti.b);
+          mbar_arrive_expect_tx(&bar.v_full[st], C::BYTES);
+          tma_load_4d(vd, &tmV, &bar.v_full[st], 0, key, ti.hk, ti.b);
+          if (D != 64) tma_load_4d(vd + C::R0, &tmV1, &bar.v_full[st], 64, key, ti.hk, ti.b);
+        }
+      }
+      // Let every load issued so far land before the CTA can retire.
+      if (*abort) {
+        for (uint32_t u = (kvc > (uint32_t)C::ST ? kvc - C::ST : 0); u < kvc; ++u) {
+          const int st = u % C::ST;
+          const unsigned long long t0 = global_timer_ns();
+          while (!mbar_try_wait(&bar.k_full[st], (u / C::ST) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+          while (!mbar_try_wait(&bar.v_full[st], (u / C::ST) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idO64 = idesc_bf16(128, 64, 0, 1);
+      constexpr uint32_t idO16 = idesc_bf16(128, 16, 0, 1);
+      const uint32_t tS[2] = {tmem, tmem + 128};
+      const uint32_t tO = tmem + 256;
+      uint32_t kvc = 0, scnt = 0, pcnt = 0, ofree = 0;
+      int lt = 0;
+      bool ok = true;
+      auto issue_pv = [&](int first, uint32_t sbuf, int st) {
+        const uint32_t vt = base + C::V_OFF + st * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+          const uint32_t a = sbuf + kk * 8;
+          umma_ts(tO, a, v_desc<D>(vt, kk, 0), idO64, acc);
+          if (D == 128) umma_ts(tO + 64, a, v_desc<D>(vt, kk, 1), idO64, acc);
+          if (D == 80) umma_ts(tO + 64, a, v_desc<D>(vt, kk, 1), idO16, acc);
+        }
+      };
+      for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x, ++lt) {
+        TileInfo ti;
+        if (MODE == kGathered) gathered_tile(p, t, ti); else query_major_tile(p, t, ti);
+        const int qb = lt & 1;
+        if (!(ok = mbar_wait(&bar.q_full[qb], (lt >> 1) & 1, abort, p.status, site0 + 3))) break;
+        tc_fence_after();
+        const uint32_t qt = base + C::Q_OFF + qb * C::TILE;
+        uint32_t prev_sbuf = 0;
+        int prev_st = 0;
+        for (int m = 0; m < ti.nc; ++m, ++kvc, ++scnt) {
+          const int st = kvc % C::ST;
+          if (!(ok = mbar_wait(&bar.k_full[st], (kvc / C::ST) & 1, abort, p.status, site0 + 4))) break;
+          tc_fence_after();
+          const uint32_t kt = base + C::K_OFF + st * C::TILE;
+          const uint32_t sb = tS[scnt & 1];
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            umma_ss(sb, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idS, ks > 0 ? 1u : 0u);
+          umma_commit(&bar.s_full[scnt & 1]);
+          if (m == ti.nc - 1) umma_commit(&bar.q_empty[qb]);
+          if (m > 0) {
+            if (!(ok = mbar_wait(&bar.p_full, pcnt & 1, abort, p.status, site0 + 5))) break;
+            ++pcnt;
+            if (!(ok = mbar_wait(&bar.v_full[prev_st], ((kvc - 1) / C::ST) & 1, abort, p.status, site0 + 6))) break;
+            if (m == 1) {
+              if (!(ok = mbar_wait(&bar.o_free, (ofree & 1) ^ 1, abort, p.status, site0 + 7))) break;
+              ++ofree;
+            }
+            tc_fence_after();
+            issue_pv(m == 1, prev_sbuf, prev_st);
+            umma_commit(&bar.o_done);
+            umma_commit(&bar.kv_empty[prev_st]);
+          }
+          prev_sbuf = sb;
+          prev_st = st;
+        }
+        if (!ok) break;
+        // PV of the last chunk.
+        if (!(ok = mbar_wait(&bar.p_full, pcnt & 1, abort, p.status, site0 + 8))) break;
+        ++pcnt;
+        if (!(ok = mbar_wait(&bar.v_full[prev_st], ((kvc - 1) / C::ST) & 1, abort, p.status, site0 + 9))) break;
+        if (ti.nc == 1) {
+          if (!(ok = mbar_wait(&bar.o_free, (ofree & 1) ^ 1, abort, p.status, site0 + 10))) break;
+          ++ofree;
+        }
+        tc_fence_after();
+        issue_pv(ti.nc == 1, prev_sbuf, prev_st);
+        umma_commit(&bar.o_done);
+        umma_commit(&bar.kv_empty[prev_st]);
+      }
+      // Every MMA issued so far completes before TMEM is released.
+      umma_commit(&bar.mma_done);
+      const unsigned long long t0 = global_timer_ns();
+      while (!mbar_try_wait(&bar.mma_done, 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------- row gather
+    if (MODE == kGathered) {
+      const int u = tid - 64;  // 0..63
+      constexpr int VPR = D / 8;  // 16-byte vectors per row
+      const int npast = p.npast;
+      int lt = 0;
+      for (int t = t_begin + blockIdx.x; t < t_end; t += gridDim.x, ++lt) {
+        TileInfo ti;
+        gathered_tile(p, t, ti);
+        const int qb = lt & 1;
+        if (!mbar_wait(&bar.q_empty[qb], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 11)) break;
+        const uint32_t qt = base + C::Q_OFF + qb * C::TILE;
+        for (int e = u; e < 128 * VPR; e += 64) {
+          const int r = e / VPR, c = e % VPR;
+          const bool valid = r < ti.rows;
+          const uint16_t *src = p.q;
+          if (valid) {
+            const uint32_t ent = __ldg(p.entries + ti.ent0 + r);
+            const uint32_t ig = ent / (uint32_t)npast;
+            const int g = (int)(ig % (uint32_t)p.G);
+            const int i = (int)(ig / (uint32_t)p.G);
+            src = p.q + ti.b * p.q_sb + (int64_t)(ti.hk * p.G + g) * p.q_sh + (int64_t)i * p.q_sn + c * 8;
+          }
+          uint32_t dst;
+          if (c < 8) {
+            dst = qt + r * 128 + ((c ^ (r & 7)) << 4);
+          } else if (D == 128) {
+            dst = qt + C::R0 + r * 128 + (((c - 8) ^ (r & 7)) << 4);
+          } else {
+            dst = qt + C::R0 + r * 32 + (((c - 8) ^ ((r >> 2) & 1)) << 4);
+          }
+          cp_async_16_zfill(dst, src, valid);
+        }
+        cp_async_commit();
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        mbar_arrive(&bar.q_full[qb]);
+      }
+    }
+  } else {
+    // ------------------------------------------- softmax + correction + epilogue
+    const int r = tid - 128;             // row within the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tS[2] = {tmem + lane_off, tmem + lane_off + 128};
+    const uint32_t tO = tmem + lane_off + 256;
+    const float sl2 = p.scale_log2;
+    uint32_t scnt = 0, ocnt = 0;
+    bool ok = true;
+    for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x) {
+      TileInfo ti;
+      if (MODE == kGathered) gathered_tile(p, t, ti); else query_major_tile(p, t, ti);
+      const bool live = r < ti.rows;
+      // Row identity.
+      int i = 0, h = ti.h, slot = 0;
+      if (MODE == kGathered) {
+        if (live) {
+          const uint32_t ent = __ldg(p.entries + ti.ent0 + r);
+          slot = (int)(ent % (uint32_t)p.npast);
+          const uint32_t ig = ent / (uint32_t)p.npast;
+          h = ti.hk * p.G + (int)(ig % (uint32_t)p.G);
+          i = (int)(ig / (uint32_t)p.G);
+        }
+      } else {
+        i = ti.i0 + r;
+      }
+      const int32_t *irow = (MODE == kQueryMajor && p.is_moba && live)
+                                ? p.idx + (((int64_t)ti.b * p.hq + h) * p.N + i) * p.topk
+                                : nullptr;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int m = 0; m < ti.nc; ++m, ++scnt) {
+        const int sbi = scnt & 1;
+        if (!(ok = mbar_wait(&bar.s_full[sbi], (scnt >> 1) & 1, abort, p.status, site0 + 12))) break;
+        tc_fence_after();
+        float s[128];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t v[32];
+          tmem_ld32(tS[sbi] + q4 * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) s[q4 * 32 + e] = __uint_as_float(v[e]);
+        }
+        // Masks.
+        const int key0 = chunk_key<MODE>(p, ti, m);
+        if (MODE == kQueryMajor) {
+          if (p.is_moba) {
+            if (m < ti.ntail) {
+              // Window tail into an earlier block: keys i - j < window that the row's
+              // own selection does not already cover.
+              bool covered = false;
+              if (irow) {
+                const int blk = key0 / p.block;
+                for (int u2 = 0; u2 < p.topk; ++u2) covered |= (__ldg(irow + u2) == blk);
+              }
+#pragma unroll
+              for (int e = 0; e < 128; ++e)
+                if (covered || !live || i - (key0 + e) >= p.window) s[e] = -INFINITY;
+            } else if (key0 + kTileKeys > ti.i0) {
+#pragma unroll
+              for (int e = 0; e < 128; ++e)
+                if (key0 + e > i) s[e] = -INFINITY;
+            }
+          } else {
+            const bool full = (key0 + kTileKeys - 1 <= ti.i0) &&
+                              (key0 >= ti.i0 + ti.rows - 1 - p.window + 1);
+            if (!full) {
+#pragma unroll
+              for (int e = 0; e < 128; ++e) {
+                const int j = key0 + e;
+                if (j > i || i - j >= p.window) s[e] = -INFINITY;
+              }
+            }
+          }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 128; ++e) mx = fmaxf(mx, s[e]);
+        const float m_new = fmaxf(m_run, mx * sl2);
+        if (m > 0) {
+          if (!(ok = mbar_wait(&bar.o_done, ocnt & 1, abort, p.status, site0 + 13))) break;
+          ++ocnt;
+          tc_fence_after();
+        }
+        if (m_new > m_run + (float)kRescaleThreshold || (m == 0)) {
+          if (m > 0 && m_run != -INFINITY) {
+            const float alpha = ex2_approx(m_run - m_new);
+            l_run *= alpha;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 16) {
+              uint32_t o[16];
+              tmem_ld16(tO + c0, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st16(tO + c0, o);
+            }
+          }
+          m_run = m_new;
+        }
+        const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+        float lsum = 0.f;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2_approx(fmaf(s[q4 * 32 + 2 * e], sl2, -mu));
+            const float p1 = ex2_approx(fmaf(s[q4 * 32 + 2 * e + 1], sl2, -mu));
+            lsum += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS[sbi] + q4 * 16, pk);
+        }
+        l_run += lsum;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar.p_full);
+      }
+      if (!ok) break;
+      // ------------------------------------------------------------ epilogue
+      if (!(ok = mbar_wait(&bar.o_done, ocnt & 1, abort, p.status, site0 + 14))) break;
+      ++ocnt;
+      tc_fence_after();
+      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      const float own_lse = (m_run + log2f(l_run)) * 0.69314718055994530942f;  // natural log
+      if (MODE == kGathered) {
+        if (live) {
+          const int il = i - p.chunk * p.chunk_rows;
+          const int64_t pidx = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + il) * p.npast + slot;
+          uint16_t *dst = p.opart + pidx * D;
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 16) {
+            uint32_t o[16];
+            tmem_ld16(tO + c0, o);
+            tmem_wait_ld();
+            uint4 w0, w1;
+            w0.x = pack_bf16x2(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l);
+            w0.y = pack_bf16x2(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l);
+            w0.z = pack_bf16x2(__uint_as_float(o[4]) * inv_l, __uint_as_float(o[5]) * inv_l);
+            w0.w = pack_bf16x2(__uint_as_float(o[6]) * inv_l, __uint_as_float(o[7]) * inv_l);
+            w1.x = pack_bf16x2(__uint_as_float(o[8]) * inv_l, __uint_as_float(o[9]) * inv_l);
+            w1.y = pack_bf16x2(__uint_as_float(o[10]) * inv_l, __uint_as_float(o[11]) * inv_l);
+            w1.z = pack_bf16x2(__uint_as_float(o[12]) * inv_l, __uint_as_float(o[13]) * inv_l);
+            w1.w = pack_bf16x2(__uint_as_float(o[14]) * inv_l, __uint_as_float(o[15]) * inv_l);
+            *reinterpret_cast<uint4 *>(dst + c0) = w0;
+            *reinterpret_cast<uint4 *>(dst + c0 + 8) = w1;
+          }
+          p.lpart[pidx] = own_lse;
+        }
+      } else if (live) {
+        // Merge with the past-block partials of this row (MoBA), then store.
+        float wown = 1.f, lse = own_lse;
+        int np = 0;
+        int64_t pbase = 0;
+        float wp[32];
+        if (p.is_moba && p.npast > 0) {
+          const int c = i / p.block;
+          for (int s2 = 0; s2 < p.npast; ++s2) {
+            const int blk = __ldg(irow + s2);
+            if (blk < 0 || blk >= c) break;
+            ++np;
+          }
+          if (np > 0) {
+            const int il = i - p.chunk * p.chunk_rows;
+            pbase = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + il) * p.npast;
+            float mx = own_lse;
+            for (int s2 = 0; s2 < np; ++s2) mx = fmaxf(mx, p.lpart[pbase + s2]);
+            float tot = __expf(own_lse - mx);
+            for (int s2 = 0; s2 < np; ++s2) tot += __expf(p.lpart[pbase + s2] - mx);
+            lse = mx + __logf(tot);
+            wown = __expf(own_lse - lse);
+            for (int s2 = 0; s2 < np; ++s2) wp[s2] = __expf(p.lpart[pbase + s2] - lse);
+          }
+        }
+        uint16_t *dst = p.out + ti.b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)i * p.o_sn;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 16) {
+          uint32_t o[16];
+          tmem_ld16(tO + c0, o);
+          tmem_wait_ld();
+          float acc[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[e]) * inv_l * wown;
+          for (int s2 = 0; s2 < np; ++s2) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.opart + (pbase + s2) * D + c0);
+            const uint4 a0 = src[0], a1 = src[1];
+            const uint32_t wv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              acc[2 * e] += wp[s2] * __uint_as_float(wv[e] << 16);
+              acc[2 * e + 1] += wp[s2] * __uint_as_float(wv[e] & 0xFFFF0000u);
+            }
+          }
+          uint4 w0, w1;
+          w0.x = pack_bf16x2(acc[0], acc[1]);
+          w0.y = pack_bf16x2(acc[2], acc[3]);
+          w0.z = pack_bf16x2(acc[4], acc[5]);
+          w0.w = pack_bf16x2(acc[6], acc[7]);
+          w1.x = pack_bf16x2(acc[8], acc[9]);
+          w1.y = pack_bf16x2(acc[10], acc[11]);
+          w1.z = pack_bf16x2(acc[12], acc[13]);
+          w1.w = pack_bf16x2(acc[14], acc[15]);
+          *reinterpret_cast<uint4 *>(dst + c0) = w0;
+          *reinterpret_cast<uint4 *>(dst + c0 + 8) = w1;
+        }
+        p.lse[((int64_t)ti.b * p.hq + h) * p.N + i] = lse;
+      }
+      tc_fence_before();
+      mbar_arrive(&bar.o_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ launch
+
+template <int D, int MODE>
+static cudaError_t launch_attn_dm(const CUtensorMap *maps, const AttnParams &p, int grid,
+                                  cudaStream_t st) {
+  using C = AttnCfg<D>;
+  auto kern = attn_fwd_kernel<D, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kAttnThreads, C::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
+  return cudaGetLastError();
+}
+
+// maps: Q (64-col box), Q tail, K, K tail, V, V tail.
+cudaError_t launch_attn(const CUtensorMap *maps, const AttnParams &p, int mode, int grid,
+                        cudaStream_t st) {
+  if (mode == kQueryMajor) {
+    switch (p.d) {
+      case 64: return launch_attn_dm<64, kQueryMajor>(maps, p, grid, st);
+      case 80: return launch_attn_dm<80, kQueryMajor>(maps, p, grid, st);
+      case 128: return launch_attn_dm<128, kQueryMajor>(maps, p, grid, st);
+    }
+  } else {
+    switch (p.d) {
+      case 64: return launch_attn_dm<64, kGathered>(maps, p, grid, st);
+      case 80: return launch_attn_dm<80, kGathered>(maps, p, grid, st);
+      case 128: return launch_attn_dm<128, kGathered>(maps, p, grid, st);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+int attn_smem_bytes(int d) {
+  switch (d) {
+    case 64: return AttnCfg<64>::SMEM;
+    case 80: return AttnCfg<80>::SMEM;
+    case 128: return AttnCfg<128>::SMEM;
+  }
+  return 0;
+}
+
+}  // namespace moba

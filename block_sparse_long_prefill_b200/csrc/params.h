@@ -1,0 +1,114 @@
+// params.h -- problem description, workspace layout and kernel parameter blocks
+// shared by the host-side ABI and the kernels.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moba {
+
+constexpr int kTileRows = 128;   // query rows per attention tile (tcgen05 M)
+constexpr int kTileKeys = 128;   // keys per attention chunk (tcgen05 N of S = QK^T)
+constexpr size_t kPartialCapBytes = size_t(4) << 30;  // partial outputs kept per pass
+
+// Block-major dispatch lists and partial outputs, carved out of the caller's workspace.
+// List L = ((chunk * batch + b) * hkv + hk) * nblk + j holds the (row, q-head, slot)
+// triples of the rows of query chunk `chunk` that picked past block j.
+struct WorkspaceLayout {
+  int nblk;         // N / block
+  int G;            // hq / hkv
+  int npast;        // topk - 1: partial slots per row
+  int chunk_rows;   // query rows per pass (multiple of 128)
+  int nchunks;
+  int nlists;       // nchunks * batch * hkv * nblk
+  size_t off_counts;   // int32 [nlists]       entries per list (atomic counts)
+  size_t off_cursor;   // int32 [nlists]       scatter cursors
+  size_t off_listoff;  // int32 [nlists + 1]   exclusive prefix of counts
+  size_t off_tileoff;  // int32 [nlists + 1]   exclusive prefix of ceil(count / 128)
+  size_t off_entries;  // uint32 [max_entries] entry = (i * G + g) * npast + slot
+  size_t off_opart;    // bf16 [batch, hq, chunk_rows, npast, d]
+  size_t off_lpart;    // f32  [batch, hq, chunk_rows, npast]
+  size_t total;
+  long long max_entries;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline WorkspaceLayout make_layout(int batch, int hq, int hkv, int N, int d, int block,
+                                   int topk) {
+  WorkspaceLayout w{};
+  w.nblk = N / block;
+  w.G = hq / hkv;
+  w.npast = topk - 1;
+  const size_t per_row = size_t(w.npast) * (size_t(d) * 2 + 4) * size_t(batch) * size_t(hq);
+  long long rows = N;
+  if (per_row > 0 && per_row * size_t(N) > kPartialCapBytes) {
+    rows = static_cast<long long>(kPartialCapBytes / per_row) / kTileRows * kTileRows;
+    if (rows < kTileRows) rows = kTileRows;
+  }
+  w.chunk_rows = static_cast<int>(rows);
+  w.nchunks = static_cast<int>((N + w.chunk_rows - 1) / w.chunk_rows);
+  w.nlists = w.nchunks * batch * hkv * w.nblk;
+  w.max_entries = static_cast<long long>(batch) * hq * N * w.npast;
+  size_t off = 0;
+  w.off_counts = off;  off = align_up(off + sizeof(int) * size_t(w.nlists), 256);
+  w.off_cursor = off;  off = align_up(off + sizeof(int) * size_t(w.nlists), 256);
+  w.off_listoff = off; off = align_up(off + sizeof(int) * size_t(w.nlists + 1), 256);
+  w.off_tileoff = off; off = align_up(off + sizeof(int) * size_t(w.nlists + 1), 256);
+  w.off_entries = off; off = align_up(off + sizeof(uint32_t) * size_t(w.max_entries), 256);
+  const size_t prow = size_t(batch) * hq * size_t(w.chunk_rows) * size_t(w.npast);
+  w.off_opart = off;   off = align_up(off + prow * size_t(d) * 2, 256);
+  w.off_lpart = off;   off = align_up(off + prow * sizeof(float), 256);
+  w.total = off;
+  return w;
+}
+
+// Parameters of the gate / top-k kernel.
+struct SelectParams {
+  const uint16_t *q;     // bf16 bits
+  int64_t q_sb, q_sh, q_sn;
+  const uint16_t *kbar_split;  // [batch, hkv, 2, nblk, d]
+  int32_t *idx;          // [batch, hq, N, topk]
+  int *counts;           // workspace list counts
+  int batch, hq, hkv, N, d, block, topk, nblk, G, chunk_rows;
+};
+
+struct ScatterParams {
+  const int32_t *idx;
+  int *cursor;
+  uint32_t *entries;
+  int batch, hq, hkv, N, block, topk, nblk, G, chunk_rows;
+};
+
+// Attention kernel modes.
+enum AttnMode : int {
+  kQueryMajor = 0,  // contiguous 128-row query tiles: own block (MoBA) or band (SWA)
+  kGathered = 1,    // gathered rows of one block-major list against one whole block
+};
+
+struct AttnParams {
+  int *status;             // device status words (see common.cuh)
+  // Tensors (bf16 bits) and strides in elements.
+  const uint16_t *q;
+  int64_t q_sb, q_sh, q_sn;
+  uint16_t *out;
+  int64_t o_sb, o_sh, o_sn;
+  float *lse;              // [batch, hq, N]
+  const int32_t *idx;      // [batch, hq, N, topk] (MoBA) or null (SWA)
+  // Problem.
+  int batch, hq, hkv, N, d, block, topk, window, G;
+  float scale_log2;        // scale * log2(e)
+  int is_moba;             // 0: sliding window only (swa_attn_fwd)
+  // Query-major pass: row range of this pass.
+  int row_begin, row_end;  // multiples of 128 except row_end == N
+  int ntiles;              // query-major tiles in this pass
+  // Block-major lists and partials (MoBA).
+  const int *listoff;
+  const int *tileoff;
+  const uint32_t *entries;
+  uint16_t *opart;         // [batch, hq, chunk_rows, npast, d]
+  float *lpart;            // [batch, hq, chunk_rows, npast]
+  int chunk, chunk_rows, npast, nblk, lists_per_chunk;
+};
+
+}  // namespace moba

@@ -1,0 +1,436 @@
+// select.cu -- MoBA selection stage on sm_100a: key mean-pooling, gate scores with
+// causal block masking, per-row top-k, and the block-major dispatch lists.
+//
+// [MoBA] = "MoBA: 어텐션에 전문가 혼합을 적용해 긴 문맥을 효율적으로 처리하는 블록 어텐션
+//          (feat. MoonshotAI)", PyTorch KR forum summary of the MoBA paper.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "params.h"
+
+namespace moba {
+
+// ------------------------------------------------------------------ pooling
+//
+// [MoBA] §"블록 분할과 top-k 게이팅": MeanPool(K[I_j]) over the keys of block j.
+// One CTA per (block, kv-head, batch).  Threads read 16-byte vectors along d
+// (coalesced rows), accumulate in fp32, and reduce across row groups in a fixed
+// order (deterministic).  Also writes the split hi = bf16(mean), lo = bf16(mean - hi)
+// that the gate multiplies with on the tensor cores.
+constexpr int kPoolThreads = 256;
+
+__global__ void __launch_bounds__(kPoolThreads)
+pool_keys_kernel(const uint16_t *__restrict__ k, int64_t sb, int64_t sh, int64_t sn, int hkv,
+                 int d, int block, int nblk, float *__restrict__ kbar,
+                 uint16_t *__restrict__ split) {
+  extern __shared__ float red[];  // [ngroups][d]
+  const int j = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int vpr = d >> 3;                   // 16-byte vectors per key row
+  const int ngroups = kPoolThreads / vpr;   // rows read concurrently
+  const int t = threadIdx.x;
+  const int vec = t % vpr, grp = t / vpr;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  if (grp < ngroups) {
+    const uint16_t *base = k + b * sb + hk * sh + (int64_t)j * block * sn + vec * 8;
+    int r = grp;
+    for (; r + 3 * ngroups < block; r += 4 * ngroups) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        v[u] = __ldg(reinterpret_cast<const uint4 *>(base + (int64_t)(r + u * ngroups) * sn));
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[2 * e] += __uint_as_float(w[e] << 16);
+          acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+        }
+      }
+    }
+    for (; r < block; r += ngroups) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(base + (int64_t)r * sn));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += __uint_as_float(w[e] << 16);
+        acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[grp * d + vec * 8 + e] = acc[e];
+  }
+  __syncthreads();
+  const int64_t bh = (int64_t)b * hkv + hk;
+  for (int c = t; c < d; c += kPoolThreads) {
+    float s = 0.f;
+    for (int g = 0; g < ngroups; ++g) s += red[g * d + c];
+    const float mean = s / (float)block;
+    kbar[(bh * nblk + j) * d + c] = mean;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(mean);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(mean - __bfloat162float(hi));
+    uint16_t *sp = split + bh * 2 * (int64_t)nblk * d;
+    sp[(int64_t)j * d + c] = __bfloat16_as_ushort(hi);
+    sp[((int64_t)nblk + j) * d + c] = __bfloat16_as_ushort(lo);
+  }
+}
+
+// ------------------------------------------------------------ gate + top-k
+//
+// [MoBA] §"블록 분할과 top-k 게이팅": s_j = <q, MeanPool(K[I_j])>, unscaled;
+// §"인과성 보존": only blocks j < c = i / block compete, block c is always kept.
+// One CTA = 64 query rows of one (batch, q-head); 4 warps of 16 rows.
+//
+// Scores come from bf16 tensor-core MMAs (mma.sync m16n8k16, fp32 accumulate):
+// q is exactly bf16, and kbar = hi + lo to about 2^-17 relative, so
+// s = q.hi + q.lo is fp32-accurate -- far inside the 1e-3 gate-gap tolerance.
+// The selection is k-1 rounds of a quad-wide arg-max over the row's scores in
+// shared memory (ties to the lower block), then a rank placement into ascending
+// order.  Each CTA also counts its picks per past block (shared-memory histogram,
+// one global atomic per non-empty block) for the dispatch lists.
+constexpr int kGateRows = 64;
+constexpr int kGateThreads = 128;
+constexpr int kGateChunk = 32;  // pooled blocks staged per pass
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t &r0, uint32_t &r1,
+                                            uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kGateThreads)
+gate_topk_kernel(const SelectParams p) {
+  constexpr int KS = D / 16;           // k-steps
+  constexpr int LDQ = D + 8;           // padded row stride (elements): conflict-free ldmatrix
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint16_t *qs = reinterpret_cast<uint16_t *>(smem);                       // [64][LDQ]
+  uint16_t *ks = qs + kGateRows * LDQ;                                     // [2][2][32][LDQ]
+  float *ss = reinterpret_cast<float *>(ks + 2 * 2 * kGateChunk * LDQ);    // [64][lds]
+  const int i0 = blockIdx.x * kGateRows;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / p.G;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rows = min(kGateRows, p.N - i0);
+  // Past blocks any row of this tile may score.
+  const int nb = min(p.nblk, (i0 + rows - 1) / p.block);
+  const int lds = ((nb + 31) & ~31) + 4;
+  int *hist = reinterpret_cast<int *>(ss + kGateRows * lds);               // [nblk]
+
+  // Stage the query tile and the first chunk of pooled keys.
+  const uint16_t *qg = p.q + b * p.q_sb + h * p.q_sh;
+  for (int e = tid; e < kGateRows * (D / 8); e += kGateThreads) {
+    const int r = e / (D / 8), c = e % (D / 8);
+    const bool ok = r < rows;
+    cp_async_16_zfill(smem_u32(qs + r * LDQ + c * 8), qg + (int64_t)(ok ? i0 + r : i0) * p.q_sn + c * 8, ok);
+  }
+  const uint16_t *kb = p.kbar_split + ((int64_t)b * p.hkv + hk) * 2 * p.nblk * D;
+  auto stage_chunk = [&](int ch, int buf) {
+    const int j0 = ch * kGateChunk;
+    for (int e = tid; e < 2 * kGateChunk * (D / 8); e += kGateThreads) {
+      const int part = e / (kGateChunk * (D / 8));
+      const int rem = e % (kGateChunk * (D / 8));
+      const int jj = rem / (D / 8), c = rem % (D / 8);
+      const bool ok = j0 + jj < nb;
+      const uint16_t *src = kb + ((int64_t)part * p.nblk + (ok ? j0 + jj : 0)) * D + c * 8;
+      cp_async_16_zfill(smem_u32(ks + ((buf * 2 + part) * kGateChunk + jj) * LDQ + c * 8), src, ok);
+    }
+  };
+  const int nchunk = (nb + kGateChunk - 1) / kGateChunk;
+  if (nchunk > 0) stage_chunk(0, 0);
+  cp_async_commit();
+  for (int j = tid; j < p.nblk; j += kGateThreads) hist[j] = 0;
+
+  const int wr0 = warp * 16;  // this warp's first row in the tile
+  const int g = lane >> 2, t4 = lane & 3;
+  // Largest own-block index among this warp's rows: n-tiles at or past it are skipped.
+  const int wlast = min(i0 + wr0 + 15, p.N - 1);
+  const int cw = (wr0 < rows) ? wlast / p.block : 0;
+
+  uint32_t afrag[KS][4];
+  for (int ch = 0; ch < nchunk; ++ch) {
+    if (ch + 1 < nchunk) stage_chunk(ch + 1, (ch + 1) & 1);
+    cp_async_commit();
+    cp_async_wait_group<1>();
+    __syncthreads();
+    if (ch == 0) {
+#pragma unroll
+      for (int s = 0; s < KS; ++s) {
+        const int r = wr0 + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int c = s * 16 + 8 * (lane >> 4);
+        ldmatrix_x4(smem_u32(qs + r * LDQ + c), afrag[s][0], afrag[s][1], afrag[s][2], afrag[s][3]);
+      }
+    }
+    const int buf = ch & 1;
+    const int j0 = ch * kGateChunk;
+#pragma unroll
+    for (int nt = 0; nt < kGateChunk / 8; ++nt) {
+      if (j0 + nt * 8 >= cw) break;  // every row of the warp has c <= these blocks
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < KS; ++s) {
+        // Matrices: (hi, k0..7), (hi, k8..15), (lo, k0..7), (lo, k8..15) for 8 blocks.
+        const int part = (lane >> 4) & 1;
+        const int jj = nt * 8 + (lane & 7);
+        const int c = s * 16 + 8 * ((lane >> 3) & 1);
+        uint32_t h0, h1, l0, l1;
+        ldmatrix_x4(smem_u32(ks + ((buf * 2 + part) * kGateChunk + jj) * LDQ + c), h0, h1, l0, l1);
+        mma_bf16_16816(acc, afrag[s], h0, h1);
+        mma_bf16_16816(acc, afrag[s], l0, l1);
+      }
+      const int col = j0 + nt * 8 + 2 * t4;
+      ss[(wr0 + g) * lds + col] = acc[0];
+      ss[(wr0 + g) * lds + col + 1] = acc[1];
+      ss[(wr0 + g + 8) * lds + col] = acc[2];
+      ss[(wr0 + g + 8) * lds + col + 1] = acc[3];
+    }
+    __syncthreads();
+  }
+  cp_async_wait_all();
+  __syncthreads();
+
+  // Top-(k-1) over past blocks; one quad of lanes per row, two passes of 8 rows.
+  // Every lane runs the warp's largest round count so the shuffles stay converged.
+  const int npick_max = p.topk - 1;
+  int *sel_base = reinterpret_cast<int *>(qs);  // reuses the query tile: [64][32]
+  for (int pass = 0; pass < 2; ++pass) {
+    const int r = wr0 + pass * 8 + g;
+    const int i = i0 + r;
+    const bool live = r < rows;
+    const int c = live ? i / p.block : 0;
+    float *srow = ss + r * lds;
+    int *sel = sel_base + r * 32;
+    const int npick = min(npick_max, c);
+    const int rounds = (live && c > npick_max) ? npick : 0;
+    const int wrounds = __reduce_max_sync(0xffffffffu, rounds);
+    for (int round = 0; round < wrounds; ++round) {
+      float best = -INFINITY;
+      int bj = 0x7fffffff;
+      if (round < rounds) {
+        for (int j = t4; j < c; j += 4) {
+          const float v = srow[j];
+          if (v > best) { best = v; bj = j; }
+        }
+      }
+#pragma unroll
+      for (int off = 1; off <= 2; off <<= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+        const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
+        if (ob > best || (ob == best && oj < bj)) { best = ob; bj = oj; }
+      }
+      if (round < rounds) {
+        if (bj != 0x7fffffff && (bj & 3) == t4) srow[bj] = -INFINITY;
+        if (t4 == 0) sel[round] = bj;
+      }
+      __syncwarp();
+    }
+    __syncwarp();
+    if (live) {
+      int32_t *orow = p.idx + (((int64_t)b * p.hq + h) * p.N + i) * p.topk;
+      if (c <= npick_max) {
+        for (int s = t4; s < p.topk; s += 4) orow[s] = (s < c) ? s : (s == c ? c : -1);
+        for (int j = t4; j < c; j += 4) atomicAdd(&hist[j], 1);
+      } else {
+        for (int s = t4; s < npick; s += 4) {
+          const int v = sel[s];
+          int rank = 0;
+          for (int u = 0; u < npick; ++u) rank += sel[u] < v;
+          orow[rank] = v;
+          atomicAdd(&hist[v], 1);
+        }
+        if (t4 == 0) orow[npick] = c;
+        for (int s = npick + 1 + t4; s < p.topk; s += 4) orow[s] = -1;
+      }
+    }
+  }
+  __syncthreads();
+  // One global atomic per (list, CTA).
+  const int chunk = i0 / p.chunk_rows;
+  int *cnt = p.counts + (((int64_t)chunk * p.batch + b) * p.hkv + hk) * p.nblk;
+  for (int j = tid; j < nb; j += kGateThreads)
+    if (hist[j]) atomicAdd(&cnt[j], hist[j]);
+}
+
+// ------------------------------------------------------------- list offsets
+//
+// Exclusive prefix sums of the list counts (entries) and of their 128-row tiles,
+// over all lists in (chunk, batch, kv-head, block) order; resets the scatter
+// cursors.  One CTA.
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads)
+list_scan_kernel(const int *__restrict__ counts, int *__restrict__ cursor, int *__restrict__ listoff,
+                 int *__restrict__ tileoff, int nlists) {
+  __shared__ int warp_e[32], warp_t[32];
+  __shared__ int carry_e, carry_t;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) { carry_e = 0; carry_t = 0; }
+  __syncthreads();
+  for (int base = 0; base < nlists; base += kScanThreads) {
+    const int L = base + tid;
+    const int ce = (L < nlists) ? counts[L] : 0;
+    const int ct = (ce + kTileRows - 1) / kTileRows;
+    int se = ce, st = ct;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int ye = __shfl_up_sync(0xffffffffu, se, off);
+      const int yt = __shfl_up_sync(0xffffffffu, st, off);
+      if (lane >= off) { se += ye; st += yt; }
+    }
+    if (lane == 31) { warp_e[warp] = se; warp_t[warp] = st; }
+    __syncthreads();
+    if (warp == 0) {
+      int we = warp_e[lane], wt = warp_t[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int ye = __shfl_up_sync(0xffffffffu, we, off);
+        const int yt = __shfl_up_sync(0xffffffffu, wt, off);
+        if (lane >= off) { we += ye; wt += yt; }
+      }
+      warp_e[lane] = we;  // inclusive per-warp totals
+      warp_t[lane] = wt;
+    }
+    __syncthreads();
+    const int pe = carry_e + (warp ? warp_e[warp - 1] : 0) + se - ce;
+    const int pt = carry_t + (warp ? warp_t[warp - 1] : 0) + st - ct;
+    if (L < nlists) {
+      listoff[L] = pe;
+      cursor[L] = pe;
+      tileoff[L] = pt;
+    }
+    __syncthreads();
+    if (tid == kScanThreads - 1) {
+      carry_e = pe + ce;
+      carry_t = pt + ct;
+    }
+    __syncthreads();
+  }
+  if (tid == 0) {
+    listoff[nlists] = carry_e;
+    tileoff[nlists] = carry_t;
+  }
+}
+
+// ----------------------------------------------------------------- scatter
+//
+// [MoBA] §"MoBA의 구현", steps 1-2: assign each (query, q-head) to the KV blocks it
+// picked and regroup the queries by block.  One CTA = 128 rows x all G q-heads of one
+// kv-head.  Entries of one CTA reserve their places with one atomic per block.
+// The order of entries inside a list is not fixed; no result depends on it (each
+// row's attention is computed independently of the rows sharing its tile).
+constexpr int kScatterThreads = 256;
+
+__global__ void __launch_bounds__(kScatterThreads)
+scatter_kernel(const ScatterParams p) {
+  extern __shared__ int sh[];
+  int *hist = sh;             // [nblk]
+  int *base = sh + p.nblk;    // [nblk]
+  const int i0 = blockIdx.x * kTileRows;
+  const int hk = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x;
+  const int npast = p.topk - 1;
+  const int rows = min(kTileRows, p.N - i0);
+  const int nb = min(p.nblk, (i0 + rows - 1) / p.block);
+  for (int j = tid; j < nb; j += kScatterThreads) hist[j] = 0;
+  __syncthreads();
+  const int pairs = p.G * kTileRows;
+  for (int e = tid; e < pairs; e += kScatterThreads) {
+    const int g = e / kTileRows, r = e % kTileRows;
+    if (r >= rows) continue;
+    const int i = i0 + r;
+    const int c = i / p.block;
+    const int32_t *row = p.idx + (((int64_t)b * p.hq + hk * p.G + g) * p.N + i) * p.topk;
+    for (int s = 0; s < npast; ++s) {
+      const int j = row[s];
+      if (j < 0 || j >= c) break;  // own block (last) or padding
+      atomicAdd(&hist[j], 1);
+    }
+  }
+  __syncthreads();
+  const int chunk = i0 / p.chunk_rows;
+  int *cur = p.cursor + (((int64_t)chunk * p.batch + b) * p.hkv + hk) * p.nblk;
+  for (int j = tid; j < nb; j += kScatterThreads) {
+    base[j] = hist[j] ? atomicAdd(&cur[j], hist[j]) : 0;
+    hist[j] = 0;
+  }
+  __syncthreads();
+  for (int e = tid; e < pairs; e += kScatterThreads) {
+    const int g = e / kTileRows, r = e % kTileRows;
+    if (r >= rows) continue;
+    const int i = i0 + r;
+    const int c = i / p.block;
+    const int32_t *row = p.idx + (((int64_t)b * p.hq + hk * p.G + g) * p.N + i) * p.topk;
+    for (int s = 0; s < npast; ++s) {
+      const int j = row[s];
+      if (j < 0 || j >= c) break;
+      const int pos = base[j] + atomicAdd(&hist[j], 1);
+      p.entries[pos] = (uint32_t)(((int64_t)i * p.G + g) * npast + s);
+    }
+  }
+}
+
+// Host-side launchers (called by the ABI layer).
+cudaError_t launch_pool(const uint16_t *k, int64_t sb, int64_t sh, int64_t sn, int batch, int hkv,
+                        int N, int d, int block, float *kbar, uint16_t *split, cudaStream_t st) {
+  const int nblk = N / block;
+  const int ngroups = kPoolThreads / (d / 8);
+  const size_t smem = sizeof(float) * ngroups * d;
+  dim3 grid(nblk, hkv, batch);
+  pool_keys_kernel<<<grid, kPoolThreads, smem, st>>>(k, sb, sh, sn, hkv, d, block, nblk, kbar, split);
+  return cudaGetLastError();
+}
+
+size_t gate_smem_bytes(int d, int nblk) {
+  const int ldq = d + 8;
+  const int lds = ((nblk + 31) & ~31) + 4;
+  return sizeof(uint16_t) * (kGateRows * ldq + 2 * 2 * kGateChunk * ldq) +
+         sizeof(float) * kGateRows * lds + sizeof(int) * nblk;
+}
+
+template <int D>
+static cudaError_t launch_gate_d(const SelectParams &p, cudaStream_t st) {
+  const size_t smem = gate_smem_bytes(D, p.nblk);
+  cudaError_t e = cudaFuncSetAttribute(gate_topk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((p.N + kGateRows - 1) / kGateRows, p.hq, p.batch);
+  gate_topk_kernel<D><<<grid, kGateThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate(const SelectParams &p, cudaStream_t st) {
+  switch (p.d) {
+    case 64: return launch_gate_d<64>(p, st);
+    case 80: return launch_gate_d<80>(p, st);
+    case 128: return launch_gate_d<128>(p, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileoff, int nlists,
+                        cudaStream_t st) {
+  list_scan_kernel<<<1, kScanThreads, 0, st>>>(counts, cursor, listoff, tileoff, nlists);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter(const ScatterParams &p, cudaStream_t st) {
+  dim3 grid((p.N + kTileRows - 1) / kTileRows, p.hkv, p.batch);
+  const size_t smem = sizeof(int) * 2 * p.nblk;
+  scatter_kernel<<<grid, kScatterThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace moba

@@ -1,0 +1,142 @@
+/*
+ * moba.h -- C ABI of libmoba: MoBA block-sparse attention prefill and sliding-window
+ * attention prefill on NVIDIA B200 (sm_100a).
+ *
+ * The method (cited by page title and section):
+ *   [MoBA] "MoBA: 어텐션에 전문가 혼합을 적용해 긴 문맥을 효율적으로 처리하는 블록 어텐션
+ *          (feat. MoonshotAI)", PyTorch KR forum summary of the MoBA paper.
+ *   [SWA]  "SWA + MoE: 어텐션과 희소 전문가", Bit-Axon architecture page.
+ *
+ * A MoBA prefill is three calls on one stream, in this order:
+ *   moba_pool_keys   -> pooled block keys
+ *   moba_select_topk -> per-row block choices (idx) + block-major dispatch lists in
+ *                       the workspace
+ *   moba_attn_fwd    -> out and per-row log-sum-exp, reading the dispatch lists
+ * swa_attn_fwd is independent (the window-only special case).
+ *
+ * Conventions shared by every call:
+ *   - Tensors are device pointers described by moba_tensor: element (b, h, n, 0) sits
+ *     at ptr + b*sb + h*sh + n*sn (strides in elements); the head dimension d is
+ *     contiguous.  ptr and every stride times the element size must be multiples of
+ *     16 bytes.  q is [batch, hq, N, d]; k, v are [batch, hkv, N, d]; out is
+ *     [batch, hq, N, d]; all bf16.
+ *   - GQA: query head h reads KV head h / (hq / hkv).
+ *   - Block j covers key positions [j*block, (j+1)*block) (0-based; the MoBA page
+ *     numbers blocks from 1).  N must be a multiple of block, and block a multiple
+ *     of 128.
+ *   - d must be 64, 80 or 128 for the attention calls (any multiple of 8 up to 256
+ *     for moba_pool_keys and moba_select_topk).
+ *   - Ownership: the caller allocates every buffer (inputs, outputs, workspace); the
+ *     library allocates no device memory and keeps no state between calls.
+ *   - Execution: every call only enqueues kernels on `stream` (a cudaStream_t, 0 for
+ *     the legacy default stream) and returns; nothing synchronises.
+ *   - Errors: calls return MOBA_OK (0) or a negative MOBA_ERR_* code.  Argument
+ *     errors are detected on the host before anything is launched.  Kernel waits are
+ *     bounded: a wait that runs out records MOBA_ERR_DEVICE in a device-side status
+ *     word that moba_device_status() reads.
+ */
+#ifndef MOBA_H
+#define MOBA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOBA_OK 0
+#define MOBA_ERR_SHAPE -1     /* N % block, hq % hkv, block % 128, sizes out of range */
+#define MOBA_ERR_DIM -2       /* unsupported head dimension */
+#define MOBA_ERR_ALIGN -3     /* pointer or stride not 16-byte aligned */
+#define MOBA_ERR_ARG -4       /* topk < 1, window < 0, null pointer, ... */
+#define MOBA_ERR_WORKSPACE -5 /* workspace missing or too small */
+#define MOBA_ERR_LAUNCH -6    /* a CUDA launch or driver call failed */
+#define MOBA_ERR_DEVICE -7    /* a kernel wait ran out (see moba_device_status) */
+#define MOBA_ERR_NODEVICE -8  /* no sm_100 device is current */
+
+typedef struct {
+    void *ptr;
+    int64_t sb, sh, sn; /* strides in elements for batch, head and position */
+} moba_tensor;
+
+/*
+ * Bytes of workspace that moba_select_topk and moba_attn_fwd need for this problem.
+ * The workspace holds the block-major dispatch lists that moba_select_topk writes
+ * and moba_attn_fwd reads, and the per-(row, past block) partial outputs that
+ * moba_attn_fwd merges.  Host-only; launches nothing.
+ */
+int moba_workspace_size(int batch, int hq, int hkv, int N, int d, int block, int topk,
+                        size_t *bytes);
+
+/*
+ * [MoBA] §"블록 분할과 top-k 게이팅": MeanPool(K[I_j]) for every block j.
+ *   k          : bf16 keys [batch, hkv, N, d]
+ *   kbar       : float32 out [batch, hkv, N/block, d], contiguous: the block means
+ *   kbar_split : bf16 out [batch, hkv, 2, N/block, d], contiguous: hi = bf16(kbar)
+ *                and lo = bf16(kbar - hi), the two bf16 terms the gate multiplies by
+ */
+int moba_pool_keys(moba_tensor k, int batch, int hkv, int N, int d, int block, float *kbar,
+                   void *kbar_split, void *stream);
+
+/*
+ * [MoBA] §"블록 분할과 top-k 게이팅" and §"인과성 보존": for every query row i (block
+ * c = i / block) score the past blocks j < c with s_j = <q_i, kbar_j> (no scale),
+ * keep the own block c and the topk-1 best past blocks (ties to the lower j; all
+ * past blocks when c <= topk-1), then build the block-major dispatch lists of
+ * §"MoBA의 구현" (steps 1-2: assign queries to KV blocks, regroup by block).
+ *   q          : bf16 queries [batch, hq, N, d]
+ *   kbar_split : as written by moba_pool_keys
+ *   idx        : int32 out [batch, hq, N, topk], contiguous: the kept blocks in
+ *                ascending order (the own block last), -1 padded
+ *   workspace  : device buffer of at least moba_workspace_size() bytes; receives
+ *                the dispatch lists
+ */
+int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, int hkv, int N,
+                     int d, int block, int topk, int32_t *idx, void *workspace,
+                     size_t workspace_bytes, void *stream);
+
+/*
+ * [MoBA] §"표준 어텐션에서 블록 어텐션으로" and §"MoBA의 구현": out_i =
+ * Softmax(scale q_i K[J_i]^T) V[J_i] with J_i = { j <= i : j / block in idx[i] },
+ * unioned with the causal window { j : 0 <= i - j < window } when window > 0.
+ * Past blocks are attended block-major (steps 3-4) into partial results that the
+ * own-block pass merges by log-sum-exp (step 5).
+ *   q, k, v    : bf16 [batch, hq|hkv, N, d], d in {64, 80, 128}
+ *   idx        : as written by moba_select_topk for the same q and shapes
+ *   workspace  : the same buffer moba_select_topk filled (read, then partly reused)
+ *   window     : 0 for none
+ *   scale      : logit scale; <= 0 selects 1/sqrt(d)
+ *   out        : bf16 out [batch, hq, N, d]
+ *   lse        : float32 out [batch, hq, N], contiguous: natural log of the sum of
+ *                exp(scale q_i . k_j) over J_i
+ */
+int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *idx, int batch,
+                  int hq, int hkv, int N, int d, int block, int topk, int window, float scale,
+                  moba_tensor out, float *lse, void *workspace, size_t workspace_bytes,
+                  void *stream);
+
+/*
+ * [SWA] §"어텐션 공식" and §"슬라이딩 윈도우 마스크": softmax(scale QK^T + M) V with
+ * M_ij = 0 iff j <= i and i - j < window, else -inf.  window >= N gives dense causal
+ * attention.  Any N >= 1 (no block constraint).
+ *   q, k, v, out : bf16 [batch, hq|hkv, N, d], d in {64, 80, 128}
+ *   lse          : float32 out [batch, hq, N], contiguous
+ */
+int swa_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq, int hkv, int N,
+                 int d, int window, float scale, moba_tensor out, float *lse, void *stream);
+
+/*
+ * Reads and clears the device-side status word that bounded kernel waits write
+ * (MOBA_OK or MOBA_ERR_DEVICE) on the current device.  Synchronises the device.
+ */
+int moba_device_status(void);
+
+/* Static description of a status code. */
+const char *moba_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOBA_H */

@@ -1,0 +1,87 @@
+"""The C-ABI library loads, exports every entry point include/moba.h declares, and
+rejects bad arguments on the host before touching a device (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import block_sparse_long_prefill_b200 as moba
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moba.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_abi():
+    assert _declared() == sorted(moba.ABI_FUNCTIONS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(moba.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    assert moba.status_string(0) == "ok"
+    for code in range(-8, 0):
+        assert moba.status_string(code) != "unknown status"
+
+
+def test_workspace_size_is_host_only_and_grows_with_topk():
+    a = moba.workspace_size(1, 32, 8, 32768, 128, 512, 3)
+    b = moba.workspace_size(1, 32, 8, 32768, 128, 512, 4)
+    assert 0 < a < b
+    # k = 1 keeps only the own block: no partials, no entries.
+    c = moba.workspace_size(1, 32, 8, 32768, 128, 512, 1)
+    assert c < a
+
+
+@pytest.mark.parametrize("args,code", [
+    ((1, 32, 8, 32768, 128, 500, 3), -1),   # block not a multiple of 128
+    ((1, 32, 8, 32000, 128, 512, 3), -1),   # N not a multiple of block
+    ((1, 30, 8, 32768, 128, 512, 3), -1),   # hq not a multiple of hkv
+    ((1, 32, 8, 32768, 96, 512, 3), -2),    # unsupported d
+    ((1, 32, 8, 32768, 128, 512, 0), -4),   # topk < 1
+    ((1, 32, 8, 32768, 128, 512, 33), -4),  # topk > 32
+])
+def test_workspace_size_rejects_bad_shapes(args, code):
+    out = ctypes.c_size_t(0)
+    assert moba.library().moba_workspace_size(*args, ctypes.byref(out)) == code
+
+
+def test_bad_arguments_are_rejected_before_any_launch():
+    lib = moba.library()
+    T = moba.MobaTensor
+    null = T(None, 0, 0, 0)
+    ok = T(1 << 20, 8 * 1024, 8 * 1024, 128)
+    mis = T((1 << 20) + 2, 8 * 1024, 8 * 1024, 128)
+    odd = T(1 << 20, 8 * 1024, 8 * 1024, 100)
+    # pool: null tensor, misaligned pointer, misaligned stride, ragged block
+    assert lib.moba_pool_keys(null, 1, 1, 1024, 128, 128, 1 << 20, 1 << 20, None) == -4
+    assert lib.moba_pool_keys(mis, 1, 1, 1024, 128, 128, 1 << 20, 1 << 20, None) == -3
+    assert lib.moba_pool_keys(odd, 1, 1, 1024, 128, 128, 1 << 20, 1 << 20, None) == -3
+    assert lib.moba_pool_keys(ok, 1, 1, 1000, 128, 128, 1 << 20, 1 << 20, None) == -1
+    # select: workspace too small
+    assert lib.moba_select_topk(ok, 1 << 20, 1, 1, 1, 1024, 128, 128, 3, 1 << 20, 1 << 20, 16,
+                                None) == -5
+    # attention: negative window, unsupported d
+    assert lib.moba_attn_fwd(ok, ok, ok, 1 << 20, 1, 1, 1, 1024, 128, 128, 3, -1, 0.0, ok,
+                             1 << 20, 1 << 20, 1 << 30, None) == -4
+    assert lib.swa_attn_fwd(ok, ok, ok, 1, 1, 1, 1024, 96, 64, 0.0, ok, 1 << 20, None) == -2
+    assert lib.swa_attn_fwd(ok, ok, ok, 1, 1, 1, 1024, 128, 0, 0.0, ok, 1 << 20, None) == -4
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_a_device_reports_no_device():
+    lib = moba.library()
+    ok = moba.MobaTensor(1 << 20, 8 * 1024, 8 * 1024, 128)
+    rc = lib.swa_attn_fwd(ok, ok, ok, 1, 1, 1, 1024, 128, 64, 0.0, ok, 1 << 20, None)
+    assert rc == -8

@@ -1,0 +1,101 @@
+"""GPU parity of the MoBA path (pool -> select -> attention) against the fp64 oracle,
+through the C ABI, on seeded synthetic inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.parity import check_idx, check_out, rows_of
+
+pytestmark = pytest.mark.gpu
+
+
+def _moba():
+    import block_sparse_long_prefill_b200 as moba
+    return moba
+
+
+def run_and_check(w: workloads.Workload, seed=0, rows=None, check_pool=True):
+    moba = _moba()
+    q, k, v = workloads.make_inputs(w, seed)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    runner = moba.MobaPrefill(w.batch, w.hq, w.hkv, w.seqlen, w.d, w.block, w.topk, w.window)
+    out, lse = runner(qd, kd, vd)
+    torch.cuda.synchronize()
+    assert moba.device_status() == 0
+    if rows is None:
+        rows = np.arange(w.seqlen, dtype=np.int32)
+    kbar_o = oracle.pool_keys(k, w.block)
+    if check_pool:
+        kb = runner.kbar.cpu().numpy().astype(np.float64)
+        scale = np.abs(kbar_o).max()
+        assert np.abs(kb - kbar_o).max() <= 1e-5 * scale + 1e-7
+        split = runner.kbar_split.float().cpu().numpy().astype(np.float64)
+        recon = split[:, :, 0] + split[:, :, 1]
+        assert np.abs(recon - kbar_o).max() <= 2e-5 * scale + 1e-7
+    scores = oracle.gate_scores(q, kbar_o, w.block, rows)
+    idx_o, gap = oracle.select_topk(scores, w.seqlen, w.block, w.topk, rows)
+    idx_g = rows_of(runner.idx, rows)
+    loose = check_idx(idx_g, idx_o, gap, scores, rows, w.block)
+    out_o, lse_o = oracle.attention(q, k, v, mode=oracle.MODE_MOBA, block=w.block, topk=w.topk,
+                                    idx=idx_g, window=w.window, rows=rows)
+    stats = check_out(rows_of(out, rows), rows_of(lse, rows), out_o, lse_o)
+    stats["loose_rows"] = loose
+    return stats, runner
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny", dict()),
+    ("gqa_small", dict(batch=1, hq=4, hkv=2, seqlen=2048, d=128, block=256, topk=3)),
+    ("d80", dict(batch=1, hq=2, hkv=1, seqlen=1024, d=80, block=128, topk=4)),
+    ("batch2_g4", dict(batch=2, hq=8, hkv=2, seqlen=1024, d=64, block=128, topk=2)),
+    ("k1", dict(batch=1, hq=2, hkv=2, seqlen=1024, d=128, block=128, topk=1)),
+    ("k_all", dict(batch=1, hq=2, hkv=1, seqlen=1024, d=64, block=128, topk=8)),
+    ("k_over", dict(batch=1, hq=1, hkv=1, seqlen=768, d=64, block=128, topk=20)),
+    ("one_block", dict(batch=1, hq=2, hkv=1, seqlen=512, d=128, block=512, topk=3)),
+    ("window", dict(batch=1, hq=4, hkv=2, seqlen=2048, d=128, block=512, topk=2, window=300)),
+    ("window_wide", dict(batch=1, hq=2, hkv=1, seqlen=1024, d=64, block=128, topk=2, window=700)),
+    ("window_dense", dict(batch=1, hq=2, hkv=1, seqlen=1024, d=128, block=256, topk=2, window=4096)),
+    ("big_k", dict(batch=1, hq=2, hkv=1, seqlen=4096, d=128, block=128, topk=16)),
+])
+def test_moba_small_full_rows(name, kw):
+    w = workloads.WORKLOADS["tiny"] if name == "tiny" else workloads.small_moba(name=name, **kw)
+    stats, _ = run_and_check(w)
+    print(name, stats)
+
+
+def test_moba_deterministic():
+    moba = _moba()
+    w = workloads.small_moba(batch=1, hq=4, hkv=2, seqlen=2048, d=128, block=256, topk=3)
+    q, k, v = (t.cuda() for t in workloads.make_inputs(w, 3))
+    r = moba.MobaPrefill(w.batch, w.hq, w.hkv, w.seqlen, w.d, w.block, w.topk)
+    o1, l1 = (t.clone() for t in r(q, k, v))
+    i1 = r.idx.clone()
+    o2, l2 = r(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(i1, r.idx)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_moba_strided_inputs():
+    """q/k/v as [b, N, h, d] storage viewed as [b, h, N, d] (non-contiguous heads)."""
+    moba = _moba()
+    w = workloads.small_moba(batch=1, hq=4, hkv=2, seqlen=1024, d=128, block=128, topk=3)
+    q, k, v = workloads.make_inputs(w, 5)
+    qs = q.transpose(1, 2).contiguous().cuda().transpose(1, 2)
+    ks = k.transpose(1, 2).contiguous().cuda().transpose(1, 2)
+    vs = v.transpose(1, 2).contiguous().cuda().transpose(1, 2)
+    out, lse, idx = moba.moba_prefill(qs, ks, vs, w.block, w.topk)
+    out2, lse2, idx2 = moba.moba_prefill(q.cuda(), k.cuda(), v.cuda(), w.block, w.topk)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
+@pytest.mark.parametrize("name", ["gqa32k", "hybrid64k"])
+def test_moba_full_size_sampled_rows(name):
+    w = workloads.WORKLOADS[name]
+    rows = workloads.sampled_rows(w, seed=0)
+    stats, _ = run_and_check(w, rows=rows)
+    print(name, stats)
