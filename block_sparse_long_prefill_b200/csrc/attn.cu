@@ -368,6 +368,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
   } else {
     // ------------------------------------------- softmax + correction + epilogue
+    // tcgen05.ld / st are warp-collective (.sync.aligned): every wait below is made
+    // warp-uniform with __all_sync, and no TMEM access sits under a per-row branch.
     const int r = tid - 128;             // row within the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t tS[2] = {tmem + lane_off, tmem + lane_off + 128};
@@ -398,7 +400,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       float m_run = -INFINITY, l_run = 0.f;
       for (int m = 0; m < ti.nc; ++m, ++scnt) {
         const int sbi = scnt & 1;
-        if (!(ok = mbar_wait(&bar.s_full[sbi], (scnt >> 1) & 1, abort, p.status, site0 + 12))) break;
+        ok = mbar_wait(&bar.s_full[sbi], (scnt >> 1) & 1, abort, p.status, site0 + 12);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
         tc_fence_after();
         float s[128];
 #pragma unroll
@@ -446,25 +449,30 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int e = 0; e < 128; ++e) mx = fmaxf(mx, s[e]);
         const float m_new = fmaxf(m_run, mx * sl2);
         if (m > 0) {
-          if (!(ok = mbar_wait(&bar.o_done, ocnt & 1, abort, p.status, site0 + 13))) break;
+          ok = mbar_wait(&bar.o_done, ocnt & 1, abort, p.status, site0 + 13);
+          if (!(ok = __all_sync(0xffffffffu, ok))) break;
           ++ocnt;
           tc_fence_after();
         }
-        if (m_new > m_run + (float)kRescaleThreshold || (m == 0)) {
-          if (m > 0 && m_run != -INFINITY) {
-            const float alpha = ex2_approx(m_run - m_new);
-            l_run *= alpha;
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 16) {
-              uint32_t o[16];
-              tmem_ld16(tO + c0, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st16(tO + c0, o);
-            }
-          }
+        // Raise the running maximum only when it grows by more than 2^8 (or from
+        // -inf); rows that keep theirs multiply O by 1 when the warp rescales.
+        const bool raise = (m == 0) || (m_new > m_run + (float)kRescaleThreshold);
+        const bool scale_o = raise && m > 0 && m_run != -INFINITY;
+        const float alpha = scale_o ? ex2_approx(m_run - m_new) : 1.f;
+        if (raise) {
+          l_run *= alpha;
           m_run = m_new;
+        }
+        if (__any_sync(0xffffffffu, scale_o)) {
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 16) {
+            uint32_t o[16];
+            tmem_ld16(tO + c0, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(tO + c0, o);
+          }
         }
         const float mu = (m_run == -INFINITY) ? 0.f : m_run;
         float lsum = 0.f;
@@ -487,21 +495,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       if (!ok) break;
       // ------------------------------------------------------------ epilogue
-      if (!(ok = mbar_wait(&bar.o_done, ocnt & 1, abort, p.status, site0 + 14))) break;
+      ok = mbar_wait(&bar.o_done, ocnt & 1, abort, p.status, site0 + 14);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
       ++ocnt;
       tc_fence_after();
       const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
       const float own_lse = (m_run + log2f(l_run)) * 0.69314718055994530942f;  // natural log
       if (MODE == kGathered) {
-        if (live) {
-          const int il = i - p.chunk * p.chunk_rows;
-          const int64_t pidx = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + il) * p.npast + slot;
-          uint16_t *dst = p.opart + pidx * D;
+        const int il = i - p.chunk * p.chunk_rows;
+        const int64_t pidx = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + il) * p.npast + slot;
+        uint16_t *dst = p.opart + pidx * D;
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 16) {
-            uint32_t o[16];
-            tmem_ld16(tO + c0, o);
-            tmem_wait_ld();
+        for (int c0 = 0; c0 < D; c0 += 16) {
+          uint32_t o[16];
+          __syncwarp();
+          tmem_ld16(tO + c0, o);
+          tmem_wait_ld();
+          if (live) {
             uint4 w0, w1;
             w0.x = pack_bf16x2(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l);
             w0.y = pack_bf16x2(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l);
@@ -514,15 +524,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             *reinterpret_cast<uint4 *>(dst + c0) = w0;
             *reinterpret_cast<uint4 *>(dst + c0 + 8) = w1;
           }
-          p.lpart[pidx] = own_lse;
         }
-      } else if (live) {
+        if (live) p.lpart[pidx] = own_lse;
+      } else {
         // Merge with the past-block partials of this row (MoBA), then store.
         float wown = 1.f, lse = own_lse;
         int np = 0;
         int64_t pbase = 0;
         float wp[32];
-        if (p.is_moba && p.npast > 0) {
+        if (live && p.is_moba && p.npast > 0) {
           const int c = i / p.block;
           for (int s2 = 0; s2 < p.npast; ++s2) {
             const int blk = __ldg(irow + s2);
@@ -545,40 +555,46 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 16) {
           uint32_t o[16];
+          __syncwarp();
           tmem_ld16(tO + c0, o);
           tmem_wait_ld();
-          float acc[16];
+          if (live) {
+            float acc[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[e]) * inv_l * wown;
-          for (int s2 = 0; s2 < np; ++s2) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.opart + (pbase + s2) * D + c0);
-            const uint4 a0 = src[0], a1 = src[1];
-            const uint32_t wv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[e]) * inv_l * wown;
+            for (int s2 = 0; s2 < np; ++s2) {
+              const uint4 *src = reinterpret_cast<const uint4 *>(p.opart + (pbase + s2) * D + c0);
+              const uint4 a0 = src[0], a1 = src[1];
+              const uint32_t wv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              acc[2 * e] += wp[s2] * __uint_as_float(wv[e] << 16);
-              acc[2 * e + 1] += wp[s2] * __uint_as_float(wv[e] & 0xFFFF0000u);
+              for (int e = 0; e < 8; ++e) {
+                acc[2 * e] += wp[s2] * __uint_as_float(wv[e] << 16);
+                acc[2 * e + 1] += wp[s2] * __uint_as_float(wv[e] & 0xFFFF0000u);
+              }
             }
+            uint4 w0, w1;
+            w0.x = pack_bf16x2(acc[0], acc[1]);
+            w0.y = pack_bf16x2(acc[2], acc[3]);
+            w0.z = pack_bf16x2(acc[4], acc[5]);
+            w0.w = pack_bf16x2(acc[6], acc[7]);
+            w1.x = pack_bf16x2(acc[8], acc[9]);
+            w1.y = pack_bf16x2(acc[10], acc[11]);
+            w1.z = pack_bf16x2(acc[12], acc[13]);
+            w1.w = pack_bf16x2(acc[14], acc[15]);
+            *reinterpret_cast<uint4 *>(dst + c0) = w0;
+            *reinterpret_cast<uint4 *>(dst + c0 + 8) = w1;
           }
-          uint4 w0, w1;
-          w0.x = pack_bf16x2(acc[0], acc[1]);
-          w0.y = pack_bf16x2(acc[2], acc[3]);
-          w0.z = pack_bf16x2(acc[4], acc[5]);
-          w0.w = pack_bf16x2(acc[6], acc[7]);
-          w1.x = pack_bf16x2(acc[8], acc[9]);
-          w1.y = pack_bf16x2(acc[10], acc[11]);
-          w1.z = pack_bf16x2(acc[12], acc[13]);
-          w1.w = pack_bf16x2(acc[14], acc[15]);
-          *reinterpret_cast<uint4 *>(dst + c0) = w0;
-          *reinterpret_cast<uint4 *>(dst + c0 + 8) = w1;
         }
-        p.lse[((int64_t)ti.b * p.hq + h) * p.N + i] = lse;
+        if (live) p.lse[((int64_t)ti.b * p.hq + h) * p.N + i] = lse;
       }
       tc_fence_before();
       mbar_arrive(&bar.o_free);
     }
   }
 
+  // Roles ran on single lanes or with per-thread waits: reconverge every warp before
+  // the CTA barrier (bar.sync is warp-aligned) and before the warp-wide dealloc.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

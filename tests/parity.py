@@ -34,8 +34,9 @@ def check_idx(idx_gpu: np.ndarray, idx_orc: np.ndarray, gap: np.ndarray, scores:
     assert np.array_equal(nvalid, np.broadcast_to(want_n, nvalid.shape)), "wrong number of blocks"
     last = np.take_along_axis(idx_gpu, (nvalid - 1)[..., None], axis=-1)[..., 0]
     assert np.array_equal(last, np.broadcast_to(c, last.shape)), "own block is not kept"
-    assert np.all(np.diff(np.where(valid, idx_gpu, np.iinfo(np.int32).max), axis=-1) > 0), \
-        "not ascending / duplicate"
+    assert np.all(valid[..., 1:] <= valid[..., :-1]), "padding before a valid entry"
+    both = valid[..., 1:] & valid[..., :-1]
+    assert np.all(np.diff(idx_gpu, axis=-1)[both] > 0), "not ascending / duplicate"
     same = np.all(idx_gpu == idx_orc, axis=-1)
     clear = gap > GAP_TOL
     bad = clear & ~same
