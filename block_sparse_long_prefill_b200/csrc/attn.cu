@@ -14,15 +14,18 @@
 //                whole past block they picked (steps 3-4, causal=False); writes a
 //                normalised partial output and its log-sum-exp per (row, slot).
 //
-// Per CTA (256 threads, one CTA per SM, 512 TMEM columns):
-//   warp 0      TMA producer: K/V chunks of 128 keys (and the query tile, query-major)
-//   warp 1      tcgen05 MMA issuer (one thread) and TMEM owner
-//   warps 2-3   query-row gather with cp.async (gathered tiles)
-//   warps 4-7   softmax, O correction and epilogue; thread r owns row r (TMEM lane r)
-// TMEM: S/P double buffer at columns [0,128) and [128,256); O at [256, 256+D).
+// Per CTA (384 threads, one CTA per SM, 512 TMEM columns), FA4-style roles:
+//   warp 0       TMA producer: K/V chunks of 128 keys, the query tile (query-major) and
+//                L2 prefetch of the partials the merge will read
+//   warp 1       tcgen05 MMA issuer (one thread) and TMEM owner
+//   warps 2-3    query-row gather with cp.async (gathered tiles)
+//   warps 4-7    softmax: thread r owns row r (TMEM lane r); S -> P in place, rescales
+//                O only when its running maximum grows by more than 2^8
+//   warps 8-11   epilogue: normalises O, merges / stores, then frees the O buffer
+// TMEM: S/P double buffer at columns [0,128) and [128,256); O double buffer at
+// [256,384) and [384,512), so a tile's epilogue overlaps the next tile's MMAs.
 // S = Q K^T is an SS MMA; P (bf16) overwrites its own S columns and is the A operand
-// (from TMEM) of O += P V.  Softmax uses exp2 with a lazily raised running maximum:
-// O and l are rescaled only when the row maximum grows by more than 2^8.
+// (from TMEM) of O += P V.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -33,8 +36,12 @@
 
 namespace moba {
 
-constexpr int kAttnThreads = 256;
+constexpr int kAttnThreads = 384;
 constexpr int kRescaleThreshold = 8;  // log2 units
+// Registers per thread after the re-split: producer/MMA/gather, softmax, epilogue.
+constexpr int kRegsWG0 = 80, kRegsSoftmax = 240, kRegsEpilogue = 184;
+constexpr int kRegSplitTotal = 128 * (kRegsWG0 + kRegsSoftmax + kRegsEpilogue);
+static_assert(kRegSplitTotal <= 65536, "register split exceeds the register file");
 
 template <int D>
 struct AttnCfg {
@@ -46,7 +53,7 @@ struct AttnCfg {
   static constexpr int K_OFF = 2 * TILE;                   // ST key stages
   static constexpr int V_OFF = K_OFF + ST * TILE;          // ST value stages
   static constexpr int BAR_OFF = V_OFF + ST * TILE;
-  static constexpr int SMEM = BAR_OFF + 1024 + 1024;       // + barriers + alignment slack
+  static constexpr int SMEM = BAR_OFF + 3072 + 1024;       // + barriers/stats + alignment slack
   static constexpr uint32_t BYTES = 128u * D * 2u;         // bytes one full tile load moves
 };
 
@@ -54,9 +61,11 @@ struct Bars {
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[3], v_full[3], kv_empty[3];
   uint64_t s_full[2];
-  uint64_t p_full, o_done, o_free, mma_done;
+  uint64_t p_full, o_done, mma_done;
+  uint64_t o_full[2], o_free[2], stat_full[2];
   uint32_t tmem_base;
   int abort;
+  float2 stat[2][128];  // per O buffer and row: running max (log2 units), row sum
 };
 
 // What one tile covers.  All roles derive it independently from the tile index.
@@ -165,6 +174,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   Bars &bar = *reinterpret_cast<Bars *>(sbase + C::BAR_OFF);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int site0 = (MODE * 16 + (D == 64 ? 0 : (D == 80 ? 1 : 2))) * 256;
+  constexpr uint32_t FULL = 0xffffffffu;
 
   // Tile range.
   int t_begin = 0, t_end = p.ntiles;
@@ -187,8 +197,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     mbar_init(&bar.s_full[1], 1);
     mbar_init(&bar.p_full, 128);
     mbar_init(&bar.o_done, 1);
-    mbar_init(&bar.o_free, 128);
     mbar_init(&bar.mma_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar.o_full[b], 1);
+      mbar_init(&bar.o_free[b], 128);
+      mbar_init(&bar.stat_full[b], 128);
+    }
     bar.abort = 0;
     fence_barrier_init();
   }
@@ -207,128 +221,134 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t tmem = bar.tmem_base;
   volatile int *abort = &bar.abort;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t kvc = 0;
-      int lt = 0;
-      bool ok = true;
-      for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x, ++lt) {
-        TileInfo ti;
-        if (MODE == kGathered) gathered_tile(p, t, ti); else query_major_tile(p, t, ti);
-        if (MODE == kQueryMajor) {
-          const int qb = lt & 1;
-          if (!(ok = mbar_wait(&bar.q_empty[qb], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 1))) break;
-          const uint32_t qt = base + C::Q_OFF + qb * C::TILE;
-          mbar_arrive_expect_tx(&bar.q_full[qb], C::BYTES);
-          tma_load_4d(sbase + (qt - base), &tmQ, &bar.q_full[qb], 0, ti.i0, ti.h, ti.b);
-          if (D == 128) tma_load_4d(sbase + (qt - base) + C::R0, &tmQ1, &bar.q_full[qb], 64, ti.i0, ti.h, ti.b);
-          if (D == 80) tma_load_4d(sbase + (qt - base) + C::R0, &tmQ1, &bar.q_full[qb], 64, ti.i0, ti.h, ti.b);
-        }
-        for (int m = 0; m < ti.nc; ++m, ++kvc) {
-          const int st = kvc % C::ST;
-          if (!(ok = mbar_wait(&bar.kv_empty[st], ((kvc / C::ST) & 1) ^ 1, abort, p.status, site0 + 2))) break;
-          const int key = chunk_key<MODE>(p, ti, m);
-          unsigned char *kd = sbase + C::K_OFF + st * C::TILE;
-          unsigned char *vd = sbase + C::V_OFF + st * C::TILE;
-          mbar_arrive_expect_tx(&bar.k_full[st], C::BYTES);
-          tma_load_4d(kd, &tmK, &bar.k_full[st], 0, key, ti.hk, ti.b);
-          if (D != 64) tma_load_4d(kd + C::R0, &tmK1, &bar.k_full[st], 64, key, ti.hk, ti.b);
-          mbar_arrive_expect_tx(&bar.v_full[st], C::BYTES);
-          tma_load_4d(vd, &tmV, &bar.v_full[st], 0, key, ti.hk, ti.b);
-          if (D != 64) tma_load_4d(vd + C::R0, &tmV1, &bar.v_full[st], 64, key, ti.hk, ti.b);
-        }
-      }
-      // Let every load issued so far land before the CTA can retire.
-      if (*abort) {
-        for (uint32_t u = (kvc > (uint32_t)C::ST ? kvc - C::ST : 0); u < kvc; ++u) {
-          const int st = u % C::ST;
-          const unsigned long long t0 = global_timer_ns();
-          while (!mbar_try_wait(&bar.k_full[st], (u / C::ST) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
-          while (!mbar_try_wait(&bar.v_full[st], (u / C::ST) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
-      constexpr uint32_t idO64 = idesc_bf16(128, 64, 0, 1);
-      constexpr uint32_t idO16 = idesc_bf16(128, 16, 0, 1);
-      const uint32_t tS[2] = {tmem, tmem + 128};
-      const uint32_t tO = tmem + 256;
-      uint32_t kvc = 0, scnt = 0, pcnt = 0, ofree = 0;
-      int lt = 0;
-      bool ok = true;
-      auto issue_pv = [&](int first, uint32_t sbuf, int st) {
-        const uint32_t vt = base + C::V_OFF + st * C::TILE;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-          const uint32_t a = sbuf + kk * 8;
-          umma_ts(tO, a, v_desc<D>(vt, kk, 0), idO64, acc);
-          if (D == 128) umma_ts(tO + 64, a, v_desc<D>(vt, kk, 1), idO64, acc);
-          if (D == 80) umma_ts(tO + 64, a, v_desc<D>(vt, kk, 1), idO16, acc);
-        }
-      };
-      for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x, ++lt) {
-        TileInfo ti;
-        if (MODE == kGathered) gathered_tile(p, t, ti); else query_major_tile(p, t, ti);
-        const int qb = lt & 1;
-        if (!(ok = mbar_wait(&bar.q_full[qb], (lt >> 1) & 1, abort, p.status, site0 + 3))) break;
-        tc_fence_after();
-        const uint32_t qt = base + C::Q_OFF + qb * C::TILE;
-        uint32_t prev_sbuf = 0;
-        int prev_st = 0;
-        for (int m = 0; m < ti.nc; ++m, ++kvc, ++scnt) {
-          const int st = kvc % C::ST;
-          if (!(ok = mbar_wait(&bar.k_full[st], (kvc / C::ST) & 1, abort, p.status, site0 + 4))) break;
-          tc_fence_after();
-          const uint32_t kt = base + C::K_OFF + st * C::TILE;
-          const uint32_t sb = tS[scnt & 1];
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            umma_ss(sb, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idS, ks > 0 ? 1u : 0u);
-          umma_commit(&bar.s_full[scnt & 1]);
-          if (m == ti.nc - 1) umma_commit(&bar.q_empty[qb]);
-          if (m > 0) {
-            if (!(ok = mbar_wait(&bar.p_full, pcnt & 1, abort, p.status, site0 + 5))) break;
-            ++pcnt;
-            if (!(ok = mbar_wait(&bar.v_full[prev_st], ((kvc - 1) / C::ST) & 1, abort, p.status, site0 + 6))) break;
-            if (m == 1) {
-              if (!(ok = mbar_wait(&bar.o_free, (ofree & 1) ^ 1, abort, p.status, site0 + 7))) break;
-              ++ofree;
+  // Register split (launch: 384 threads x 168): 128 x (80 + 240 + 184) = 64512.
+  if (warp < 4) {
+    setmaxnreg_dec<kRegsWG0>();
+    if (warp == 0) {
+      // ---------------------------------------------------------- producer
+      if (lane == 0) {
+        uint32_t kvc = 0;
+        int lt = 0;
+        bool ok = true;
+        for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x, ++lt) {
+          TileInfo ti;
+          if (MODE == kGathered) gathered_tile(p, t, ti); else query_major_tile(p, t, ti);
+          if (MODE == kQueryMajor) {
+            if (p.is_moba && p.npast > 0) {
+              // The merge reads this tile's partials: pull them into L2 now.
+              const int il = ti.i0 - p.chunk * p.chunk_rows;
+              const int64_t prow = ((int64_t)ti.b * p.hq + ti.h) * p.chunk_rows + il;
+              const char *po = reinterpret_cast<const char *>(p.opart + prow * p.npast * D);
+              const uint32_t pbytes = (uint32_t)ti.rows * p.npast * D * 2;
+              for (uint32_t off = 0; off < pbytes; off += 65536)
+                prefetch_l2_bulk(po + off, min(65536u, pbytes - off));
+              const char *pl = reinterpret_cast<const char *>(p.lpart + prow * p.npast);
+              prefetch_l2_bulk(pl, ((uint32_t)ti.rows * p.npast * 4 + 15) & ~15u);
             }
-            tc_fence_after();
-            issue_pv(m == 1, prev_sbuf, prev_st);
-            umma_commit(&bar.o_done);
-            umma_commit(&bar.kv_empty[prev_st]);
+            const int qb = lt & 1;
+            if (!(ok = mbar_wait(&bar.q_empty[qb], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 1))) break;
+            unsigned char *qd = sbase + C::Q_OFF + qb * C::TILE;
+            mbar_arrive_expect_tx(&bar.q_full[qb], C::BYTES);
+            tma_load_4d(qd, &tmQ, &bar.q_full[qb], 0, ti.i0, ti.h, ti.b);
+            if (D != 64) tma_load_4d(qd + C::R0, &tmQ1, &bar.q_full[qb], 64, ti.i0, ti.h, ti.b);
           }
-          prev_sbuf = sb;
-          prev_st = st;
+          for (int m = 0; m < ti.nc; ++m, ++kvc) {
+            const int st = kvc % C::ST;
+            if (!(ok = mbar_wait(&bar.kv_empty[st], ((kvc / C::ST) & 1) ^ 1, abort, p.status, site0 + 2))) break;
+            const int key = chunk_key<MODE>(p, ti, m);
+            unsigned char *kd = sbase + C::K_OFF + st * C::TILE;
+            unsigned char *vd = sbase + C::V_OFF + st * C::TILE;
+            mbar_arrive_expect_tx(&bar.k_full[st], C::BYTES);
+            tma_load_4d(kd, &tmK, &bar.k_full[st], 0, key, ti.hk, ti.b);
+            if (D != 64) tma_load_4d(kd + C::R0, &tmK1, &bar.k_full[st], 64, key, ti.hk, ti.b);
+            mbar_arrive_expect_tx(&bar.v_full[st], C::BYTES);
+            tma_load_4d(vd, &tmV, &bar.v_full[st], 0, key, ti.hk, ti.b);
+            if (D != 64) tma_load_4d(vd + C::R0, &tmV1, &bar.v_full[st], 64, key, ti.hk, ti.b);
+          }
         }
-        if (!ok) break;
-        // PV of the last chunk.
-        if (!(ok = mbar_wait(&bar.p_full, pcnt & 1, abort, p.status, site0 + 8))) break;
-        ++pcnt;
-        if (!(ok = mbar_wait(&bar.v_full[prev_st], ((kvc - 1) / C::ST) & 1, abort, p.status, site0 + 9))) break;
-        if (ti.nc == 1) {
-          if (!(ok = mbar_wait(&bar.o_free, (ofree & 1) ^ 1, abort, p.status, site0 + 10))) break;
-          ++ofree;
+        // Let every load issued so far land before the CTA can retire.
+        if (*abort) {
+          for (uint32_t u = (kvc > (uint32_t)C::ST ? kvc - C::ST : 0); u < kvc; ++u) {
+            const int st = u % C::ST;
+            const unsigned long long t0 = global_timer_ns();
+            while (!mbar_try_wait(&bar.k_full[st], (u / C::ST) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+            while (!mbar_try_wait(&bar.v_full[st], (u / C::ST) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+          }
         }
-        tc_fence_after();
-        issue_pv(ti.nc == 1, prev_sbuf, prev_st);
-        umma_commit(&bar.o_done);
-        umma_commit(&bar.kv_empty[prev_st]);
       }
-      // Every MMA issued so far completes before TMEM is released.
-      umma_commit(&bar.mma_done);
-      const unsigned long long t0 = global_timer_ns();
-      while (!mbar_try_wait(&bar.mma_done, 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
-    }
-  } else if (warp < 4) {
-    // ------------------------------------------------------- row gather
-    if (MODE == kGathered) {
+    } else if (warp == 1) {
+      // -------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+        constexpr uint32_t idO64 = idesc_bf16(128, 64, 0, 1);
+        constexpr uint32_t idO16 = idesc_bf16(128, 16, 0, 1);
+        uint32_t kvc = 0, scnt = 0, pcnt = 0;
+        int lt = 0;
+        bool ok = true;
+        auto issue_pv = [&](uint32_t tO, int first, uint32_t sbuf, int st) {
+          const uint32_t vt = base + C::V_OFF + st * C::TILE;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+            const uint32_t a = sbuf + kk * 8;
+            umma_ts(tO, a, v_desc<D>(vt, kk, 0), idO64, acc);
+            if (D == 128) umma_ts(tO + 64, a, v_desc<D>(vt, kk, 1), idO64, acc);
+            if (D == 80) umma_ts(tO + 64, a, v_desc<D>(vt, kk, 1), idO16, acc);
+          }
+        };
+        for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x, ++lt) {
+          TileInfo ti;
+          if (MODE == kGathered) gathered_tile(p, t, ti); else query_major_tile(p, t, ti);
+          const int qb = lt & 1, ob = lt & 1;
+          const uint32_t tO = tmem + 256 + 128 * ob;
+          if (!(ok = mbar_wait(&bar.q_full[qb], (lt >> 1) & 1, abort, p.status, site0 + 3))) break;
+          tc_fence_after();
+          const uint32_t qt = base + C::Q_OFF + qb * C::TILE;
+          uint32_t prev_sbuf = 0;
+          int prev_st = 0;
+          for (int m = 0; m <= ti.nc; ++m) {
+            if (m < ti.nc) {
+              const int st = kvc % C::ST;
+              if (!(ok = mbar_wait(&bar.k_full[st], (kvc / C::ST) & 1, abort, p.status, site0 + 4))) break;
+              tc_fence_after();
+              const uint32_t kt = base + C::K_OFF + st * C::TILE;
+              const uint32_t sb = tmem + 128 * (scnt & 1);
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                umma_ss(sb, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idS, ks > 0 ? 1u : 0u);
+              umma_commit(&bar.s_full[scnt & 1]);
+              if (m == ti.nc - 1) umma_commit(&bar.q_empty[qb]);
+            }
+            if (m > 0) {
+              // O += P V for chunk m-1.
+              if (!(ok = mbar_wait(&bar.p_full, pcnt & 1, abort, p.status, site0 + 5))) break;
+              ++pcnt;
+              // Chunk m-1 used pipeline slot kvc - 1 (kvc advances after each S).
+              if (!(ok = mbar_wait(&bar.v_full[prev_st], ((kvc - 1) / C::ST) & 1, abort, p.status, site0 + 6))) break;
+              if (m == 1) {
+                if (!(ok = mbar_wait(&bar.o_free[ob], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 7))) break;
+              }
+              tc_fence_after();
+              issue_pv(tO, m == 1, prev_sbuf, prev_st);
+              if (m < ti.nc) umma_commit(&bar.o_done);
+              else umma_commit(&bar.o_full[ob]);
+              umma_commit(&bar.kv_empty[prev_st]);
+            }
+            if (m < ti.nc) {
+              prev_sbuf = tmem + 128 * (scnt & 1);
+              prev_st = kvc % C::ST;
+              ++scnt;
+              ++kvc;
+            }
+          }
+        }
+        // Every MMA issued so far completes before TMEM is released.
+        umma_commit(&bar.mma_done);
+        const unsigned long long t0 = global_timer_ns();
+        while (!mbar_try_wait(&bar.mma_done, 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+      }
+    } else if (MODE == kGathered) {
+      // -------------------------------------------------------- row gather
       const int u = tid - 64;  // 0..63
       constexpr int VPR = D / 8;  // 16-byte vectors per row
       const int npast = p.npast;
@@ -366,52 +386,41 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_arrive(&bar.q_full[qb]);
       }
     }
-  } else {
-    // ------------------------------------------- softmax + correction + epilogue
-    // tcgen05.ld / st are warp-collective (.sync.aligned): every wait below is made
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax
+    // tcgen05.ld / st are warp-collective (.sync.aligned): every wait is made
     // warp-uniform with __all_sync, and no TMEM access sits under a per-row branch.
+    setmaxnreg_inc<kRegsSoftmax>();
     const int r = tid - 128;             // row within the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t tS[2] = {tmem + lane_off, tmem + lane_off + 128};
-    const uint32_t tO = tmem + lane_off + 256;
     const float sl2 = p.scale_log2;
     uint32_t scnt = 0, ocnt = 0;
+    int lt = 0;
     bool ok = true;
-    for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x) {
+    for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x, ++lt) {
       TileInfo ti;
       if (MODE == kGathered) gathered_tile(p, t, ti); else query_major_tile(p, t, ti);
+      const int ob = lt & 1;
+      const uint32_t tO = tmem + lane_off + 256 + 128 * ob;
       const bool live = r < ti.rows;
-      // Row identity.
-      int i = 0, h = ti.h, slot = 0;
-      if (MODE == kGathered) {
-        if (live) {
-          const uint32_t ent = __ldg(p.entries + ti.ent0 + r);
-          slot = (int)(ent % (uint32_t)p.npast);
-          const uint32_t ig = ent / (uint32_t)p.npast;
-          h = ti.hk * p.G + (int)(ig % (uint32_t)p.G);
-          i = (int)(ig / (uint32_t)p.G);
-        }
-      } else {
-        i = ti.i0 + r;
-      }
+      const int i = ti.i0 + r;  // query-major row
       const int32_t *irow = (MODE == kQueryMajor && p.is_moba && live)
-                                ? p.idx + (((int64_t)ti.b * p.hq + h) * p.N + i) * p.topk
+                                ? p.idx + (((int64_t)ti.b * p.hq + ti.h) * p.N + i) * p.topk
                                 : nullptr;
       float m_run = -INFINITY, l_run = 0.f;
       for (int m = 0; m < ti.nc; ++m, ++scnt) {
         const int sbi = scnt & 1;
+        const uint32_t tS = tmem + lane_off + 128 * sbi;
         ok = mbar_wait(&bar.s_full[sbi], (scnt >> 1) & 1, abort, p.status, site0 + 12);
-        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+        if (!(ok = __all_sync(FULL, ok))) break;
         tc_fence_after();
-        float s[128];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t v[32];
-          tmem_ld32(tS[sbi] + q4 * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) s[q4 * 32 + e] = __uint_as_float(v[e]);
-        }
+        uint32_t sv[128];
+        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+        tmem_wait_ld();
+        float *s = reinterpret_cast<float *>(sv);
         // Masks.
         const int key0 = chunk_key<MODE>(p, ti, m);
         if (MODE == kQueryMajor) {
@@ -444,16 +453,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             }
           }
         }
-        float mx = -INFINITY;
+        float mx4[8];
 #pragma unroll
-        for (int e = 0; e < 128; ++e) mx = fmaxf(mx, s[e]);
+        for (int u2 = 0; u2 < 8; ++u2) mx4[u2] = s[u2];
+#pragma unroll
+        for (int e = 8; e < 128; ++e) mx4[e & 7] = fmaxf(mx4[e & 7], s[e]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])),
+                               fmaxf(fmaxf(mx4[4], mx4[5]), fmaxf(mx4[6], mx4[7])));
         const float m_new = fmaxf(m_run, mx * sl2);
-        if (m > 0) {
-          ok = mbar_wait(&bar.o_done, ocnt & 1, abort, p.status, site0 + 13);
-          if (!(ok = __all_sync(0xffffffffu, ok))) break;
-          ++ocnt;
-          tc_fence_after();
-        }
         // Raise the running maximum only when it grows by more than 2^8 (or from
         // -inf); rows that keep theirs multiply O by 1 when the warp rescales.
         const bool raise = (m == 0) || (m_new > m_run + (float)kRescaleThreshold);
@@ -463,47 +470,107 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           l_run *= alpha;
           m_run = m_new;
         }
-        if (__any_sync(0xffffffffu, scale_o)) {
-#pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 16) {
-            uint32_t o[16];
-            tmem_ld16(tO + c0, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st16(tO + c0, o);
-          }
-        }
         const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-        float lsum = 0.f;
+        float ls[8];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t pk[16];
+        for (int u2 = 0; u2 < 8; ++u2) ls[u2] = 0.f;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2_approx(fmaf(s[q4 * 32 + 2 * e], sl2, -mu));
-            const float p1 = ex2_approx(fmaf(s[q4 * 32 + 2 * e + 1], sl2, -mu));
-            lsum += p0 + p1;
+        for (int q4 = 0; q4 < 8; ++q4) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            // One element in four takes the FMA-pipe 2^x, the rest the MUFU unit.
+            const float p0 = ex2_approx(fmaf(s[q4 * 16 + 2 * e], sl2, -mu));
+            const float x1 = fmaf(s[q4 * 16 + 2 * e + 1], sl2, -mu);
+            const float p1 = (e & 1) ? exp2_fma(x1) : ex2_approx(x1);
+            ls[e] += p0 + p1;
             pk[e] = pack_bf16x2(p0, p1);
           }
-          tmem_st16(tS[sbi] + q4 * 16, pk);
+          sv[q4 * 8 + 0] = pk[0]; sv[q4 * 8 + 1] = pk[1]; sv[q4 * 8 + 2] = pk[2]; sv[q4 * 8 + 3] = pk[3];
+          sv[q4 * 8 + 4] = pk[4]; sv[q4 * 8 + 5] = pk[5]; sv[q4 * 8 + 6] = pk[6]; sv[q4 * 8 + 7] = pk[7];
         }
-        l_run += lsum;
+        tmem_st16(tS, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+        tmem_st16(tS + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+        tmem_st16(tS + 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[32]));
+        tmem_st16(tS + 48, *reinterpret_cast<uint32_t(*)[16]>(&sv[48]));
+        l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        if (m > 0) {
+          // O holds chunks 0..m-1 once their last P V is done; rescale it if any row
+          // of this warp raised its maximum.
+          ok = mbar_wait(&bar.o_done, ocnt & 1, abort, p.status, site0 + 13);
+          if (!(ok = __all_sync(FULL, ok))) break;
+          ++ocnt;
+          tc_fence_after();
+          if (__any_sync(FULL, scale_o)) {
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 16) {
+              uint32_t o[16];
+              tmem_ld16(tO + c0, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st16(tO + c0, o);
+            }
+          }
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bar.p_full);
       }
       if (!ok) break;
-      // ------------------------------------------------------------ epilogue
-      ok = mbar_wait(&bar.o_done, ocnt & 1, abort, p.status, site0 + 14);
-      if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      ++ocnt;
+      // Hand the row statistics to the epilogue once it has drained this O buffer's
+      // previous tile.
+      ok = mbar_wait(&bar.o_free[ob], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 14);
+      if (!(ok = __all_sync(FULL, ok))) break;
+      bar.stat[ob][r] = make_float2(m_run, l_run);
+      mbar_arrive(&bar.stat_full[ob]);
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    setmaxnreg_inc<kRegsEpilogue>();
+    const int r = tid - 256;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    int lt = 0;
+    bool ok = true;
+    for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x, ++lt) {
+      TileInfo ti;
+      if (MODE == kGathered) gathered_tile(p, t, ti); else query_major_tile(p, t, ti);
+      const int ob = lt & 1;
+      const uint32_t tO = tmem + lane_off + 256 + 128 * ob;
+      const bool live = r < ti.rows;
+      int i = ti.i0 + r, h = ti.h, slot = 0;
+      if (MODE == kGathered && live) {
+        const uint32_t ent = __ldg(p.entries + ti.ent0 + r);
+        slot = (int)(ent % (uint32_t)p.npast);
+        const uint32_t ig = ent / (uint32_t)p.npast;
+        h = ti.hk * p.G + (int)(ig % (uint32_t)p.G);
+        i = (int)(ig / (uint32_t)p.G);
+      }
+      // Merge inputs that do not depend on this tile's result: read them first.
+      int np = 0;
+      int64_t pbase = 0;
+      float lp[32];
+      if (MODE == kQueryMajor && live && p.is_moba && p.npast > 0) {
+        const int32_t *irow = p.idx + (((int64_t)ti.b * p.hq + h) * p.N + i) * p.topk;
+        const int c = i / p.block;
+        for (int s2 = 0; s2 < p.npast; ++s2) {
+          const int blk = __ldg(irow + s2);
+          if (blk < 0 || blk >= c) break;
+          ++np;
+        }
+        pbase = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + (i - p.chunk * p.chunk_rows)) * p.npast;
+        for (int s2 = 0; s2 < np; ++s2) lp[s2] = p.lpart[pbase + s2];
+      }
+      ok = mbar_wait(&bar.stat_full[ob], (lt >> 1) & 1, abort, p.status, site0 + 15);
+      ok = ok && mbar_wait(&bar.o_full[ob], (lt >> 1) & 1, abort, p.status, site0 + 16);
+      if (!(ok = __all_sync(FULL, ok))) break;
       tc_fence_after();
+      const float2 st = bar.stat[ob][r];
+      const float m_run = st.x, l_run = st.y;
       const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
       const float own_lse = (m_run + log2f(l_run)) * 0.69314718055994530942f;  // natural log
       if (MODE == kGathered) {
-        const int il = i - p.chunk * p.chunk_rows;
-        const int64_t pidx = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + il) * p.npast + slot;
+        const int64_t pidx = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + (i - p.chunk * p.chunk_rows)) * p.npast + slot;
         uint16_t *dst = p.opart + pidx * D;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 16) {
@@ -529,27 +596,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       } else {
         // Merge with the past-block partials of this row (MoBA), then store.
         float wown = 1.f, lse = own_lse;
-        int np = 0;
-        int64_t pbase = 0;
         float wp[32];
-        if (live && p.is_moba && p.npast > 0) {
-          const int c = i / p.block;
-          for (int s2 = 0; s2 < p.npast; ++s2) {
-            const int blk = __ldg(irow + s2);
-            if (blk < 0 || blk >= c) break;
-            ++np;
-          }
-          if (np > 0) {
-            const int il = i - p.chunk * p.chunk_rows;
-            pbase = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + il) * p.npast;
-            float mx = own_lse;
-            for (int s2 = 0; s2 < np; ++s2) mx = fmaxf(mx, p.lpart[pbase + s2]);
-            float tot = __expf(own_lse - mx);
-            for (int s2 = 0; s2 < np; ++s2) tot += __expf(p.lpart[pbase + s2] - mx);
-            lse = mx + __logf(tot);
-            wown = __expf(own_lse - lse);
-            for (int s2 = 0; s2 < np; ++s2) wp[s2] = __expf(p.lpart[pbase + s2] - lse);
-          }
+        if (np > 0) {
+          float mx = own_lse;
+          for (int s2 = 0; s2 < np; ++s2) mx = fmaxf(mx, lp[s2]);
+          float tot = __expf(own_lse - mx);
+          for (int s2 = 0; s2 < np; ++s2) tot += __expf(lp[s2] - mx);
+          lse = mx + __logf(tot);
+          wown = __expf(own_lse - lse);
+          for (int s2 = 0; s2 < np; ++s2) wp[s2] = __expf(lp[s2] - lse);
         }
         uint16_t *dst = p.out + ti.b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)i * p.o_sn;
 #pragma unroll
@@ -588,7 +643,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (live) p.lse[((int64_t)ti.b * p.hq + h) * p.N + i] = lse;
       }
       tc_fence_before();
-      mbar_arrive(&bar.o_free);
+      mbar_arrive(&bar.o_free[ob]);
     }
   }
 
@@ -608,6 +663,17 @@ static cudaError_t launch_attn_dm(const CUtensorMap *maps, const AttnParams &p, 
                                   cudaStream_t st) {
   using C = AttnCfg<D>;
   auto kern = attn_fwd_kernel<D, MODE>;
+  // The warpgroups re-split the registers the CTA is launched with (setmaxnreg); a
+  // build that launched with fewer than 168 per thread would leave an increase
+  // waiting forever, so refuse to launch it.
+  static int regs = 0;
+  if (regs == 0) {
+    cudaFuncAttributes fa;
+    cudaError_t e0 = cudaFuncGetAttributes(&fa, kern);
+    if (e0 != cudaSuccess) return e0;
+    regs = fa.numRegs;
+  }
+  if (regs * kAttnThreads < kRegSplitTotal) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   kern<<<grid, kAttnThreads, C::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);

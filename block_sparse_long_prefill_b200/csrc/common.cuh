@@ -103,6 +103,11 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, u
       : "memory");
 }
 
+// Prefetch [src, src + bytes) of global memory into L2 (bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ---------------------------------------------------------------- cp.async
 
 __device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void *src) {
@@ -254,10 +259,37 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Software 2^x on the FMA pipes (no MUFU): Cody-Waite range reduction x = n + f,
+// n = rint(x) via the 1.5 * 2^23 rounding constant, f in [-1/2, 1/2]; 2^f from a cubic
+// near-minimax fit (weighted least squares on Chebyshev nodes, p(0) = 1; the constants
+// come from exp2_poly.py); 2^n enters through the exponent field.  Relative error
+// about 1.1e-4 on [-127, 8], below the bf16 step the probabilities are rounded to.
+// Inputs below -127 are clamped (their result, about 1e-38, is negligible).
+constexpr float kExp2C1 = 0.6933686f;
+constexpr float kExp2C2 = 0.24221784f;
+constexpr float kExp2C3 = 0.054592825f;
+
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -127.f);
+  const float t = x + 12582912.f;
+  const float r = x - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(kExp2C3, r, kExp2C2), r, kExp2C1), r, 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
