@@ -349,6 +349,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     } else if (MODE == kGathered) {
       // -------------------------------------------------------- row gather
+      // Thread u owns rows u and u + 64 of the tile: it reads their list entries
+      // first, then issues all of their 16-byte copies (no dependent loads between).
       const int u = tid - 64;  // 0..63
       constexpr int VPR = D / 8;  // 16-byte vectors per row
       const int npast = p.npast;
@@ -357,28 +359,35 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         TileInfo ti;
         gathered_tile(p, t, ti);
         const int qb = lt & 1;
+        uint32_t ent[2] = {0u, 0u};
+#pragma unroll
+        for (int k2 = 0; k2 < 2; ++k2)
+          if (u + 64 * k2 < ti.rows) ent[k2] = __ldg(p.entries + ti.ent0 + u + 64 * k2);
         if (!mbar_wait(&bar.q_empty[qb], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 11)) break;
         const uint32_t qt = base + C::Q_OFF + qb * C::TILE;
-        for (int e = u; e < 128 * VPR; e += 64) {
-          const int r = e / VPR, c = e % VPR;
+#pragma unroll
+        for (int k2 = 0; k2 < 2; ++k2) {
+          const int r = u + 64 * k2;
           const bool valid = r < ti.rows;
-          const uint16_t *src = p.q;
+          const uint16_t *row = p.q;
           if (valid) {
-            const uint32_t ent = __ldg(p.entries + ti.ent0 + r);
-            const uint32_t ig = ent / (uint32_t)npast;
+            const uint32_t ig = ent[k2] / (uint32_t)npast;
             const int g = (int)(ig % (uint32_t)p.G);
             const int i = (int)(ig / (uint32_t)p.G);
-            src = p.q + ti.b * p.q_sb + (int64_t)(ti.hk * p.G + g) * p.q_sh + (int64_t)i * p.q_sn + c * 8;
+            row = p.q + ti.b * p.q_sb + (int64_t)(ti.hk * p.G + g) * p.q_sh + (int64_t)i * p.q_sn;
           }
-          uint32_t dst;
-          if (c < 8) {
-            dst = qt + r * 128 + ((c ^ (r & 7)) << 4);
-          } else if (D == 128) {
-            dst = qt + C::R0 + r * 128 + (((c - 8) ^ (r & 7)) << 4);
-          } else {
-            dst = qt + C::R0 + r * 32 + (((c - 8) ^ ((r >> 2) & 1)) << 4);
+#pragma unroll
+          for (int c = 0; c < VPR; ++c) {
+            uint32_t dst;
+            if (c < 8) {
+              dst = qt + r * 128 + ((c ^ (r & 7)) << 4);
+            } else if (D == 128) {
+              dst = qt + C::R0 + r * 128 + (((c - 8) ^ (r & 7)) << 4);
+            } else {
+              dst = qt + C::R0 + r * 32 + (((c - 8) ^ ((r >> 2) & 1)) << 4);
+            }
+            cp_async_16_zfill(dst, valid ? row + c * 8 : p.q, valid);
           }
-          cp_async_16_zfill(dst, src, valid);
         }
         cp_async_commit();
         cp_async_wait_all();
@@ -607,37 +616,87 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int s2 = 0; s2 < np; ++s2) wp[s2] = __expf(lp[s2] - lse);
         }
         uint16_t *dst = p.out + ti.b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)i * p.o_sn;
+        // 32 columns at a time: the partial pieces of up to two slots are loaded
+        // together before the TMEM read, so their latencies overlap.
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 16) {
-          uint32_t o[16];
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          constexpr int W = (D == 80) ? 16 : 32;  // D = 80: pieces of 32, 32, 16
+          (void)W;
+          const int cols = (D - c0) < 32 ? (D - c0) : 32;
+          uint32_t o[32];
           __syncwarp();
-          tmem_ld16(tO + c0, o);
+          if (cols == 32) {
+            tmem_ld32(tO + c0, o);
+          } else {
+            tmem_ld16(tO + c0, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+          }
+          float acc[32];
+          uint4 pa[2][4];
+          if (live && np > 0) {
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2)
+              if (s2 < np) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(p.opart + (pbase + s2) * D + c0);
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4)
+                  if (v4 * 8 < cols) pa[s2][v4] = src[v4];
+              }
+          }
           tmem_wait_ld();
           if (live) {
-            float acc[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[e]) * inv_l * wown;
-            for (int s2 = 0; s2 < np; ++s2) {
-              const uint4 *src = reinterpret_cast<const uint4 *>(p.opart + (pbase + s2) * D + c0);
-              const uint4 a0 = src[0], a1 = src[1];
-              const uint32_t wv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(o[e]) * inv_l * wown;
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                acc[2 * e] += wp[s2] * __uint_as_float(wv[e] << 16);
-                acc[2 * e + 1] += wp[s2] * __uint_as_float(wv[e] & 0xFFFF0000u);
+            for (int s2 = 0; s2 < 2; ++s2)
+              if (s2 < np) {
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4) {
+                  if (v4 * 8 >= cols) break;
+                  const uint32_t wv[4] = {pa[s2][v4].x, pa[s2][v4].y, pa[s2][v4].z, pa[s2][v4].w};
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    acc[v4 * 8 + 2 * e] += wp[s2] * __uint_as_float(wv[e] << 16);
+                    acc[v4 * 8 + 2 * e + 1] += wp[s2] * __uint_as_float(wv[e] & 0xFFFF0000u);
+                  }
+                }
               }
+            // Slots beyond the second (large top-k), two at a time.
+            for (int s2 = 2; s2 < np; s2 += 2) {
+              uint4 pb[2][4];
+#pragma unroll
+              for (int k2 = 0; k2 < 2; ++k2)
+                if (s2 + k2 < np) {
+                  const uint4 *src = reinterpret_cast<const uint4 *>(p.opart + (pbase + s2 + k2) * D + c0);
+#pragma unroll
+                  for (int v4 = 0; v4 < 4; ++v4)
+                    if (v4 * 8 < cols) pb[k2][v4] = src[v4];
+                }
+#pragma unroll
+              for (int k2 = 0; k2 < 2; ++k2)
+                if (s2 + k2 < np) {
+                  const float wk = wp[s2 + k2];
+#pragma unroll
+                  for (int v4 = 0; v4 < 4; ++v4) {
+                    if (v4 * 8 >= cols) break;
+                    const uint32_t wv[4] = {pb[k2][v4].x, pb[k2][v4].y, pb[k2][v4].z, pb[k2][v4].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                      acc[v4 * 8 + 2 * e] += wk * __uint_as_float(wv[e] << 16);
+                      acc[v4 * 8 + 2 * e + 1] += wk * __uint_as_float(wv[e] & 0xFFFF0000u);
+                    }
+                  }
+                }
             }
-            uint4 w0, w1;
-            w0.x = pack_bf16x2(acc[0], acc[1]);
-            w0.y = pack_bf16x2(acc[2], acc[3]);
-            w0.z = pack_bf16x2(acc[4], acc[5]);
-            w0.w = pack_bf16x2(acc[6], acc[7]);
-            w1.x = pack_bf16x2(acc[8], acc[9]);
-            w1.y = pack_bf16x2(acc[10], acc[11]);
-            w1.z = pack_bf16x2(acc[12], acc[13]);
-            w1.w = pack_bf16x2(acc[14], acc[15]);
-            *reinterpret_cast<uint4 *>(dst + c0) = w0;
-            *reinterpret_cast<uint4 *>(dst + c0 + 8) = w1;
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              if (v4 * 8 >= cols) break;
+              uint4 w;
+              w.x = pack_bf16x2(acc[v4 * 8 + 0], acc[v4 * 8 + 1]);
+              w.y = pack_bf16x2(acc[v4 * 8 + 2], acc[v4 * 8 + 3]);
+              w.z = pack_bf16x2(acc[v4 * 8 + 4], acc[v4 * 8 + 5]);
+              w.w = pack_bf16x2(acc[v4 * 8 + 6], acc[v4 * 8 + 7]);
+              *reinterpret_cast<uint4 *>(dst + c0 + v4 * 8) = w;
+            }
           }
         }
         if (live) p.lse[((int64_t)ti.b * p.hq + h) * p.N + i] = lse;

@@ -115,11 +115,10 @@ template <int D>
 __global__ void __launch_bounds__(kGateThreads)
 gate_topk_kernel(const SelectParams p) {
   constexpr int KS = D / 16;           // k-steps
-  constexpr int LDQ = D + 8;           // padded row stride (elements): conflict-free ldmatrix
+  constexpr int LDK = D + 8;           // padded row stride (elements): conflict-free ldmatrix
   extern __shared__ __align__(128) unsigned char smem[];
-  uint16_t *qs = reinterpret_cast<uint16_t *>(smem);                       // [64][LDQ]
-  uint16_t *ks = qs + kGateRows * LDQ;                                     // [2][2][32][LDQ]
-  float *ss = reinterpret_cast<float *>(ks + 2 * 2 * kGateChunk * LDQ);    // [64][lds]
+  uint16_t *ks = reinterpret_cast<uint16_t *>(smem);                       // [2][32][LDK]
+  float *ss = reinterpret_cast<float *>(ks + 2 * kGateChunk * LDK);        // [64][lds]
   const int i0 = blockIdx.x * kGateRows;
   const int h = blockIdx.y, b = blockIdx.z;
   const int hk = h / p.G;
@@ -129,75 +128,81 @@ gate_topk_kernel(const SelectParams p) {
   const int nb = min(p.nblk, (i0 + rows - 1) / p.block);
   const int lds = ((nb + 31) & ~31) + 4;
   int *hist = reinterpret_cast<int *>(ss + kGateRows * lds);               // [nblk]
+  const int wr0 = warp * 16;  // this warp's first row in the tile
+  const int g = lane >> 2, t4 = lane & 3;
 
-  // Stage the query tile and the first chunk of pooled keys.
-  const uint16_t *qg = p.q + b * p.q_sb + h * p.q_sh;
-  for (int e = tid; e < kGateRows * (D / 8); e += kGateThreads) {
-    const int r = e / (D / 8), c = e % (D / 8);
-    const bool ok = r < rows;
-    cp_async_16_zfill(smem_u32(qs + r * LDQ + c * 8), qg + (int64_t)(ok ? i0 + r : i0) * p.q_sn + c * 8, ok);
+  // Query fragments straight from global memory (every load in flight at once):
+  // A of m16n8k16 holds rows g, g+8 and columns 2*t4 (+1), (+8) of each 16-wide step.
+  uint32_t afrag[KS][4];
+  {
+    const uint16_t *qg = p.q + b * p.q_sb + h * p.q_sh;
+    const int ra = i0 + wr0 + g, rb = ra + 8;
+    const bool va = ra < p.N, vb = rb < p.N;
+    const uint32_t *qa = reinterpret_cast<const uint32_t *>(qg + (int64_t)(va ? ra : 0) * p.q_sn);
+    const uint32_t *qb = reinterpret_cast<const uint32_t *>(qg + (int64_t)(vb ? rb : 0) * p.q_sn);
+#pragma unroll
+    for (int s = 0; s < KS; ++s) {
+      const int w0 = s * 8 + t4;  // 32-bit word of column s*16 + 2*t4
+      afrag[s][0] = va ? __ldg(qa + w0) : 0u;
+      afrag[s][1] = vb ? __ldg(qb + w0) : 0u;
+      afrag[s][2] = va ? __ldg(qa + w0 + 4) : 0u;
+      afrag[s][3] = vb ? __ldg(qb + w0 + 4) : 0u;
+    }
   }
+  for (int j = tid; j < p.nblk; j += kGateThreads) hist[j] = 0;
+
   const uint16_t *kb = p.kbar_split + ((int64_t)b * p.hkv + hk) * 2 * p.nblk * D;
-  auto stage_chunk = [&](int ch, int buf) {
+  // Largest own-block index among this warp's rows: n-tiles at or past it are skipped.
+  const int wlast = min(i0 + wr0 + 15, p.N - 1);
+  const int cw = (wr0 < rows) ? wlast / p.block : 0;
+  const int nchunk = (nb + kGateChunk - 1) / kGateChunk;
+  for (int ch = 0; ch < nchunk; ++ch) {
     const int j0 = ch * kGateChunk;
+    if (ch > 0) __syncthreads();  // previous chunk's ldmatrix reads are done
     for (int e = tid; e < 2 * kGateChunk * (D / 8); e += kGateThreads) {
       const int part = e / (kGateChunk * (D / 8));
       const int rem = e % (kGateChunk * (D / 8));
       const int jj = rem / (D / 8), c = rem % (D / 8);
       const bool ok = j0 + jj < nb;
       const uint16_t *src = kb + ((int64_t)part * p.nblk + (ok ? j0 + jj : 0)) * D + c * 8;
-      cp_async_16_zfill(smem_u32(ks + ((buf * 2 + part) * kGateChunk + jj) * LDQ + c * 8), src, ok);
+      cp_async_16_zfill(smem_u32(ks + (part * kGateChunk + jj) * LDK + c * 8), src, ok);
     }
-  };
-  const int nchunk = (nb + kGateChunk - 1) / kGateChunk;
-  if (nchunk > 0) stage_chunk(0, 0);
-  cp_async_commit();
-  for (int j = tid; j < p.nblk; j += kGateThreads) hist[j] = 0;
-
-  const int wr0 = warp * 16;  // this warp's first row in the tile
-  const int g = lane >> 2, t4 = lane & 3;
-  // Largest own-block index among this warp's rows: n-tiles at or past it are skipped.
-  const int wlast = min(i0 + wr0 + 15, p.N - 1);
-  const int cw = (wr0 < rows) ? wlast / p.block : 0;
-
-  uint32_t afrag[KS][4];
-  for (int ch = 0; ch < nchunk; ++ch) {
-    if (ch + 1 < nchunk) stage_chunk(ch + 1, (ch + 1) & 1);
     cp_async_commit();
-    cp_async_wait_group<1>();
+    cp_async_wait_all();
     __syncthreads();
-    if (ch == 0) {
+    // n-tiles of 8 blocks this warp needs in this chunk (warp-uniform).
+    const int ntc = min(kGateChunk / 8, max(0, (cw - j0 + 7) / 8));
+    float acc_hi[kGateChunk / 8][4], acc_lo[kGateChunk / 8][4];
 #pragma unroll
-      for (int s = 0; s < KS; ++s) {
-        const int r = wr0 + (lane & 7) + 8 * ((lane >> 3) & 1);
-        const int c = s * 16 + 8 * (lane >> 4);
-        ldmatrix_x4(smem_u32(qs + r * LDQ + c), afrag[s][0], afrag[s][1], afrag[s][2], afrag[s][3]);
+    for (int nt = 0; nt < kGateChunk / 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) { acc_hi[nt][e] = 0.f; acc_lo[nt][e] = 0.f; }
+#pragma unroll
+    for (int s = 0; s < KS; ++s) {
+#pragma unroll
+      for (int nt = 0; nt < kGateChunk / 8; ++nt) {
+        if (nt < ntc) {
+          // Matrices: (hi, k0..7), (hi, k8..15), (lo, k0..7), (lo, k8..15) for 8 blocks.
+          const int part = (lane >> 4) & 1;
+          const int jj = nt * 8 + (lane & 7);
+          const int c = s * 16 + 8 * ((lane >> 3) & 1);
+          uint32_t h0, h1, l0, l1;
+          ldmatrix_x4(smem_u32(ks + (part * kGateChunk + jj) * LDK + c), h0, h1, l0, l1);
+          mma_bf16_16816(acc_hi[nt], afrag[s], h0, h1);
+          mma_bf16_16816(acc_lo[nt], afrag[s], l0, l1);
+        }
       }
     }
-    const int buf = ch & 1;
-    const int j0 = ch * kGateChunk;
 #pragma unroll
     for (int nt = 0; nt < kGateChunk / 8; ++nt) {
-      if (j0 + nt * 8 >= cw) break;  // every row of the warp has c <= these blocks
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int s = 0; s < KS; ++s) {
-        // Matrices: (hi, k0..7), (hi, k8..15), (lo, k0..7), (lo, k8..15) for 8 blocks.
-        const int part = (lane >> 4) & 1;
-        const int jj = nt * 8 + (lane & 7);
-        const int c = s * 16 + 8 * ((lane >> 3) & 1);
-        uint32_t h0, h1, l0, l1;
-        ldmatrix_x4(smem_u32(ks + ((buf * 2 + part) * kGateChunk + jj) * LDQ + c), h0, h1, l0, l1);
-        mma_bf16_16816(acc, afrag[s], h0, h1);
-        mma_bf16_16816(acc, afrag[s], l0, l1);
+      if (nt < ntc) {
+        const int col = j0 + nt * 8 + 2 * t4;
+        ss[(wr0 + g) * lds + col] = acc_hi[nt][0] + acc_lo[nt][0];
+        ss[(wr0 + g) * lds + col + 1] = acc_hi[nt][1] + acc_lo[nt][1];
+        ss[(wr0 + g + 8) * lds + col] = acc_hi[nt][2] + acc_lo[nt][2];
+        ss[(wr0 + g + 8) * lds + col + 1] = acc_hi[nt][3] + acc_lo[nt][3];
       }
-      const int col = j0 + nt * 8 + 2 * t4;
-      ss[(wr0 + g) * lds + col] = acc[0];
-      ss[(wr0 + g) * lds + col + 1] = acc[1];
-      ss[(wr0 + g + 8) * lds + col] = acc[2];
-      ss[(wr0 + g + 8) * lds + col + 1] = acc[3];
     }
-    __syncthreads();
   }
   cp_async_wait_all();
   __syncthreads();
@@ -205,7 +210,7 @@ gate_topk_kernel(const SelectParams p) {
   // Top-(k-1) over past blocks; one quad of lanes per row, two passes of 8 rows.
   // Every lane runs the warp's largest round count so the shuffles stay converged.
   const int npick_max = p.topk - 1;
-  int *sel_base = reinterpret_cast<int *>(qs);  // reuses the query tile: [64][32]
+  int *sel_base = reinterpret_cast<int *>(ks);  // reuses the key staging: [64][32]
   for (int pass = 0; pass < 2; ++pass) {
     const int r = wr0 + pass * 8 + g;
     const int i = i0 + r;
@@ -394,10 +399,12 @@ cudaError_t launch_pool(const uint16_t *k, int64_t sb, int64_t sh, int64_t sn, i
 }
 
 size_t gate_smem_bytes(int d, int nblk) {
-  const int ldq = d + 8;
+  const int ldk = d + 8;
   const int lds = ((nblk + 31) & ~31) + 4;
-  return sizeof(uint16_t) * (kGateRows * ldq + 2 * 2 * kGateChunk * ldq) +
-         sizeof(float) * kGateRows * lds + sizeof(int) * nblk;
+  // Key staging (also holds the 64 x 32 selection scratch afterwards), scores, counts.
+  const size_t stage = sizeof(uint16_t) * 2 * kGateChunk * ldk;
+  const size_t sel = sizeof(int) * kGateRows * 32;
+  return (stage > sel ? stage : sel) + sizeof(float) * kGateRows * lds + sizeof(int) * nblk;
 }
 
 template <int D>
