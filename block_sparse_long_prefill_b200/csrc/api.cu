@@ -19,8 +19,8 @@ __device__ int g_device_status[2] = {MOBA_OK, 0};
 cudaError_t launch_pool(const uint16_t *k, int64_t sb, int64_t sh, int64_t sn, int batch, int hkv,
                         int N, int d, int block, float *kbar, uint16_t *split, cudaStream_t st);
 cudaError_t launch_gate(const SelectParams &p, cudaStream_t st);
-cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileoff, int nlists,
-                        cudaStream_t st);
+cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileoff, int4 *tiles,
+                        int nlists, cudaStream_t st);
 cudaError_t launch_scatter(const ScatterParams &p, cudaStream_t st);
 cudaError_t launch_attn(const CUtensorMap *maps, const AttnParams &p, int mode, int grid,
                         cudaStream_t st);
@@ -184,7 +184,8 @@ int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, i
   int *cursor = reinterpret_cast<int *>(ws + w.off_cursor);
   int *listoff = reinterpret_cast<int *>(ws + w.off_listoff);
   int *tileoff = reinterpret_cast<int *>(ws + w.off_tileoff);
-  if ((rc = launch_status(launch_scan(counts, cursor, listoff, tileoff, w.nlists, st)))) return rc;
+  int4 *tiles = reinterpret_cast<int4 *>(ws + w.off_tiles);
+  if ((rc = launch_status(launch_scan(counts, cursor, listoff, tileoff, tiles, w.nlists, st)))) return rc;
   ScatterParams cp{};
   cp.idx = idx;
   cp.cursor = cursor;
@@ -231,6 +232,7 @@ int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *id
   p.is_moba = 1;
   p.listoff = reinterpret_cast<const int *>(ws + w.off_listoff);
   p.tileoff = reinterpret_cast<const int *>(ws + w.off_tileoff);
+  p.tiles = reinterpret_cast<const int4 *>(ws + w.off_tiles);
   p.entries = reinterpret_cast<const uint32_t *>(ws + w.off_entries);
   p.opart = reinterpret_cast<uint16_t *>(ws + w.off_opart);
   p.lpart = reinterpret_cast<float *>(ws + w.off_lpart);

@@ -59,7 +59,7 @@ struct AttnCfg {
 
 struct Bars {
   uint64_t q_full[2], q_empty[2];
-  uint64_t k_full[3], v_full[3], kv_empty[3];
+  uint64_t k_full[3], v_full[3], k_empty[3], v_empty[3];
   uint64_t s_full[2];
   uint64_t p_full, o_done, mma_done;
   uint64_t o_full[2], o_free[2], stat_full[2];
@@ -113,26 +113,42 @@ __device__ __forceinline__ void query_major_tile(const AttnParams &p, int t, Til
   }
 }
 
-__device__ __forceinline__ void gathered_tile(const AttnParams &p, int t, TileInfo &ti) {
-  // Binary search the list whose tile range holds t (lists of this chunk only).
-  int lo = p.chunk * p.lists_per_chunk, hi = lo + p.lists_per_chunk;  // tileoff[lo] <= t < tileoff[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(p.tileoff + mid) <= t) lo = mid; else hi = mid;
-  }
-  const int L = lo;
-  const int first = __ldg(p.listoff + L);
-  const int count = __ldg(p.listoff + L + 1) - first;
-  const int start = (t - __ldg(p.tileoff + L)) * kTileRows;
+__device__ __forceinline__ void gathered_tile(const AttnParams &p, int4 rec, TileInfo &ti) {
+  const int L = rec.x;
   ti.list = L;
-  ti.ent0 = first + start;
-  ti.rows = min(kTileRows, count - start);
+  ti.ent0 = rec.y;
+  ti.rows = rec.z;
   ti.j = L % p.nblk;
   ti.hk = (L / p.nblk) % p.hkv;
   ti.b = (L / (p.nblk * p.hkv)) % p.batch;
   ti.h = -1;
+  ti.i0 = 0;
   ti.nc = p.block / kTileKeys;
 }
+
+// Walks this CTA's tiles t = t_begin + blockIdx.x, t += gridDim.x.  Gathered tiles
+// come from the tile table; the next record is loaded one tile ahead.
+template <int MODE>
+struct TileIter {
+  int t, t_end;
+  int4 nxt;
+  __device__ __forceinline__ TileIter(const AttnParams &p, int t_begin, int t_end_) {
+    t = t_begin + (int)blockIdx.x;
+    t_end = t_end_;
+    if (MODE == kGathered && t < t_end) nxt = __ldg(p.tiles + t);
+  }
+  __device__ __forceinline__ bool valid() const { return t < t_end; }
+  __device__ __forceinline__ void get(const AttnParams &p, TileInfo &ti) {
+    if (MODE == kGathered) {
+      const int4 cur = nxt;
+      if (t + (int)gridDim.x < t_end) nxt = __ldg(p.tiles + t + gridDim.x);
+      gathered_tile(p, cur, ti);
+    } else {
+      query_major_tile(p, t, ti);
+    }
+  }
+  __device__ __forceinline__ void next() { t += gridDim.x; }
+};
 
 // Key of chunk m of a tile.
 template <int MODE>
@@ -191,7 +207,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     for (int s = 0; s < 3; ++s) {
       mbar_init(&bar.k_full[s], 1);
       mbar_init(&bar.v_full[s], 1);
-      mbar_init(&bar.kv_empty[s], 1);
+      mbar_init(&bar.k_empty[s], 1);
+      mbar_init(&bar.v_empty[s], 1);
     }
     mbar_init(&bar.s_full[0], 1);
     mbar_init(&bar.s_full[1], 1);
@@ -221,29 +238,36 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t tmem = bar.tmem_base;
   volatile int *abort = &bar.abort;
 
-  // Register split (launch: 384 threads x 168): 128 x (80 + 240 + 184) = 64512.
+  // Register split (launch: 384 threads x 168): see kRegSplitTotal.
   if (warp < 4) {
     setmaxnreg_dec<kRegsWG0>();
     if (warp == 0) {
-      // ---------------------------------------------------------- producer
-      if (lane == 0) {
-        uint32_t kvc = 0;
+      // ---------------------------------------------------------- producers
+      // Lane 0 loads query tiles (query-major) and K chunks; lane 1 loads V chunks.
+      // K and V have separate rings: a K slot frees once its S = Q K^T is done, long
+      // before the V slot of the same chunk (freed by P V).
+      if (lane < 2) {
+        const bool kside = lane == 0;
+        uint64_t *full = kside ? bar.k_full : bar.v_full;
+        uint64_t *empty = kside ? bar.k_empty : bar.v_empty;
+        const CUtensorMap *m0 = kside ? &tmK : &tmV;
+        const CUtensorMap *m1 = kside ? &tmK1 : &tmV1;
+        const int off = kside ? C::K_OFF : C::V_OFF;
+        uint32_t cnt = 0;
         int lt = 0;
         bool ok = true;
-        for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x, ++lt) {
+        for (TileIter<MODE> it(p, t_begin, t_end); ok && it.valid(); it.next(), ++lt) {
           TileInfo ti;
-          if (MODE == kGathered) gathered_tile(p, t, ti); else query_major_tile(p, t, ti);
-          if (MODE == kQueryMajor) {
+          it.get(p, ti);
+          if (MODE == kQueryMajor && kside) {
             if (p.is_moba && p.npast > 0) {
               // The merge reads this tile's partials: pull them into L2 now.
               const int il = ti.i0 - p.chunk * p.chunk_rows;
               const int64_t prow = ((int64_t)ti.b * p.hq + ti.h) * p.chunk_rows + il;
               const char *po = reinterpret_cast<const char *>(p.opart + prow * p.npast * D);
               const uint32_t pbytes = (uint32_t)ti.rows * p.npast * D * 2;
-              for (uint32_t off = 0; off < pbytes; off += 65536)
-                prefetch_l2_bulk(po + off, min(65536u, pbytes - off));
-              const char *pl = reinterpret_cast<const char *>(p.lpart + prow * p.npast);
-              prefetch_l2_bulk(pl, ((uint32_t)ti.rows * p.npast * 4 + 15) & ~15u);
+              for (uint32_t o2 = 0; o2 < pbytes; o2 += 65536)
+                prefetch_l2_bulk(po + o2, min(65536u, pbytes - o2));
             }
             const int qb = lt & 1;
             if (!(ok = mbar_wait(&bar.q_empty[qb], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 1))) break;
@@ -252,27 +276,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tma_load_4d(qd, &tmQ, &bar.q_full[qb], 0, ti.i0, ti.h, ti.b);
             if (D != 64) tma_load_4d(qd + C::R0, &tmQ1, &bar.q_full[qb], 64, ti.i0, ti.h, ti.b);
           }
-          for (int m = 0; m < ti.nc; ++m, ++kvc) {
-            const int st = kvc % C::ST;
-            if (!(ok = mbar_wait(&bar.kv_empty[st], ((kvc / C::ST) & 1) ^ 1, abort, p.status, site0 + 2))) break;
+          for (int m = 0; m < ti.nc; ++m, ++cnt) {
+            const int st = cnt % C::ST;
+            if (!(ok = mbar_wait(&empty[st], ((cnt / C::ST) & 1) ^ 1, abort, p.status, site0 + 2))) break;
             const int key = chunk_key<MODE>(p, ti, m);
-            unsigned char *kd = sbase + C::K_OFF + st * C::TILE;
-            unsigned char *vd = sbase + C::V_OFF + st * C::TILE;
-            mbar_arrive_expect_tx(&bar.k_full[st], C::BYTES);
-            tma_load_4d(kd, &tmK, &bar.k_full[st], 0, key, ti.hk, ti.b);
-            if (D != 64) tma_load_4d(kd + C::R0, &tmK1, &bar.k_full[st], 64, key, ti.hk, ti.b);
-            mbar_arrive_expect_tx(&bar.v_full[st], C::BYTES);
-            tma_load_4d(vd, &tmV, &bar.v_full[st], 0, key, ti.hk, ti.b);
-            if (D != 64) tma_load_4d(vd + C::R0, &tmV1, &bar.v_full[st], 64, key, ti.hk, ti.b);
+            unsigned char *dst = sbase + off + st * C::TILE;
+            mbar_arrive_expect_tx(&full[st], C::BYTES);
+            tma_load_4d(dst, m0, &full[st], 0, key, ti.hk, ti.b);
+            if (D != 64) tma_load_4d(dst + C::R0, m1, &full[st], 64, key, ti.hk, ti.b);
           }
         }
         // Let every load issued so far land before the CTA can retire.
         if (*abort) {
-          for (uint32_t u = (kvc > (uint32_t)C::ST ? kvc - C::ST : 0); u < kvc; ++u) {
-            const int st = u % C::ST;
+          for (uint32_t u = (cnt > (uint32_t)C::ST ? cnt - C::ST : 0); u < cnt; ++u) {
             const unsigned long long t0 = global_timer_ns();
-            while (!mbar_try_wait(&bar.k_full[st], (u / C::ST) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
-            while (!mbar_try_wait(&bar.v_full[st], (u / C::ST) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+            while (!mbar_try_wait(&full[u % C::ST], (u / C::ST) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
           }
         }
       }
@@ -296,9 +314,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (D == 80) umma_ts(tO + 64, a, v_desc<D>(vt, kk, 1), idO16, acc);
           }
         };
-        for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x, ++lt) {
+        for (TileIter<MODE> it(p, t_begin, t_end); ok && it.valid(); it.next(), ++lt) {
           TileInfo ti;
-          if (MODE == kGathered) gathered_tile(p, t, ti); else query_major_tile(p, t, ti);
+          it.get(p, ti);
           const int qb = lt & 1, ob = lt & 1;
           const uint32_t tO = tmem + 256 + 128 * ob;
           if (!(ok = mbar_wait(&bar.q_full[qb], (lt >> 1) & 1, abort, p.status, site0 + 3))) break;
@@ -317,13 +335,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               for (int ks = 0; ks < D / 16; ++ks)
                 umma_ss(sb, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idS, ks > 0 ? 1u : 0u);
               umma_commit(&bar.s_full[scnt & 1]);
+              umma_commit(&bar.k_empty[st]);
               if (m == ti.nc - 1) umma_commit(&bar.q_empty[qb]);
             }
             if (m > 0) {
-              // O += P V for chunk m-1.
+              // O += P V for chunk m-1 (pipeline slot kvc - 1: kvc advances after each S).
               if (!(ok = mbar_wait(&bar.p_full, pcnt & 1, abort, p.status, site0 + 5))) break;
               ++pcnt;
-              // Chunk m-1 used pipeline slot kvc - 1 (kvc advances after each S).
               if (!(ok = mbar_wait(&bar.v_full[prev_st], ((kvc - 1) / C::ST) & 1, abort, p.status, site0 + 6))) break;
               if (m == 1) {
                 if (!(ok = mbar_wait(&bar.o_free[ob], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 7))) break;
@@ -332,7 +350,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               issue_pv(tO, m == 1, prev_sbuf, prev_st);
               if (m < ti.nc) umma_commit(&bar.o_done);
               else umma_commit(&bar.o_full[ob]);
-              umma_commit(&bar.kv_empty[prev_st]);
+              umma_commit(&bar.v_empty[prev_st]);
             }
             if (m < ti.nc) {
               prev_sbuf = tmem + 128 * (scnt & 1);
@@ -355,9 +373,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       constexpr int VPR = D / 8;  // 16-byte vectors per row
       const int npast = p.npast;
       int lt = 0;
-      for (int t = t_begin + blockIdx.x; t < t_end; t += gridDim.x, ++lt) {
+      for (TileIter<MODE> it(p, t_begin, t_end); it.valid(); it.next(), ++lt) {
         TileInfo ti;
-        gathered_tile(p, t, ti);
+        it.get(p, ti);
         const int qb = lt & 1;
         uint32_t ent[2] = {0u, 0u};
 #pragma unroll
@@ -406,9 +424,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     uint32_t scnt = 0, ocnt = 0;
     int lt = 0;
     bool ok = true;
-    for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x, ++lt) {
+    for (TileIter<MODE> it(p, t_begin, t_end); ok && it.valid(); it.next(), ++lt) {
       TileInfo ti;
-      if (MODE == kGathered) gathered_tile(p, t, ti); else query_major_tile(p, t, ti);
+      it.get(p, ti);
       const int ob = lt & 1;
       const uint32_t tO = tmem + lane_off + 256 + 128 * ob;
       const bool live = r < ti.rows;
@@ -541,9 +559,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     int lt = 0;
     bool ok = true;
-    for (int t = t_begin + blockIdx.x; ok && t < t_end; t += gridDim.x, ++lt) {
+    for (TileIter<MODE> it(p, t_begin, t_end); ok && it.valid(); it.next(), ++lt) {
       TileInfo ti;
-      if (MODE == kGathered) gathered_tile(p, t, ti); else query_major_tile(p, t, ti);
+      it.get(p, ti);
       const int ob = lt & 1;
       const uint32_t tO = tmem + lane_off + 256 + 128 * ob;
       const bool live = r < ti.rows;
@@ -555,20 +573,54 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         h = ti.hk * p.G + (int)(ig % (uint32_t)p.G);
         i = (int)(ig / (uint32_t)p.G);
       }
-      // Merge inputs that do not depend on this tile's result: read them first.
-      int np = 0;
-      int64_t pbase = 0;
-      float lp[32];
-      if (MODE == kQueryMajor && live && p.is_moba && p.npast > 0) {
-        const int32_t *irow = p.idx + (((int64_t)ti.b * p.hq + h) * p.N + i) * p.topk;
-        const int c = i / p.block;
-        for (int s2 = 0; s2 < p.npast; ++s2) {
-          const int blk = __ldg(irow + s2);
-          if (blk < 0 || blk >= c) break;
-          ++np;
+      // Query-major MoBA: combine this row's past-block partials while the tile is
+      // still being computed: accp = sum_s exp(lse_s - lse_p) o_s, lse_p = logsumexp.
+      float accp[D];
+      float lse_p = -INFINITY;
+      if (MODE == kQueryMajor && p.is_moba && p.npast > 0) {
+        int np = 0;
+        int64_t pbase = 0;
+        if (live) {
+          const int32_t *irow = p.idx + (((int64_t)ti.b * p.hq + h) * p.N + i) * p.topk;
+          const int c = i / p.block;
+          for (int s2 = 0; s2 < p.npast; ++s2) {
+            const int blk = __ldg(irow + s2);
+            if (blk < 0 || blk >= c) break;
+            ++np;
+          }
+          pbase = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + (i - p.chunk * p.chunk_rows)) * p.npast;
         }
-        pbase = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + (i - p.chunk * p.chunk_rows)) * p.npast;
-        for (int s2 = 0; s2 < np; ++s2) lp[s2] = p.lpart[pbase + s2];
+#pragma unroll
+        for (int c = 0; c < D; ++c) accp[c] = 0.f;
+        if (np > 0) {
+          float mx = -INFINITY;
+          for (int s2 = 0; s2 < np; ++s2) mx = fmaxf(mx, p.lpart[pbase + s2]);
+          float tot = 0.f;
+          for (int s2 = 0; s2 < np; ++s2) tot += __expf(p.lpart[pbase + s2] - mx);
+          lse_p = mx + __logf(tot);
+          for (int s2 = 0; s2 < np; ++s2) {
+            const float wgt = __expf(p.lpart[pbase + s2] - lse_p);
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.opart + (pbase + s2) * D);
+            // Half a row (up to 8 x 16 bytes) per round, all in flight together.
+#pragma unroll
+            for (int h0 = 0; h0 < D / 8; h0 += 8) {
+              uint4 v[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                if (h0 + j < D / 8) v[j] = src[h0 + j];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                if (h0 + j >= D / 8) break;
+                const uint32_t wv[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  accp[(h0 + j) * 8 + 2 * e] += wgt * __uint_as_float(wv[e] << 16);
+                  accp[(h0 + j) * 8 + 2 * e + 1] += wgt * __uint_as_float(wv[e] & 0xFFFF0000u);
+                }
+              }
+            }
+          }
+        }
       }
       ok = mbar_wait(&bar.stat_full[ob], (lt >> 1) & 1, abort, p.status, site0 + 15);
       ok = ok && mbar_wait(&bar.o_full[ob], (lt >> 1) & 1, abort, p.status, site0 + 16);
@@ -603,100 +655,39 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
         if (live) p.lpart[pidx] = own_lse;
       } else {
-        // Merge with the past-block partials of this row (MoBA), then store.
-        float wown = 1.f, lse = own_lse;
-        float wp[32];
-        if (np > 0) {
-          float mx = own_lse;
-          for (int s2 = 0; s2 < np; ++s2) mx = fmaxf(mx, lp[s2]);
-          float tot = __expf(own_lse - mx);
-          for (int s2 = 0; s2 < np; ++s2) tot += __expf(lp[s2] - mx);
-          lse = mx + __logf(tot);
-          wown = __expf(own_lse - lse);
-          for (int s2 = 0; s2 < np; ++s2) wp[s2] = __expf(lp[s2] - lse);
+        // out = a * O + b * accp with a = exp(own - lse) / l, b = exp(lse_p - lse).
+        float lse = own_lse, a = inv_l, bw = 0.f;
+        if (lse_p != -INFINITY) {
+          const float mx = fmaxf(own_lse, lse_p);
+          lse = mx + __logf(__expf(own_lse - mx) + __expf(lse_p - mx));
+          a = __expf(own_lse - lse) * inv_l;
+          bw = __expf(lse_p - lse);
         }
         uint16_t *dst = p.out + ti.b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)i * p.o_sn;
-        // 32 columns at a time: the partial pieces of up to two slots are loaded
-        // together before the TMEM read, so their latencies overlap.
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          constexpr int W = (D == 80) ? 16 : 32;  // D = 80: pieces of 32, 32, 16
-          (void)W;
-          const int cols = (D - c0) < 32 ? (D - c0) : 32;
-          uint32_t o[32];
+        for (int c0 = 0; c0 < D; c0 += 16) {
+          uint32_t o[16];
           __syncwarp();
-          if (cols == 32) {
-            tmem_ld32(tO + c0, o);
-          } else {
-            tmem_ld16(tO + c0, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
-          }
-          float acc[32];
-          uint4 pa[2][4];
-          if (live && np > 0) {
-#pragma unroll
-            for (int s2 = 0; s2 < 2; ++s2)
-              if (s2 < np) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(p.opart + (pbase + s2) * D + c0);
-#pragma unroll
-                for (int v4 = 0; v4 < 4; ++v4)
-                  if (v4 * 8 < cols) pa[s2][v4] = src[v4];
-              }
-          }
+          tmem_ld16(tO + c0, o);
           tmem_wait_ld();
           if (live) {
+            float y[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(o[e]) * inv_l * wown;
-#pragma unroll
-            for (int s2 = 0; s2 < 2; ++s2)
-              if (s2 < np) {
-#pragma unroll
-                for (int v4 = 0; v4 < 4; ++v4) {
-                  if (v4 * 8 >= cols) break;
-                  const uint32_t wv[4] = {pa[s2][v4].x, pa[s2][v4].y, pa[s2][v4].z, pa[s2][v4].w};
-#pragma unroll
-                  for (int e = 0; e < 4; ++e) {
-                    acc[v4 * 8 + 2 * e] += wp[s2] * __uint_as_float(wv[e] << 16);
-                    acc[v4 * 8 + 2 * e + 1] += wp[s2] * __uint_as_float(wv[e] & 0xFFFF0000u);
-                  }
-                }
-              }
-            // Slots beyond the second (large top-k), two at a time.
-            for (int s2 = 2; s2 < np; s2 += 2) {
-              uint4 pb[2][4];
-#pragma unroll
-              for (int k2 = 0; k2 < 2; ++k2)
-                if (s2 + k2 < np) {
-                  const uint4 *src = reinterpret_cast<const uint4 *>(p.opart + (pbase + s2 + k2) * D + c0);
-#pragma unroll
-                  for (int v4 = 0; v4 < 4; ++v4)
-                    if (v4 * 8 < cols) pb[k2][v4] = src[v4];
-                }
-#pragma unroll
-              for (int k2 = 0; k2 < 2; ++k2)
-                if (s2 + k2 < np) {
-                  const float wk = wp[s2 + k2];
-#pragma unroll
-                  for (int v4 = 0; v4 < 4; ++v4) {
-                    if (v4 * 8 >= cols) break;
-                    const uint32_t wv[4] = {pb[k2][v4].x, pb[k2][v4].y, pb[k2][v4].z, pb[k2][v4].w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                      acc[v4 * 8 + 2 * e] += wk * __uint_as_float(wv[e] << 16);
-                      acc[v4 * 8 + 2 * e + 1] += wk * __uint_as_float(wv[e] & 0xFFFF0000u);
-                    }
-                  }
-                }
+            for (int e = 0; e < 16; ++e) {
+              const float pv = (MODE == kQueryMajor && p.is_moba && p.npast > 0) ? accp[c0 + e] : 0.f;
+              y[e] = fmaf(a, __uint_as_float(o[e]), bw * pv);
             }
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) {
-              if (v4 * 8 >= cols) break;
-              uint4 w;
-              w.x = pack_bf16x2(acc[v4 * 8 + 0], acc[v4 * 8 + 1]);
-              w.y = pack_bf16x2(acc[v4 * 8 + 2], acc[v4 * 8 + 3]);
-              w.z = pack_bf16x2(acc[v4 * 8 + 4], acc[v4 * 8 + 5]);
-              w.w = pack_bf16x2(acc[v4 * 8 + 6], acc[v4 * 8 + 7]);
-              *reinterpret_cast<uint4 *>(dst + c0 + v4 * 8) = w;
-            }
+            uint4 w0, w1;
+            w0.x = pack_bf16x2(y[0], y[1]);
+            w0.y = pack_bf16x2(y[2], y[3]);
+            w0.z = pack_bf16x2(y[4], y[5]);
+            w0.w = pack_bf16x2(y[6], y[7]);
+            w1.x = pack_bf16x2(y[8], y[9]);
+            w1.y = pack_bf16x2(y[10], y[11]);
+            w1.z = pack_bf16x2(y[12], y[13]);
+            w1.w = pack_bf16x2(y[14], y[15]);
+            *reinterpret_cast<uint4 *>(dst + c0) = w0;
+            *reinterpret_cast<uint4 *>(dst + c0 + 8) = w1;
           }
         }
         if (live) p.lse[((int64_t)ti.b * p.hq + h) * p.N + i] = lse;

@@ -4,6 +4,7 @@
 
 #include <stddef.h>
 #include <stdint.h>
+#include <vector_types.h>
 
 namespace moba {
 
@@ -26,10 +27,12 @@ struct WorkspaceLayout {
   size_t off_listoff;  // int32 [nlists + 1]   exclusive prefix of counts
   size_t off_tileoff;  // int32 [nlists + 1]   exclusive prefix of ceil(count / 128)
   size_t off_entries;  // uint32 [max_entries] entry = (i * G + g) * npast + slot
+  size_t off_tiles;    // int4 [max_tiles]      per 128-row tile: list, first entry, rows
   size_t off_opart;    // bf16 [batch, hq, chunk_rows, npast, d]
   size_t off_lpart;    // f32  [batch, hq, chunk_rows, npast]
   size_t total;
   long long max_entries;
+  long long max_tiles;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -50,12 +53,14 @@ inline WorkspaceLayout make_layout(int batch, int hq, int hkv, int N, int d, int
   w.nchunks = static_cast<int>((N + w.chunk_rows - 1) / w.chunk_rows);
   w.nlists = w.nchunks * batch * hkv * w.nblk;
   w.max_entries = static_cast<long long>(batch) * hq * N * w.npast;
+  w.max_tiles = w.max_entries / kTileRows + w.nlists + 1;
   size_t off = 0;
   w.off_counts = off;  off = align_up(off + sizeof(int) * size_t(w.nlists), 256);
   w.off_cursor = off;  off = align_up(off + sizeof(int) * size_t(w.nlists), 256);
   w.off_listoff = off; off = align_up(off + sizeof(int) * size_t(w.nlists + 1), 256);
   w.off_tileoff = off; off = align_up(off + sizeof(int) * size_t(w.nlists + 1), 256);
   w.off_entries = off; off = align_up(off + sizeof(uint32_t) * size_t(w.max_entries), 256);
+  w.off_tiles = off;   off = align_up(off + 16 * size_t(w.max_tiles), 256);
   const size_t prow = size_t(batch) * hq * size_t(w.chunk_rows) * size_t(w.npast);
   w.off_opart = off;   off = align_up(off + prow * size_t(d) * 2, 256);
   w.off_lpart = off;   off = align_up(off + prow * sizeof(float), 256);
@@ -105,6 +110,7 @@ struct AttnParams {
   // Block-major lists and partials (MoBA).
   const int *listoff;
   const int *tileoff;
+  const int4 *tiles;       // per gathered tile: list, first entry, rows
   const uint32_t *entries;
   uint16_t *opart;         // [batch, hq, chunk_rows, npast, d]
   float *lpart;            // [batch, hq, chunk_rows, npast]

@@ -278,7 +278,7 @@ constexpr int kScanThreads = 1024;
 
 __global__ void __launch_bounds__(kScanThreads)
 list_scan_kernel(const int *__restrict__ counts, int *__restrict__ cursor, int *__restrict__ listoff,
-                 int *__restrict__ tileoff, int nlists) {
+                 int *__restrict__ tileoff, int4 *__restrict__ tiles, int nlists) {
   __shared__ int warp_e[32], warp_t[32];
   __shared__ int carry_e, carry_t;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -326,6 +326,14 @@ list_scan_kernel(const int *__restrict__ counts, int *__restrict__ cursor, int *
   if (tid == 0) {
     listoff[nlists] = carry_e;
     tileoff[nlists] = carry_t;
+  }
+  __syncthreads();
+  // Tile table: one {list, first entry, rows} record per 128-entry tile, so the
+  // attention kernel reads a tile's description with a single load.
+  for (int L = tid; L < nlists; L += kScanThreads) {
+    const int first = listoff[L], cnt = counts[L], t0 = tileoff[L];
+    for (int k = 0; k * kTileRows < cnt; ++k)
+      tiles[t0 + k] = make_int4(L, first + k * kTileRows, min(kTileRows, cnt - k * kTileRows), 0);
   }
 }
 
@@ -427,9 +435,9 @@ cudaError_t launch_gate(const SelectParams &p, cudaStream_t st) {
   }
 }
 
-cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileoff, int nlists,
-                        cudaStream_t st) {
-  list_scan_kernel<<<1, kScanThreads, 0, st>>>(counts, cursor, listoff, tileoff, nlists);
+cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileoff, int4 *tiles,
+                        int nlists, cudaStream_t st) {
+  list_scan_kernel<<<1, kScanThreads, 0, st>>>(counts, cursor, listoff, tileoff, tiles, nlists);
   return cudaGetLastError();
 }
 
