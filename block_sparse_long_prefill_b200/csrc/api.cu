@@ -24,6 +24,7 @@ cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileo
 cudaError_t launch_scatter(const ScatterParams &p, cudaStream_t st);
 cudaError_t launch_attn(const CUtensorMap *maps, const AttnParams &p, int mode, int grid,
                         cudaStream_t st);
+cudaError_t launch_merge(const MergeParams &p, cudaStream_t st);
 
 namespace {
 
@@ -252,6 +253,20 @@ int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *id
     p.ntiles = nq * hq * batch;
     const int grid = p.ntiles < nsm ? p.ntiles : nsm;
     if ((rc = launch_status(launch_attn(maps, p, kQueryMajor, grid, st)))) return rc;
+    if (w.npast > 0) {
+      MergeParams mp{};
+      mp.opart = p.opart;
+      mp.lpart = p.lpart;
+      mp.idx = idx;
+      mp.out = p.out;
+      mp.o_sb = out.sb; mp.o_sh = out.sh; mp.o_sn = out.sn;
+      mp.lse = lse;
+      mp.batch = batch; mp.hq = hq; mp.N = N; mp.d = d; mp.block = block; mp.topk = topk;
+      mp.chunk_rows = w.chunk_rows;
+      mp.row_begin = p.row_begin;
+      mp.row_end = p.row_end;
+      if ((rc = launch_status(launch_merge(mp, st)))) return rc;
+    }
   }
   return MOBA_OK;
 }

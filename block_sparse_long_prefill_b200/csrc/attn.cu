@@ -260,15 +260,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           TileInfo ti;
           it.get(p, ti);
           if (MODE == kQueryMajor && kside) {
-            if (p.is_moba && p.npast > 0) {
-              // The merge reads this tile's partials: pull them into L2 now.
-              const int il = ti.i0 - p.chunk * p.chunk_rows;
-              const int64_t prow = ((int64_t)ti.b * p.hq + ti.h) * p.chunk_rows + il;
-              const char *po = reinterpret_cast<const char *>(p.opart + prow * p.npast * D);
-              const uint32_t pbytes = (uint32_t)ti.rows * p.npast * D * 2;
-              for (uint32_t o2 = 0; o2 < pbytes; o2 += 65536)
-                prefetch_l2_bulk(po + o2, min(65536u, pbytes - o2));
-            }
             const int qb = lt & 1;
             if (!(ok = mbar_wait(&bar.q_empty[qb], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 1))) break;
             unsigned char *qd = sbase + C::Q_OFF + qb * C::TILE;
@@ -301,6 +292,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         constexpr uint32_t idO64 = idesc_bf16(128, 64, 0, 1);
         constexpr uint32_t idO16 = idesc_bf16(128, 16, 0, 1);
         uint32_t kvc = 0, scnt = 0, pcnt = 0;
+        uint32_t ofree_uses[2] = {0u, 0u};  // tiles started per O buffer
+        auto ofree_parity = [&](int b) -> uint32_t { return ((ofree_uses[b]++) & 1) ^ 1; };
         int lt = 0;
         bool ok = true;
         auto issue_pv = [&](uint32_t tO, int first, uint32_t sbuf, int st) {
@@ -314,6 +307,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (D == 80) umma_ts(tO + 64, a, v_desc<D>(vt, kk, 1), idO16, acc);
           }
         };
+        // Chunks of consecutive tiles form one stream: S of chunk g is issued before
+        // P V of chunk g-1, also across a tile boundary, so the next tile's first
+        // S = Q K^T overlaps the current tile's last softmax.
+        struct Pending { bool valid, first, last; uint32_t sbuf, tO; int st, ob; };
+        Pending pend = {false, false, false, 0u, 0u, 0, 0};
+        uint32_t pv_slot = 0;  // pipeline slot of the pending P V
+        auto issue_pending = [&]() -> bool {
+          if (!mbar_wait(&bar.p_full, pcnt & 1, abort, p.status, site0 + 5)) return false;
+          ++pcnt;
+          if (!mbar_wait(&bar.v_full[pend.st], (pv_slot / C::ST) & 1, abort, p.status, site0 + 6)) return false;
+          if (pend.first) {
+            if (!mbar_wait(&bar.o_free[pend.ob], ofree_parity(pend.ob), abort, p.status, site0 + 7)) return false;
+          }
+          tc_fence_after();
+          issue_pv(pend.tO, pend.first, pend.sbuf, pend.st);
+          if (pend.last) umma_commit(&bar.o_full[pend.ob]);
+          else umma_commit(&bar.o_done);
+          umma_commit(&bar.v_empty[pend.st]);
+          pend.valid = false;
+          return true;
+        };
         for (TileIter<MODE> it(p, t_begin, t_end); ok && it.valid(); it.next(), ++lt) {
           TileInfo ti;
           it.get(p, ti);
@@ -322,44 +336,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (!(ok = mbar_wait(&bar.q_full[qb], (lt >> 1) & 1, abort, p.status, site0 + 3))) break;
           tc_fence_after();
           const uint32_t qt = base + C::Q_OFF + qb * C::TILE;
-          uint32_t prev_sbuf = 0;
-          int prev_st = 0;
-          for (int m = 0; m <= ti.nc; ++m) {
-            if (m < ti.nc) {
-              const int st = kvc % C::ST;
-              if (!(ok = mbar_wait(&bar.k_full[st], (kvc / C::ST) & 1, abort, p.status, site0 + 4))) break;
-              tc_fence_after();
-              const uint32_t kt = base + C::K_OFF + st * C::TILE;
-              const uint32_t sb = tmem + 128 * (scnt & 1);
+          for (int m = 0; m < ti.nc; ++m) {
+            const int st = kvc % C::ST;
+            if (!(ok = mbar_wait(&bar.k_full[st], (kvc / C::ST) & 1, abort, p.status, site0 + 4))) break;
+            tc_fence_after();
+            const uint32_t kt = base + C::K_OFF + st * C::TILE;
+            const uint32_t sb = tmem + 128 * (scnt & 1);
 #pragma unroll
-              for (int ks = 0; ks < D / 16; ++ks)
-                umma_ss(sb, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idS, ks > 0 ? 1u : 0u);
-              umma_commit(&bar.s_full[scnt & 1]);
-              umma_commit(&bar.k_empty[st]);
-              if (m == ti.nc - 1) umma_commit(&bar.q_empty[qb]);
-            }
-            if (m > 0) {
-              // O += P V for chunk m-1 (pipeline slot kvc - 1: kvc advances after each S).
-              if (!(ok = mbar_wait(&bar.p_full, pcnt & 1, abort, p.status, site0 + 5))) break;
-              ++pcnt;
-              if (!(ok = mbar_wait(&bar.v_full[prev_st], ((kvc - 1) / C::ST) & 1, abort, p.status, site0 + 6))) break;
-              if (m == 1) {
-                if (!(ok = mbar_wait(&bar.o_free[ob], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 7))) break;
-              }
-              tc_fence_after();
-              issue_pv(tO, m == 1, prev_sbuf, prev_st);
-              if (m < ti.nc) umma_commit(&bar.o_done);
-              else umma_commit(&bar.o_full[ob]);
-              umma_commit(&bar.v_empty[prev_st]);
-            }
-            if (m < ti.nc) {
-              prev_sbuf = tmem + 128 * (scnt & 1);
-              prev_st = kvc % C::ST;
-              ++scnt;
-              ++kvc;
-            }
+            for (int ks = 0; ks < D / 16; ++ks)
+              umma_ss(sb, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idS, ks > 0 ? 1u : 0u);
+            umma_commit(&bar.s_full[scnt & 1]);
+            umma_commit(&bar.k_empty[st]);
+            if (m == ti.nc - 1) umma_commit(&bar.q_empty[qb]);
+            if (pend.valid && !(ok = issue_pending())) break;
+            pend = {true, m == 0, m == ti.nc - 1, sb, tO, st, ob};
+            pv_slot = kvc;
+            ++scnt;
+            ++kvc;
           }
         }
+        if (ok && pend.valid) ok = issue_pending();
         // Every MMA issued so far completes before TMEM is released.
         umma_commit(&bar.mma_done);
         const unsigned long long t0 = global_timer_ns();
@@ -573,55 +569,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         h = ti.hk * p.G + (int)(ig % (uint32_t)p.G);
         i = (int)(ig / (uint32_t)p.G);
       }
-      // Query-major MoBA: combine this row's past-block partials while the tile is
-      // still being computed: accp = sum_s exp(lse_s - lse_p) o_s, lse_p = logsumexp.
-      float accp[D];
-      float lse_p = -INFINITY;
-      if (MODE == kQueryMajor && p.is_moba && p.npast > 0) {
-        int np = 0;
-        int64_t pbase = 0;
-        if (live) {
-          const int32_t *irow = p.idx + (((int64_t)ti.b * p.hq + h) * p.N + i) * p.topk;
-          const int c = i / p.block;
-          for (int s2 = 0; s2 < p.npast; ++s2) {
-            const int blk = __ldg(irow + s2);
-            if (blk < 0 || blk >= c) break;
-            ++np;
-          }
-          pbase = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + (i - p.chunk * p.chunk_rows)) * p.npast;
-        }
-#pragma unroll
-        for (int c = 0; c < D; ++c) accp[c] = 0.f;
-        if (np > 0) {
-          float mx = -INFINITY;
-          for (int s2 = 0; s2 < np; ++s2) mx = fmaxf(mx, p.lpart[pbase + s2]);
-          float tot = 0.f;
-          for (int s2 = 0; s2 < np; ++s2) tot += __expf(p.lpart[pbase + s2] - mx);
-          lse_p = mx + __logf(tot);
-          for (int s2 = 0; s2 < np; ++s2) {
-            const float wgt = __expf(p.lpart[pbase + s2] - lse_p);
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.opart + (pbase + s2) * D);
-            // Half a row (up to 8 x 16 bytes) per round, all in flight together.
-#pragma unroll
-            for (int h0 = 0; h0 < D / 8; h0 += 8) {
-              uint4 v[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-                if (h0 + j < D / 8) v[j] = src[h0 + j];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                if (h0 + j >= D / 8) break;
-                const uint32_t wv[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  accp[(h0 + j) * 8 + 2 * e] += wgt * __uint_as_float(wv[e] << 16);
-                  accp[(h0 + j) * 8 + 2 * e + 1] += wgt * __uint_as_float(wv[e] & 0xFFFF0000u);
-                }
-              }
-            }
-          }
-        }
-      }
       ok = mbar_wait(&bar.stat_full[ob], (lt >> 1) & 1, abort, p.status, site0 + 15);
       ok = ok && mbar_wait(&bar.o_full[ob], (lt >> 1) & 1, abort, p.status, site0 + 16);
       if (!(ok = __all_sync(FULL, ok))) break;
@@ -630,68 +577,41 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const float m_run = st.x, l_run = st.y;
       const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
       const float own_lse = (m_run + log2f(l_run)) * 0.69314718055994530942f;  // natural log
-      if (MODE == kGathered) {
-        const int64_t pidx = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + (i - p.chunk * p.chunk_rows)) * p.npast + slot;
-        uint16_t *dst = p.opart + pidx * D;
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 16) {
-          uint32_t o[16];
-          __syncwarp();
-          tmem_ld16(tO + c0, o);
-          tmem_wait_ld();
-          if (live) {
-            uint4 w0, w1;
-            w0.x = pack_bf16x2(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l);
-            w0.y = pack_bf16x2(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l);
-            w0.z = pack_bf16x2(__uint_as_float(o[4]) * inv_l, __uint_as_float(o[5]) * inv_l);
-            w0.w = pack_bf16x2(__uint_as_float(o[6]) * inv_l, __uint_as_float(o[7]) * inv_l);
-            w1.x = pack_bf16x2(__uint_as_float(o[8]) * inv_l, __uint_as_float(o[9]) * inv_l);
-            w1.y = pack_bf16x2(__uint_as_float(o[10]) * inv_l, __uint_as_float(o[11]) * inv_l);
-            w1.z = pack_bf16x2(__uint_as_float(o[12]) * inv_l, __uint_as_float(o[13]) * inv_l);
-            w1.w = pack_bf16x2(__uint_as_float(o[14]) * inv_l, __uint_as_float(o[15]) * inv_l);
-            *reinterpret_cast<uint4 *>(dst + c0) = w0;
-            *reinterpret_cast<uint4 *>(dst + c0 + 8) = w1;
-          }
-        }
-        if (live) p.lpart[pidx] = own_lse;
+      // Destination: a partial slot (gathered tiles: the row's past-block slot; MoBA
+      // query-major tiles: the own-block slot topk-1, merged afterwards), or the
+      // output itself when nothing needs merging (SWA, or topk = 1).
+      uint16_t *dst;
+      float *ldst;
+      if (MODE == kGathered || (p.is_moba && p.npast > 0)) {
+        const int sl = (MODE == kGathered) ? slot : p.npast;
+        const int64_t pidx = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + (i - p.chunk * p.chunk_rows)) * p.topk + sl;
+        dst = p.opart + pidx * D;
+        ldst = p.lpart + pidx;
       } else {
-        // out = a * O + b * accp with a = exp(own - lse) / l, b = exp(lse_p - lse).
-        float lse = own_lse, a = inv_l, bw = 0.f;
-        if (lse_p != -INFINITY) {
-          const float mx = fmaxf(own_lse, lse_p);
-          lse = mx + __logf(__expf(own_lse - mx) + __expf(lse_p - mx));
-          a = __expf(own_lse - lse) * inv_l;
-          bw = __expf(lse_p - lse);
-        }
-        uint16_t *dst = p.out + ti.b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)i * p.o_sn;
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 16) {
-          uint32_t o[16];
-          __syncwarp();
-          tmem_ld16(tO + c0, o);
-          tmem_wait_ld();
-          if (live) {
-            float y[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float pv = (MODE == kQueryMajor && p.is_moba && p.npast > 0) ? accp[c0 + e] : 0.f;
-              y[e] = fmaf(a, __uint_as_float(o[e]), bw * pv);
-            }
-            uint4 w0, w1;
-            w0.x = pack_bf16x2(y[0], y[1]);
-            w0.y = pack_bf16x2(y[2], y[3]);
-            w0.z = pack_bf16x2(y[4], y[5]);
-            w0.w = pack_bf16x2(y[6], y[7]);
-            w1.x = pack_bf16x2(y[8], y[9]);
-            w1.y = pack_bf16x2(y[10], y[11]);
-            w1.z = pack_bf16x2(y[12], y[13]);
-            w1.w = pack_bf16x2(y[14], y[15]);
-            *reinterpret_cast<uint4 *>(dst + c0) = w0;
-            *reinterpret_cast<uint4 *>(dst + c0 + 8) = w1;
-          }
-        }
-        if (live) p.lse[((int64_t)ti.b * p.hq + h) * p.N + i] = lse;
+        dst = p.out + ti.b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)i * p.o_sn;
+        ldst = p.lse + ((int64_t)ti.b * p.hq + h) * p.N + i;
       }
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 16) {
+        uint32_t o[16];
+        __syncwarp();
+        tmem_ld16(tO + c0, o);
+        tmem_wait_ld();
+        if (live) {
+          uint4 w0, w1;
+          w0.x = pack_bf16x2(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l);
+          w0.y = pack_bf16x2(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l);
+          w0.z = pack_bf16x2(__uint_as_float(o[4]) * inv_l, __uint_as_float(o[5]) * inv_l);
+          w0.w = pack_bf16x2(__uint_as_float(o[6]) * inv_l, __uint_as_float(o[7]) * inv_l);
+          w1.x = pack_bf16x2(__uint_as_float(o[8]) * inv_l, __uint_as_float(o[9]) * inv_l);
+          w1.y = pack_bf16x2(__uint_as_float(o[10]) * inv_l, __uint_as_float(o[11]) * inv_l);
+          w1.z = pack_bf16x2(__uint_as_float(o[12]) * inv_l, __uint_as_float(o[13]) * inv_l);
+          w1.w = pack_bf16x2(__uint_as_float(o[14]) * inv_l, __uint_as_float(o[15]) * inv_l);
+          *reinterpret_cast<uint4 *>(dst + c0) = w0;
+          *reinterpret_cast<uint4 *>(dst + c0 + 8) = w1;
+        }
+      }
+      if (live) *ldst = own_lse;
       tc_fence_before();
       mbar_arrive(&bar.o_free[ob]);
     }

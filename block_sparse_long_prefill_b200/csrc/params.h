@@ -28,8 +28,9 @@ struct WorkspaceLayout {
   size_t off_tileoff;  // int32 [nlists + 1]   exclusive prefix of ceil(count / 128)
   size_t off_entries;  // uint32 [max_entries] entry = (i * G + g) * npast + slot
   size_t off_tiles;    // int4 [max_tiles]      per 128-row tile: list, first entry, rows
-  size_t off_opart;    // bf16 [batch, hq, chunk_rows, npast, d]
-  size_t off_lpart;    // f32  [batch, hq, chunk_rows, npast]
+  size_t off_opart;    // bf16 [batch, hq, chunk_rows, topk, d]: slots 0..npast-1 past
+                       //      blocks, slot npast the own block
+  size_t off_lpart;    // f32  [batch, hq, chunk_rows, topk]
   size_t total;
   long long max_entries;
   long long max_tiles;
@@ -43,7 +44,9 @@ inline WorkspaceLayout make_layout(int batch, int hq, int hkv, int N, int d, int
   w.nblk = N / block;
   w.G = hq / hkv;
   w.npast = topk - 1;
-  const size_t per_row = size_t(w.npast) * (size_t(d) * 2 + 4) * size_t(batch) * size_t(hq);
+  // Partials exist only when a row can attend past blocks: topk slots per row then.
+  const size_t nslots = w.npast > 0 ? size_t(topk) : 0;
+  const size_t per_row = nslots * (size_t(d) * 2 + 4) * size_t(batch) * size_t(hq);
   long long rows = N;
   if (per_row > 0 && per_row * size_t(N) > kPartialCapBytes) {
     rows = static_cast<long long>(kPartialCapBytes / per_row) / kTileRows * kTileRows;
@@ -61,7 +64,7 @@ inline WorkspaceLayout make_layout(int batch, int hq, int hkv, int N, int d, int
   w.off_tileoff = off; off = align_up(off + sizeof(int) * size_t(w.nlists + 1), 256);
   w.off_entries = off; off = align_up(off + sizeof(uint32_t) * size_t(w.max_entries), 256);
   w.off_tiles = off;   off = align_up(off + 16 * size_t(w.max_tiles), 256);
-  const size_t prow = size_t(batch) * hq * size_t(w.chunk_rows) * size_t(w.npast);
+  const size_t prow = size_t(batch) * hq * size_t(w.chunk_rows) * nslots;
   w.off_opart = off;   off = align_up(off + prow * size_t(d) * 2, 256);
   w.off_lpart = off;   off = align_up(off + prow * sizeof(float), 256);
   w.total = off;
@@ -112,9 +115,20 @@ struct AttnParams {
   const int *tileoff;
   const int4 *tiles;       // per gathered tile: list, first entry, rows
   const uint32_t *entries;
-  uint16_t *opart;         // [batch, hq, chunk_rows, npast, d]
-  float *lpart;            // [batch, hq, chunk_rows, npast]
+  uint16_t *opart;         // [batch, hq, chunk_rows, topk, d]
+  float *lpart;            // [batch, hq, chunk_rows, topk]
   int chunk, chunk_rows, npast, nblk, lists_per_chunk;
+};
+
+// Parameters of the merge pass (one query chunk).
+struct MergeParams {
+  const uint16_t *opart;   // [batch, hq, chunk_rows, topk, d]
+  const float *lpart;      // [batch, hq, chunk_rows, topk]
+  const int32_t *idx;      // [batch, hq, N, topk]
+  uint16_t *out;
+  int64_t o_sb, o_sh, o_sn;
+  float *lse;              // [batch, hq, N]
+  int batch, hq, N, d, block, topk, chunk_rows, row_begin, row_end;
 };
 
 }  // namespace moba
