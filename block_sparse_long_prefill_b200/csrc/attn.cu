@@ -14,14 +14,17 @@
 //                whole past block they picked (steps 3-4, causal=False); writes a
 //                normalised partial output and its log-sum-exp per (row, slot).
 //
-// Per CTA (384 threads, one CTA per SM, 512 TMEM columns), FA4-style roles:
-//   warp 0       TMA producer: K/V chunks of 128 keys, the query tile (query-major) and
-//                L2 prefetch of the partials the merge will read
+// Per CTA (512 threads, one CTA per SM, 512 TMEM columns):
+//   warp 0       TMA producers: lane 0 the query tile (query-major) and K chunks of 128
+//                keys, lane 1 the V chunks (separate K and V rings)
 //   warp 1       tcgen05 MMA issuer (one thread) and TMEM owner
 //   warps 2-3    query-row gather with cp.async (gathered tiles)
-//   warps 4-7    softmax: thread r owns row r (TMEM lane r); S -> P in place, rescales
-//                O only when its running maximum grows by more than 2^8
-//   warps 8-11   epilogue: normalises O, merges / stores, then frees the O buffer
+//   warps 4-11   softmax, two warpgroups: thread r of group h owns row r (TMEM lane r)
+//                and keys [64 h, 64 h + 64) of each chunk; the two halves of a row
+//                exchange their maxima through shared memory; S -> P in place; O is
+//                rescaled only when the running maximum grows by more than 2^8
+//   warps 12-15  epilogue: normalises O and stores it (a partial or the output),
+//                then frees the O buffer
 // TMEM: S/P double buffer at columns [0,128) and [128,256); O double buffer at
 // [256,384) and [384,512), so a tile's epilogue overlaps the next tile's MMAs.
 // S = Q K^T is an SS MMA; P (bf16) overwrites its own S columns and is the A operand
@@ -36,12 +39,13 @@
 
 namespace moba {
 
-constexpr int kAttnThreads = 384;
+constexpr int kAttnThreads = 512;
 constexpr int kRescaleThreshold = 8;  // log2 units
 // Registers per thread after the re-split: producer/MMA/gather, softmax, epilogue.
-constexpr int kRegsWG0 = 80, kRegsSoftmax = 240, kRegsEpilogue = 184;
-constexpr int kRegSplitTotal = 128 * (kRegsWG0 + kRegsSoftmax + kRegsEpilogue);
+constexpr int kRegsWG0 = 64, kRegsSoftmax = 160, kRegsEpilogue = 128;
+constexpr int kRegSplitTotal = 128 * (kRegsWG0 + 2 * kRegsSoftmax + kRegsEpilogue);
 static_assert(kRegSplitTotal <= 65536, "register split exceeds the register file");
+static_assert(kRegsEpilogue * kAttnThreads == 65536, "the epilogue keeps the launch budget");
 
 template <int D>
 struct AttnCfg {
@@ -53,7 +57,7 @@ struct AttnCfg {
   static constexpr int K_OFF = 2 * TILE;                   // ST key stages
   static constexpr int V_OFF = K_OFF + ST * TILE;          // ST value stages
   static constexpr int BAR_OFF = V_OFF + ST * TILE;
-  static constexpr int SMEM = BAR_OFF + 3072 + 1024;       // + barriers/stats + alignment slack
+  static constexpr int SMEM = BAR_OFF + 8192 + 1024;       // + barriers/stats + alignment slack
   static constexpr uint32_t BYTES = 128u * D * 2u;         // bytes one full tile load moves
 };
 
@@ -65,7 +69,8 @@ struct Bars {
   uint64_t o_full[2], o_free[2], stat_full[2];
   uint32_t tmem_base;
   int abort;
-  float2 stat[2][128];  // per O buffer and row: running max (log2 units), row sum
+  float2 stat[2][2][128];  // per O buffer, key half and row: running max (log2), row sum
+  float xmax[2][2][128];   // per S buffer, key half and row: the half-row maximum
 };
 
 // What one tile covers.  All roles derive it independently from the tile index.
@@ -167,12 +172,15 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int ks) {
   return smem_desc(tile + AttnCfg<D>::R0, 16, 256, kSwizzle32);
 }
 
-// V as the MN-major B operand of O += P V: keys [16 kk, 16 kk + 16), columns of region
-// `rg` (64 columns with 128-byte swizzle, or 16 columns with 32-byte swizzle).
+// V as the MN-major B operand of O += P V, keys [16 kk, 16 kk + 16).  rg = 0: the 64
+// columns of region 0 (128-byte swizzle; 8-key groups 1024 bytes apart).  rg = 1: the
+// 16 columns of the D = 80 tail region (32-byte swizzle, groups 256 bytes apart).
+// rg = 2 (D = 128): all 128 columns in one operand, the second 64-column atom a
+// leading-byte-offset of one region away.
 template <int D>
 __device__ __forceinline__ uint64_t v_desc(uint32_t tile, int kk, int rg) {
   if (rg == 0) return smem_desc(tile + kk * 2048, 16, 1024, kSwizzle128);
-  if (D == 128) return smem_desc(tile + AttnCfg<D>::R0 + kk * 2048, 16, 1024, kSwizzle128);
+  if (rg == 2) return smem_desc(tile + kk * 2048, AttnCfg<D>::R0, 1024, kSwizzle128);
   return smem_desc(tile + AttnCfg<D>::R0 + kk * 512, 16, 256, kSwizzle32);
 }
 
@@ -212,13 +220,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     mbar_init(&bar.s_full[0], 1);
     mbar_init(&bar.s_full[1], 1);
-    mbar_init(&bar.p_full, 128);
+    mbar_init(&bar.p_full, 256);
     mbar_init(&bar.o_done, 1);
     mbar_init(&bar.mma_done, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar.o_full[b], 1);
       mbar_init(&bar.o_free[b], 128);
-      mbar_init(&bar.stat_full[b], 128);
+      mbar_init(&bar.stat_full[b], 256);
     }
     bar.abort = 0;
     fence_barrier_init();
@@ -238,7 +246,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t tmem = bar.tmem_base;
   volatile int *abort = &bar.abort;
 
-  // Register split (launch: 384 threads x 168): see kRegSplitTotal.
+  // Register split (launch: 512 threads x 128): see kRegSplitTotal.
   if (warp < 4) {
     setmaxnreg_dec<kRegsWG0>();
     if (warp == 0) {
@@ -290,6 +298,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (lane == 0) {
         constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
         constexpr uint32_t idO64 = idesc_bf16(128, 64, 0, 1);
+        constexpr uint32_t idO128 = idesc_bf16(128, 128, 0, 1);
         constexpr uint32_t idO16 = idesc_bf16(128, 16, 0, 1);
         uint32_t kvc = 0, scnt = 0, pcnt = 0;
         uint32_t ofree_uses[2] = {0u, 0u};  // tiles started per O buffer
@@ -302,9 +311,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t acc = (first && kk == 0) ? 0u : 1u;
             const uint32_t a = sbuf + kk * 8;
-            umma_ts(tO, a, v_desc<D>(vt, kk, 0), idO64, acc);
-            if (D == 128) umma_ts(tO + 64, a, v_desc<D>(vt, kk, 1), idO64, acc);
-            if (D == 80) umma_ts(tO + 64, a, v_desc<D>(vt, kk, 1), idO16, acc);
+            if (D == 128) {
+              umma_ts(tO, a, v_desc<D>(vt, kk, 2), idO128, acc);
+            } else {
+              umma_ts(tO, a, v_desc<D>(vt, kk, 0), idO64, acc);
+              if (D == 80) umma_ts(tO + 64, a, v_desc<D>(vt, kk, 1), idO16, acc);
+            }
           }
         };
         // Chunks of consecutive tiles form one stream: S of chunk g is issued before
@@ -409,13 +421,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_arrive(&bar.q_full[qb]);
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ------------------------------------------------------------ softmax
     // tcgen05.ld / st are warp-collective (.sync.aligned): every wait is made
     // warp-uniform with __all_sync, and no TMEM access sits under a per-row branch.
     setmaxnreg_inc<kRegsSoftmax>();
-    const int r = tid - 128;             // row within the tile == TMEM lane
+    const int half = (warp - 4) >> 2;       // key half of each chunk
+    const int r = (tid - 128) & 127;        // row within the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    // O columns this half rescales: [oc0, oc1).
+    constexpr int OH = ((D / 2 + 15) / 16) * 16;
+    const int oc0 = half ? OH : 0, oc1 = half ? D : OH;
     const float sl2 = p.scale_log2;
     uint32_t scnt = 0, ocnt = 0;
     int lt = 0;
@@ -434,18 +450,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int m = 0; m < ti.nc; ++m, ++scnt) {
         const int sbi = scnt & 1;
         const uint32_t tS = tmem + lane_off + 128 * sbi;
+        // The two halves must take every decision together (they meet at named
+        // barriers), so each wait's outcome is AND-ed over both warpgroups.
         ok = mbar_wait(&bar.s_full[sbi], (scnt >> 1) & 1, abort, p.status, site0 + 12);
-        if (!(ok = __all_sync(FULL, ok))) break;
+        if (!(ok = named_barrier_and(1, 256, ok))) break;
         tc_fence_after();
-        uint32_t sv[128];
-        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+        uint32_t sv[64];
+        tmem_ld32(tS + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tS + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
         tmem_wait_ld();
         float *s = reinterpret_cast<float *>(sv);
         // Masks.
-        const int key0 = chunk_key<MODE>(p, ti, m);
+        const int key0 = chunk_key<MODE>(p, ti, m) + 64 * half;
         if (MODE == kQueryMajor) {
           if (p.is_moba) {
             if (m < ti.ntail) {
@@ -457,19 +473,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 for (int u2 = 0; u2 < p.topk; ++u2) covered |= (__ldg(irow + u2) == blk);
               }
 #pragma unroll
-              for (int e = 0; e < 128; ++e)
+              for (int e = 0; e < 64; ++e)
                 if (covered || !live || i - (key0 + e) >= p.window) s[e] = -INFINITY;
-            } else if (key0 + kTileKeys > ti.i0) {
+            } else if (key0 + 64 > ti.i0) {
 #pragma unroll
-              for (int e = 0; e < 128; ++e)
+              for (int e = 0; e < 64; ++e)
                 if (key0 + e > i) s[e] = -INFINITY;
             }
           } else {
-            const bool full = (key0 + kTileKeys - 1 <= ti.i0) &&
-                              (key0 >= ti.i0 + ti.rows - 1 - p.window + 1);
+            const bool full = (key0 + 63 <= ti.i0) && (key0 >= ti.i0 + ti.rows - 1 - p.window + 1);
             if (!full) {
 #pragma unroll
-              for (int e = 0; e < 128; ++e) {
+              for (int e = 0; e < 64; ++e) {
                 const int j = key0 + e;
                 if (j > i || i - j >= p.window) s[e] = -INFINITY;
               }
@@ -480,12 +495,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
         for (int u2 = 0; u2 < 8; ++u2) mx4[u2] = s[u2];
 #pragma unroll
-        for (int e = 8; e < 128; ++e) mx4[e & 7] = fmaxf(mx4[e & 7], s[e]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])),
-                               fmaxf(fmaxf(mx4[4], mx4[5]), fmaxf(mx4[6], mx4[7])));
+        for (int e = 8; e < 64; ++e) mx4[e & 7] = fmaxf(mx4[e & 7], s[e]);
+        // The row maximum over both halves of the chunk.
+        bar.xmax[sbi][half][r] = fmaxf(fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])),
+                                       fmaxf(fmaxf(mx4[4], mx4[5]), fmaxf(mx4[6], mx4[7])));
+        named_barrier_sync(1, 256);
+        const float mx = fmaxf(bar.xmax[sbi][0][r], bar.xmax[sbi][1][r]);
         const float m_new = fmaxf(m_run, mx * sl2);
         // Raise the running maximum only when it grows by more than 2^8 (or from
-        // -inf); rows that keep theirs multiply O by 1 when the warp rescales.
+        // -inf); rows that keep theirs multiply O by 1 when the warp rescales.  Both
+        // halves of a row take the same decision from the same numbers.
         const bool raise = (m == 0) || (m_new > m_run + (float)kRescaleThreshold);
         const bool scale_o = raise && m > 0 && m_run != -INFINITY;
         const float alpha = scale_o ? ex2_approx(m_run - m_new) : 1.f;
@@ -498,35 +517,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
         for (int u2 = 0; u2 < 8; ++u2) ls[u2] = 0.f;
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            // One element in four takes the FMA-pipe 2^x, the rest the MUFU unit.
-            const float p0 = ex2_approx(fmaf(s[q4 * 16 + 2 * e], sl2, -mu));
-            const float x1 = fmaf(s[q4 * 16 + 2 * e + 1], sl2, -mu);
-            const float p1 = (e & 1) ? exp2_fma(x1) : ex2_approx(x1);
-            ls[e] += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
-          }
-          sv[q4 * 8 + 0] = pk[0]; sv[q4 * 8 + 1] = pk[1]; sv[q4 * 8 + 2] = pk[2]; sv[q4 * 8 + 3] = pk[3];
-          sv[q4 * 8 + 4] = pk[4]; sv[q4 * 8 + 5] = pk[5]; sv[q4 * 8 + 6] = pk[6]; sv[q4 * 8 + 7] = pk[7];
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = ex2_approx(fmaf(s[2 * e], sl2, -mu));
+          const float p1 = ex2_approx(fmaf(s[2 * e + 1], sl2, -mu));
+          ls[e & 7] += p0 + p1;
+          sv[e] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(tS, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-        tmem_st16(tS + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
-        tmem_st16(tS + 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[32]));
-        tmem_st16(tS + 48, *reinterpret_cast<uint32_t(*)[16]>(&sv[48]));
+        // P of keys [64 half, 64 half + 64) -> TMEM columns [32 half, 32 half + 32).
+        tmem_st16(tS + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+        tmem_st16(tS + 32 * half + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
         l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         if (m > 0) {
-          // O holds chunks 0..m-1 once their last P V is done; rescale it if any row
-          // of this warp raised its maximum.
+          // O holds chunks 0..m-1 once their last P V is done; rescale this half's
+          // columns if any row of the warp raised its maximum.
           ok = mbar_wait(&bar.o_done, ocnt & 1, abort, p.status, site0 + 13);
-          if (!(ok = __all_sync(FULL, ok))) break;
+          if (!(ok = named_barrier_and(1, 256, ok))) break;
           ++ocnt;
           tc_fence_after();
           if (__any_sync(FULL, scale_o)) {
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 16) {
+              if (c0 < oc0 || c0 >= oc1) continue;
               uint32_t o[16];
               tmem_ld16(tO + c0, o);
               tmem_wait_ld();
@@ -544,14 +555,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // Hand the row statistics to the epilogue once it has drained this O buffer's
       // previous tile.
       ok = mbar_wait(&bar.o_free[ob], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 14);
-      if (!(ok = __all_sync(FULL, ok))) break;
-      bar.stat[ob][r] = make_float2(m_run, l_run);
+      if (!(ok = named_barrier_and(1, 256, ok))) break;
+      bar.stat[ob][half][r] = make_float2(m_run, l_run);
       mbar_arrive(&bar.stat_full[ob]);
     }
   } else {
     // ----------------------------------------------------------- epilogue
-    setmaxnreg_inc<kRegsEpilogue>();
-    const int r = tid - 256;
+    // Keeps the registers it was launched with (kRegsEpilogue).
+    const int r = tid - 384;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     int lt = 0;
     bool ok = true;
@@ -573,8 +584,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       ok = ok && mbar_wait(&bar.o_full[ob], (lt >> 1) & 1, abort, p.status, site0 + 16);
       if (!(ok = __all_sync(FULL, ok))) break;
       tc_fence_after();
-      const float2 st = bar.stat[ob][r];
-      const float m_run = st.x, l_run = st.y;
+      const float2 st0 = bar.stat[ob][0][r], st1 = bar.stat[ob][1][r];
+      const float m_run = st0.x, l_run = st0.y + st1.y;
       const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
       const float own_lse = (m_run + log2f(l_run)) * 0.69314718055994530942f;  // natural log
       // Destination: a partial slot (gathered tiles: the row's past-block slot; MoBA
