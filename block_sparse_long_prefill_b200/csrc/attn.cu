@@ -41,6 +41,12 @@ namespace moba {
 
 constexpr int kAttnThreads = 512;
 constexpr int kRescaleThreshold = 8;  // log2 units
+// Of every 16 probabilities, this many take the FMA-pipe 2^x (exp2_fma) instead of
+// the MUFU unit, whose 16 results per clock and SM bound the softmax otherwise.
+#ifndef MOBA_EXP_EMU_PER16
+#define MOBA_EXP_EMU_PER16 4
+#endif
+constexpr int kExpEmuPer16 = MOBA_EXP_EMU_PER16;
 // Registers per thread after the re-split: producer/MMA/gather, softmax, epilogue.
 constexpr int kRegsWG0 = 64, kRegsSoftmax = 160, kRegsEpilogue = 128;
 constexpr int kRegSplitTotal = 128 * (kRegsWG0 + 2 * kRegsSoftmax + kRegsEpilogue);
@@ -65,7 +71,7 @@ struct Bars {
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[3], v_full[3], k_empty[3], v_empty[3];
   uint64_t s_full[2];
-  uint64_t p_full, o_done, mma_done;
+  uint64_t p_full, o_done[2], mma_done;
   uint64_t o_full[2], o_free[2], stat_full[2];
   uint32_t tmem_base;
   int abort;
@@ -221,7 +227,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     mbar_init(&bar.s_full[0], 1);
     mbar_init(&bar.s_full[1], 1);
     mbar_init(&bar.p_full, 256);
-    mbar_init(&bar.o_done, 1);
+    mbar_init(&bar.o_done[0], 1);
+    mbar_init(&bar.o_done[1], 1);
     mbar_init(&bar.mma_done, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar.o_full[b], 1);
@@ -334,8 +341,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
           tc_fence_after();
           issue_pv(pend.tO, pend.first, pend.sbuf, pend.st);
+          // Every P V completes a phase of o_done[its index & 1] (the softmax tracks
+          // them in order); a tile's last one also hands the O buffer to the epilogue.
+          umma_commit(&bar.o_done[pv_slot & 1]);
           if (pend.last) umma_commit(&bar.o_full[pend.ob]);
-          else umma_commit(&bar.o_done);
           umma_commit(&bar.v_empty[pend.st]);
           pend.valid = false;
           return true;
@@ -433,7 +442,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     constexpr int OH = ((D / 2 + 15) / 16) * 16;
     const int oc0 = half ? OH : 0, oc1 = half ? D : OH;
     const float sl2 = p.scale_log2;
-    uint32_t scnt = 0, ocnt = 0;
+    uint32_t scnt = 0;
+    // P V number k (counted over all chunks of this CTA, like scnt) completes phase
+    // k >> 1 of o_done[k & 1].  pv_seen: P Vs whose completion was already awaited.
+    uint32_t pv_seen = 0;
     int lt = 0;
     bool ok = true;
     for (TileIter<MODE> it(p, t_begin, t_end); ok && it.valid(); it.next(), ++lt) {
@@ -518,8 +530,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int u2 = 0; u2 < 8; ++u2) ls[u2] = 0.f;
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float p0 = ex2_approx(fmaf(s[2 * e], sl2, -mu));
-          const float p1 = ex2_approx(fmaf(s[2 * e + 1], sl2, -mu));
+          const float x0 = fmaf(s[2 * e], sl2, -mu), x1 = fmaf(s[2 * e + 1], sl2, -mu);
+          const float p0 = ((2 * e) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x0) : ex2_approx(x0);
+          const float p1 = ((2 * e + 1) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x1) : ex2_approx(x1);
           ls[e & 7] += p0 + p1;
           sv[e] = pack_bf16x2(p0, p1);
         }
@@ -527,12 +540,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_st16(tS + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
         tmem_st16(tS + 32 * half + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
         l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-        if (m > 0) {
-          // O holds chunks 0..m-1 once their last P V is done; rescale this half's
-          // columns if any row of the warp raised its maximum.
-          ok = mbar_wait(&bar.o_done, ocnt & 1, abort, p.status, site0 + 13);
+        // Before P V number scnt may be issued, the P V two back must be complete
+        // (o_done[scnt & 1] is reused by it); if this chunk rescales O, the previous
+        // one too.  The pair of warpgroups decides together.
+        const bool rescale = (m > 0) && named_barrier_and(2, 256, !__any_sync(FULL, scale_o)) == false;
+        const uint32_t need = rescale ? scnt : (scnt >= 1 ? scnt - 1 : 0);
+        while (pv_seen < need) {
+          ok = mbar_wait(&bar.o_done[pv_seen & 1], (pv_seen >> 1) & 1, abort, p.status, site0 + 13);
           if (!(ok = named_barrier_and(1, 256, ok))) break;
-          ++ocnt;
+          ++pv_seen;
+        }
+        if (!ok) break;
+        if (rescale) {
+          // O holds chunks 0..m-1 now; rescale this half's columns where a row of the
+          // warp raised its maximum.
           tc_fence_after();
           if (__any_sync(FULL, scale_o)) {
 #pragma unroll
@@ -553,7 +574,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       if (!ok) break;
       // Hand the row statistics to the epilogue once it has drained this O buffer's
-      // previous tile.
+      // previous tile (that also orders every earlier P V before this point).
       ok = mbar_wait(&bar.o_free[ob], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 14);
       if (!(ok = named_barrier_and(1, 256, ok))) break;
       bar.stat[ob][half][r] = make_float2(m_run, l_run);
@@ -603,23 +624,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         ldst = p.lse + ((int64_t)ti.b * p.hq + h) * p.N + i;
       }
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 16) {
-        uint32_t o[16];
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        const int cols = (D - c0) < 32 ? (D - c0) : 32;  // D = 80 ends with 16
+        uint32_t o[32];
         __syncwarp();
-        tmem_ld16(tO + c0, o);
+        if (cols == 32) tmem_ld32(tO + c0, o);
+        else tmem_ld16(tO + c0, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
         tmem_wait_ld();
         if (live) {
-          uint4 w0, w1;
-          w0.x = pack_bf16x2(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l);
-          w0.y = pack_bf16x2(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l);
-          w0.z = pack_bf16x2(__uint_as_float(o[4]) * inv_l, __uint_as_float(o[5]) * inv_l);
-          w0.w = pack_bf16x2(__uint_as_float(o[6]) * inv_l, __uint_as_float(o[7]) * inv_l);
-          w1.x = pack_bf16x2(__uint_as_float(o[8]) * inv_l, __uint_as_float(o[9]) * inv_l);
-          w1.y = pack_bf16x2(__uint_as_float(o[10]) * inv_l, __uint_as_float(o[11]) * inv_l);
-          w1.z = pack_bf16x2(__uint_as_float(o[12]) * inv_l, __uint_as_float(o[13]) * inv_l);
-          w1.w = pack_bf16x2(__uint_as_float(o[14]) * inv_l, __uint_as_float(o[15]) * inv_l);
-          *reinterpret_cast<uint4 *>(dst + c0) = w0;
-          *reinterpret_cast<uint4 *>(dst + c0 + 8) = w1;
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            if (v4 * 8 >= cols) break;
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv_l, __uint_as_float(o[8 * v4 + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * v4 + 2]) * inv_l, __uint_as_float(o[8 * v4 + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * v4 + 4]) * inv_l, __uint_as_float(o[8 * v4 + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * v4 + 6]) * inv_l, __uint_as_float(o[8 * v4 + 7]) * inv_l);
+            *reinterpret_cast<uint4 *>(dst + c0 + 8 * v4) = w;
+          }
         }
       }
       if (live) *ldst = own_lse;
