@@ -44,7 +44,7 @@ constexpr int kRescaleThreshold = 8;  // log2 units
 // Of every 16 probabilities, this many take the FMA-pipe 2^x (exp2_fma) instead of
 // the MUFU unit, whose 16 results per clock and SM bound the softmax otherwise.
 #ifndef MOBA_EXP_EMU_PER16
-#define MOBA_EXP_EMU_PER16 4
+#define MOBA_EXP_EMU_PER16 0
 #endif
 constexpr int kExpEmuPer16 = MOBA_EXP_EMU_PER16;
 // Registers per thread after the re-split: producer/MMA/gather, softmax, epilogue.
