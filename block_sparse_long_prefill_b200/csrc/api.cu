@@ -25,6 +25,8 @@ cudaError_t launch_scatter(const ScatterParams &p, cudaStream_t st);
 cudaError_t launch_attn(const CUtensorMap *maps, const AttnParams &p, int mode, int grid,
                         cudaStream_t st);
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t st);
+int query_major_units(int batch, int hq, int hkv, int block, int is_moba, int row_begin,
+                      int row_end);
 
 namespace {
 
@@ -249,8 +251,7 @@ int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *id
       p.ntiles = 0;  // read from the workspace by the kernel
       if ((rc = launch_status(launch_attn(maps, p, kGathered, nsm, st)))) return rc;
     }
-    const int nq = (p.row_end - p.row_begin + kTileRows - 1) / kTileRows;
-    p.ntiles = nq * hq * batch;
+    p.ntiles = query_major_units(batch, hq, hkv, block, 1, p.row_begin, p.row_end);
     const int grid = p.ntiles < nsm ? p.ntiles : nsm;
     if ((rc = launch_status(launch_attn(maps, p, kQueryMajor, grid, st)))) return rc;
     if (w.npast > 0) {
@@ -302,8 +303,7 @@ int swa_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq,
   p.is_moba = 0;
   p.row_begin = 0;
   p.row_end = N;
-  const int nq = (N + kTileRows - 1) / kTileRows;
-  p.ntiles = nq * hq * batch;
+  p.ntiles = query_major_units(batch, hq, hkv, 0, 0, 0, N);
   p.npast = 0;
   const int grid = p.ntiles < nsm ? p.ntiles : nsm;
   return launch_status(launch_attn(maps, p, kQueryMajor, grid, static_cast<cudaStream_t>(stream)));

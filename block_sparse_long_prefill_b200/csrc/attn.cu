@@ -4,31 +4,34 @@
 //          (feat. MoonshotAI)", PyTorch KR forum summary of the MoBA paper.
 // [SWA]  = "SWA + MoE: 어텐션과 희소 전문가", Bit-Axon architecture page.
 //
-// One persistent kernel, two tile kinds:
-//   kQueryMajor  128 contiguous query rows of one (batch, q-head).  MoBA: the causal own
-//                block (§"MoBA의 구현": current block with causal=True), the window
-//                tail into earlier unselected blocks, and the merge of the past-block
-//                partials by log-sum-exp (step 5).  SWA: the causal band of [SWA]
-//                §"슬라이딩 윈도우 마스크".
-//   kGathered    up to 128 (row, q-head) pairs of one block-major list against the
-//                whole past block they picked (steps 3-4, causal=False); writes a
-//                normalised partial output and its log-sum-exp per (row, slot).
+// One persistent kernel, two work kinds:
+//   kQueryMajor  contiguous 128-row query tiles of one (batch, q-head).  MoBA: the causal
+//                own block (§"MoBA의 구현": current block with causal=True) plus the
+//                window tail into earlier blocks the row did not select; the result is
+//                the own-block partial that the merge pass combines with the past-block
+//                partials (step 5).  SWA: the causal band of [SWA] §"슬라이딩 윈도우
+//                마스크", written straight to the output.
+//   kGathered    gathered (row, q-head) pairs of one block-major list against the whole
+//                past block they picked (steps 3-4, causal=False); writes a normalised
+//                partial output and its log-sum-exp per (row, slot).
 //
-// Per CTA (512 threads, one CTA per SM, 512 TMEM columns):
-//   warp 0       TMA producers: lane 0 the query tile (query-major) and K chunks of 128
+// Each CTA runs two tile streams, A and B, over a shared K/V chunk sequence: a work
+// unit is a pair of 128-row tiles that attend to the same keys (two q-heads of one KV
+// head, two row tiles of one head, or 256 entries of one block list).  While one
+// stream's softmax runs, the tensor core works on the other stream's S = Q K^T and
+// O += P V, so the exponentials and the MMAs overlap (the FA4 ping-pong).
+//   warp 0       TMA producers: lane 0 the query tiles (query-major) and K chunks of 128
 //                keys, lane 1 the V chunks (separate K and V rings)
 //   warp 1       tcgen05 MMA issuer (one thread) and TMEM owner
-//   warps 2-3    query-row gather with cp.async (gathered tiles)
-//   warps 4-11   softmax, two warpgroups: thread r of group h owns row r (TMEM lane r)
-//                and keys [64 h, 64 h + 64) of each chunk; the two halves of a row
-//                exchange their maxima through shared memory; S -> P in place; O is
-//                rescaled only when the running maximum grows by more than 2^8
-//   warps 12-15  epilogue: normalises O and stores it (a partial or the output),
-//                then frees the O buffer
-// TMEM: S/P double buffer at columns [0,128) and [128,256); O double buffer at
-// [256,384) and [384,512), so a tile's epilogue overlaps the next tile's MMAs.
-// S = Q K^T is an SS MMA; P (bf16) overwrites its own S columns and is the A operand
-// (from TMEM) of O += P V.
+//   warps 2-3    query-row gather with cp.async (gathered work)
+//   warps 4-7    stream A softmax + epilogue; thread r owns row r (TMEM lane r)
+//   warps 8-11   stream B softmax + epilogue
+// TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).  P (bf16) overwrites
+// its own S columns and is the A operand (from TMEM) of O += P V.  A stream's S of
+// chunk m is issued after its P V of chunk m-1, so when the softmax sees S(m) complete
+// (commit semantics: every earlier MMA is complete) it may rescale O at once.  The
+// running maximum is raised lazily: O and l are rescaled only when it grows by more
+// than 2^8.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -39,134 +42,166 @@
 
 namespace moba {
 
-constexpr int kAttnThreads = 512;
+constexpr int kAttnThreads = 384;
 constexpr int kRescaleThreshold = 8;  // log2 units
 // Of every 16 probabilities, this many take the FMA-pipe 2^x (exp2_fma) instead of
-// the MUFU unit, whose 16 results per clock and SM bound the softmax otherwise.
+// the MUFU unit.
 #ifndef MOBA_EXP_EMU_PER16
 #define MOBA_EXP_EMU_PER16 0
 #endif
 constexpr int kExpEmuPer16 = MOBA_EXP_EMU_PER16;
-// Registers per thread after the re-split: producer/MMA/gather, softmax, epilogue.
-constexpr int kRegsWG0 = 64, kRegsSoftmax = 160, kRegsEpilogue = 128;
-constexpr int kRegSplitTotal = 128 * (kRegsWG0 + 2 * kRegsSoftmax + kRegsEpilogue);
+// Registers per thread after the re-split: producer/MMA/gather, each softmax stream.
+constexpr int kRegsWG0 = 72, kRegsSoftmax = 216;
+constexpr int kRegSplitTotal = 128 * (kRegsWG0 + 2 * kRegsSoftmax);
 static_assert(kRegSplitTotal <= 65536, "register split exceeds the register file");
-static_assert(kRegsEpilogue * kAttnThreads == 65536, "the epilogue keeps the launch budget");
 
 template <int D>
 struct AttnCfg {
-  static constexpr int ST = (D == 128) ? 2 : 3;            // K/V pipeline stages
+  static constexpr int ST = (D == 128) ? 2 : 3;            // K and V ring stages each
   static constexpr int R0 = 128 * 128;                     // bytes of the 64-column region
   static constexpr int R1 = (D == 128) ? 128 * 128 : (D == 80 ? 128 * 32 : 0);
   static constexpr int TILE = R0 + ((R1 + 1023) / 1024) * 1024;  // one 128 x D operand tile
-  static constexpr int Q_OFF = 0;                          // 2 query buffers
-  static constexpr int K_OFF = 2 * TILE;                   // ST key stages
-  static constexpr int V_OFF = K_OFF + ST * TILE;          // ST value stages
+  static constexpr int Q_OFF = 0;                          // Q_A, Q_B
+  static constexpr int K_OFF = 2 * TILE;                   // K ring
+  static constexpr int V_OFF = K_OFF + ST * TILE;          // V ring
   static constexpr int BAR_OFF = V_OFF + ST * TILE;
-  static constexpr int SMEM = BAR_OFF + 8192 + 1024;       // + barriers/stats + alignment slack
+  static constexpr int SMEM = BAR_OFF + 1024 + 1024;       // + barriers + alignment slack
   static constexpr uint32_t BYTES = 128u * D * 2u;         // bytes one full tile load moves
 };
 
 struct Bars {
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[2], q_empty[2];                          // per stream
   uint64_t k_full[3], v_full[3], k_empty[3], v_empty[3];
-  uint64_t s_full[2];
-  uint64_t p_full, o_done[2], mma_done;
-  uint64_t o_full[2], o_free[2], stat_full[2];
+  uint64_t s_full[2], p_full[2], o_full[2];                // per stream
+  uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
-  float2 stat[2][2][128];  // per O buffer, key half and row: running max (log2), row sum
-  float xmax[2][2][128];   // per S buffer, key half and row: the half-row maximum
 };
 
-// What one tile covers.  All roles derive it independently from the tile index.
-struct TileInfo {
+// One stream's tile of a work unit.
+struct Tile {
   int b, h, hk;
-  int i0;          // query-major: first row
-  int rows;        // valid rows
-  int nc;          // key chunks
-  int key0;        // query-major MoBA: first key of the tail (window) range
-  int ntail;       // query-major MoBA: chunks before the own block
-  int cB;          // query-major MoBA: first key of the own block
-  // gathered
-  int list;        // list id
-  int ent0;        // first entry of this tile in the entry array
-  int j;           // past block
+  int i0;      // query-major: first row
+  int rows;    // valid rows (0: the stream is idle in this unit)
+  int ent0;    // gathered: first list entry
+  int cB;      // query-major MoBA: first key of the own block
 };
 
-__device__ __forceinline__ void query_major_tile(const AttnParams &p, int t, TileInfo &ti) {
-  const int HB = p.hq * p.batch;
+// A work unit: two tiles over one key-chunk sequence.
+struct Unit {
+  Tile t[2];
+  int b, hk;
+  int key0;    // first key of chunk 0
+  int nc;      // chunks
+  int j;       // gathered: the past block
+};
+
+// Query-major units.  With GQA (G >= 2) a unit is two q-heads of one KV head at the
+// same rows; otherwise two consecutive row tiles of one head (MoBA: of one block),
+// attending to the union of their key ranges with per-row masks.
+__device__ __forceinline__ void query_major_unit(const AttnParams &p, int u, Unit &w) {
   const int nq = (p.row_end - p.row_begin + kTileRows - 1) / kTileRows;
-  const int qt = nq - 1 - t / HB;  // later (heavier) tiles first
-  const int hb = t % HB;
-  ti.h = hb % p.hq;
-  ti.b = hb / p.hq;
-  ti.hk = ti.h / p.G;
-  ti.i0 = p.row_begin + qt * kTileRows;
-  ti.rows = min(kTileRows, p.row_end - ti.i0);
-  const int ilast = ti.i0 + ti.rows - 1;
-  if (p.is_moba) {
-    ti.cB = (ti.i0 / p.block) * p.block;
-    int tl = ti.cB;
-    if (p.window > 0) {
-      const int lo = max(0, ti.i0 - p.window + 1);
-      tl = min(ti.cB, (lo / kTileKeys) * kTileKeys);
-    }
-    ti.key0 = tl;
-    ti.ntail = (ti.cB - tl) / kTileKeys;
-    ti.nc = ti.ntail + (ti.i0 - ti.cB) / kTileKeys + 1;
+  int qt0, qt1, g0, g1, hb;
+  if (p.G >= 2) {
+    const int per_hk = (p.G + 1) / 2;                      // head pairs per KV head
+    const int HB = p.batch * p.hkv * per_hk;
+    const int slot = nq - 1 - u / HB;                      // later (heavier) rows first
+    hb = u % HB;
+    qt0 = qt1 = slot;
+    const int ph = hb % per_hk;
+    g0 = 2 * ph;
+    g1 = (2 * ph + 1 < p.G) ? 2 * ph + 1 : -1;
+    hb /= per_hk;                                          // (b, hk)
   } else {
-    const int lo = max(0, ti.i0 - p.window + 1);
-    ti.key0 = (lo / kTileKeys) * kTileKeys;
-    ti.ntail = 0;
-    ti.cB = 0;
-    ti.nc = (ilast - ti.key0) / kTileKeys + 1;
+    // Row-tile pairs; for MoBA a pair never crosses a block boundary.
+    const int tpb = p.is_moba ? p.block / kTileRows : nq;   // tiles per pairing group
+    const int ppg = (tpb + 1) / 2;                         // pairs per group
+    const int ngroups = (nq + tpb - 1) / tpb;
+    const int HB = p.batch * p.hkv;
+    const int pr = ngroups * ppg - 1 - u / HB;             // later rows first
+    hb = u % HB;
+    const int grp = pr / ppg, k = pr % ppg;
+    qt0 = grp * tpb + 2 * k;
+    const int lim = min(nq, (grp + 1) * tpb);
+    qt1 = (qt0 + 1 < lim) ? qt0 + 1 : -1;
+    g0 = 0;
+    g1 = (qt1 >= 0) ? 0 : -1;
+    if (qt1 < 0) qt1 = qt0;
   }
+  w.b = hb / p.hkv;
+  w.hk = hb % p.hkv;
+  w.j = 0;
+  int lo = 0x7fffffff, hi = -1;
+  for (int x = 0; x < 2; ++x) {
+    Tile &t = w.t[x];
+    const int g = x ? g1 : g0;
+    const int qt = x ? qt1 : qt0;
+    t.b = w.b;
+    t.hk = w.hk;
+    t.h = w.hk * p.G + (g < 0 ? 0 : g);
+    t.i0 = p.row_begin + qt * kTileRows;
+    t.rows = (g < 0) ? 0 : min(kTileRows, p.row_end - t.i0);
+    t.ent0 = 0;
+    t.cB = 0;
+    if (t.rows == 0) continue;
+    const int ilast = t.i0 + t.rows - 1;
+    int first;
+    if (p.is_moba) {
+      t.cB = (t.i0 / p.block) * p.block;
+      first = t.cB;
+      if (p.window > 0) first = min(t.cB, (max(0, t.i0 - p.window + 1) / kTileKeys) * kTileKeys);
+    } else {
+      first = (max(0, t.i0 - p.window + 1) / kTileKeys) * kTileKeys;
+    }
+    lo = min(lo, first);
+    hi = max(hi, ilast);
+  }
+  w.key0 = lo;
+  w.nc = (hi - lo) / kTileKeys + 1;
 }
 
-__device__ __forceinline__ void gathered_tile(const AttnParams &p, int4 rec, TileInfo &ti) {
+__device__ __forceinline__ void gathered_unit(const AttnParams &p, int4 rec, Unit &w) {
   const int L = rec.x;
-  ti.list = L;
-  ti.ent0 = rec.y;
-  ti.rows = rec.z;
-  ti.j = L % p.nblk;
-  ti.hk = (L / p.nblk) % p.hkv;
-  ti.b = (L / (p.nblk * p.hkv)) % p.batch;
-  ti.h = -1;
-  ti.i0 = 0;
-  ti.nc = p.block / kTileKeys;
+  w.j = L % p.nblk;
+  w.hk = (L / p.nblk) % p.hkv;
+  w.b = (L / (p.nblk * p.hkv)) % p.batch;
+  w.key0 = w.j * p.block;
+  w.nc = p.block / kTileKeys;
+  for (int x = 0; x < 2; ++x) {
+    Tile &t = w.t[x];
+    t.b = w.b;
+    t.hk = w.hk;
+    t.h = -1;
+    t.i0 = 0;
+    t.cB = 0;
+    t.ent0 = rec.y + x * kTileRows;
+    t.rows = max(0, min(kTileRows, rec.z - x * kTileRows));
+  }
 }
 
-// Walks this CTA's tiles t = t_begin + blockIdx.x, t += gridDim.x.  Gathered tiles
-// come from the tile table; the next record is loaded one tile ahead.
+// Walks this CTA's units u = u_begin + blockIdx.x, u += gridDim.x.  Gathered units
+// come from the unit table; the next record is loaded one unit ahead.
 template <int MODE>
-struct TileIter {
-  int t, t_end;
+struct UnitIter {
+  int u, u_end;
   int4 nxt;
-  __device__ __forceinline__ TileIter(const AttnParams &p, int t_begin, int t_end_) {
-    t = t_begin + (int)blockIdx.x;
-    t_end = t_end_;
-    if (MODE == kGathered && t < t_end) nxt = __ldg(p.tiles + t);
+  __device__ __forceinline__ UnitIter(const AttnParams &p, int u_begin, int u_end_) {
+    u = u_begin + (int)blockIdx.x;
+    u_end = u_end_;
+    if (MODE == kGathered && u < u_end) nxt = __ldg(p.tiles + u);
   }
-  __device__ __forceinline__ bool valid() const { return t < t_end; }
-  __device__ __forceinline__ void get(const AttnParams &p, TileInfo &ti) {
+  __device__ __forceinline__ bool valid() const { return u < u_end; }
+  __device__ __forceinline__ void get(const AttnParams &p, Unit &w) {
     if (MODE == kGathered) {
       const int4 cur = nxt;
-      if (t + (int)gridDim.x < t_end) nxt = __ldg(p.tiles + t + gridDim.x);
-      gathered_tile(p, cur, ti);
+      if (u + (int)gridDim.x < u_end) nxt = __ldg(p.tiles + u + gridDim.x);
+      gathered_unit(p, cur, w);
     } else {
-      query_major_tile(p, t, ti);
+      query_major_unit(p, u, w);
     }
   }
-  __device__ __forceinline__ void next() { t += gridDim.x; }
+  __device__ __forceinline__ void next() { u += gridDim.x; }
 };
-
-// Key of chunk m of a tile.
-template <int MODE>
-__device__ __forceinline__ int chunk_key(const AttnParams &p, const TileInfo &ti, int m) {
-  if (MODE == kGathered) return ti.j * p.block + m * kTileKeys;
-  return ti.key0 + m * kTileKeys;
-}
 
 // Operand descriptors.  Region 0 holds columns [0, 64) of a 128-row tile (128-byte
 // rows, 128-byte swizzle); region 1 holds columns [64, 128) the same way (D = 128) or
@@ -206,35 +241,28 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int site0 = (MODE * 16 + (D == 64 ? 0 : (D == 80 ? 1 : 2))) * 256;
   constexpr uint32_t FULL = 0xffffffffu;
 
-  // Tile range.
-  int t_begin = 0, t_end = p.ntiles;
+  // Unit range.
+  int u_begin = 0, u_end = p.ntiles;
   if (MODE == kGathered) {
-    t_begin = __ldg(p.tileoff + p.chunk * p.lists_per_chunk);
-    t_end = __ldg(p.tileoff + (p.chunk + 1) * p.lists_per_chunk);
+    u_begin = __ldg(p.tileoff + p.chunk * p.lists_per_chunk);
+    u_end = __ldg(p.tileoff + (p.chunk + 1) * p.lists_per_chunk);
   }
 
   if (tid == 0) {
-    mbar_init(&bar.q_full[0], MODE == kGathered ? 64 : 1);
-    mbar_init(&bar.q_full[1], MODE == kGathered ? 64 : 1);
-    mbar_init(&bar.q_empty[0], 1);
-    mbar_init(&bar.q_empty[1], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bar.q_full[x], MODE == kGathered ? 64 : 1);
+      mbar_init(&bar.q_empty[x], 1);
+      mbar_init(&bar.s_full[x], 1);
+      mbar_init(&bar.p_full[x], 128);
+      mbar_init(&bar.o_full[x], 1);
+    }
     for (int s = 0; s < 3; ++s) {
       mbar_init(&bar.k_full[s], 1);
       mbar_init(&bar.v_full[s], 1);
       mbar_init(&bar.k_empty[s], 1);
       mbar_init(&bar.v_empty[s], 1);
     }
-    mbar_init(&bar.s_full[0], 1);
-    mbar_init(&bar.s_full[1], 1);
-    mbar_init(&bar.p_full, 256);
-    mbar_init(&bar.o_done[0], 1);
-    mbar_init(&bar.o_done[1], 1);
     mbar_init(&bar.mma_done, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bar.o_full[b], 1);
-      mbar_init(&bar.o_free[b], 128);
-      mbar_init(&bar.stat_full[b], 256);
-    }
     bar.abort = 0;
     fence_barrier_init();
   }
@@ -253,14 +281,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t tmem = bar.tmem_base;
   volatile int *abort = &bar.abort;
 
-  // Register split (launch: 512 threads x 128): see kRegSplitTotal.
+  // Register split (launch: 384 threads x 168): see kRegSplitTotal.
   if (warp < 4) {
     setmaxnreg_dec<kRegsWG0>();
     if (warp == 0) {
       // ---------------------------------------------------------- producers
-      // Lane 0 loads query tiles (query-major) and K chunks; lane 1 loads V chunks.
-      // K and V have separate rings: a K slot frees once its S = Q K^T is done, long
-      // before the V slot of the same chunk (freed by P V).
+      // Lane 0 loads the query tiles (query-major) and K chunks; lane 1 the V chunks.
       if (lane < 2) {
         const bool kside = lane == 0;
         uint64_t *full = kside ? bar.k_full : bar.v_full;
@@ -269,27 +295,33 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const CUtensorMap *m1 = kside ? &tmK1 : &tmV1;
         const int off = kside ? C::K_OFF : C::V_OFF;
         uint32_t cnt = 0;
-        int lt = 0;
+        uint32_t quse[2] = {0u, 0u};
         bool ok = true;
-        for (TileIter<MODE> it(p, t_begin, t_end); ok && it.valid(); it.next(), ++lt) {
-          TileInfo ti;
-          it.get(p, ti);
+        for (UnitIter<MODE> it(p, u_begin, u_end); ok && it.valid(); it.next()) {
+          Unit w;
+          it.get(p, w);
           if (MODE == kQueryMajor && kside) {
-            const int qb = lt & 1;
-            if (!(ok = mbar_wait(&bar.q_empty[qb], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 1))) break;
-            unsigned char *qd = sbase + C::Q_OFF + qb * C::TILE;
-            mbar_arrive_expect_tx(&bar.q_full[qb], C::BYTES);
-            tma_load_4d(qd, &tmQ, &bar.q_full[qb], 0, ti.i0, ti.h, ti.b);
-            if (D != 64) tma_load_4d(qd + C::R0, &tmQ1, &bar.q_full[qb], 64, ti.i0, ti.h, ti.b);
+            for (int x = 0; x < 2 && ok; ++x) {
+              const Tile &t = w.t[x];
+              if (t.rows == 0) continue;
+              ok = mbar_wait(&bar.q_empty[x], (quse[x] & 1) ^ 1, abort, p.status, site0 + 1);
+              if (!ok) break;
+              ++quse[x];
+              unsigned char *qd = sbase + C::Q_OFF + x * C::TILE;
+              mbar_arrive_expect_tx(&bar.q_full[x], C::BYTES);
+              tma_load_4d(qd, &tmQ, &bar.q_full[x], 0, t.i0, t.h, t.b);
+              if (D != 64) tma_load_4d(qd + C::R0, &tmQ1, &bar.q_full[x], 64, t.i0, t.h, t.b);
+            }
+            if (!ok) break;
           }
-          for (int m = 0; m < ti.nc; ++m, ++cnt) {
+          for (int m = 0; m < w.nc; ++m, ++cnt) {
             const int st = cnt % C::ST;
             if (!(ok = mbar_wait(&empty[st], ((cnt / C::ST) & 1) ^ 1, abort, p.status, site0 + 2))) break;
-            const int key = chunk_key<MODE>(p, ti, m);
+            const int key = w.key0 + m * kTileKeys;
             unsigned char *dst = sbase + off + st * C::TILE;
             mbar_arrive_expect_tx(&full[st], C::BYTES);
-            tma_load_4d(dst, m0, &full[st], 0, key, ti.hk, ti.b);
-            if (D != 64) tma_load_4d(dst + C::R0, m1, &full[st], 64, key, ti.hk, ti.b);
+            tma_load_4d(dst, m0, &full[st], 0, key, w.hk, w.b);
+            if (D != 64) tma_load_4d(dst + C::R0, m1, &full[st], 64, key, w.hk, w.b);
           }
         }
         // Let every load issued so far land before the CTA can retire.
@@ -307,76 +339,69 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         constexpr uint32_t idO64 = idesc_bf16(128, 64, 0, 1);
         constexpr uint32_t idO128 = idesc_bf16(128, 128, 0, 1);
         constexpr uint32_t idO16 = idesc_bf16(128, 16, 0, 1);
-        uint32_t kvc = 0, scnt = 0, pcnt = 0;
-        uint32_t ofree_uses[2] = {0u, 0u};  // tiles started per O buffer
-        auto ofree_parity = [&](int b) -> uint32_t { return ((ofree_uses[b]++) & 1) ^ 1; };
-        int lt = 0;
+        uint32_t kvc = 0;                      // pipeline slot of chunk 0 of this unit
+        uint32_t quse[2] = {0u, 0u}, pcnt[2] = {0u, 0u};
         bool ok = true;
-        auto issue_pv = [&](uint32_t tO, int first, uint32_t sbuf, int st) {
-          const uint32_t vt = base + C::V_OFF + st * C::TILE;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-            const uint32_t a = sbuf + kk * 8;
-            if (D == 128) {
-              umma_ts(tO, a, v_desc<D>(vt, kk, 2), idO128, acc);
-            } else {
-              umma_ts(tO, a, v_desc<D>(vt, kk, 0), idO64, acc);
-              if (D == 80) umma_ts(tO + 64, a, v_desc<D>(vt, kk, 1), idO16, acc);
+        for (UnitIter<MODE> it(p, u_begin, u_end); ok && it.valid(); it.next()) {
+          Unit w;
+          it.get(p, w);
+          const bool act[2] = {w.t[0].rows > 0, w.t[1].rows > 0};
+          for (int x = 0; x < 2 && ok; ++x) {
+            if (!act[x]) continue;
+            ok = mbar_wait(&bar.q_full[x], quse[x] & 1, abort, p.status, site0 + 3);
+            ++quse[x];
+          }
+          if (!ok) break;
+          tc_fence_after();
+          // Per chunk m, for each active stream: O += P V of chunk m-1, then S = Q K^T
+          // of chunk m (the stream's S buffer is free once its P was consumed).
+          for (int m = 0; m <= w.nc && ok; ++m) {
+            const uint32_t slot_m = kvc + m, slot_p = kvc + m - 1;
+            const int st_m = slot_m % C::ST, st_p = slot_p % C::ST;
+            if (m < w.nc) {
+              if (!(ok = mbar_wait(&bar.k_full[st_m], (slot_m / C::ST) & 1, abort, p.status, site0 + 4))) break;
             }
-          }
-        };
-        // Chunks of consecutive tiles form one stream: S of chunk g is issued before
-        // P V of chunk g-1, also across a tile boundary, so the next tile's first
-        // S = Q K^T overlaps the current tile's last softmax.
-        struct Pending { bool valid, first, last; uint32_t sbuf, tO; int st, ob; };
-        Pending pend = {false, false, false, 0u, 0u, 0, 0};
-        uint32_t pv_slot = 0;  // pipeline slot of the pending P V
-        auto issue_pending = [&]() -> bool {
-          if (!mbar_wait(&bar.p_full, pcnt & 1, abort, p.status, site0 + 5)) return false;
-          ++pcnt;
-          if (!mbar_wait(&bar.v_full[pend.st], (pv_slot / C::ST) & 1, abort, p.status, site0 + 6)) return false;
-          if (pend.first) {
-            if (!mbar_wait(&bar.o_free[pend.ob], ofree_parity(pend.ob), abort, p.status, site0 + 7)) return false;
-          }
-          tc_fence_after();
-          issue_pv(pend.tO, pend.first, pend.sbuf, pend.st);
-          // Every P V completes a phase of o_done[its index & 1] (the softmax tracks
-          // them in order); a tile's last one also hands the O buffer to the epilogue.
-          umma_commit(&bar.o_done[pv_slot & 1]);
-          if (pend.last) umma_commit(&bar.o_full[pend.ob]);
-          umma_commit(&bar.v_empty[pend.st]);
-          pend.valid = false;
-          return true;
-        };
-        for (TileIter<MODE> it(p, t_begin, t_end); ok && it.valid(); it.next(), ++lt) {
-          TileInfo ti;
-          it.get(p, ti);
-          const int qb = lt & 1, ob = lt & 1;
-          const uint32_t tO = tmem + 256 + 128 * ob;
-          if (!(ok = mbar_wait(&bar.q_full[qb], (lt >> 1) & 1, abort, p.status, site0 + 3))) break;
-          tc_fence_after();
-          const uint32_t qt = base + C::Q_OFF + qb * C::TILE;
-          for (int m = 0; m < ti.nc; ++m) {
-            const int st = kvc % C::ST;
-            if (!(ok = mbar_wait(&bar.k_full[st], (kvc / C::ST) & 1, abort, p.status, site0 + 4))) break;
-            tc_fence_after();
-            const uint32_t kt = base + C::K_OFF + st * C::TILE;
-            const uint32_t sb = tmem + 128 * (scnt & 1);
+            if (m > 0) {
+              if (!(ok = mbar_wait(&bar.v_full[st_p], (slot_p / C::ST) & 1, abort, p.status, site0 + 6))) break;
+            }
+            for (int x = 0; x < 2; ++x) {
+              if (!act[x]) continue;
+              const uint32_t sb = tmem + 128 * x;
+              const uint32_t tO = tmem + 256 + 128 * x;
+              if (m > 0) {
+                if (!(ok = mbar_wait(&bar.p_full[x], pcnt[x] & 1, abort, p.status, site0 + 5))) break;
+                ++pcnt[x];
+                tc_fence_after();
+                const uint32_t vt = base + C::V_OFF + st_p * C::TILE;
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks)
-              umma_ss(sb, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idS, ks > 0 ? 1u : 0u);
-            umma_commit(&bar.s_full[scnt & 1]);
-            umma_commit(&bar.k_empty[st]);
-            if (m == ti.nc - 1) umma_commit(&bar.q_empty[qb]);
-            if (pend.valid && !(ok = issue_pending())) break;
-            pend = {true, m == 0, m == ti.nc - 1, sb, tO, st, ob};
-            pv_slot = kvc;
-            ++scnt;
-            ++kvc;
+                for (int kk = 0; kk < 8; ++kk) {
+                  const uint32_t acc = (m == 1 && kk == 0) ? 0u : 1u;
+                  const uint32_t a = sb + kk * 8;
+                  if (D == 128) {
+                    umma_ts(tO, a, v_desc<D>(vt, kk, 2), idO128, acc);
+                  } else {
+                    umma_ts(tO, a, v_desc<D>(vt, kk, 0), idO64, acc);
+                    if (D == 80) umma_ts(tO + 64, a, v_desc<D>(vt, kk, 1), idO16, acc);
+                  }
+                }
+                if (m == w.nc) umma_commit(&bar.o_full[x]);
+              }
+              if (m < w.nc) {
+                const uint32_t qt = base + C::Q_OFF + x * C::TILE;
+                const uint32_t kt = base + C::K_OFF + st_m * C::TILE;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                  umma_ss(sb, kmajor_desc<D>(qt, ks), kmajor_desc<D>(kt, ks), idS, ks > 0 ? 1u : 0u);
+                umma_commit(&bar.s_full[x]);
+                if (m == w.nc - 1) umma_commit(&bar.q_empty[x]);
+              }
+            }
+            if (!ok) break;
+            if (m < w.nc) umma_commit(&bar.k_empty[st_m]);
+            if (m > 0) umma_commit(&bar.v_empty[st_p]);
           }
+          kvc += w.nc;
         }
-        if (ok && pend.valid) ok = issue_pending();
         // Every MMA issued so far completes before TMEM is released.
         umma_commit(&bar.mma_done);
         const unsigned long long t0 = global_timer_ns();
@@ -384,99 +409,105 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     } else if (MODE == kGathered) {
       // -------------------------------------------------------- row gather
-      // Thread u owns rows u and u + 64 of the tile: it reads their list entries
-      // first, then issues all of their 16-byte copies (no dependent loads between).
+      // Thread u owns rows u and u + 64 of each stream's tile: it reads their list
+      // entries first, then issues all of their 16-byte copies.
       const int u = tid - 64;  // 0..63
       constexpr int VPR = D / 8;  // 16-byte vectors per row
       const int npast = p.npast;
-      int lt = 0;
-      for (TileIter<MODE> it(p, t_begin, t_end); it.valid(); it.next(), ++lt) {
-        TileInfo ti;
-        it.get(p, ti);
-        const int qb = lt & 1;
-        uint32_t ent[2] = {0u, 0u};
+      uint32_t quse[2] = {0u, 0u};
+      bool ok = true;
+      for (UnitIter<MODE> it(p, u_begin, u_end); ok && it.valid(); it.next()) {
+        Unit w;
+        it.get(p, w);
+        for (int x = 0; x < 2; ++x) {
+          const Tile &t = w.t[x];
+          if (t.rows == 0) continue;
+          uint32_t ent[2] = {0u, 0u};
 #pragma unroll
-        for (int k2 = 0; k2 < 2; ++k2)
-          if (u + 64 * k2 < ti.rows) ent[k2] = __ldg(p.entries + ti.ent0 + u + 64 * k2);
-        if (!mbar_wait(&bar.q_empty[qb], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 11)) break;
-        const uint32_t qt = base + C::Q_OFF + qb * C::TILE;
+          for (int k2 = 0; k2 < 2; ++k2)
+            if (u + 64 * k2 < t.rows) ent[k2] = __ldg(p.entries + t.ent0 + u + 64 * k2);
+          if (!(ok = mbar_wait(&bar.q_empty[x], (quse[x] & 1) ^ 1, abort, p.status, site0 + 11))) break;
+          ++quse[x];
+          const uint32_t qt = base + C::Q_OFF + x * C::TILE;
 #pragma unroll
-        for (int k2 = 0; k2 < 2; ++k2) {
-          const int r = u + 64 * k2;
-          const bool valid = r < ti.rows;
-          const uint16_t *row = p.q;
-          if (valid) {
-            const uint32_t ig = ent[k2] / (uint32_t)npast;
-            const int g = (int)(ig % (uint32_t)p.G);
-            const int i = (int)(ig / (uint32_t)p.G);
-            row = p.q + ti.b * p.q_sb + (int64_t)(ti.hk * p.G + g) * p.q_sh + (int64_t)i * p.q_sn;
-          }
-#pragma unroll
-          for (int c = 0; c < VPR; ++c) {
-            uint32_t dst;
-            if (c < 8) {
-              dst = qt + r * 128 + ((c ^ (r & 7)) << 4);
-            } else if (D == 128) {
-              dst = qt + C::R0 + r * 128 + (((c - 8) ^ (r & 7)) << 4);
-            } else {
-              dst = qt + C::R0 + r * 32 + (((c - 8) ^ ((r >> 2) & 1)) << 4);
+          for (int k2 = 0; k2 < 2; ++k2) {
+            const int r = u + 64 * k2;
+            const bool valid = r < t.rows;
+            const uint16_t *row = p.q;
+            if (valid) {
+              const uint32_t ig = ent[k2] / (uint32_t)npast;
+              const int g = (int)(ig % (uint32_t)p.G);
+              const int i = (int)(ig / (uint32_t)p.G);
+              row = p.q + t.b * p.q_sb + (int64_t)(t.hk * p.G + g) * p.q_sh + (int64_t)i * p.q_sn;
             }
-            cp_async_16_zfill(dst, valid ? row + c * 8 : p.q, valid);
+#pragma unroll
+            for (int c = 0; c < VPR; ++c) {
+              uint32_t dst;
+              if (c < 8) {
+                dst = qt + r * 128 + ((c ^ (r & 7)) << 4);
+              } else if (D == 128) {
+                dst = qt + C::R0 + r * 128 + (((c - 8) ^ (r & 7)) << 4);
+              } else {
+                dst = qt + C::R0 + r * 32 + (((c - 8) ^ ((r >> 2) & 1)) << 4);
+              }
+              cp_async_16_zfill(dst, valid ? row + c * 8 : p.q, valid);
+            }
           }
+          cp_async_commit();
+          cp_async_wait_all();
+          fence_proxy_async_smem();
+          mbar_arrive(&bar.q_full[x]);
         }
-        cp_async_commit();
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        mbar_arrive(&bar.q_full[qb]);
       }
     }
-  } else if (warp < 12) {
-    // ------------------------------------------------------------ softmax
+  } else {
+    // ------------------------------------------------- softmax + epilogue
     // tcgen05.ld / st are warp-collective (.sync.aligned): every wait is made
     // warp-uniform with __all_sync, and no TMEM access sits under a per-row branch.
     setmaxnreg_inc<kRegsSoftmax>();
-    const int half = (warp - 4) >> 2;       // key half of each chunk
+    const int x = (warp - 4) >> 2;          // stream
     const int r = (tid - 128) & 127;        // row within the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    // O columns this half rescales: [oc0, oc1).
-    constexpr int OH = ((D / 2 + 15) / 16) * 16;
-    const int oc0 = half ? OH : 0, oc1 = half ? D : OH;
+    const uint32_t tS = tmem + lane_off + 128 * x;
+    const uint32_t tO = tmem + lane_off + 256 + 128 * x;
     const float sl2 = p.scale_log2;
-    uint32_t scnt = 0;
-    // P V number k (counted over all chunks of this CTA, like scnt) completes phase
-    // k >> 1 of o_done[k & 1].  pv_seen: P Vs whose completion was already awaited.
-    uint32_t pv_seen = 0;
-    int lt = 0;
+    uint32_t scnt = 0, ocnt = 0;
     bool ok = true;
-    for (TileIter<MODE> it(p, t_begin, t_end); ok && it.valid(); it.next(), ++lt) {
-      TileInfo ti;
-      it.get(p, ti);
-      const int ob = lt & 1;
-      const uint32_t tO = tmem + lane_off + 256 + 128 * ob;
-      const bool live = r < ti.rows;
-      const int i = ti.i0 + r;  // query-major row
+    for (UnitIter<MODE> it(p, u_begin, u_end); ok && it.valid(); it.next()) {
+      Unit w;
+      it.get(p, w);
+      const Tile &t = w.t[x];
+      if (t.rows == 0) continue;
+      const bool live = r < t.rows;
+      // Row identity.
+      int i = t.i0 + r, h = t.h, slot = 0;
+      if (MODE == kGathered && live) {
+        const uint32_t ent = __ldg(p.entries + t.ent0 + r);
+        slot = (int)(ent % (uint32_t)p.npast);
+        const uint32_t ig = ent / (uint32_t)p.npast;
+        h = t.hk * p.G + (int)(ig % (uint32_t)p.G);
+        i = (int)(ig / (uint32_t)p.G);
+      }
       const int32_t *irow = (MODE == kQueryMajor && p.is_moba && live)
-                                ? p.idx + (((int64_t)ti.b * p.hq + ti.h) * p.N + i) * p.topk
+                                ? p.idx + (((int64_t)t.b * p.hq + h) * p.N + i) * p.topk
                                 : nullptr;
       float m_run = -INFINITY, l_run = 0.f;
-      for (int m = 0; m < ti.nc; ++m, ++scnt) {
-        const int sbi = scnt & 1;
-        const uint32_t tS = tmem + lane_off + 128 * sbi;
-        // The two halves must take every decision together (they meet at named
-        // barriers), so each wait's outcome is AND-ed over both warpgroups.
-        ok = mbar_wait(&bar.s_full[sbi], (scnt >> 1) & 1, abort, p.status, site0 + 12);
-        if (!(ok = named_barrier_and(1, 256, ok))) break;
+      for (int m = 0; m < w.nc; ++m, ++scnt) {
+        ok = mbar_wait(&bar.s_full[x], scnt & 1, abort, p.status, site0 + 12);
+        if (!(ok = __all_sync(FULL, ok))) break;
         tc_fence_after();
-        uint32_t sv[64];
-        tmem_ld32(tS + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tS + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        uint32_t sv[128];
+        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
         tmem_wait_ld();
         float *s = reinterpret_cast<float *>(sv);
         // Masks.
-        const int key0 = chunk_key<MODE>(p, ti, m) + 64 * half;
+        const int key0 = w.key0 + m * kTileKeys;
         if (MODE == kQueryMajor) {
           if (p.is_moba) {
-            if (m < ti.ntail) {
+            if (key0 < t.cB) {
               // Window tail into an earlier block: keys i - j < window that the row's
               // own selection does not already cover.
               bool covered = false;
@@ -484,39 +515,37 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 const int blk = key0 / p.block;
                 for (int u2 = 0; u2 < p.topk; ++u2) covered |= (__ldg(irow + u2) == blk);
               }
+              const bool none = covered || !live || p.window <= 0;
 #pragma unroll
-              for (int e = 0; e < 64; ++e)
-                if (covered || !live || i - (key0 + e) >= p.window) s[e] = -INFINITY;
-            } else if (key0 + 64 > ti.i0) {
+              for (int e = 0; e < 128; ++e)
+                if (none || i - (key0 + e) >= p.window) s[e] = -INFINITY;
+            } else if (key0 + kTileKeys > t.i0) {
 #pragma unroll
-              for (int e = 0; e < 64; ++e)
+              for (int e = 0; e < 128; ++e)
                 if (key0 + e > i) s[e] = -INFINITY;
             }
           } else {
-            const bool full = (key0 + 63 <= ti.i0) && (key0 >= ti.i0 + ti.rows - 1 - p.window + 1);
+            const bool full = (key0 + kTileKeys - 1 <= t.i0) &&
+                              (key0 >= t.i0 + t.rows - 1 - p.window + 1);
             if (!full) {
 #pragma unroll
-              for (int e = 0; e < 64; ++e) {
+              for (int e = 0; e < 128; ++e) {
                 const int j = key0 + e;
                 if (j > i || i - j >= p.window) s[e] = -INFINITY;
               }
             }
           }
         }
-        float mx4[8];
+        float mx8[8];
 #pragma unroll
-        for (int u2 = 0; u2 < 8; ++u2) mx4[u2] = s[u2];
+        for (int u2 = 0; u2 < 8; ++u2) mx8[u2] = s[u2];
 #pragma unroll
-        for (int e = 8; e < 64; ++e) mx4[e & 7] = fmaxf(mx4[e & 7], s[e]);
-        // The row maximum over both halves of the chunk.
-        bar.xmax[sbi][half][r] = fmaxf(fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])),
-                                       fmaxf(fmaxf(mx4[4], mx4[5]), fmaxf(mx4[6], mx4[7])));
-        named_barrier_sync(1, 256);
-        const float mx = fmaxf(bar.xmax[sbi][0][r], bar.xmax[sbi][1][r]);
+        for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[e]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_new = fmaxf(m_run, mx * sl2);
         // Raise the running maximum only when it grows by more than 2^8 (or from
-        // -inf); rows that keep theirs multiply O by 1 when the warp rescales.  Both
-        // halves of a row take the same decision from the same numbers.
+        // -inf); rows that keep theirs multiply O by 1 when the warp rescales.
         const bool raise = (m == 0) || (m_new > m_run + (float)kRescaleThreshold);
         const bool scale_o = raise && m > 0 && m_run != -INFINITY;
         const float alpha = scale_o ? ex2_approx(m_run - m_new) : 1.f;
@@ -524,104 +553,60 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           l_run *= alpha;
           m_run = m_new;
         }
+        if (__any_sync(FULL, scale_o)) {
+          // S(m) complete implies P V of chunk m-1 complete: O is final for now.
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 16) {
+            uint32_t o[16];
+            tmem_ld16(tO + c0, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(tO + c0, o);
+          }
+        }
         const float mu = (m_run == -INFINITY) ? 0.f : m_run;
         float ls[8];
 #pragma unroll
         for (int u2 = 0; u2 < 8; ++u2) ls[u2] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < 64; ++e) {
           const float x0 = fmaf(s[2 * e], sl2, -mu), x1 = fmaf(s[2 * e + 1], sl2, -mu);
           const float p0 = ((2 * e) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x0) : ex2_approx(x0);
           const float p1 = ((2 * e + 1) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x1) : ex2_approx(x1);
           ls[e & 7] += p0 + p1;
           sv[e] = pack_bf16x2(p0, p1);
         }
-        // P of keys [64 half, 64 half + 64) -> TMEM columns [32 half, 32 half + 32).
-        tmem_st16(tS + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-        tmem_st16(tS + 32 * half + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+        tmem_st16(tS, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+        tmem_st16(tS + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+        tmem_st16(tS + 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[32]));
+        tmem_st16(tS + 48, *reinterpret_cast<uint32_t(*)[16]>(&sv[48]));
         l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-        // Before P V number scnt may be issued, the P V two back must be complete
-        // (o_done[scnt & 1] is reused by it); if this chunk rescales O, the previous
-        // one too.  The pair of warpgroups decides together.
-        const bool rescale = (m > 0) && named_barrier_and(2, 256, !__any_sync(FULL, scale_o)) == false;
-        const uint32_t need = rescale ? scnt : (scnt >= 1 ? scnt - 1 : 0);
-        while (pv_seen < need) {
-          ok = mbar_wait(&bar.o_done[pv_seen & 1], (pv_seen >> 1) & 1, abort, p.status, site0 + 13);
-          if (!(ok = named_barrier_and(1, 256, ok))) break;
-          ++pv_seen;
-        }
-        if (!ok) break;
-        if (rescale) {
-          // O holds chunks 0..m-1 now; rescale this half's columns where a row of the
-          // warp raised its maximum.
-          tc_fence_after();
-          if (__any_sync(FULL, scale_o)) {
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 16) {
-              if (c0 < oc0 || c0 >= oc1) continue;
-              uint32_t o[16];
-              tmem_ld16(tO + c0, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st16(tO + c0, o);
-            }
-          }
-        }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bar.p_full);
+        mbar_arrive(&bar.p_full[x]);
       }
       if (!ok) break;
-      // Hand the row statistics to the epilogue once it has drained this O buffer's
-      // previous tile (that also orders every earlier P V before this point).
-      ok = mbar_wait(&bar.o_free[ob], ((lt >> 1) & 1) ^ 1, abort, p.status, site0 + 14);
-      if (!(ok = named_barrier_and(1, 256, ok))) break;
-      bar.stat[ob][half][r] = make_float2(m_run, l_run);
-      mbar_arrive(&bar.stat_full[ob]);
-    }
-  } else {
-    // ----------------------------------------------------------- epilogue
-    // Keeps the registers it was launched with (kRegsEpilogue).
-    const int r = tid - 384;
-    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    int lt = 0;
-    bool ok = true;
-    for (TileIter<MODE> it(p, t_begin, t_end); ok && it.valid(); it.next(), ++lt) {
-      TileInfo ti;
-      it.get(p, ti);
-      const int ob = lt & 1;
-      const uint32_t tO = tmem + lane_off + 256 + 128 * ob;
-      const bool live = r < ti.rows;
-      int i = ti.i0 + r, h = ti.h, slot = 0;
-      if (MODE == kGathered && live) {
-        const uint32_t ent = __ldg(p.entries + ti.ent0 + r);
-        slot = (int)(ent % (uint32_t)p.npast);
-        const uint32_t ig = ent / (uint32_t)p.npast;
-        h = ti.hk * p.G + (int)(ig % (uint32_t)p.G);
-        i = (int)(ig / (uint32_t)p.G);
-      }
-      ok = mbar_wait(&bar.stat_full[ob], (lt >> 1) & 1, abort, p.status, site0 + 15);
-      ok = ok && mbar_wait(&bar.o_full[ob], (lt >> 1) & 1, abort, p.status, site0 + 16);
+      // ------------------------------------------------------------ epilogue
+      ok = mbar_wait(&bar.o_full[x], ocnt & 1, abort, p.status, site0 + 14);
       if (!(ok = __all_sync(FULL, ok))) break;
+      ++ocnt;
       tc_fence_after();
-      const float2 st0 = bar.stat[ob][0][r], st1 = bar.stat[ob][1][r];
-      const float m_run = st0.x, l_run = st0.y + st1.y;
       const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
       const float own_lse = (m_run + log2f(l_run)) * 0.69314718055994530942f;  // natural log
-      // Destination: a partial slot (gathered tiles: the row's past-block slot; MoBA
-      // query-major tiles: the own-block slot topk-1, merged afterwards), or the
-      // output itself when nothing needs merging (SWA, or topk = 1).
+      // Destination: a partial slot (gathered: the row's past-block slot; MoBA
+      // query-major: the own-block slot topk-1, merged afterwards), or the output
+      // itself when nothing needs merging (SWA, or topk = 1).
       uint16_t *dst;
       float *ldst;
       if (MODE == kGathered || (p.is_moba && p.npast > 0)) {
         const int sl = (MODE == kGathered) ? slot : p.npast;
-        const int64_t pidx = (((int64_t)ti.b * p.hq + h) * p.chunk_rows + (i - p.chunk * p.chunk_rows)) * p.topk + sl;
+        const int64_t pidx = (((int64_t)t.b * p.hq + h) * p.chunk_rows + (i - p.chunk * p.chunk_rows)) * p.topk + sl;
         dst = p.opart + pidx * D;
         ldst = p.lpart + pidx;
       } else {
-        dst = p.out + ti.b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)i * p.o_sn;
-        ldst = p.lse + ((int64_t)ti.b * p.hq + h) * p.N + i;
+        dst = p.out + t.b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)i * p.o_sn;
+        ldst = p.lse + ((int64_t)t.b * p.hq + h) * p.N + i;
       }
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
@@ -635,18 +620,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4) {
             if (v4 * 8 >= cols) break;
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv_l, __uint_as_float(o[8 * v4 + 1]) * inv_l);
-            w.y = pack_bf16x2(__uint_as_float(o[8 * v4 + 2]) * inv_l, __uint_as_float(o[8 * v4 + 3]) * inv_l);
-            w.z = pack_bf16x2(__uint_as_float(o[8 * v4 + 4]) * inv_l, __uint_as_float(o[8 * v4 + 5]) * inv_l);
-            w.w = pack_bf16x2(__uint_as_float(o[8 * v4 + 6]) * inv_l, __uint_as_float(o[8 * v4 + 7]) * inv_l);
-            *reinterpret_cast<uint4 *>(dst + c0 + 8 * v4) = w;
+            uint4 q4;
+            q4.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv_l, __uint_as_float(o[8 * v4 + 1]) * inv_l);
+            q4.y = pack_bf16x2(__uint_as_float(o[8 * v4 + 2]) * inv_l, __uint_as_float(o[8 * v4 + 3]) * inv_l);
+            q4.z = pack_bf16x2(__uint_as_float(o[8 * v4 + 4]) * inv_l, __uint_as_float(o[8 * v4 + 5]) * inv_l);
+            q4.w = pack_bf16x2(__uint_as_float(o[8 * v4 + 6]) * inv_l, __uint_as_float(o[8 * v4 + 7]) * inv_l);
+            *reinterpret_cast<uint4 *>(dst + c0 + 8 * v4) = q4;
           }
         }
       }
       if (live) *ldst = own_lse;
+      // The O reads are done before this stream's next P lets a P V overwrite O.
+      __syncwarp();
       tc_fence_before();
-      mbar_arrive(&bar.o_free[ob]);
     }
   }
 
@@ -667,7 +653,7 @@ static cudaError_t launch_attn_dm(const CUtensorMap *maps, const AttnParams &p, 
   using C = AttnCfg<D>;
   auto kern = attn_fwd_kernel<D, MODE>;
   // The warpgroups re-split the registers the CTA is launched with (setmaxnreg); a
-  // build that launched with fewer than 168 per thread would leave an increase
+  // build that launched with fewer than the split needs would leave an increase
   // waiting forever, so refuse to launch it.
   static int regs = 0;
   if (regs == 0) {
@@ -700,6 +686,17 @@ cudaError_t launch_attn(const CUtensorMap *maps, const AttnParams &p, int mode, 
     }
   }
   return cudaErrorInvalidValue;
+}
+
+// Query-major work units for rows [row_begin, row_end) (see query_major_unit).
+int query_major_units(int batch, int hq, int hkv, int block, int is_moba, int row_begin,
+                      int row_end) {
+  const int nq = (row_end - row_begin + kTileRows - 1) / kTileRows;
+  const int G = hq / hkv;
+  if (G >= 2) return nq * batch * hkv * ((G + 1) / 2);
+  const int tpb = is_moba ? block / kTileRows : nq;
+  const int ngroups = (nq + tpb - 1) / tpb;
+  return ngroups * ((tpb + 1) / 2) * batch * hkv;
 }
 
 int attn_smem_bytes(int d) {

@@ -9,6 +9,7 @@
 namespace moba {
 
 constexpr int kTileRows = 128;   // query rows per attention tile (tcgen05 M)
+constexpr int kUnitRows = 256;   // list entries per gathered work unit (two tiles)
 constexpr int kTileKeys = 128;   // keys per attention chunk (tcgen05 N of S = QK^T)
 constexpr size_t kPartialCapBytes = size_t(4) << 30;  // partial outputs kept per pass
 
@@ -25,9 +26,9 @@ struct WorkspaceLayout {
   size_t off_counts;   // int32 [nlists]       entries per list (atomic counts)
   size_t off_cursor;   // int32 [nlists]       scatter cursors
   size_t off_listoff;  // int32 [nlists + 1]   exclusive prefix of counts
-  size_t off_tileoff;  // int32 [nlists + 1]   exclusive prefix of ceil(count / 128)
+  size_t off_tileoff;  // int32 [nlists + 1]   exclusive prefix of ceil(count / 256)
   size_t off_entries;  // uint32 [max_entries] entry = (i * G + g) * npast + slot
-  size_t off_tiles;    // int4 [max_tiles]      per 128-row tile: list, first entry, rows
+  size_t off_tiles;    // int4 [max_tiles]      per 256-entry unit: list, first entry, rows
   size_t off_opart;    // bf16 [batch, hq, chunk_rows, topk, d]: slots 0..npast-1 past
                        //      blocks, slot npast the own block
   size_t off_lpart;    // f32  [batch, hq, chunk_rows, topk]
@@ -56,7 +57,7 @@ inline WorkspaceLayout make_layout(int batch, int hq, int hkv, int N, int d, int
   w.nchunks = static_cast<int>((N + w.chunk_rows - 1) / w.chunk_rows);
   w.nlists = w.nchunks * batch * hkv * w.nblk;
   w.max_entries = static_cast<long long>(batch) * hq * N * w.npast;
-  w.max_tiles = w.max_entries / kTileRows + w.nlists + 1;
+  w.max_tiles = w.max_entries / kUnitRows + w.nlists + 1;
   size_t off = 0;
   w.off_counts = off;  off = align_up(off + sizeof(int) * size_t(w.nlists), 256);
   w.off_cursor = off;  off = align_up(off + sizeof(int) * size_t(w.nlists), 256);
@@ -109,11 +110,11 @@ struct AttnParams {
   int is_moba;             // 0: sliding window only (swa_attn_fwd)
   // Query-major pass: row range of this pass.
   int row_begin, row_end;  // multiples of 128 except row_end == N
-  int ntiles;              // query-major tiles in this pass
+  int ntiles;              // query-major work units in this pass
   // Block-major lists and partials (MoBA).
   const int *listoff;
   const int *tileoff;
-  const int4 *tiles;       // per gathered tile: list, first entry, rows
+  const int4 *tiles;       // per gathered unit: list, first entry, rows (<= 256)
   const uint32_t *entries;
   uint16_t *opart;         // [batch, hq, chunk_rows, topk, d]
   float *lpart;            // [batch, hq, chunk_rows, topk]

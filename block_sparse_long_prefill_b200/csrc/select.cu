@@ -271,7 +271,7 @@ gate_topk_kernel(const SelectParams p) {
 
 // ------------------------------------------------------------- list offsets
 //
-// Exclusive prefix sums of the list counts (entries) and of their 128-row tiles,
+// Exclusive prefix sums of the list counts (entries) and of their 256-entry units,
 // over all lists in (chunk, batch, kv-head, block) order; resets the scatter
 // cursors.  One CTA.
 constexpr int kScanThreads = 1024;
@@ -287,7 +287,7 @@ list_scan_kernel(const int *__restrict__ counts, int *__restrict__ cursor, int *
   for (int base = 0; base < nlists; base += kScanThreads) {
     const int L = base + tid;
     const int ce = (L < nlists) ? counts[L] : 0;
-    const int ct = (ce + kTileRows - 1) / kTileRows;
+    const int ct = (ce + kUnitRows - 1) / kUnitRows;
     int se = ce, st = ct;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -328,12 +328,13 @@ list_scan_kernel(const int *__restrict__ counts, int *__restrict__ cursor, int *
     tileoff[nlists] = carry_t;
   }
   __syncthreads();
-  // Tile table: one {list, first entry, rows} record per 128-entry tile, so the
-  // attention kernel reads a tile's description with a single load.
+  // Unit table: one {list, first entry, rows} record per unit of up to 256 entries
+  // (two 128-row tiles over the same block), so the attention kernel reads a unit's
+  // description with a single load.
   for (int L = tid; L < nlists; L += kScanThreads) {
     const int first = listoff[L], cnt = counts[L], t0 = tileoff[L];
-    for (int k = 0; k * kTileRows < cnt; ++k)
-      tiles[t0 + k] = make_int4(L, first + k * kTileRows, min(kTileRows, cnt - k * kTileRows), 0);
+    for (int k = 0; k * kUnitRows < cnt; ++k)
+      tiles[t0 + k] = make_int4(L, first + k * kUnitRows, min(kUnitRows, cnt - k * kUnitRows), 0);
   }
 }
 
