@@ -64,7 +64,8 @@ struct AttnCfg {
   static constexpr int Q_OFF = 0;                          // Q_A, Q_B
   static constexpr int K_OFF = 2 * TILE;                   // K ring
   static constexpr int V_OFF = K_OFF + ST * TILE;          // V ring
-  static constexpr int BAR_OFF = V_OFF + ST * TILE;
+  static constexpr int EPI_OFF = V_OFF + ST * TILE;       // 8 softmax warps x 32 rows x 64 B
+  static constexpr int BAR_OFF = EPI_OFF + 8 * 2048;
   static constexpr int SMEM = BAR_OFF + 1024 + 1024;       // + barriers + alignment slack
   static constexpr uint32_t BYTES = 128u * D * 2u;         // bytes one full tile load moves
 };
@@ -250,7 +251,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (tid == 0) {
     for (int x = 0; x < 2; ++x) {
-      mbar_init(&bar.q_full[x], MODE == kGathered ? 64 : 1);
+      mbar_init(&bar.q_full[x], MODE == kGathered ? 32 : 1);
       mbar_init(&bar.q_empty[x], 1);
       mbar_init(&bar.s_full[x], 1);
       mbar_init(&bar.p_full[x], 128);
@@ -409,55 +410,55 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     } else if (MODE == kGathered) {
       // -------------------------------------------------------- row gather
-      // Thread u owns rows u and u + 64 of each stream's tile: it reads their list
-      // entries first, then issues all of their 16-byte copies.
-      const int u = tid - 64;  // 0..63
+      // Warp 2 fills stream A's query tile, warp 3 stream B's: lane l owns rows l,
+      // l + 32, l + 64, l + 96; it reads their list entries first, then issues all of
+      // their 16-byte copies.
+      const int x = warp - 2;
+      const int l = lane;
       constexpr int VPR = D / 8;  // 16-byte vectors per row
       const int npast = p.npast;
-      uint32_t quse[2] = {0u, 0u};
+      uint32_t quse = 0;
       bool ok = true;
       for (UnitIter<MODE> it(p, u_begin, u_end); ok && it.valid(); it.next()) {
         Unit w;
         it.get(p, w);
-        for (int x = 0; x < 2; ++x) {
-          const Tile &t = w.t[x];
-          if (t.rows == 0) continue;
-          uint32_t ent[2] = {0u, 0u};
+        const Tile &t = w.t[x];
+        if (t.rows == 0) continue;
+        uint32_t ent[4];
 #pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2)
-            if (u + 64 * k2 < t.rows) ent[k2] = __ldg(p.entries + t.ent0 + u + 64 * k2);
-          if (!(ok = mbar_wait(&bar.q_empty[x], (quse[x] & 1) ^ 1, abort, p.status, site0 + 11))) break;
-          ++quse[x];
-          const uint32_t qt = base + C::Q_OFF + x * C::TILE;
+        for (int k2 = 0; k2 < 4; ++k2)
+          ent[k2] = (l + 32 * k2 < t.rows) ? __ldg(p.entries + t.ent0 + l + 32 * k2) : 0u;
+        if (!(ok = mbar_wait(&bar.q_empty[x], (quse & 1) ^ 1, abort, p.status, site0 + 11))) break;
+        ++quse;
+        const uint32_t qt = base + C::Q_OFF + x * C::TILE;
 #pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2) {
-            const int r = u + 64 * k2;
-            const bool valid = r < t.rows;
-            const uint16_t *row = p.q;
-            if (valid) {
-              const uint32_t ig = ent[k2] / (uint32_t)npast;
-              const int g = (int)(ig % (uint32_t)p.G);
-              const int i = (int)(ig / (uint32_t)p.G);
-              row = p.q + t.b * p.q_sb + (int64_t)(t.hk * p.G + g) * p.q_sh + (int64_t)i * p.q_sn;
-            }
-#pragma unroll
-            for (int c = 0; c < VPR; ++c) {
-              uint32_t dst;
-              if (c < 8) {
-                dst = qt + r * 128 + ((c ^ (r & 7)) << 4);
-              } else if (D == 128) {
-                dst = qt + C::R0 + r * 128 + (((c - 8) ^ (r & 7)) << 4);
-              } else {
-                dst = qt + C::R0 + r * 32 + (((c - 8) ^ ((r >> 2) & 1)) << 4);
-              }
-              cp_async_16_zfill(dst, valid ? row + c * 8 : p.q, valid);
-            }
+        for (int k2 = 0; k2 < 4; ++k2) {
+          const int r = l + 32 * k2;
+          const bool valid = r < t.rows;
+          const uint16_t *row = p.q;
+          if (valid) {
+            const uint32_t ig = ent[k2] / (uint32_t)npast;
+            const int g = (int)(ig % (uint32_t)p.G);
+            const int i = (int)(ig / (uint32_t)p.G);
+            row = p.q + t.b * p.q_sb + (int64_t)(t.hk * p.G + g) * p.q_sh + (int64_t)i * p.q_sn;
           }
-          cp_async_commit();
-          cp_async_wait_all();
-          fence_proxy_async_smem();
-          mbar_arrive(&bar.q_full[x]);
+#pragma unroll
+          for (int c = 0; c < VPR; ++c) {
+            uint32_t dst;
+            if (c < 8) {
+              dst = qt + r * 128 + ((c ^ (r & 7)) << 4);
+            } else if (D == 128) {
+              dst = qt + C::R0 + r * 128 + (((c - 8) ^ (r & 7)) << 4);
+            } else {
+              dst = qt + C::R0 + r * 32 + (((c - 8) ^ ((r >> 2) & 1)) << 4);
+            }
+            cp_async_16_zfill(dst, valid ? row + c * 8 : p.q, valid);
+          }
         }
+        cp_async_commit();
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        mbar_arrive(&bar.q_full[x]);
       }
     }
   } else {
@@ -608,6 +609,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         dst = p.out + t.b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)i * p.o_sn;
         ldst = p.lse + ((int64_t)t.b * p.hq + h) * p.N + i;
       }
+      // Stores go through a per-warp staging buffer (32 rows x 64 bytes, chunk index
+      // XOR-swizzled by row pair): lane r writes its row's piece, then each lane stores
+      // 16 bytes of eight whole 64-byte row segments per instruction (coalesced).
+      unsigned char *stg = sbase + C::EPI_OFF + (warp - 4) * 2048;
+      const int wl = r & 31;                  // this lane's row within the warp
+      uint16_t *rdst[4];
+      bool rlive[4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int src = jj * 8 + (lane >> 2);
+        rdst[jj] = reinterpret_cast<uint16_t *>(__shfl_sync(FULL, reinterpret_cast<uintptr_t>(dst), src));
+        rlive[jj] = __shfl_sync(FULL, live ? 1 : 0, src) != 0;
+      }
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         const int cols = (D - c0) < 32 ? (D - c0) : 32;  // D = 80 ends with 16
@@ -616,16 +630,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (cols == 32) tmem_ld32(tO + c0, o);
         else tmem_ld16(tO + c0, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
         tmem_wait_ld();
-        if (live) {
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            if (v4 * 8 >= cols) break;
-            uint4 q4;
-            q4.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv_l, __uint_as_float(o[8 * v4 + 1]) * inv_l);
-            q4.y = pack_bf16x2(__uint_as_float(o[8 * v4 + 2]) * inv_l, __uint_as_float(o[8 * v4 + 3]) * inv_l);
-            q4.z = pack_bf16x2(__uint_as_float(o[8 * v4 + 4]) * inv_l, __uint_as_float(o[8 * v4 + 5]) * inv_l);
-            q4.w = pack_bf16x2(__uint_as_float(o[8 * v4 + 6]) * inv_l, __uint_as_float(o[8 * v4 + 7]) * inv_l);
-            *reinterpret_cast<uint4 *>(dst + c0 + 8 * v4) = q4;
+        for (int v4 = 0; v4 < 4; ++v4) {
+          if (v4 * 8 >= cols) break;
+          uint4 q4;
+          q4.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv_l, __uint_as_float(o[8 * v4 + 1]) * inv_l);
+          q4.y = pack_bf16x2(__uint_as_float(o[8 * v4 + 2]) * inv_l, __uint_as_float(o[8 * v4 + 3]) * inv_l);
+          q4.z = pack_bf16x2(__uint_as_float(o[8 * v4 + 4]) * inv_l, __uint_as_float(o[8 * v4 + 5]) * inv_l);
+          q4.w = pack_bf16x2(__uint_as_float(o[8 * v4 + 6]) * inv_l, __uint_as_float(o[8 * v4 + 7]) * inv_l);
+          *reinterpret_cast<uint4 *>(stg + wl * 64 + ((v4 ^ ((wl >> 1) & 3)) << 4)) = q4;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int row = jj * 8 + (lane >> 2), ch = lane & 3;
+          if (ch * 8 < cols && rlive[jj]) {
+            const uint4 q4 = *reinterpret_cast<const uint4 *>(stg + row * 64 + ((ch ^ ((row >> 1) & 3)) << 4));
+            *reinterpret_cast<uint4 *>(rdst[jj] + c0 + ch * 8) = q4;
           }
         }
       }
