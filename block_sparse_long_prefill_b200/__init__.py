@@ -25,11 +25,12 @@ MOBA_OK = 0
 _STATUS = {
     -1: "MOBA_ERR_SHAPE", -2: "MOBA_ERR_DIM", -3: "MOBA_ERR_ALIGN", -4: "MOBA_ERR_ARG",
     -5: "MOBA_ERR_WORKSPACE", -6: "MOBA_ERR_LAUNCH", -7: "MOBA_ERR_DEVICE", -8: "MOBA_ERR_NODEVICE",
+    -9: "MOBA_ERR_TOO_LARGE",
 }
 
 # Entry points declared in include/moba.h.
 ABI_FUNCTIONS = ("moba_workspace_size", "moba_pool_keys", "moba_select_topk", "moba_attn_fwd",
-                 "swa_attn_fwd", "moba_device_status", "moba_status_string")
+                 "swa_attn_fwd", "moba_prefill_static", "moba_device_status", "moba_status_string")
 
 
 class MobaError(RuntimeError):
@@ -55,6 +56,7 @@ def _load():
     lib.moba_select_topk.argtypes = [T, P, I, I, I, I, I, I, I, P, P, S, P]
     lib.moba_attn_fwd.argtypes = [T, T, T, P, I, I, I, I, I, I, I, I, ctypes.c_float, T, P, P, S, P]
     lib.swa_attn_fwd.argtypes = [T, T, T, I, I, I, I, I, I, ctypes.c_float, T, P, P]
+    lib.moba_prefill_static.argtypes = [T, T, T, I, I, I, I, I, I, I, I, ctypes.c_float, T, P, P]
     lib.moba_device_status.argtypes = []
     lib.moba_status_string.argtypes = [I]
     lib.moba_status_string.restype = ctypes.c_char_p
@@ -158,6 +160,22 @@ def swa_attn_fwd(q, k, v, window: int, scale: float = 0.0, out=None, lse=None, s
     _check("swa_attn_fwd",
            _lib.swa_attn_fwd(_t(q), _t(k), _t(v), b, hq, hkv, N, d, window, float(scale), _t(out),
                              lse.data_ptr(), _stream(stream)))
+    return out, lse
+
+
+def moba_prefill_static(q, k, v, block: int, topk: int, window: int = 0, scale: float = 0.0,
+                        out=None, lse=None, stream=None):
+    """The whole prefill with the library's own fixed scratch (no workspace): for
+    callers that cannot allocate device memory.  Returns (out, lse)."""
+    b, hq, N, d = q.shape
+    hkv = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device)
+    _check("moba_prefill_static",
+           _lib.moba_prefill_static(_t(q), _t(k), _t(v), b, hq, hkv, N, d, block, topk, window,
+                                    float(scale), _t(out), lse.data_ptr(), _stream(stream)))
     return out, lse
 
 

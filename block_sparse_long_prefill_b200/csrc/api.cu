@@ -329,6 +329,7 @@ const char *moba_status_string(int status) {
     case MOBA_ERR_LAUNCH: return "CUDA launch or driver call failed";
     case MOBA_ERR_DEVICE: return "a kernel wait timed out on the device";
     case MOBA_ERR_NODEVICE: return "no sm_100 device is current";
+    case MOBA_ERR_TOO_LARGE: return "problem exceeds the 32 MiB static scratch of moba_prefill_static";
   }
   return "unknown status";
 }

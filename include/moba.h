@@ -27,7 +27,8 @@
  *   - d must be 64, 80 or 128 for the attention calls (any multiple of 8 up to 256
  *     for moba_pool_keys and moba_select_topk).
  *   - Ownership: the caller allocates every buffer (inputs, outputs, workspace); the
- *     library allocates no device memory and keeps no state between calls.
+ *     library allocates no device memory and keeps no state between calls (except the
+ *     fixed scratch array of moba_prefill_static, below).
  *   - Execution: every call only enqueues kernels on `stream` (a cudaStream_t, 0 for
  *     the legacy default stream) and returns; nothing synchronises.
  *   - Errors: calls return MOBA_OK (0) or a negative MOBA_ERR_* code.  Argument
@@ -54,6 +55,7 @@ extern "C" {
 #define MOBA_ERR_LAUNCH -6    /* a CUDA launch or driver call failed */
 #define MOBA_ERR_DEVICE -7    /* a kernel wait ran out (see moba_device_status) */
 #define MOBA_ERR_NODEVICE -8  /* no sm_100 device is current */
+#define MOBA_ERR_TOO_LARGE -9 /* problem needs more than moba_prefill_static's scratch */
 
 typedef struct {
     void *ptr;
@@ -125,6 +127,24 @@ int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *id
  */
 int swa_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq, int hkv, int N,
                  int d, int window, float scale, moba_tensor out, float *lse, void *stream);
+
+/*
+ * The whole MoBA prefill (moba_pool_keys, moba_select_topk, moba_attn_fwd) without any
+ * caller-provided workspace, for callers that cannot allocate device memory: code
+ * inside a CUDA-graph capture that forbids allocation, plugins whose host framework
+ * owns all allocations, runtimes with a memory budget fixed up front.  The paper has
+ * no counterpart; it is a deployment convenience.
+ *   Arguments as for moba_attn_fwd; out and lse are written, nothing else is.
+ *   Scratch: one 32 MiB device array inside the library (held, on each GPU that runs
+ *   this call, until the process exits).  Problems whose pooled keys, block choices
+ *   and workspace (moba_workspace_size) need more return MOBA_ERR_TOO_LARGE.
+ *   The first call on a device looks up the array's device address (keep it outside
+ *   any stream capture).  All calls share the array: calls that overlap on the GPU
+ *   (other streams, other host threads) race and must be serialised by the caller.
+ */
+int moba_prefill_static(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq, int hkv,
+                        int N, int d, int block, int topk, int window, float scale,
+                        moba_tensor out, float *lse, void *stream);
 
 /*
  * Reads and clears the device-side status word that bounded kernel waits write

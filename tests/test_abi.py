@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings():
     assert moba.status_string(0) == "ok"
-    for code in range(-8, 0):
+    for code in range(-9, 0):
         assert moba.status_string(code) != "unknown status"
 
 
