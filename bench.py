@@ -61,6 +61,50 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+# ------------------------------------------------------------------ multi-rank
+
+def max_over_ranks(value: float, device) -> float:
+    """The largest of every rank's value (one all-reduce; identity without a group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_rate(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job rate: every rank processed units_per_rank in at most max_ms."""
+    return units_per_rank * world / (max_ms * 1e-3)
+
+
+def source_digest() -> str:
+    """sha256 over the library sources: ties a stored ncu traffic figure to the
+    kernels it was measured on."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_long_prefill_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()
+
+
+def stored_traffic(workload: str):
+    """DRAM bytes per attention step from the committed ncu summary, or None when the
+    kernels changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    rec = d.get(workload)
+    if not rec or rec.get("sources_sha256") != source_digest():
+        return None
+    return rec.get("attention_dram_bytes_per_step")
+
+
 # ------------------------------------------------------------------ accounting
 
 def attended_pairs_moba(idx: torch.Tensor, w: workloads.Workload) -> int:
@@ -191,14 +235,16 @@ def run_ours(args, rank, world, device):
         out_t, lse_t = runner.out, runner.lse
         layout_chunks = 1
         try:
-            per_row = (w.topk - 1) * (w.d * 2 + 4) * w.batch * w.hq
+            per_row = (w.topk if w.topk > 1 else 0) * (w.d * 2 + 4) * w.batch * w.hq
             cap = 4 << 30
             if per_row * w.seqlen > cap:
                 rows = max(128, (cap // per_row) // 128 * 128)
                 layout_chunks = math.ceil(w.seqlen / rows)
         except ZeroDivisionError:
             pass
-        launches_per_step = 2 + (2 if w.topk > 1 else 0) + layout_chunks * (2 if w.topk > 1 else 1)
+        # pool, gate (+ scan, scatter), and per query chunk: past-block pass, own-block
+        # pass, merge (only the own-block pass when topk = 1).
+        launches_per_step = 2 + (2 if w.topk > 1 else 0) + layout_chunks * (3 if w.topk > 1 else 1)
     else:
         out_t = torch.empty_like(qd)
         lse_t = torch.empty(w.batch, w.hq, w.seqlen, dtype=torch.float32, device=device)
@@ -242,25 +288,25 @@ def run_ours(args, rank, world, device):
             for a, b_, n in zip(evs[:-1], evs[1:], names):
                 per_stage.setdefault(n, []).append(a.elapsed_time(b_))
     torch.cuda.synchronize()
+    total_ms = max_over_ranks(total_ms, device)
     if world > 1:
-        t = torch.tensor([total_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
         torch.distributed.barrier()
     assert moba.device_status() == 0
     assert torch.isfinite(out_t.float()).all().item(), "non-finite output"
     ms = total_ms / args.steps
-    tflops_total = flops * world / (ms * 1e-3) / 1e12
-    tokens = w.batch * w.seqlen * world / (ms * 1e-3)
+    tflops_total = weak_scaling_rate(flops, world, ms) / 1e12
+    tokens = weak_scaling_rate(w.batch * w.seqlen, world, ms)
 
     hbm, tc_peak, tc_sus, peak_kind = peaks()
     stage_ms = {n: sum(v) / len(v) for n, v in per_stage.items()}
     attn_ms = stage_ms["attention"]
     achieved = flops / (attn_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": tc_peak,
-                "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4), "traffic": None,
-                "kernel": "moba_attn_fwd (past-block pass + own-block pass)" if w.kind == "moba"
-                else "swa_attn_fwd", "peak_kind": f"bf16 dense burst, {peak_kind}"}
+                "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
+                "traffic": stored_traffic(w.name),
+                "kernel": ("moba_attn_fwd: past-block pass, own-block pass and merge "
+                           "(3 launches per query chunk)") if w.kind == "moba" else "swa_attn_fwd",
+                "peak_kind": f"bf16 dense burst, {peak_kind}"}
     extra = {}
     if w.kind == "moba":
         sel_ms = stage_ms["pool"] + stage_ms["select"]
@@ -291,11 +337,7 @@ def run_ours(args, rank, world, device):
         torch.cuda.synchronize()
         if it >= args.warmup:
             e2e_ms += e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_ms /= args.steps
+    e2e_ms = max_over_ranks(e2e_ms, device) / args.steps
     h2d = (qh.numel() + kh.numel() + vh.numel()) * 2
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
     e2e = {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,

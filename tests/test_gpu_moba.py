@@ -93,8 +93,10 @@ def test_moba_strided_inputs():
     assert torch.equal(out, out2) and torch.equal(lse, lse2)
 
 
-@pytest.mark.parametrize("name", ["gqa32k", "hybrid64k"])
+@pytest.mark.parametrize("name", ["gqa32k", "hybrid64k", "moba1m"])
 def test_moba_full_size_sampled_rows(name):
+    """The full-size workloads in the launch configuration the benchmark times
+    (moba1m: 1M tokens, 25 query chunks of partials), checked on sampled rows."""
     w = workloads.WORKLOADS[name]
     rows = workloads.sampled_rows(w, seed=0)
     stats, _ = run_and_check(w, rows=rows)
