@@ -149,59 +149,139 @@ def physical_gpu(local: int) -> str:
     return vis[local] if local < len(vis) else str(local)
 
 
+_REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+            ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
+
+
 class ClockSampler:
-    def __init__(self, gpu_index: str):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    """Samples the SM clock, its maximum and the active clock-event reasons of one GPU
+    while the timed region runs.  NVML (the library nvidia-smi reads) is polled every
+    few milliseconds from a thread, so that even a timed region of tens of
+    milliseconds is covered; `mark_start()` / `mark_stop()` bracket the region and
+    only samples inside it are summarised.  Without NVML it falls back to nvidia-smi
+    at its shortest period.  Read-only: nothing about the GPU is changed."""
+
+    def __init__(self, device: int, period_s: float = 0.002):
+        self.device = device
+        self.period = period_s
+        self.samples = []          # (t, sm_mhz, max_mhz, reasons bitmask, power_w)
+        self.t0 = self.t1 = None
+        self._stop = False
+        self._thread = None
+        self._smi = None
+        self._path = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device)
+        try:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId_v2(bus.encode())
+        except Exception:
+            pass
+        try:
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + str(props.uuid)).encode())
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(int(physical_gpu(self.device)))
+
+    def _poll(self, nv, h):
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self._stop:
+            try:
+                self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                     mx, int(get_reasons(h)), nv.nvmlDeviceGetPowerUsage(h) / 1000.0))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def __enter__(self):
         try:
+            import threading
+            nv, h = self._nvml_handle()
+            self._thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self._thread.start()
+            deadline = time.perf_counter() + 2.0
+            while not self.samples and time.perf_counter() < deadline:
+                time.sleep(0.001)
+        except Exception:
+            self._thread = None
+            self._start_smi()
+        return self
+
+    def _start_smi(self):
+        try:
             import tempfile
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            fd, self._path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.gpu,
+            self._smi = subprocess.Popen(
+                ["nvidia-smi", "-i", physical_gpu(self.device),
                  "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=open(self._path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(1.0)
         except Exception:
-            self.proc = None
-        return self
+            self._smi = None
+
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_stop(self):
+        self.t1 = time.perf_counter()
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+        self._stop = True
+        if self._thread is not None:
+            self._thread.join(timeout=2)
+        if self._smi is not None:
+            self._smi.terminate()
             try:
-                self.proc.wait(timeout=5)
+                self._smi.wait(timeout=5)
             except Exception:
-                self.proc.kill()
+                self._smi.kill()
 
-    def summary(self):
-        if self.proc is None or not self.path or not os.path.exists(self.path):
-            return None
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
+    def _smi_samples(self):
+        out = []
+        if not self._path or not os.path.exists(self._path):
+            return out
+        names = [n for n, _ in _REASONS[:4]]
+        with open(self._path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
                 if len(parts) < 8:
                     continue
                 try:
-                    sm.append(float(parts[0]))
-                    mx = float(parts[1])
+                    sm, mx = float(parts[0]), float(parts[1])
                 except ValueError:
                     continue
-                for n, v in zip(names, parts[4:8]):
+                mask = 0
+                for (n, bit), v in zip(_REASONS[:4], parts[4:8]):
                     if v.lower().startswith("active"):
-                        reasons.add(n)
-        os.unlink(self.path)
-        if not sm:
+                        mask |= bit
+                out.append((None, sm, mx, mask, None))
+        os.unlink(self._path)
+        return out
+
+    def summary(self):
+        if self._thread is not None:
+            inside = [x for x in self.samples
+                      if self.t0 is not None and self.t1 is not None and self.t0 <= x[0] <= self.t1]
+            source = "nvml"
+        else:
+            inside = self._smi_samples()
+            source = "nvidia-smi"
+        if not inside:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = sorted({n for x in inside for n, bit in _REASONS if x[3] & bit})
+        pw = [x[4] for x in inside if x[4] is not None]
+        return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": inside[0][2],
+                "sm_mhz_min": min(x[1] for x in inside), "reasons": reasons,
+                "power_w_median": round(statistics.median(pw), 1) if pw else None,
+                "samples": len(inside), "source": source}
 
 
 # ------------------------------------------------------------------- our arm
@@ -279,7 +359,8 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize()
     per_stage = {}
     total_ms = 0.0
-    with ClockSampler(physical_gpu(torch.cuda.current_device())) as clk:
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        clk.mark_start()
         for _ in range(args.steps):
             flush.zero_()
             evs, names = step_timed()
@@ -287,6 +368,7 @@ def run_ours(args, rank, world, device):
             total_ms += evs[0].elapsed_time(evs[-1])
             for a, b_, n in zip(evs[:-1], evs[1:], names):
                 per_stage.setdefault(n, []).append(a.elapsed_time(b_))
+        clk.mark_stop()
     torch.cuda.synchronize()
     total_ms = max_over_ranks(total_ms, device)
     if world > 1:
