@@ -116,6 +116,36 @@ int make_attn_maps(CUtensorMap *maps, const moba_tensor &q, const moba_tensor &k
   return MOBA_OK;
 }
 
+// 2-D maps over q viewed as rows ((b * hq + h) * N + i) of d columns, one row high, for
+// the TMA gather of the gathered pass: a 64-column box (128-byte swizzle) and, for d = 80,
+// a 16-column tail box (32-byte swizzle).  Returns false when q's strides give no such
+// uniform row view or the row count does not fit the gather's int32 coordinates.
+bool make_gather_maps(CUtensorMap *maps, const moba_tensor &q, int batch, int hq, int N, int d) {
+  const long long rows = (long long)batch * hq * N;
+  if (rows >= (1ll << 31)) return false;
+  if (hq > 1 && q.sh != (int64_t)N * q.sn) return false;
+  if (batch > 1 && q.sb != (int64_t)hq * N * q.sn) return false;
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)q.sn * 2};
+  cuuint32_t estr[2] = {1u, 1u};
+  cuuint32_t box0[2] = {64u, 1u};
+  if (enc(&maps[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q.ptr, dims, strides, box0, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  maps[1] = maps[0];
+  if (d == 80) {
+    cuuint32_t box1[2] = {16u, 1u};
+    if (enc(&maps[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q.ptr, dims, strides, box1, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  return true;
+}
+
 int launch_status(cudaError_t e) { return e == cudaSuccess ? MOBA_OK : MOBA_ERR_LAUNCH; }
 
 // Device address of the status words on the current device.
@@ -218,6 +248,10 @@ int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *id
   if ((rc = check_device(&nsm))) return rc;
   CUtensorMap maps[6];
   if ((rc = make_attn_maps(maps, q, k, v, batch, hq, hkv, N, d))) return rc;
+  // The gathered pass reads q through 2-D row maps in place of the 4-D tile maps.
+  CUtensorMap gmaps[6];
+  for (int a = 0; a < 6; ++a) gmaps[a] = maps[a];
+  const int q_gather_tma = make_gather_maps(gmaps, q, batch, hq, N, d) ? 1 : 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char *ws = static_cast<char *>(workspace);
   AttnParams p{};
@@ -249,7 +283,9 @@ int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *id
     p.row_end = (c + 1) * w.chunk_rows < N ? (c + 1) * w.chunk_rows : N;
     if (w.npast > 0) {
       p.ntiles = 0;  // read from the workspace by the kernel
-      if ((rc = launch_status(launch_attn(maps, p, kGathered, nsm, st)))) return rc;
+      p.q_gather_tma = q_gather_tma;
+      if ((rc = launch_status(launch_attn(gmaps, p, kGathered, nsm, st)))) return rc;
+      p.q_gather_tma = 0;
     }
     p.ntiles = query_major_units(batch, hq, hkv, block, 1, p.row_begin, p.row_end);
     const int grid = p.ntiles < nsm ? p.ntiles : nsm;

@@ -23,7 +23,8 @@
 //   warp 0       TMA producers: lane 0 the query tiles (query-major) and K chunks of 128
 //                keys, lane 1 the V chunks (separate K and V rings)
 //   warp 1       tcgen05 MMA issuer (one thread) and TMEM owner
-//   warps 2-3    query-row gather with cp.async (gathered work)
+//   warps 2-3    query-row gather (gathered work): TMA gather4 of four rows per
+//                instruction, or cp.async when q's strides admit no 2-D row view
 //   warps 4-7    stream A softmax + epilogue; thread r owns row r (TMEM lane r)
 //   warps 8-11   stream B softmax + epilogue
 // TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).  P (bf16) overwrites
@@ -251,7 +252,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (tid == 0) {
     for (int x = 0; x < 2; ++x) {
-      mbar_init(&bar.q_full[x], MODE == kGathered ? 32 : 1);
+      mbar_init(&bar.q_full[x], (MODE == kGathered && !p.q_gather_tma) ? 32 : 1);
       mbar_init(&bar.q_empty[x], 1);
       mbar_init(&bar.s_full[x], 1);
       mbar_init(&bar.p_full[x], 128);
@@ -270,7 +271,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    if (MODE == kQueryMajor) tma_prefetch_desc(&tmQ);
+    if (MODE == kQueryMajor || p.q_gather_tma) tma_prefetch_desc(&tmQ);
   }
   if (warp == 1) {
     tmem_alloc(&bar.tmem_base, 512);
@@ -330,6 +331,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (uint32_t u = (cnt > (uint32_t)C::ST ? cnt - C::ST : 0); u < cnt; ++u) {
             const unsigned long long t0 = global_timer_ns();
             while (!mbar_try_wait(&full[u % C::ST], (u / C::ST) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+          }
+          for (int x = 0; x < 2; ++x) {
+            if (quse[x] == 0) continue;
+            const unsigned long long t0 = global_timer_ns();
+            while (!mbar_try_wait(&bar.q_full[x], (quse[x] - 1) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
           }
         }
       }
@@ -410,55 +416,107 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     } else if (MODE == kGathered) {
       // -------------------------------------------------------- row gather
-      // Warp 2 fills stream A's query tile, warp 3 stream B's: lane l owns rows l,
-      // l + 32, l + 64, l + 96; it reads their list entries first, then issues all of
-      // their 16-byte copies.
+      // Warp 2 fills stream A's query tile, warp 3 stream B's.
       const int x = warp - 2;
-      const int l = lane;
-      constexpr int VPR = D / 8;  // 16-byte vectors per row
       const int npast = p.npast;
+      const uint32_t qt = base + C::Q_OFF + x * C::TILE;
       uint32_t quse = 0;
       bool ok = true;
-      for (UnitIter<MODE> it(p, u_begin, u_end); ok && it.valid(); it.next()) {
-        Unit w;
-        it.get(p, w);
-        const Tile &t = w.t[x];
-        if (t.rows == 0) continue;
-        uint32_t ent[4];
+      if (p.q_gather_tma) {
+        // TMA gather4: lane l owns tile rows 4l .. 4l+3 and fetches them, 64 columns
+        // (and the 16-column tail for D = 80) per instruction, into the swizzled tile
+        // layout; rows past the unit's end repeat a valid row and are never stored.
+        // While a unit's copies are in flight the warp decodes the next unit's rows.
+        auto rows_of = [&](const Tile &t, int (&rr)[4]) {
 #pragma unroll
-        for (int k2 = 0; k2 < 4; ++k2)
-          ent[k2] = (l + 32 * k2 < t.rows) ? __ldg(p.entries + t.ent0 + l + 32 * k2) : 0u;
-        if (!(ok = mbar_wait(&bar.q_empty[x], (quse & 1) ^ 1, abort, p.status, site0 + 11))) break;
-        ++quse;
-        const uint32_t qt = base + C::Q_OFF + x * C::TILE;
-#pragma unroll
-        for (int k2 = 0; k2 < 4; ++k2) {
-          const int r = l + 32 * k2;
-          const bool valid = r < t.rows;
-          const uint16_t *row = p.q;
-          if (valid) {
-            const uint32_t ig = ent[k2] / (uint32_t)npast;
+          for (int e = 0; e < 4; ++e) {
+            const int r = 4 * lane + e;
+            const uint32_t ent = __ldg(p.entries + t.ent0 + (r < t.rows ? r : 0));
+            const uint32_t ig = ent / (uint32_t)npast;
             const int g = (int)(ig % (uint32_t)p.G);
             const int i = (int)(ig / (uint32_t)p.G);
-            row = p.q + t.b * p.q_sb + (int64_t)(t.hk * p.G + g) * p.q_sh + (int64_t)i * p.q_sn;
+            rr[e] = ((t.b * p.hq + t.hk * p.G + g) * p.N) + i;
           }
-#pragma unroll
-          for (int c = 0; c < VPR; ++c) {
-            uint32_t dst;
-            if (c < 8) {
-              dst = qt + r * 128 + ((c ^ (r & 7)) << 4);
-            } else if (D == 128) {
-              dst = qt + C::R0 + r * 128 + (((c - 8) ^ (r & 7)) << 4);
-            } else {
-              dst = qt + C::R0 + r * 32 + (((c - 8) ^ ((r >> 2) & 1)) << 4);
+        };
+        int u = u_begin + (int)blockIdx.x;
+        int rr[4];
+        Unit w;
+        w.t[x].rows = 0;
+        if (u < u_end) {
+          gathered_unit(p, __ldg(p.tiles + u), w);
+          if (w.t[x].rows > 0) rows_of(w.t[x], rr);
+        }
+        for (; ok && u < u_end; u += gridDim.x) {
+          if (w.t[x].rows > 0) {
+            if (!(ok = mbar_wait(&bar.q_empty[x], (quse & 1) ^ 1, abort, p.status, site0 + 11))) break;
+            ++quse;
+            if (lane == 0) mbar_arrive_expect_tx(&bar.q_full[x], C::BYTES);
+            __syncwarp();
+            tma_gather4_2d(qt + lane * 512, &tmQ, &bar.q_full[x], 0, rr[0], rr[1], rr[2], rr[3]);
+            if (D == 128)
+              tma_gather4_2d(qt + C::R0 + lane * 512, &tmQ, &bar.q_full[x], 64, rr[0], rr[1], rr[2], rr[3]);
+            if (D == 80)
+              tma_gather4_2d(qt + C::R0 + lane * 128, &tmQ1, &bar.q_full[x], 64, rr[0], rr[1], rr[2], rr[3]);
+          }
+          const int un = u + (int)gridDim.x;
+          w.t[x].rows = 0;
+          if (un < u_end) {
+            gathered_unit(p, __ldg(p.tiles + un), w);
+            if (w.t[x].rows > 0) {
+              rows_of(w.t[x], rr);
             }
-            cp_async_16_zfill(dst, valid ? row + c * 8 : p.q, valid);
           }
         }
-        cp_async_commit();
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        mbar_arrive(&bar.q_full[x]);
+        // After an abort, let the last gather land before the CTA can retire.
+        if (*abort && quse > 0) {
+          const unsigned long long t0 = global_timer_ns();
+          while (!mbar_try_wait(&bar.q_full[x], (quse - 1) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+        }
+      } else {
+        // cp.async: lane l owns rows l, l + 32, l + 64, l + 96; it reads their list
+        // entries first, then issues all of their 16-byte copies.
+        const int l = lane;
+        constexpr int VPR = D / 8;  // 16-byte vectors per row
+        for (UnitIter<MODE> it(p, u_begin, u_end); ok && it.valid(); it.next()) {
+          Unit w;
+          it.get(p, w);
+          const Tile &t = w.t[x];
+          if (t.rows == 0) continue;
+          uint32_t ent[4];
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2)
+            ent[k2] = (l + 32 * k2 < t.rows) ? __ldg(p.entries + t.ent0 + l + 32 * k2) : 0u;
+          if (!(ok = mbar_wait(&bar.q_empty[x], (quse & 1) ^ 1, abort, p.status, site0 + 11))) break;
+          ++quse;
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) {
+            const int r = l + 32 * k2;
+            const bool valid = r < t.rows;
+            const uint16_t *row = p.q;
+            if (valid) {
+              const uint32_t ig = ent[k2] / (uint32_t)npast;
+              const int g = (int)(ig % (uint32_t)p.G);
+              const int i = (int)(ig / (uint32_t)p.G);
+              row = p.q + t.b * p.q_sb + (int64_t)(t.hk * p.G + g) * p.q_sh + (int64_t)i * p.q_sn;
+            }
+#pragma unroll
+            for (int c = 0; c < VPR; ++c) {
+              uint32_t dst;
+              if (c < 8) {
+                dst = qt + r * 128 + ((c ^ (r & 7)) << 4);
+              } else if (D == 128) {
+                dst = qt + C::R0 + r * 128 + (((c - 8) ^ (r & 7)) << 4);
+              } else {
+                dst = qt + C::R0 + r * 32 + (((c - 8) ^ ((r >> 2) & 1)) << 4);
+              }
+              cp_async_16_zfill(dst, valid ? row + c * 8 : p.q, valid);
+            }
+          }
+          cp_async_commit();
+          cp_async_wait_all();
+          fence_proxy_async_smem();
+          mbar_arrive(&bar.q_full[x]);
+        }
       }
     }
   } else {

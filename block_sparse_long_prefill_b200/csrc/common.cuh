@@ -103,6 +103,18 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, u
       : "memory");
 }
 
+// Four rows (r0..r3) of a 2-D tensor map whose box is one row high, columns from c0:
+// written to consecutive box rows at dst (swizzled by the map's mode).
+__device__ __forceinline__ void tma_gather4_2d(uint32_t dst, const CUtensorMap *map, uint64_t *bar,
+                                               int c0, int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1),
+      "r"(r2), "r"(r3)
+      : "memory");
+}
+
 // Prefetch [src, src + bytes) of global memory into L2 (bytes a multiple of 16).
 __device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");

@@ -108,6 +108,10 @@ struct AttnParams {
   int batch, hq, hkv, N, d, block, topk, window, G;
   float scale_log2;        // scale * log2(e)
   int is_moba;             // 0: sliding window only (swa_attn_fwd)
+  // Gathered pass: 1 when the query rows are fetched by TMA gather4 through a 2-D map
+  // over q (row ((b * hq + h) * N + i)); 0 when by cp.async (q's strides admit no
+  // single row stride, or the row count exceeds int32).
+  int q_gather_tma;
   // Query-major pass: row range of this pass.
   int row_begin, row_end;  // multiples of 128 except row_end == N
   int ntiles;              // query-major work units in this pass
