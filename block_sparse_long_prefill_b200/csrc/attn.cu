@@ -75,6 +75,7 @@ struct Bars {
   uint64_t q_full[2], q_empty[2];                          // per stream
   uint64_t k_full[3], v_full[3], k_empty[3], v_empty[3];
   uint64_t s_full[2], p_full[2], o_full[2];                // per stream
+  uint64_t turn[2][4];   // exponential-phase token of stream x, per sub-partition pair
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
@@ -264,6 +265,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(&bar.k_empty[s], 1);
       mbar_init(&bar.v_empty[s], 1);
     }
+    for (int x = 0; x < 2; ++x)
+      for (int q = 0; q < 4; ++q) mbar_init(&bar.turn[x][q], 1);
     mbar_init(&bar.mma_done, 1);
     bar.abort = 0;
     fence_barrier_init();
@@ -303,7 +306,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           Unit w;
           it.get(p, w);
           if (MODE == kQueryMajor && kside) {
-            for (int x = 0; x < 2 && ok; ++x) {
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              if (!ok) break;
               const Tile &t = w.t[x];
               if (t.rows == 0) continue;
               ok = mbar_wait(&bar.q_empty[x], (quse[x] & 1) ^ 1, abort, p.status, site0 + 1);
@@ -353,8 +358,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           Unit w;
           it.get(p, w);
           const bool act[2] = {w.t[0].rows > 0, w.t[1].rows > 0};
-          for (int x = 0; x < 2 && ok; ++x) {
-            if (!act[x]) continue;
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            if (!act[x] || !ok) continue;
             ok = mbar_wait(&bar.q_full[x], quse[x] & 1, abort, p.status, site0 + 3);
             ++quse[x];
           }
@@ -371,8 +377,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (m > 0) {
               if (!(ok = mbar_wait(&bar.v_full[st_p], (slot_p / C::ST) & 1, abort, p.status, site0 + 6))) break;
             }
+#pragma unroll
             for (int x = 0; x < 2; ++x) {
-              if (!act[x]) continue;
+              if (!act[x] || !ok) continue;
               const uint32_t sb = tmem + 128 * x;
               const uint32_t tO = tmem + 256 + 128 * x;
               if (m > 0) {
@@ -441,13 +448,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         int u = u_begin + (int)blockIdx.x;
         int rr[4];
         Unit w;
-        w.t[x].rows = 0;
+        Tile tx;
+        tx.rows = 0;
         if (u < u_end) {
           gathered_unit(p, __ldg(p.tiles + u), w);
-          if (w.t[x].rows > 0) rows_of(w.t[x], rr);
+          tx = x ? w.t[1] : w.t[0];
+          if (tx.rows > 0) rows_of(tx, rr);
         }
         for (; ok && u < u_end; u += gridDim.x) {
-          if (w.t[x].rows > 0) {
+          if (tx.rows > 0) {
             if (!(ok = mbar_wait(&bar.q_empty[x], (quse & 1) ^ 1, abort, p.status, site0 + 11))) break;
             ++quse;
             if (lane == 0) mbar_arrive_expect_tx(&bar.q_full[x], C::BYTES);
@@ -459,12 +468,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               tma_gather4_2d(qt + C::R0 + lane * 128, &tmQ1, &bar.q_full[x], 64, rr[0], rr[1], rr[2], rr[3]);
           }
           const int un = u + (int)gridDim.x;
-          w.t[x].rows = 0;
+          tx.rows = 0;
           if (un < u_end) {
             gathered_unit(p, __ldg(p.tiles + un), w);
-            if (w.t[x].rows > 0) {
-              rows_of(w.t[x], rr);
-            }
+            tx = x ? w.t[1] : w.t[0];
+            if (tx.rows > 0) rows_of(tx, rr);
           }
         }
         // After an abort, let the last gather land before the CTA can retire.
@@ -480,7 +488,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (UnitIter<MODE> it(p, u_begin, u_end); ok && it.valid(); it.next()) {
           Unit w;
           it.get(p, w);
-          const Tile &t = w.t[x];
+          const Tile t = x ? w.t[1] : w.t[0];
           if (t.rows == 0) continue;
           uint32_t ent[4];
 #pragma unroll
@@ -531,12 +539,32 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t tO = tmem + lane_off + 256 + 128 * x;
     const float sl2 = p.scale_log2;
     uint32_t scnt = 0, ocnt = 0;
+    // Ping-pong of the exponential phases: the softmax warps of streams A and B that
+    // share a sub-partition (warps w and w + 4) take turns, so that one stream's
+    // exponentials run while the tensor core works on the other stream's MMAs instead
+    // of both streams contending for the same exponential units at once.  Stream x
+    // waits on turn[x][q] before its exponentials and passes turn[x ^ 1][q] after them;
+    // stream B hands stream A the first turn.  Both streams take one turn per chunk of
+    // every unit (an idle stream passes its turns on at once), so the turns stay paired.
+    const int q4 = warp & 3;
+    uint64_t *my_turn = &bar.turn[x][q4];
+    uint64_t *other_turn = &bar.turn[x ^ 1][q4];
+    uint32_t tcnt = 0;
+    if (x == 1 && lane == 0) mbar_arrive(other_turn);
     bool ok = true;
     for (UnitIter<MODE> it(p, u_begin, u_end); ok && it.valid(); it.next()) {
       Unit w;
       it.get(p, w);
-      const Tile &t = w.t[x];
-      if (t.rows == 0) continue;
+      const Tile t = x ? w.t[1] : w.t[0];   // (a select: w stays in registers)
+      if (t.rows == 0) {
+        for (int m = 0; m < w.nc && ok; ++m, ++tcnt) {
+          ok = mbar_wait(my_turn, tcnt & 1, abort, p.status, site0 + 15);
+          ok = __all_sync(FULL, ok);
+          __syncwarp();
+          if (ok && lane == 0) mbar_arrive(other_turn);
+        }
+        continue;
+      }
       const bool live = r < t.rows;
       // Row identity.
       int i = t.i0 + r, h = t.h, slot = 0;
@@ -624,6 +652,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tmem_st16(tO + c0, o);
           }
         }
+        ok = mbar_wait(my_turn, tcnt & 1, abort, p.status, site0 + 15);
+        ++tcnt;
+        if (!(ok = __all_sync(FULL, ok))) break;
         const float mu = (m_run == -INFINITY) ? 0.f : m_run;
         float ls[8];
 #pragma unroll
@@ -636,6 +667,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           ls[e & 7] += p0 + p1;
           sv[e] = pack_bf16x2(p0, p1);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(other_turn);
         tmem_st16(tS, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
         tmem_st16(tS + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
         tmem_st16(tS + 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[32]));
