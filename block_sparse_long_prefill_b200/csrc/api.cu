@@ -22,6 +22,8 @@ cudaError_t launch_gate(const SelectParams &p, cudaStream_t st);
 cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileoff, int4 *tiles,
                         int nlists, cudaStream_t st);
 cudaError_t launch_scatter(const ScatterParams &p, cudaStream_t st);
+cudaError_t launch_gate_tc(const CUtensorMap *maps, const GateParams &p, int grid, cudaStream_t st);
+int gate_tc_rows_staged();
 cudaError_t launch_attn(const CUtensorMap *maps, const AttnParams &p, int mode, int grid,
                         cudaStream_t st);
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t st);
@@ -146,6 +148,34 @@ bool make_gather_maps(CUtensorMap *maps, const moba_tensor &q, int batch, int hq
   return true;
 }
 
+// 3-D maps over the pooled-key split [batch, hkv, 2, nblk, d] viewed as planes
+// (b * hkv + hk) * 2 + part of nblk rows: a 64-column box of `rows` rows (128-byte
+// swizzle) and, for d = 80, a 16-column tail box (32-byte swizzle).  Rows past nblk
+// read as zero.
+int make_kbar_maps(CUtensorMap *maps, const void *split, int batch, int hkv, int nblk, int d,
+                   int rows) {
+  auto enc = get_encode();
+  if (!enc) return MOBA_ERR_LAUNCH;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)nblk, (cuuint64_t)batch * hkv * 2};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)nblk * d * 2};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  cuuint32_t box0[3] = {64u, (cuuint32_t)rows, 1u};
+  void *ptr = const_cast<void *>(split);
+  if (enc(&maps[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box0, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return MOBA_ERR_LAUNCH;
+  maps[1] = maps[0];
+  if (d == 80) {
+    cuuint32_t box1[3] = {16u, (cuuint32_t)rows, 1u};
+    if (enc(&maps[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box1, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MOBA_ERR_LAUNCH;
+  }
+  return MOBA_OK;
+}
+
 int launch_status(cudaError_t e) { return e == cudaSuccess ? MOBA_OK : MOBA_ERR_LAUNCH; }
 
 // Device address of the status words on the current device.
@@ -204,15 +234,39 @@ int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, i
   int *counts = reinterpret_cast<int *>(ws + w.off_counts);
   if (cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)w.nlists, st) != cudaSuccess)
     return MOBA_ERR_LAUNCH;
-  SelectParams sp{};
-  sp.q = static_cast<const uint16_t *>(q.ptr);
-  sp.q_sb = q.sb; sp.q_sh = q.sh; sp.q_sn = q.sn;
-  sp.kbar_split = static_cast<const uint16_t *>(kbar_split);
-  sp.idx = idx;
-  sp.counts = counts;
-  sp.batch = batch; sp.hq = hq; sp.hkv = hkv; sp.N = N; sp.d = d; sp.block = block;
-  sp.topk = topk; sp.nblk = w.nblk; sp.G = w.G; sp.chunk_rows = w.chunk_rows;
-  if ((rc = launch_status(launch_gate(sp, st)))) return rc;
+  if (w.nblk <= gate_tc_rows_staged()) {
+    // Tensor-core gate: q tiles and the pooled keys through TMA.
+    int nsm = 0;
+    if ((rc = check_device(&nsm))) return rc;
+    CUtensorMap maps[4];
+    if ((rc = make_map(&maps[0], q, batch, hq, N, d, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+    if (d == 80) {
+      if ((rc = make_map(&maps[1], q, batch, hq, N, d, 16, CU_TENSOR_MAP_SWIZZLE_32B))) return rc;
+    } else {
+      maps[1] = maps[0];
+    }
+    const int rows = (w.nblk + 15) & ~15;
+    if ((rc = make_kbar_maps(&maps[2], kbar_split, batch, hkv, w.nblk, d, rows))) return rc;
+    GateParams gp{};
+    if ((rc = status_words(&gp.status))) return rc;
+    gp.idx = idx;
+    gp.counts = counts;
+    gp.batch = batch; gp.hq = hq; gp.hkv = hkv; gp.N = N; gp.d = d; gp.block = block;
+    gp.topk = topk; gp.nblk = w.nblk; gp.G = w.G; gp.chunk_rows = w.chunk_rows;
+    const long long tiles = (long long)batch * hkv * (N / kTileRows) * w.G;
+    const int grid = (int)(tiles < nsm ? tiles : nsm);
+    if ((rc = launch_status(launch_gate_tc(maps, gp, grid, st)))) return rc;
+  } else {
+    SelectParams sp{};
+    sp.q = static_cast<const uint16_t *>(q.ptr);
+    sp.q_sb = q.sb; sp.q_sh = q.sh; sp.q_sn = q.sn;
+    sp.kbar_split = static_cast<const uint16_t *>(kbar_split);
+    sp.idx = idx;
+    sp.counts = counts;
+    sp.batch = batch; sp.hq = hq; sp.hkv = hkv; sp.N = N; sp.d = d; sp.block = block;
+    sp.topk = topk; sp.nblk = w.nblk; sp.G = w.G; sp.chunk_rows = w.chunk_rows;
+    if ((rc = launch_status(launch_gate(sp, st)))) return rc;
+  }
   if (w.npast == 0) return MOBA_OK;
   int *cursor = reinterpret_cast<int *>(ws + w.off_cursor);
   int *listoff = reinterpret_cast<int *>(ws + w.off_listoff);

@@ -1,0 +1,413 @@
+// gate.cu -- MoBA gate scores and top-k on the sm_100a tensor cores (tcgen05 + TMA).
+//
+// [MoBA] = "MoBA: 어텐션에 전문가 혼합을 적용해 긴 문맥을 효율적으로 처리하는 블록 어텐션
+//          (feat. MoonshotAI)", PyTorch KR forum summary of the MoBA paper.
+//
+// §"블록 분할과 top-k 게이팅": the gate score of query i for block j is the unscaled
+// inner product s_j = <q_i, MeanPool(K[I_j])>; each query keeps the k blocks with the
+// highest scores.  §"인과성 보존": only blocks wholly before the query's own block
+// c = i / block compete (j < c), block c is always kept, later blocks never.
+//
+// One persistent CTA per SM walks a contiguous range of 128-row query tiles ordered
+// (batch, kv-head, row tile, q-head), so that the pooled keys of one kv-head are staged
+// in shared memory once per range.  Since block % 128 == 0, every row of a tile has the
+// same own block c, and the tile needs the scores of blocks [0, c) only.
+//   warp 0     TMA producer: query tiles (a ring of up to eight) and, per kv-head, the
+//              pooled keys kbar = hi + lo (two bf16 matrices of up to 256 rows)
+//   warp 1     tcgen05 MMA issuer and TMEM owner: S = Q hi^T + Q lo^T in fp32, into
+//              one of two TMEM accumulators (N = c rounded up to 16 columns)
+//   warps 2-5  top-k: thread r owns row r (TMEM lane r) and scans its c scores in
+//              ascending block order, keeping the best k-1 in registers (a strictly
+//              greater score displaces; ties keep the lower block), then writes the
+//              row's choices in ascending order, the own block, and -1 padding; it
+//              also counts the picks per past block for the dispatch lists.
+// q is exactly bf16 and kbar = hi + lo to about 2^-17 relative, so the fp32 scores
+// match an fp32 inner product with the pooled keys far inside the ranking tolerance.
+#include <cuda.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "params.h"
+
+namespace moba {
+
+constexpr int kGateTcThreads = 192;
+constexpr int kGateMaxBlocks = 256;   // pooled keys staged at once (MMA N <= 256)
+
+constexpr int kGateMaxStages = 8;     // query tile ring depth limit
+constexpr int kGateSmemLimit = 227 * 1024;
+
+// Shared memory: a ring of qst query tiles, the pooled keys hi and lo (kc16 rows each),
+// four per-warp pick histograms, barriers.  qst is chosen on the host to fill the
+// shared memory the staged pooled keys leave.
+template <int D>
+struct GateCfg {
+  static constexpr int QR0 = 128 * 128;                                // query region 0 bytes
+  static constexpr int QR1 = (D == 128) ? 128 * 128 : (D == 80 ? 128 * 32 : 0);
+  static constexpr int QTILE = QR0 + ((QR1 + 1023) / 1024) * 1024;
+  static constexpr uint32_t QBYTES = 128u * D * 2u;
+  static constexpr int R1ROW = (D == 128) ? 128 : (D == 80 ? 32 : 0);  // region 1 bytes per row
+  __host__ __device__ static constexpr int kmat(int kc16) {           // one of hi / lo
+    return kc16 * 128 + ((kc16 * R1ROW + 1023) / 1024) * 1024;
+  }
+  __host__ __device__ static constexpr int k_off(int qst) { return qst * QTILE; }
+  __host__ __device__ static constexpr int hist_off(int qst, int kc16) { return k_off(qst) + 2 * kmat(kc16); }
+  __host__ __device__ static constexpr int bar_off(int qst, int kc16) {
+    return hist_off(qst, kc16) + 4 * 4 * kGateMaxBlocks;
+  }
+  __host__ __device__ static constexpr int smem(int qst, int kc16) { return bar_off(qst, kc16) + 512 + 1024; }
+};
+
+struct GateBars {
+  uint64_t q_full[kGateMaxStages], q_empty[kGateMaxStages];
+  uint64_t k_full, k_empty;
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// K-major operand descriptor for k-step ks of a tile whose region 0 holds columns
+// [0, 64) of `rows` rows (128-byte rows, 128-byte swizzle) and whose region 1 holds
+// the remaining columns (D = 128: 64 more, same layout; D = 80: 16, 32-byte rows and
+// 32-byte swizzle).
+template <int D>
+__device__ __forceinline__ uint64_t gate_desc(uint32_t tile, int ks, int rows) {
+  if (ks < 4) return smem_desc(tile + ks * 32, 16, 1024, kSwizzle128);
+  if (D == 128) return smem_desc(tile + rows * 128 + (ks - 4) * 32, 16, 1024, kSwizzle128);
+  return smem_desc(tile + rows * 128, 16, 256, kSwizzle32);
+}
+
+// Tile t of the range -> (b, hk, row tile, g): rows [128 rt, 128 rt + 128) of q-head
+// hk * G + g.  Ordered so that consecutive tiles share the kv-head.
+struct GateTile {
+  int b, hk, g, rt;
+};
+__device__ __forceinline__ GateTile gate_tile(const GateParams &p, int t) {
+  GateTile r;
+  r.g = t % p.G;
+  t /= p.G;
+  const int nrt = p.N / 128;
+  r.rt = t % nrt;
+  t /= nrt;
+  r.hk = t % p.hkv;
+  r.b = t / p.hkv;
+  return r;
+}
+
+// Insertion of (v, j) into the descending list val / idx.  Entries past the npick in
+// use hold +inf and are never displaced, so the element carried past the last used
+// entry falls off; an entry is displaced only by a strictly greater score, so ties
+// keep the block that came first, the lower one.
+template <int KM>
+__device__ __forceinline__ void topk_insert(float (&val)[KM], int (&idx)[KM], float v, int j) {
+#pragma unroll
+  for (int e = 0; e < KM; ++e) {
+    const bool take = v > val[e];
+    const float tv = val[e];
+    const int tj = idx[e];
+    val[e] = take ? v : tv;
+    idx[e] = take ? j : tj;
+    v = take ? tv : v;
+    j = take ? tj : j;
+  }
+}
+
+template <int D, int KM>
+__global__ void __launch_bounds__(kGateTcThreads, 1)
+gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ1,
+               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK1,
+               const GateParams p) {
+  using C = GateCfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char *sbase = smem_raw + (base - raw);
+  // Pooled-key rows staged per kv-head: every past block of the last row tile.
+  const int kc16 = (min(p.nblk, kGateMaxBlocks) + 15) & ~15;
+  const int qst = p.qstages;
+  const int kmat = C::kmat(kc16);
+  const int k_off = C::k_off(qst);
+  GateBars &bar = *reinterpret_cast<GateBars *>(sbase + C::bar_off(qst, kc16));
+  int *hist = reinterpret_cast<int *>(sbase + C::hist_off(qst, kc16));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int site0 = (3 * 16 + (D == 64 ? 0 : (D == 80 ? 1 : 2))) * 256;
+  constexpr uint32_t FULL = 0xffffffffu;
+
+  // This CTA's contiguous tile range.
+  const int ntiles = p.batch * p.hkv * (p.N / 128) * p.G;
+  const int per = (ntiles + gridDim.x - 1) / gridDim.x;
+  const int t_begin = blockIdx.x * per;
+  const int t_end = min(ntiles, t_begin + per);
+
+  if (tid == 0) {
+    for (int s = 0; s < qst; ++s) {
+      mbar_init(&bar.q_full[s], 1);
+      mbar_init(&bar.q_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar.acc_full[s], 1);
+      mbar_init(&bar.acc_empty[s], 4);
+    }
+    mbar_init(&bar.k_full, 1);
+    mbar_init(&bar.k_empty, 1);
+    mbar_init(&bar.mma_done, 1);
+    bar.abort = 0;
+    fence_barrier_init();
+  }
+  for (int j = tid; j < 4 * kGateMaxBlocks; j += kGateTcThreads) hist[j] = 0;
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+  }
+  if (warp == 1) {
+    tmem_alloc(&bar.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+  volatile int *abort = &bar.abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      int cur = -1;
+      uint32_t kuse = 0, quse = 0;
+      for (int t = t_begin; ok && t < t_end; ++t) {
+        const GateTile gt = gate_tile(p, t);
+        const int grp = gt.b * p.hkv + gt.hk;
+        if (grp != cur) {
+          cur = grp;
+          if (!(ok = mbar_wait(&bar.k_empty, (kuse & 1) ^ 1, abort, p.status, site0 + 1))) break;
+          ++kuse;
+          const uint32_t kbytes = 2u * (uint32_t)kc16 * (uint32_t)D * 2u;
+          mbar_arrive_expect_tx(&bar.k_full, kbytes);
+          for (int part = 0; part < 2; ++part) {
+            unsigned char *kd = sbase + k_off + part * kmat;
+            const int plane = grp * 2 + part;
+            tma_load_3d(kd, &tmK, &bar.k_full, 0, 0, plane);
+            if (D != 64) tma_load_3d(kd + kc16 * 128, &tmK1, &bar.k_full, 64, 0, plane);
+          }
+        }
+        const int s = quse % qst;
+        if (!(ok = mbar_wait(&bar.q_empty[s], ((quse / qst) & 1) ^ 1, abort, p.status, site0 + 2))) break;
+        unsigned char *qd = sbase + s * C::QTILE;
+        const int h = gt.hk * p.G + gt.g;
+        mbar_arrive_expect_tx(&bar.q_full[s], C::QBYTES);
+        tma_load_4d(qd, &tmQ, &bar.q_full[s], 0, gt.rt * 128, h, gt.b);
+        if (D != 64) tma_load_4d(qd + C::QR0, &tmQ1, &bar.q_full[s], 64, gt.rt * 128, h, gt.b);
+        ++quse;
+      }
+      if (*abort) {
+        // Let issued loads land before the CTA can retire.
+        const unsigned long long t0 = global_timer_ns();
+        for (uint32_t u = (quse > (uint32_t)qst ? quse - qst : 0u); u < quse; ++u)
+          while (!mbar_try_wait(&bar.q_full[u % qst], (u / qst) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+        while (kuse > 0 && !mbar_try_wait(&bar.k_full, (kuse - 1) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      int cur = -1;
+      uint32_t kuse = 0, quse = 0, ause = 0;
+      for (int t = t_begin; ok && t < t_end; ++t) {
+        const GateTile gt = gate_tile(p, t);
+        const int grp = gt.b * p.hkv + gt.hk;
+        if (grp != cur) {
+          cur = grp;
+          if (!(ok = mbar_wait(&bar.k_full, kuse & 1, abort, p.status, site0 + 3))) break;
+          ++kuse;
+        }
+        const int s = quse % qst, a = ause & 1;
+        if (!(ok = mbar_wait(&bar.q_full[s], (quse / qst) & 1, abort, p.status, site0 + 4))) break;
+        if (!(ok = mbar_wait(&bar.acc_empty[a], ((ause >> 1) & 1) ^ 1, abort, p.status, site0 + 5))) break;
+        tc_fence_after();
+        const int c = (gt.rt * 128) / p.block;              // own block of every row
+        // Score columns needed (none when every past block is kept anyway).
+        const int nn = (c > p.topk - 1) ? min((c + 15) & ~15, kc16) : 0;
+        if (nn > 0) {
+          const uint32_t idesc = idesc_bf16(128, nn, 0, 0);
+          const uint32_t qt = base + s * C::QTILE;
+          const uint32_t acc = tmem + 256 * a;
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+            const uint32_t kt = base + k_off + part * kmat;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+              umma_ss(acc, gate_desc<D>(qt, ks, 128), gate_desc<D>(kt, ks, kc16), idesc,
+                      (part > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(&bar.acc_full[a]);
+        umma_commit(&bar.q_empty[s]);
+        // Last tile of this kv-head in the range: the pooled keys may be replaced.
+        const bool last = (t + 1 == t_end) || ([&] {
+          const GateTile nx = gate_tile(p, t + 1);
+          return nx.b * p.hkv + nx.hk != grp;
+        })();
+        if (last) umma_commit(&bar.k_empty);
+        ++quse;
+        ++ause;
+      }
+      umma_commit(&bar.mma_done);
+      const unsigned long long t0 = global_timer_ns();
+      while (!mbar_try_wait(&bar.mma_done, 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+    }
+  } else {
+    // ------------------------------------------------------------ top-k
+    // Each warp counts its rows' picks in its own shared histogram and adds it to the
+    // list counts when its rows move to another (chunk, batch, kv-head) list, so no
+    // barrier across warps is needed.
+    const int r = 32 * (warp & 3) + lane;                  // row within the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    int *whist = hist + (warp & 3) * kGateMaxBlocks;
+    const int npast = p.topk - 1;
+    bool ok = true;
+    uint32_t ause = 0;
+    int cur_list = -1;
+    auto flush = [&](int list) {
+      __syncwarp();
+      for (int j = lane; j < p.nblk; j += 32) {
+        const int v = whist[j];
+        if (v) {
+          atomicAdd(&p.counts[(int64_t)list * p.nblk + j], v);
+          whist[j] = 0;
+        }
+      }
+      __syncwarp();
+    };
+    for (int t = t_begin; ok && t < t_end; ++t) {
+      const GateTile gt = gate_tile(p, t);
+      const int i = gt.rt * 128 + r;
+      const int c = (gt.rt * 128) / p.block;
+      const int h = gt.hk * p.G + gt.g;
+      const int a = ause & 1;
+      const int list = ((gt.rt * 128) / p.chunk_rows * p.batch + gt.b) * p.hkv + gt.hk;
+      if (list != cur_list) {
+        if (cur_list >= 0) flush(cur_list);
+        cur_list = list;
+      }
+      ok = mbar_wait(&bar.acc_full[a], (ause >> 1) & 1, abort, p.status, site0 + 6);
+      if (!(ok = __all_sync(FULL, ok))) break;
+      tc_fence_after();
+      int32_t *orow = p.idx + (((int64_t)gt.b * p.hq + h) * p.N + i) * p.topk;
+      if (c <= npast || npast == 0) {
+        // Every past block is kept (or none is asked for): no scores needed.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.acc_empty[a]);
+        const int nk = min(c, npast);
+        for (int s = 0; s < p.topk; ++s) orow[s] = (s < nk) ? s : (s == nk ? c : -1);
+        if (lane == 0)
+          for (int j = 0; j < nk; ++j) whist[j] += 32;
+      } else {
+        const int npick = npast;                            // c > npast here
+        float val[KM];
+        int idx[KM];
+#pragma unroll
+        for (int e = 0; e < KM; ++e) {
+          val[e] = (e < npick) ? -INFINITY : INFINITY;
+          idx[e] = -1;
+        }
+        const uint32_t acc = tmem + lane_off + 256 * a;
+        float thr = -INFINITY;                              // val[npick - 1]
+        for (int j0 = 0; j0 < c; j0 += 32) {
+          uint32_t sc[32];
+          tmem_ld32(acc + j0, sc);
+          tmem_wait_ld();
+          if (KM <= 4) {
+            // Short lists: every score goes through the list, with no branch.
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              topk_insert<KM>(val, idx, (j0 + e < c) ? __uint_as_float(sc[e]) : -INFINITY, j0 + e);
+          } else {
+            // Long lists: only scores above the current k-1-th best go in.
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float v = __uint_as_float(sc[e]);
+              if (j0 + e < c && v > thr) {
+                topk_insert<KM>(val, idx, v, j0 + e);
+                thr = val[0];
+#pragma unroll
+                for (int f = 1; f < KM; ++f) thr = (f < npick) ? val[f] : thr;
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.acc_empty[a]);
+        // Ascending block order: each choice goes to its rank among the choices.
+#pragma unroll
+        for (int e = 0; e < KM; ++e) {
+          if (e < npick) {
+            int rank = 0;
+#pragma unroll
+            for (int f = 0; f < KM; ++f)
+              if (f < npick) rank += idx[f] < idx[e];
+            orow[rank] = idx[e];
+            atomicAdd(&whist[idx[e]], 1);
+          }
+        }
+        orow[npick] = c;
+        for (int s = npick + 1; s < p.topk; ++s) orow[s] = -1;
+      }
+      ++ause;
+    }
+    if (cur_list >= 0) flush(cur_list);
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int D, int KM>
+static cudaError_t launch_gate_tc_dk(const CUtensorMap *maps, GateParams p, int grid,
+                                     cudaStream_t st) {
+  using C = GateCfg<D>;
+  auto kern = gate_tc_kernel<D, KM>;
+  const int kc16 = (min(p.nblk, kGateMaxBlocks) + 15) & ~15;
+  // As many query stages as the shared memory left by the pooled keys holds.
+  int qst = kGateMaxStages;
+  while (qst > 2 && C::smem(qst, kc16) > kGateSmemLimit) --qst;
+  if (C::smem(qst, kc16) > kGateSmemLimit) return cudaErrorInvalidConfiguration;
+  p.qstages = qst;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem(qst, kc16));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kGateTcThreads, C::smem(qst, kc16), st>>>(maps[0], maps[1], maps[2], maps[3], p);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_gate_tc_d(const CUtensorMap *maps, const GateParams &p, int grid,
+                                    cudaStream_t st) {
+  const int npast = p.topk - 1;
+  if (npast <= 2) return launch_gate_tc_dk<D, 2>(maps, p, grid, st);
+  if (npast <= 4) return launch_gate_tc_dk<D, 4>(maps, p, grid, st);
+  if (npast <= 8) return launch_gate_tc_dk<D, 8>(maps, p, grid, st);
+  if (npast <= 16) return launch_gate_tc_dk<D, 16>(maps, p, grid, st);
+  return launch_gate_tc_dk<D, 32>(maps, p, grid, st);
+}
+
+// maps: Q (64-column box of 128 rows), Q tail, kbar planes (64-column box of
+// min(nblk, 256) rounded to 16 rows), kbar tail.
+cudaError_t launch_gate_tc(const CUtensorMap *maps, const GateParams &p, int grid, cudaStream_t st) {
+  switch (p.d) {
+    case 64: return launch_gate_tc_d<64>(maps, p, grid, st);
+    case 80: return launch_gate_tc_d<80>(maps, p, grid, st);
+    case 128: return launch_gate_tc_d<128>(maps, p, grid, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+int gate_tc_rows_staged() { return kGateMaxBlocks; }
+
+}  // namespace moba

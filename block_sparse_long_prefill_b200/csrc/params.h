@@ -82,6 +82,16 @@ struct SelectParams {
   int batch, hq, hkv, N, d, block, topk, nblk, G, chunk_rows;
 };
 
+// Parameters of the tensor-core gate / top-k kernel (q and the pooled keys arrive
+// through TMA maps).
+struct GateParams {
+  int *status;           // device status words
+  int32_t *idx;          // [batch, hq, N, topk]
+  int *counts;           // workspace list counts
+  int batch, hq, hkv, N, d, block, topk, nblk, G, chunk_rows;
+  int qstages;           // query tile ring depth (set by the launcher)
+};
+
 struct ScatterParams {
   const int32_t *idx;
   int *cursor;

@@ -93,6 +93,20 @@ def test_moba_strided_inputs():
     assert torch.equal(out, out2) and torch.equal(lse, lse2)
 
 
+@pytest.mark.parametrize("name,kw", [
+    # 512 blocks: more pooled keys than the tensor-core gate stages at once, so the
+    # selection takes the general (mma.sync) gate kernel.
+    ("many_blocks", dict(batch=1, hq=2, hkv=1, seqlen=65536, d=64, block=128, topk=4)),
+    # exactly the tensor-core gate's limit of 256 blocks, with d = 80 and GQA.
+    ("blocks256_d80", dict(batch=1, hq=4, hkv=2, seqlen=32768, d=80, block=128, topk=6)),
+])
+def test_moba_block_count_limits_sampled_rows(name, kw):
+    w = workloads.small_moba(name=name, **kw)
+    rows = workloads.sampled_rows(w, seed=2)
+    stats, _ = run_and_check(w, rows=rows)
+    print(name, stats)
+
+
 @pytest.mark.parametrize("name", ["gqa32k", "hybrid64k", "moba1m"])
 def test_moba_full_size_sampled_rows(name):
     """The full-size workloads in the launch configuration the benchmark times
