@@ -8,6 +8,7 @@
 // A streaming kernel: LPR = d/8 lanes cover one row with 16-byte vectors, so every
 // partial row (slots contiguous per row) and the output row move in coalesced
 // 16-byte accesses; the per-row weights are computed redundantly by those lanes.
+// Warps walk the rows grid-stride.
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
@@ -29,18 +30,15 @@ __device__ __forceinline__ void add_scaled(float (&acc)[8], float w, uint4 v) {
   }
 }
 
+// One row: LPR lanes (a sub-group) own 16 bytes of the row each.  Lane v of the
+// sub-group also loads block choice v and partial log-sum-exp v of the row (v < topk,
+// for topk <= LPR), so that every load of the row is issued at once; the sub-group
+// then shares them with shuffles.
 template <int D>
-__global__ void __launch_bounds__(kMergeThreads)
-merge_partials_kernel(const MergeParams p) {
-  constexpr int LPR = D / 8;       // lanes per row
-  constexpr int RPW = 32 / LPR;    // rows per warp
-  const int lane = threadIdx.x & 31;
-  const int sub = lane / LPR, v = lane % LPR;
-  const int64_t warp_id = ((int64_t)blockIdx.x * kMergeThreads + threadIdx.x) >> 5;
+__device__ __forceinline__ void merge_row(const MergeParams &p, int64_t row, int v, unsigned gmask,
+                                          int gbase) {
+  constexpr int LPR = D / 8;
   const int nrows = p.row_end - p.row_begin;
-  const int64_t total = (int64_t)p.batch * p.hq * nrows;
-  const int64_t row = warp_id * RPW + sub;
-  if (sub >= RPW || row >= total) return;
   const int il = (int)(row % nrows);
   const int64_t bh = row / nrows;
   const int h = (int)(bh % p.hq), b = (int)(bh / p.hq);
@@ -50,34 +48,64 @@ merge_partials_kernel(const MergeParams p) {
   // Chunk-local row: the pass covers rows [row_begin, row_end) of one chunk.
   const int64_t pbase = (bh * p.chunk_rows + il) * p.topk;
   const uint4 *po = reinterpret_cast<const uint4 *>(p.opart) + pbase * LPR + v;
-  // Issue the row's loads before any of them is needed.
   const int32_t *irow = p.idx + (bh * p.N + i) * p.topk;
-  uint4 own = po[(int64_t)npast * LPR];
+  const bool spread = p.topk <= LPR;
+  int my_blk = -1;
+  float my_l = 0.f;
+  if (spread && v < p.topk) {
+    my_blk = __ldg(irow + v);
+    my_l = p.lpart[pbase + v];
+  }
+  const uint4 own = po[(int64_t)npast * LPR];
   uint4 early[kMergeEager];
 #pragma unroll
   for (int s = 0; s < kMergeEager; ++s)
     if (s < npast) early[s] = po[(int64_t)s * LPR];
+  // Valid past slots: the leading choices below the own block.
   int np = 0;
-  for (int s = 0; s < npast; ++s) {
-    const int blk = __ldg(irow + s);
-    if (blk < 0 || blk >= c) break;
-    ++np;
+  float l_own;
+  if (spread) {
+    const bool bad = v < npast && (my_blk < 0 || my_blk >= c);
+    const unsigned badm = (__ballot_sync(gmask, bad) >> gbase) & ((1u << LPR) - 1u);
+    np = badm ? (__ffs(badm) - 1) : npast;
+    l_own = __shfl_sync(gmask, my_l, gbase + npast);
+  } else {
+    for (int s = 0; s < npast; ++s) {
+      const int blk = __ldg(irow + s);
+      if (blk < 0 || blk >= c) break;
+      ++np;
+    }
+    l_own = p.lpart[pbase + npast];
   }
-  const float l_own = p.lpart[pbase + npast];
+  auto lse_of = [&](int s) -> float {
+    return spread ? __shfl_sync(gmask, my_l, gbase + s) : p.lpart[pbase + s];
+  };
   float mx = l_own;
-  for (int s = 0; s < np; ++s) mx = fmaxf(mx, p.lpart[pbase + s]);
+  for (int s = 0; s < npast; ++s) {
+    const float ls = lse_of(s);
+    if (s < np) mx = fmaxf(mx, ls);
+  }
   float tot = __expf(l_own - mx);
-  for (int s = 0; s < np; ++s) tot += __expf(p.lpart[pbase + s] - mx);
+  for (int s = 0; s < npast; ++s) {
+    const float ls = lse_of(s);
+    if (s < np) tot += __expf(ls - mx);
+  }
   const float lse = mx + __logf(tot);
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   add_scaled(acc, __expf(l_own - lse), own);
 #pragma unroll
-  for (int s = 0; s < kMergeEager; ++s)
-    if (s < np) add_scaled(acc, __expf(p.lpart[pbase + s] - lse), early[s]);
-  for (int s = kMergeEager; s < np; ++s)
-    add_scaled(acc, __expf(p.lpart[pbase + s] - lse), po[(int64_t)s * LPR]);
+  for (int s = 0; s < kMergeEager; ++s) {
+    if (s < npast) {
+      const float ls = lse_of(s);
+      if (s < np) add_scaled(acc, __expf(ls - lse), early[s]);
+    }
+  }
+  for (int s = kMergeEager; s < npast; ++s) {
+    const float ls = lse_of(s);
+    if (s < np) add_scaled(acc, __expf(ls - lse), po[(int64_t)s * LPR]);
+  }
   uint4 w;
   w.x = pack_bf16x2(acc[0], acc[1]);
   w.y = pack_bf16x2(acc[2], acc[3]);
@@ -88,11 +116,35 @@ merge_partials_kernel(const MergeParams p) {
   if (v == 0) p.lse[bh * p.N + i] = lse;
 }
 
+template <int D>
+__global__ void __launch_bounds__(kMergeThreads)
+merge_partials_kernel(const MergeParams p) {
+  constexpr int LPR = D / 8;       // lanes per row
+  constexpr int RPW = 32 / LPR;    // rows per warp
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPR, v = lane % LPR;
+  if (sub >= RPW) return;          // D = 80: the last two lanes idle
+  const int gbase = sub * LPR;
+  const unsigned gmask = (LPR == 32 ? 0xffffffffu : ((1u << LPR) - 1u)) << gbase;
+  const int64_t nwarps = ((int64_t)gridDim.x * kMergeThreads) >> 5;
+  const int64_t warp_id = ((int64_t)blockIdx.x * kMergeThreads + threadIdx.x) >> 5;
+  const int64_t total = (int64_t)p.batch * p.hq * (p.row_end - p.row_begin);
+  // Rows warp_id * RPW + sub, then a grid-stride walk.
+  for (int64_t row = warp_id * RPW + sub; row < total; row += nwarps * RPW)
+    merge_row<D>(p, row, v, gmask, gbase);
+}
+
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t st) {
   const int64_t rows = (int64_t)p.batch * p.hq * (p.row_end - p.row_begin);
   const int rpw = 32 / (p.d / 8);
   const int64_t warps = (rows + rpw - 1) / rpw;
-  const int64_t blocks = (warps * 32 + kMergeThreads - 1) / kMergeThreads;
+  int64_t blocks = (warps * 32 + kMergeThreads - 1) / kMergeThreads;
+  // Enough CTAs to fill every SM several times over; each warp then walks rows.
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t cap = (int64_t)nsm * 8 * 4;
+  if (blocks > cap) blocks = cap;
   if (blocks <= 0) return cudaSuccess;
   switch (p.d) {
     case 64: merge_partials_kernel<64><<<(unsigned)blocks, kMergeThreads, 0, st>>>(p); break;
