@@ -91,9 +91,9 @@ def source_digest() -> str:
     return h.hexdigest()
 
 
-def stored_traffic(workload: str):
-    """DRAM bytes per attention step from the committed ncu summary, or None when the
-    kernels changed since it was taken."""
+def stored_traffic(workload: str, kernel: str = None):
+    """DRAM bytes per launch of `kernel` (or of the whole attention stage) from the
+    committed ncu summary, or None when the kernels changed since it was taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -102,7 +102,9 @@ def stored_traffic(workload: str):
     rec = d.get(workload)
     if not rec or rec.get("sources_sha256") != source_digest():
         return None
-    return rec.get("attention_dram_bytes_per_step")
+    if kernel is None:
+        return rec.get("attention_dram_bytes_per_step")
+    return rec.get("per_kernel_bytes", {}).get(kernel)
 
 
 # ------------------------------------------------------------------ accounting
@@ -135,6 +137,31 @@ def attended_pairs_moba(idx: torch.Tensor, w: workloads.Workload) -> int:
 def attended_pairs_swa(w: workloads.Workload) -> int:
     i = np.arange(w.seqlen, dtype=np.int64)
     return int(np.minimum(i + 1, w.window).sum()) * w.batch * w.hq
+
+
+def pass_work_moba(idx: torch.Tensor, w: workloads.Workload, chunk_rows: int) -> dict:
+    """Algorithmic work of each moba_attn_fwd pass over rows [0, chunk_rows): attended
+    FLOPs (4*d per (query, key) pair) of the past-block pass (whole selected past
+    blocks) and of the own-block pass (causal own block plus window tail keys), and
+    the bytes the merge pass must move (topk partial rows and log-sum-exps read, block
+    choices read, the output row and its log-sum-exp written)."""
+    B, N = w.block, w.seqlen
+    rows = min(chunk_rows, N)
+    sub = idx[:, :, :rows]
+    i = torch.arange(rows, device=idx.device)
+    c = i // B
+    past = int(((sub >= 0) & (sub < c[None, None, :, None])).sum().item()) * B
+    own = int(((i % B) + 1).sum().item()) * w.batch * w.hq
+    if w.window > 0:
+        total_rows = attended_pairs_moba(idx, w)  # all rows; window extras scaled below
+        base = int(((torch.arange(N, device=idx.device) % B) + 1).sum().item()) * w.batch * w.hq
+        base += int(((idx >= 0) & (idx < (torch.arange(N, device=idx.device) // B)[None, None, :, None]))
+                    .sum().item()) * B
+        own += int(round((total_rows - base) * rows / N))
+    rowcount = w.batch * w.hq * rows
+    merge_bytes = rowcount * (w.topk * (w.d * 2 + 4) + w.topk * 4 + w.d * 2 + 4)
+    return {"past_block_pass": 4.0 * w.d * past, "own_block_pass": 4.0 * w.d * own,
+            "merge_pass": merge_bytes}
 
 
 def dense_pairs(w: workloads.Workload) -> int:
@@ -314,12 +341,13 @@ def run_ours(args, rank, world, device):
             yield "attention"
         out_t, lse_t = runner.out, runner.lse
         layout_chunks = 1
+        chunk_rows = w.seqlen
         try:
             per_row = (w.topk if w.topk > 1 else 0) * (w.d * 2 + 4) * w.batch * w.hq
             cap = 4 << 30
             if per_row * w.seqlen > cap:
-                rows = max(128, (cap // per_row) // 128 * 128)
-                layout_chunks = math.ceil(w.seqlen / rows)
+                chunk_rows = max(128, (cap // per_row) // 128 * 128)
+                layout_chunks = math.ceil(w.seqlen / chunk_rows)
         except ZeroDivisionError:
             pass
         # pool, gate (+ scan, scatter), and per query chunk: past-block pass, own-block
@@ -333,6 +361,15 @@ def run_ours(args, rank, world, device):
             moba.swa_attn_fwd(qd, kd, vd, w.window, out=out_t, lse=lse_t)
             yield "attention"
         launches_per_step = 1
+
+    # Per-pass events inside moba_attn_fwd (first query chunk): the dominant kernel's
+    # own launch duration, timed on the stream it runs on.
+    pass_names = []
+    if w.kind == "moba":
+        pass_names = (["past_block_pass", "own_block_pass", "merge_pass"] if w.topk > 1
+                      else ["own_block_pass"])
+    pass_evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(pass_names) + 1)]
+    per_pass = {n: [] for n in pass_names}
 
     def step_timed():
         evs = [torch.cuda.Event(enable_timing=True)]
@@ -359,6 +396,8 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize()
     per_stage = {}
     total_ms = 0.0
+    if pass_names:
+        moba.set_pass_events(pass_evs)
     with ClockSampler(torch.cuda.current_device()) as clk:
         clk.mark_start()
         for _ in range(args.steps):
@@ -368,8 +407,12 @@ def run_ours(args, rank, world, device):
             total_ms += evs[0].elapsed_time(evs[-1])
             for a, b_, n in zip(evs[:-1], evs[1:], names):
                 per_stage.setdefault(n, []).append(a.elapsed_time(b_))
+            for a, b_, n in zip(pass_evs[:-1], pass_evs[1:], pass_names):
+                per_pass[n].append(a.elapsed_time(b_))
         clk.mark_stop()
     torch.cuda.synchronize()
+    if pass_names:
+        moba.set_pass_events(None)
     total_ms = max_over_ranks(total_ms, device)
     if world > 1:
         torch.distributed.barrier()
@@ -383,13 +426,42 @@ def run_ours(args, rank, world, device):
     stage_ms = {n: sum(v) / len(v) for n, v in per_stage.items()}
     attn_ms = stage_ms["attention"]
     achieved = flops / (attn_ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": tc_peak,
-                "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
-                "traffic": stored_traffic(w.name),
-                "kernel": ("moba_attn_fwd: past-block pass, own-block pass and merge "
-                           "(3 launches per query chunk)") if w.kind == "moba" else "swa_attn_fwd",
-                "peak_kind": f"bf16 dense burst, {peak_kind}"}
     extra = {}
+    kname = f"attn_fwd_kernel<{w.d}, 0>"
+    if w.kind == "moba":
+        # Work of each pass over the first query chunk (all of it for one chunk).
+        work = pass_work_moba(runner.idx, w, chunk_rows)
+        pass_ms = {n: sum(v) / len(v) for n, v in per_pass.items()}
+        passes = {}
+        for n in pass_names:
+            t = pass_ms[n] * 1e-3
+            if n == "merge_pass":
+                gbs = work[n] / t / 1e9
+                passes[n] = {"ms": round(pass_ms[n], 4), "bytes": work[n], "gbs": round(gbs, 1),
+                             "frac_hbm": round(gbs / hbm, 4)}
+            else:
+                tf = work[n] / t / 1e12
+                passes[n] = {"ms": round(pass_ms[n], 4), "flops": work[n], "tflops": round(tf, 2),
+                             "frac": round(tf / tc_peak, 4)}
+        extra["passes"] = passes
+        extra["attention_stage"] = {"ms": round(attn_ms, 4), "tflops": round(achieved, 2),
+                                    "frac": round(achieved / tc_peak, 4),
+                                    "note": "whole moba_attn_fwd call: all passes, all query chunks"}
+        dom = max((n for n in pass_names if n != "merge_pass"), key=lambda n: pass_ms[n])
+        kname = f"attn_fwd_kernel<{w.d}, {1 if dom == 'past_block_pass' else 0}>"
+        roofline = {"bound": "tensor", "achieved": passes[dom]["tflops"], "peak": tc_peak,
+                    "unit": "TFLOP/s", "frac": passes[dom]["frac"],
+                    "traffic": stored_traffic(w.name, kname),
+                    "kernel": f"{kname} ({dom.replace('_', ' ')}; first query chunk)",
+                    "work": "4*d FLOPs per attended (query, key) pair of the pass",
+                    "peak_kind": f"bf16 dense burst, {peak_kind}"}
+    else:
+        roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": tc_peak,
+                    "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
+                    "traffic": stored_traffic(w.name, kname),
+                    "kernel": f"{kname} (swa_attn_fwd: one launch)",
+                    "work": "4*d FLOPs per attended (query, key) pair",
+                    "peak_kind": f"bf16 dense burst, {peak_kind}"}
     if w.kind == "moba":
         sel_ms = stage_ms["pool"] + stage_ms["select"]
         n_entries = int(((runner.idx >= 0).sum().item()) - w.batch * w.hq * w.seqlen)

@@ -30,7 +30,8 @@ _STATUS = {
 
 # Entry points declared in include/moba.h.
 ABI_FUNCTIONS = ("moba_workspace_size", "moba_pool_keys", "moba_select_topk", "moba_attn_fwd",
-                 "swa_attn_fwd", "moba_prefill_static", "moba_device_status", "moba_status_string")
+                 "swa_attn_fwd", "moba_prefill_static", "moba_device_status", "moba_set_pass_events",
+                 "moba_status_string")
 
 
 class MobaError(RuntimeError):
@@ -58,6 +59,7 @@ def _load():
     lib.swa_attn_fwd.argtypes = [T, T, T, I, I, I, I, I, I, ctypes.c_float, T, P, P]
     lib.moba_prefill_static.argtypes = [T, T, T, I, I, I, I, I, I, I, I, ctypes.c_float, T, P, P]
     lib.moba_device_status.argtypes = []
+    lib.moba_set_pass_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), I]
     lib.moba_status_string.argtypes = [I]
     lib.moba_status_string.restype = ctypes.c_char_p
     for name in ABI_FUNCTIONS[:-1]:
@@ -177,6 +179,19 @@ def moba_prefill_static(q, k, v, block: int, topk: int, window: int = 0, scale: 
            _lib.moba_prefill_static(_t(q), _t(k), _t(v), b, hq, hkv, N, d, block, topk, window,
                                     float(scale), _t(out), lse.data_ptr(), _stream(stream)))
     return out, lse
+
+
+def set_pass_events(events) -> None:
+    """Diagnostics: moba_attn_fwd records these torch.cuda.Event objects before its
+    first kernel and after each pass (past blocks, own block, merge) of its first query
+    chunk; None or [] switches it off.  Each event is recorded once here first so that
+    its CUDA handle exists."""
+    events = list(events or [])
+    for e in events:
+        if not e.cuda_event:
+            e.record()
+    arr = (ctypes.c_void_p * max(1, len(events)))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check("moba_set_pass_events", _lib.moba_set_pass_events(arr, len(events)))
 
 
 def device_status() -> int:

@@ -23,7 +23,7 @@ cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileo
                         int nlists, cudaStream_t st);
 cudaError_t launch_scatter(const ScatterParams &p, cudaStream_t st);
 cudaError_t launch_gate_tc(const CUtensorMap *maps, const GateParams &p, int grid, cudaStream_t st);
-int gate_tc_rows_staged();
+bool gate_tc_supports(int nblk, int topk);
 cudaError_t launch_attn(const CUtensorMap *maps, const AttnParams &p, int mode, int grid,
                         cudaStream_t st);
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t st);
@@ -178,6 +178,14 @@ int make_kbar_maps(CUtensorMap *maps, const void *split, int batch, int hkv, int
 
 int launch_status(cudaError_t e) { return e == cudaSuccess ? MOBA_OK : MOBA_ERR_LAUNCH; }
 
+// Per-pass timing events of moba_attn_fwd (diagnostics; see moba_set_pass_events).
+cudaEvent_t g_pass_events[8];
+int g_pass_nevents = 0;
+
+void record_pass_event(int k, int chunk, cudaStream_t st) {
+  if (chunk == 0 && k < g_pass_nevents && g_pass_events[k]) cudaEventRecord(g_pass_events[k], st);
+}
+
 // Device address of the status words on the current device.
 int status_words(int **ptr) {
   void *p = nullptr;
@@ -234,7 +242,7 @@ int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, i
   int *counts = reinterpret_cast<int *>(ws + w.off_counts);
   if (cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)w.nlists, st) != cudaSuccess)
     return MOBA_ERR_LAUNCH;
-  if (w.nblk <= gate_tc_rows_staged()) {
+  if (gate_tc_supports(w.nblk, topk)) {
     // Tensor-core gate: q tiles and the pooled keys through TMA.
     int nsm = 0;
     if ((rc = check_device(&nsm))) return rc;
@@ -331,6 +339,8 @@ int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *id
   p.npast = w.npast;
   p.nblk = w.nblk;
   p.lists_per_chunk = batch * hkv * w.nblk;
+  int ev = 0;
+  record_pass_event(ev++, 0, st);
   for (int c = 0; c < w.nchunks; ++c) {
     p.chunk = c;
     p.row_begin = c * w.chunk_rows;
@@ -340,10 +350,12 @@ int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *id
       p.q_gather_tma = q_gather_tma;
       if ((rc = launch_status(launch_attn(gmaps, p, kGathered, nsm, st)))) return rc;
       p.q_gather_tma = 0;
+      record_pass_event(ev++, c, st);
     }
     p.ntiles = query_major_units(batch, hq, hkv, block, 1, p.row_begin, p.row_end);
     const int grid = p.ntiles < nsm ? p.ntiles : nsm;
     if ((rc = launch_status(launch_attn(maps, p, kQueryMajor, grid, st)))) return rc;
+    record_pass_event(ev++, c, st);
     if (w.npast > 0) {
       MergeParams mp{};
       mp.opart = p.opart;
@@ -357,8 +369,17 @@ int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *id
       mp.row_begin = p.row_begin;
       mp.row_end = p.row_end;
       if ((rc = launch_status(launch_merge(mp, st)))) return rc;
+      record_pass_event(ev++, c, st);
     }
   }
+  return MOBA_OK;
+}
+
+int moba_set_pass_events(void *const *events, int count) {
+  if (count < 0 || count > 8) return MOBA_ERR_ARG;
+  if (!events) count = 0;
+  for (int k = 0; k < 8; ++k) g_pass_events[k] = (k < count) ? static_cast<cudaEvent_t>(events[k]) : nullptr;
+  g_pass_nevents = count;
   return MOBA_OK;
 }
 

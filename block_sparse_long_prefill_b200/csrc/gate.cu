@@ -8,6 +8,8 @@
 // highest scores.  §"인과성 보존": only blocks wholly before the query's own block
 // c = i / block compete (j < c), block c is always kept, later blocks never.
 //
+// It takes problems of at most 256 blocks and k - 1 <= kGateMaxPicks; the general
+// gate of select.cu takes the others.
 // One persistent CTA per SM walks a contiguous range of 128-row query tiles ordered
 // (batch, kv-head, row tile, q-head), so that the pooled keys of one kv-head are staged
 // in shared memory once per range.  Since block % 128 == 0, every row of a tile has the
@@ -17,8 +19,9 @@
 //   warp 1     tcgen05 MMA issuer and TMEM owner: S = Q hi^T + Q lo^T in fp32, into
 //              one of two TMEM accumulators (N = c rounded up to 16 columns)
 //   warps 2-5  top-k: thread r owns row r (TMEM lane r) and scans its c scores in
-//              ascending block order, keeping the best k-1 in registers (a strictly
-//              greater score displaces; ties keep the lower block), then writes the
+//              ascending block order, keeping the best k-1 (at most kGateMaxPicks) in
+//              a register list without branches (a strictly greater score displaces;
+//              ties keep the lower block), then writes the
 //              row's choices in ascending order, the own block, and -1 padding; it
 //              also counts the picks per past block for the dispatch lists.
 // q is exactly bf16 and kbar = hi + lo to about 2^-17 relative, so the fp32 scores
@@ -33,6 +36,7 @@ namespace moba {
 
 constexpr int kGateTcThreads = 192;
 constexpr int kGateMaxBlocks = 256;   // pooled keys staged at once (MMA N <= 256)
+constexpr int kGateMaxPicks = 4;      // past blocks per row kept in the register list
 
 constexpr int kGateMaxStages = 8;     // query tile ring depth limit
 constexpr int kGateSmemLimit = 227 * 1024;
@@ -315,29 +319,14 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           idx[e] = -1;
         }
         const uint32_t acc = tmem + lane_off + 256 * a;
-        float thr = -INFINITY;                              // val[npick - 1]
         for (int j0 = 0; j0 < c; j0 += 32) {
           uint32_t sc[32];
           tmem_ld32(acc + j0, sc);
           tmem_wait_ld();
-          if (KM <= 4) {
-            // Short lists: every score goes through the list, with no branch.
+          // Every score goes through the short list, with no branch.
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              topk_insert<KM>(val, idx, (j0 + e < c) ? __uint_as_float(sc[e]) : -INFINITY, j0 + e);
-          } else {
-            // Long lists: only scores above the current k-1-th best go in.
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float v = __uint_as_float(sc[e]);
-              if (j0 + e < c && v > thr) {
-                topk_insert<KM>(val, idx, v, j0 + e);
-                thr = val[0];
-#pragma unroll
-                for (int f = 1; f < KM; ++f) thr = (f < npick) ? val[f] : thr;
-              }
-            }
-          }
+          for (int e = 0; e < 32; ++e)
+            topk_insert<KM>(val, idx, (j0 + e < c) ? __uint_as_float(sc[e]) : -INFINITY, j0 + e);
         }
         tc_fence_before();
         __syncwarp();
@@ -391,10 +380,8 @@ static cudaError_t launch_gate_tc_d(const CUtensorMap *maps, const GateParams &p
                                     cudaStream_t st) {
   const int npast = p.topk - 1;
   if (npast <= 2) return launch_gate_tc_dk<D, 2>(maps, p, grid, st);
-  if (npast <= 4) return launch_gate_tc_dk<D, 4>(maps, p, grid, st);
-  if (npast <= 8) return launch_gate_tc_dk<D, 8>(maps, p, grid, st);
-  if (npast <= 16) return launch_gate_tc_dk<D, 16>(maps, p, grid, st);
-  return launch_gate_tc_dk<D, 32>(maps, p, grid, st);
+  if (npast <= kGateMaxPicks) return launch_gate_tc_dk<D, kGateMaxPicks>(maps, p, grid, st);
+  return cudaErrorInvalidValue;
 }
 
 // maps: Q (64-column box of 128 rows), Q tail, kbar planes (64-column box of
@@ -408,6 +395,8 @@ cudaError_t launch_gate_tc(const CUtensorMap *maps, const GateParams &p, int gri
   return cudaErrorInvalidValue;
 }
 
-int gate_tc_rows_staged() { return kGateMaxBlocks; }
+// Whether this kernel takes the problem: at most 256 pooled blocks (all staged at once)
+// and at most 4 past picks per row (a short register list scanned without branches).
+bool gate_tc_supports(int nblk, int topk) { return nblk <= kGateMaxBlocks && topk - 1 <= kGateMaxPicks; }
 
 }  // namespace moba

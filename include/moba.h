@@ -24,8 +24,8 @@
  *   - Block j covers key positions [j*block, (j+1)*block) (0-based; the MoBA page
  *     numbers blocks from 1).  N must be a multiple of block, and block a multiple
  *     of 128.
- *   - d must be 64, 80 or 128 for the attention calls (any multiple of 8 up to 256
- *     for moba_pool_keys and moba_select_topk).
+ *   - d must be 64, 80 or 128 (moba_pool_keys alone takes any multiple of 8 up to
+ *     256).
  *   - Ownership: the caller allocates every buffer (inputs, outputs, workspace); the
  *     library allocates no device memory and keeps no state between calls (except the
  *     fixed scratch array of moba_prefill_static, below).
@@ -154,6 +154,17 @@ int moba_device_status(void);
 
 /* Static description of a status code. */
 const char *moba_status_string(int status);
+
+/* Diagnostics for benchmarks: per-pass timing of moba_attn_fwd.  `events` holds
+ * `count` cudaEvent_t handles created by the caller (count 0 or events NULL switches
+ * this off).  While set, every moba_attn_fwd call records, on its stream, events[0]
+ * before its first kernel and events[k] after its k-th kernel (k = 1, 2, 3: the
+ * past-block pass, the own-block pass and the merge pass; with topk = 1 only the
+ * own-block pass runs), for its first query chunk and as far as count allows.  The
+ * library keeps the handles, not the events: they must outlive their use.  A
+ * process-wide setting, not synchronised between host threads.
+ * Returns MOBA_OK, or MOBA_ERR_ARG when count is outside [0, 8]. */
+int moba_set_pass_events(void *const *events, int count);
 
 #ifdef __cplusplus
 }

@@ -95,10 +95,10 @@ def test_moba_strided_inputs():
 
 @pytest.mark.parametrize("name,kw", [
     # 512 blocks: more pooled keys than the tensor-core gate stages at once, so the
-    # selection takes the general (mma.sync) gate kernel.
+    # selection takes the general (mma.sync) gate kernel (as do rows with > 4 picks).
     ("many_blocks", dict(batch=1, hq=2, hkv=1, seqlen=65536, d=64, block=128, topk=4)),
-    # exactly the tensor-core gate's limit of 256 blocks, with d = 80 and GQA.
-    ("blocks256_d80", dict(batch=1, hq=4, hkv=2, seqlen=32768, d=80, block=128, topk=6)),
+    # exactly the tensor-core gate's limits (256 blocks, 4 past picks), d = 80, GQA.
+    ("blocks256_d80", dict(batch=1, hq=4, hkv=2, seqlen=32768, d=80, block=128, topk=5)),
 ])
 def test_moba_block_count_limits_sampled_rows(name, kw):
     w = workloads.small_moba(name=name, **kw)
