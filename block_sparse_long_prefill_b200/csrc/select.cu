@@ -36,13 +36,13 @@ pool_keys_kernel(const uint16_t *__restrict__ k, int64_t sb, int64_t sh, int64_t
   if (grp < ngroups) {
     const uint16_t *base = k + b * sb + hk * sh + (int64_t)j * block * sn + vec * 8;
     int r = grp;
-    for (; r + 3 * ngroups < block; r += 4 * ngroups) {
-      uint4 v[4];
+    for (; r + 7 * ngroups < block; r += 8 * ngroups) {
+      uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < 8; ++u)
         v[u] = __ldg(reinterpret_cast<const uint4 *>(base + (int64_t)(r + u * ngroups) * sn));
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
