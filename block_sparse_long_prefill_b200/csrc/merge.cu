@@ -32,23 +32,23 @@ __device__ __forceinline__ void add_scaled(float (&acc)[8], float w, uint4 v) {
 
 // One row: LPR lanes (a sub-group) own 16 bytes of the row each.  Lane v of the
 // sub-group also loads block choice v and partial log-sum-exp v of the row (v < topk,
-// for topk <= LPR), so that every load of the row is issued at once; the sub-group
-// then shares them with shuffles.
+// for topk <= LPR), so that every load of the row is in flight at once.  Lane v then
+// computes the weight of slot v alone (one exponential), and the sub-group shares the
+// maximum, the sum and the weights with shuffles.  Row indices fit 32 bits: the host
+// bounds batch * hq * N below 2^31 whenever partials exist.
 template <int D>
-__device__ __forceinline__ void merge_row(const MergeParams &p, int64_t row, int v, unsigned gmask,
-                                          int gbase) {
+__device__ __forceinline__ void merge_row(const MergeParams &p, int row, int nrows, int v,
+                                          unsigned gmask, int gbase) {
   constexpr int LPR = D / 8;
-  const int nrows = p.row_end - p.row_begin;
-  const int il = (int)(row % nrows);
-  const int64_t bh = row / nrows;
-  const int h = (int)(bh % p.hq), b = (int)(bh / p.hq);
+  const int bh = row / nrows, il = row - bh * nrows;
+  const int h = bh % p.hq, b = bh / p.hq;
   const int i = p.row_begin + il;
   const int c = i / p.block;
   const int npast = p.topk - 1;
   // Chunk-local row: the pass covers rows [row_begin, row_end) of one chunk.
-  const int64_t pbase = (bh * p.chunk_rows + il) * p.topk;
+  const int64_t pbase = ((int64_t)bh * p.chunk_rows + il) * p.topk;
   const uint4 *po = reinterpret_cast<const uint4 *>(p.opart) + pbase * LPR + v;
-  const int32_t *irow = p.idx + (bh * p.N + i) * p.topk;
+  const int32_t *irow = p.idx + ((int64_t)bh * p.N + i) * p.topk;
   const bool spread = p.topk <= LPR;
   int my_blk = -1;
   float my_l = 0.f;
@@ -61,50 +61,57 @@ __device__ __forceinline__ void merge_row(const MergeParams &p, int64_t row, int
 #pragma unroll
   for (int s = 0; s < kMergeEager; ++s)
     if (s < npast) early[s] = po[(int64_t)s * LPR];
-  // Valid past slots: the leading choices below the own block.
-  int np = 0;
-  float l_own;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  float lse;
   if (spread) {
+    // Valid past slots: the leading choices below the own block; slot npast is the
+    // own block.
     const bool bad = v < npast && (my_blk < 0 || my_blk >= c);
     const unsigned badm = (__ballot_sync(gmask, bad) >> gbase) & ((1u << LPR) - 1u);
-    np = badm ? (__ffs(badm) - 1) : npast;
-    l_own = __shfl_sync(gmask, my_l, gbase + npast);
+    const int np = badm ? (__ffs(badm) - 1) : npast;
+    float mx = -INFINITY;
+    for (int s = 0; s < p.topk; ++s) {
+      const float ls = __shfl_sync(gmask, my_l, gbase + s);
+      if (s < np || s == npast) mx = fmaxf(mx, ls);
+    }
+    const float e_mine = (v < np || v == npast) ? __expf(my_l - mx) : 0.f;
+    float tot = 0.f;
+    for (int s = 0; s < p.topk; ++s) tot += __shfl_sync(gmask, e_mine, gbase + s);
+    const float inv = 1.f / tot;
+    lse = mx + __logf(tot);
+    add_scaled(acc, __shfl_sync(gmask, e_mine, gbase + npast) * inv, own);
+#pragma unroll
+    for (int s = 0; s < kMergeEager; ++s) {
+      if (s < npast) {
+        const float w = __shfl_sync(gmask, e_mine, gbase + s) * inv;
+        if (s < np) add_scaled(acc, w, early[s]);
+      }
+    }
+    for (int s = kMergeEager; s < npast; ++s) {
+      const float w = __shfl_sync(gmask, e_mine, gbase + s) * inv;
+      if (s < np) add_scaled(acc, w, po[(int64_t)s * LPR]);
+    }
   } else {
+    int np = 0;
     for (int s = 0; s < npast; ++s) {
       const int blk = __ldg(irow + s);
       if (blk < 0 || blk >= c) break;
       ++np;
     }
-    l_own = p.lpart[pbase + npast];
-  }
-  auto lse_of = [&](int s) -> float {
-    return spread ? __shfl_sync(gmask, my_l, gbase + s) : p.lpart[pbase + s];
-  };
-  float mx = l_own;
-  for (int s = 0; s < npast; ++s) {
-    const float ls = lse_of(s);
-    if (s < np) mx = fmaxf(mx, ls);
-  }
-  float tot = __expf(l_own - mx);
-  for (int s = 0; s < npast; ++s) {
-    const float ls = lse_of(s);
-    if (s < np) tot += __expf(ls - mx);
-  }
-  const float lse = mx + __logf(tot);
-  float acc[8];
+    const float l_own = p.lpart[pbase + npast];
+    float mx = l_own;
+    for (int s = 0; s < np; ++s) mx = fmaxf(mx, p.lpart[pbase + s]);
+    float tot = __expf(l_own - mx);
+    for (int s = 0; s < np; ++s) tot += __expf(p.lpart[pbase + s] - mx);
+    lse = mx + __logf(tot);
+    add_scaled(acc, __expf(l_own - lse), own);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  add_scaled(acc, __expf(l_own - lse), own);
-#pragma unroll
-  for (int s = 0; s < kMergeEager; ++s) {
-    if (s < npast) {
-      const float ls = lse_of(s);
-      if (s < np) add_scaled(acc, __expf(ls - lse), early[s]);
-    }
-  }
-  for (int s = kMergeEager; s < npast; ++s) {
-    const float ls = lse_of(s);
-    if (s < np) add_scaled(acc, __expf(ls - lse), po[(int64_t)s * LPR]);
+    for (int s = 0; s < kMergeEager; ++s)
+      if (s < np) add_scaled(acc, __expf(p.lpart[pbase + s] - lse), early[s]);
+    for (int s = kMergeEager; s < np; ++s)
+      add_scaled(acc, __expf(p.lpart[pbase + s] - lse), po[(int64_t)s * LPR]);
   }
   uint4 w;
   w.x = pack_bf16x2(acc[0], acc[1]);
@@ -113,7 +120,7 @@ __device__ __forceinline__ void merge_row(const MergeParams &p, int64_t row, int
   w.w = pack_bf16x2(acc[6], acc[7]);
   uint16_t *dst = p.out + b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)i * p.o_sn + v * 8;
   *reinterpret_cast<uint4 *>(dst) = w;
-  if (v == 0) p.lse[bh * p.N + i] = lse;
+  if (v == 0) p.lse[(int64_t)bh * p.N + i] = lse;
 }
 
 template <int D>
@@ -126,12 +133,13 @@ merge_partials_kernel(const MergeParams p) {
   if (sub >= RPW) return;          // D = 80: the last two lanes idle
   const int gbase = sub * LPR;
   const unsigned gmask = (LPR == 32 ? 0xffffffffu : ((1u << LPR) - 1u)) << gbase;
-  const int64_t nwarps = ((int64_t)gridDim.x * kMergeThreads) >> 5;
-  const int64_t warp_id = ((int64_t)blockIdx.x * kMergeThreads + threadIdx.x) >> 5;
-  const int64_t total = (int64_t)p.batch * p.hq * (p.row_end - p.row_begin);
+  const int nwarps = (int)((gridDim.x * kMergeThreads) >> 5);
+  const int warp_id = (int)((blockIdx.x * kMergeThreads + threadIdx.x) >> 5);
+  const int nrows = p.row_end - p.row_begin;
+  const int total = p.batch * p.hq * nrows;
   // Rows warp_id * RPW + sub, then a grid-stride walk.
-  for (int64_t row = warp_id * RPW + sub; row < total; row += nwarps * RPW)
-    merge_row<D>(p, row, v, gmask, gbase);
+  for (int row = warp_id * RPW + sub; row < total; row += nwarps * RPW)
+    merge_row<D>(p, row, nrows, v, gmask, gbase);
 }
 
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t st) {
