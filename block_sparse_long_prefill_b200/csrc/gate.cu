@@ -86,6 +86,8 @@ __device__ __forceinline__ uint64_t gate_desc(uint32_t tile, int ks, int rows) {
 // hk * G + g.  Ordered so that consecutive tiles share the kv-head.
 struct GateTile {
   int b, hk, g, rt;
+  int c;        // own block of the tile's rows: 128 rt / block
+  int chunk;    // query chunk of the tile's rows: 128 rt / chunk_rows
 };
 __device__ __forceinline__ GateTile gate_tile(const GateParams &p, int t) {
   GateTile r;
@@ -96,7 +98,25 @@ __device__ __forceinline__ GateTile gate_tile(const GateParams &p, int t) {
   t /= nrt;
   r.hk = t % p.hkv;
   r.b = t / p.hkv;
+  r.c = (r.rt * 128) / p.block;
+  r.chunk = (r.rt * 128) / p.chunk_rows;
   return r;
+}
+
+// The next tile in that order, without divisions (one decode per range, then steps).
+__device__ __forceinline__ void gate_tile_next(const GateParams &p, GateTile &r) {
+  if (++r.g < p.G) return;
+  r.g = 0;
+  ++r.rt;
+  if (r.rt * 128 == (r.c + 1) * p.block) ++r.c;
+  if (r.rt * 128 == (r.chunk + 1) * p.chunk_rows) ++r.chunk;
+  if (r.rt < p.N / 128) return;
+  r.rt = 0;
+  r.c = 0;
+  r.chunk = 0;
+  if (++r.hk < p.hkv) return;
+  r.hk = 0;
+  ++r.b;
 }
 
 // Insertion of (v, j) into the descending list val / idx.  Entries past the npick in
@@ -180,8 +200,8 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool ok = true;
       int cur = -1;
       uint32_t kuse = 0, quse = 0;
-      for (int t = t_begin; ok && t < t_end; ++t) {
-        const GateTile gt = gate_tile(p, t);
+      GateTile gt = gate_tile(p, t_begin);
+      for (int t = t_begin; ok && t < t_end; ++t, gate_tile_next(p, gt)) {
         const int grp = gt.b * p.hkv + gt.hk;
         if (grp != cur) {
           cur = grp;
@@ -219,8 +239,8 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool ok = true;
       int cur = -1;
       uint32_t kuse = 0, quse = 0, ause = 0;
-      for (int t = t_begin; ok && t < t_end; ++t) {
-        const GateTile gt = gate_tile(p, t);
+      GateTile gt = gate_tile(p, t_begin);
+      for (int t = t_begin; ok && t < t_end; ++t, gate_tile_next(p, gt)) {
         const int grp = gt.b * p.hkv + gt.hk;
         if (grp != cur) {
           cur = grp;
@@ -231,7 +251,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!(ok = mbar_wait(&bar.q_full[s], (quse / qst) & 1, abort, p.status, site0 + 4))) break;
         if (!(ok = mbar_wait(&bar.acc_empty[a], ((ause >> 1) & 1) ^ 1, abort, p.status, site0 + 5))) break;
         tc_fence_after();
-        const int c = (gt.rt * 128) / p.block;              // own block of every row
+        const int c = gt.c;                                 // own block of every row
         // Score columns needed (none when every past block is kept anyway).
         const int nn = (c > p.topk - 1) ? min((c + 15) & ~15, kc16) : 0;
         if (nn > 0) {
@@ -250,10 +270,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         umma_commit(&bar.acc_full[a]);
         umma_commit(&bar.q_empty[s]);
         // Last tile of this kv-head in the range: the pooled keys may be replaced.
-        const bool last = (t + 1 == t_end) || ([&] {
-          const GateTile nx = gate_tile(p, t + 1);
-          return nx.b * p.hkv + nx.hk != grp;
-        })();
+        const bool last = (t + 1 == t_end) || (gt.g == p.G - 1 && gt.rt == p.N / 128 - 1);
         if (last) umma_commit(&bar.k_empty);
         ++quse;
         ++ause;
@@ -285,13 +302,13 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       __syncwarp();
     };
-    for (int t = t_begin; ok && t < t_end; ++t) {
-      const GateTile gt = gate_tile(p, t);
+    GateTile gt = gate_tile(p, t_begin);
+    for (int t = t_begin; ok && t < t_end; ++t, gate_tile_next(p, gt)) {
       const int i = gt.rt * 128 + r;
-      const int c = (gt.rt * 128) / p.block;
+      const int c = gt.c;
       const int h = gt.hk * p.G + gt.g;
       const int a = ause & 1;
-      const int list = ((gt.rt * 128) / p.chunk_rows * p.batch + gt.b) * p.hkv + gt.hk;
+      const int list = (gt.chunk * p.batch + gt.b) * p.hkv + gt.hk;
       if (list != cur_list) {
         if (cur_list >= 0) flush(cur_list);
         cur_list = list;
