@@ -18,7 +18,8 @@
 //              pooled keys kbar = hi + lo (two bf16 matrices of up to 256 rows)
 //   warp 1     tcgen05 MMA issuer and TMEM owner: S = Q hi^T + Q lo^T in fp32, into
 //              one of two TMEM accumulators (N = c rounded up to 16 columns)
-//   warps 2-5  top-k: thread r owns row r (TMEM lane r) and scans its c scores in
+//   warps 2-9  top-k, two groups of four warps taking the tiles (and accumulators) in
+//              turn: thread r owns row r (TMEM lane r) and scans its c scores in
 //              ascending block order, keeping the best k-1 (at most kGateMaxPicks) in
 //              a register list without branches (a strictly greater score displaces;
 //              ties keep the lower block), then writes the
@@ -34,7 +35,7 @@
 
 namespace moba {
 
-constexpr int kGateTcThreads = 192;
+constexpr int kGateTcThreads = 320;
 constexpr int kGateMaxBlocks = 256;   // pooled keys staged at once (MMA N <= 256)
 constexpr int kGateMaxPicks = 4;      // past blocks per row kept in the register list
 
@@ -57,7 +58,7 @@ struct GateCfg {
   __host__ __device__ static constexpr int k_off(int qst) { return qst * QTILE; }
   __host__ __device__ static constexpr int hist_off(int qst, int kc16) { return k_off(qst) + 2 * kmat(kc16); }
   __host__ __device__ static constexpr int bar_off(int qst, int kc16) {
-    return hist_off(qst, kc16) + 4 * 4 * kGateMaxBlocks;
+    return hist_off(qst, kc16) + 8 * 4 * kGateMaxBlocks;
   }
   __host__ __device__ static constexpr int smem(int qst, int kc16) { return bar_off(qst, kc16) + 512 + 1024; }
 };
@@ -179,7 +180,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     bar.abort = 0;
     fence_barrier_init();
   }
-  for (int j = tid; j < 4 * kGateMaxBlocks; j += kGateTcThreads) hist[j] = 0;
+  for (int j = tid; j < 8 * kGateMaxBlocks; j += kGateTcThreads) hist[j] = 0;
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -284,9 +285,12 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // Each warp counts its rows' picks in its own shared histogram and adds it to the
     // list counts when its rows move to another (chunk, batch, kv-head) list, so no
     // barrier across warps is needed.
+    // Two groups of four warps take the tiles in turn: group gi (warps 2-5 or 6-9)
+    // reads accumulator gi and handles tiles t_begin + gi, t_begin + gi + 2, ...
+    const int gi = (warp - 2) >> 2;
     const int r = 32 * (warp & 3) + lane;                  // row within the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    int *whist = hist + (warp & 3) * kGateMaxBlocks;
+    int *whist = hist + (warp - 2) * kGateMaxBlocks;
     const int npast = p.topk - 1;
     bool ok = true;
     uint32_t ause = 0;
@@ -303,17 +307,18 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       __syncwarp();
     };
     GateTile gt = gate_tile(p, t_begin);
-    for (int t = t_begin; ok && t < t_end; ++t, gate_tile_next(p, gt)) {
+    if (gi) gate_tile_next(p, gt);
+    for (int t = t_begin + gi; ok && t < t_end; t += 2, gate_tile_next(p, gt), gate_tile_next(p, gt)) {
       const int i = gt.rt * 128 + r;
       const int c = gt.c;
       const int h = gt.hk * p.G + gt.g;
-      const int a = ause & 1;
+      const int a = gi;
       const int list = (gt.chunk * p.batch + gt.b) * p.hkv + gt.hk;
       if (list != cur_list) {
         if (cur_list >= 0) flush(cur_list);
         cur_list = list;
       }
-      ok = mbar_wait(&bar.acc_full[a], (ause >> 1) & 1, abort, p.status, site0 + 6);
+      ok = mbar_wait(&bar.acc_full[a], ause & 1, abort, p.status, site0 + 6);
       if (!(ok = __all_sync(FULL, ok))) break;
       tc_fence_after();
       int32_t *orow = p.idx + (((int64_t)gt.b * p.hq + h) * p.N + i) * p.topk;
