@@ -97,8 +97,12 @@ def test_moba_strided_inputs():
     # 512 blocks: more pooled keys than the tensor-core gate stages at once, so the
     # selection takes the general (mma.sync) gate kernel (as do rows with > 4 picks).
     ("many_blocks", dict(batch=1, hq=2, hkv=1, seqlen=65536, d=64, block=128, topk=4)),
-    # exactly the tensor-core gate's limits (256 blocks, 4 past picks), d = 80, GQA.
+    # exactly the tensor-core gate's block limit (256 blocks), d = 80, GQA.
     ("blocks256_d80", dict(batch=1, hq=4, hkv=2, seqlen=32768, d=80, block=128, topk=5)),
+    # long top-k lists (k - 1 > 4: the general gate), 128 / 256 / 64 blocks.
+    ("k9_blocks128", dict(batch=1, hq=2, hkv=1, seqlen=16384, d=64, block=128, topk=9)),
+    ("k13_blocks256", dict(batch=1, hq=2, hkv=2, seqlen=32768, d=128, block=128, topk=13)),
+    ("k32_blocks64", dict(batch=1, hq=2, hkv=1, seqlen=8192, d=128, block=128, topk=32)),
 ])
 def test_moba_block_count_limits_sampled_rows(name, kw):
     w = workloads.small_moba(name=name, **kw)
