@@ -584,10 +584,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (!(ok = __all_sync(FULL, ok))) break;
         tc_fence_after();
         uint32_t sv[128];
-        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+        tmem_ld64(tS, *reinterpret_cast<uint32_t(*)[64]>(&sv[0]));
+        tmem_ld64(tS + 64, *reinterpret_cast<uint32_t(*)[64]>(&sv[64]));
         tmem_wait_ld();
         float *s = reinterpret_cast<float *>(sv);
         // Masks.
@@ -669,10 +667,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(other_turn);
-        tmem_st16(tS, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-        tmem_st16(tS + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
-        tmem_st16(tS + 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[32]));
-        tmem_st16(tS + 48, *reinterpret_cast<uint32_t(*)[16]>(&sv[48]));
+        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
         l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         tmem_wait_st();
         tc_fence_before();

@@ -119,3 +119,29 @@ def test_moba_full_size_sampled_rows(name):
     rows = workloads.sampled_rows(w, seed=0)
     stats, _ = run_and_check(w, rows=rows)
     print(name, stats)
+
+
+def test_pass_events_time_each_pass():
+    """moba_set_pass_events: the events recorded between the passes of moba_attn_fwd
+    bracket the passes in order, and recording them changes no result."""
+    moba = _moba()
+    w = workloads.small_moba(batch=1, hq=4, hkv=2, seqlen=4096, d=128, block=256, topk=3)
+    q, k, v = (t.cuda() for t in workloads.make_inputs(w, 4))
+    r = moba.MobaPrefill(w.batch, w.hq, w.hkv, w.seqlen, w.d, w.block, w.topk)
+    o1, l1 = (t.clone() for t in r(q, k, v))
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    moba.set_pass_events(evs)
+    try:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        o2, l2 = r(q, k, v)
+        end.record()
+        torch.cuda.synchronize()
+    finally:
+        moba.set_pass_events(None)
+    assert moba.device_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    passes = [a.elapsed_time(b) for a, b in zip(evs[:-1], evs[1:])]
+    assert all(t > 0 for t in passes), passes
+    assert start.elapsed_time(evs[0]) >= 0 and evs[-1].elapsed_time(end) >= 0
+    assert sum(passes) <= start.elapsed_time(end) + 1e-3
