@@ -19,9 +19,9 @@ __device__ int g_device_status[2] = {MOBA_OK, 0};
 cudaError_t launch_pool(const uint16_t *k, int64_t sb, int64_t sh, int64_t sn, int batch, int hkv,
                         int N, int d, int block, float *kbar, uint16_t *split, cudaStream_t st);
 cudaError_t launch_gate(const SelectParams &p, cudaStream_t st);
-cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileoff, int4 *tiles,
-                        int nlists, cudaStream_t st);
-cudaError_t launch_scatter(const ScatterParams &p, cudaStream_t st);
+cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileoff, int nlists,
+                        cudaStream_t st);
+cudaError_t launch_scatter(ScatterParams p, cudaStream_t st);
 cudaError_t launch_gate_tc(const CUtensorMap *maps, const GateParams &p, int grid, cudaStream_t st);
 bool gate_tc_supports(int nblk, int topk);
 cudaError_t launch_attn(const CUtensorMap *maps, const AttnParams &p, int mode, int grid,
@@ -240,7 +240,8 @@ int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, i
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char *ws = static_cast<char *>(workspace);
   int *counts = reinterpret_cast<int *>(ws + w.off_counts);
-  if (cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)w.nlists, st) != cudaSuccess)
+  // The list counts and the tensor-core gate's tile counter after them.
+  if (cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)(w.nlists + 1), st) != cudaSuccess)
     return MOBA_ERR_LAUNCH;
   if (gate_tc_supports(w.nblk, topk)) {
     // Tensor-core gate: q tiles and the pooled keys through TMA.
@@ -259,6 +260,7 @@ int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, i
     if ((rc = status_words(&gp.status))) return rc;
     gp.idx = idx;
     gp.counts = counts;
+    gp.sched = counts + w.nlists;
     gp.batch = batch; gp.hq = hq; gp.hkv = hkv; gp.N = N; gp.d = d; gp.block = block;
     gp.topk = topk; gp.nblk = w.nblk; gp.G = w.G; gp.chunk_rows = w.chunk_rows;
     const long long tiles = (long long)batch * hkv * (N / kTileRows) * w.G;
@@ -280,9 +282,14 @@ int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, i
   int *listoff = reinterpret_cast<int *>(ws + w.off_listoff);
   int *tileoff = reinterpret_cast<int *>(ws + w.off_tileoff);
   int4 *tiles = reinterpret_cast<int4 *>(ws + w.off_tiles);
-  if ((rc = launch_status(launch_scan(counts, cursor, listoff, tileoff, tiles, w.nlists, st)))) return rc;
+  if ((rc = launch_status(launch_scan(counts, cursor, listoff, tileoff, w.nlists, st)))) return rc;
   ScatterParams cp{};
   cp.idx = idx;
+  cp.counts = counts;
+  cp.listoff = listoff;
+  cp.tileoff = tileoff;
+  cp.tiles = tiles;
+  cp.nlists = w.nlists;
   cp.cursor = cursor;
   cp.entries = reinterpret_cast<uint32_t *>(ws + w.off_entries);
   cp.batch = batch; cp.hq = hq; cp.hkv = hkv; cp.N = N; cp.block = block; cp.topk = topk;

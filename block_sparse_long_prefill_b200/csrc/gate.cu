@@ -8,11 +8,13 @@
 // highest scores.  §"인과성 보존": only blocks wholly before the query's own block
 // c = i / block compete (j < c), block c is always kept, later blocks never.
 //
-// It takes problems of at most 256 blocks and k - 1 <= kGateMaxPicks; the general
-// gate of select.cu takes the others.
-// One persistent CTA per SM walks a contiguous range of 128-row query tiles ordered
-// (batch, kv-head, row tile, q-head), so that the pooled keys of one kv-head are staged
-// in shared memory once per range.  Since block % 128 == 0, every row of a tile has the
+// It takes problems of at most 256 blocks with k - 1 <= kGateMaxPicks, and problems of
+// at most 33 blocks with any k (rank selection); the general gate of select.cu takes
+// the others.
+// One persistent CTA per SM takes chunks of consecutive 128-row query tiles, ordered
+// (batch, kv-head, row tile, q-head), from a global counter (the cost of a tile grows
+// with its row position, so a static split would leave SMs idle); the pooled keys of a
+// kv-head stay staged in shared memory while the CTA's tiles stay in that kv-head.  Since block % 128 == 0, every row of a tile has the
 // same own block c, and the tile needs the scores of blocks [0, c) only.
 //   warp 0     TMA producer: query tiles (a ring of up to eight) and, per kv-head, the
 //              pooled keys kbar = hi + lo (two bf16 matrices of up to 256 rows)
@@ -30,6 +32,8 @@
 #include <cuda.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "params.h"
 
@@ -37,14 +41,16 @@ namespace moba {
 
 constexpr int kGateTcThreads = 320;
 constexpr int kGateMaxBlocks = 256;   // pooled keys staged at once (MMA N <= 256)
-constexpr int kGateMaxPicks = 4;      // past blocks per row kept in the register list
+constexpr int kGateMaxPicks = 4;      // past blocks per row kept in the float list
+constexpr int kGateMaxList = 32;      // packed-key list length limit: k - 1 <= 31
 
 constexpr int kGateMaxStages = 8;     // query tile ring depth limit
 constexpr int kGateSmemLimit = 227 * 1024;
 
 // Shared memory: a ring of qst query tiles, the pooled keys hi and lo (kc16 rows each),
-// four per-warp pick histograms, barriers.  qst is chosen on the host to fill the
-// shared memory the staged pooled keys leave.
+// eight per-warp pick histograms, eight per-warp output staging areas (32 rows of str
+// words, str = topk | 1 so that the rows start in distinct banks), barriers.  qst is
+// chosen on the host to fill the shared memory the staged pooled keys leave.
 template <int D>
 struct GateCfg {
   static constexpr int QR0 = 128 * 128;                                // query region 0 bytes
@@ -57,17 +63,26 @@ struct GateCfg {
   }
   __host__ __device__ static constexpr int k_off(int qst) { return qst * QTILE; }
   __host__ __device__ static constexpr int hist_off(int qst, int kc16) { return k_off(qst) + 2 * kmat(kc16); }
-  __host__ __device__ static constexpr int bar_off(int qst, int kc16) {
+  __host__ __device__ static constexpr int stg_off(int qst, int kc16) {
     return hist_off(qst, kc16) + 8 * 4 * kGateMaxBlocks;
   }
-  __host__ __device__ static constexpr int smem(int qst, int kc16) { return bar_off(qst, kc16) + 512 + 1024; }
+  __host__ __device__ static constexpr int bar_off(int qst, int kc16, int str) {
+    return stg_off(qst, kc16) + ((8 * 32 * str * 4 + 15) & ~15);
+  }
+  __host__ __device__ static constexpr int smem(int qst, int kc16, int str) {
+    return bar_off(qst, kc16, str) + 512 + 1024;
+  }
 };
+
+constexpr int kGateSchedRing = 4;     // tile chunks handed from the producer to the others
 
 struct GateBars {
   uint64_t q_full[kGateMaxStages], q_empty[kGateMaxStages];
   uint64_t k_full, k_empty;
   uint64_t acc_full[2], acc_empty[2];
+  uint64_t sched_full[kGateSchedRing], sched_empty[kGateSchedRing];
   uint64_t mma_done;
+  int sched[kGateSchedRing];   // first tile of each handed-out chunk, -1 at the end
   uint32_t tmem_base;
   int abort;
 };
@@ -138,6 +153,113 @@ __device__ __forceinline__ void topk_insert(float (&val)[KM], int (&idx)[KM], fl
   }
 }
 
+// The k-1 best (score, block) pairs of one row over blocks [0, c), from the TMEM
+// accumulator row at `acc`, in the float list above.
+template <int KM>
+__device__ __forceinline__ void topk_scan(uint32_t acc, int c, int npick, float (&val)[KM],
+                                          int (&idx)[KM]) {
+#pragma unroll
+  for (int e = 0; e < KM; ++e) {
+    val[e] = (e < npick) ? -INFINITY : INFINITY;
+    idx[e] = -1;
+  }
+  for (int j0 = 0; j0 < c; j0 += 32) {
+    uint32_t sc[32];
+    tmem_ld32(acc + j0, sc);
+    tmem_wait_ld();
+    // Every score goes through the short list, with no branch.
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      topk_insert<KM>(val, idx, (j0 + e < c) ? __uint_as_float(sc[e]) : -INFINITY, j0 + e);
+  }
+}
+
+// Insertion of key v into the descending list L of packed keys: two unsigned min / max
+// per entry.  Entries past the npick + 1 in use hold all ones and are never displaced.
+template <int KM, typename K>
+__device__ __forceinline__ void packed_insert(K (&L)[KM], K v) {
+#pragma unroll
+  for (int e = 0; e < KM; ++e) {
+    const K hi = max(L[e], v);
+    v = min(L[e], v);
+    L[e] = hi;
+  }
+}
+
+// Sorting networks on packed keys (one unsigned min and max per comparator).
+// Batcher's odd-even merge sort of W keys, as a comparator list built at compile time
+// (so that every index is a constant once the loop over it is unrolled).
+template <int W>
+struct SortNet {
+  int lo[W * W], hi[W * W];
+  int n;
+  constexpr SortNet() : lo(), hi(), n(0) {
+    for (int p = 1; p < W; p *= 2)
+      for (int k = p; k >= 1; k /= 2)
+        for (int j = k % p; j + k < W; j += 2 * k)
+          for (int i = 0; i < k; ++i)
+            if (i + j + k < W && (i + j) / (2 * p) == (i + j + k) / (2 * p)) {
+              lo[n] = i + j;
+              hi[n] = i + j + k;
+              ++n;
+            }
+  }
+};
+
+// B := B in ascending order.
+template <int W>
+__device__ __forceinline__ void sort_asc(uint32_t (&B)[W]) {
+  constexpr SortNet<W> net;
+#pragma unroll
+  for (int t = 0; t < net.n; ++t) {
+    const uint32_t a = B[net.lo[t]], b = B[net.hi[t]];
+    B[net.lo[t]] = min(a, b);
+    B[net.hi[t]] = max(a, b);
+  }
+}
+
+// L (W keys, descending) := the W greatest of L and the batch B (W keys, ascending):
+// the element-wise maximum of a descending and an ascending sequence is bitonic and
+// holds the W greatest; half-cleaners then sort it descending.
+template <int W>
+__device__ __forceinline__ void merge_top(uint32_t (&L)[W], const uint32_t (&B)[W]) {
+#pragma unroll
+  for (int e = 0; e < W; ++e) L[e] = max(L[e], B[e]);
+#pragma unroll
+  for (int k = W / 2; k >= 1; k /= 2) {
+#pragma unroll
+    for (int i = 0; i < W; ++i) {
+      if ((i & k) == 0) {
+        const uint32_t a = L[i], b = L[i + k];
+        L[i] = max(a, b);
+        L[i + k] = min(a, b);
+      }
+    }
+  }
+}
+
+// The scores of blocks j0 .. j0 + 15 (raw fp32 bits in s) into the list L, KM at a time:
+// packed keys (blocks at or after c: key 0, never kept), a sort, a merge.
+template <int KM>
+__device__ __forceinline__ void net_batches(uint32_t (&L)[KM], const uint32_t (&s)[16], int j0,
+                                            int c, uint32_t imask) {
+  const uint32_t jb = imask - (uint32_t)j0;
+#pragma unroll
+  for (int h = 0; h < 16; h += KM) {
+    if (j0 + h < c) {
+      uint32_t B[KM];
+#pragma unroll
+      for (int e = 0; e < KM; ++e) {
+        const uint32_t b = s[h + e];
+        const uint32_t ord = b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
+        B[e] = (j0 + h + e < c) ? ((ord & ~imask) | (jb - (uint32_t)(h + e))) : 0u;
+      }
+      sort_asc<KM>(B);
+      merge_top<KM>(L, B);
+    }
+  }
+}
+
 template <int D, int KM>
 __global__ void __launch_bounds__(kGateTcThreads, 1)
 gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ1,
@@ -153,17 +275,18 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int qst = p.qstages;
   const int kmat = C::kmat(kc16);
   const int k_off = C::k_off(qst);
-  GateBars &bar = *reinterpret_cast<GateBars *>(sbase + C::bar_off(qst, kc16));
+  const int str = p.topk | 1;
+  GateBars &bar = *reinterpret_cast<GateBars *>(sbase + C::bar_off(qst, kc16, str));
   int *hist = reinterpret_cast<int *>(sbase + C::hist_off(qst, kc16));
+  int *stg_all = reinterpret_cast<int *>(sbase + C::stg_off(qst, kc16));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int site0 = (3 * 16 + (D == 64 ? 0 : (D == 80 ? 1 : 2))) * 256;
   constexpr uint32_t FULL = 0xffffffffu;
 
-  // This CTA's contiguous tile range.
+  // Tiles are handed out in chunks of p.chunk_tiles consecutive tiles from a global
+  // counter: the producer takes a chunk and passes its first tile through the sched
+  // ring to the MMA issuer and the top-k warps, which walk the same tiles in order.
   const int ntiles = p.batch * p.hkv * (p.N / 128) * p.G;
-  const int per = (ntiles + gridDim.x - 1) / gridDim.x;
-  const int t_begin = blockIdx.x * per;
-  const int t_end = min(ntiles, t_begin + per);
 
   if (tid == 0) {
     for (int s = 0; s < qst; ++s) {
@@ -173,6 +296,10 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar.acc_full[s], 1);
       mbar_init(&bar.acc_empty[s], 4);
+    }
+    for (int s = 0; s < kGateSchedRing; ++s) {
+      mbar_init(&bar.sched_full[s], 1);
+      mbar_init(&bar.sched_empty[s], 9);   // the MMA issuer and the eight top-k warps
     }
     mbar_init(&bar.k_full, 1);
     mbar_init(&bar.k_empty, 1);
@@ -194,6 +321,13 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
   volatile int *abort = &bar.abort;
+  // The first tile of chunk kq of this CTA (-1: no more tiles), or -1 with ok = false
+  // when the wait gave up.
+  auto take_chunk = [&](uint32_t kq, int site, bool &ok) -> int {
+    const int slot = kq % kGateSchedRing;
+    ok = mbar_wait(&bar.sched_full[slot], (kq / kGateSchedRing) & 1, abort, p.status, site);
+    return ok ? *reinterpret_cast<volatile int *>(&bar.sched[slot]) : -1;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -201,8 +335,19 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool ok = true;
       int cur = -1;
       uint32_t kuse = 0, quse = 0;
-      GateTile gt = gate_tile(p, t_begin);
-      for (int t = t_begin; ok && t < t_end; ++t, gate_tile_next(p, gt)) {
+      for (uint32_t kq = 0; ok; ++kq) {
+        // Take the next chunk and hand it on.
+        int start = atomicAdd(p.sched, p.chunk_tiles);
+        if (start >= ntiles) start = -1;
+        const int slot = kq % kGateSchedRing;
+        if (!(ok = mbar_wait(&bar.sched_empty[slot], ((kq / kGateSchedRing) & 1) ^ 1, abort, p.status,
+                             site0 + 7))) break;
+        *reinterpret_cast<volatile int *>(&bar.sched[slot]) = start;
+        mbar_arrive(&bar.sched_full[slot]);
+        if (start < 0) break;
+        const int end = min(start + p.chunk_tiles, ntiles);
+        GateTile gt = gate_tile(p, start);
+      for (int t = start; ok && t < end; ++t, gate_tile_next(p, gt)) {
         const int grp = gt.b * p.hkv + gt.hk;
         if (grp != cur) {
           cur = grp;
@@ -226,6 +371,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (D != 64) tma_load_4d(qd + C::QR0, &tmQ1, &bar.q_full[s], 64, gt.rt * 128, h, gt.b);
         ++quse;
       }
+      }
       if (*abort) {
         // Let issued loads land before the CTA can retire.
         const unsigned long long t0 = global_timer_ns();
@@ -240,10 +386,17 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool ok = true;
       int cur = -1;
       uint32_t kuse = 0, quse = 0, ause = 0;
-      GateTile gt = gate_tile(p, t_begin);
-      for (int t = t_begin; ok && t < t_end; ++t, gate_tile_next(p, gt)) {
+      for (uint32_t kq = 0; ok; ++kq) {
+        const int start = take_chunk(kq, site0 + 8, ok);
+        if (ok) mbar_arrive(&bar.sched_empty[kq % kGateSchedRing]);
+        if (!ok || start < 0) break;
+        const int end = min(start + p.chunk_tiles, ntiles);
+        GateTile gt = gate_tile(p, start);
+      for (int t = start; ok && t < end; ++t, gate_tile_next(p, gt)) {
         const int grp = gt.b * p.hkv + gt.hk;
         if (grp != cur) {
+          // The staged pooled keys may be replaced once the MMAs issued so far are done.
+          if (cur >= 0) umma_commit(&bar.k_empty);
           cur = grp;
           if (!(ok = mbar_wait(&bar.k_full, kuse & 1, abort, p.status, site0 + 3))) break;
           ++kuse;
@@ -270,11 +423,9 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         umma_commit(&bar.acc_full[a]);
         umma_commit(&bar.q_empty[s]);
-        // Last tile of this kv-head in the range: the pooled keys may be replaced.
-        const bool last = (t + 1 == t_end) || (gt.g == p.G - 1 && gt.rt == p.N / 128 - 1);
-        if (last) umma_commit(&bar.k_empty);
         ++quse;
         ++ause;
+      }
       }
       umma_commit(&bar.mma_done);
       const unsigned long long t0 = global_timer_ns();
@@ -286,12 +437,20 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // list counts when its rows move to another (chunk, batch, kv-head) list, so no
     // barrier across warps is needed.
     // Two groups of four warps take the tiles in turn: group gi (warps 2-5 or 6-9)
-    // reads accumulator gi and handles tiles t_begin + gi, t_begin + gi + 2, ...
+    // reads accumulator gi and handles the CTA's tiles u = gi, gi + 2, ...
     const int gi = (warp - 2) >> 2;
     const int r = 32 * (warp & 3) + lane;                  // row within the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     int *whist = hist + (warp - 2) * kGateMaxBlocks;
+    // The warp's 32 output rows are staged here, then written as one contiguous run of
+    // 32 * topk words with coalesced stores.
+    int *stg = stg_all + (warp - 2) * 32 * str;
+    int *orow = stg + lane * str;
+    const int r0 = lane / p.topk, s0 = lane - r0 * p.topk;
+    const int dq = 32 / p.topk, dr = 32 - dq * p.topk;
     const int npast = p.topk - 1;
+    // Low key bits that carry the block index of a packed key.
+    const uint32_t imask = (1u << (32 - __clz(max(p.nblk - 1, 1)))) - 1u;
     bool ok = true;
     uint32_t ause = 0;
     int cur_list = -1;
@@ -306,9 +465,16 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       __syncwarp();
     };
-    GateTile gt = gate_tile(p, t_begin);
-    if (gi) gate_tile_next(p, gt);
-    for (int t = t_begin + gi; ok && t < t_end; t += 2, gate_tile_next(p, gt), gate_tile_next(p, gt)) {
+    uint32_t u = 0;                                        // tile number within this CTA
+    for (uint32_t kq = 0; ok; ++kq) {
+      const int start = take_chunk(kq, site0 + 9, ok);
+      ok = __all_sync(FULL, ok);
+      if (ok && lane == 0) mbar_arrive(&bar.sched_empty[kq % kGateSchedRing]);
+      if (!ok || start < 0) break;
+      const int end = min(start + p.chunk_tiles, ntiles);
+      GateTile gt = gate_tile(p, start);
+    for (int t = start; ok && t < end; ++t, ++u, gate_tile_next(p, gt)) {
+      if ((int)(u & 1) != gi) continue;                    // the other group's tile
       const int i = gt.rt * 128 + r;
       const int c = gt.c;
       const int h = gt.hk * p.G + gt.g;
@@ -321,7 +487,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       ok = mbar_wait(&bar.acc_full[a], ause & 1, abort, p.status, site0 + 6);
       if (!(ok = __all_sync(FULL, ok))) break;
       tc_fence_after();
-      int32_t *orow = p.idx + (((int64_t)gt.b * p.hq + h) * p.N + i) * p.topk;
+      int32_t *gout = p.idx + (((int64_t)gt.b * p.hq + h) * p.N + (i - lane)) * p.topk;
       if (c <= npast || npast == 0) {
         // Every past block is kept (or none is asked for): no scores needed.
         tc_fence_before();
@@ -333,42 +499,135 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int j = 0; j < nk; ++j) whist[j] += 32;
       } else {
         const int npick = npast;                            // c > npast here
-        float val[KM];
-        int idx[KM];
-#pragma unroll
-        for (int e = 0; e < KM; ++e) {
-          val[e] = (e < npick) ? -INFINITY : INFINITY;
-          idx[e] = -1;
-        }
         const uint32_t acc = tmem + lane_off + 256 * a;
-        for (int j0 = 0; j0 < c; j0 += 32) {
-          uint32_t sc[32];
-          tmem_ld32(acc + j0, sc);
-          tmem_wait_ld();
-          // Every score goes through the short list, with no branch.
+        int pk[KM];                                         // the row's picks, any order
+        if constexpr (KM <= kGateMaxPicks) {
+          float val[KM];
+          int idx[KM];
+          topk_scan<KM>(acc, c, npick, val, idx);
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            topk_insert<KM>(val, idx, (j0 + e < c) ? __uint_as_float(sc[e]) : -INFINITY, j0 + e);
+          for (int e = 0; e < KM; ++e) pk[e] = idx[e];
+        } else {
+          // Packed keys: the order-preserving integer image of the score with its low
+          // index bits replaced by (imask - j), so that one unsigned comparison ranks a
+          // greater score first and, between equal truncated scores, the lower block.
+          uint32_t L[KM];
+          if constexpr (KM == 8 || KM == 16) {
+            // Batches of KM keys, sorted by a network and merged into the list; scores
+            // come in 16-column TMEM loads, the next one in flight during the sort.
+#pragma unroll
+            for (int e = 0; e < KM; ++e) L[e] = 0u;
+            uint32_t s0[16], s1[16];
+            tmem_ld16(acc, s0);
+            tmem_wait_ld();
+            for (int j0 = 0; j0 < c; j0 += 32) {
+              if (j0 + 16 < c) tmem_ld16(acc + j0 + 16, s1);
+              net_batches<KM>(L, s0, j0, c, imask);
+              tmem_wait_ld();
+              if (j0 + 16 < c) {
+                if (j0 + 32 < c) tmem_ld16(acc + j0 + 32, s0);
+                net_batches<KM>(L, s1, j0 + 16, c, imask);
+                tmem_wait_ld();
+              }
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < KM; ++e) L[e] = (e <= npick) ? 0u : 0xFFFFFFFFu;
+            for (int j0 = 0; j0 < c; j0 += 32) {
+              uint32_t sc[32];
+              tmem_ld32(acc + j0, sc);
+              tmem_wait_ld();
+              const uint32_t jb = imask - (uint32_t)j0;
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const uint32_t b = sc[e];
+                const uint32_t ord = b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
+                packed_insert<KM>(L, (j0 + e < c) ? ((ord & ~imask) | (jb - (uint32_t)e)) : 0u);
+              }
+            }
+          }
+          // L[0..npick] holds the npick + 1 greatest keys in descending order.  When the last
+          // kept and the first dropped key differ in their score bits, every kept score
+          // exceeds every dropped one and the choice is the exact one; otherwise the
+          // row is decided again on the full fp32 scores.
+          // (Written as a reduction over adjacent pairs: a select of L[npick] would
+          // index L at run time and move it to local memory.)
+          bool near_tie = false;
+#pragma unroll
+          for (int e = 0; e + 1 < KM; ++e)
+            near_tie |= (e + 1 == npick) & (((L[e] ^ L[e + 1]) & ~imask) == 0u);
+#pragma unroll
+          for (int e = 0; e < KM; ++e) pk[e] = (int)(imask - (L[e] & imask));
+          if (__any_sync(FULL, near_tie)) {
+            // The same scan on 64-bit keys: the full 32-bit score image above the block
+            // index, i.e. the exact rule (greater score first, then the lower block).
+            unsigned long long X[KM];
+#pragma unroll
+            for (int e = 0; e < KM; ++e) X[e] = (e < npick) ? 0ull : ~0ull;
+            for (int j0 = 0; j0 < c; j0 += 32) {
+              uint32_t sc[32];
+              tmem_ld32(acc + j0, sc);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const uint32_t b = sc[e];
+                const uint32_t ord = b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
+                const unsigned long long key =
+                    ((unsigned long long)ord << 32) | (0xFFFFFFFFu - (uint32_t)(j0 + e));
+                packed_insert<KM>(X, (j0 + e < c) ? key : 0ull);
+              }
+            }
+            if (near_tie) {
+#pragma unroll
+              for (int e = 0; e < KM; ++e) pk[e] = (int)(0xFFFFFFFFu - (uint32_t)X[e]);
+            }
+          }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar.acc_empty[a]);
-        // Ascending block order: each choice goes to its rank among the choices.
+        // Ascending block order.
+        if (c <= 64) {
+          unsigned long long m = 0;
 #pragma unroll
-        for (int e = 0; e < KM; ++e) {
-          if (e < npick) {
-            int rank = 0;
+          for (int e = 0; e < KM; ++e)
+            if (e < npick) m |= 1ull << pk[e];
+          for (int s = 0; s < npick; ++s) {
+            orow[s] = __ffsll((long long)m) - 1;
+            m &= m - 1;
+          }
+        } else {
 #pragma unroll
-            for (int f = 0; f < KM; ++f)
-              if (f < npick) rank += idx[f] < idx[e];
-            orow[rank] = idx[e];
-            atomicAdd(&whist[idx[e]], 1);
+          for (int e = 0; e < KM; ++e) {
+            if (e < npick) {
+              int rank = 0;
+#pragma unroll
+              for (int f = 0; f < KM; ++f)
+                if (f < npick) rank += pk[f] < pk[e];
+              orow[rank] = pk[e];
+            }
           }
         }
+#pragma unroll
+        for (int e = 0; e < KM; ++e)
+          if (e < npick && pk[e] >= 0) atomicAdd(&whist[pk[e]], 1);  // < 0 only for NaN scores
         orow[npick] = c;
         for (int s = npick + 1; s < p.topk; ++s) orow[s] = -1;
       }
+      // Staged rows -> idx: word w = 32 m + lane of the run is entry (r, s) of the warp.
+      __syncwarp();
+      {
+        int rr = r0, ss = s0;
+        for (int w = lane; w < 32 * p.topk; w += 32) {
+          gout[w] = stg[rr * str + ss];
+          rr += dq;
+          ss += dr;
+          if (ss >= p.topk) { ss -= p.topk; ++rr; }
+        }
+      }
+      __syncwarp();
       ++ause;
+    }
     }
     if (cur_list >= 0) flush(cur_list);
   }
@@ -384,16 +643,21 @@ template <int D, int KM>
 static cudaError_t launch_gate_tc_dk(const CUtensorMap *maps, GateParams p, int grid,
                                      cudaStream_t st) {
   using C = GateCfg<D>;
+  // About sixteen chunks per CTA.
+  const long long ntiles = (long long)p.batch * p.hkv * (p.N / 128) * p.G;
+  p.chunk_tiles = (int)std::max(1LL, std::min(32LL, ntiles / (16LL * grid)));
   auto kern = gate_tc_kernel<D, KM>;
   const int kc16 = (min(p.nblk, kGateMaxBlocks) + 15) & ~15;
   // As many query stages as the shared memory left by the pooled keys holds.
+  const int str = p.topk | 1;
   int qst = kGateMaxStages;
-  while (qst > 2 && C::smem(qst, kc16) > kGateSmemLimit) --qst;
-  if (C::smem(qst, kc16) > kGateSmemLimit) return cudaErrorInvalidConfiguration;
+  while (qst > 2 && C::smem(qst, kc16, str) > kGateSmemLimit) --qst;
+  if (C::smem(qst, kc16, str) > kGateSmemLimit) return cudaErrorInvalidConfiguration;
   p.qstages = qst;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem(qst, kc16));
+  const int bytes = C::smem(qst, kc16, str);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kGateTcThreads, C::smem(qst, kc16), st>>>(maps[0], maps[1], maps[2], maps[3], p);
+  kern<<<grid, kGateTcThreads, bytes, st>>>(maps[0], maps[1], maps[2], maps[3], p);
   return cudaGetLastError();
 }
 
@@ -403,6 +667,11 @@ static cudaError_t launch_gate_tc_d(const CUtensorMap *maps, const GateParams &p
   const int npast = p.topk - 1;
   if (npast <= 2) return launch_gate_tc_dk<D, 2>(maps, p, grid, st);
   if (npast <= kGateMaxPicks) return launch_gate_tc_dk<D, kGateMaxPicks>(maps, p, grid, st);
+  // Packed lists hold npast + 1 keys.
+  if (npast + 1 <= 8) return launch_gate_tc_dk<D, 8>(maps, p, grid, st);
+  if (npast + 1 <= 16) return launch_gate_tc_dk<D, 16>(maps, p, grid, st);
+  if (npast + 1 <= 24) return launch_gate_tc_dk<D, 24>(maps, p, grid, st);
+  if (npast + 1 <= kGateMaxList) return launch_gate_tc_dk<D, kGateMaxList>(maps, p, grid, st);
   return cudaErrorInvalidValue;
 }
 
@@ -418,7 +687,9 @@ cudaError_t launch_gate_tc(const CUtensorMap *maps, const GateParams &p, int gri
 }
 
 // Whether this kernel takes the problem: at most 256 pooled blocks (all staged at once)
-// and at most 4 past picks per row (a short register list scanned without branches).
-bool gate_tc_supports(int nblk, int topk) { return nblk <= kGateMaxBlocks && topk - 1 <= kGateMaxPicks; }
+// and at most 31 past picks per row (a register list scanned without branches).
+bool gate_tc_supports(int nblk, int topk) {
+  return nblk <= kGateMaxBlocks && topk - 1 < kGateMaxList;
+}
 
 }  // namespace moba

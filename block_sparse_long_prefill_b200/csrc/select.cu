@@ -273,12 +273,13 @@ gate_topk_kernel(const SelectParams p) {
 //
 // Exclusive prefix sums of the list counts (entries) and of their 256-entry units,
 // over all lists in (chunk, batch, kv-head, block) order; resets the scatter
-// cursors.  One CTA.
+// cursors.  One CTA.  (The unit table that these offsets index is written by the
+// scatter kernel's grid.)
 constexpr int kScanThreads = 1024;
 
 __global__ void __launch_bounds__(kScanThreads)
 list_scan_kernel(const int *__restrict__ counts, int *__restrict__ cursor, int *__restrict__ listoff,
-                 int *__restrict__ tileoff, int4 *__restrict__ tiles, int nlists) {
+                 int *__restrict__ tileoff, int nlists) {
   __shared__ int warp_e[32], warp_t[32];
   __shared__ int carry_e, carry_t;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -327,15 +328,6 @@ list_scan_kernel(const int *__restrict__ counts, int *__restrict__ cursor, int *
     listoff[nlists] = carry_e;
     tileoff[nlists] = carry_t;
   }
-  __syncthreads();
-  // Unit table: one {list, first entry, rows} record per unit of up to 256 entries
-  // (two 128-row tiles over the same block), so the attention kernel reads a unit's
-  // description with a single load.
-  for (int L = tid; L < nlists; L += kScanThreads) {
-    const int first = listoff[L], cnt = counts[L], t0 = tileoff[L];
-    for (int k = 0; k * kUnitRows < cnt; ++k)
-      tiles[t0 + k] = make_int4(L, first + k * kUnitRows, min(kUnitRows, cnt - k * kUnitRows), 0);
-  }
 }
 
 // ----------------------------------------------------------------- scatter
@@ -345,31 +337,69 @@ list_scan_kernel(const int *__restrict__ counts, int *__restrict__ cursor, int *
 // kv-head.  Entries of one CTA reserve their places with one atomic per block.
 // The order of entries inside a list is not fixed; no result depends on it (each
 // row's attention is computed independently of the rows sharing its tile).
+//
+// The CTA's block choices are read once into shared memory when they fit.
+// The grid also writes the unit table: one {list, first entry, rows} record per unit
+// of up to 256 entries (two 128-row tiles over the same block), so the attention
+// kernel reads a unit's description with a single load.
 constexpr int kScatterThreads = 256;
+constexpr size_t kScatterCacheBytes = 96 * 1024;
 
 __global__ void __launch_bounds__(kScatterThreads)
 scatter_kernel(const ScatterParams p) {
   extern __shared__ int sh[];
   int *hist = sh;             // [nblk]
   int *base = sh + p.nblk;    // [nblk]
+  int *picks = sh + 2 * p.nblk;  // [G][128][ps] when p.cache_rows (ps = topk | 1: rows of a
+                                 // warp start in distinct banks)
+  const int ps = p.topk | 1;
   const int i0 = blockIdx.x * kTileRows;
   const int hk = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x;
   const int npast = p.topk - 1;
   const int rows = min(kTileRows, p.N - i0);
   const int nb = min(p.nblk, (i0 + rows - 1) / p.block);
+
+  {
+    // Unit table, grid-stride over the lists.
+    const long long nthreads = (long long)gridDim.x * gridDim.y * gridDim.z * kScatterThreads;
+    const long long gtid =
+        (((long long)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * kScatterThreads + tid;
+    for (long long L = gtid; L < p.nlists; L += nthreads) {
+      const int first = p.listoff[L], cnt = p.counts[L], t0 = p.tileoff[L];
+      for (int k = 0; k * kUnitRows < cnt; ++k)
+        p.tiles[t0 + k] = make_int4((int)L, first + k * kUnitRows, min(kUnitRows, cnt - k * kUnitRows), 0);
+    }
+  }
+
   for (int j = tid; j < nb; j += kScatterThreads) hist[j] = 0;
+  const int64_t head0 = ((int64_t)b * p.hq + (int64_t)hk * p.G) * p.N + i0;  // row (b, hk*G, i0)
+  if (p.cache_rows) {
+    // Each head's rows i0 .. i0 + rows - 1 are one contiguous run of rows * topk words.
+    const int run = rows * p.topk;
+    for (int g = 0; g < p.G; ++g) {
+      const int32_t *src = p.idx + (head0 + (int64_t)g * p.N) * p.topk;
+      for (int e = tid; e < run; e += kScatterThreads) {
+        const int r = e / p.topk;
+        picks[(g * kTileRows + r) * ps + (e - r * p.topk)] = src[e];
+      }
+    }
+  }
   __syncthreads();
+  // Pair e = (g, r) of the tile; a warp holds 32 rows of one head (128 % 32 == 0).
   const int pairs = p.G * kTileRows;
+  auto pick = [&](int g, int r, int s) -> int {
+    return p.cache_rows ? picks[(g * kTileRows + r) * ps + s]
+                        : p.idx[(head0 + (int64_t)g * p.N + r) * p.topk + s];
+  };
   for (int e = tid; e < pairs; e += kScatterThreads) {
     const int g = e / kTileRows, r = e % kTileRows;
-    if (r >= rows) continue;
-    const int i = i0 + r;
-    const int c = i / p.block;
-    const int32_t *row = p.idx + (((int64_t)b * p.hq + hk * p.G + g) * p.N + i) * p.topk;
+    const bool row_ok = r < rows;
+    const int c = (i0 + r) / p.block;
     for (int s = 0; s < npast; ++s) {
-      const int j = row[s];
-      if (j < 0 || j >= c) break;  // own block (last) or padding
+      const int j = row_ok ? pick(g, r, s) : -1;
+      // Past picks come first; the own block and the -1 padding end them.
+      if (j < 0 || j >= c) break;
       atomicAdd(&hist[j], 1);
     }
   }
@@ -383,12 +413,11 @@ scatter_kernel(const ScatterParams p) {
   __syncthreads();
   for (int e = tid; e < pairs; e += kScatterThreads) {
     const int g = e / kTileRows, r = e % kTileRows;
-    if (r >= rows) continue;
+    const bool row_ok = r < rows;
     const int i = i0 + r;
     const int c = i / p.block;
-    const int32_t *row = p.idx + (((int64_t)b * p.hq + hk * p.G + g) * p.N + i) * p.topk;
     for (int s = 0; s < npast; ++s) {
-      const int j = row[s];
+      const int j = row_ok ? pick(g, r, s) : -1;
       if (j < 0 || j >= c) break;
       const int pos = base[j] + atomicAdd(&hist[j], 1);
       p.entries[pos] = (uint32_t)(((int64_t)i * p.G + g) * npast + s);
@@ -436,15 +465,22 @@ cudaError_t launch_gate(const SelectParams &p, cudaStream_t st) {
   }
 }
 
-cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileoff, int4 *tiles,
-                        int nlists, cudaStream_t st) {
-  list_scan_kernel<<<1, kScanThreads, 0, st>>>(counts, cursor, listoff, tileoff, tiles, nlists);
+cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileoff, int nlists,
+                        cudaStream_t st) {
+  list_scan_kernel<<<1, kScanThreads, 0, st>>>(counts, cursor, listoff, tileoff, nlists);
   return cudaGetLastError();
 }
 
-cudaError_t launch_scatter(const ScatterParams &p, cudaStream_t st) {
+cudaError_t launch_scatter(ScatterParams p, cudaStream_t st) {
   dim3 grid((p.N + kTileRows - 1) / kTileRows, p.hkv, p.batch);
-  const size_t smem = sizeof(int) * 2 * p.nblk;
+  const size_t cache = sizeof(int) * (size_t)p.G * kTileRows * (p.topk | 1);
+  p.cache_rows = cache <= kScatterCacheBytes ? 1 : 0;
+  const size_t smem = sizeof(int) * 2 * p.nblk + (p.cache_rows ? cache : 0);
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)smem);
+    if (e != cudaSuccess) return e;
+  }
   scatter_kernel<<<grid, kScatterThreads, smem, st>>>(p);
   return cudaGetLastError();
 }

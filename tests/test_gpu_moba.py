@@ -99,10 +99,13 @@ def test_moba_strided_inputs():
     ("many_blocks", dict(batch=1, hq=2, hkv=1, seqlen=65536, d=64, block=128, topk=4)),
     # exactly the tensor-core gate's block limit (256 blocks), d = 80, GQA.
     ("blocks256_d80", dict(batch=1, hq=4, hkv=2, seqlen=32768, d=80, block=128, topk=5)),
-    # long top-k lists (k - 1 > 4: the general gate), 128 / 256 / 64 blocks.
+    # long top-k lists (k - 1 > 4: packed-key lists), 128 / 256 / 64 blocks.
     ("k9_blocks128", dict(batch=1, hq=2, hkv=1, seqlen=16384, d=64, block=128, topk=9)),
     ("k13_blocks256", dict(batch=1, hq=2, hkv=2, seqlen=32768, d=128, block=128, topk=13)),
     ("k32_blocks64", dict(batch=1, hq=2, hkv=1, seqlen=8192, d=128, block=128, topk=32)),
+    # packed-key lists of 8 (k - 1 = 5) and 24 (k - 1 = 19) entries
+    ("k6_blocks64", dict(batch=1, hq=2, hkv=1, seqlen=8192, d=64, block=128, topk=6)),
+    ("k20_blocks64", dict(batch=1, hq=2, hkv=1, seqlen=8192, d=128, block=128, topk=20)),
 ])
 def test_moba_block_count_limits_sampled_rows(name, kw):
     w = workloads.small_moba(name=name, **kw)
@@ -145,3 +148,50 @@ def test_pass_events_time_each_pass():
     assert all(t > 0 for t in passes), passes
     assert start.elapsed_time(evs[0]) >= 0 and evs[-1].elapsed_time(end) >= 0
     assert sum(passes) <= start.elapsed_time(end) + 1e-3
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("float_list", dict(batch=1, hq=2, hkv=1, seqlen=8192, d=128, block=128, topk=4)),
+    ("packed12", dict(batch=1, hq=2, hkv=1, seqlen=8192, d=128, block=128, topk=10)),
+    ("packed16_d64", dict(batch=1, hq=2, hkv=2, seqlen=16384, d=64, block=128, topk=14)),
+])
+def test_moba_tied_blocks_keep_the_lower_block(name, kw):
+    """Blocks 2m and 2m+1 hold identical keys, so their gate scores are equal in every
+    precision and the top-k boundary often splits a pair.  The choice is then decided
+    by the lower block alone: it must equal the oracle's on every row whose boundary
+    score is clear (by 1e-3) of every score it does not equal."""
+    moba = _moba()
+    w = workloads.small_moba(name=name, **kw)
+    q, k, v = workloads.make_inputs(w, 7)
+    kb = k.view(w.batch, w.hkv, w.seqlen // w.block, w.block, w.d)
+    kb[:, :, 1::2] = kb[:, :, 0::2]
+    runner = moba.MobaPrefill(w.batch, w.hq, w.hkv, w.seqlen, w.d, w.block, w.topk, w.window)
+    runner(q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    assert moba.device_status() == 0
+    rows = np.arange(w.seqlen, dtype=np.int32)
+    kbar_o = oracle.pool_keys(k, w.block)
+    scores = oracle.gate_scores(q, kbar_o, w.block, rows)
+    idx_o, _ = oracle.select_topk(scores, w.seqlen, w.block, w.topk, rows)
+    idx_g = rows_of(runner.idx, rows)
+    npast = w.topk - 1
+    checked = split = 0
+    for bb in range(w.batch):
+        for hh in range(w.hq):
+            for r in rows:
+                c = int(r) // w.block
+                if c <= npast:
+                    assert np.array_equal(idx_g[bb, hh, r], idx_o[bb, hh, r])
+                    continue
+                s = scores[bb, hh, r, :c]
+                past = [int(x) for x in idx_o[bb, hh, r] if 0 <= x < c]
+                vb = min(s[j] for j in past)
+                others = s[s != vb]
+                if others.size and np.abs(others - vb).min() <= 1e-3:
+                    continue
+                checked += 1
+                split += int(np.sum(s == vb) > sum(1 for j in past if s[j] == vb))
+                assert np.array_equal(idx_g[bb, hh, r], idx_o[bb, hh, r]), (bb, hh, r)
+    assert checked > 0.9 * w.batch * w.hq * (w.seqlen - (npast + 1) * w.block)
+    assert split > 100  # the boundary splits a tied pair on many rows
+    print(name, "checked", checked, "split pairs", split)
