@@ -350,9 +350,13 @@ def run_ours(args, rank, world, device):
                 layout_chunks = math.ceil(w.seqlen / chunk_rows)
         except ZeroDivisionError:
             pass
-        # pool, gate (+ scan, scatter), and per query chunk: past-block pass, own-block
-        # pass, merge (only the own-block pass when topk = 1).
-        launches_per_step = 2 + (2 if w.topk > 1 else 0) + layout_chunks * (3 if w.topk > 1 else 1)
+        # pool, gate, scatter (+ a scan launch when the general gate runs: the
+        # tensor-core gate's last CTA writes the list offsets itself), and per query
+        # chunk: past-block pass, own-block pass, merge (only the own-block pass when
+        # topk = 1).
+        tc_gate = w.seqlen // w.block <= 256 and w.topk - 1 < 32
+        launches_per_step = (2 + ((1 if tc_gate else 2) if w.topk > 1 else 0)
+                             + layout_chunks * (3 if w.topk > 1 else 1))
     else:
         out_t = torch.empty_like(qd)
         lse_t = torch.empty(w.batch, w.hq, w.seqlen, dtype=torch.float32, device=device)

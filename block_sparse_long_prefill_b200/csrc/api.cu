@@ -240,9 +240,14 @@ int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, i
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char *ws = static_cast<char *>(workspace);
   int *counts = reinterpret_cast<int *>(ws + w.off_counts);
-  // The list counts and the tensor-core gate's tile counter after them.
-  if (cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)(w.nlists + 1), st) != cudaSuccess)
+  // The list counts and the tensor-core gate's two counters after them.
+  if (cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)(w.nlists + 2), st) != cudaSuccess)
     return MOBA_ERR_LAUNCH;
+  int *cursor = reinterpret_cast<int *>(ws + w.off_cursor);
+  int *listoff = reinterpret_cast<int *>(ws + w.off_listoff);
+  int *tileoff = reinterpret_cast<int *>(ws + w.off_tileoff);
+  int4 *tiles = reinterpret_cast<int4 *>(ws + w.off_tiles);
+  bool scanned = false;  // list offsets already written by the gate kernel
   if (gate_tc_supports(w.nblk, topk)) {
     // Tensor-core gate: q tiles and the pooled keys through TMA.
     int nsm = 0;
@@ -261,10 +266,15 @@ int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, i
     gp.idx = idx;
     gp.counts = counts;
     gp.sched = counts + w.nlists;
+    if (w.npast > 0) {
+      gp.done = counts + w.nlists + 1;
+      gp.cursor = cursor; gp.listoff = listoff; gp.tileoff = tileoff; gp.nlists = w.nlists;
+      scanned = true;
+    }
     gp.batch = batch; gp.hq = hq; gp.hkv = hkv; gp.N = N; gp.d = d; gp.block = block;
     gp.topk = topk; gp.nblk = w.nblk; gp.G = w.G; gp.chunk_rows = w.chunk_rows;
-    const long long tiles = (long long)batch * hkv * (N / kTileRows) * w.G;
-    const int grid = (int)(tiles < nsm ? tiles : nsm);
+    const long long ntiles = (long long)batch * hkv * (N / kTileRows) * w.G;
+    const int grid = (int)(ntiles < nsm ? ntiles : nsm);
     if ((rc = launch_status(launch_gate_tc(maps, gp, grid, st)))) return rc;
   } else {
     SelectParams sp{};
@@ -278,11 +288,8 @@ int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, i
     if ((rc = launch_status(launch_gate(sp, st)))) return rc;
   }
   if (w.npast == 0) return MOBA_OK;
-  int *cursor = reinterpret_cast<int *>(ws + w.off_cursor);
-  int *listoff = reinterpret_cast<int *>(ws + w.off_listoff);
-  int *tileoff = reinterpret_cast<int *>(ws + w.off_tileoff);
-  int4 *tiles = reinterpret_cast<int4 *>(ws + w.off_tiles);
-  if ((rc = launch_status(launch_scan(counts, cursor, listoff, tileoff, w.nlists, st)))) return rc;
+  if (!scanned && (rc = launch_status(launch_scan(counts, cursor, listoff, tileoff, w.nlists, st))))
+    return rc;
   ScatterParams cp{};
   cp.idx = idx;
   cp.counts = counts;

@@ -19,7 +19,7 @@
 //   warp 0     TMA producer: query tiles (a ring of up to eight) and, per kv-head, the
 //              pooled keys kbar = hi + lo (two bf16 matrices of up to 256 rows)
 //   warp 1     tcgen05 MMA issuer and TMEM owner: S = Q hi^T + Q lo^T in fp32, into
-//              one of two TMEM accumulators (N = c rounded up to 16 columns)
+//              one of 2-4 TMEM accumulators (N = c rounded up to 16 columns)
 //   warps 2-9  top-k, two groups of four warps taking the tiles (and accumulators) in
 //              turn: thread r owns row r (TMEM lane r) and scans its c scores in
 //              ascending block order, keeping the best k-1 (at most kGateMaxPicks) in
@@ -35,6 +35,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "lists.cuh"
 #include "params.h"
 
 namespace moba {
@@ -62,24 +63,28 @@ struct GateCfg {
     return kc16 * 128 + ((kc16 * R1ROW + 1023) / 1024) * 1024;
   }
   __host__ __device__ static constexpr int k_off(int qst) { return qst * QTILE; }
-  __host__ __device__ static constexpr int hist_off(int qst, int kc16) { return k_off(qst) + 2 * kmat(kc16); }
-  __host__ __device__ static constexpr int stg_off(int qst, int kc16) {
-    return hist_off(qst, kc16) + 8 * 4 * kGateMaxBlocks;
+  // ks staging slots for the pooled keys, each holding hi and lo.
+  __host__ __device__ static constexpr int hist_off(int qst, int kc16, int ks) {
+    return k_off(qst) + ks * 2 * kmat(kc16);
   }
-  __host__ __device__ static constexpr int bar_off(int qst, int kc16, int str) {
-    return stg_off(qst, kc16) + ((8 * 32 * str * 4 + 15) & ~15);
+  __host__ __device__ static constexpr int stg_off(int qst, int kc16, int ks) {
+    return hist_off(qst, kc16, ks) + 8 * 4 * kGateMaxBlocks;
   }
-  __host__ __device__ static constexpr int smem(int qst, int kc16, int str) {
-    return bar_off(qst, kc16, str) + 512 + 1024;
+  __host__ __device__ static constexpr int bar_off(int qst, int kc16, int ks, int str) {
+    return stg_off(qst, kc16, ks) + ((8 * 32 * str * 4 + 15) & ~15);
+  }
+  __host__ __device__ static constexpr int smem(int qst, int kc16, int ks, int str) {
+    return bar_off(qst, kc16, ks, str) + 512 + 1024;
   }
 };
 
 constexpr int kGateSchedRing = 4;     // tile chunks handed from the producer to the others
+constexpr int kGateMaxAcc = 4;        // TMEM accumulators (score tiles in flight)
 
 struct GateBars {
   uint64_t q_full[kGateMaxStages], q_empty[kGateMaxStages];
-  uint64_t k_full, k_empty;
-  uint64_t acc_full[2], acc_empty[2];
+  uint64_t k_full[2], k_empty[2];
+  uint64_t acc_full[kGateMaxAcc], acc_empty[kGateMaxAcc];
   uint64_t sched_full[kGateSchedRing], sched_empty[kGateSchedRing];
   uint64_t mma_done;
   int sched[kGateSchedRing];   // first tile of each handed-out chunk, -1 at the end
@@ -276,9 +281,15 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int kmat = C::kmat(kc16);
   const int k_off = C::k_off(qst);
   const int str = p.topk | 1;
-  GateBars &bar = *reinterpret_cast<GateBars *>(sbase + C::bar_off(qst, kc16, str));
-  int *hist = reinterpret_cast<int *>(sbase + C::hist_off(qst, kc16));
-  int *stg_all = reinterpret_cast<int *>(sbase + C::stg_off(qst, kc16));
+  // TMEM accumulators of accw columns (a power of two >= kc16) share the 512 columns:
+  // tile u of the CTA uses accumulator u % nacc (nacc even, so a group's tiles never
+  // use the other group's accumulators).
+  const int accw = kc16 <= 32 ? 32 : (kc16 <= 64 ? 64 : (kc16 <= 128 ? 128 : 256));
+  const int nacc = min(kGateMaxAcc, 512 / accw);
+  const int ks = p.kslots;
+  GateBars &bar = *reinterpret_cast<GateBars *>(sbase + C::bar_off(qst, kc16, ks, str));
+  int *hist = reinterpret_cast<int *>(sbase + C::hist_off(qst, kc16, ks));
+  int *stg_all = reinterpret_cast<int *>(sbase + C::stg_off(qst, kc16, ks));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int site0 = (3 * 16 + (D == 64 ? 0 : (D == 80 ? 1 : 2))) * 256;
   constexpr uint32_t FULL = 0xffffffffu;
@@ -293,7 +304,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(&bar.q_full[s], 1);
       mbar_init(&bar.q_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kGateMaxAcc; ++s) {
       mbar_init(&bar.acc_full[s], 1);
       mbar_init(&bar.acc_empty[s], 4);
     }
@@ -301,8 +312,10 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(&bar.sched_full[s], 1);
       mbar_init(&bar.sched_empty[s], 9);   // the MMA issuer and the eight top-k warps
     }
-    mbar_init(&bar.k_full, 1);
-    mbar_init(&bar.k_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar.k_full[s], 1);
+      mbar_init(&bar.k_empty[s], 1);
+    }
     mbar_init(&bar.mma_done, 1);
     bar.abort = 0;
     fence_barrier_init();
@@ -335,10 +348,13 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool ok = true;
       int cur = -1;
       uint32_t kuse = 0, quse = 0;
+      // The counter is read one chunk ahead, so its latency overlaps a chunk's loads.
+      int next = atomicAdd(p.sched, p.chunk_tiles);
       for (uint32_t kq = 0; ok; ++kq) {
-        // Take the next chunk and hand it on.
-        int start = atomicAdd(p.sched, p.chunk_tiles);
+        // Hand on the chunk taken last time, take the following one.
+        int start = next;
         if (start >= ntiles) start = -1;
+        else next = atomicAdd(p.sched, p.chunk_tiles);
         const int slot = kq % kGateSchedRing;
         if (!(ok = mbar_wait(&bar.sched_empty[slot], ((kq / kGateSchedRing) & 1) ^ 1, abort, p.status,
                              site0 + 7))) break;
@@ -351,15 +367,19 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int grp = gt.b * p.hkv + gt.hk;
         if (grp != cur) {
           cur = grp;
-          if (!(ok = mbar_wait(&bar.k_empty, (kuse & 1) ^ 1, abort, p.status, site0 + 1))) break;
+          // Slot kuse % ks; with two slots the next kv-head's keys load while the
+          // MMAs of the current one still run.
+          const int ksl = kuse % ks;
+          if (!(ok = mbar_wait(&bar.k_empty[ksl], ((kuse / ks) & 1) ^ 1, abort, p.status, site0 + 1)))
+            break;
           ++kuse;
           const uint32_t kbytes = 2u * (uint32_t)kc16 * (uint32_t)D * 2u;
-          mbar_arrive_expect_tx(&bar.k_full, kbytes);
+          mbar_arrive_expect_tx(&bar.k_full[ksl], kbytes);
           for (int part = 0; part < 2; ++part) {
-            unsigned char *kd = sbase + k_off + part * kmat;
+            unsigned char *kd = sbase + k_off + (ksl * 2 + part) * kmat;
             const int plane = grp * 2 + part;
-            tma_load_3d(kd, &tmK, &bar.k_full, 0, 0, plane);
-            if (D != 64) tma_load_3d(kd + kc16 * 128, &tmK1, &bar.k_full, 64, 0, plane);
+            tma_load_3d(kd, &tmK, &bar.k_full[ksl], 0, 0, plane);
+            if (D != 64) tma_load_3d(kd + kc16 * 128, &tmK1, &bar.k_full[ksl], 64, 0, plane);
           }
         }
         const int s = quse % qst;
@@ -377,7 +397,8 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const unsigned long long t0 = global_timer_ns();
         for (uint32_t u = (quse > (uint32_t)qst ? quse - qst : 0u); u < quse; ++u)
           while (!mbar_try_wait(&bar.q_full[u % qst], (u / qst) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
-        while (kuse > 0 && !mbar_try_wait(&bar.k_full, (kuse - 1) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+        for (uint32_t u = (kuse > (uint32_t)ks ? kuse - ks : 0u); u < kuse; ++u)
+          while (!mbar_try_wait(&bar.k_full[u % ks], (u / ks) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
       }
     }
   } else if (warp == 1) {
@@ -386,6 +407,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool ok = true;
       int cur = -1;
       uint32_t kuse = 0, quse = 0, ause = 0;
+      uint32_t kslot = base + k_off;                        // staged keys in use
       for (uint32_t kq = 0; ok; ++kq) {
         const int start = take_chunk(kq, site0 + 8, ok);
         if (ok) mbar_arrive(&bar.sched_empty[kq % kGateSchedRing]);
@@ -395,15 +417,18 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int t = start; ok && t < end; ++t, gate_tile_next(p, gt)) {
         const int grp = gt.b * p.hkv + gt.hk;
         if (grp != cur) {
-          // The staged pooled keys may be replaced once the MMAs issued so far are done.
-          if (cur >= 0) umma_commit(&bar.k_empty);
+          // The slot in use may be refilled once the MMAs issued so far are done.
+          if (cur >= 0) umma_commit(&bar.k_empty[(kuse - 1) % ks]);
           cur = grp;
-          if (!(ok = mbar_wait(&bar.k_full, kuse & 1, abort, p.status, site0 + 3))) break;
+          const int ksl = kuse % ks;
+          if (!(ok = mbar_wait(&bar.k_full[ksl], (kuse / ks) & 1, abort, p.status, site0 + 3))) break;
           ++kuse;
+          kslot = base + k_off + ksl * 2 * kmat;
         }
-        const int s = quse % qst, a = ause & 1;
+        const int s = quse % qst, a = ause % nacc;
         if (!(ok = mbar_wait(&bar.q_full[s], (quse / qst) & 1, abort, p.status, site0 + 4))) break;
-        if (!(ok = mbar_wait(&bar.acc_empty[a], ((ause >> 1) & 1) ^ 1, abort, p.status, site0 + 5))) break;
+        if (!(ok = mbar_wait(&bar.acc_empty[a], ((ause / nacc) & 1) ^ 1, abort, p.status, site0 + 5)))
+          break;
         tc_fence_after();
         const int c = gt.c;                                 // own block of every row
         // Score columns needed (none when every past block is kept anyway).
@@ -411,10 +436,10 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (nn > 0) {
           const uint32_t idesc = idesc_bf16(128, nn, 0, 0);
           const uint32_t qt = base + s * C::QTILE;
-          const uint32_t acc = tmem + 256 * a;
+          const uint32_t acc = tmem + accw * a;
 #pragma unroll
           for (int part = 0; part < 2; ++part) {
-            const uint32_t kt = base + k_off + part * kmat;
+            const uint32_t kt = kslot + part * kmat;
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks)
               umma_ss(acc, gate_desc<D>(qt, ks, 128), gate_desc<D>(kt, ks, kc16), idesc,
@@ -437,7 +462,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // list counts when its rows move to another (chunk, batch, kv-head) list, so no
     // barrier across warps is needed.
     // Two groups of four warps take the tiles in turn: group gi (warps 2-5 or 6-9)
-    // reads accumulator gi and handles the CTA's tiles u = gi, gi + 2, ...
+    // handles the CTA's tiles u = gi, gi + 2, ... (accumulator u % nacc).
     const int gi = (warp - 2) >> 2;
     const int r = 32 * (warp & 3) + lane;                  // row within the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
@@ -452,7 +477,6 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // Low key bits that carry the block index of a packed key.
     const uint32_t imask = (1u << (32 - __clz(max(p.nblk - 1, 1)))) - 1u;
     bool ok = true;
-    uint32_t ause = 0;
     int cur_list = -1;
     auto flush = [&](int list) {
       __syncwarp();
@@ -478,13 +502,13 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int i = gt.rt * 128 + r;
       const int c = gt.c;
       const int h = gt.hk * p.G + gt.g;
-      const int a = gi;
+      const int a = u % nacc;
       const int list = (gt.chunk * p.batch + gt.b) * p.hkv + gt.hk;
       if (list != cur_list) {
         if (cur_list >= 0) flush(cur_list);
         cur_list = list;
       }
-      ok = mbar_wait(&bar.acc_full[a], ause & 1, abort, p.status, site0 + 6);
+      ok = mbar_wait(&bar.acc_full[a], (u / nacc) & 1, abort, p.status, site0 + 6);
       if (!(ok = __all_sync(FULL, ok))) break;
       tc_fence_after();
       int32_t *gout = p.idx + (((int64_t)gt.b * p.hq + h) * p.N + (i - lane)) * p.topk;
@@ -499,7 +523,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int j = 0; j < nk; ++j) whist[j] += 32;
       } else {
         const int npick = npast;                            // c > npast here
-        const uint32_t acc = tmem + lane_off + 256 * a;
+        const uint32_t acc = tmem + lane_off + accw * a;
         int pk[KM];                                         // the row's picks, any order
         if constexpr (KM <= kGateMaxPicks) {
           float val[KM];
@@ -626,7 +650,6 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
       }
       __syncwarp();
-      ++ause;
     }
     }
     if (cur_list >= 0) flush(cur_list);
@@ -634,27 +657,41 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   __syncwarp();
   tc_fence_before();
+  __threadfence();  // this thread's count atomics, before the CTA's ticket below
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, 512);
+  if (p.done != nullptr) {
+    // The last CTA to finish turns the list counts into list offsets.
+    int *ticket = hist + 64;  // the histograms are flushed and free
+    if (tid == 0) ticket[0] = atomicAdd(p.done, 1);
+    __syncthreads();
+    if (ticket[0] == (int)gridDim.x - 1) {
+      __threadfence();
+      scan_lists<kGateTcThreads>(p.counts, p.cursor, p.listoff, p.tileoff, p.nlists, hist);
+    }
+  }
 }
 
 template <int D, int KM>
 static cudaError_t launch_gate_tc_dk(const CUtensorMap *maps, GateParams p, int grid,
                                      cudaStream_t st) {
   using C = GateCfg<D>;
-  // About sixteen chunks per CTA.
+  // About eight chunks per CTA.
   const long long ntiles = (long long)p.batch * p.hkv * (p.N / 128) * p.G;
-  p.chunk_tiles = (int)std::max(1LL, std::min(32LL, ntiles / (16LL * grid)));
+  p.chunk_tiles = (int)std::max(1LL, std::min(32LL, ntiles / (8LL * grid)));
   auto kern = gate_tc_kernel<D, KM>;
   const int kc16 = (min(p.nblk, kGateMaxBlocks) + 15) & ~15;
-  // As many query stages as the shared memory left by the pooled keys holds.
   const int str = p.topk | 1;
+  // Two pooled-key slots when they leave room for three query stages; then as many
+  // query stages as the shared memory holds.
+  const int ks = C::smem(3, kc16, 2, str) <= kGateSmemLimit ? 2 : 1;
   int qst = kGateMaxStages;
-  while (qst > 2 && C::smem(qst, kc16, str) > kGateSmemLimit) --qst;
-  if (C::smem(qst, kc16, str) > kGateSmemLimit) return cudaErrorInvalidConfiguration;
+  while (qst > 2 && C::smem(qst, kc16, ks, str) > kGateSmemLimit) --qst;
+  if (C::smem(qst, kc16, ks, str) > kGateSmemLimit) return cudaErrorInvalidConfiguration;
   p.qstages = qst;
-  const int bytes = C::smem(qst, kc16, str);
+  p.kslots = ks;
+  const int bytes = C::smem(qst, kc16, ks, str);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, kGateTcThreads, bytes, st>>>(maps[0], maps[1], maps[2], maps[3], p);

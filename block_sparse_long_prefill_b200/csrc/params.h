@@ -23,8 +23,8 @@ struct WorkspaceLayout {
   int chunk_rows;   // query rows per pass (multiple of 128)
   int nchunks;
   int nlists;       // nchunks * batch * hkv * nblk
-  size_t off_counts;   // int32 [nlists + 1]   entries per list (atomic counts), then the
-                       //                      gate's tile counter
+  size_t off_counts;   // int32 [nlists + 2]   entries per list (atomic counts), then the
+                       //                      gate's tile counter and finished-CTA count
   size_t off_cursor;   // int32 [nlists]       scatter cursors
   size_t off_listoff;  // int32 [nlists + 1]   exclusive prefix of counts
   size_t off_tileoff;  // int32 [nlists + 1]   exclusive prefix of ceil(count / 256)
@@ -60,7 +60,7 @@ inline WorkspaceLayout make_layout(int batch, int hq, int hkv, int N, int d, int
   w.max_entries = static_cast<long long>(batch) * hq * N * w.npast;
   w.max_tiles = w.max_entries / kUnitRows + w.nlists + 1;
   size_t off = 0;
-  w.off_counts = off;  off = align_up(off + sizeof(int) * size_t(w.nlists + 1), 256);
+  w.off_counts = off;  off = align_up(off + sizeof(int) * size_t(w.nlists + 2), 256);
   w.off_cursor = off;  off = align_up(off + sizeof(int) * size_t(w.nlists), 256);
   w.off_listoff = off; off = align_up(off + sizeof(int) * size_t(w.nlists + 1), 256);
   w.off_tileoff = off; off = align_up(off + sizeof(int) * size_t(w.nlists + 1), 256);
@@ -91,8 +91,14 @@ struct GateParams {
   int *counts;           // workspace list counts
   int batch, hq, hkv, N, d, block, topk, nblk, G, chunk_rows;
   int qstages;           // query tile ring depth (set by the launcher)
+  int kslots;            // pooled-key staging slots, 1 or 2 (set by the launcher)
   int *sched;            // tile counter, zero at launch (the word after the list counts)
   int chunk_tiles;       // tiles per chunk taken from it (set by the launcher)
+  // When done is set (zero at launch, the second word after the counts), the last
+  // CTA to finish writes the list offsets (cursor, listoff, tileoff over nlists).
+  int *done;
+  int *cursor, *listoff, *tileoff;
+  int nlists;
 };
 
 struct ScatterParams {

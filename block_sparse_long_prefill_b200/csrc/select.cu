@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "lists.cuh"
 #include "params.h"
 
 namespace moba {
@@ -280,54 +281,8 @@ constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads)
 list_scan_kernel(const int *__restrict__ counts, int *__restrict__ cursor, int *__restrict__ listoff,
                  int *__restrict__ tileoff, int nlists) {
-  __shared__ int warp_e[32], warp_t[32];
-  __shared__ int carry_e, carry_t;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) { carry_e = 0; carry_t = 0; }
-  __syncthreads();
-  for (int base = 0; base < nlists; base += kScanThreads) {
-    const int L = base + tid;
-    const int ce = (L < nlists) ? counts[L] : 0;
-    const int ct = (ce + kUnitRows - 1) / kUnitRows;
-    int se = ce, st = ct;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int ye = __shfl_up_sync(0xffffffffu, se, off);
-      const int yt = __shfl_up_sync(0xffffffffu, st, off);
-      if (lane >= off) { se += ye; st += yt; }
-    }
-    if (lane == 31) { warp_e[warp] = se; warp_t[warp] = st; }
-    __syncthreads();
-    if (warp == 0) {
-      int we = warp_e[lane], wt = warp_t[lane];
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int ye = __shfl_up_sync(0xffffffffu, we, off);
-        const int yt = __shfl_up_sync(0xffffffffu, wt, off);
-        if (lane >= off) { we += ye; wt += yt; }
-      }
-      warp_e[lane] = we;  // inclusive per-warp totals
-      warp_t[lane] = wt;
-    }
-    __syncthreads();
-    const int pe = carry_e + (warp ? warp_e[warp - 1] : 0) + se - ce;
-    const int pt = carry_t + (warp ? warp_t[warp - 1] : 0) + st - ct;
-    if (L < nlists) {
-      listoff[L] = pe;
-      cursor[L] = pe;
-      tileoff[L] = pt;
-    }
-    __syncthreads();
-    if (tid == kScanThreads - 1) {
-      carry_e = pe + ce;
-      carry_t = pt + ct;
-    }
-    __syncthreads();
-  }
-  if (tid == 0) {
-    listoff[nlists] = carry_e;
-    tileoff[nlists] = carry_t;
-  }
+  __shared__ int sh[2 * kScanThreads / 32];
+  scan_lists<kScanThreads>(counts, cursor, listoff, tileoff, nlists, sh);
 }
 
 // ----------------------------------------------------------------- scatter
@@ -474,7 +429,8 @@ cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileo
 cudaError_t launch_scatter(ScatterParams p, cudaStream_t st) {
   dim3 grid((p.N + kTileRows - 1) / kTileRows, p.hkv, p.batch);
   const size_t cache = sizeof(int) * (size_t)p.G * kTileRows * (p.topk | 1);
-  p.cache_rows = cache <= kScatterCacheBytes ? 1 : 0;
+  // Staging pays for itself when a row has several picks to read twice.
+  p.cache_rows = (p.topk - 1 >= 4 && cache <= kScatterCacheBytes) ? 1 : 0;
   const size_t smem = sizeof(int) * 2 * p.nblk + (p.cache_rows ? cache : 0);
   if (smem > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
