@@ -89,14 +89,20 @@ def num_threads() -> int:
     return int(_load().orc_num_threads())
 
 
+def n_blocks(N: int, block: int) -> int:
+    """ceil(N / block): when block does not divide N the last block is partial."""
+    return -(-N // block)
+
+
 def pool_keys(k, block: int) -> np.ndarray:
-    """[MoBA] §블록 분할과 top-k 게이팅: kbar[b,hk,j] = mean of K[b,hk,j*B:(j+1)*B].
-    ``k``: bf16 [b, hkv, N, d].  Returns float64 [b, hkv, N/B, d]."""
+    """[MoBA] §블록 분할과 top-k 게이팅: kbar[b,hk,j] = mean of K[b,hk,j*B:min((j+1)*B,N)]
+    (a partial last block: the mean of the keys it holds).
+    ``k``: bf16 [b, hkv, N, d].  Returns float64 [b, hkv, ceil(N/B), d]."""
     kb = bf16_bits(k)
     b, hkv, N, d = kb.shape
-    if block < 1 or N % block:
-        raise ValueError("N must be a multiple of the block size")
-    out = np.empty((b, hkv, N // block, d), dtype=np.float64)
+    if block < 1:
+        raise ValueError("block must be positive")
+    out = np.empty((b, hkv, n_blocks(N, block), d), dtype=np.float64)
     _check(_load().orc_pool_keys(_ptr(kb), b, hkv, N, d, block, _ptr(out)))
     return out
 
@@ -108,7 +114,7 @@ def gate_scores(q, kbar: np.ndarray, block: int, rows=None) -> np.ndarray:
     b, hq, N, d = qb.shape
     kbar = np.ascontiguousarray(kbar, dtype=np.float64)
     hkv, n = kbar.shape[1], kbar.shape[2]
-    assert kbar.shape == (b, hkv, N // block, d)
+    assert kbar.shape == (b, hkv, n_blocks(N, block), d)
     r = _rows(rows, N)
     out = np.empty((b, hq, len(r), n), dtype=np.float64)
     _check(_load().orc_gate_scores(_ptr(qb), _ptr(kbar), b, hq, hkv, N, d, block,
@@ -123,7 +129,7 @@ def select_topk(scores: np.ndarray, N: int, block: int, topk: int, rows=None):
     scores = np.ascontiguousarray(scores, dtype=np.float64)
     b, hq, R, n = scores.shape
     r = _rows(rows, N)
-    assert len(r) == R and n == N // block
+    assert len(r) == R and n == n_blocks(N, block)
     idx = np.empty((b, hq, R, topk), dtype=np.int32)
     gap = np.empty((b, hq, R), dtype=np.float64)
     _check(_load().orc_select_topk(_ptr(scores), b, hq, N, block, topk, _ptr(r), R,

@@ -24,7 +24,10 @@
  *   - with fewer than k-1 past blocks every past block is kept;
  *   - each GQA query head selects on its own; head h reads KV head h / (Hq/Hkv);
  *   - the optional causal window is a set union with the selected blocks;
- *   - lse is the natural log of the sum of exp(scaled logits) over the key set.
+ *   - lse is the natural log of the sum of exp(scaled logits) over the key set;
+ *   - when B does not divide N, the last block holds the remaining N mod B
+ *     positions and is pooled by the mean of those keys (it is only ever a row's
+ *     own block, never a past block of any row).
  */
 #include <math.h>
 #include <stdint.h>
@@ -57,30 +60,35 @@ int orc_num_threads(void)
 #endif
 }
 
+/* Number of blocks: ceil(N / B).  When B does not divide N the last block is
+   partial: it holds the N mod B remaining positions. */
+static int n_blocks(int N, int B) { return (N + B - 1) / B; }
+
 /*
  * [MoBA] §"블록 분할과 top-k 게이팅" (block partition and top-k gating): block j covers
- * key positions [j*B, (j+1)*B) and is represented by the mean of its keys,
- * MeanPool(K[I_j]).
+ * key positions [j*B, min((j+1)*B, N)) and is represented by the mean of its keys,
+ * MeanPool(K[I_j]) (a partial last block: the mean of the keys it holds).
  *   k    : bf16 [b, hkv, N, d]
- *   kbar : double [b, hkv, N/B, d]
+ *   kbar : double [b, hkv, ceil(N/B), d]
  */
 int orc_pool_keys(const uint16_t *k, int b, int hkv, int N, int d, int B, double *kbar)
 {
-    if (b < 1 || hkv < 1 || N < 1 || d < 1 || B < 1 || N % B != 0)
+    if (b < 1 || hkv < 1 || N < 1 || d < 1 || B < 1)
         return ORC_ERR_ARG;
-    const int n = N / B;
+    const int n = n_blocks(N, B);
     const long total = (long)b * hkv * n;
 #pragma omp parallel for schedule(static)
     for (long u = 0; u < total; ++u) {
         const long bh = u / n;
         const int j = (int)(u % n);
+        const int len = (N - j * B < B) ? N - j * B : B;
         const uint16_t *kb = k + (bh * N + (long)j * B) * d;
         double *dst = kbar + u * d;
         for (int t = 0; t < d; ++t) {
             double sum = 0.0;
-            for (int r = 0; r < B; ++r)
+            for (int r = 0; r < len; ++r)
                 sum += bf16_to_double(kb[(long)r * d + t]);
-            dst[t] = sum / (double)B;
+            dst[t] = sum / (double)len;
         }
     }
     return ORC_OK;
@@ -92,16 +100,16 @@ int orc_pool_keys(const uint16_t *k, int b, int hkv, int N, int d, int B, double
  * c = i / B compete; the own block is forced and later blocks are excluded, so only
  * j < c gets a score.  Entries j >= c are written as -INFINITY.
  *   q      : bf16 [b, hq, N, d]
- *   kbar   : double [b, hkv, N/B, d]
+ *   kbar   : double [b, hkv, ceil(N/B), d]
  *   rows   : nrows query positions (applied to every batch and head)
- *   scores : double [b, hq, nrows, N/B]
+ *   scores : double [b, hq, nrows, ceil(N/B)]
  */
 int orc_gate_scores(const uint16_t *q, const double *kbar, int b, int hq, int hkv, int N,
                     int d, int B, const int32_t *rows, int nrows, double *scores)
 {
-    if (b < 1 || hq < 1 || hkv < 1 || hq % hkv != 0 || N < 1 || d < 1 || B < 1 || N % B != 0)
+    if (b < 1 || hq < 1 || hkv < 1 || hq % hkv != 0 || N < 1 || d < 1 || B < 1)
         return ORC_ERR_ARG;
-    const int n = N / B, G = hq / hkv;
+    const int n = n_blocks(N, B), G = hq / hkv;
     const long total = (long)b * hq * nrows;
     int bad = 0;
 #pragma omp parallel for schedule(static) reduction(| : bad)
@@ -158,9 +166,9 @@ static int by_score_desc(const void *a, const void *b)
 int orc_select_topk(const double *scores, int b, int hq, int N, int B, int topk,
                     const int32_t *rows, int nrows, int32_t *idx, double *gap)
 {
-    if (b < 1 || hq < 1 || N < 1 || B < 1 || N % B != 0 || topk < 1)
+    if (b < 1 || hq < 1 || N < 1 || B < 1 || topk < 1)
         return ORC_ERR_ARG;
-    const int n = N / B;
+    const int n = n_blocks(N, B);
     const long total = (long)b * hq * nrows;
     int bad = 0;
 #pragma omp parallel reduction(| : bad)
@@ -230,14 +238,14 @@ int orc_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, int b
 {
     if (b < 1 || hq < 1 || hkv < 1 || hq % hkv != 0 || N < 1 || d < 1)
         return ORC_ERR_ARG;
-    if (mode == ORC_MODE_MOBA && (B < 1 || N % B != 0 || topk < 1 || !idx))
+    if (mode == ORC_MODE_MOBA && (B < 1 || topk < 1 || !idx))
         return ORC_ERR_ARG;
     if (mode == ORC_MODE_SWA && window < 1)
         return ORC_ERR_ARG;
     if (mode < 0 || mode > 2)
         return ORC_ERR_ARG;
     const int G = hq / hkv;
-    const int n = (mode == ORC_MODE_MOBA) ? N / B : 1;
+    const int n = (mode == ORC_MODE_MOBA) ? n_blocks(N, B) : 1;
     const long total = (long)b * hq * nrows;
     int bad = 0;
 #pragma omp parallel reduction(| : bad)

@@ -174,3 +174,42 @@ def test_sampled_rows_equal_full_rows():
     part = oracle.moba(q, k, v, block=64, topk=3, window=40, rows=rows)
     assert np.array_equal(part["idx"], full["idx"][:, :, rows])
     np.testing.assert_allclose(part["out"], full["out"][:, :, rows], rtol=0, atol=0)
+
+
+# ------------------------------------------------------------- partial last block
+
+@pytest.mark.parametrize("N,B,topk,window", [(500, 64, 100, 0), (300, 128, 3, 0), (200, 64, 1, 10_000)])
+def test_moba_with_partial_block_reduces_to_dense_causal(N, B, topk, window):
+    """B does not divide N: top-k >= n (or a window >= N) still attends every causal
+    key, the partial last block included (torch SDPA, float64)."""
+    q, k, v = _qkv(1, 2, 1, N, 16, seed=13)
+    r = _moba(q, k, v, B, topk, window)
+    ref, rlse = _sdpa(q, k, v, causal=True)
+    np.testing.assert_allclose(r["out"], ref, **TOL)
+    np.testing.assert_allclose(r["lse"], rlse, **TOL)
+
+
+@pytest.mark.parametrize("N,B,topk,window", [(250, 32, 3, 0), (230, 16, 4, 24), (100, 64, 2, 0)])
+def test_gathered_with_partial_block_matches_naive_mask(N, B, topk, window):
+    d = 16
+    q, k, v = _qkv(1, 2, 1, N, d, seed=14)
+    r = _moba(q, k, v, B, topk, window)
+    qd, kd, vd = (oracle.bf16_to_f64(t)[0] for t in (q, k, v))
+    for h in range(2):
+        mask = naive.block_mask(N, B, naive.block_sets_from_idx(r["idx"][0, h]), window)
+        out, lse = naive.masked_attention(qd[h], kd[0], vd[0], mask)
+        np.testing.assert_allclose(r["out"][0, h], out, **TOL)
+        np.testing.assert_allclose(r["lse"][0, h], lse, **TOL)
+
+
+def test_topk_one_with_partial_block_is_block_diagonal_causal():
+    """k = 1: each row attends its own block causally, the partial last block as a
+    shorter causal block (SDPA per block)."""
+    N, B = 200, 64
+    q, k, v = _qkv(1, 2, 2, N, 16, seed=15)
+    r = _moba(q, k, v, B, 1)
+    for j in range(-(-N // B)):
+        sl = slice(j * B, min((j + 1) * B, N))
+        ref, rlse = _sdpa(q[:, :, sl], k[:, :, sl], v[:, :, sl], causal=True)
+        np.testing.assert_allclose(r["out"][:, :, sl], ref, **TOL)
+        np.testing.assert_allclose(r["lse"][:, :, sl], rlse, **TOL)

@@ -43,9 +43,18 @@ def test_pool_matches_numpy_mean(B):
     np.testing.assert_allclose(kbar, ref, rtol=0, atol=1e-15)
 
 
-def test_pool_rejects_ragged_block():
-    with pytest.raises(ValueError):
-        oracle.pool_keys(_bf16((1, 1, 100, 8), 0), 64)
+def test_pool_partial_last_block_is_the_mean_of_its_keys():
+    """N = 100, B = 64: block 1 holds positions 64..99 and is pooled over those 36
+    keys only (numpy mean of the slice); a constant partial block pools exactly."""
+    k = _bf16((2, 2, 100, 16), seed=2)
+    kbar = oracle.pool_keys(k, 64)
+    assert kbar.shape == (2, 2, 2, 16)
+    kd = oracle.bf16_to_f64(k)
+    np.testing.assert_allclose(kbar[:, :, 0], kd[:, :, :64].mean(axis=2), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(kbar[:, :, 1], kd[:, :, 64:].mean(axis=2), rtol=0, atol=1e-15)
+    kc = torch.zeros(1, 1, 100, 8)
+    kc[:, :, 64:] = 0.375
+    assert np.all(oracle.pool_keys(kc.to(torch.bfloat16), 64)[0, 0, 1] == 0.375)
 
 
 # ---------------------------------------------------------------------- selection
@@ -215,3 +224,43 @@ def test_selection_invariant_under_a_common_key_shift():
     assert np.array_equal(i1, i2)
     finite = np.isfinite(g1)
     np.testing.assert_allclose(g1[finite], g2[finite], atol=1e-12)
+
+
+# ------------------------------------------------------------- partial last block
+
+@pytest.mark.parametrize("B", [2, 8, 128])
+def test_select_with_partial_last_block_matches_brute_force(B):
+    """N = 6B + B/2: the last block is partial.  It is only ever a row's own block, so
+    every past block is full, and the choice equals brute force for all k."""
+    n_full = 6
+    N = n_full * B + B // 2
+    d = 8
+    q = _bf16((1, 2, N, d), seed=40 + B)
+    k = _bf16((1, 1, N, d), seed=50 + B)
+    kbar = oracle.pool_keys(k, B)
+    assert kbar.shape[2] == n_full + 1
+    rows = np.arange(N, dtype=np.int32)
+    s = oracle.gate_scores(q, kbar, B, rows)
+    for k_ in range(1, n_full + 2):
+        idx, _ = oracle.select_topk(s, N, B, k_, rows)
+        for h in range(2):
+            for i in rows:
+                c = i // B
+                got = [x for x in idx[0, h, i] if x >= 0]
+                assert len(got) == min(k_, c + 1)
+                assert set(got) == _brute_force_sets(s[0, h, i], c, k_), (B, k_, h, i)
+
+
+def test_rows_before_a_partial_block_ignore_it():
+    """Causality: rows in the full blocks of an N = 5B + 40 problem choose exactly as
+    in the problem cut at 5B (they never see the partial block)."""
+    B, d, k_ = 64, 16, 3
+    N = 5 * B + 40
+    q = _bf16((1, 2, N, d), seed=61)
+    k = _bf16((1, 1, N, d), seed=62)
+    full = oracle.select_topk(oracle.gate_scores(q, oracle.pool_keys(k, B), B), N, B, k_)
+    Nc = 5 * B
+    cut = oracle.select_topk(oracle.gate_scores(q[:, :, :Nc], oracle.pool_keys(k[:, :, :Nc], B), B),
+                             Nc, B, k_)
+    assert np.array_equal(full[0][:, :, :Nc], cut[0])
+    assert np.array_equal(full[1][:, :, :Nc], cut[1])

@@ -66,8 +66,11 @@ def make_inputs(w: Workload, seed: int = 0, device: str = "cpu"):
     k32 = torch.randn((b, w.hkv, N, d), generator=g, dtype=torch.float32)
     v = _randn_bf16((b, w.hkv, N, d), g)
     if w.key_offset_std > 0:
-        off = torch.randn((b, w.hkv, N // w.block, d), generator=g, dtype=torch.float32)
-        k32 += (w.key_offset_std * off).repeat_interleave(w.block, dim=2)
+        # One offset per block, the partial last block (when block does not divide N)
+        # included.
+        nb = -(-N // w.block)
+        off = torch.randn((b, w.hkv, nb, d), generator=g, dtype=torch.float32)
+        k32 += (w.key_offset_std * off).repeat_interleave(w.block, dim=2)[:, :, :N]
     k = k32.to(torch.bfloat16)
     del k32
     return q.to(device), k.to(device), v.to(device)
