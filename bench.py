@@ -354,7 +354,7 @@ def run_ours(args, rank, world, device):
         # tensor-core gate's last CTA writes the list offsets itself), and per query
         # chunk: past-block pass, own-block pass, merge (only the own-block pass when
         # topk = 1).
-        tc_gate = w.seqlen // w.block <= 256 and w.topk - 1 < 32
+        tc_gate = -(-w.seqlen // w.block) <= 256 and w.topk - 1 < 32
         launches_per_step = (2 + ((1 if tc_gate else 2) if w.topk > 1 else 0)
                              + layout_chunks * (3 if w.topk > 1 else 1))
     else:

@@ -109,7 +109,7 @@ def moba_pool_keys(k: torch.Tensor, block: int, kbar=None, kbar_split=None, stre
     """[MoBA] §블록 분할과 top-k 게이팅: block means of the keys.  Returns (kbar float32
     [b, hkv, n, d], kbar_split bf16 [b, hkv, 2, n, d])."""
     b, hkv, N, d = k.shape
-    n = N // block
+    n = -(-N // block)  # a partial last block when block does not divide N
     if kbar is None:
         kbar = torch.empty(b, hkv, n, d, dtype=torch.float32, device=k.device)
     if kbar_split is None:
@@ -205,7 +205,7 @@ class MobaPrefill:
     def __init__(self, batch, hq, hkv, N, d, block, topk, window=0, device="cuda"):
         self.shape = (batch, hq, hkv, N, d)
         self.block, self.topk, self.window = block, topk, window
-        n = N // block
+        n = -(-N // block)  # a partial last block when block does not divide N
         self.workspace = torch.empty(workspace_size(batch, hq, hkv, N, d, block, topk),
                                      dtype=torch.uint8, device=device)
         self.kbar = torch.empty(batch, hkv, n, d, dtype=torch.float32, device=device)

@@ -60,7 +60,9 @@ int check_attn_dim(int d) { return (d == 64 || d == 80 || d == 128) ? MOBA_OK : 
 int check_moba_shape(int batch, int hq, int hkv, int N, int d, int block, int topk) {
   if (batch < 1 || hq < 1 || hkv < 1 || N < 1 || block < 1) return MOBA_ERR_SHAPE;
   if (hq % hkv) return MOBA_ERR_SHAPE;
-  if (block % kTileRows || N % block) return MOBA_ERR_SHAPE;
+  // 128-row query tiles: N and block multiples of 128 (block need not divide N: the
+  // last block is then partial).
+  if (block % kTileRows || N % kTileRows) return MOBA_ERR_SHAPE;
   if (topk < 1 || topk > 32) return MOBA_ERR_ARG;
   const long long G = hq / hkv;
   if ((long long)N * G * (topk - 1) >= (1ll << 31)) return MOBA_ERR_SHAPE;
@@ -212,7 +214,7 @@ int moba_workspace_size(int batch, int hq, int hkv, int N, int d, int block, int
 
 int moba_pool_keys(moba_tensor k, int batch, int hkv, int N, int d, int block, float *kbar,
                    void *kbar_split, void *stream) {
-  if (batch < 1 || hkv < 1 || N < 1 || block < 1 || N % block) return MOBA_ERR_SHAPE;
+  if (batch < 1 || hkv < 1 || N < 1 || block < 1) return MOBA_ERR_SHAPE;
   if (d < 8 || d > 256 || d % 8) return MOBA_ERR_DIM;
   int rc = check_tensor(k);
   if (rc) return rc;
@@ -446,7 +448,7 @@ int moba_device_status(void) {
 const char *moba_status_string(int status) {
   switch (status) {
     case MOBA_OK: return "ok";
-    case MOBA_ERR_SHAPE: return "unsupported shape (N % block, hq % hkv, block % 128, size limits)";
+    case MOBA_ERR_SHAPE: return "unsupported shape (N % 128, hq % hkv, block % 128, size limits)";
     case MOBA_ERR_DIM: return "unsupported head dimension";
     case MOBA_ERR_ALIGN: return "pointer or stride not 16-byte aligned";
     case MOBA_ERR_ARG: return "invalid argument";

@@ -63,7 +63,7 @@ int moba_prefill_static(moba_tensor q, moba_tensor k, moba_tensor v, int batch, 
   int rc = moba_workspace_size(batch, hq, hkv, N, d, block, topk, &ws);
   if (rc) return rc;
   // Carve: pooled keys (f32), their bf16 split, block choices, workspace.
-  const size_t nblk = size_t(N / block);
+  const size_t nblk = size_t((N + block - 1) / block);
   const size_t kbar_bytes = align_up(size_t(batch) * hkv * nblk * d * 4, 256);
   const size_t split_bytes = align_up(size_t(batch) * hkv * 2 * nblk * d * 2, 256);
   const size_t idx_bytes = align_up(size_t(batch) * hq * size_t(N) * topk * 4, 256);

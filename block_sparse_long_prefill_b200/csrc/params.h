@@ -17,7 +17,7 @@ constexpr size_t kPartialCapBytes = size_t(4) << 30;  // partial outputs kept pe
 // List L = ((chunk * batch + b) * hkv + hk) * nblk + j holds the (row, q-head, slot)
 // triples of the rows of query chunk `chunk` that picked past block j.
 struct WorkspaceLayout {
-  int nblk;         // N / block
+  int nblk;         // ceil(N / block): a partial last block when block does not divide N
   int G;            // hq / hkv
   int npast;        // topk - 1: partial slots per row
   int chunk_rows;   // query rows per pass (multiple of 128)
@@ -43,7 +43,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline WorkspaceLayout make_layout(int batch, int hq, int hkv, int N, int d, int block,
                                    int topk) {
   WorkspaceLayout w{};
-  w.nblk = N / block;
+  w.nblk = (N + block - 1) / block;
   w.G = hq / hkv;
   w.npast = topk - 1;
   // Partials exist only when a row can attend past blocks: topk slots per row then.

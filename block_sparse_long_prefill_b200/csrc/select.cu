@@ -14,8 +14,9 @@ namespace moba {
 
 // ------------------------------------------------------------------ pooling
 //
-// [MoBA] §"블록 분할과 top-k 게이팅": MeanPool(K[I_j]) over the keys of block j.
-// One CTA per (block, kv-head, batch).  Threads read 16-byte vectors along d
+// [MoBA] §"블록 분할과 top-k 게이팅": MeanPool(K[I_j]) over the keys of block j
+// (positions [j*block, min((j+1)*block, N)): a partial last block when block does
+// not divide N).  One CTA per (block, kv-head, batch).  Threads read 16-byte vectors along d
 // (coalesced rows), accumulate in fp32, and reduce across row groups in a fixed
 // order (deterministic).  Also writes the split hi = bf16(mean), lo = bf16(mean - hi)
 // that the gate multiplies with on the tensor cores.
@@ -23,7 +24,7 @@ constexpr int kPoolThreads = 256;
 
 __global__ void __launch_bounds__(kPoolThreads)
 pool_keys_kernel(const uint16_t *__restrict__ k, int64_t sb, int64_t sh, int64_t sn, int hkv,
-                 int d, int block, int nblk, float *__restrict__ kbar,
+                 int d, int block, int N, int nblk, float *__restrict__ kbar,
                  uint16_t *__restrict__ split) {
   extern __shared__ float red[];  // [ngroups][d]
   const int j = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
@@ -31,13 +32,14 @@ pool_keys_kernel(const uint16_t *__restrict__ k, int64_t sb, int64_t sh, int64_t
   const int ngroups = kPoolThreads / vpr;   // rows read concurrently
   const int t = threadIdx.x;
   const int vec = t % vpr, grp = t / vpr;
+  const int len = min(block, N - j * block);  // keys in this block
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   if (grp < ngroups) {
     const uint16_t *base = k + b * sb + hk * sh + (int64_t)j * block * sn + vec * 8;
     int r = grp;
-    for (; r + 7 * ngroups < block; r += 8 * ngroups) {
+    for (; r + 7 * ngroups < len; r += 8 * ngroups) {
       uint4 v[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u)
@@ -52,7 +54,7 @@ pool_keys_kernel(const uint16_t *__restrict__ k, int64_t sb, int64_t sh, int64_t
         }
       }
     }
-    for (; r < block; r += ngroups) {
+    for (; r < len; r += ngroups) {
       const uint4 v = __ldg(reinterpret_cast<const uint4 *>(base + (int64_t)r * sn));
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -69,7 +71,7 @@ pool_keys_kernel(const uint16_t *__restrict__ k, int64_t sb, int64_t sh, int64_t
   for (int c = t; c < d; c += kPoolThreads) {
     float s = 0.f;
     for (int g = 0; g < ngroups; ++g) s += red[g * d + c];
-    const float mean = s / (float)block;
+    const float mean = s / (float)len;
     kbar[(bh * nblk + j) * d + c] = mean;
     const __nv_bfloat16 hi = __float2bfloat16_rn(mean);
     const __nv_bfloat16 lo = __float2bfloat16_rn(mean - __bfloat162float(hi));
@@ -383,11 +385,12 @@ scatter_kernel(const ScatterParams p) {
 // Host-side launchers (called by the ABI layer).
 cudaError_t launch_pool(const uint16_t *k, int64_t sb, int64_t sh, int64_t sn, int batch, int hkv,
                         int N, int d, int block, float *kbar, uint16_t *split, cudaStream_t st) {
-  const int nblk = N / block;
+  const int nblk = (N + block - 1) / block;
   const int ngroups = kPoolThreads / (d / 8);
   const size_t smem = sizeof(float) * ngroups * d;
   dim3 grid(nblk, hkv, batch);
-  pool_keys_kernel<<<grid, kPoolThreads, smem, st>>>(k, sb, sh, sn, hkv, d, block, nblk, kbar, split);
+  pool_keys_kernel<<<grid, kPoolThreads, smem, st>>>(k, sb, sh, sn, hkv, d, block, N, nblk, kbar,
+                                                      split);
   return cudaGetLastError();
 }
 

@@ -21,9 +21,11 @@
  *     16 bytes.  q is [batch, hq, N, d]; k, v are [batch, hkv, N, d]; out is
  *     [batch, hq, N, d]; all bf16.
  *   - GQA: query head h reads KV head h / (hq / hkv).
- *   - Block j covers key positions [j*block, (j+1)*block) (0-based; the MoBA page
- *     numbers blocks from 1).  N must be a multiple of block, and block a multiple
- *     of 128.
+ *   - Block j covers key positions [j*block, min((j+1)*block, N)) (0-based; the MoBA
+ *     page numbers blocks from 1); there are n = ceil(N / block) blocks.  When block
+ *     does not divide N the last block is partial: it holds the N mod block remaining
+ *     positions and is pooled over those keys.  block and N must be multiples of 128
+ *     (moba_pool_keys alone takes any N and block >= 1).
  *   - d must be 64, 80 or 128 (moba_pool_keys alone takes any multiple of 8 up to
  *     256).
  *   - Ownership: the caller allocates every buffer (inputs, outputs, workspace); the
@@ -47,7 +49,7 @@ extern "C" {
 #endif
 
 #define MOBA_OK 0
-#define MOBA_ERR_SHAPE -1     /* N % block, hq % hkv, block % 128, sizes out of range */
+#define MOBA_ERR_SHAPE -1     /* N % 128, hq % hkv, block % 128, sizes out of range */
 #define MOBA_ERR_DIM -2       /* unsupported head dimension */
 #define MOBA_ERR_ALIGN -3     /* pointer or stride not 16-byte aligned */
 #define MOBA_ERR_ARG -4       /* topk < 1, window < 0, null pointer, ... */
@@ -74,8 +76,9 @@ int moba_workspace_size(int batch, int hq, int hkv, int N, int d, int block, int
 /*
  * [MoBA] §"블록 분할과 top-k 게이팅": MeanPool(K[I_j]) for every block j.
  *   k          : bf16 keys [batch, hkv, N, d]
- *   kbar       : float32 out [batch, hkv, N/block, d], contiguous: the block means
- *   kbar_split : bf16 out [batch, hkv, 2, N/block, d], contiguous: hi = bf16(kbar)
+ *   kbar       : float32 out [batch, hkv, n, d], contiguous: the block means
+ *                (n = ceil(N / block); a partial last block: the mean of its keys)
+ *   kbar_split : bf16 out [batch, hkv, 2, n, d], contiguous: hi = bf16(kbar)
  *                and lo = bf16(kbar - hi), the two bf16 terms the gate multiplies by
  */
 int moba_pool_keys(moba_tensor k, int batch, int hkv, int N, int d, int block, float *kbar,

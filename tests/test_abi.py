@@ -46,7 +46,7 @@ def test_workspace_size_is_host_only_and_grows_with_topk():
 
 @pytest.mark.parametrize("args,code", [
     ((1, 32, 8, 32768, 128, 500, 3), -1),   # block not a multiple of 128
-    ((1, 32, 8, 32000, 128, 512, 3), -1),   # N not a multiple of block
+    ((1, 32, 8, 32064, 128, 512, 3), -1),   # N not a multiple of 128
     ((1, 30, 8, 32768, 128, 512, 3), -1),   # hq not a multiple of hkv
     ((1, 32, 8, 32768, 96, 512, 3), -2),    # unsupported d
     ((1, 32, 8, 32768, 128, 512, 0), -4),   # topk < 1
@@ -57,6 +57,13 @@ def test_workspace_size_rejects_bad_shapes(args, code):
     assert moba.library().moba_workspace_size(*args, ctypes.byref(out)) == code
 
 
+def test_block_need_not_divide_n():
+    """N = 250 * 128 with blocks of 512: 63 blocks, the last one partial."""
+    a = moba.workspace_size(1, 32, 8, 32000, 128, 512, 3)
+    b = moba.workspace_size(1, 32, 8, 32256, 128, 512, 3)  # 63 full blocks
+    assert 0 < a <= b
+
+
 def test_bad_arguments_are_rejected_before_any_launch():
     lib = moba.library()
     T = moba.MobaTensor
@@ -64,11 +71,15 @@ def test_bad_arguments_are_rejected_before_any_launch():
     ok = T(1 << 20, 8 * 1024, 8 * 1024, 128)
     mis = T((1 << 20) + 2, 8 * 1024, 8 * 1024, 128)
     odd = T(1 << 20, 8 * 1024, 8 * 1024, 100)
-    # pool: null tensor, misaligned pointer, misaligned stride, ragged block
+    # pool: null tensor, misaligned pointer, misaligned stride, empty sequence, no block
     assert lib.moba_pool_keys(null, 1, 1, 1024, 128, 128, 1 << 20, 1 << 20, None) == -4
     assert lib.moba_pool_keys(mis, 1, 1, 1024, 128, 128, 1 << 20, 1 << 20, None) == -3
     assert lib.moba_pool_keys(odd, 1, 1, 1024, 128, 128, 1 << 20, 1 << 20, None) == -3
-    assert lib.moba_pool_keys(ok, 1, 1, 1000, 128, 128, 1 << 20, 1 << 20, None) == -1
+    assert lib.moba_pool_keys(ok, 1, 1, 0, 128, 128, 1 << 20, 1 << 20, None) == -1
+    assert lib.moba_pool_keys(ok, 1, 1, 1000, 128, 0, 1 << 20, 1 << 20, None) == -1
+    # select: N not a multiple of 128
+    assert lib.moba_select_topk(ok, 1 << 20, 1, 1, 1, 1000, 128, 128, 3, 1 << 20, 1 << 20,
+                                1 << 30, None) == -1
     # select: workspace too small
     assert lib.moba_select_topk(ok, 1 << 20, 1, 1, 1, 1024, 128, 128, 3, 1 << 20, 1 << 20, 16,
                                 None) == -5

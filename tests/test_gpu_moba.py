@@ -58,6 +58,12 @@ def run_and_check(w: workloads.Workload, seed=0, rows=None, check_pool=True):
     ("window_wide", dict(batch=1, hq=2, hkv=1, seqlen=1024, d=64, block=128, topk=2, window=700)),
     ("window_dense", dict(batch=1, hq=2, hkv=1, seqlen=1024, d=128, block=256, topk=2, window=4096)),
     ("big_k", dict(batch=1, hq=2, hkv=1, seqlen=4096, d=128, block=128, topk=16)),
+    # block does not divide N: the last block is partial (its rows' own block)
+    ("partial_block", dict(batch=1, hq=4, hkv=2, seqlen=1280, d=128, block=512, topk=2)),
+    ("partial_d80_k3", dict(batch=1, hq=2, hkv=1, seqlen=1664, d=80, block=256, topk=3)),
+    ("partial_window", dict(batch=1, hq=2, hkv=1, seqlen=2432, d=64, block=512, topk=2, window=300)),
+    ("partial_long_list", dict(batch=1, hq=2, hkv=2, seqlen=4224, d=128, block=256, topk=12)),
+    ("partial_k_all", dict(batch=2, hq=2, hkv=1, seqlen=1152, d=64, block=256, topk=8)),
 ])
 def test_moba_small_full_rows(name, kw):
     w = workloads.WORKLOADS["tiny"] if name == "tiny" else workloads.small_moba(name=name, **kw)

@@ -29,6 +29,8 @@ def test_static_scratch_matches_the_allocating_path_twice():
     cases = [
         _case(0, batch=1, hq=4, hkv=2, seqlen=2048, d=128, block=256, topk=3),
         _case(1, batch=2, hq=2, hkv=1, seqlen=1024, d=64, block=128, topk=4, window=200),
+        # a partial last block (block does not divide N)
+        _case(3, batch=1, hq=2, hkv=1, seqlen=1408, d=128, block=512, topk=2),
     ]
     for w, q, k, v in cases:
         ref = moba.MobaPrefill(w.batch, w.hq, w.hkv, w.seqlen, w.d, w.block, w.topk, w.window)
