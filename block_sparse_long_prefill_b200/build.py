@@ -10,7 +10,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoba.so")
 SOURCES = ["api.cu", "select.cu", "gate.cu", "attn.cu", "merge.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "params.h"]
+HEADERS = ["common.cuh", "params.h", "lists.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
