@@ -111,9 +111,10 @@ def stored_traffic(workload: str, kernel: str = None):
 
 def attended_pairs_moba(idx: torch.Tensor, w: workloads.Workload) -> int:
     """Sum over rows, heads and batch of |J_i| for the blocks in idx (own block causal,
-    past blocks whole) unioned with the causal window."""
-    B, N = w.block, w.seqlen
-    i = torch.arange(N, device=idx.device)
+    past blocks whole) unioned with the causal window.  Row r of idx sits at key
+    position q_off + r (q_off > 0 for a chunked prefill)."""
+    B = w.block
+    i = w.q_off + torch.arange(w.nq, device=idx.device)
     c = i // B
     own = (i % B) + 1
     past = ((idx >= 0) & (idx < c[None, None, :, None])).sum(-1)  # [b, h, N]
@@ -145,18 +146,18 @@ def pass_work_moba(idx: torch.Tensor, w: workloads.Workload, chunk_rows: int) ->
     blocks) and of the own-block pass (causal own block plus window tail keys), and
     the bytes the merge pass must move (topk partial rows and log-sum-exps read, block
     choices read, the output row and its log-sum-exp written)."""
-    B, N = w.block, w.seqlen
+    B, N = w.block, w.nq
     rows = min(chunk_rows, N)
     sub = idx[:, :, :rows]
-    i = torch.arange(rows, device=idx.device)
+    i = w.q_off + torch.arange(rows, device=idx.device)   # key positions of the rows
     c = i // B
     past = int(((sub >= 0) & (sub < c[None, None, :, None])).sum().item()) * B
     own = int(((i % B) + 1).sum().item()) * w.batch * w.hq
     if w.window > 0:
         total_rows = attended_pairs_moba(idx, w)  # all rows; window extras scaled below
-        base = int(((torch.arange(N, device=idx.device) % B) + 1).sum().item()) * w.batch * w.hq
-        base += int(((idx >= 0) & (idx < (torch.arange(N, device=idx.device) // B)[None, None, :, None]))
-                    .sum().item()) * B
+        pos = w.q_off + torch.arange(N, device=idx.device)
+        base = int(((pos % B) + 1).sum().item()) * w.batch * w.hq
+        base += int(((idx >= 0) & (idx < (pos // B)[None, None, :, None])).sum().item()) * B
         own += int(round((total_rows - base) * rows / N))
     rowcount = w.batch * w.hq * rows
     merge_bytes = rowcount * (w.topk * (w.d * 2 + 4) + w.topk * 4 + w.d * 2 + 4)
@@ -165,7 +166,9 @@ def pass_work_moba(idx: torch.Tensor, w: workloads.Workload, chunk_rows: int) ->
 
 
 def dense_pairs(w: workloads.Workload) -> int:
-    return w.seqlen * (w.seqlen + 1) // 2 * w.batch * w.hq
+    """Causal pairs of the query rows (positions q_off .. seqlen - 1)."""
+    Nk, off = w.seqlen, w.q_off
+    return (Nk * (Nk + 1) // 2 - off * (off + 1) // 2) * w.batch * w.hq
 
 
 # --------------------------------------------------------------------- clocks
@@ -321,33 +324,35 @@ def run_ours(args, rank, world, device):
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream()
     q, k, v = workloads.make_inputs(w, seed=args.seed + rank)
+    if w.q_off:
+        q = q[:, :, w.q_off:].contiguous()  # chunked prefill: the last nq query rows
     qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
     qd, kd, vd = q.to(device), k.to(device), v.to(device)
     del q, k, v
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
 
     if w.kind == "moba":
-        runner = MobaPrefill(w.batch, w.hq, w.hkv, w.seqlen, w.d, w.block, w.topk, w.window,
-                             device=device)
+        runner = MobaPrefill(w.batch, w.hq, w.hkv, w.nq, w.d, w.block, w.topk, w.window,
+                             device=device, kv_len=w.seqlen)
 
         def stages():
             moba.moba_pool_keys(kd, w.block, runner.kbar, runner.kbar_split)
             yield "pool"
-            moba.moba_select_topk(qd, runner.kbar_split, w.block, w.topk, runner.workspace,
-                                  runner.idx)
+            moba.moba_select_topk_chunk(qd, runner.kbar_split, w.block, w.topk, w.seqlen,
+                                        runner.workspace, runner.idx)
             yield "select"
-            moba.moba_attn_fwd(qd, kd, vd, runner.idx, w.block, w.topk, runner.workspace,
-                               w.window, out=runner.out, lse=runner.lse)
+            moba.moba_attn_fwd_chunk(qd, kd, vd, runner.idx, w.block, w.topk, runner.workspace,
+                                     w.window, out=runner.out, lse=runner.lse)
             yield "attention"
         out_t, lse_t = runner.out, runner.lse
         layout_chunks = 1
-        chunk_rows = w.seqlen
+        chunk_rows = w.nq
         try:
             per_row = (w.topk if w.topk > 1 else 0) * (w.d * 2 + 4) * w.batch * w.hq
             cap = 4 << 30
-            if per_row * w.seqlen > cap:
+            if per_row * w.nq > cap:
                 chunk_rows = max(128, (cap // per_row) // 128 * 128)
-                layout_chunks = math.ceil(w.seqlen / chunk_rows)
+                layout_chunks = math.ceil(w.nq / chunk_rows)
         except ZeroDivisionError:
             pass
         # pool, gate, scatter (+ a scan launch when the general gate runs: the
@@ -424,7 +429,7 @@ def run_ours(args, rank, world, device):
     assert torch.isfinite(out_t.float()).all().item(), "non-finite output"
     ms = total_ms / args.steps
     tflops_total = weak_scaling_rate(flops, world, ms) / 1e12
-    tokens = weak_scaling_rate(w.batch * w.seqlen, world, ms)
+    tokens = weak_scaling_rate(w.batch * w.nq, world, ms)
 
     hbm, tc_peak, tc_sus, peak_kind = peaks()
     stage_ms = {n: sum(v) / len(v) for n, v in per_stage.items()}
@@ -468,9 +473,9 @@ def run_ours(args, rank, world, device):
                     "peak_kind": f"bf16 dense burst, {peak_kind}"}
     if w.kind == "moba":
         sel_ms = stage_ms["pool"] + stage_ms["select"]
-        n_entries = int(((runner.idx >= 0).sum().item()) - w.batch * w.hq * w.seqlen)
-        sel_bytes = (w.batch * w.hkv * w.seqlen * w.d * 2 + w.batch * w.hq * w.seqlen * w.d * 2
-                     + 2 * w.batch * w.hq * w.seqlen * w.topk * 4 + 2 * n_entries * 4)
+        n_entries = int(((runner.idx >= 0).sum().item()) - w.batch * w.hq * w.nq)
+        sel_bytes = (w.batch * w.hkv * w.seqlen * w.d * 2 + w.batch * w.hq * w.nq * w.d * 2
+                     + 2 * w.batch * w.hq * w.nq * w.topk * 4 + 2 * n_entries * 4)
         extra["selection"] = {"ms": round(sel_ms, 4), "bytes": sel_bytes,
                               "gbs": round(sel_bytes / (sel_ms * 1e-3) / 1e9, 1),
                               "frac_hbm": round(sel_bytes / (sel_ms * 1e-3) / 1e9 / hbm, 4)}
@@ -526,19 +531,22 @@ def run_ours(args, rank, world, device):
                 tot += a.elapsed_time(b_)
             return tot / reps
 
-        sd_ms = timeit(lambda: F.scaled_dot_product_attention(qd, kr, vr, is_causal=True),
-                       max(3, args.steps // 4))
         own_out = torch.empty_like(qd)
-        own_lse = torch.empty(w.batch, w.hq, w.seqlen, dtype=torch.float32, device=device)
-        od_ms = timeit(lambda: moba.swa_attn_fwd(qd, kd, vd, w.seqlen, out=own_out, lse=own_lse),
+        own_lse = torch.empty(w.batch, w.hq, w.nq, dtype=torch.float32, device=device)
+        od_ms = timeit(lambda: moba.swa_attn_fwd_chunk(qd, kd, vd, w.seqlen, out=own_out, lse=own_lse),
                        max(3, args.steps // 4))
-        comps = {"dense_causal_sdpa": {"ms": round(sd_ms, 4),
-                                       "tflops": round(dflops / (sd_ms * 1e-3) / 1e12, 2),
-                                       "speedup_of_moba": round(sd_ms / ms, 3)},
-                 "dense_causal_own_kernel": {"ms": round(od_ms, 4),
+        comps = {"dense_causal_own_kernel": {"ms": round(od_ms, 4),
                                              "tflops": round(dflops / (od_ms * 1e-3) / 1e12, 2),
                                              "frac_of_peak": round(dflops / (od_ms * 1e-3) / 1e12
                                                                    / tc_peak, 4)}}
+        if not w.q_off:
+            # torch's is_causal aligns the queries with the first keys, so it times whole
+            # prefills only.
+            sd_ms = timeit(lambda: F.scaled_dot_product_attention(qd, kr, vr, is_causal=True),
+                           max(3, args.steps // 4))
+            comps["dense_causal_sdpa"] = {"ms": round(sd_ms, 4),
+                                          "tflops": round(dflops / (sd_ms * 1e-3) / 1e12, 2),
+                                          "speedup_of_moba": round(sd_ms / ms, 3)}
         del kr, vr
 
     cpu = None
@@ -551,7 +559,7 @@ def run_ours(args, rank, world, device):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) q,k,v; per-block key offsets; no dataset)",
             "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv,
-                       "seq_len": w.seqlen, "d": w.d, "block": w.block, "topk": w.topk,
+                       "seq_len": w.seqlen, "q_len": w.nq, "d": w.d, "block": w.block, "topk": w.topk,
                        "window": w.window, "parallelism": f"replicas x{world}" if world > 1 else "1 gpu",
                        "l2": "flushed between timed steps (256 MB write)"},
             "tokens_per_s": round(tokens, 1), "attended_flops_per_step": flops,
@@ -573,16 +581,16 @@ def cpu_baseline(w: workloads.Workload, seed: int, target_s: float):
 
     q, k, v = workloads.make_inputs(w, seed)
     rng = np.random.default_rng(seed + 2000)
-    N = w.seqlen
+    N = w.nq  # query rows: positions q_off .. seqlen - 1
 
     def run(nrows):
-        rows = np.sort(rng.choice(N, size=nrows, replace=False)).astype(np.int32)
+        rows = (w.q_off + np.sort(rng.choice(N, size=nrows, replace=False))).astype(np.int32)
         t0 = time.perf_counter()
         if w.kind == "moba":
             kbar = oracle.pool_keys(k, w.block)
             t1 = time.perf_counter()
             s = oracle.gate_scores(q, kbar, w.block, rows)
-            idx, _ = oracle.select_topk(s, N, w.block, w.topk, rows)
+            idx, _ = oracle.select_topk(s, w.seqlen, w.block, w.topk, rows)
             oracle.attention(q, k, v, mode=oracle.MODE_MOBA, block=w.block, topk=w.topk, idx=idx,
                              window=w.window, rows=rows)
             t2 = time.perf_counter()
@@ -603,7 +611,7 @@ def cpu_baseline(w: workloads.Workload, seed: int, target_s: float):
     full_s = tp + ta * N / nrows
     pairs = attended_pairs_swa(w) if w.kind == "swa" else None
     if pairs is None:
-        i = np.arange(N, dtype=np.int64)
+        i = w.q_off + np.arange(N, dtype=np.int64)
         pairs = int(((i % w.block) + 1 + np.minimum(w.topk - 1, i // w.block) * w.block).sum()) * w.batch * w.hq
     flops = 4.0 * w.d * pairs
     return {"value": flops / full_s / 1e12, "unit": UNIT, "cores": oracle.num_threads(),
@@ -630,7 +638,7 @@ def run_reference(args, rank, world):
             "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv,
-                       "seq_len": w.seqlen, "d": w.d, "block": w.block, "topk": w.topk,
+                       "seq_len": w.seqlen, "q_len": w.nq, "d": w.d, "block": w.block, "topk": w.topk,
                        "window": w.window},
             "cpu_baseline": {**last, "value": value},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

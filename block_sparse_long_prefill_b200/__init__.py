@@ -30,8 +30,9 @@ _STATUS = {
 
 # Entry points declared in include/moba.h.
 ABI_FUNCTIONS = ("moba_workspace_size", "moba_pool_keys", "moba_select_topk", "moba_attn_fwd",
-                 "swa_attn_fwd", "moba_prefill_static", "moba_device_status", "moba_set_pass_events",
-                 "moba_status_string")
+                 "swa_attn_fwd", "moba_workspace_size_chunk", "moba_select_topk_chunk",
+                 "moba_attn_fwd_chunk", "swa_attn_fwd_chunk", "moba_prefill_static",
+                 "moba_device_status", "moba_set_pass_events", "moba_status_string")
 
 
 class MobaError(RuntimeError):
@@ -57,6 +58,11 @@ def _load():
     lib.moba_select_topk.argtypes = [T, P, I, I, I, I, I, I, I, P, P, S, P]
     lib.moba_attn_fwd.argtypes = [T, T, T, P, I, I, I, I, I, I, I, I, ctypes.c_float, T, P, P, S, P]
     lib.swa_attn_fwd.argtypes = [T, T, T, I, I, I, I, I, I, ctypes.c_float, T, P, P]
+    lib.moba_workspace_size_chunk.argtypes = [I, I, I, I, I, I, I, I, ctypes.POINTER(S)]
+    lib.moba_select_topk_chunk.argtypes = [T, P, I, I, I, I, I, I, I, I, P, P, S, P]
+    lib.moba_attn_fwd_chunk.argtypes = [T, T, T, P, I, I, I, I, I, I, I, I, I, ctypes.c_float, T, P,
+                                        P, S, P]
+    lib.swa_attn_fwd_chunk.argtypes = [T, T, T, I, I, I, I, I, I, I, ctypes.c_float, T, P, P]
     lib.moba_prefill_static.argtypes = [T, T, T, I, I, I, I, I, I, I, I, ctypes.c_float, T, P, P]
     lib.moba_device_status.argtypes = []
     lib.moba_set_pass_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), I]
@@ -165,6 +171,72 @@ def swa_attn_fwd(q, k, v, window: int, scale: float = 0.0, out=None, lse=None, s
     return out, lse
 
 
+def workspace_size_chunk(batch, hq, hkv, N, Nk, d, block, topk) -> int:
+    out = ctypes.c_size_t(0)
+    _check("moba_workspace_size_chunk",
+           _lib.moba_workspace_size_chunk(batch, hq, hkv, N, Nk, d, block, topk, ctypes.byref(out)))
+    return out.value
+
+
+def moba_select_topk_chunk(q, kbar_split: torch.Tensor, block: int, topk: int, kv_len: int,
+                           workspace: torch.Tensor, idx=None, stream=None):
+    """Block choices for the N query rows of ``q``, which are the last N of ``kv_len``
+    positions (pooled keys of all kv_len positions in ``kbar_split``)."""
+    b, hq, N, d = q.shape
+    hkv = kbar_split.shape[1]
+    if idx is None:
+        idx = torch.empty(b, hq, N, topk, dtype=torch.int32, device=q.device)
+    _check("moba_select_topk_chunk",
+           _lib.moba_select_topk_chunk(_t(q), kbar_split.data_ptr(), b, hq, hkv, N, kv_len, d, block,
+                                       topk, idx.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                       _stream(stream)))
+    return idx
+
+
+def moba_attn_fwd_chunk(q, k, v, idx, block: int, topk: int, workspace: torch.Tensor,
+                        window: int = 0, scale: float = 0.0, out=None, lse=None, stream=None):
+    """Attention of the N query rows of ``q`` (the last N positions) over the keys and
+    values of all k.shape[2] positions.  Returns (out, lse) for the N rows."""
+    b, hq, N, d = q.shape
+    hkv, Nk = k.shape[1], k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device)
+    _check("moba_attn_fwd_chunk",
+           _lib.moba_attn_fwd_chunk(_t(q), _t(k), _t(v), idx.data_ptr(), b, hq, hkv, N, Nk, d, block,
+                                    topk, window, float(scale), _t(out), lse.data_ptr(),
+                                    workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def swa_attn_fwd_chunk(q, k, v, window: int, scale: float = 0.0, out=None, lse=None, stream=None):
+    """Sliding-window attention of the last N positions (q) over k.shape[2] positions."""
+    b, hq, N, d = q.shape
+    hkv, Nk = k.shape[1], k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device)
+    _check("swa_attn_fwd_chunk",
+           _lib.swa_attn_fwd_chunk(_t(q), _t(k), _t(v), b, hq, hkv, N, Nk, d, window, float(scale),
+                                   _t(out), lse.data_ptr(), _stream(stream)))
+    return out, lse
+
+
+def moba_prefill_chunk(q, k, v, block: int, topk: int, window: int = 0, stream=None):
+    """Chunked prefill: q holds the last N of the k.shape[2] positions.  Pools all keys,
+    selects and attends for the N rows; returns (out, lse, idx)."""
+    b, hq, N, d = q.shape
+    hkv, Nk = k.shape[1], k.shape[2]
+    _, ks = moba_pool_keys(k, block, stream=stream)
+    ws = torch.empty(workspace_size_chunk(b, hq, hkv, N, Nk, d, block, topk), dtype=torch.uint8,
+                     device=q.device)
+    idx = moba_select_topk_chunk(q, ks, block, topk, Nk, ws, stream=stream)
+    out, lse = moba_attn_fwd_chunk(q, k, v, idx, block, topk, ws, window, stream=stream)
+    return out, lse, idx
+
+
 def moba_prefill_static(q, k, v, block: int, topk: int, window: int = 0, scale: float = 0.0,
                         out=None, lse=None, stream=None):
     """The whole prefill with the library's own fixed scratch (no workspace): for
@@ -200,13 +272,17 @@ def device_status() -> int:
 
 
 class MobaPrefill:
-    """The three MoBA calls with their buffers allocated once for a fixed shape."""
+    """The three MoBA calls with their buffers allocated once for a fixed shape.  N query
+    rows; with ``kv_len`` (> N) they are the last N of kv_len positions (chunked
+    prefill: k and v hold all kv_len positions)."""
 
-    def __init__(self, batch, hq, hkv, N, d, block, topk, window=0, device="cuda"):
+    def __init__(self, batch, hq, hkv, N, d, block, topk, window=0, device="cuda", kv_len=None):
+        kv = kv_len or N
         self.shape = (batch, hq, hkv, N, d)
+        self.kv_len = kv
         self.block, self.topk, self.window = block, topk, window
-        n = -(-N // block)  # a partial last block when block does not divide N
-        self.workspace = torch.empty(workspace_size(batch, hq, hkv, N, d, block, topk),
+        n = -(-kv // block)  # a partial last block when block does not divide kv_len
+        self.workspace = torch.empty(workspace_size_chunk(batch, hq, hkv, N, kv, d, block, topk),
                                      dtype=torch.uint8, device=device)
         self.kbar = torch.empty(batch, hkv, n, d, dtype=torch.float32, device=device)
         self.kbar_split = torch.empty(batch, hkv, 2, n, d, dtype=torch.bfloat16, device=device)
@@ -216,9 +292,10 @@ class MobaPrefill:
 
     def __call__(self, q, k, v, stream=None):
         moba_pool_keys(k, self.block, self.kbar, self.kbar_split, stream)
-        moba_select_topk(q, self.kbar_split, self.block, self.topk, self.workspace, self.idx, stream)
-        moba_attn_fwd(q, k, v, self.idx, self.block, self.topk, self.workspace, self.window,
-                      out=self.out, lse=self.lse, stream=stream)
+        moba_select_topk_chunk(q, self.kbar_split, self.block, self.topk, self.kv_len,
+                               self.workspace, self.idx, stream)
+        moba_attn_fwd_chunk(q, k, v, self.idx, self.block, self.topk, self.workspace, self.window,
+                            out=self.out, lse=self.lse, stream=stream)
         return self.out, self.lse
 
 

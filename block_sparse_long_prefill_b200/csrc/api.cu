@@ -57,12 +57,14 @@ int check_device(int *num_sms) {
 
 int check_attn_dim(int d) { return (d == 64 || d == 80 || d == 128) ? MOBA_OK : MOBA_ERR_DIM; }
 
-int check_moba_shape(int batch, int hq, int hkv, int N, int d, int block, int topk) {
+// N query rows at key positions q_off .. q_off + N - 1 (q_off = 0: a whole prefill).
+int check_moba_shape(int batch, int hq, int hkv, int N, int d, int block, int topk, int q_off = 0) {
   if (batch < 1 || hq < 1 || hkv < 1 || N < 1 || block < 1) return MOBA_ERR_SHAPE;
   if (hq % hkv) return MOBA_ERR_SHAPE;
-  // 128-row query tiles: N and block multiples of 128 (block need not divide N: the
-  // last block is then partial).
+  // 128-row query tiles: N, q_off and block multiples of 128 (block need not divide the
+  // key count: the last block is then partial).
   if (block % kTileRows || N % kTileRows) return MOBA_ERR_SHAPE;
+  if (q_off < 0 || q_off % kTileRows || (long long)q_off + N >= (1ll << 31)) return MOBA_ERR_SHAPE;
   if (topk < 1 || topk > 32) return MOBA_ERR_ARG;
   const long long G = hq / hkv;
   if ((long long)N * G * (topk - 1) >= (1ll << 31)) return MOBA_ERR_SHAPE;
@@ -104,15 +106,17 @@ int make_map(CUtensorMap *map, const moba_tensor &t, int batch, int heads, int N
 }
 
 // Q, Q tail, K, K tail, V, V tail.
+// q has Nq rows, k and v Nk rows.
 int make_attn_maps(CUtensorMap *maps, const moba_tensor &q, const moba_tensor &k,
-                   const moba_tensor &v, int batch, int hq, int hkv, int N, int d) {
+                   const moba_tensor &v, int batch, int hq, int hkv, int Nq, int Nk, int d) {
   const moba_tensor *ts[3] = {&q, &k, &v};
   const int heads[3] = {hq, hkv, hkv};
+  const int rows[3] = {Nq, Nk, Nk};
   for (int a = 0; a < 3; ++a) {
-    int rc = make_map(&maps[2 * a], *ts[a], batch, heads[a], N, d, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    int rc = make_map(&maps[2 * a], *ts[a], batch, heads[a], rows[a], d, 64, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
     if (d == 80)
-      rc = make_map(&maps[2 * a + 1], *ts[a], batch, heads[a], N, d, 16, CU_TENSOR_MAP_SWIZZLE_32B);
+      rc = make_map(&maps[2 * a + 1], *ts[a], batch, heads[a], rows[a], d, 16, CU_TENSOR_MAP_SWIZZLE_32B);
     else
       maps[2 * a + 1] = maps[2 * a];
     if (rc) return rc;
@@ -203,13 +207,18 @@ using namespace moba;
 
 extern "C" {
 
+int moba_workspace_size_chunk(int batch, int hq, int hkv, int Nq, int Nk, int d, int block,
+                              int topk, size_t *bytes) {
+  if (!bytes) return MOBA_ERR_ARG;
+  const int rc = check_moba_shape(batch, hq, hkv, Nq, d, block, topk, Nk - Nq);
+  if (rc) return rc;
+  *bytes = make_layout(batch, hq, hkv, Nq, d, block, topk, Nk - Nq).total;
+  return MOBA_OK;
+}
+
 int moba_workspace_size(int batch, int hq, int hkv, int N, int d, int block, int topk,
                         size_t *bytes) {
-  if (!bytes) return MOBA_ERR_ARG;
-  const int rc = check_moba_shape(batch, hq, hkv, N, d, block, topk);
-  if (rc) return rc;
-  *bytes = make_layout(batch, hq, hkv, N, d, block, topk).total;
-  return MOBA_OK;
+  return moba_workspace_size_chunk(batch, hq, hkv, N, N, d, block, topk, bytes);
 }
 
 int moba_pool_keys(moba_tensor k, int batch, int hkv, int N, int d, int block, float *kbar,
@@ -227,15 +236,16 @@ int moba_pool_keys(moba_tensor k, int batch, int hkv, int N, int d, int block, f
                                    static_cast<cudaStream_t>(stream)));
 }
 
-int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, int hkv, int N,
-                     int d, int block, int topk, int32_t *idx, void *workspace,
-                     size_t workspace_bytes, void *stream) {
-  int rc = check_moba_shape(batch, hq, hkv, N, d, block, topk);
+int moba_select_topk_chunk(moba_tensor q, const void *kbar_split, int batch, int hq, int hkv,
+                           int N, int Nk, int d, int block, int topk, int32_t *idx,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+  const int q_off = Nk - N;
+  int rc = check_moba_shape(batch, hq, hkv, N, d, block, topk, q_off);
   if (rc) return rc;
   if ((rc = check_tensor(q))) return rc;
   if (!kbar_split || !idx) return MOBA_ERR_ARG;
   if (!aligned16(kbar_split) || (reinterpret_cast<uintptr_t>(idx) & 3u)) return MOBA_ERR_ALIGN;
-  const WorkspaceLayout w = make_layout(batch, hq, hkv, N, d, block, topk);
+  const WorkspaceLayout w = make_layout(batch, hq, hkv, N, d, block, topk, q_off);
   if (!workspace || workspace_bytes < w.total) return MOBA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return MOBA_ERR_ALIGN;
   if ((rc = check_device(nullptr))) return rc;
@@ -275,6 +285,7 @@ int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, i
     }
     gp.batch = batch; gp.hq = hq; gp.hkv = hkv; gp.N = N; gp.d = d; gp.block = block;
     gp.topk = topk; gp.nblk = w.nblk; gp.G = w.G; gp.chunk_rows = w.chunk_rows;
+    gp.q_off = q_off;
     const long long ntiles = (long long)batch * hkv * (N / kTileRows) * w.G;
     const int grid = (int)(ntiles < nsm ? ntiles : nsm);
     if ((rc = launch_status(launch_gate_tc(maps, gp, grid, st)))) return rc;
@@ -287,6 +298,7 @@ int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, i
     sp.counts = counts;
     sp.batch = batch; sp.hq = hq; sp.hkv = hkv; sp.N = N; sp.d = d; sp.block = block;
     sp.topk = topk; sp.nblk = w.nblk; sp.G = w.G; sp.chunk_rows = w.chunk_rows;
+    sp.q_off = q_off;
     if ((rc = launch_status(launch_gate(sp, st)))) return rc;
   }
   if (w.npast == 0) return MOBA_OK;
@@ -303,14 +315,23 @@ int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, i
   cp.entries = reinterpret_cast<uint32_t *>(ws + w.off_entries);
   cp.batch = batch; cp.hq = hq; cp.hkv = hkv; cp.N = N; cp.block = block; cp.topk = topk;
   cp.nblk = w.nblk; cp.G = w.G; cp.chunk_rows = w.chunk_rows;
+  cp.q_off = q_off;
   return launch_status(launch_scatter(cp, st));
 }
 
-int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *idx, int batch,
-                  int hq, int hkv, int N, int d, int block, int topk, int window, float scale,
-                  moba_tensor out, float *lse, void *workspace, size_t workspace_bytes,
-                  void *stream) {
-  int rc = check_moba_shape(batch, hq, hkv, N, d, block, topk);
+int moba_select_topk(moba_tensor q, const void *kbar_split, int batch, int hq, int hkv, int N,
+                     int d, int block, int topk, int32_t *idx, void *workspace,
+                     size_t workspace_bytes, void *stream) {
+  return moba_select_topk_chunk(q, kbar_split, batch, hq, hkv, N, N, d, block, topk, idx,
+                                workspace, workspace_bytes, stream);
+}
+
+int moba_attn_fwd_chunk(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *idx,
+                        int batch, int hq, int hkv, int N, int Nk, int d, int block, int topk,
+                        int window, float scale, moba_tensor out, float *lse, void *workspace,
+                        size_t workspace_bytes, void *stream) {
+  const int q_off = Nk - N;
+  int rc = check_moba_shape(batch, hq, hkv, N, d, block, topk, q_off);
   if (rc) return rc;
   if (window < 0) return MOBA_ERR_ARG;
   if ((rc = check_tensor(q)) || (rc = check_tensor(k)) || (rc = check_tensor(v)) ||
@@ -319,13 +340,13 @@ int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *id
   if (!idx || !lse) return MOBA_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
     return MOBA_ERR_ALIGN;
-  const WorkspaceLayout w = make_layout(batch, hq, hkv, N, d, block, topk);
+  const WorkspaceLayout w = make_layout(batch, hq, hkv, N, d, block, topk, q_off);
   if (!workspace || workspace_bytes < w.total) return MOBA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return MOBA_ERR_ALIGN;
   int nsm = 0;
   if ((rc = check_device(&nsm))) return rc;
   CUtensorMap maps[6];
-  if ((rc = make_attn_maps(maps, q, k, v, batch, hq, hkv, N, d))) return rc;
+  if ((rc = make_attn_maps(maps, q, k, v, batch, hq, hkv, N, Nk, d))) return rc;
   // The gathered pass reads q through 2-D row maps in place of the 4-D tile maps.
   CUtensorMap gmaps[6];
   for (int a = 0; a < 6; ++a) gmaps[a] = maps[a];
@@ -342,6 +363,7 @@ int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *id
   p.idx = idx;
   p.batch = batch; p.hq = hq; p.hkv = hkv; p.N = N; p.d = d; p.block = block; p.topk = topk;
   p.window = window; p.G = w.G;
+  p.q_off = q_off;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
   p.scale_log2 = sc * 1.4426950408889634f;
   p.is_moba = 1;
@@ -384,11 +406,20 @@ int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *id
       mp.chunk_rows = w.chunk_rows;
       mp.row_begin = p.row_begin;
       mp.row_end = p.row_end;
+      mp.q_off = q_off;
       if ((rc = launch_status(launch_merge(mp, st)))) return rc;
       record_pass_event(ev++, c, st);
     }
   }
   return MOBA_OK;
+}
+
+int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *idx, int batch,
+                  int hq, int hkv, int N, int d, int block, int topk, int window, float scale,
+                  moba_tensor out, float *lse, void *workspace, size_t workspace_bytes,
+                  void *stream) {
+  return moba_attn_fwd_chunk(q, k, v, idx, batch, hq, hkv, N, N, d, block, topk, window, scale,
+                             out, lse, workspace, workspace_bytes, stream);
 }
 
 int moba_set_pass_events(void *const *events, int count) {
@@ -399,9 +430,14 @@ int moba_set_pass_events(void *const *events, int count) {
   return MOBA_OK;
 }
 
-int swa_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq, int hkv, int N,
-                 int d, int window, float scale, moba_tensor out, float *lse, void *stream) {
+int swa_attn_fwd_chunk(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq, int hkv,
+                       int N, int Nk, int d, int window, float scale, moba_tensor out, float *lse,
+                       void *stream) {
   if (batch < 1 || hq < 1 || hkv < 1 || N < 1 || hq % hkv) return MOBA_ERR_SHAPE;
+  // Query row i sits at key position Nk - N + i; with a chunk (Nk > N) the offset must
+  // be a multiple of 128 (query tiles).
+  const int q_off = Nk - N;
+  if (q_off < 0 || q_off % kTileRows || (long long)Nk >= (1ll << 31)) return MOBA_ERR_SHAPE;
   if (window < 1) return MOBA_ERR_ARG;
   int rc = check_attn_dim(d);
   if (rc) return rc;
@@ -413,7 +449,7 @@ int swa_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq,
   int nsm = 0;
   if ((rc = check_device(&nsm))) return rc;
   CUtensorMap maps[6];
-  if ((rc = make_attn_maps(maps, q, k, v, batch, hq, hkv, N, d))) return rc;
+  if ((rc = make_attn_maps(maps, q, k, v, batch, hq, hkv, N, Nk, d))) return rc;
   AttnParams p{};
   if ((rc = status_words(&p.status))) return rc;
   p.q = static_cast<const uint16_t *>(q.ptr);
@@ -423,7 +459,8 @@ int swa_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq,
   p.lse = lse;
   p.idx = nullptr;
   p.batch = batch; p.hq = hq; p.hkv = hkv; p.N = N; p.d = d; p.block = 0; p.topk = 0;
-  p.window = window < N ? window : N;
+  p.window = window < Nk ? window : Nk;
+  p.q_off = q_off;
   p.G = hq / hkv;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
   p.scale_log2 = sc * 1.4426950408889634f;
@@ -434,6 +471,11 @@ int swa_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq,
   p.npast = 0;
   const int grid = p.ntiles < nsm ? p.ntiles : nsm;
   return launch_status(launch_attn(maps, p, kQueryMajor, grid, static_cast<cudaStream_t>(stream)));
+}
+
+int swa_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq, int hkv, int N,
+                 int d, int window, float scale, moba_tensor out, float *lse, void *stream) {
+  return swa_attn_fwd_chunk(q, k, v, batch, hq, hkv, N, N, d, window, scale, out, lse, stream);
 }
 
 int moba_device_status(void) {

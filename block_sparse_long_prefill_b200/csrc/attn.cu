@@ -84,10 +84,10 @@ struct Bars {
 // One stream's tile of a work unit.
 struct Tile {
   int b, h, hk;
-  int i0;      // query-major: first row
+  int i0;      // query-major: first query row (at key position q_off + i0)
   int rows;    // valid rows (0: the stream is idle in this unit)
   int ent0;    // gathered: first list entry
-  int cB;      // query-major MoBA: first key of the own block
+  int cB;      // query-major MoBA: first key (position) of the own block
 };
 
 // A work unit: two tiles over one key-chunk sequence.
@@ -116,7 +116,10 @@ __device__ __forceinline__ void query_major_unit(const AttnParams &p, int u, Uni
     g1 = (2 * ph + 1 < p.G) ? 2 * ph + 1 : -1;
     hb /= per_hk;                                          // (b, hk)
   } else {
-    // Row-tile pairs; for MoBA a pair never crosses a block boundary.
+    // Row-tile pairs, grouped by tpb tiles from the pass's first row: for MoBA a pair
+    // stays inside one block when that row starts a block; otherwise (a chunk that
+    // starts mid-block) a pair may span two blocks, which the union key range and the
+    // per-row masks below handle.
     const int tpb = p.is_moba ? p.block / kTileRows : nq;   // tiles per pairing group
     const int ppg = (tpb + 1) / 2;                         // pairs per group
     const int ngroups = (nq + tpb - 1) / tpb;
@@ -147,14 +150,16 @@ __device__ __forceinline__ void query_major_unit(const AttnParams &p, int u, Uni
     t.ent0 = 0;
     t.cB = 0;
     if (t.rows == 0) continue;
-    const int ilast = t.i0 + t.rows - 1;
+    // Key positions: row i0 of q sits at position q_off + i0.
+    const int a0 = p.q_off + t.i0;
+    const int ilast = a0 + t.rows - 1;
     int first;
     if (p.is_moba) {
-      t.cB = (t.i0 / p.block) * p.block;
+      t.cB = (a0 / p.block) * p.block;
       first = t.cB;
-      if (p.window > 0) first = min(t.cB, (max(0, t.i0 - p.window + 1) / kTileKeys) * kTileKeys);
+      if (p.window > 0) first = min(t.cB, (max(0, a0 - p.window + 1) / kTileKeys) * kTileKeys);
     } else {
-      first = (max(0, t.i0 - p.window + 1) / kTileKeys) * kTileKeys;
+      first = (max(0, a0 - p.window + 1) / kTileKeys) * kTileKeys;
     }
     lo = min(lo, first);
     hi = max(hi, ilast);
@@ -578,6 +583,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const int32_t *irow = (MODE == kQueryMajor && p.is_moba && live)
                                 ? p.idx + (((int64_t)t.b * p.hq + h) * p.N + i) * p.topk
                                 : nullptr;
+      const int pos = p.q_off + i;        // the row's key position (masks)
+      const int a0 = p.q_off + t.i0;      // query-major: the tile's first key position
       float m_run = -INFINITY, l_run = 0.f;
       for (int m = 0; m < w.nc; ++m, ++scnt) {
         ok = mbar_wait(&bar.s_full[x], scnt & 1, abort, p.status, site0 + 12);
@@ -603,20 +610,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               const bool none = covered || !live || p.window <= 0;
 #pragma unroll
               for (int e = 0; e < 128; ++e)
-                if (none || i - (key0 + e) >= p.window) s[e] = -INFINITY;
-            } else if (key0 + kTileKeys > t.i0) {
+                if (none || pos - (key0 + e) >= p.window) s[e] = -INFINITY;
+            } else if (key0 + kTileKeys > a0) {
 #pragma unroll
               for (int e = 0; e < 128; ++e)
-                if (key0 + e > i) s[e] = -INFINITY;
+                if (key0 + e > pos) s[e] = -INFINITY;
             }
           } else {
-            const bool full = (key0 + kTileKeys - 1 <= t.i0) &&
-                              (key0 >= t.i0 + t.rows - 1 - p.window + 1);
+            const bool full = (key0 + kTileKeys - 1 <= a0) &&
+                              (key0 >= a0 + t.rows - 1 - p.window + 1);
             if (!full) {
 #pragma unroll
               for (int e = 0; e < 128; ++e) {
                 const int j = key0 + e;
-                if (j > i || i - j >= p.window) s[e] = -INFINITY;
+                if (j > pos || pos - j >= p.window) s[e] = -INFINITY;
               }
             }
           }

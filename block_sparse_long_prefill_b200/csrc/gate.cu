@@ -107,7 +107,7 @@ __device__ __forceinline__ uint64_t gate_desc(uint32_t tile, int ks, int rows) {
 // hk * G + g.  Ordered so that consecutive tiles share the kv-head.
 struct GateTile {
   int b, hk, g, rt;
-  int c;        // own block of the tile's rows: 128 rt / block
+  int c;        // own block of the tile's rows: (q_off + 128 rt) / block
   int chunk;    // query chunk of the tile's rows: 128 rt / chunk_rows
 };
 __device__ __forceinline__ GateTile gate_tile(const GateParams &p, int t) {
@@ -119,7 +119,7 @@ __device__ __forceinline__ GateTile gate_tile(const GateParams &p, int t) {
   t /= nrt;
   r.hk = t % p.hkv;
   r.b = t / p.hkv;
-  r.c = (r.rt * 128) / p.block;
+  r.c = (p.q_off + r.rt * 128) / p.block;
   r.chunk = (r.rt * 128) / p.chunk_rows;
   return r;
 }
@@ -129,11 +129,11 @@ __device__ __forceinline__ void gate_tile_next(const GateParams &p, GateTile &r)
   if (++r.g < p.G) return;
   r.g = 0;
   ++r.rt;
-  if (r.rt * 128 == (r.c + 1) * p.block) ++r.c;
+  if (p.q_off + r.rt * 128 == (r.c + 1) * p.block) ++r.c;
   if (r.rt * 128 == (r.chunk + 1) * p.chunk_rows) ++r.chunk;
   if (r.rt < p.N / 128) return;
   r.rt = 0;
-  r.c = 0;
+  r.c = p.q_off / p.block;
   r.chunk = 0;
   if (++r.hk < p.hkv) return;
   r.hk = 0;

@@ -43,7 +43,7 @@ __device__ __forceinline__ void merge_row(const MergeParams &p, int row, int nro
   const int bh = row / nrows, il = row - bh * nrows;
   const int h = bh % p.hq, b = bh / p.hq;
   const int i = p.row_begin + il;
-  const int c = i / p.block;
+  const int c = (p.q_off + i) / p.block;  // own block of the row's key position
   const int npast = p.topk - 1;
   // Chunk-local row: the pass covers rows [row_begin, row_end) of one chunk.
   const int64_t pbase = ((int64_t)bh * p.chunk_rows + il) * p.topk;

@@ -17,7 +17,8 @@ constexpr size_t kPartialCapBytes = size_t(4) << 30;  // partial outputs kept pe
 // List L = ((chunk * batch + b) * hkv + hk) * nblk + j holds the (row, q-head, slot)
 // triples of the rows of query chunk `chunk` that picked past block j.
 struct WorkspaceLayout {
-  int nblk;         // ceil(N / block): a partial last block when block does not divide N
+  int nblk;         // ceil((q_off + N) / block): a partial last block when block does not
+                    // divide the key count
   int G;            // hq / hkv
   int npast;        // topk - 1: partial slots per row
   int chunk_rows;   // query rows per pass (multiple of 128)
@@ -40,10 +41,12 @@ struct WorkspaceLayout {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// N query rows; the keys run over q_off + N positions (q_off > 0: a chunk of a longer
+// prefill whose queries are the last N positions).
 inline WorkspaceLayout make_layout(int batch, int hq, int hkv, int N, int d, int block,
-                                   int topk) {
+                                   int topk, int q_off = 0) {
   WorkspaceLayout w{};
-  w.nblk = (N + block - 1) / block;
+  w.nblk = (q_off + N + block - 1) / block;
   w.G = hq / hkv;
   w.npast = topk - 1;
   // Partials exist only when a row can attend past blocks: topk slots per row then.
@@ -81,6 +84,7 @@ struct SelectParams {
   int32_t *idx;          // [batch, hq, N, topk]
   int *counts;           // workspace list counts
   int batch, hq, hkv, N, d, block, topk, nblk, G, chunk_rows;
+  int q_off;             // position of query row 0 among the keys
 };
 
 // Parameters of the tensor-core gate / top-k kernel (q and the pooled keys arrive
@@ -90,6 +94,7 @@ struct GateParams {
   int32_t *idx;          // [batch, hq, N, topk]
   int *counts;           // workspace list counts
   int batch, hq, hkv, N, d, block, topk, nblk, G, chunk_rows;
+  int q_off;             // position of query row 0 among the keys (a multiple of 128)
   int qstages;           // query tile ring depth (set by the launcher)
   int kslots;            // pooled-key staging slots, 1 or 2 (set by the launcher)
   int *sched;            // tile counter, zero at launch (the word after the list counts)
@@ -106,6 +111,7 @@ struct ScatterParams {
   int *cursor;
   uint32_t *entries;
   int batch, hq, hkv, N, block, topk, nblk, G, chunk_rows;
+  int q_off;               // position of query row 0 among the keys
   // Unit table (written by the scatter grid from the scanned offsets).
   const int *counts;
   const int *listoff;
@@ -130,8 +136,10 @@ struct AttnParams {
   int64_t o_sb, o_sh, o_sn;
   float *lse;              // [batch, hq, N]
   const int32_t *idx;      // [batch, hq, N, topk] (MoBA) or null (SWA)
-  // Problem.
+  // Problem: N query rows; keys and values run over q_off + N positions, query row i
+  // sits at position q_off + i (q_off a multiple of 128).
   int batch, hq, hkv, N, d, block, topk, window, G;
+  int q_off;
   float scale_log2;        // scale * log2(e)
   int is_moba;             // 0: sliding window only (swa_attn_fwd)
   // Gathered pass: 1 when the query rows are fetched by TMA gather4 through a 2-D map
@@ -160,6 +168,7 @@ struct MergeParams {
   int64_t o_sb, o_sh, o_sn;
   float *lse;              // [batch, hq, N]
   int batch, hq, N, d, block, topk, chunk_rows, row_begin, row_end;
+  int q_off;               // position of query row 0 among the keys
 };
 
 }  // namespace moba

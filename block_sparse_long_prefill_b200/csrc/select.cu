@@ -127,8 +127,9 @@ gate_topk_kernel(const SelectParams p) {
   const int hk = h / p.G;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rows = min(kGateRows, p.N - i0);
-  // Past blocks any row of this tile may score.
-  const int nb = min(p.nblk, (i0 + rows - 1) / p.block);
+  // Past blocks any row of this tile may score (query row i sits at key position
+  // q_off + i).
+  const int nb = min(p.nblk, (p.q_off + i0 + rows - 1) / p.block);
   const int lds = ((nb + 31) & ~31) + 4;
   int *hist = reinterpret_cast<int *>(ss + kGateRows * lds);               // [nblk]
   const int wr0 = warp * 16;  // this warp's first row in the tile
@@ -157,7 +158,7 @@ gate_topk_kernel(const SelectParams p) {
   const uint16_t *kb = p.kbar_split + ((int64_t)b * p.hkv + hk) * 2 * p.nblk * D;
   // Largest own-block index among this warp's rows: n-tiles at or past it are skipped.
   const int wlast = min(i0 + wr0 + 15, p.N - 1);
-  const int cw = (wr0 < rows) ? wlast / p.block : 0;
+  const int cw = (wr0 < rows) ? (p.q_off + wlast) / p.block : 0;
   const int nchunk = (nb + kGateChunk - 1) / kGateChunk;
   for (int ch = 0; ch < nchunk; ++ch) {
     const int j0 = ch * kGateChunk;
@@ -218,7 +219,7 @@ gate_topk_kernel(const SelectParams p) {
     const int r = wr0 + pass * 8 + g;
     const int i = i0 + r;
     const bool live = r < rows;
-    const int c = live ? i / p.block : 0;
+    const int c = live ? (p.q_off + i) / p.block : 0;
     float *srow = ss + r * lds;
     int *sel = sel_base + r * 32;
     const int npick = min(npick_max, c);
@@ -315,7 +316,7 @@ scatter_kernel(const ScatterParams p) {
   const int tid = threadIdx.x;
   const int npast = p.topk - 1;
   const int rows = min(kTileRows, p.N - i0);
-  const int nb = min(p.nblk, (i0 + rows - 1) / p.block);
+  const int nb = min(p.nblk, (p.q_off + i0 + rows - 1) / p.block);
 
   {
     // Unit table, grid-stride over the lists.
@@ -352,7 +353,7 @@ scatter_kernel(const ScatterParams p) {
   for (int e = tid; e < pairs; e += kScatterThreads) {
     const int g = e / kTileRows, r = e % kTileRows;
     const bool row_ok = r < rows;
-    const int c = (i0 + r) / p.block;
+    const int c = (p.q_off + i0 + r) / p.block;
     for (int s = 0; s < npast; ++s) {
       const int j = row_ok ? pick(g, r, s) : -1;
       // Past picks come first; the own block and the -1 padding end them.
@@ -372,7 +373,7 @@ scatter_kernel(const ScatterParams p) {
     const int g = e / kTileRows, r = e % kTileRows;
     const bool row_ok = r < rows;
     const int i = i0 + r;
-    const int c = i / p.block;
+    const int c = (p.q_off + i) / p.block;
     for (int s = 0; s < npast; ++s) {
       const int j = row_ok ? pick(g, r, s) : -1;
       if (j < 0 || j >= c) break;

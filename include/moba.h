@@ -132,6 +132,32 @@ int swa_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq,
                  int d, int window, float scale, moba_tensor out, float *lse, void *stream);
 
 /*
+ * Chunked prefill: N query rows that are the last N of Nk positions (query row i sits
+ * at position Nk - N + i, as when a long prompt is prefilled chunk by chunk against
+ * the keys and values cached so far).  Each row's block choice and attention are those
+ * of the same row in a whole prefill of the Nk positions ([MoBA] §"인과성 보존": a row
+ * sees only keys at or before its own position, so it does not depend on the other
+ * rows).  k and v hold the Nk positions ([batch, hkv, Nk, d]); pool them with
+ * moba_pool_keys(k, ..., Nk, ...).  q, idx, out and lse hold the N query rows.
+ * Nk - N must be a multiple of 128 (and N, block as for the whole prefill); Nk = N is
+ * the whole prefill, and the calls without _chunk are exactly that.  The workspace is
+ * sized by moba_workspace_size_chunk for the same (N, Nk).  swa_attn_fwd_chunk takes
+ * any N and window with Nk - N a multiple of 128.
+ */
+int moba_workspace_size_chunk(int batch, int hq, int hkv, int N, int Nk, int d, int block,
+                              int topk, size_t *bytes);
+int moba_select_topk_chunk(moba_tensor q, const void *kbar_split, int batch, int hq, int hkv,
+                           int N, int Nk, int d, int block, int topk, int32_t *idx,
+                           void *workspace, size_t workspace_bytes, void *stream);
+int moba_attn_fwd_chunk(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *idx,
+                        int batch, int hq, int hkv, int N, int Nk, int d, int block, int topk,
+                        int window, float scale, moba_tensor out, float *lse, void *workspace,
+                        size_t workspace_bytes, void *stream);
+int swa_attn_fwd_chunk(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq, int hkv,
+                       int N, int Nk, int d, int window, float scale, moba_tensor out, float *lse,
+                       void *stream);
+
+/*
  * The whole MoBA prefill (moba_pool_keys, moba_select_topk, moba_attn_fwd) without any
  * caller-provided workspace, for callers that cannot allocate device memory: code
  * inside a CUDA-graph capture that forbids allocation, plugins whose host framework

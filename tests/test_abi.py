@@ -96,3 +96,20 @@ def test_valid_call_without_a_device_reports_no_device():
     ok = moba.MobaTensor(1 << 20, 8 * 1024, 8 * 1024, 128)
     rc = lib.swa_attn_fwd(ok, ok, ok, 1, 1, 1, 1024, 128, 64, 0.0, ok, 1 << 20, None)
     assert rc == -8
+
+
+def test_chunk_workspace_and_offset_checks():
+    """Chunked prefill (N query rows, the last N of Nk positions): the workspace of the
+    last 8K rows of a 32K context is smaller than the whole prefill's, and the query
+    offset Nk - N must be a non-negative multiple of 128."""
+    whole = moba.workspace_size(1, 32, 8, 32768, 128, 512, 3)
+    chunk = moba.workspace_size_chunk(1, 32, 8, 8192, 32768, 128, 512, 3)
+    assert 0 < chunk < whole
+    assert moba.workspace_size_chunk(1, 32, 8, 32768, 32768, 128, 512, 3) == whole
+    lib = moba.library()
+    out = ctypes.c_size_t(0)
+    assert lib.moba_workspace_size_chunk(1, 32, 8, 8192, 8192 + 64, 128, 512, 3, ctypes.byref(out)) == -1
+    assert lib.moba_workspace_size_chunk(1, 32, 8, 8192, 4096, 128, 512, 3, ctypes.byref(out)) == -1
+    ok = moba.MobaTensor(1 << 20, 8 * 1024, 8 * 1024, 128)
+    assert lib.swa_attn_fwd_chunk(ok, ok, ok, 1, 1, 1, 1000, 1064, 128, 64, 0.0, ok, 1 << 20, None) == -1
+    assert lib.swa_attn_fwd_chunk(ok, ok, ok, 1, 1, 1, 1000, 900, 128, 64, 0.0, ok, 1 << 20, None) == -1

@@ -31,6 +31,7 @@ class Workload:
     window: int = 0         # causal window (0 = none)
     key_offset_std: float = 0.0
     sampled_rows: bool = False   # the oracle checks sampled rows only
+    q_len: int = 0               # chunked prefill: the queries are the last q_len positions
     note: str = ""
 
     @property
@@ -39,7 +40,17 @@ class Workload:
 
     @property
     def nblocks(self) -> int:
-        return self.seqlen // self.block if self.block else 0
+        return -(-self.seqlen // self.block) if self.block else 0
+
+    @property
+    def nq(self) -> int:
+        """Query rows: q_len for a chunked prefill, else all seqlen positions."""
+        return self.q_len or self.seqlen
+
+    @property
+    def q_off(self) -> int:
+        """Position of query row 0 among the keys."""
+        return self.seqlen - self.nq
 
 
 # The five workloads the method is measured and checked on.
@@ -55,6 +66,10 @@ WORKLOADS = {
                           note="GQA 8/4, 32 blocks of 2048, top-16 unioned with window 512"),
     "moba1m": Workload("moba1m", 1, 32, 8, 1 << 20, 128, block=4096, topk=12, key_offset_std=0.5,
                        sampled_rows=True, note="1M tokens, 256 blocks of 4096, top-12"),
+    "gqa32k_chunk8k": Workload("gqa32k_chunk8k", 1, 32, 8, 32768, 128, block=512, topk=3,
+                               key_offset_std=0.5, q_len=8192,
+                               note="chunked prefill: the last 8192 queries of the gqa32k "
+                                    "context against all 32768 keys"),
 }
 
 
