@@ -137,6 +137,31 @@ def select_topk(scores: np.ndarray, N: int, block: int, topk: int, rows=None):
     return idx, gap
 
 
+def select_static(N: int, block: int, topk: int, sink: int, rows=None, batch: int = 1,
+                  hq: int = 1) -> np.ndarray:
+    """[MoBA] §"MoBA의 구현" preamble on static sparse attention as special cases of MoBA:
+    sliding-window attention is MoBA whose gate always picks the most recent blocks, and
+    an attention sink is MoBA whose gate always picks the first block together with the
+    most recent ones.  Row i (own block c = i / block) keeps its own block and k-1 past
+    blocks: the first ``sink`` blocks and the k-1-sink most recent blocks before c (all
+    past blocks when c <= k-1).  No score is involved.  Returns int32
+    [batch, hq, len(rows), topk], ascending, -1 padded (the same for every batch and
+    head)."""
+    if not 0 <= sink <= topk - 1:
+        raise ValueError("need 0 <= sink <= topk - 1")
+    r = _rows(rows, N)
+    out = np.full((len(r), topk), -1, dtype=np.int32)
+    for t, i in enumerate(r):
+        c = int(i) // block
+        if c <= topk - 1:
+            keep = list(range(c + 1))
+        else:
+            recent = topk - 1 - sink
+            keep = list(range(sink)) + list(range(c - recent, c)) + [c]
+        out[t, :len(keep)] = keep
+    return np.broadcast_to(out, (batch, hq, len(r), topk)).copy()
+
+
 def attention(q, k, v, *, mode: int, block: int = 1, topk: int = 1, idx=None,
               window: int = 0, scale: float | None = None, rows=None):
     """Softmax attention over each row's key set (see ``orc_attention``).

@@ -264,3 +264,32 @@ def test_rows_before_a_partial_block_ignore_it():
                              Nc, B, k_)
     assert np.array_equal(full[0][:, :, :Nc], cut[0])
     assert np.array_equal(full[1][:, :, :Nc], cut[1])
+
+
+# ------------------------------------------------------------------- static gates
+
+@pytest.mark.parametrize("sink", [0, 1, 2])
+def test_static_gate_is_moba_top_k_on_scores_that_rank_those_blocks(sink):
+    """The MoBA page: sliding-window attention is MoBA whose gate always picks the most
+    recent blocks, an attention sink MoBA whose gate also picks the first block.  With
+    pooled keys whose scores rise with the block index (and the first `sink` blocks
+    above all of them), the score-based top-k picks exactly the static rule's blocks."""
+    B, n, d, k_ = 16, 12, 4, 5
+    N = n * B
+    q = torch.ones(1, 1, N, d)
+    k = torch.zeros(1, 1, N, d)
+    for j in range(n):
+        k[0, 0, j * B:(j + 1) * B, :] = 100.0 + 4.0 * j if j >= sink else 1000.0 + j
+    q, k = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    s = oracle.gate_scores(q, oracle.pool_keys(k, B), B)
+    idx, _ = oracle.select_topk(s, N, B, k_)
+    assert np.array_equal(idx, oracle.select_static(N, B, k_, sink))
+
+
+def test_static_gate_definition():
+    """Closed form of a few rows: B = 4, k = 4, sink = 1."""
+    idx = oracle.select_static(40, 4, 4, 1, rows=[0, 5, 9, 13, 39])
+    assert idx[0, 0].tolist() == [[0, -1, -1, -1], [0, 1, -1, -1], [0, 1, 2, -1], [0, 1, 2, 3],
+                                  [0, 7, 8, 9]]
+    with pytest.raises(ValueError):
+        oracle.select_static(40, 4, 4, 4)
