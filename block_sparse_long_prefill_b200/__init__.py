@@ -31,7 +31,8 @@ _STATUS = {
 # Entry points declared in include/moba.h.
 ABI_FUNCTIONS = ("moba_workspace_size", "moba_pool_keys", "moba_select_topk", "moba_attn_fwd",
                  "swa_attn_fwd", "moba_workspace_size_chunk", "moba_select_topk_chunk",
-                 "moba_attn_fwd_chunk", "swa_attn_fwd_chunk", "moba_prefill_static",
+                 "moba_attn_fwd_chunk", "swa_attn_fwd_chunk", "moba_select_static",
+                 "moba_prefill_static",
                  "moba_device_status", "moba_set_pass_events", "moba_status_string")
 
 
@@ -63,6 +64,7 @@ def _load():
     lib.moba_attn_fwd_chunk.argtypes = [T, T, T, P, I, I, I, I, I, I, I, I, I, ctypes.c_float, T, P,
                                         P, S, P]
     lib.swa_attn_fwd_chunk.argtypes = [T, T, T, I, I, I, I, I, I, I, ctypes.c_float, T, P, P]
+    lib.moba_select_static.argtypes = [I, I, I, I, I, I, I, I, I, P, P, S, P]
     lib.moba_prefill_static.argtypes = [T, T, T, I, I, I, I, I, I, I, I, ctypes.c_float, T, P, P]
     lib.moba_device_status.argtypes = []
     lib.moba_set_pass_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), I]
@@ -222,6 +224,21 @@ def swa_attn_fwd_chunk(q, k, v, window: int, scale: float = 0.0, out=None, lse=N
            _lib.swa_attn_fwd_chunk(_t(q), _t(k), _t(v), b, hq, hkv, N, Nk, d, window, float(scale),
                                    _t(out), lse.data_ptr(), _stream(stream)))
     return out, lse
+
+
+def moba_select_static(batch: int, hq: int, hkv: int, N: int, d: int, block: int, topk: int,
+                       sink: int, workspace: torch.Tensor, kv_len=None, idx=None, stream=None,
+                       device="cuda"):
+    """Static gate in place of moba_select_topk: own block, the first ``sink`` blocks and
+    the most recent past blocks (sink = 0: sliding window at block granularity; sink = 1:
+    an attention sink).  N query rows, the last N of ``kv_len`` (default N) positions."""
+    kv = kv_len or N
+    if idx is None:
+        idx = torch.empty(batch, hq, N, topk, dtype=torch.int32, device=device)
+    _check("moba_select_static",
+           _lib.moba_select_static(batch, hq, hkv, N, kv, d, block, topk, sink, idx.data_ptr(),
+                                   workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return idx
 
 
 def moba_prefill_chunk(q, k, v, block: int, topk: int, window: int = 0, stream=None):

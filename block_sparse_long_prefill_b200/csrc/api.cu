@@ -22,6 +22,9 @@ cudaError_t launch_gate(const SelectParams &p, cudaStream_t st);
 cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileoff, int nlists,
                         cudaStream_t st);
 cudaError_t launch_scatter(ScatterParams p, cudaStream_t st);
+cudaError_t launch_static_select(int32_t *idx, int *counts, int batch, int hq, int hkv, int N,
+                                 int q_off, int block, int topk, int sink, int nblk, int chunk_rows,
+                                 cudaStream_t st);
 cudaError_t launch_gate_tc(const CUtensorMap *maps, const GateParams &p, int grid, cudaStream_t st);
 bool gate_tc_supports(int nblk, int topk);
 cudaError_t launch_attn(const CUtensorMap *maps, const AttnParams &p, int mode, int grid,
@@ -310,6 +313,47 @@ int moba_select_topk_chunk(moba_tensor q, const void *kbar_split, int batch, int
   cp.listoff = listoff;
   cp.tileoff = tileoff;
   cp.tiles = tiles;
+  cp.nlists = w.nlists;
+  cp.cursor = cursor;
+  cp.entries = reinterpret_cast<uint32_t *>(ws + w.off_entries);
+  cp.batch = batch; cp.hq = hq; cp.hkv = hkv; cp.N = N; cp.block = block; cp.topk = topk;
+  cp.nblk = w.nblk; cp.G = w.G; cp.chunk_rows = w.chunk_rows;
+  cp.q_off = q_off;
+  return launch_status(launch_scatter(cp, st));
+}
+
+int moba_select_static(int batch, int hq, int hkv, int N, int Nk, int d, int block, int topk,
+                       int sink, int32_t *idx, void *workspace, size_t workspace_bytes,
+                       void *stream) {
+  const int q_off = Nk - N;
+  int rc = check_moba_shape(batch, hq, hkv, N, d, block, topk, q_off);
+  if (rc) return rc;
+  if (sink < 0 || sink > topk - 1) return MOBA_ERR_ARG;
+  if (!idx) return MOBA_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(idx) & 3u) return MOBA_ERR_ALIGN;
+  const WorkspaceLayout w = make_layout(batch, hq, hkv, N, d, block, topk, q_off);
+  if (!workspace || workspace_bytes < w.total) return MOBA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MOBA_ERR_ALIGN;
+  if ((rc = check_device(nullptr))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char *ws = static_cast<char *>(workspace);
+  int *counts = reinterpret_cast<int *>(ws + w.off_counts);
+  if (cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)(w.nlists + 2), st) != cudaSuccess)
+    return MOBA_ERR_LAUNCH;
+  if ((rc = launch_status(launch_static_select(idx, counts, batch, hq, hkv, N, q_off, block, topk,
+                                               sink, w.nblk, w.chunk_rows, st))))
+    return rc;
+  if (w.npast == 0) return MOBA_OK;
+  int *cursor = reinterpret_cast<int *>(ws + w.off_cursor);
+  int *listoff = reinterpret_cast<int *>(ws + w.off_listoff);
+  int *tileoff = reinterpret_cast<int *>(ws + w.off_tileoff);
+  if ((rc = launch_status(launch_scan(counts, cursor, listoff, tileoff, w.nlists, st)))) return rc;
+  ScatterParams cp{};
+  cp.idx = idx;
+  cp.counts = counts;
+  cp.listoff = listoff;
+  cp.tileoff = tileoff;
+  cp.tiles = reinterpret_cast<int4 *>(ws + w.off_tiles);
   cp.nlists = w.nlists;
   cp.cursor = cursor;
   cp.entries = reinterpret_cast<uint32_t *>(ws + w.off_entries);

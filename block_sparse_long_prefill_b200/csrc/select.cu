@@ -383,6 +383,59 @@ scatter_kernel(const ScatterParams p) {
   }
 }
 
+// ------------------------------------------------------------ static gates
+//
+// [MoBA] §"MoBA의 구현" preamble: sliding-window attention is MoBA whose gate always
+// picks the most recent blocks; an attention sink is MoBA whose gate picks the first
+// block together with the most recent ones.  Row i (own block c) keeps block c, the
+// first `sink` blocks and the k-1-sink most recent blocks before c (all past blocks
+// when c <= k-1).  The choice depends on c alone, so one CTA = one 128-row tile (one
+// c) of one (batch, kv-head): it writes the tile's G * 128 idx rows and adds G * 128 per
+// past pick to the list counts.
+constexpr int kStaticThreads = 256;
+
+__global__ void __launch_bounds__(kStaticThreads)
+static_select_kernel(int32_t *__restrict__ idx, int *__restrict__ counts, int batch, int hq,
+                     int hkv, int N, int q_off, int block, int topk, int sink, int nblk,
+                     int chunk_rows) {
+  const int i0 = blockIdx.x * kTileRows;
+  const int hk = blockIdx.y, b = blockIdx.z;
+  const int G = hq / hkv;
+  const int rows = min(kTileRows, N - i0);
+  const int c = (q_off + i0) / block;
+  const int npast = topk - 1;
+  const int recent = npast - sink;
+  // Entry s of the tile's (shared) choice list.
+  auto pick = [&](int s) -> int {
+    if (c <= npast) return s < c ? s : (s == c ? c : -1);
+    if (s < sink) return s;
+    if (s < npast) return c - recent + (s - sink);
+    return s == npast ? c : -1;
+  };
+  // Each head's rows i0 .. i0 + rows - 1 are one contiguous run of rows * topk words.
+  const int run = rows * topk;
+  for (int g = 0; g < G; ++g) {
+    int32_t *dst = idx + (((int64_t)b * hq + (int64_t)hk * G + g) * N + i0) * topk;
+    for (int e = threadIdx.x; e < run; e += kStaticThreads) dst[e] = pick(e % topk);
+  }
+  if (threadIdx.x < npast) {
+    const int j = pick(threadIdx.x);
+    if (j >= 0 && j < c) {
+      const int chunk = i0 / chunk_rows;
+      atomicAdd(&counts[(((int64_t)chunk * batch + b) * hkv + hk) * nblk + j], rows * G);
+    }
+  }
+}
+
+cudaError_t launch_static_select(int32_t *idx, int *counts, int batch, int hq, int hkv, int N,
+                                 int q_off, int block, int topk, int sink, int nblk, int chunk_rows,
+                                 cudaStream_t st) {
+  dim3 grid((N + kTileRows - 1) / kTileRows, hkv, batch);
+  static_select_kernel<<<grid, kStaticThreads, 0, st>>>(idx, counts, batch, hq, hkv, N, q_off,
+                                                        block, topk, sink, nblk, chunk_rows);
+  return cudaGetLastError();
+}
+
 // Host-side launchers (called by the ABI layer).
 cudaError_t launch_pool(const uint16_t *k, int64_t sb, int64_t sh, int64_t sn, int batch, int hkv,
                         int N, int d, int block, float *kbar, uint16_t *split, cudaStream_t st) {

@@ -158,6 +158,20 @@ int swa_attn_fwd_chunk(moba_tensor q, moba_tensor k, moba_tensor v, int batch, i
                        void *stream);
 
 /*
+ * Static gates ([MoBA] §"MoBA의 구현" preamble: sliding-window attention is MoBA whose
+ * gate always picks the most recent blocks; an attention sink is MoBA whose gate picks
+ * the first block together with the most recent ones): in place of moba_select_topk,
+ * row i (own block c, at position Nk - N + i) keeps block c, the first `sink` blocks and
+ * the topk-1-sink most recent blocks before c (all past blocks when c <= topk-1).  No
+ * score, no pooled keys.  Writes idx and the dispatch lists exactly as
+ * moba_select_topk_chunk does, for moba_attn_fwd_chunk (Nk = N: the whole prefill).
+ *   sink : 0 <= sink <= topk-1 (MOBA_ERR_ARG otherwise)
+ */
+int moba_select_static(int batch, int hq, int hkv, int N, int Nk, int d, int block, int topk,
+                       int sink, int32_t *idx, void *workspace, size_t workspace_bytes,
+                       void *stream);
+
+/*
  * The whole MoBA prefill (moba_pool_keys, moba_select_topk, moba_attn_fwd) without any
  * caller-provided workspace, for callers that cannot allocate device memory: code
  * inside a CUDA-graph capture that forbids allocation, plugins whose host framework

@@ -113,3 +113,11 @@ def test_chunk_workspace_and_offset_checks():
     ok = moba.MobaTensor(1 << 20, 8 * 1024, 8 * 1024, 128)
     assert lib.swa_attn_fwd_chunk(ok, ok, ok, 1, 1, 1, 1000, 1064, 128, 64, 0.0, ok, 1 << 20, None) == -1
     assert lib.swa_attn_fwd_chunk(ok, ok, ok, 1, 1, 1, 1000, 900, 128, 64, 0.0, ok, 1 << 20, None) == -1
+
+
+def test_static_gate_rejects_a_sink_beyond_the_list():
+    lib = moba.library()
+    assert lib.moba_select_static(1, 2, 1, 1024, 1024, 128, 128, 3, 3, 1 << 20, 1 << 20, 1 << 30,
+                                  None) == -4
+    assert lib.moba_select_static(1, 2, 1, 1024, 1024, 128, 128, 3, -1, 1 << 20, 1 << 20, 1 << 30,
+                                  None) == -4
