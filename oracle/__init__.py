@@ -137,6 +137,44 @@ def select_topk(scores: np.ndarray, N: int, block: int, topk: int, rows=None):
     return idx, gap
 
 
+def pool_minmax(k, block: int):
+    """The MoBA page: Quest is MoBA with smaller blocks and a min/max pooled block
+    representation.  Element-wise maximum and minimum of the keys of each block
+    (positions [j*B, min((j+1)*B, N))).  Returns (kmax, kmin) float64
+    [b, hkv, ceil(N/B), d]."""
+    kd = bf16_to_f64(k)
+    b, hkv, N, d = kd.shape
+    n = n_blocks(N, block)
+    kmax = np.empty((b, hkv, n, d))
+    kmin = np.empty((b, hkv, n, d))
+    for j in range(n):
+        blk = kd[:, :, j * block:min((j + 1) * block, N)]
+        kmax[:, :, j] = blk.max(axis=2)
+        kmin[:, :, j] = blk.min(axis=2)
+    return kmax, kmin
+
+
+def minmax_scores(q, kmax: np.ndarray, kmin: np.ndarray, block: int, rows=None) -> np.ndarray:
+    """Score of past block j for query row i: the largest inner product q_i can have
+    with a key inside block j's min/max box, sum_d max(q_d kmax_jd, q_d kmin_jd) (the
+    reading taken of the page's min/max pooled representation); -inf for j >= c, as in
+    gate_scores.  Returns float64 [b, hq, len(rows), n]."""
+    qd = bf16_to_f64(q)
+    b, hq, N, d = qd.shape
+    hkv, n = kmax.shape[1], kmax.shape[2]
+    G = hq // hkv
+    r = _rows(rows, N)
+    out = np.full((b, hq, len(r), n), -np.inf)
+    for h in range(hq):
+        qi = qd[:, h, r]                                     # [b, R, d]
+        hi = qi[:, :, None, :] * kmax[:, h // G][:, None]    # [b, R, n, d]
+        lo = qi[:, :, None, :] * kmin[:, h // G][:, None]
+        s = np.maximum(hi, lo).sum(-1)                       # [b, R, n]
+        c = (r // block)[None, :, None]
+        out[:, h] = np.where(np.arange(n)[None, None, :] < c, s, -np.inf)
+    return out
+
+
 def select_static(N: int, block: int, topk: int, sink: int, rows=None, batch: int = 1,
                   hq: int = 1) -> np.ndarray:
     """[MoBA] §"MoBA의 구현" preamble on static sparse attention as special cases of MoBA:

@@ -293,3 +293,41 @@ def test_static_gate_definition():
                                   [0, 7, 8, 9]]
     with pytest.raises(ValueError):
         oracle.select_static(40, 4, 4, 4)
+
+
+# ----------------------------------------------------------------- min/max pooling
+
+def test_minmax_pool_and_scores_bound_every_key():
+    """The min/max block score is an upper bound of q . k for every key k of the block,
+    reached when one key holds every coordinate's extreme of q's sign pattern; with one
+    key per block it is q . k itself (B = 1: token-level, like the mean)."""
+    B, N, d = 8, 64, 16
+    q = _bf16((1, 2, N, d), seed=71)
+    k = _bf16((1, 1, N, d), seed=72)
+    kmax, kmin = oracle.pool_minmax(k, B)
+    kd = oracle.bf16_to_f64(k)[0, 0]
+    np.testing.assert_array_equal(kmax[0, 0], kd.reshape(N // B, B, d).max(axis=1))
+    np.testing.assert_array_equal(kmin[0, 0], kd.reshape(N // B, B, d).min(axis=1))
+    s = oracle.minmax_scores(q, kmax, kmin, B)
+    qd = oracle.bf16_to_f64(q)[0]
+    for h in range(2):
+        for i in range(0, N, 5):
+            c = i // B
+            for j in range(c):
+                dots = qd[h, i] @ kd[j * B:(j + 1) * B].T
+                assert s[0, h, i, j] >= dots.max() - 1e-12
+                # the box corner that matches q's signs attains the score
+                corner = np.where(qd[h, i] >= 0, kmax[0, 0, j], kmin[0, 0, j])
+                assert abs(s[0, h, i, j] - qd[h, i] @ corner) <= 1e-12
+            assert np.all(np.isneginf(s[0, h, i, c:]))
+    s1 = oracle.minmax_scores(q, *oracle.pool_minmax(k, 1), 1)
+    ref = oracle.gate_scores(q, oracle.pool_keys(k, 1), 1)
+    np.testing.assert_allclose(s1, ref, rtol=0, atol=1e-12)
+
+
+def test_minmax_pool_partial_block():
+    k = _bf16((1, 1, 100, 8), seed=73)
+    kmax, kmin = oracle.pool_minmax(k, 64)
+    kd = oracle.bf16_to_f64(k)[0, 0]
+    np.testing.assert_array_equal(kmax[0, 0, 1], kd[64:].max(axis=0))
+    np.testing.assert_array_equal(kmin[0, 0, 1], kd[64:].min(axis=0))
