@@ -32,6 +32,7 @@ _STATUS = {
 ABI_FUNCTIONS = ("moba_workspace_size", "moba_pool_keys", "moba_select_topk", "moba_attn_fwd",
                  "swa_attn_fwd", "moba_workspace_size_chunk", "moba_select_topk_chunk",
                  "moba_attn_fwd_chunk", "swa_attn_fwd_chunk", "moba_select_static",
+                 "moba_pool_keys_minmax", "moba_select_topk_minmax",
                  "moba_prefill_static",
                  "moba_device_status", "moba_set_pass_events", "moba_status_string")
 
@@ -65,6 +66,8 @@ def _load():
                                         P, S, P]
     lib.swa_attn_fwd_chunk.argtypes = [T, T, T, I, I, I, I, I, I, I, ctypes.c_float, T, P, P]
     lib.moba_select_static.argtypes = [I, I, I, I, I, I, I, I, I, P, P, S, P]
+    lib.moba_pool_keys_minmax.argtypes = [T, I, I, I, I, I, P, P]
+    lib.moba_select_topk_minmax.argtypes = [T, P, I, I, I, I, I, I, I, I, P, P, S, P]
     lib.moba_prefill_static.argtypes = [T, T, T, I, I, I, I, I, I, I, I, ctypes.c_float, T, P, P]
     lib.moba_device_status.argtypes = []
     lib.moba_set_pass_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), I]
@@ -238,6 +241,33 @@ def moba_select_static(batch: int, hq: int, hkv: int, N: int, d: int, block: int
     _check("moba_select_static",
            _lib.moba_select_static(batch, hq, hkv, N, kv, d, block, topk, sink, idx.data_ptr(),
                                    workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return idx
+
+
+def moba_pool_keys_minmax(k: torch.Tensor, block: int, out=None, stream=None):
+    """Min/max pooling: bf16 [b, hkv, 2, n, d] with the block maxima (plane 0) and minima
+    (plane 1) of the keys."""
+    b, hkv, N, d = k.shape
+    n = -(-N // block)
+    if out is None:
+        out = torch.empty(b, hkv, 2, n, d, dtype=torch.bfloat16, device=k.device)
+    _check("moba_pool_keys_minmax",
+           _lib.moba_pool_keys_minmax(_t(k), b, hkv, N, d, block, out.data_ptr(), _stream(stream)))
+    return out
+
+
+def moba_select_topk_minmax(q, kminmax: torch.Tensor, block: int, topk: int, kv_len: int,
+                            workspace: torch.Tensor, idx=None, stream=None):
+    """Selection on min/max pooled blocks (score q+ . kmax + q- . kmin); N query rows,
+    the last N of ``kv_len`` positions."""
+    b, hq, N, d = q.shape
+    hkv = kminmax.shape[1]
+    if idx is None:
+        idx = torch.empty(b, hq, N, topk, dtype=torch.int32, device=q.device)
+    _check("moba_select_topk_minmax",
+           _lib.moba_select_topk_minmax(_t(q), kminmax.data_ptr(), b, hq, hkv, N, kv_len, d, block,
+                                        topk, idx.data_ptr(), workspace.data_ptr(),
+                                        workspace.numel(), _stream(stream)))
     return idx
 
 

@@ -22,6 +22,8 @@ cudaError_t launch_gate(const SelectParams &p, cudaStream_t st);
 cudaError_t launch_scan(const int *counts, int *cursor, int *listoff, int *tileoff, int nlists,
                         cudaStream_t st);
 cudaError_t launch_scatter(ScatterParams p, cudaStream_t st);
+cudaError_t launch_pool_minmax(const uint16_t *k, int64_t sb, int64_t sh, int64_t sn, int batch,
+                               int hkv, int N, int d, int block, uint16_t *planes, cudaStream_t st);
 cudaError_t launch_static_select(int32_t *idx, int *counts, int batch, int hq, int hkv, int N,
                                  int q_off, int block, int topk, int sink, int nblk, int chunk_rows,
                                  cudaStream_t st);
@@ -239,9 +241,14 @@ int moba_pool_keys(moba_tensor k, int batch, int hkv, int N, int d, int block, f
                                    static_cast<cudaStream_t>(stream)));
 }
 
-int moba_select_topk_chunk(moba_tensor q, const void *kbar_split, int batch, int hq, int hkv,
-                           int N, int Nk, int d, int block, int topk, int32_t *idx,
-                           void *workspace, size_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+// Selection over the block representation in `kbar_split`: the hi / lo split of the
+// means (minmax = 0; the tensor-core gate when it takes the problem) or the maxima /
+// minima planes of min/max pooling (minmax = 1; the general gate).
+static int select_topk_impl(moba_tensor q, const void *kbar_split, int batch, int hq, int hkv,
+                            int N, int Nk, int d, int block, int topk, int32_t *idx,
+                            void *workspace, size_t workspace_bytes, void *stream, int minmax) {
   const int q_off = Nk - N;
   int rc = check_moba_shape(batch, hq, hkv, N, d, block, topk, q_off);
   if (rc) return rc;
@@ -263,7 +270,7 @@ int moba_select_topk_chunk(moba_tensor q, const void *kbar_split, int batch, int
   int *tileoff = reinterpret_cast<int *>(ws + w.off_tileoff);
   int4 *tiles = reinterpret_cast<int4 *>(ws + w.off_tiles);
   bool scanned = false;  // list offsets already written by the gate kernel
-  if (gate_tc_supports(w.nblk, topk)) {
+  if (!minmax && gate_tc_supports(w.nblk, topk)) {
     // Tensor-core gate: q tiles and the pooled keys through TMA.
     int nsm = 0;
     if ((rc = check_device(&nsm))) return rc;
@@ -302,6 +309,7 @@ int moba_select_topk_chunk(moba_tensor q, const void *kbar_split, int batch, int
     sp.batch = batch; sp.hq = hq; sp.hkv = hkv; sp.N = N; sp.d = d; sp.block = block;
     sp.topk = topk; sp.nblk = w.nblk; sp.G = w.G; sp.chunk_rows = w.chunk_rows;
     sp.q_off = q_off;
+    sp.minmax = minmax;
     if ((rc = launch_status(launch_gate(sp, st)))) return rc;
   }
   if (w.npast == 0) return MOBA_OK;
@@ -320,6 +328,37 @@ int moba_select_topk_chunk(moba_tensor q, const void *kbar_split, int batch, int
   cp.nblk = w.nblk; cp.G = w.G; cp.chunk_rows = w.chunk_rows;
   cp.q_off = q_off;
   return launch_status(launch_scatter(cp, st));
+}
+
+extern "C" {
+
+int moba_select_topk_chunk(moba_tensor q, const void *kbar_split, int batch, int hq, int hkv,
+                           int N, int Nk, int d, int block, int topk, int32_t *idx,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+  return select_topk_impl(q, kbar_split, batch, hq, hkv, N, Nk, d, block, topk, idx, workspace,
+                          workspace_bytes, stream, 0);
+}
+
+int moba_pool_keys_minmax(moba_tensor k, int batch, int hkv, int N, int d, int block,
+                          void *kminmax, void *stream) {
+  if (batch < 1 || hkv < 1 || N < 1 || block < 1) return MOBA_ERR_SHAPE;
+  if (d < 8 || d > 256 || d % 8) return MOBA_ERR_DIM;
+  int rc = check_tensor(k);
+  if (rc) return rc;
+  if (!kminmax) return MOBA_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(kminmax) & 1u) return MOBA_ERR_ALIGN;
+  if ((rc = check_device(nullptr))) return rc;
+  return launch_status(launch_pool_minmax(static_cast<const uint16_t *>(k.ptr), k.sb, k.sh, k.sn,
+                                          batch, hkv, N, d, block,
+                                          static_cast<uint16_t *>(kminmax),
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int moba_select_topk_minmax(moba_tensor q, const void *kminmax, int batch, int hq, int hkv, int N,
+                            int Nk, int d, int block, int topk, int32_t *idx, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+  return select_topk_impl(q, kminmax, batch, hq, hkv, N, Nk, d, block, topk, idx, workspace,
+                          workspace_bytes, stream, 1);
 }
 
 int moba_select_static(int batch, int hq, int hkv, int N, int Nk, int d, int block, int topk,

@@ -85,6 +85,8 @@ struct SelectParams {
   int *counts;           // workspace list counts
   int batch, hq, hkv, N, d, block, topk, nblk, G, chunk_rows;
   int q_off;             // position of query row 0 among the keys
+  int minmax;            // 1: the planes are block maxima and minima (min/max pooling), and
+                         // the score is q+ . kmax + q- . kmin; 0: hi + lo of the means
 };
 
 // Parameters of the tensor-core gate / top-k kernel (q and the pooled keys arrive

@@ -81,6 +81,58 @@ pool_keys_kernel(const uint16_t *__restrict__ k, int64_t sb, int64_t sh, int64_t
   }
 }
 
+// Min/max pooling (the MoBA page: Quest is MoBA with smaller blocks and a min/max
+// pooled block representation): kmax_j and kmin_j, the element-wise maximum and minimum
+// of the keys of block j, written as bf16 planes [batch, hkv, 2, nblk, d] (plane 0 the
+// maxima, plane 1 the minima; exact, the keys are bf16).  Same CTA layout as the mean.
+__global__ void __launch_bounds__(kPoolThreads)
+pool_minmax_kernel(const uint16_t *__restrict__ k, int64_t sb, int64_t sh, int64_t sn, int hkv,
+                   int d, int block, int N, int nblk, uint16_t *__restrict__ planes) {
+  extern __shared__ float red[];  // [2][ngroups][d]
+  const int j = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int vpr = d >> 3;
+  const int ngroups = kPoolThreads / vpr;
+  const int t = threadIdx.x;
+  const int vec = t % vpr, grp = t / vpr;
+  const int len = min(block, N - j * block);
+  float mx[8], mn[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) { mx[e] = -INFINITY; mn[e] = INFINITY; }
+  if (grp < ngroups) {
+    const uint16_t *base = k + b * sb + hk * sh + (int64_t)j * block * sn + vec * 8;
+    for (int r = grp; r < len; r += ngroups) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(base + (int64_t)r * sn));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
+        mx[2 * e] = fmaxf(mx[2 * e], lo);
+        mn[2 * e] = fminf(mn[2 * e], lo);
+        mx[2 * e + 1] = fmaxf(mx[2 * e + 1], hi);
+        mn[2 * e + 1] = fminf(mn[2 * e + 1], hi);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      red[grp * d + vec * 8 + e] = mx[e];
+      red[(ngroups + grp) * d + vec * 8 + e] = mn[e];
+    }
+  }
+  __syncthreads();
+  const int64_t bh = (int64_t)b * hkv + hk;
+  uint16_t *pl = planes + bh * 2 * (int64_t)nblk * d;
+  for (int c = t; c < d; c += kPoolThreads) {
+    float a = -INFINITY, z = INFINITY;
+    for (int g = 0; g < ngroups; ++g) {
+      a = fmaxf(a, red[g * d + c]);
+      z = fminf(z, red[(ngroups + g) * d + c]);
+    }
+    // Exact: a and z are bf16 values.
+    pl[(int64_t)j * d + c] = (uint16_t)(__float_as_uint(a) >> 16);
+    pl[((int64_t)nblk + j) * d + c] = (uint16_t)(__float_as_uint(z) >> 16);
+  }
+}
+
 // ------------------------------------------------------------ gate + top-k
 //
 // [MoBA] §"블록 분할과 top-k 게이팅": s_j = <q, MeanPool(K[I_j])>, unscaled;
@@ -192,8 +244,24 @@ gate_topk_kernel(const SelectParams p) {
           const int c = s * 16 + 8 * ((lane >> 3) & 1);
           uint32_t h0, h1, l0, l1;
           ldmatrix_x4(smem_u32(ks + (part * kGateChunk + jj) * LDK + c), h0, h1, l0, l1);
-          mma_bf16_16816(acc_hi[nt], afrag[s], h0, h1);
-          mma_bf16_16816(acc_lo[nt], afrag[s], l0, l1);
+          if (p.minmax) {
+            // max(q_d kmax_d, q_d kmin_d) = q+_d kmax_d + q-_d kmin_d: the positive part
+            // of q against the maxima, the negative part against the minima (exact).
+            uint32_t ap[4], an[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&afrag[s][e]);
+              const __nv_bfloat162 z = __float2bfloat162_rn(0.f);
+              const __nv_bfloat162 xp = __hmax2(x, z), xn = __hmin2(x, z);
+              ap[e] = *reinterpret_cast<const uint32_t *>(&xp);
+              an[e] = *reinterpret_cast<const uint32_t *>(&xn);
+            }
+            mma_bf16_16816(acc_hi[nt], ap, h0, h1);
+            mma_bf16_16816(acc_lo[nt], an, l0, l1);
+          } else {
+            mma_bf16_16816(acc_hi[nt], afrag[s], h0, h1);
+            mma_bf16_16816(acc_lo[nt], afrag[s], l0, l1);
+          }
         }
       }
     }
@@ -445,6 +513,21 @@ cudaError_t launch_pool(const uint16_t *k, int64_t sb, int64_t sh, int64_t sn, i
   dim3 grid(nblk, hkv, batch);
   pool_keys_kernel<<<grid, kPoolThreads, smem, st>>>(k, sb, sh, sn, hkv, d, block, N, nblk, kbar,
                                                       split);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pool_minmax(const uint16_t *k, int64_t sb, int64_t sh, int64_t sn, int batch,
+                               int hkv, int N, int d, int block, uint16_t *planes, cudaStream_t st) {
+  const int nblk = (N + block - 1) / block;
+  const int ngroups = kPoolThreads / (d / 8);
+  const size_t smem = sizeof(float) * 2 * ngroups * d;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(pool_minmax_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(nblk, hkv, batch);
+  pool_minmax_kernel<<<grid, kPoolThreads, smem, st>>>(k, sb, sh, sn, hkv, d, block, N, nblk, planes);
   return cudaGetLastError();
 }
 

@@ -158,6 +158,23 @@ int swa_attn_fwd_chunk(moba_tensor q, moba_tensor k, moba_tensor v, int batch, i
                        void *stream);
 
 /*
+ * Min/max pooling (the MoBA page: Quest is MoBA with smaller blocks and a min/max
+ * pooled block representation).  moba_pool_keys_minmax writes, per block, the
+ * element-wise maximum and minimum of its keys as bf16 planes [batch, hkv, 2, n, d]
+ * (plane 0 maxima, plane 1 minima; n = ceil(N / block); exact).  N is the key count.
+ * moba_select_topk_minmax then scores the past blocks of each query row with
+ * s_j = sum_d max(q_d kmax_jd, q_d kmin_jd) -- the largest inner product q can have
+ * with a key inside block j's min/max box, computed as q+ . kmax_j + q- . kmin_j -- and
+ * keeps the own block and the topk-1 best past blocks like moba_select_topk_chunk
+ * (same idx, lists and workspace; N query rows, the last N of Nk positions).
+ */
+int moba_pool_keys_minmax(moba_tensor k, int batch, int hkv, int N, int d, int block,
+                          void *kminmax, void *stream);
+int moba_select_topk_minmax(moba_tensor q, const void *kminmax, int batch, int hq, int hkv, int N,
+                            int Nk, int d, int block, int topk, int32_t *idx, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/*
  * Static gates ([MoBA] §"MoBA의 구현" preamble: sliding-window attention is MoBA whose
  * gate always picks the most recent blocks; an attention sink is MoBA whose gate picks
  * the first block together with the most recent ones): in place of moba_select_topk,

@@ -121,3 +121,12 @@ def test_static_gate_rejects_a_sink_beyond_the_list():
                                   None) == -4
     assert lib.moba_select_static(1, 2, 1, 1024, 1024, 128, 128, 3, -1, 1 << 20, 1 << 20, 1 << 30,
                                   None) == -4
+
+
+def test_minmax_entries_check_arguments():
+    lib = moba.library()
+    ok = moba.MobaTensor(1 << 20, 8 * 1024, 8 * 1024, 128)
+    assert lib.moba_pool_keys_minmax(ok, 1, 1, 1024, 128, 0, 1 << 20, None) == -1
+    assert lib.moba_pool_keys_minmax(ok, 1, 1, 1024, 128, 128, None, None) == -4
+    assert lib.moba_select_topk_minmax(ok, 1 << 20, 1, 2, 1, 1024, 1088, 128, 128, 3, 1 << 20,
+                                       1 << 20, 1 << 30, None) == -1  # offset not a multiple of 128
