@@ -336,10 +336,21 @@ def run_ours(args, rank, world, device):
                              device=device, kv_len=w.seqlen)
 
         def stages():
-            moba.moba_pool_keys(kd, w.block, runner.kbar, runner.kbar_split)
-            yield "pool"
-            moba.moba_select_topk_chunk(qd, runner.kbar_split, w.block, w.topk, w.seqlen,
-                                        runner.workspace, runner.idx)
+            if w.gate == "minmax":
+                moba.moba_pool_keys_minmax(kd, w.block, out=runner.kbar_split)
+                yield "pool"
+                moba.moba_select_topk_minmax(qd, runner.kbar_split, w.block, w.topk, w.seqlen,
+                                             runner.workspace, runner.idx)
+            elif w.gate == "static":
+                yield "pool"  # no pooled keys
+                moba.moba_select_static(w.batch, w.hq, w.hkv, w.nq, w.d, w.block, w.topk, w.sink,
+                                        runner.workspace, kv_len=w.seqlen, idx=runner.idx,
+                                        device=device)
+            else:
+                moba.moba_pool_keys(kd, w.block, runner.kbar, runner.kbar_split)
+                yield "pool"
+                moba.moba_select_topk_chunk(qd, runner.kbar_split, w.block, w.topk, w.seqlen,
+                                            runner.workspace, runner.idx)
             yield "select"
             moba.moba_attn_fwd_chunk(qd, kd, vd, runner.idx, w.block, w.topk, runner.workspace,
                                      w.window, out=runner.out, lse=runner.lse)
@@ -359,9 +370,12 @@ def run_ours(args, rank, world, device):
         # tensor-core gate's last CTA writes the list offsets itself), and per query
         # chunk: past-block pass, own-block pass, merge (only the own-block pass when
         # topk = 1).
-        tc_gate = -(-w.seqlen // w.block) <= 256 and w.topk - 1 < 32
-        launches_per_step = (2 + ((1 if tc_gate else 2) if w.topk > 1 else 0)
-                             + layout_chunks * (3 if w.topk > 1 else 1))
+        tc_gate = -(-w.seqlen // w.block) <= 256 and w.topk - 1 < 32 and w.gate == "mean"
+        if w.gate == "static":
+            sel_launches = 1 + (2 if w.topk > 1 else 0)       # static gate, scan, scatter
+        else:
+            sel_launches = 2 + ((1 if tc_gate else 2) if w.topk > 1 else 0)
+        launches_per_step = sel_launches + layout_chunks * (3 if w.topk > 1 else 1)
     else:
         out_t = torch.empty_like(qd)
         lse_t = torch.empty(w.batch, w.hq, w.seqlen, dtype=torch.float32, device=device)
@@ -474,8 +488,9 @@ def run_ours(args, rank, world, device):
     if w.kind == "moba":
         sel_ms = stage_ms["pool"] + stage_ms["select"]
         n_entries = int(((runner.idx >= 0).sum().item()) - w.batch * w.hq * w.nq)
-        sel_bytes = (w.batch * w.hkv * w.seqlen * w.d * 2 + w.batch * w.hq * w.nq * w.d * 2
-                     + 2 * w.batch * w.hq * w.nq * w.topk * 4 + 2 * n_entries * 4)
+        sel_bytes = 2 * w.batch * w.hq * w.nq * w.topk * 4 + 2 * n_entries * 4
+        if w.gate != "static":  # the keys and the queries are read once
+            sel_bytes += w.batch * w.hkv * w.seqlen * w.d * 2 + w.batch * w.hq * w.nq * w.d * 2
         extra["selection"] = {"ms": round(sel_ms, 4), "bytes": sel_bytes,
                               "gbs": round(sel_bytes / (sel_ms * 1e-3) / 1e9, 1),
                               "frac_hbm": round(sel_bytes / (sel_ms * 1e-3) / 1e9 / hbm, 4)}
@@ -559,7 +574,8 @@ def run_ours(args, rank, world, device):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) q,k,v; per-block key offsets; no dataset)",
             "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv,
-                       "seq_len": w.seqlen, "q_len": w.nq, "d": w.d, "block": w.block, "topk": w.topk,
+                       "seq_len": w.seqlen, "q_len": w.nq, "gate": w.gate, "d": w.d,
+                       "block": w.block, "topk": w.topk,
                        "window": w.window, "parallelism": f"replicas x{world}" if world > 1 else "1 gpu",
                        "l2": "flushed between timed steps (256 MB write)"},
             "tokens_per_s": round(tokens, 1), "attended_flops_per_step": flops,
@@ -587,10 +603,19 @@ def cpu_baseline(w: workloads.Workload, seed: int, target_s: float):
         rows = (w.q_off + np.sort(rng.choice(N, size=nrows, replace=False))).astype(np.int32)
         t0 = time.perf_counter()
         if w.kind == "moba":
-            kbar = oracle.pool_keys(k, w.block)
-            t1 = time.perf_counter()
-            s = oracle.gate_scores(q, kbar, w.block, rows)
-            idx, _ = oracle.select_topk(s, w.seqlen, w.block, w.topk, rows)
+            if w.gate == "static":
+                t1 = time.perf_counter()
+                idx = oracle.select_static(w.seqlen, w.block, w.topk, w.sink, rows, w.batch, w.hq)
+            elif w.gate == "minmax":
+                kmax, kmin = oracle.pool_minmax(k, w.block)
+                t1 = time.perf_counter()
+                s = oracle.minmax_scores(q, kmax, kmin, w.block, rows)
+                idx, _ = oracle.select_topk(s, w.seqlen, w.block, w.topk, rows)
+            else:
+                kbar = oracle.pool_keys(k, w.block)
+                t1 = time.perf_counter()
+                s = oracle.gate_scores(q, kbar, w.block, rows)
+                idx, _ = oracle.select_topk(s, w.seqlen, w.block, w.topk, rows)
             oracle.attention(q, k, v, mode=oracle.MODE_MOBA, block=w.block, topk=w.topk, idx=idx,
                              window=w.window, rows=rows)
             t2 = time.perf_counter()
@@ -638,7 +663,8 @@ def run_reference(args, rank, world):
             "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv,
-                       "seq_len": w.seqlen, "q_len": w.nq, "d": w.d, "block": w.block, "topk": w.topk,
+                       "seq_len": w.seqlen, "q_len": w.nq, "gate": w.gate, "d": w.d,
+                       "block": w.block, "topk": w.topk,
                        "window": w.window},
             "cpu_baseline": {**last, "value": value},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

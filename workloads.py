@@ -32,6 +32,10 @@ class Workload:
     key_offset_std: float = 0.0
     sampled_rows: bool = False   # the oracle checks sampled rows only
     q_len: int = 0               # chunked prefill: the queries are the last q_len positions
+    gate: str = "mean"           # block selection: "mean" (MoBA), "minmax" (min/max pooled
+                                 # blocks) or "static" (own block, `sink` first blocks and the
+                                 # most recent ones, no scores)
+    sink: int = 0
     note: str = ""
 
     @property
@@ -70,6 +74,13 @@ WORKLOADS = {
                                key_offset_std=0.5, q_len=8192,
                                note="chunked prefill: the last 8192 queries of the gqa32k "
                                     "context against all 32768 keys"),
+    "gqa32k_minmax": Workload("gqa32k_minmax", 1, 32, 8, 32768, 128, block=512, topk=3,
+                              key_offset_std=0.5, gate="minmax",
+                              note="gqa32k with min/max pooled blocks"),
+    "gqa32k_sink": Workload("gqa32k_sink", 1, 32, 8, 32768, 128, block=512, topk=3,
+                            key_offset_std=0.5, gate="static", sink=1,
+                            note="gqa32k with a static gate: the first block, the most recent "
+                                 "block and the own block"),
 }
 
 
