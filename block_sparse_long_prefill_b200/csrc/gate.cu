@@ -6,27 +6,32 @@
 // §"블록 분할과 top-k 게이팅": the gate score of query i for block j is the unscaled
 // inner product s_j = <q_i, MeanPool(K[I_j])>; each query keeps the k blocks with the
 // highest scores.  §"인과성 보존": only blocks wholly before the query's own block
-// c = i / block compete (j < c), block c is always kept, later blocks never.
+// c = (q_off + i) / block compete (j < c), block c is always kept, later blocks never.
 //
-// It takes problems of at most 256 blocks with k - 1 <= kGateMaxPicks, and problems of
-// at most 33 blocks with any k (rank selection); the general gate of select.cu takes
-// the others.
+// It takes problems of at most 256 blocks with k - 1 <= 31; the general gate of
+// select.cu takes the others (and the min/max pooled variant).
 // One persistent CTA per SM takes chunks of consecutive 128-row query tiles, ordered
 // (batch, kv-head, row tile, q-head), from a global counter (the cost of a tile grows
 // with its row position, so a static split would leave SMs idle); the pooled keys of a
-// kv-head stay staged in shared memory while the CTA's tiles stay in that kv-head.  Since block % 128 == 0, every row of a tile has the
-// same own block c, and the tile needs the scores of blocks [0, c) only.
+// kv-head stay staged in shared memory while the CTA's tiles stay in that kv-head.
+// Since block % 128 == 0 and q_off % 128 == 0, every row of a tile has the same own
+// block c, and the tile needs the scores of blocks [0, c) only.
 //   warp 0     TMA producer: query tiles (a ring of up to eight) and, per kv-head, the
-//              pooled keys kbar = hi + lo (two bf16 matrices of up to 256 rows)
+//              pooled keys kbar = hi + lo (two bf16 matrices of up to 256 rows; two
+//              slots when they fit, so the next kv-head's keys load early); it also
+//              takes the tile chunks from the counter and hands them on
 //   warp 1     tcgen05 MMA issuer and TMEM owner: S = Q hi^T + Q lo^T in fp32, into
 //              one of 2-4 TMEM accumulators (N = c rounded up to 16 columns)
 //   warps 2-9  top-k, two groups of four warps taking the tiles (and accumulators) in
-//              turn: thread r owns row r (TMEM lane r) and scans its c scores in
-//              ascending block order, keeping the best k-1 (at most kGateMaxPicks) in
-//              a register list without branches (a strictly greater score displaces;
-//              ties keep the lower block), then writes the
-//              row's choices in ascending order, the own block, and -1 padding; it
-//              also counts the picks per past block for the dispatch lists.
+//              turn: thread r owns row r (TMEM lane r) and ranks its c scores --
+//              k - 1 <= 4: a float register list without branches (a strictly greater
+//              score displaces; ties keep the lower block); longer lists: 32-bit packed
+//              keys merged by sorting networks (lists of 8, 16) or inserted (24, 32),
+//              with an exact 64-bit rescan of rows whose boundary keys tie in their
+//              score bits -- then stages the row's choices in ascending order, the own
+//              block and -1 padding (stored coalesced per warp), and counts the picks
+//              per past block for the dispatch lists.
+// The last CTA to finish turns the list counts into list offsets.
 // q is exactly bf16 and kbar = hi + lo to about 2^-17 relative, so the fp32 scores
 // match an fp32 inner product with the pooled keys far inside the ranking tolerance.
 #include <cuda.h>
