@@ -352,3 +352,73 @@ def moba_prefill(q, k, v, block: int, topk: int, window: int = 0, stream=None):
     runner = MobaPrefill(b, hq, k.shape[1], N, d, block, topk, window, device=q.device)
     out, lse = runner(q, k, v, stream)
     return out, lse, runner.idx
+
+
+class MobaPrefillHost:
+    """The whole MoBA prefill from pinned host buffers to pinned host buffers, pipelined
+    over KV-head groups.  The path needs no exchange between KV heads (a q-head reads its
+    own KV head only), so the heads split into ``groups`` independent sub-problems: the
+    upload of group g+1, the kernels of group g and the download of group g-1 run on
+    three streams at once, through two sets of device buffers.  The results are those of
+    MobaPrefill on the whole problem.
+
+    q_h: [batch, hq, N, d], k_h, v_h: [batch, hkv, N, d] bf16, pinned; out_h like q_h and
+    lse_h [batch, hq, N] float32, pinned.  Per batch item and group the head range is
+    contiguous in host memory."""
+
+    def __init__(self, batch, hq, hkv, N, d, block, topk, window=0, device="cuda", groups=None):
+        G = hq // hkv
+        if groups is None:
+            groups = max(g for g in (1, 2, 4, 8) if hkv % g == 0)
+        if hkv % groups:
+            raise ValueError("groups must divide hkv")
+        self.batch, self.hq, self.hkv, self.N, self.d = batch, hq, hkv, N, d
+        self.groups, self.G = groups, G
+        self.hkv_g, self.hq_g = hkv // groups, hq // groups
+        self.device = torch.device(device)
+        self.runners = [MobaPrefill(1, self.hq_g, self.hkv_g, N, d, block, topk, window, device=device)
+                        for _ in range(2)]
+        self.qd = [torch.empty(1, self.hq_g, N, d, dtype=torch.bfloat16, device=device) for _ in range(2)]
+        self.kd = [torch.empty(1, self.hkv_g, N, d, dtype=torch.bfloat16, device=device) for _ in range(2)]
+        self.vd = [torch.empty(1, self.hkv_g, N, d, dtype=torch.bfloat16, device=device) for _ in range(2)]
+        self.s_h2d = torch.cuda.Stream(device)
+        self.s_run = torch.cuda.Stream(device)
+        self.s_d2h = torch.cuda.Stream(device)
+
+    def __call__(self, q_h, k_h, v_h, out_h, lse_h):
+        cur = torch.cuda.current_stream(self.device)
+        for s in (self.s_h2d, self.s_run, self.s_d2h):
+            s.wait_stream(cur)
+        inputs_free = [None, None]   # the kernels of the slot's last use have read its inputs
+        outputs_free = [None, None]  # the download of the slot's last output is done
+        units = [(b, g) for b in range(self.batch) for g in range(self.groups)]
+        for u, (b, g) in enumerate(units):
+            slot = u % 2
+            hq0, hk0 = g * self.hq_g, g * self.hkv_g
+            with torch.cuda.stream(self.s_h2d):
+                if inputs_free[slot] is not None:
+                    self.s_h2d.wait_event(inputs_free[slot])
+                self.qd[slot].copy_(q_h[b:b + 1, hq0:hq0 + self.hq_g], non_blocking=True)
+                self.kd[slot].copy_(k_h[b:b + 1, hk0:hk0 + self.hkv_g], non_blocking=True)
+                self.vd[slot].copy_(v_h[b:b + 1, hk0:hk0 + self.hkv_g], non_blocking=True)
+                loaded = torch.cuda.Event()
+                loaded.record(self.s_h2d)
+            with torch.cuda.stream(self.s_run):
+                self.s_run.wait_event(loaded)
+                if outputs_free[slot] is not None:
+                    self.s_run.wait_event(outputs_free[slot])
+                self.runners[slot](self.qd[slot], self.kd[slot], self.vd[slot], self.s_run)
+                done = torch.cuda.Event()
+                done.record(self.s_run)
+                inputs_free[slot] = done
+            with torch.cuda.stream(self.s_d2h):
+                self.s_d2h.wait_event(done)
+                r = self.runners[slot]
+                out_h[b:b + 1, hq0:hq0 + self.hq_g].copy_(r.out, non_blocking=True)
+                lse_h[b:b + 1, hq0:hq0 + self.hq_g].copy_(r.lse, non_blocking=True)
+                fetched = torch.cuda.Event()
+                fetched.record(self.s_d2h)
+                outputs_free[slot] = fetched
+        for s in (self.s_h2d, self.s_run, self.s_d2h):
+            cur.wait_stream(s)
+        return out_h, lse_h

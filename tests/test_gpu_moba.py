@@ -201,3 +201,26 @@ def test_moba_tied_blocks_keep_the_lower_block(name, kw):
     assert checked > 0.9 * w.batch * w.hq * (w.seqlen - (npast + 1) * w.block)
     assert split > 100  # the boundary splits a tied pair on many rows
     print(name, "checked", checked, "split pairs", split)
+
+
+@pytest.mark.parametrize("batch,hq,hkv,groups", [(1, 8, 4, 4), (2, 4, 2, 2), (1, 2, 1, 1)])
+def test_host_pipeline_equals_device_path(batch, hq, hkv, groups):
+    """MobaPrefillHost (pinned host buffers, KV-head groups pipelined over three streams)
+    gives exactly the device path's results."""
+    moba = _moba()
+    w = workloads.small_moba(batch=batch, hq=hq, hkv=hkv, seqlen=2048, d=128, block=256, topk=3,
+                             window=100)
+    q, k, v = workloads.make_inputs(w, 9)
+    ref = moba.MobaPrefill(w.batch, w.hq, w.hkv, w.seqlen, w.d, w.block, w.topk, w.window)
+    o_ref, l_ref = (t.cpu() for t in ref(q.cuda(), k.cuda(), v.cuda()))
+    host = moba.MobaPrefillHost(w.batch, w.hq, w.hkv, w.seqlen, w.d, w.block, w.topk, w.window,
+                                groups=groups)
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    out_h = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    lse_h = torch.empty(w.batch, w.hq, w.seqlen, dtype=torch.float32).pin_memory()
+    for _ in range(2):
+        out_h.zero_()
+        host(qh, kh, vh, out_h, lse_h)
+        torch.cuda.synchronize()
+        assert moba.device_status() == 0
+        assert torch.equal(out_h, o_ref) and torch.equal(lse_h, l_ref)
