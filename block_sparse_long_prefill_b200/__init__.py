@@ -422,3 +422,55 @@ class MobaPrefillHost:
         for s in (self.s_h2d, self.s_run, self.s_d2h):
             cur.wait_stream(s)
         return out_h, lse_h
+
+
+def moba_prefill_varlen(q, k, v, cu_seqlens, block: int, topk: int, window: int = 0,
+                        stream=None):
+    """MoBA prefill of a batch of sequences of different lengths, packed along the token
+    axis (FlashAttention's varlen layout): q [total, hq, d], k, v [total, hkv, d] bf16,
+    ``cu_seqlens`` the prefix offsets (batch + 1 ints from 0 to total; a list or a CPU
+    tensor).  Sequence s is positions cu_seqlens[s] .. cu_seqlens[s+1] - 1 and is its own
+    prefill: its own blocks, its own causal order.  A length must be a multiple of 128
+    (not necessarily of ``block``: its last block may be partial).  Each sequence goes
+    through the library's calls as a [1, heads, N_s, d] strided view of the packed
+    tensors (no copy); the pooled keys, block choices and workspace are sized for the
+    longest sequence and reused in stream order.  Returns (out [total, hq, d] bf16, lse
+    [hq, total] float32)."""
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    offs = [int(x) for x in (cu_seqlens.tolist() if torch.is_tensor(cu_seqlens) else cu_seqlens)]
+    if len(offs) < 2 or offs[0] != 0 or offs[-1] != T or any(b < a for a, b in zip(offs, offs[1:])):
+        raise ValueError("cu_seqlens must rise from 0 to the token count")
+    lens = [b - a for a, b in zip(offs, offs[1:])]
+    nmax = max(lens)
+    out = torch.empty_like(q)
+    lse = torch.empty(hq, T, dtype=torch.float32, device=q.device)
+    if nmax == 0:
+        return out, lse
+    nb = -(-nmax // block)
+    dev = q.device
+    ws = torch.empty(workspace_size(1, hq, hkv, nmax, d, block, topk), dtype=torch.uint8, device=dev)
+    kbar_f = torch.empty(hkv * nb * d, dtype=torch.float32, device=dev)
+    ks_f = torch.empty(hkv * 2 * nb * d, dtype=torch.bfloat16, device=dev)
+    idx_f = torch.empty(hq * nmax * topk, dtype=torch.int32, device=dev)
+    lse_f = torch.empty(hq * nmax, dtype=torch.float32, device=dev)
+
+    def view(t, a, n):  # packed [total, heads, d] -> [1, heads, n, d] over positions a .. a+n-1
+        return t[a:a + n].permute(1, 0, 2).unsqueeze(0)
+
+    cur = torch.cuda.current_stream(dev) if stream is None else stream
+    for a, n in zip(offs, lens):
+        if n == 0:
+            continue
+        nbs = -(-n // block)
+        kbar = kbar_f[:hkv * nbs * d].view(1, hkv, nbs, d)
+        ks = ks_f[:hkv * 2 * nbs * d].view(1, hkv, 2, nbs, d)
+        idx = idx_f[:hq * n * topk].view(1, hq, n, topk)
+        lse_s = lse_f[:hq * n].view(1, hq, n)
+        qs, kk, vv, os_ = view(q, a, n), view(k, a, n), view(v, a, n), view(out, a, n)
+        moba_pool_keys(kk, block, kbar, ks, stream)
+        moba_select_topk(qs, ks, block, topk, ws, idx, stream)
+        moba_attn_fwd(qs, kk, vv, idx, block, topk, ws, window, out=os_, lse=lse_s, stream=stream)
+        with torch.cuda.stream(cur):
+            lse[:, a:a + n].copy_(lse_s[0], non_blocking=True)
+    return out, lse
