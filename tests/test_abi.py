@@ -130,3 +130,11 @@ def test_minmax_entries_check_arguments():
     assert lib.moba_pool_keys_minmax(ok, 1, 1, 1024, 128, 128, None, None) == -4
     assert lib.moba_select_topk_minmax(ok, 1 << 20, 1, 2, 1, 1024, 1088, 128, 128, 3, 1 << 20,
                                        1 << 20, 1 << 30, None) == -1  # offset not a multiple of 128
+
+
+@pytest.mark.parametrize("cu", [[1, 256], [0, 128, 64], [0, 100], []])
+def test_varlen_rejects_bad_offsets_before_any_launch(cu):
+    q = torch.empty(256, 2, 64, dtype=torch.bfloat16)
+    k = torch.empty(256, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        moba.moba_prefill_varlen(q, k, k, cu, 128, 2)
