@@ -138,3 +138,8 @@ def test_varlen_rejects_bad_offsets_before_any_launch(cu):
     k = torch.empty(256, 1, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         moba.moba_prefill_varlen(q, k, k, cu, 128, 2)
+
+
+def test_host_pipeline_needs_groups_that_divide_the_kv_heads():
+    with pytest.raises(ValueError):
+        moba.MobaPrefillHost(1, 8, 4, 1024, 128, 512, 3, groups=3)
