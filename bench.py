@@ -4,11 +4,13 @@ One step is the whole hot path over one batch of the workload: key pooling, gate
 scores + top-k + dispatch lists, and block-sparse attention with the merge
 (moba_pool_keys -> moba_select_topk -> moba_attn_fwd), inputs resident in HBM.
 `value` is attended TFLOP/s (4 d |J_i| summed over rows, heads and batch, divided by
-the device time of the step); tokens/s, per-stage times, the dense-causal comparators
-(torch SDPA and this library's own kernel with a window >= N) and the roofline of the
-attention stage ride along.  `e2e` measures the same through the C ABI with host
-buffers (host->device copies of q, k, v and device->host copies of out, lse inside the
-timed region).  `--impl reference` times the fp64 CPU oracle instead.
+the device time of the step); tokens/s, per-stage and per-pass times, the dense-causal
+comparators (torch SDPA and this library's own kernel with a window >= N) and the
+roofline of the dominant kernel ride along.  `e2e` measures the same through the
+binding's host-buffer entry (host->device copies of q, k, v and device->host copies of
+out, lse inside the timed region).  The default workload is the 1M-token prefill; the
+32K, hybrid 64K and sliding-window 16K workloads are measured after it in the same run
+and reported under "workloads".  `--impl reference` times the fp64 CPU oracle instead.
 
 Multi-GPU (torchrun): every rank runs its own copy of the workload (the method
 shards over batch / kv-head groups with no exchange): weak scaling, no collective on
@@ -45,10 +47,14 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="gqa32k", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="moba1m", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--extra-workloads", default="gqa32k,hybrid64k,swa16k",
+                    help="comma-separated workloads measured after the main one (rank 0 "
+                         "reports them under 'workloads'); empty for none")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-comparators", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
     return ap.parse_args()
 
 
@@ -140,26 +146,20 @@ def attended_pairs_swa(w: workloads.Workload) -> int:
     return int(np.minimum(i + 1, w.window).sum()) * w.batch * w.hq
 
 
-def pass_work_moba(idx: torch.Tensor, w: workloads.Workload, chunk_rows: int) -> dict:
-    """Algorithmic work of each moba_attn_fwd pass over rows [0, chunk_rows): attended
-    FLOPs (4*d per (query, key) pair) of the past-block pass (whole selected past
-    blocks) and of the own-block pass (causal own block plus window tail keys), and
-    the bytes the merge pass must move (topk partial rows and log-sum-exps read, block
-    choices read, the output row and its log-sum-exp written)."""
+def pass_work_moba(idx: torch.Tensor, w: workloads.Workload) -> dict:
+    """Algorithmic work of each moba_attn_fwd pass, summed over all query chunks:
+    attended FLOPs (4*d per (query, key) pair) of the past-block pass (whole selected
+    past blocks) and of the own-block pass (causal own block plus window tail keys),
+    and the bytes the merge pass must move (topk partial rows and log-sum-exps read,
+    block choices read, the output row and its log-sum-exp written)."""
     B, N = w.block, w.nq
-    rows = min(chunk_rows, N)
-    sub = idx[:, :, :rows]
-    i = w.q_off + torch.arange(rows, device=idx.device)   # key positions of the rows
+    i = w.q_off + torch.arange(N, device=idx.device)   # key positions of the rows
     c = i // B
-    past = int(((sub >= 0) & (sub < c[None, None, :, None])).sum().item()) * B
+    past = int(((idx >= 0) & (idx < c[None, None, :, None])).sum().item()) * B
     own = int(((i % B) + 1).sum().item()) * w.batch * w.hq
     if w.window > 0:
-        total_rows = attended_pairs_moba(idx, w)  # all rows; window extras scaled below
-        pos = w.q_off + torch.arange(N, device=idx.device)
-        base = int(((pos % B) + 1).sum().item()) * w.batch * w.hq
-        base += int(((idx >= 0) & (idx < (pos // B)[None, None, :, None])).sum().item()) * B
-        own += int(round((total_rows - base) * rows / N))
-    rowcount = w.batch * w.hq * rows
+        own += attended_pairs_moba(idx, w) - own - past  # window keys outside the choices
+    rowcount = w.batch * w.hq * N
     merge_bytes = rowcount * (w.topk * (w.d * 2 + 4) + w.topk * 4 + w.d * 2 + 4)
     return {"past_block_pass": 4.0 * w.d * past, "own_block_pass": 4.0 * w.d * own,
             "merge_pass": merge_bytes}
@@ -316,21 +316,49 @@ class ClockSampler:
 
 # ------------------------------------------------------------------- our arm
 
-def run_ours(args, rank, world, device):
+def layout_chunks(w: workloads.Workload) -> int:
+    """Query chunks moba_attn_fwd runs (the partials of one chunk stay below 4 GiB)."""
+    per_row = (w.topk if w.topk > 1 else 0) * (w.d * 2 + 4) * w.batch * w.hq
+    if per_row == 0 or per_row * w.nq <= (4 << 30):
+        return 1
+    chunk_rows = max(128, ((4 << 30) // per_row) // 128 * 128)
+    return math.ceil(w.nq / chunk_rows)
+
+
+def launches_per_step(w: workloads.Workload) -> int:
+    """Library kernels one step launches: pool, gate, scatter (+ a scan launch when the
+    general gate runs: the tensor-core gate's last CTA writes the list offsets itself),
+    and per query chunk: past-block pass, own-block pass, merge (only the own-block
+    pass when topk = 1)."""
+    if w.kind != "moba":
+        return 1
+    tc_gate = -(-w.seqlen // w.block) <= 256 and w.topk - 1 < 32 and w.gate == "mean"
+    if w.gate == "static":
+        sel = 1 + (2 if w.topk > 1 else 0)       # static gate, scan, scatter
+    else:
+        sel = 2 + ((1 if tc_gate else 2) if w.topk > 1 else 0)
+    return sel + layout_chunks(w) * (3 if w.topk > 1 else 1)
+
+
+def measure(w, steps, warmup, rank, world, device, seed, full=True, cpu=True, comparators=True):
+    """Times `steps` steps of workload w (after `warmup` untimed ones) and returns the
+    result dict.  full: also the end-to-end host-buffer leg; cpu: the CPU oracle
+    baseline (rank 0, one GPU); comparators: the dense comparators (rank 0)."""
     import block_sparse_long_prefill_b200 as moba
     from block_sparse_long_prefill_b200 import MobaPrefill
 
-    w = workloads.WORKLOADS[args.workload]
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream()
-    q, k, v = workloads.make_inputs(w, seed=args.seed + rank)
+    q, k, v = workloads.make_inputs(w, seed=seed + rank)
     if w.q_off:
         q = q[:, :, w.q_off:].contiguous()  # chunked prefill: the last nq query rows
-    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
     qd, kd, vd = q.to(device), k.to(device), v.to(device)
+    if full:
+        qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
     del q, k, v
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
 
+    nchunks = layout_chunks(w) if w.kind == "moba" else 1
     if w.kind == "moba":
         runner = MobaPrefill(w.batch, w.hq, w.hkv, w.nq, w.d, w.block, w.topk, w.window,
                              device=device, kv_len=w.seqlen)
@@ -344,8 +372,7 @@ def run_ours(args, rank, world, device):
             elif w.gate == "static":
                 yield "pool"  # no pooled keys
                 moba.moba_select_static(w.batch, w.hq, w.hkv, w.nq, w.d, w.block, w.topk, w.sink,
-                                        runner.workspace, kv_len=w.seqlen, idx=runner.idx,
-                                        device=device)
+                                        runner.workspace, kv_len=w.seqlen, idx=runner.idx)
             else:
                 moba.moba_pool_keys(kd, w.block, runner.kbar, runner.kbar_split)
                 yield "pool"
@@ -356,26 +383,6 @@ def run_ours(args, rank, world, device):
                                      w.window, out=runner.out, lse=runner.lse)
             yield "attention"
         out_t, lse_t = runner.out, runner.lse
-        layout_chunks = 1
-        chunk_rows = w.nq
-        try:
-            per_row = (w.topk if w.topk > 1 else 0) * (w.d * 2 + 4) * w.batch * w.hq
-            cap = 4 << 30
-            if per_row * w.nq > cap:
-                chunk_rows = max(128, (cap // per_row) // 128 * 128)
-                layout_chunks = math.ceil(w.nq / chunk_rows)
-        except ZeroDivisionError:
-            pass
-        # pool, gate, scatter (+ a scan launch when the general gate runs: the
-        # tensor-core gate's last CTA writes the list offsets itself), and per query
-        # chunk: past-block pass, own-block pass, merge (only the own-block pass when
-        # topk = 1).
-        tc_gate = -(-w.seqlen // w.block) <= 256 and w.topk - 1 < 32 and w.gate == "mean"
-        if w.gate == "static":
-            sel_launches = 1 + (2 if w.topk > 1 else 0)       # static gate, scan, scatter
-        else:
-            sel_launches = 2 + ((1 if tc_gate else 2) if w.topk > 1 else 0)
-        launches_per_step = sel_launches + layout_chunks * (3 if w.topk > 1 else 1)
     else:
         out_t = torch.empty_like(qd)
         lse_t = torch.empty(w.batch, w.hq, w.seqlen, dtype=torch.float32, device=device)
@@ -383,16 +390,17 @@ def run_ours(args, rank, world, device):
         def stages():
             moba.swa_attn_fwd(qd, kd, vd, w.window, out=out_t, lse=lse_t)
             yield "attention"
-        launches_per_step = 1
 
-    # Per-pass events inside moba_attn_fwd (first query chunk): the dominant kernel's
-    # own launch duration, timed on the stream it runs on.
-    pass_names = []
+    # Events recorded by moba_attn_fwd before its first kernel and after each launch
+    # (every pass of every query chunk), so that each kernel is timed over all of its
+    # launches on the stream it runs on.
+    chunk_passes = []
     if w.kind == "moba":
-        pass_names = (["past_block_pass", "own_block_pass", "merge_pass"] if w.topk > 1
-                      else ["own_block_pass"])
-    pass_evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(pass_names) + 1)]
-    per_pass = {n: [] for n in pass_names}
+        chunk_passes = (["past_block_pass", "own_block_pass", "merge_pass"] if w.topk > 1
+                        else ["own_block_pass"])
+    pass_seq = chunk_passes * nchunks
+    pass_evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(pass_seq) + 1)]
+    per_pass = {n: 0.0 for n in chunk_passes}
 
     def step_timed():
         evs = [torch.cuda.Event(enable_timing=True)]
@@ -405,7 +413,7 @@ def run_ours(args, rank, world, device):
             names.append(name)
         return evs, names
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         for _ in stages():
             pass
     torch.cuda.synchronize()
@@ -419,69 +427,71 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize()
     per_stage = {}
     total_ms = 0.0
-    if pass_names:
+    if pass_seq:
         moba.set_pass_events(pass_evs)
     with ClockSampler(torch.cuda.current_device()) as clk:
         clk.mark_start()
-        for _ in range(args.steps):
+        for _ in range(steps):
             flush.zero_()
             evs, names = step_timed()
             torch.cuda.synchronize()
             total_ms += evs[0].elapsed_time(evs[-1])
             for a, b_, n in zip(evs[:-1], evs[1:], names):
                 per_stage.setdefault(n, []).append(a.elapsed_time(b_))
-            for a, b_, n in zip(pass_evs[:-1], pass_evs[1:], pass_names):
-                per_pass[n].append(a.elapsed_time(b_))
+            for a, b_, n in zip(pass_evs[:-1], pass_evs[1:], pass_seq):
+                per_pass[n] += a.elapsed_time(b_) / steps
         clk.mark_stop()
     torch.cuda.synchronize()
-    if pass_names:
+    if pass_seq:
         moba.set_pass_events(None)
     total_ms = max_over_ranks(total_ms, device)
     if world > 1:
         torch.distributed.barrier()
     assert moba.device_status() == 0
     assert torch.isfinite(out_t.float()).all().item(), "non-finite output"
-    ms = total_ms / args.steps
+    ms = total_ms / steps
     tflops_total = weak_scaling_rate(flops, world, ms) / 1e12
     tokens = weak_scaling_rate(w.batch * w.nq, world, ms)
 
     hbm, tc_peak, tc_sus, peak_kind = peaks()
-    stage_ms = {n: sum(v) / len(v) for n, v in per_stage.items()}
+    stage_ms = {n: sum(v_) / len(v_) for n, v_ in per_stage.items()}
     attn_ms = stage_ms["attention"]
     achieved = flops / (attn_ms * 1e-3) / 1e12
     extra = {}
     kname = f"attn_fwd_kernel<{w.d}, 0>"
     if w.kind == "moba":
-        # Work of each pass over the first query chunk (all of it for one chunk).
-        work = pass_work_moba(runner.idx, w, chunk_rows)
-        pass_ms = {n: sum(v) / len(v) for n, v in per_pass.items()}
+        work = pass_work_moba(runner.idx, w)
         passes = {}
-        for n in pass_names:
-            t = pass_ms[n] * 1e-3
+        for n in chunk_passes:
+            t = per_pass[n] * 1e-3
+            rec = {"ms": round(per_pass[n], 4), "launches": nchunks}
             if n == "merge_pass":
                 gbs = work[n] / t / 1e9
-                passes[n] = {"ms": round(pass_ms[n], 4), "bytes": work[n], "gbs": round(gbs, 1),
-                             "frac_hbm": round(gbs / hbm, 4)}
+                rec.update({"bytes": work[n], "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)})
             else:
                 tf = work[n] / t / 1e12
-                passes[n] = {"ms": round(pass_ms[n], 4), "flops": work[n], "tflops": round(tf, 2),
-                             "frac": round(tf / tc_peak, 4)}
+                rec.update({"flops": work[n], "tflops": round(tf, 2), "frac": round(tf / tc_peak, 4)})
+            passes[n] = rec
         extra["passes"] = passes
         extra["attention_stage"] = {"ms": round(attn_ms, 4), "tflops": round(achieved, 2),
                                     "frac": round(achieved / tc_peak, 4),
                                     "note": "whole moba_attn_fwd call: all passes, all query chunks"}
-        dom = max((n for n in pass_names if n != "merge_pass"), key=lambda n: pass_ms[n])
+        dom = max((n for n in chunk_passes if n != "merge_pass"), key=lambda n: per_pass[n])
         kname = f"attn_fwd_kernel<{w.d}, {1 if dom == 'past_block_pass' else 0}>"
+        traffic = stored_traffic(w.name, kname)
         roofline = {"bound": "tensor", "achieved": passes[dom]["tflops"], "peak": tc_peak,
                     "unit": "TFLOP/s", "frac": passes[dom]["frac"],
-                    "traffic": stored_traffic(w.name, kname),
-                    "kernel": f"{kname} ({dom.replace('_', ' ')}; first query chunk)",
-                    "work": "4*d FLOPs per attended (query, key) pair of the pass",
-                    "peak_kind": f"bf16 dense burst, {peak_kind}"}
+                    "traffic": None if traffic is None else traffic / nchunks,
+                    "kernel": f"{kname} ({dom.replace('_', ' ')}; {nchunks} launches per step, "
+                              "one per query chunk)",
+                    "work": "4*d FLOPs per attended (query, key) pair of the pass, all launches",
+                    "peak_kind": f"bf16 dense burst, {peak_kind}",
+                    "frac_of_sustained": round(passes[dom]["tflops"] / tc_sus, 4) if tc_sus else None}
     else:
+        traffic = stored_traffic(w.name, kname)
         roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": tc_peak,
                     "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
-                    "traffic": stored_traffic(w.name, kname),
+                    "traffic": traffic,
                     "kernel": f"{kname} (swa_attn_fwd: one launch)",
                     "work": "4*d FLOPs per attended (query, key) pair",
                     "peak_kind": f"bf16 dense burst, {peak_kind}"}
@@ -496,97 +506,63 @@ def run_ours(args, rank, world, device):
                               "frac_hbm": round(sel_bytes / (sel_ms * 1e-3) / 1e9 / hbm, 4)}
 
     # ---------------------------------------------------------------- e2e (host buffers)
-    out_h = torch.empty(out_t.shape, dtype=out_t.dtype, pin_memory=True)
-    lse_h = torch.empty(lse_t.shape, dtype=lse_t.dtype, pin_memory=True)
-    e2e_ms = 0.0
-    # The MoBA prefill from host buffers goes through MobaPrefillHost, which overlaps the
-    # copies of one KV-head group with the kernels of the previous one; the variants
-    # (chunks, other gates) copy in, run and copy out in sequence.
-    host = None
-    if w.kind == "moba" and w.gate == "mean" and not w.q_off:
-        host = moba.MobaPrefillHost(w.batch, w.hq, w.hkv, w.seqlen, w.d, w.block, w.topk,
-                                    w.window, device=device)
-    for it in range(args.warmup + args.steps):
-        flush.zero_()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+    e2e = None
+    if full:
+        out_h = torch.empty(out_t.shape, dtype=out_t.dtype, pin_memory=True)
+        lse_h = torch.empty(lse_t.shape, dtype=lse_t.dtype, pin_memory=True)
+        e2e_ms = 0.0
+        # The MoBA prefill from host buffers goes through MobaPrefillHost, which overlaps
+        # the copies of one KV-head group with the kernels of the previous one; the
+        # variants (chunks, other gates) copy in, run and copy out in sequence.
+        host = None
+        if w.kind == "moba" and w.gate == "mean" and not w.q_off:
+            host = moba.MobaPrefillHost(w.batch, w.hq, w.hkv, w.seqlen, w.d, w.block, w.topk,
+                                        w.window, device=device)
+        for it in range(warmup + steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            if host is not None:
+                host(qh, kh, vh, out_h, lse_h)
+            else:
+                qd.copy_(qh, non_blocking=True)
+                kd.copy_(kh, non_blocking=True)
+                vd.copy_(vh, non_blocking=True)
+                for _ in stages():
+                    pass
+                out_h.copy_(out_t, non_blocking=True)
+                lse_h.copy_(lse_t, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if it >= warmup:
+                e2e_ms += e0.elapsed_time(e1)
         if host is not None:
-            host(qh, kh, vh, out_h, lse_h)
-        else:
-            qd.copy_(qh, non_blocking=True)
-            kd.copy_(kh, non_blocking=True)
-            vd.copy_(vh, non_blocking=True)
-            for _ in stages():
-                pass
-            out_h.copy_(out_t, non_blocking=True)
-            lse_h.copy_(lse_t, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        if it >= args.warmup:
-            e2e_ms += e0.elapsed_time(e1)
-    if host is not None:
-        # The pipelined result is the device path's (checked on the last step).
-        assert torch.equal(out_h, out_t.cpu()) and torch.equal(lse_h, lse_t.cpu()), "e2e mismatch"
-        del host
-    e2e_ms = max_over_ranks(e2e_ms, device) / args.steps
-    h2d = (qh.numel() + kh.numel() + vh.numel()) * 2
-    d2h = out_h.numel() * 2 + lse_h.numel() * 4
-    e2e = {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
-           "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            # The pipelined result is the device path's (checked on the last step).
+            assert torch.equal(out_h, out_t.cpu()) and torch.equal(lse_h, lse_t.cpu()), "e2e mismatch"
+            del host
+        e2e_ms = max_over_ranks(e2e_ms, device) / steps
+        h2d = (qh.numel() + kh.numel() + vh.numel()) * 2
+        d2h = out_h.numel() * 2 + lse_h.numel() * 4
+        e2e = {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+               "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h,
+               "path": "MobaPrefillHost (pinned host buffers, KV-head groups pipelined)"
+                       if (w.kind == "moba" and w.gate == "mean" and not w.q_off)
+                       else "copies in, the step, copies out"}
+        del out_h, lse_h
 
     # ---------------------------------------------------------------- comparators
     comps = {}
-    if not args.no_comparators and rank == 0:
-        dflops = 4.0 * w.d * dense_pairs(w)
-        G = w.hq // w.hkv
-        kr = kd.repeat_interleave(G, dim=1) if G > 1 else kd
-        vr = vd.repeat_interleave(G, dim=1) if G > 1 else vd
-        import torch.nn.functional as F
-
-        def timeit(fn, reps):
-            for _ in range(2):
-                fn()
-            torch.cuda.synchronize()
-            tot = 0.0
-            for _ in range(reps):
-                flush.zero_()
-                a = torch.cuda.Event(enable_timing=True)
-                b_ = torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                fn()
-                b_.record(stream)
-                torch.cuda.synchronize()
-                tot += a.elapsed_time(b_)
-            return tot / reps
-
-        own_out = torch.empty_like(qd)
-        own_lse = torch.empty(w.batch, w.hq, w.nq, dtype=torch.float32, device=device)
-        od_ms = timeit(lambda: moba.swa_attn_fwd_chunk(qd, kd, vd, w.seqlen, out=own_out, lse=own_lse),
-                       max(3, args.steps // 4))
-        comps = {"dense_causal_own_kernel": {"ms": round(od_ms, 4),
-                                             "tflops": round(dflops / (od_ms * 1e-3) / 1e12, 2),
-                                             "frac_of_peak": round(dflops / (od_ms * 1e-3) / 1e12
-                                                                   / tc_peak, 4)}}
-        if not w.q_off:
-            # torch's is_causal aligns the queries with the first keys, so it times whole
-            # prefills only.
-            sd_ms = timeit(lambda: F.scaled_dot_product_attention(qd, kr, vr, is_causal=True),
-                           max(3, args.steps // 4))
-            comps["dense_causal_sdpa"] = {"ms": round(sd_ms, 4),
-                                          "tflops": round(dflops / (sd_ms * 1e-3) / 1e12, 2),
-                                          "speedup_of_moba": round(sd_ms / ms, 3)}
-        del kr, vr
+    if comparators and rank == 0:
+        comps = dense_comparators(w, qd, kd, vd, flush, stream, ms, steps, tc_peak)
 
     cpu = None
-    if not args.no_cpu_baseline and rank == 0 and world == 1:
-        cpu = cpu_baseline(w, args.seed, target_s=12.0)
+    if full and cpu and rank == 0 and world == 1:
+        cpu = cpu_baseline(w, seed, target_s=12.0, tensors=None if w.q_off else (qh, kh, vh))
 
     clocks = clk.summary()
-    line = {"metric": METRIC, "value": round(tflops_total, 2), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0,1) q,k,v; per-block key offsets; no dataset)",
+    line = {"value": round(tflops_total, 2), "ms_per_step": round(ms, 4),
             "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv,
                        "seq_len": w.seqlen, "q_len": w.nq, "gate": w.gate, "d": w.d,
                        "block": w.block, "topk": w.topk,
@@ -595,21 +571,102 @@ def run_ours(args, rank, world, device):
             "tokens_per_s": round(tokens, 1), "attended_flops_per_step": flops,
             "stages_ms": {k_: round(v_, 4) for k_, v_ in stage_ms.items()},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
+            "gpu_launches": launches_per_step(w) * steps, "clocks": clocks}
     line.update(extra)
     line.update(comps)
     return line
 
 
+def dense_comparators(w, qd, kd, vd, flush, stream, moba_ms, steps, tc_peak):
+    """Dense causal attention on the same inputs: this library's own kernel (sliding
+    window >= N) and torch SDPA (a library call).  Problems above a PFLOP are timed
+    once, after a warm-up on their first 8192 rows."""
+    import torch.nn.functional as F
+
+    import block_sparse_long_prefill_b200 as moba
+    dflops = 4.0 * w.d * dense_pairs(w)
+    big = dflops > 1e15
+    reps = 1 if big else max(3, steps // 4)
+
+    def timeit(fn, warm):
+        for _ in range(1 if big else 2):
+            warm()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b_ = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b_.record(stream)
+            torch.cuda.synchronize()
+            tot += a.elapsed_time(b_)
+        return tot / reps
+
+    def sl(t):  # the first 8192 rows (warm-up of the big problems)
+        return t[:, :, :8192] if big else t
+
+    own_out = torch.empty_like(qd)
+    own_lse = torch.empty(w.batch, w.hq, w.nq, dtype=torch.float32, device=qd.device)
+    od_ms = timeit(lambda: moba.swa_attn_fwd_chunk(qd, kd, vd, w.seqlen, out=own_out, lse=own_lse),
+                   lambda: moba.swa_attn_fwd(sl(qd), sl(kd), sl(vd), w.seqlen))
+    del own_out, own_lse
+    comps = {"dense_causal_own_kernel": {"ms": round(od_ms, 4), "reps": reps,
+                                         "tflops": round(dflops / (od_ms * 1e-3) / 1e12, 2),
+                                         "frac_of_peak": round(dflops / (od_ms * 1e-3) / 1e12
+                                                               / tc_peak, 4)}}
+    if not w.q_off:
+        # torch's is_causal aligns the queries with the first keys, so it times whole
+        # prefills only.
+        G = w.hq // w.hkv
+        kr = kd.repeat_interleave(G, dim=1) if G > 1 else kd
+        vr = vd.repeat_interleave(G, dim=1) if G > 1 else vd
+        sd_ms = timeit(lambda: F.scaled_dot_product_attention(qd, kr, vr, is_causal=True),
+                       lambda: F.scaled_dot_product_attention(sl(qd), sl(kr), sl(vr), is_causal=True))
+        del kr, vr
+        comps["dense_causal_sdpa"] = {"ms": round(sd_ms, 4), "reps": reps,
+                                      "tflops": round(dflops / (sd_ms * 1e-3) / 1e12, 2),
+                                      "speedup_of_moba": round(sd_ms / moba_ms, 3)}
+    return comps
+
+
+def run_ours(args, rank, world, device):
+    w = workloads.WORKLOADS[args.workload]
+    main = measure(w, args.steps, args.warmup, rank, world, device, args.seed,
+                   full=not args.no_e2e, cpu=not args.no_cpu_baseline,
+                   comparators=not args.no_comparators)
+    line = {"metric": METRIC, "value": main.pop("value"), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": main.pop("ms_per_step"),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) q,k,v; per-block key offsets; no dataset)"}
+    line.update(main)
+    extras = [x for x in args.extra_workloads.split(",") if x and x != w.name]
+    if extras:
+        torch.cuda.empty_cache()
+        line["workloads"] = {}
+        for name in extras:
+            we = workloads.WORKLOADS[name]
+            r = measure(we, max(5, min(args.steps, 10)), args.warmup, rank, world, device,
+                        args.seed, full=False, comparators=not args.no_comparators)
+            for key in ("cpu_baseline", "e2e"):
+                r.pop(key, None)
+            r["steps"] = max(5, min(args.steps, 10))
+            line["workloads"][name] = r
+            torch.cuda.empty_cache()
+    return line
+
+
 # ------------------------------------------------------------ oracle timing
 
-def cpu_baseline(w: workloads.Workload, seed: int, target_s: float):
+def cpu_baseline(w: workloads.Workload, seed: int, target_s: float, tensors=None):
     """Times the fp64 oracle on this workload: the full key pooling plus selection and
     attention for a seeded sample of query rows (all heads), sized to about target_s
-    seconds; reports the attended TFLOP/s extrapolated to the whole workload."""
+    seconds; reports the attended TFLOP/s extrapolated to the whole workload.
+    ``tensors``: the workload's (q, k, v) host tensors when already drawn."""
     import oracle
 
-    q, k, v = workloads.make_inputs(w, seed)
+    q, k, v = tensors if tensors is not None else workloads.make_inputs(w, seed)
     rng = np.random.default_rng(seed + 2000)
     N = w.nq  # query rows: positions q_off .. seqlen - 1
 
@@ -667,9 +724,10 @@ def run_reference(args, rank, world):
         return None
     per_step = []
     last = None
+    # The inputs are drawn once; every step times the oracle on its own row sample.
+    tensors = workloads.make_inputs(w, args.seed)
     for it in range(args.warmup + args.steps):
-        t0 = time.perf_counter()
-        last = cpu_baseline(w, args.seed + it, target_s=3.0)
+        last = cpu_baseline(w, args.seed + it, target_s=3.0, tensors=tensors)
         if it >= args.warmup:
             per_step.append(last["value"])
     value = statistics.median(per_step)

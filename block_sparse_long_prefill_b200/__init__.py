@@ -103,6 +103,35 @@ def _t(x: torch.Tensor) -> MobaTensor:
     return MobaTensor(x.data_ptr(), x.stride(0), x.stride(1), x.stride(2))
 
 
+_BF16, _F32, _I32 = torch.bfloat16, torch.float32, torch.int32
+
+
+def _device(fn: str, *specs):
+    """Checks the tensors a call passes to the library and returns their device.
+
+    Each spec is (name, tensor, dtype, must_be_contiguous, shape or None); None tensors
+    are skipped.  Every tensor must be a CUDA tensor of the given dtype, and all of them
+    must sit on one device: the library launches on the current device, which the
+    wrappers make that device."""
+    dev = None
+    for name, t, dt, contig, shape in specs:
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise ValueError(f"{fn}: {name} must be a CUDA tensor")
+        if dt is not None and t.dtype != dt:
+            raise ValueError(f"{fn}: {name} must be {dt}, not {t.dtype}")
+        if contig and not t.is_contiguous():
+            raise ValueError(f"{fn}: {name} must be contiguous")
+        if shape is not None and tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{fn}: {name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{fn}: every tensor must be on {dev}; {name} is on {t.device}")
+    return dev
+
+
 def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -121,12 +150,16 @@ def moba_pool_keys(k: torch.Tensor, block: int, kbar=None, kbar_split=None, stre
     [b, hkv, n, d], kbar_split bf16 [b, hkv, 2, n, d])."""
     b, hkv, N, d = k.shape
     n = -(-N // block)  # a partial last block when block does not divide N
-    if kbar is None:
-        kbar = torch.empty(b, hkv, n, d, dtype=torch.float32, device=k.device)
-    if kbar_split is None:
-        kbar_split = torch.empty(b, hkv, 2, n, d, dtype=torch.bfloat16, device=k.device)
-    _check("moba_pool_keys", _lib.moba_pool_keys(_t(k), b, hkv, N, d, block, kbar.data_ptr(),
-                                                 kbar_split.data_ptr(), _stream(stream)))
+    dev = _device("moba_pool_keys", ("k", k, _BF16, False, None),
+                  ("kbar", kbar, _F32, True, (b, hkv, n, d)),
+                  ("kbar_split", kbar_split, _BF16, True, (b, hkv, 2, n, d)))
+    with torch.cuda.device(dev):
+        if kbar is None:
+            kbar = torch.empty(b, hkv, n, d, dtype=torch.float32, device=dev)
+        if kbar_split is None:
+            kbar_split = torch.empty(b, hkv, 2, n, d, dtype=torch.bfloat16, device=dev)
+        _check("moba_pool_keys", _lib.moba_pool_keys(_t(k), b, hkv, N, d, block, kbar.data_ptr(),
+                                                     kbar_split.data_ptr(), _stream(stream)))
     return kbar, kbar_split
 
 
@@ -135,45 +168,20 @@ def moba_select_topk(q: torch.Tensor, kbar_split: torch.Tensor, block: int, topk
     """[MoBA] §블록 분할과 top-k 게이팅 + §인과성 보존: per-row block choices (int32
     [b, hq, N, topk], ascending, -1 padded) and the dispatch lists in ``workspace``."""
     b, hq, N, d = q.shape
-    hkv = kbar_split.shape[1]
-    if idx is None:
-        idx = torch.empty(b, hq, N, topk, dtype=torch.int32, device=q.device)
-    _check("moba_select_topk",
-           _lib.moba_select_topk(_t(q), kbar_split.data_ptr(), b, hq, hkv, N, d, block, topk,
-                                 idx.data_ptr(), workspace.data_ptr(), workspace.numel(),
-                                 _stream(stream)))
-    return idx
+    return moba_select_topk_chunk(q, kbar_split, block, topk, N, workspace, idx, stream)
 
 
 def moba_attn_fwd(q, k, v, idx, block: int, topk: int, workspace: torch.Tensor, window: int = 0,
                   scale: float = 0.0, out=None, lse=None, stream=None):
     """[MoBA] §MoBA의 구현: attention over the selected blocks (unioned with the causal
     window).  Returns (out bf16 [b, hq, N, d], lse float32 [b, hq, N])."""
-    b, hq, N, d = q.shape
-    hkv = k.shape[1]
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device)
-    _check("moba_attn_fwd",
-           _lib.moba_attn_fwd(_t(q), _t(k), _t(v), idx.data_ptr(), b, hq, hkv, N, d, block, topk,
-                              window, float(scale), _t(out), lse.data_ptr(), workspace.data_ptr(),
-                              workspace.numel(), _stream(stream)))
-    return out, lse
+    return moba_attn_fwd_chunk(q, k, v, idx, block, topk, workspace, window, scale, out, lse,
+                               stream)
 
 
 def swa_attn_fwd(q, k, v, window: int, scale: float = 0.0, out=None, lse=None, stream=None):
     """[SWA] §슬라이딩 윈도우 마스크: causal band attention (window >= N is dense causal)."""
-    b, hq, N, d = q.shape
-    hkv = k.shape[1]
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device)
-    _check("swa_attn_fwd",
-           _lib.swa_attn_fwd(_t(q), _t(k), _t(v), b, hq, hkv, N, d, window, float(scale), _t(out),
-                             lse.data_ptr(), _stream(stream)))
-    return out, lse
+    return swa_attn_fwd_chunk(q, k, v, window, scale, out, lse, stream)
 
 
 def workspace_size_chunk(batch, hq, hkv, N, Nk, d, block, topk) -> int:
@@ -189,12 +197,18 @@ def moba_select_topk_chunk(q, kbar_split: torch.Tensor, block: int, topk: int, k
     positions (pooled keys of all kv_len positions in ``kbar_split``)."""
     b, hq, N, d = q.shape
     hkv = kbar_split.shape[1]
-    if idx is None:
-        idx = torch.empty(b, hq, N, topk, dtype=torch.int32, device=q.device)
-    _check("moba_select_topk_chunk",
-           _lib.moba_select_topk_chunk(_t(q), kbar_split.data_ptr(), b, hq, hkv, N, kv_len, d, block,
-                                       topk, idx.data_ptr(), workspace.data_ptr(), workspace.numel(),
-                                       _stream(stream)))
+    dev = _device("moba_select_topk", ("q", q, _BF16, False, None),
+                  ("kbar_split", kbar_split, _BF16, True, None),
+                  ("workspace", workspace, None, True, None),
+                  ("idx", idx, _I32, True, (b, hq, N, topk)))
+    with torch.cuda.device(dev):
+        if idx is None:
+            idx = torch.empty(b, hq, N, topk, dtype=torch.int32, device=dev)
+        _check("moba_select_topk",
+               _lib.moba_select_topk_chunk(_t(q), kbar_split.data_ptr(), b, hq, hkv, N, kv_len, d,
+                                           block, topk, idx.data_ptr(), workspace.data_ptr(),
+                                           workspace.numel() * workspace.element_size(),
+                                           _stream(stream)))
     return idx
 
 
@@ -204,14 +218,23 @@ def moba_attn_fwd_chunk(q, k, v, idx, block: int, topk: int, workspace: torch.Te
     values of all k.shape[2] positions.  Returns (out, lse) for the N rows."""
     b, hq, N, d = q.shape
     hkv, Nk = k.shape[1], k.shape[2]
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device)
-    _check("moba_attn_fwd_chunk",
-           _lib.moba_attn_fwd_chunk(_t(q), _t(k), _t(v), idx.data_ptr(), b, hq, hkv, N, Nk, d, block,
-                                    topk, window, float(scale), _t(out), lse.data_ptr(),
-                                    workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    dev = _device("moba_attn_fwd", ("q", q, _BF16, False, None), ("k", k, _BF16, False, None),
+                  ("v", v, _BF16, False, tuple(k.shape)),
+                  ("idx", idx, _I32, True, (b, hq, N, topk)),
+                  ("workspace", workspace, None, True, None),
+                  ("out", out, _BF16, False, tuple(q.shape)),
+                  ("lse", lse, _F32, True, (b, hq, N)))
+    with torch.cuda.device(dev):
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty(b, hq, N, dtype=torch.float32, device=dev)
+        _check("moba_attn_fwd",
+               _lib.moba_attn_fwd_chunk(_t(q), _t(k), _t(v), idx.data_ptr(), b, hq, hkv, N, Nk, d,
+                                        block, topk, window, float(scale), _t(out), lse.data_ptr(),
+                                        workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)))
     return out, lse
 
 
@@ -219,28 +242,40 @@ def swa_attn_fwd_chunk(q, k, v, window: int, scale: float = 0.0, out=None, lse=N
     """Sliding-window attention of the last N positions (q) over k.shape[2] positions."""
     b, hq, N, d = q.shape
     hkv, Nk = k.shape[1], k.shape[2]
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device)
-    _check("swa_attn_fwd_chunk",
-           _lib.swa_attn_fwd_chunk(_t(q), _t(k), _t(v), b, hq, hkv, N, Nk, d, window, float(scale),
-                                   _t(out), lse.data_ptr(), _stream(stream)))
+    dev = _device("swa_attn_fwd", ("q", q, _BF16, False, None), ("k", k, _BF16, False, None),
+                  ("v", v, _BF16, False, tuple(k.shape)),
+                  ("out", out, _BF16, False, tuple(q.shape)),
+                  ("lse", lse, _F32, True, (b, hq, N)))
+    with torch.cuda.device(dev):
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty(b, hq, N, dtype=torch.float32, device=dev)
+        _check("swa_attn_fwd",
+               _lib.swa_attn_fwd_chunk(_t(q), _t(k), _t(v), b, hq, hkv, N, Nk, d, window,
+                                       float(scale), _t(out), lse.data_ptr(), _stream(stream)))
     return out, lse
 
 
 def moba_select_static(batch: int, hq: int, hkv: int, N: int, d: int, block: int, topk: int,
                        sink: int, workspace: torch.Tensor, kv_len=None, idx=None, stream=None,
-                       device="cuda"):
+                       device=None):
     """Static gate in place of moba_select_topk: own block, the first ``sink`` blocks and
     the most recent past blocks (sink = 0: sliding window at block granularity; sink = 1:
     an attention sink).  N query rows, the last N of ``kv_len`` (default N) positions."""
     kv = kv_len or N
-    if idx is None:
-        idx = torch.empty(batch, hq, N, topk, dtype=torch.int32, device=device)
-    _check("moba_select_static",
-           _lib.moba_select_static(batch, hq, hkv, N, kv, d, block, topk, sink, idx.data_ptr(),
-                                   workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    dev = _device("moba_select_static", ("workspace", workspace, None, True, None),
+                  ("idx", idx, _I32, True, (batch, hq, N, topk)))
+    if device is not None and torch.device(device) != dev and torch.device(device).index is not None:
+        raise ValueError(f"moba_select_static: device {device} differs from the workspace's {dev}")
+    with torch.cuda.device(dev):
+        if idx is None:
+            idx = torch.empty(batch, hq, N, topk, dtype=torch.int32, device=dev)
+        _check("moba_select_static",
+               _lib.moba_select_static(batch, hq, hkv, N, kv, d, block, topk, sink, idx.data_ptr(),
+                                       workspace.data_ptr(),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream(stream)))
     return idx
 
 
@@ -249,10 +284,14 @@ def moba_pool_keys_minmax(k: torch.Tensor, block: int, out=None, stream=None):
     (plane 1) of the keys."""
     b, hkv, N, d = k.shape
     n = -(-N // block)
-    if out is None:
-        out = torch.empty(b, hkv, 2, n, d, dtype=torch.bfloat16, device=k.device)
-    _check("moba_pool_keys_minmax",
-           _lib.moba_pool_keys_minmax(_t(k), b, hkv, N, d, block, out.data_ptr(), _stream(stream)))
+    dev = _device("moba_pool_keys_minmax", ("k", k, _BF16, False, None),
+                  ("out", out, _BF16, True, (b, hkv, 2, n, d)))
+    with torch.cuda.device(dev):
+        if out is None:
+            out = torch.empty(b, hkv, 2, n, d, dtype=torch.bfloat16, device=dev)
+        _check("moba_pool_keys_minmax",
+               _lib.moba_pool_keys_minmax(_t(k), b, hkv, N, d, block, out.data_ptr(),
+                                          _stream(stream)))
     return out
 
 
@@ -262,12 +301,18 @@ def moba_select_topk_minmax(q, kminmax: torch.Tensor, block: int, topk: int, kv_
     the last N of ``kv_len`` positions."""
     b, hq, N, d = q.shape
     hkv = kminmax.shape[1]
-    if idx is None:
-        idx = torch.empty(b, hq, N, topk, dtype=torch.int32, device=q.device)
-    _check("moba_select_topk_minmax",
-           _lib.moba_select_topk_minmax(_t(q), kminmax.data_ptr(), b, hq, hkv, N, kv_len, d, block,
-                                        topk, idx.data_ptr(), workspace.data_ptr(),
-                                        workspace.numel(), _stream(stream)))
+    dev = _device("moba_select_topk_minmax", ("q", q, _BF16, False, None),
+                  ("kminmax", kminmax, _BF16, True, None),
+                  ("workspace", workspace, None, True, None),
+                  ("idx", idx, _I32, True, (b, hq, N, topk)))
+    with torch.cuda.device(dev):
+        if idx is None:
+            idx = torch.empty(b, hq, N, topk, dtype=torch.int32, device=dev)
+        _check("moba_select_topk_minmax",
+               _lib.moba_select_topk_minmax(_t(q), kminmax.data_ptr(), b, hq, hkv, N, kv_len, d,
+                                            block, topk, idx.data_ptr(), workspace.data_ptr(),
+                                            workspace.numel() * workspace.element_size(),
+                                            _stream(stream)))
     return idx
 
 
@@ -276,11 +321,13 @@ def moba_prefill_chunk(q, k, v, block: int, topk: int, window: int = 0, stream=N
     selects and attends for the N rows; returns (out, lse, idx)."""
     b, hq, N, d = q.shape
     hkv, Nk = k.shape[1], k.shape[2]
-    _, ks = moba_pool_keys(k, block, stream=stream)
-    ws = torch.empty(workspace_size_chunk(b, hq, hkv, N, Nk, d, block, topk), dtype=torch.uint8,
-                     device=q.device)
-    idx = moba_select_topk_chunk(q, ks, block, topk, Nk, ws, stream=stream)
-    out, lse = moba_attn_fwd_chunk(q, k, v, idx, block, topk, ws, window, stream=stream)
+    dev = _device("moba_prefill_chunk", ("q", q, _BF16, False, None), ("k", k, _BF16, False, None))
+    with torch.cuda.device(dev):
+        _, ks = moba_pool_keys(k, block, stream=stream)
+        ws = torch.empty(workspace_size_chunk(b, hq, hkv, N, Nk, d, block, topk),
+                         dtype=torch.uint8, device=dev)
+        idx = moba_select_topk_chunk(q, ks, block, topk, Nk, ws, stream=stream)
+        out, lse = moba_attn_fwd_chunk(q, k, v, idx, block, topk, ws, window, stream=stream)
     return out, lse, idx
 
 
@@ -290,13 +337,19 @@ def moba_prefill_static(q, k, v, block: int, topk: int, window: int = 0, scale: 
     callers that cannot allocate device memory.  Returns (out, lse)."""
     b, hq, N, d = q.shape
     hkv = k.shape[1]
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device)
-    _check("moba_prefill_static",
-           _lib.moba_prefill_static(_t(q), _t(k), _t(v), b, hq, hkv, N, d, block, topk, window,
-                                    float(scale), _t(out), lse.data_ptr(), _stream(stream)))
+    dev = _device("moba_prefill_static", ("q", q, _BF16, False, None),
+                  ("k", k, _BF16, False, None), ("v", v, _BF16, False, tuple(k.shape)),
+                  ("out", out, _BF16, False, tuple(q.shape)),
+                  ("lse", lse, _F32, True, (b, hq, N)))
+    with torch.cuda.device(dev):
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty(b, hq, N, dtype=torch.float32, device=dev)
+        _check("moba_prefill_static",
+               _lib.moba_prefill_static(_t(q), _t(k), _t(v), b, hq, hkv, N, d, block, topk,
+                                        window, float(scale), _t(out), lse.data_ptr(),
+                                        _stream(stream)))
     return out, lse
 
 

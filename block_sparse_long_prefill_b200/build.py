@@ -36,15 +36,34 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    """Compile libmoba.so for sm_100a (cross-compiles without a GPU)."""
+    """Compile libmoba.so for sm_100a (cross-compiles without a GPU).  Each source is
+    compiled to an object file in parallel, then the objects are linked."""
     if not force and not _stale():
         return LIB
+    from concurrent.futures import ThreadPoolExecutor
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+
+    def compile_one(f):
+        obj = os.path.join(objdir, f.replace(".cu", f".{os.getpid()}.o"))
+        cmd = [_nvcc(), *compile_flags, *extra, "-I", INCLUDE, "-I", CSRC, "-c",
+               os.path.join(CSRC, f), "-o", obj]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        subprocess.check_call(cmd)
+        return obj
+
+    with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
+        objs = list(ex.map(compile_one, SOURCES))
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC,
-           *[os.path.join(CSRC, f) for f in SOURCES], "-o", tmp]
+    cmd = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC",
+           *objs, "-o", tmp]
     if verbose:
-        print(" ".join(cmd))
+        print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
+    for o in objs:
+        os.remove(o)
     os.replace(tmp, LIB)
     return LIB
 

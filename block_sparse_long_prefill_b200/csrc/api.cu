@@ -190,11 +190,12 @@ int make_kbar_maps(CUtensorMap *maps, const void *split, int batch, int hkv, int
 int launch_status(cudaError_t e) { return e == cudaSuccess ? MOBA_OK : MOBA_ERR_LAUNCH; }
 
 // Per-pass timing events of moba_attn_fwd (diagnostics; see moba_set_pass_events).
-cudaEvent_t g_pass_events[8];
+constexpr int kMaxPassEvents = 1024;
+cudaEvent_t g_pass_events[kMaxPassEvents];
 int g_pass_nevents = 0;
 
-void record_pass_event(int k, int chunk, cudaStream_t st) {
-  if (chunk == 0 && k < g_pass_nevents && g_pass_events[k]) cudaEventRecord(g_pass_events[k], st);
+void record_pass_event(int k, cudaStream_t st) {
+  if (k < g_pass_nevents && g_pass_events[k]) cudaEventRecord(g_pass_events[k], st);
 }
 
 // Device address of the status words on the current device.
@@ -461,7 +462,7 @@ int moba_attn_fwd_chunk(moba_tensor q, moba_tensor k, moba_tensor v, const int32
   p.nblk = w.nblk;
   p.lists_per_chunk = batch * hkv * w.nblk;
   int ev = 0;
-  record_pass_event(ev++, 0, st);
+  record_pass_event(ev++, st);
   for (int c = 0; c < w.nchunks; ++c) {
     p.chunk = c;
     p.row_begin = c * w.chunk_rows;
@@ -471,12 +472,12 @@ int moba_attn_fwd_chunk(moba_tensor q, moba_tensor k, moba_tensor v, const int32
       p.q_gather_tma = q_gather_tma;
       if ((rc = launch_status(launch_attn(gmaps, p, kGathered, nsm, st)))) return rc;
       p.q_gather_tma = 0;
-      record_pass_event(ev++, c, st);
+      record_pass_event(ev++, st);
     }
     p.ntiles = query_major_units(batch, hq, hkv, block, 1, p.row_begin, p.row_end);
     const int grid = p.ntiles < nsm ? p.ntiles : nsm;
     if ((rc = launch_status(launch_attn(maps, p, kQueryMajor, grid, st)))) return rc;
-    record_pass_event(ev++, c, st);
+    record_pass_event(ev++, st);
     if (w.npast > 0) {
       MergeParams mp{};
       mp.opart = p.opart;
@@ -491,7 +492,7 @@ int moba_attn_fwd_chunk(moba_tensor q, moba_tensor k, moba_tensor v, const int32
       mp.row_end = p.row_end;
       mp.q_off = q_off;
       if ((rc = launch_status(launch_merge(mp, st)))) return rc;
-      record_pass_event(ev++, c, st);
+      record_pass_event(ev++, st);
     }
   }
   return MOBA_OK;
@@ -506,9 +507,10 @@ int moba_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, const int32_t *id
 }
 
 int moba_set_pass_events(void *const *events, int count) {
-  if (count < 0 || count > 8) return MOBA_ERR_ARG;
+  if (count < 0 || count > kMaxPassEvents) return MOBA_ERR_ARG;
   if (!events) count = 0;
-  for (int k = 0; k < 8; ++k) g_pass_events[k] = (k < count) ? static_cast<cudaEvent_t>(events[k]) : nullptr;
+  for (int k = 0; k < kMaxPassEvents; ++k)
+    g_pass_events[k] = (k < count) ? static_cast<cudaEvent_t>(events[k]) : nullptr;
   g_pass_nevents = count;
   return MOBA_OK;
 }

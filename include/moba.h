@@ -190,17 +190,23 @@ int moba_select_static(int batch, int hq, int hkv, int N, int Nk, int d, int blo
 
 /*
  * The whole MoBA prefill (moba_pool_keys, moba_select_topk, moba_attn_fwd) without any
- * caller-provided workspace, for callers that cannot allocate device memory: code
- * inside a CUDA-graph capture that forbids allocation, plugins whose host framework
- * owns all allocations, runtimes with a memory budget fixed up front.  The paper has
- * no counterpart; it is a deployment convenience.
- *   Arguments as for moba_attn_fwd; out and lse are written, nothing else is.
+ * caller-provided workspace, for callers that cannot allocate device memory: plugins
+ * whose host framework owns every device allocation and hands them only their inputs
+ * and outputs, and runtimes whose memory budget is fixed and fully assigned up front.
+ * The paper has no counterpart; it is a deployment convenience.
+ *   Arguments as for moba_attn_fwd; out and lse are written, nothing else is.  Every
+ *   argument is checked before anything is enqueued.
  *   Scratch: one 32 MiB device array inside the library (held, on each GPU that runs
  *   this call, until the process exits).  Problems whose pooled keys, block choices
  *   and workspace (moba_workspace_size) need more return MOBA_ERR_TOO_LARGE.
- *   The first call on a device looks up the array's device address (keep it outside
- *   any stream capture).  All calls share the array: calls that overlap on the GPU
- *   (other streams, other host threads) race and must be serialised by the caller.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   The first call on a device (that device current) looks up the array's device
+ *   address and caches it per device and CUDA context, so a call after a
+ *   cudaDeviceReset looks it up again; make that first call before any stream
+ *   capture.  All calls share the array and it keeps the last call's contents (the
+ *   counters that must start at zero are cleared by every call): calls that overlap
+ *   on the GPU (other streams, other host threads) race and must be serialised by the
+ *   caller.
  */
 int moba_prefill_static(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq, int hkv,
                         int N, int d, int block, int topk, int window, float scale,
@@ -218,12 +224,13 @@ const char *moba_status_string(int status);
 /* Diagnostics for benchmarks: per-pass timing of moba_attn_fwd.  `events` holds
  * `count` cudaEvent_t handles created by the caller (count 0 or events NULL switches
  * this off).  While set, every moba_attn_fwd call records, on its stream, events[0]
- * before its first kernel and events[k] after its k-th kernel (k = 1, 2, 3: the
- * past-block pass, the own-block pass and the merge pass; with topk = 1 only the
- * own-block pass runs), for its first query chunk and as far as count allows.  The
- * library keeps the handles, not the events: they must outlive their use.  A
- * process-wide setting, not synchronised between host threads.
- * Returns MOBA_OK, or MOBA_ERR_ARG when count is outside [0, 8]. */
+ * before its first kernel and events[k] after its k-th kernel, as far as count
+ * allows.  The kernels run per query chunk, in launch order: the past-block pass, the
+ * own-block pass and the merge pass of chunk 0, then those of chunk 1, and so on (with
+ * topk = 1 only the own-block pass runs).  The library keeps the handles, not the
+ * events: they must outlive their use.  A process-wide setting, not synchronised
+ * between host threads.
+ * Returns MOBA_OK, or MOBA_ERR_ARG when count is outside [0, 1024]. */
 int moba_set_pass_events(void *const *events, int count);
 
 #ifdef __cplusplus

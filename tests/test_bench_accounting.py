@@ -46,8 +46,8 @@ def test_attended_pairs_equal_the_dense_mask_count(kw):
     assert got == _brute_pairs(w, idx)
     if w.topk >= w.nblocks and w.window == 0:
         assert got == bench.dense_pairs(w)
-    # The per-pass split covers the same work (one query chunk holds every row).
-    work = bench.pass_work_moba(torch.from_numpy(idx), w, w.nq)
+    # The per-pass split (summed over all query chunks) covers the same work.
+    work = bench.pass_work_moba(torch.from_numpy(idx), w)
     assert work["past_block_pass"] + work["own_block_pass"] == 4.0 * w.d * got
 
 
@@ -57,3 +57,16 @@ def test_swa_pairs_closed_form():
     j = np.arange(777)
     band = (j[None, :] <= i[:, None]) & (i[:, None] - j[None, :] < 100)
     assert bench.attended_pairs_swa(w) == int(band.sum()) * 3
+
+
+def test_layout_chunks_and_launch_counts_follow_the_workspace_rule():
+    """The benchmark's launch count per step: the selection launches plus three passes
+    per query chunk, with the chunk count of the 4 GiB partials rule."""
+    w = workloads.WORKLOADS["moba1m"]
+    per_row = w.topk * (w.d * 2 + 4) * w.batch * w.hq
+    rows = ((4 << 30) // per_row) // 128 * 128
+    assert bench.layout_chunks(w) == -(-w.nq // rows) > 1
+    assert bench.launches_per_step(w) == 3 + 3 * bench.layout_chunks(w)
+    assert bench.layout_chunks(workloads.WORKLOADS["gqa32k"]) == 1
+    assert bench.launches_per_step(workloads.WORKLOADS["gqa32k"]) == 6
+    assert bench.launches_per_step(workloads.WORKLOADS["swa16k"]) == 1

@@ -1,11 +1,11 @@
 """moba_prefill_static: the whole MoBA prefill for callers that cannot allocate device
-memory (code running under a CUDA-graph capture that forbids allocation, plugins
-whose host framework owns every allocation, runtimes with a fixed memory budget).
-It keeps its scratch in one fixed device array inside the library, so the caller
-passes only q, k, v and the outputs.  Its results must equal the allocating entry
-points' (moba_pool_keys -> moba_select_topk -> moba_attn_fwd) within the parity
-tolerance, on consecutive calls (the shared array keeps the previous call's
-contents, and the selection step must clear what has to start at zero)."""
+memory (plugins whose host framework owns every device allocation, runtimes whose
+memory budget is fixed and fully assigned up front).  It keeps its scratch in one fixed
+device array inside the library, so the caller passes only q, k, v and the outputs.
+Its results must equal the allocating entry points' (moba_pool_keys ->
+moba_select_topk -> moba_attn_fwd) within the parity tolerance, on consecutive calls
+(the shared array keeps the previous call's contents, and the selection step must
+clear what has to start at zero)."""
 import pytest
 import torch
 

@@ -4,11 +4,15 @@ This module holds no step of the method: it only draws q, k, v (and nothing else
 from seeded generators.  Both the CUDA path and the CPU oracle take their inputs from
 here, so they see the same bf16 values.
 
-Recipe: with ``torch.Generator('cpu').manual_seed(seed)`` draw q, k, v in that order
-as float32 N(0, 1) of shapes [b, hq, N, d], [b, hkv, N, d], [b, hkv, N, d]; for the
-MoBA workloads draw one offset vector per (batch, kv-head, block), N(0, 0.5^2) of
-shape [b, hkv, N/B, d], add it to every key of its block (so that the pooled keys
-separate and the gate's choices are not near-ties); cast all three to bf16.
+Recipe: every tensor is viewed as rows of d values ([b, h, N, d] flattened to
+[b*h*N, d]) and split into chunks of 2^17 rows; chunk c of stream s (0: q, 1: k, 2: v,
+3: the key offsets) is drawn as float32 N(0, 1) from its own
+``torch.Generator('cpu').manual_seed(seed * 2^32 + s * 2^24 + c)``, so the chunks are
+independent and are drawn in parallel threads.  q is [b, hq, N, d], k and v are
+[b, hkv, N, d].  For the MoBA workloads one offset vector per (batch, kv-head, block),
+N(0, 0.5^2) of shape [b, hkv, ceil(N/B), d] (stream 3), is added to every key of its
+block (so that the pooled keys separate and the gate's choices are not near-ties);
+all three are then cast to bf16.
 """
 from __future__ import annotations
 
@@ -70,6 +74,10 @@ WORKLOADS = {
                           note="GQA 8/4, 32 blocks of 2048, top-16 unioned with window 512"),
     "moba1m": Workload("moba1m", 1, 32, 8, 1 << 20, 128, block=4096, topk=12, key_offset_std=0.5,
                        sampled_rows=True, note="1M tokens, 256 blocks of 4096, top-12"),
+    "moba1m_4h": Workload("moba1m_4h", 1, 4, 1, 1 << 20, 128, block=4096, topk=12,
+                          key_offset_std=0.5, sampled_rows=True,
+                          note="one KV head of the 1M-token workload (4 q-heads): the same "
+                               "256 blocks and top-12 at an eighth of the size"),
     "gqa32k_chunk8k": Workload("gqa32k_chunk8k", 1, 32, 8, 32768, 128, block=512, topk=3,
                                key_offset_std=0.5, q_len=8192,
                                note="chunked prefill: the last 8192 queries of the gqa32k "
@@ -84,33 +92,57 @@ WORKLOADS = {
 }
 
 
+_CHUNK_ROWS = 1 << 17
+
+
+def _seed(seed: int, stream: int, chunk: int) -> int:
+    return seed * (1 << 32) + stream * (1 << 24) + chunk
+
+
+def _draw_rows(shape, seed: int, stream: int, pool, row_fn=None) -> torch.Tensor:
+    """bf16 tensor of ``shape`` (last dim d) drawn chunk by chunk: chunk c holds rows
+    [c * 2^17, (c + 1) * 2^17) of the [rows, d] view, float32 N(0, 1) from its own
+    generator; ``row_fn(r0, r1, x)`` may adjust the float32 chunk before the cast."""
+    d = shape[-1]
+    out = torch.empty(shape, dtype=torch.bfloat16)
+    flat = out.view(-1, d)
+    rows = flat.shape[0]
+
+    def one(c):
+        r0, r1 = c * _CHUNK_ROWS, min(rows, (c + 1) * _CHUNK_ROWS)
+        g = torch.Generator("cpu").manual_seed(_seed(seed, stream, c))
+        x = torch.randn((r1 - r0, d), generator=g, dtype=torch.float32)
+        if row_fn is not None:
+            row_fn(r0, r1, x)
+        flat[r0:r1] = x.to(torch.bfloat16)
+
+    list(pool.map(one, range(-(-rows // _CHUNK_ROWS))))
+    return out
+
+
 def make_inputs(w: Workload, seed: int = 0, device: str = "cpu"):
     """q [b,hq,N,d], k, v [b,hkv,N,d] as bf16 tensors on ``device`` (drawn on the CPU)."""
-    g = torch.Generator("cpu").manual_seed(seed)
+    import os
+    from concurrent.futures import ThreadPoolExecutor
     b, N, d = w.batch, w.seqlen, w.d
-    q = _randn_bf16((b, w.hq, N, d), g)
-    k32 = torch.randn((b, w.hkv, N, d), generator=g, dtype=torch.float32)
-    v = _randn_bf16((b, w.hkv, N, d), g)
-    if w.key_offset_std > 0:
-        # One offset per block, the partial last block (when block does not divide N)
-        # included.
-        nb = -(-N // w.block)
-        off = torch.randn((b, w.hkv, nb, d), generator=g, dtype=torch.float32)
-        k32 += (w.key_offset_std * off).repeat_interleave(w.block, dim=2)[:, :, :N]
-    k = k32.to(torch.bfloat16)
-    del k32
+    with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as pool:
+        q = _draw_rows((b, w.hq, N, d), seed, 0, pool)
+        row_fn = None
+        if w.key_offset_std > 0:
+            # One offset per block, the partial last block (when block does not divide
+            # N) included; row r of the [b*hkv*N, d] view sits at position r mod N of
+            # plane r div N.
+            nb = -(-N // w.block)
+            g = torch.Generator("cpu").manual_seed(_seed(seed, 3, 0))
+            off = (w.key_offset_std *
+                   torch.randn((b * w.hkv * nb, d), generator=g, dtype=torch.float32))
+
+            def row_fn(r0, r1, x):
+                r = torch.arange(r0, r1, dtype=torch.int64)
+                x += off[(r // N) * nb + (r % N) // w.block]
+        k = _draw_rows((b, w.hkv, N, d), seed, 1, pool, row_fn)
+        v = _draw_rows((b, w.hkv, N, d), seed, 2, pool)
     return q.to(device), k.to(device), v.to(device)
-
-
-def _randn_bf16(shape, g, chunk: int = 1 << 26):
-    """N(0,1) float32 draws cast to bf16, drawn in row chunks to bound host memory."""
-    out = torch.empty(shape, dtype=torch.bfloat16)
-    flat = out.view(-1)
-    total = flat.numel()
-    for s in range(0, total, chunk):
-        e = min(total, s + chunk)
-        flat[s:e] = torch.randn(e - s, generator=g, dtype=torch.float32).to(torch.bfloat16)
-    return out
 
 
 def small_moba(batch=1, hq=2, hkv=1, seqlen=1024, d=64, block=128, topk=3, window=0,
