@@ -46,7 +46,10 @@ def _load():
         lib.orc_select_topk.argtypes = [P, I, I, I, I, I, P, I, P, P]
         lib.orc_attention.argtypes = [P, P, P, I, I, I, I, I, I, I, I, P, I,
                                       ctypes.c_double, P, I, P, P]
-        for f in (lib.orc_pool_keys, lib.orc_gate_scores, lib.orc_select_topk, lib.orc_attention):
+        lib.orc_attention_bwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, I, ctypes.c_double,
+                                          P, I, P, P, I, P, P]
+        for f in (lib.orc_pool_keys, lib.orc_gate_scores, lib.orc_select_topk, lib.orc_attention,
+                  lib.orc_attention_bwd):
             f.restype = I
         _lib = lib
     return _lib

@@ -28,7 +28,7 @@ import math
 
 import numpy as np
 
-from . import bf16_to_f64, n_blocks
+from . import _check, _load, _ptr, bf16_bits, bf16_to_f64, n_blocks
 
 
 def key_set(i: int, idx_row, block: int, window: int) -> np.ndarray:
@@ -78,3 +78,30 @@ def moba_backward(q, k, v, idx: np.ndarray, dout: np.ndarray, *, block: int, win
                 dk[bb, hk, J] += scale * np.outer(dz, qd[bb, h, i])
                 dv[bb, hk, J] += np.outer(p, do[bb, h, i])
     return out, lse, dq, dk, dv
+
+
+def moba_backward_sampled(q, k, v, idx: np.ndarray, dout, *, block: int, rows, keys,
+                          window: int = 0, scale: float | None = None):
+    """The same gradients from the C oracle (``orc_attention_bwd``, float64, OpenMP) at
+    a sample: dQ at the row positions ``rows`` of every q-head, dK and dV at the key
+    positions ``keys`` of every KV head (each key's sums run over every row of its
+    group that attends it).  ``idx`` int32 [b, hq, N, topk] is the choice of every
+    row; q, k, v, dout bf16 tensors.  Returns (dq [b, hq, R, d], dk, dv [b, hkv, K, d])
+    in float64."""
+    qb, kb, vb, ob = bf16_bits(q), bf16_bits(k), bf16_bits(v), bf16_bits(dout)
+    b, hq, N, d = qb.shape
+    hkv = kb.shape[1]
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    topk = idx.shape[-1]
+    assert idx.shape == (b, hq, N, topk) and ob.shape == qb.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    kk = np.ascontiguousarray(np.asarray(keys, dtype=np.int32))
+    dq = np.empty((b, hq, len(r), d))
+    dk = np.empty((b, hkv, len(kk), d))
+    dv = np.empty((b, hkv, len(kk), d))
+    _check(_load().orc_attention_bwd(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(ob), b, hq, hkv, N, d,
+                                     block, topk, _ptr(idx), window, float(scale), _ptr(r), len(r),
+                                     _ptr(dq), _ptr(kk), len(kk), _ptr(dk), _ptr(dv)))
+    return dq, dk, dv

@@ -336,3 +336,259 @@ int orc_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, int b
     if (bad & 2) return ORC_ERR_IDX;
     return ORC_OK;
 }
+
+/*
+ * Key set J_i of row i under MoBA with block choice `ir` (topk entries, -1 padded)
+ * and an optional causal window, in ascending key order: the keys j <= i whose block
+ * is listed, and (window > 0) the keys with 0 <= i - j < window.  `sel` is scratch of
+ * n bytes.  Returns the key count, or -1 when an entry names a block the row may not
+ * see.
+ */
+static int moba_keys(int i, int B, int n, int topk, const int32_t *ir, int window, char *sel,
+                     int32_t *key)
+{
+    const int c = i / B;
+    memset(sel, 0, (size_t)n);
+    for (int t = 0; t < topk; ++t) {
+        if (ir[t] == -1) continue;
+        if (ir[t] < 0 || ir[t] > c) return -1;
+        sel[ir[t]] = 1;
+    }
+    int nk = 0;
+    for (int blk = 0; blk <= c; ++blk) {
+        const int lo = blk * B;
+        const int hi = (blk * B + B - 1 < i) ? blk * B + B - 1 : i;
+        int from = lo;
+        if (!sel[blk]) {
+            if (window <= 0) continue;
+            from = (i - window + 1 > lo) ? i - window + 1 : lo;
+        }
+        for (int j = from; j <= hi; ++j) key[nk++] = j;
+    }
+    return nk;
+}
+
+/*
+ * Gradients of MoBA attention for a fixed block choice.  [MoBA] §"MoBA와 전체 어텐션의
+ * 하이브리드" trains models whose layers are MoBA attention, so gradients flow through
+ * it; the gate is a parameter-free top-k and passes no gradient, so for the choice in
+ * idx the layer is plain softmax attention over each row's key set J_i (§"MoBA의 구현",
+ * unioned with the optional causal window).  With z_ij = scale q_i . k_j on J_i,
+ * p_ij = exp(z_ij - lse_i), o_i = sum_j p_ij v_j and the upstream gradient dO:
+ *     D_i = dO_i . o_i,   dp_ij = dO_i . v_j,   dz_ij = p_ij (dp_ij - D_i)
+ *     dQ_i = scale sum_j dz_ij k_j
+ *     dK_j = scale sum_i dz_ij q_i,   dV_j = sum_i p_ij dO_i
+ * where a KV head's dK and dV sum over the q-heads that read it (GQA).
+ * dQ is computed at the listed rows (every q-head), dK and dV at the listed key
+ * positions (every KV head): a key's sums run over every row of every q-head of its
+ * group whose key set holds it, each with that row's own lse_i and D_i.
+ *   q, dout : bf16 [b, hq, N, d];  k, v : bf16 [b, hkv, N, d]
+ *   idx     : int32 [b, hq, N, topk], the choice of EVERY row
+ *   rows    : R row positions -> dq double [b, hq, R, d]
+ *   keys    : K key positions -> dk, dv double [b, hkv, K, d]
+ */
+int orc_attention_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                      const uint16_t *dout, int b, int hq, int hkv, int N, int d, int B, int topk,
+                      const int32_t *idx, int window, double scale, const int32_t *rows, int R,
+                      double *dq, const int32_t *keys, int K, double *dk, double *dv)
+{
+    if (b < 1 || hq < 1 || hkv < 1 || hq % hkv != 0 || N < 1 || d < 1 || B < 1 || topk < 1 ||
+        !idx || R < 0 || K < 0)
+        return ORC_ERR_ARG;
+    for (int r = 0; r < R; ++r)
+        if (rows[r] < 0 || rows[r] >= N) return ORC_ERR_ARG;
+    for (int e = 0; e < K; ++e)
+        if (keys[e] < 0 || keys[e] >= N) return ORC_ERR_ARG;
+    const int G = hq / hkv;
+    const int n = n_blocks(N, B);
+    const long nrows_all = (long)b * hq * N;
+    /* Row statistics (lse_i, D_i) of the rows a listed key's sums need. */
+    char *need = (char *)calloc((size_t)nrows_all, 1);
+    double *lse = (double *)malloc(sizeof(double) * (size_t)nrows_all);
+    double *D = (double *)malloc(sizeof(double) * (size_t)nrows_all);
+    if (!need || !lse || !D) {
+        free(need);
+        free(lse);
+        free(D);
+        return ORC_ERR_MEM;
+    }
+    int bad = 0;
+    /* A row needs its statistics when it is a listed row or when its key set holds a
+       listed key of its KV head. */
+#pragma omp parallel for schedule(dynamic, 64)
+    for (long u = 0; u < nrows_all; ++u) {
+        const long bh = u / N;
+        const int bb = (int)(bh / hq), h = (int)(bh % hq), i = (int)(u % N);
+        const int32_t *ir = idx + u * topk;
+        char hit = 0;
+        for (int e = 0; e < K && !hit; ++e) {
+            const int j = keys[e];
+            if (j > i) continue;
+            const int cj = j / B;
+            if (window > 0 && i - j < window) hit = 1;
+            for (int t = 0; t < topk && !hit; ++t) hit = (ir[t] == cj);
+        }
+        (void)bb;
+        (void)h;
+        need[u] = hit;
+    }
+    for (long bh = 0; bh < (long)b * hq; ++bh)
+        for (int r = 0; r < R; ++r) need[bh * N + rows[r]] = 1;
+
+#pragma omp parallel reduction(| : bad)
+    {
+        double *z = (double *)malloc(sizeof(double) * (size_t)N);
+        int32_t *key = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+        char *sel = (char *)malloc((size_t)n);
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+        double *od = (double *)malloc(sizeof(double) * (size_t)d);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!z || !key || !sel || !qd || !od || !acc) {
+            bad |= 4;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long u = 0; u < nrows_all; ++u) {
+                if (!need[u]) continue;
+                const long bh = u / N;
+                const int bb = (int)(bh / hq), h = (int)(bh % hq), i = (int)(u % N);
+                const int nk = moba_keys(i, B, n, topk, idx + u * topk, window, sel, key);
+                if (nk < 0) {
+                    bad |= 2;
+                    continue;
+                }
+                const long kvh = (long)bb * hkv + h / G;
+                const uint16_t *kh = k + kvh * N * (long)d;
+                const uint16_t *vh = v + kvh * N * (long)d;
+                for (int t = 0; t < d; ++t) {
+                    qd[t] = bf16_to_double(q[u * d + t]);
+                    od[t] = bf16_to_double(dout[u * d + t]);
+                }
+                double m = -INFINITY;
+                for (int e = 0; e < nk; ++e) {
+                    const uint16_t *kj = kh + (long)key[e] * d;
+                    double dot = 0.0;
+                    for (int t = 0; t < d; ++t) dot += qd[t] * bf16_to_double(kj[t]);
+                    z[e] = scale * dot;
+                    if (z[e] > m) m = z[e];
+                }
+                double l = 0.0;
+                for (int t = 0; t < d; ++t) acc[t] = 0.0;
+                for (int e = 0; e < nk; ++e) {
+                    const double p = exp(z[e] - m);
+                    const uint16_t *vj = vh + (long)key[e] * d;
+                    l += p;
+                    for (int t = 0; t < d; ++t) acc[t] += p * bf16_to_double(vj[t]);
+                }
+                double Di = 0.0;
+                for (int t = 0; t < d; ++t) Di += od[t] * (acc[t] / l);
+                lse[u] = m + log(l);
+                D[u] = Di;
+            }
+        }
+        free(z);
+        free(key);
+        free(sel);
+        free(qd);
+        free(od);
+        free(acc);
+    }
+    if (bad) {
+        free(need);
+        free(lse);
+        free(D);
+        return (bad & 4) ? ORC_ERR_MEM : ORC_ERR_IDX;
+    }
+
+    /* dQ at the listed rows. */
+#pragma omp parallel reduction(| : bad)
+    {
+        int32_t *key = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+        char *sel = (char *)malloc((size_t)n);
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+        double *od = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!key || !sel || !qd || !od) {
+            bad |= 4;
+        } else {
+#pragma omp for schedule(dynamic, 4)
+            for (long w = 0; w < (long)b * hq * R; ++w) {
+                const long bh = w / R;
+                const int bb = (int)(bh / hq), h = (int)(bh % hq), i = rows[w % R];
+                const long u = bh * N + i;
+                const int nk = moba_keys(i, B, n, topk, idx + u * topk, window, sel, key);
+                const long kvh = (long)bb * hkv + h / G;
+                const uint16_t *kh = k + kvh * N * (long)d;
+                const uint16_t *vh = v + kvh * N * (long)d;
+                for (int t = 0; t < d; ++t) {
+                    qd[t] = bf16_to_double(q[u * d + t]);
+                    od[t] = bf16_to_double(dout[u * d + t]);
+                }
+                double *g = dq + w * d;
+                for (int t = 0; t < d; ++t) g[t] = 0.0;
+                for (int e = 0; e < nk; ++e) {
+                    const uint16_t *kj = kh + (long)key[e] * d;
+                    const uint16_t *vj = vh + (long)key[e] * d;
+                    double zq = 0.0, dp = 0.0;
+                    for (int t = 0; t < d; ++t) {
+                        zq += qd[t] * bf16_to_double(kj[t]);
+                        dp += od[t] * bf16_to_double(vj[t]);
+                    }
+                    const double p = exp(scale * zq - lse[u]);
+                    const double dz = p * (dp - D[u]);
+                    for (int t = 0; t < d; ++t) g[t] += scale * dz * bf16_to_double(kj[t]);
+                }
+            }
+        }
+        free(key);
+        free(sel);
+        free(qd);
+        free(od);
+    }
+
+    /* dK and dV at the listed keys: every row of the group whose key set holds it. */
+#pragma omp parallel reduction(| : bad)
+    {
+        char *sel = (char *)malloc((size_t)n);
+        if (!sel) {
+            bad |= 4;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long w = 0; w < (long)b * hkv * K; ++w) {
+                const long bk = w / K;
+                const int bb = (int)(bk / hkv), hk = (int)(bk % hkv), j = keys[w % K];
+                const int cj = j / B;
+                const uint16_t *kj = k + (bk * N + j) * (long)d;
+                const uint16_t *vj = v + (bk * N + j) * (long)d;
+                double *gk = dk + w * d, *gv = dv + w * d;
+                for (int t = 0; t < d; ++t) gk[t] = gv[t] = 0.0;
+                for (int g = 0; g < G; ++g) {
+                    const long bh = (long)bb * hq + (long)hk * G + g;
+                    for (int i = j; i < N; ++i) {
+                        const long u = bh * N + i;
+                        const int32_t *ir = idx + u * topk;
+                        int in = (window > 0 && i - j < window);
+                        for (int t = 0; t < topk && !in; ++t) in = (ir[t] == cj);
+                        if (!in) continue;
+                        const uint16_t *qi = q + u * d;
+                        const uint16_t *oi = dout + u * d;
+                        double zq = 0.0, dp = 0.0;
+                        for (int t = 0; t < d; ++t) {
+                            zq += bf16_to_double(qi[t]) * bf16_to_double(kj[t]);
+                            dp += bf16_to_double(oi[t]) * bf16_to_double(vj[t]);
+                        }
+                        const double p = exp(scale * zq - lse[u]);
+                        const double dz = p * (dp - D[u]);
+                        for (int t = 0; t < d; ++t) {
+                            gk[t] += scale * dz * bf16_to_double(qi[t]);
+                            gv[t] += p * bf16_to_double(oi[t]);
+                        }
+                    }
+                }
+            }
+        }
+        free(sel);
+    }
+    free(need);
+    free(lse);
+    free(D);
+    return (bad & 4) ? ORC_ERR_MEM : ORC_OK;
+}

@@ -80,3 +80,58 @@ def test_backward_matches_finite_differences():
             xm = [minus if a is arr else a for a in args]
             fd = (loss(*xp) - loss(*xm)) / (2 * eps)
             assert abs(fd - grad[pos]) <= 1e-6 * max(1.0, abs(fd)), (name, pos, fd, grad[pos])
+
+
+def _bf16(x):
+    return torch.as_tensor(x).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("b,hq,hkv,N,d,block,topk,window", [
+    (1, 2, 1, 96, 8, 16, 3, 0),
+    (2, 4, 2, 80, 8, 16, 2, 10),     # GQA, a window, a partial last block
+    (1, 1, 1, 64, 4, 8, 20, 0),      # k >= n: dense causal
+    (1, 4, 1, 130, 16, 32, 2, 0),    # G = 4, N not a multiple of the block
+])
+def test_sampled_backward_equals_the_row_by_row_oracle(b, hq, hkv, N, d, block, topk, window):
+    """The C oracle's sampled gradients (dQ at listed rows, dK / dV at listed keys, each
+    key summed over every row of its group that attends it) equal the row-by-row
+    numpy oracle, which autograd and finite differences pin, at every row and key."""
+    q, k, v, _ = _inputs(b, hq, hkv, N, d, seed=3 * N + hq)
+    do = _bf16(torch.randn(b, hq, N, d, generator=torch.Generator().manual_seed(N)))
+    idx = oracle.moba(q, k, v, block=block, topk=topk, window=window)["idx"]
+    _, _, dq, dk, dv = backward.moba_backward(q, k, v, idx, oracle.bf16_to_f64(do), block=block,
+                                              window=window)
+    allr = np.arange(N, dtype=np.int32)
+    sq, sk, sv = backward.moba_backward_sampled(q, k, v, idx, do, block=block, rows=allr,
+                                                keys=allr, window=window)
+    for got, want in ((sq, dq), (sk, dk), (sv, dv)):
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-10)
+    # A sample is the matching slice of the whole.
+    rows, keys = np.array([N - 1, 0, N // 2], dtype=np.int32), np.array([3, N - 2], dtype=np.int32)
+    tq, tk, tv = backward.moba_backward_sampled(q, k, v, idx, do, block=block, rows=rows, keys=keys,
+                                                window=window)
+    np.testing.assert_allclose(tq, dq[:, :, rows], rtol=0, atol=1e-10)
+    np.testing.assert_allclose(tk, dk[:, :, keys], rtol=0, atol=1e-10)
+    np.testing.assert_allclose(tv, dv[:, :, keys], rtol=0, atol=1e-10)
+
+
+def test_backward_sum_identities():
+    """Identities of softmax attention that hold for any key sets, per KV head:
+    sum_j dV_j = sum over its q-heads' rows of dO_i (the weights of a row sum to one);
+    sum_j dK_j = 0 (the dz of a row sum to zero); sum_j k_j . dK_j = sum_i q_i . dQ_i
+    (both are sum_ij dz_ij z_ij); sum_j v_j . dV_j = sum_i dO_i . o_i."""
+    b, hq, hkv, N, d, block, topk, window = 1, 4, 2, 72, 8, 16, 2, 12
+    q, k, v, do = _inputs(b, hq, hkv, N, d, seed=11)
+    idx = oracle.moba(q, k, v, block=block, topk=topk, window=window)["idx"]
+    out, _, dq, dk, dv = backward.moba_backward(q, k, v, idx, do.numpy(), block=block, window=window)
+    qd, kd, vd = (oracle.bf16_to_f64(t) for t in (q, k, v))
+    G = hq // hkv
+    dod = do.numpy()
+    for hk in range(hkv):
+        hs = slice(hk * G, (hk + 1) * G)
+        np.testing.assert_allclose(dv[0, hk].sum(0), dod[0, hs].sum((0, 1)), atol=1e-10)
+        np.testing.assert_allclose(dk[0, hk].sum(0), 0.0, atol=1e-10)
+        np.testing.assert_allclose((kd[0, hk] * dk[0, hk]).sum(), (qd[0, hs] * dq[0, hs]).sum(),
+                                   atol=1e-10)
+        np.testing.assert_allclose((vd[0, hk] * dv[0, hk]).sum(), (dod[0, hs] * out[0, hs]).sum(),
+                                   atol=1e-10)

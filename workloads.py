@@ -6,7 +6,7 @@ here, so they see the same bf16 values.
 
 Recipe: every tensor is viewed as rows of d values ([b, h, N, d] flattened to
 [b*h*N, d]) and split into chunks of 2^17 rows; chunk c of stream s (0: q, 1: k, 2: v,
-3: the key offsets) is drawn as float32 N(0, 1) from its own
+3: the key offsets, 4: the upstream gradient of the backward) is drawn as float32 N(0, 1) from its own
 ``torch.Generator('cpu').manual_seed(seed * 2^32 + s * 2^24 + c)``, so the chunks are
 independent and are drawn in parallel threads.  q is [b, hq, N, d], k and v are
 [b, hkv, N, d].  For the MoBA workloads one offset vector per (batch, kv-head, block),
@@ -143,6 +143,16 @@ def make_inputs(w: Workload, seed: int = 0, device: str = "cpu"):
         k = _draw_rows((b, w.hkv, N, d), seed, 1, pool, row_fn)
         v = _draw_rows((b, w.hkv, N, d), seed, 2, pool)
     return q.to(device), k.to(device), v.to(device)
+
+
+def make_grad(w: Workload, seed: int = 0, device: str = "cpu"):
+    """An upstream gradient dO for the backward, [b, hq, nq, d] bf16: float32 N(0, 1)
+    draws of stream 4 (chunked like the inputs), cast to bf16."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as pool:
+        g = _draw_rows((w.batch, w.hq, w.nq, w.d), seed, 4, pool)
+    return g.to(device)
 
 
 def small_moba(batch=1, hq=2, hkv=1, seqlen=1024, d=64, block=128, topk=3, window=0,
