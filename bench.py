@@ -340,9 +340,10 @@ def launches_per_step(w: workloads.Workload) -> int:
     return sel + layout_chunks(w) * (3 if w.topk > 1 else 1)
 
 
-def measure(w, steps, warmup, rank, world, device, seed, full=True, cpu=True, comparators=True):
+def measure(w, steps, warmup, rank, world, device, seed, full=True, cpu_leg=True,
+            comparators=True):
     """Times `steps` steps of workload w (after `warmup` untimed ones) and returns the
-    result dict.  full: also the end-to-end host-buffer leg; cpu: the CPU oracle
+    result dict.  full: also the end-to-end host-buffer leg; cpu_leg: the CPU oracle
     baseline (rank 0, one GPU); comparators: the dense comparators (rank 0)."""
     import block_sparse_long_prefill_b200 as moba
     from block_sparse_long_prefill_b200 import MobaPrefill
@@ -505,6 +506,14 @@ def measure(w, steps, warmup, rank, world, device, seed, full=True, cpu=True, co
                               "gbs": round(sel_bytes / (sel_ms * 1e-3) / 1e9, 1),
                               "frac_hbm": round(sel_bytes / (sel_ms * 1e-3) / 1e9 / hbm, 4)}
 
+    # ---------------------------------------------------------------- backward
+    if (w.kind == "moba" and w.gate == "mean" and w.window == 0 and not w.q_off
+            and w.d in (64, 128)):
+        bws_bytes = moba.bwd_workspace_size(w.batch, w.hq, w.hkv, w.nq, w.d, w.block, w.topk)
+        if bws_bytes <= (16 << 30):
+            extra["backward"] = time_backward(w, qd, kd, vd, runner, flush, stream, steps,
+                                              warmup, flops / (4.0 * w.d), tc_peak, seed + rank)
+
     # ---------------------------------------------------------------- e2e (host buffers)
     e2e = None
     if full:
@@ -558,7 +567,7 @@ def measure(w, steps, warmup, rank, world, device, seed, full=True, cpu=True, co
         comps = dense_comparators(w, qd, kd, vd, flush, stream, ms, steps, tc_peak)
 
     cpu = None
-    if full and cpu and rank == 0 and world == 1:
+    if full and cpu_leg and rank == 0 and world == 1:
         cpu = cpu_baseline(w, seed, target_s=12.0, tensors=None if w.q_off else (qh, kh, vh))
 
     clocks = clk.summary()
@@ -575,6 +584,44 @@ def measure(w, steps, warmup, rank, world, device, seed, full=True, cpu=True, co
     line.update(extra)
     line.update(comps)
     return line
+
+
+def time_backward(w, qd, kd, vd, runner, flush, stream, steps, warmup, pairs, tc_peak, seed):
+    """moba_attn_bwd over the forward's choices: one call (prep, dQ, dK/dV and dQ merge
+    kernels) timed with CUDA events, L2 flushed between calls.  Algorithmic work is
+    10 d FLOPs per attended pair (the five products of softmax attention's backward);
+    the kernels execute 14 d (the dQ pass recomputes S and dP)."""
+    import block_sparse_long_prefill_b200 as moba
+    do = workloads.make_grad(w, seed).to(qd.device)
+    bws = torch.empty(moba.bwd_workspace_size(w.batch, w.hq, w.hkv, w.nq, w.d, w.block, w.topk),
+                      dtype=torch.uint8, device=qd.device)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+
+    def call():
+        moba.moba_attn_bwd(qd, kd, vd, runner.out, runner.lse, do, runner.idx, w.block, w.topk,
+                           runner.workspace, dq=dq, dk=dk, dv=dv, bwd_workspace=bws)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(steps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b_ = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        tot += a.elapsed_time(b_)
+    assert moba.device_status() == 0
+    ms = tot / steps
+    flops = 10.0 * w.d * pairs
+    del do, bws, dq, dk, dv
+    return {"ms": round(ms, 4), "flops": flops, "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+            "frac": round(flops / (ms * 1e-3) / 1e12 / tc_peak, 4),
+            "executed_flops": 14.0 * w.d * pairs, "launches": 4,
+            "work": "10*d FLOPs per attended pair (dQ, dK, dV of softmax attention)"}
 
 
 def dense_comparators(w, qd, kd, vd, flush, stream, moba_ms, steps, tc_peak):
@@ -634,7 +681,7 @@ def dense_comparators(w, qd, kd, vd, flush, stream, moba_ms, steps, tc_peak):
 def run_ours(args, rank, world, device):
     w = workloads.WORKLOADS[args.workload]
     main = measure(w, args.steps, args.warmup, rank, world, device, args.seed,
-                   full=not args.no_e2e, cpu=not args.no_cpu_baseline,
+                   full=not args.no_e2e, cpu_leg=not args.no_cpu_baseline,
                    comparators=not args.no_comparators)
     line = {"metric": METRIC, "value": main.pop("value"), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": main.pop("ms_per_step"),

@@ -33,8 +33,9 @@ ABI_FUNCTIONS = ("moba_workspace_size", "moba_pool_keys", "moba_select_topk", "m
                  "swa_attn_fwd", "moba_workspace_size_chunk", "moba_select_topk_chunk",
                  "moba_attn_fwd_chunk", "swa_attn_fwd_chunk", "moba_select_static",
                  "moba_pool_keys_minmax", "moba_select_topk_minmax",
-                 "moba_prefill_static",
-                 "moba_device_status", "moba_set_pass_events", "moba_status_string")
+                 "moba_prefill_static", "moba_bwd_workspace_size", "moba_attn_bwd",
+                 "moba_device_status", "moba_debug_set_wait_limit_us",
+                 "moba_debug_fault_next_launch", "moba_set_pass_events", "moba_status_string")
 
 
 class MobaError(RuntimeError):
@@ -69,7 +70,12 @@ def _load():
     lib.moba_pool_keys_minmax.argtypes = [T, I, I, I, I, I, P, P]
     lib.moba_select_topk_minmax.argtypes = [T, P, I, I, I, I, I, I, I, I, P, P, S, P]
     lib.moba_prefill_static.argtypes = [T, T, T, I, I, I, I, I, I, I, I, ctypes.c_float, T, P, P]
+    lib.moba_bwd_workspace_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(S)]
+    lib.moba_attn_bwd.argtypes = [T, T, T, T, T, P, P, P, S, I, I, I, I, I, I, I, I,
+                                  ctypes.c_float, T, T, T, P, S, P]
     lib.moba_device_status.argtypes = []
+    lib.moba_debug_set_wait_limit_us.argtypes = [I]
+    lib.moba_debug_fault_next_launch.argtypes = [I]
     lib.moba_set_pass_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), I]
     lib.moba_status_string.argtypes = [I]
     lib.moba_status_string.restype = ctypes.c_char_p
@@ -353,6 +359,46 @@ def moba_prefill_static(q, k, v, block: int, topk: int, window: int = 0, scale: 
     return out, lse
 
 
+def bwd_workspace_size(batch, hq, hkv, N, d, block, topk) -> int:
+    out = ctypes.c_size_t(0)
+    _check("moba_bwd_workspace_size",
+           _lib.moba_bwd_workspace_size(batch, hq, hkv, N, d, block, topk, ctypes.byref(out)))
+    return out.value
+
+
+def moba_attn_bwd(q, k, v, out, lse, dout, idx, block: int, topk: int, workspace: torch.Tensor,
+                  scale: float = 0.0, dq=None, dk=None, dv=None, bwd_workspace=None, stream=None):
+    """[MoBA] §MoBA와 전체 어텐션의 하이브리드 (training through MoBA layers): gradients of
+    MoBA attention for the block choice ``idx`` of the forward.  ``workspace`` is the
+    one moba_select_topk filled (its dispatch lists are read).  Returns (dq, dk, dv)."""
+    b, hq, N, d = q.shape
+    hkv = k.shape[1]
+    dev = _device("moba_attn_bwd", ("q", q, _BF16, False, None), ("k", k, _BF16, False, None),
+                  ("v", v, _BF16, False, tuple(k.shape)), ("out", out, _BF16, False, tuple(q.shape)),
+                  ("dout", dout, _BF16, False, tuple(q.shape)),
+                  ("lse", lse, _F32, True, (b, hq, N)), ("idx", idx, _I32, True, (b, hq, N, topk)),
+                  ("workspace", workspace, None, True, None),
+                  ("dq", dq, _BF16, False, tuple(q.shape)), ("dk", dk, _BF16, False, tuple(k.shape)),
+                  ("dv", dv, _BF16, False, tuple(k.shape)),
+                  ("bwd_workspace", bwd_workspace, None, True, None))
+    with torch.cuda.device(dev):
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
+        if bwd_workspace is None:
+            bwd_workspace = torch.empty(bwd_workspace_size(b, hq, hkv, N, d, block, topk),
+                                        dtype=torch.uint8, device=dev)
+        _check("moba_attn_bwd",
+               _lib.moba_attn_bwd(_t(q), _t(k), _t(v), _t(out), _t(dout), lse.data_ptr(),
+                                  idx.data_ptr(), workspace.data_ptr(),
+                                  workspace.numel() * workspace.element_size(), b, hq, hkv, N, d,
+                                  block, topk, 0, float(scale), _t(dq), _t(dk), _t(dv),
+                                  bwd_workspace.data_ptr(),
+                                  bwd_workspace.numel() * bwd_workspace.element_size(),
+                                  _stream(stream)))
+    return dq, dk, dv
+
+
 def set_pass_events(events) -> None:
     """Diagnostics: moba_attn_fwd records these torch.cuda.Event objects before its
     first kernel and after each pass (past blocks, own block, merge) of its first query
@@ -364,6 +410,17 @@ def set_pass_events(events) -> None:
             e.record()
     arr = (ctypes.c_void_p * max(1, len(events)))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _check("moba_set_pass_events", _lib.moba_set_pass_events(arr, len(events)))
+
+
+def debug_set_wait_limit_us(microseconds: int) -> None:
+    """Test hook: kernel waits give up after this many microseconds (0: the default)."""
+    _check("moba_debug_set_wait_limit_us", _lib.moba_debug_set_wait_limit_us(int(microseconds)))
+
+
+def debug_fault_next_launch(kind: int = 1) -> None:
+    """Test hook: the next attention launch leaves one load undone so that a bounded wait
+    runs out (MOBA_ERR_DEVICE from device_status()); 0 clears a pending request."""
+    _check("moba_debug_fault_next_launch", _lib.moba_debug_fault_next_launch(int(kind)))
 
 
 def device_status() -> int:
@@ -483,8 +540,8 @@ def moba_prefill_varlen(q, k, v, cu_seqlens, block: int, topk: int, window: int 
     axis (FlashAttention's varlen layout): q [total, hq, d], k, v [total, hkv, d] bf16,
     ``cu_seqlens`` the prefix offsets (batch + 1 ints from 0 to total; a list or a CPU
     tensor).  Sequence s is positions cu_seqlens[s] .. cu_seqlens[s+1] - 1 and is its own
-    prefill: its own blocks, its own causal order.  A length must be a multiple of 128
-    (not necessarily of ``block``: its last block may be partial).  Each sequence goes
+    prefill: its own blocks, its own causal order.  Any lengths (its last block may be
+    partial).  Each sequence goes
     through the library's calls as a [1, heads, N_s, d] strided view of the packed
     tensors (no copy); the pooled keys, block choices and workspace are sized for the
     longest sequence and reused in stream order.  Returns (out [total, hq, d] bf16, lse

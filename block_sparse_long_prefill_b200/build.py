@@ -9,7 +9,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoba.so")
-SOURCES = ["api.cu", "select.cu", "gate.cu", "attn.cu", "merge.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "select.cu", "gate.cu", "attn.cu", "merge.cu", "noalloc.cu", "bwd.cu"]
 HEADERS = ["common.cuh", "params.h", "lists.cuh"]
 
 NVCC_FLAGS = [

@@ -14,7 +14,7 @@
 
 namespace moba {
 
-__device__ int g_device_status[2] = {MOBA_OK, 0};
+__device__ int g_device_status[kStatusWords] = {MOBA_OK, 0, 0, 0};
 
 cudaError_t launch_pool(const uint16_t *k, int64_t sb, int64_t sh, int64_t sn, int batch, int hkv,
                         int N, int d, int block, float *kbar, uint16_t *split, cudaStream_t st);
@@ -34,6 +34,7 @@ cudaError_t launch_attn(const CUtensorMap *maps, const AttnParams &p, int mode, 
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t st);
 int query_major_units(int batch, int hq, int hkv, int block, int is_moba, int row_begin,
                       int row_end);
+cudaError_t launch_bwd(const CUtensorMap *maps, const BwdParams &p, int nsm, cudaStream_t st);
 
 namespace {
 
@@ -66,10 +67,11 @@ int check_attn_dim(int d) { return (d == 64 || d == 80 || d == 128) ? MOBA_OK : 
 int check_moba_shape(int batch, int hq, int hkv, int N, int d, int block, int topk, int q_off = 0) {
   if (batch < 1 || hq < 1 || hkv < 1 || N < 1 || block < 1) return MOBA_ERR_SHAPE;
   if (hq % hkv) return MOBA_ERR_SHAPE;
-  // 128-row query tiles: N, q_off and block multiples of 128 (block need not divide the
-  // key count: the last block is then partial).
-  if (block % kTileRows || N % kTileRows) return MOBA_ERR_SHAPE;
-  if (q_off < 0 || q_off % kTileRows || (long long)q_off + N >= (1ll << 31)) return MOBA_ERR_SHAPE;
+  // Any N and q_off (the last query tile may be partial and a tile may span two blocks);
+  // block a multiple of the kernels' 128-key chunks, so that a chunk never holds keys of
+  // two blocks (block need not divide the key count: the last block is then partial).
+  if (block % kTileKeys) return MOBA_ERR_SHAPE;
+  if (q_off < 0 || (long long)q_off + N >= (1ll << 31)) return MOBA_ERR_SHAPE;
   if (topk < 1 || topk > 32) return MOBA_ERR_ARG;
   const long long G = hq / hkv;
   if ((long long)N * G * (topk - 1) >= (1ll << 31)) return MOBA_ERR_SHAPE;
@@ -297,7 +299,7 @@ static int select_topk_impl(moba_tensor q, const void *kbar_split, int batch, in
     gp.batch = batch; gp.hq = hq; gp.hkv = hkv; gp.N = N; gp.d = d; gp.block = block;
     gp.topk = topk; gp.nblk = w.nblk; gp.G = w.G; gp.chunk_rows = w.chunk_rows;
     gp.q_off = q_off;
-    const long long ntiles = (long long)batch * hkv * (N / kTileRows) * w.G;
+    const long long ntiles = (long long)batch * hkv * ((N + kTileRows - 1) / kTileRows) * w.G;
     const int grid = (int)(ntiles < nsm ? ntiles : nsm);
     if ((rc = launch_status(launch_gate_tc(maps, gp, grid, st)))) return rc;
   } else {
@@ -519,10 +521,9 @@ int swa_attn_fwd_chunk(moba_tensor q, moba_tensor k, moba_tensor v, int batch, i
                        int N, int Nk, int d, int window, float scale, moba_tensor out, float *lse,
                        void *stream) {
   if (batch < 1 || hq < 1 || hkv < 1 || N < 1 || hq % hkv) return MOBA_ERR_SHAPE;
-  // Query row i sits at key position Nk - N + i; with a chunk (Nk > N) the offset must
-  // be a multiple of 128 (query tiles).
+  // Query row i sits at key position Nk - N + i (any offset).
   const int q_off = Nk - N;
-  if (q_off < 0 || q_off % kTileRows || (long long)Nk >= (1ll << 31)) return MOBA_ERR_SHAPE;
+  if (q_off < 0 || (long long)Nk >= (1ll << 31)) return MOBA_ERR_SHAPE;
   if (window < 1) return MOBA_ERR_ARG;
   int rc = check_attn_dim(d);
   if (rc) return rc;
@@ -563,6 +564,73 @@ int swa_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq,
   return swa_attn_fwd_chunk(q, k, v, batch, hq, hkv, N, N, d, window, scale, out, lse, stream);
 }
 
+int moba_bwd_workspace_size(int batch, int hq, int hkv, int N, int d, int block, int topk,
+                            size_t *bytes) {
+  if (!bytes) return MOBA_ERR_ARG;
+  const int rc = check_moba_shape(batch, hq, hkv, N, d, block, topk, 0);
+  if (rc) return rc;
+  if (d != 64 && d != 128) return MOBA_ERR_DIM;
+  *bytes = bwd_workspace_bytes(batch, hq, N, d, topk, nullptr);
+  return MOBA_OK;
+}
+
+int moba_attn_bwd(moba_tensor q, moba_tensor k, moba_tensor v, moba_tensor out, moba_tensor dout,
+                  const float *lse, const int32_t *idx, const void *workspace,
+                  size_t workspace_bytes, int batch, int hq, int hkv, int N, int d, int block,
+                  int topk, int window, float scale, moba_tensor dq, moba_tensor dk,
+                  moba_tensor dv, void *bwd_workspace, size_t bwd_workspace_bytes_, void *stream) {
+  int rc = check_moba_shape(batch, hq, hkv, N, d, block, topk, 0);
+  if (rc) return rc;
+  if (d != 64 && d != 128) return MOBA_ERR_DIM;
+  if (window != 0) return MOBA_ERR_ARG;
+  const moba_tensor ts[8] = {q, k, v, out, dout, dq, dk, dv};
+  for (const moba_tensor &t : ts)
+    if ((rc = check_tensor(t))) return rc;
+  if (!lse || !idx) return MOBA_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(idx) & 3u))
+    return MOBA_ERR_ALIGN;
+  const WorkspaceLayout w = make_layout(batch, hq, hkv, N, d, block, topk, 0);
+  if (!workspace || workspace_bytes < w.total) return MOBA_ERR_WORKSPACE;
+  size_t off_dqp = 0;
+  const size_t need = bwd_workspace_bytes(batch, hq, N, d, topk, &off_dqp);
+  if (!bwd_workspace || bwd_workspace_bytes_ < need) return MOBA_ERR_WORKSPACE;
+  if (!aligned16(workspace) || !aligned16(bwd_workspace)) return MOBA_ERR_ALIGN;
+  int nsm = 0;
+  if ((rc = check_device(&nsm))) return rc;
+  CUtensorMap maps[6];
+  if ((rc = make_attn_maps(maps, q, k, v, batch, hq, hkv, N, N, d))) return rc;
+  const CUtensorMap kv[2] = {maps[2], maps[4]};
+  const char *ws = static_cast<const char *>(workspace);
+  char *bws = static_cast<char *>(bwd_workspace);
+  BwdParams p{};
+  if ((rc = status_words(&p.status))) return rc;
+  p.q = static_cast<const uint16_t *>(q.ptr);
+  p.q_sb = q.sb; p.q_sh = q.sh; p.q_sn = q.sn;
+  p.out = static_cast<const uint16_t *>(out.ptr);
+  p.o_sb = out.sb; p.o_sh = out.sh; p.o_sn = out.sn;
+  p.dout = static_cast<const uint16_t *>(dout.ptr);
+  p.do_sb = dout.sb; p.do_sh = dout.sh; p.do_sn = dout.sn;
+  p.lse = lse;
+  p.dq = static_cast<uint16_t *>(dq.ptr);
+  p.dq_sb = dq.sb; p.dq_sh = dq.sh; p.dq_sn = dq.sn;
+  p.dk = static_cast<uint16_t *>(dk.ptr);
+  p.dk_sb = dk.sb; p.dk_sh = dk.sh; p.dk_sn = dk.sn;
+  p.dv = static_cast<uint16_t *>(dv.ptr);
+  p.dv_sb = dv.sb; p.dv_sh = dv.sh; p.dv_sn = dv.sn;
+  p.rowstat = reinterpret_cast<float2 *>(bws);
+  p.dqp = reinterpret_cast<float *>(bws + off_dqp);
+  p.batch = batch; p.hq = hq; p.hkv = hkv; p.N = N; p.d = d; p.block = block; p.topk = topk;
+  p.npast = topk - 1; p.nblk = w.nblk; p.G = w.G; p.nchunks = w.nchunks; p.nlists = w.nlists;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+  p.scale = sc;
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.entries = reinterpret_cast<const uint32_t *>(ws + w.off_entries);
+  p.tiles = reinterpret_cast<const int4 *>(ws + w.off_tiles);
+  p.tileoff = reinterpret_cast<const int *>(ws + w.off_tileoff);
+  p.listoff = reinterpret_cast<const int *>(ws + w.off_listoff);
+  return launch_status(launch_bwd(kv, p, nsm, static_cast<cudaStream_t>(stream)));
+}
+
 int moba_device_status(void) {
   int v[2] = {MOBA_OK, 0};
   if (cudaDeviceSynchronize() != cudaSuccess) return MOBA_ERR_LAUNCH;
@@ -572,10 +640,26 @@ int moba_device_status(void) {
   return v[0];
 }
 
+int moba_debug_set_wait_limit_us(int microseconds) {
+  if (microseconds < 0) return MOBA_ERR_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOBA_ERR_LAUNCH;
+  if (cudaMemcpyToSymbol(g_device_status, &microseconds, sizeof(int), 2 * sizeof(int)) != cudaSuccess)
+    return MOBA_ERR_LAUNCH;
+  return MOBA_OK;
+}
+
+int moba_debug_fault_next_launch(int kind) {
+  if (kind < 0 || kind > 1) return MOBA_ERR_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOBA_ERR_LAUNCH;
+  if (cudaMemcpyToSymbol(g_device_status, &kind, sizeof(int), 3 * sizeof(int)) != cudaSuccess)
+    return MOBA_ERR_LAUNCH;
+  return MOBA_OK;
+}
+
 const char *moba_status_string(int status) {
   switch (status) {
     case MOBA_OK: return "ok";
-    case MOBA_ERR_SHAPE: return "unsupported shape (N % 128, hq % hkv, block % 128, size limits)";
+    case MOBA_ERR_SHAPE: return "unsupported shape (hq % hkv, block % 128, size limits)";
     case MOBA_ERR_DIM: return "unsupported head dimension";
     case MOBA_ERR_ALIGN: return "pointer or stride not 16-byte aligned";
     case MOBA_ERR_ARG: return "invalid argument";

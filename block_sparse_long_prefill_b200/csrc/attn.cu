@@ -87,7 +87,8 @@ struct Tile {
   int i0;      // query-major: first query row (at key position q_off + i0)
   int rows;    // valid rows (0: the stream is idle in this unit)
   int ent0;    // gathered: first list entry
-  int cB;      // query-major MoBA: first key (position) of the own block
+  int cB;      // query-major MoBA: first key (position) of the own block of the tile's
+               // first row (the tile's later rows may sit in the next block)
 };
 
 // A work unit: two tiles over one key-chunk sequence.
@@ -307,6 +308,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         uint32_t cnt = 0;
         uint32_t quse[2] = {0u, 0u};
         bool ok = true;
+        // Test hook (moba_debug_fault_next_launch): the V loader of CTA 0 of the launch
+        // that finds the one-shot flag set takes it and leaves its first V chunk unloaded,
+        // so that the MMA issuer's wait for it runs out and the launch ends through the
+        // bounded-wait path with MOBA_ERR_DEVICE.
+        bool skip_first = false;
+        if (!kside && blockIdx.x == 0 && atomicExch(&p.status[3], 0) == 1) skip_first = true;
         for (UnitIter<MODE> it(p, u_begin, u_end); ok && it.valid(); it.next()) {
           Unit w;
           it.get(p, w);
@@ -331,6 +338,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (!(ok = mbar_wait(&empty[st], ((cnt / C::ST) & 1) ^ 1, abort, p.status, site0 + 2))) break;
             const int key = w.key0 + m * kTileKeys;
             unsigned char *dst = sbase + off + st * C::TILE;
+            if (skip_first && cnt == 0) continue;   // nothing issued, nothing to drain
             mbar_arrive_expect_tx(&full[st], C::BYTES);
             tma_load_4d(dst, m0, &full[st], 0, key, w.hk, w.b);
             if (D != 64) tma_load_4d(dst + C::R0, m1, &full[st], 64, key, w.hk, w.b);
@@ -340,12 +348,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (*abort) {
           for (uint32_t u = (cnt > (uint32_t)C::ST ? cnt - C::ST : 0); u < cnt; ++u) {
             const unsigned long long t0 = global_timer_ns();
-            while (!mbar_try_wait(&full[u % C::ST], (u / C::ST) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+            while (!mbar_try_wait(&full[u % C::ST], (u / C::ST) & 1) && global_timer_ns() - t0 < wait_limit_ns(p.status)) {}
           }
           for (int x = 0; x < 2; ++x) {
             if (quse[x] == 0) continue;
             const unsigned long long t0 = global_timer_ns();
-            while (!mbar_try_wait(&bar.q_full[x], (quse[x] - 1) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+            while (!mbar_try_wait(&bar.q_full[x], (quse[x] - 1) & 1) && global_timer_ns() - t0 < wait_limit_ns(p.status)) {}
           }
         }
       }
@@ -424,7 +432,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // Every MMA issued so far completes before TMEM is released.
         umma_commit(&bar.mma_done);
         const unsigned long long t0 = global_timer_ns();
-        while (!mbar_try_wait(&bar.mma_done, 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+        while (!mbar_try_wait(&bar.mma_done, 0) && global_timer_ns() - t0 < wait_limit_ns(p.status)) {}
       }
     } else if (MODE == kGathered) {
       // -------------------------------------------------------- row gather
@@ -483,7 +491,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // After an abort, let the last gather land before the CTA can retire.
         if (*abort && quse > 0) {
           const unsigned long long t0 = global_timer_ns();
-          while (!mbar_try_wait(&bar.q_full[x], (quse - 1) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+          while (!mbar_try_wait(&bar.q_full[x], (quse - 1) & 1) && global_timer_ns() - t0 < wait_limit_ns(p.status)) {}
         }
       } else {
         // cp.async: lane l owns rows l, l + 32, l + 64, l + 96; it reads their list
@@ -585,6 +593,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                                 : nullptr;
       const int pos = p.q_off + i;        // the row's key position (masks)
       const int a0 = p.q_off + t.i0;      // query-major: the tile's first key position
+      // Query-major MoBA: the first key of the row's own block (a tile's rows may span
+      // two blocks when its first row does not start at a multiple of 128).
+      const int cBr = (MODE == kQueryMajor && p.is_moba) ? (pos / p.block) * p.block : 0;
       float m_run = -INFINITY, l_run = 0.f;
       for (int m = 0; m < w.nc; ++m, ++scnt) {
         ok = mbar_wait(&bar.s_full[x], scnt & 1, abort, p.status, site0 + 12);
@@ -599,9 +610,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int key0 = w.key0 + m * kTileKeys;
         if (MODE == kQueryMajor) {
           if (p.is_moba) {
-            if (key0 < t.cB) {
+            if (key0 < cBr) {
               // Window tail into an earlier block: keys i - j < window that the row's
-              // own selection does not already cover.
+              // own selection does not already cover.  (block is a multiple of 128, so
+              // the chunk's keys all lie in one block.)
               bool covered = false;
               if (irow) {
                 const int blk = key0 / p.block;
@@ -611,7 +623,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
               for (int e = 0; e < 128; ++e)
                 if (none || pos - (key0 + e) >= p.window) s[e] = -INFINITY;
-            } else if (key0 + kTileKeys > a0) {
+            } else if (key0 + kTileKeys - 1 > pos) {
 #pragma unroll
               for (int e = 0; e < 128; ++e)
                 if (key0 + e > pos) s[e] = -INFINITY;

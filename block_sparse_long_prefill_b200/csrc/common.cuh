@@ -14,10 +14,19 @@ namespace moba {
 
 // Device-side status: status[0] is MOBA_OK, or MOBA_ERR_DEVICE once any bounded wait
 // ran out; status[1] records where the first failing wait was (kernel id * 256 + wait
-// site).  The words live in the library's module (api.cu); kernels get their address
-// as a parameter, and moba_device_status() reads and clears them.
-// A wait gives up after this many nanoseconds of %globaltimer time.
+// site); status[2] is the wait limit in microseconds (0: the default below);
+// status[3] is a one-shot test flag (see moba_debug_fault_next_launch).  The words live
+// in the library's module (api.cu); kernels get their address as a parameter, and
+// moba_device_status() reads and clears the first two.
+// A wait gives up after this many nanoseconds of %globaltimer time by default.
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
+constexpr int kStatusWords = 4;
+
+// The wait limit in nanoseconds (read from the status words).
+__device__ __forceinline__ unsigned long long wait_limit_ns(const int *status) {
+  const int us = *reinterpret_cast<const volatile int *>(status + 2);
+  return us > 0 ? 1000ull * (unsigned long long)us : kWaitTimeoutNs;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -68,17 +77,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits until the phase with the given parity has completed.  Gives up (returns
-// false and records MOBA_ERR_DEVICE) after kWaitTimeoutNs, or at once when *abort
+// false and records MOBA_ERR_DEVICE) after the wait limit, or at once when *abort
 // is set by another role of the same CTA.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           int *status, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
+  const unsigned long long lim = wait_limit_ns(status);
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      if (global_timer_ns() - t0 > lim) {
         record_device_error(status, site);
         *abort = 1;
         return false;

@@ -14,8 +14,10 @@
 // (batch, kv-head, row tile, q-head), from a global counter (the cost of a tile grows
 // with its row position, so a static split would leave SMs idle); the pooled keys of a
 // kv-head stay staged in shared memory while the CTA's tiles stay in that kv-head.
-// Since block % 128 == 0 and q_off % 128 == 0, every row of a tile has the same own
-// block c, and the tile needs the scores of blocks [0, c) only.
+// A tile's 128 rows span at most two blocks (block >= 128): rows before the boundary
+// have own block c, the others c + 1, and the tile needs the scores of blocks [0, c_hi)
+// for its last row's own block c_hi.  The last tile of a head may hold fewer than 128
+// rows (its missing rows load as zeros and are never written).
 //   warp 0     TMA producer: query tiles (a ring of up to eight) and, per kv-head, the
 //              pooled keys kbar = hi + lo (two bf16 matrices of up to 256 rows; two
 //              slots when they fit, so the next kv-head's keys load early); it also
@@ -112,34 +114,45 @@ __device__ __forceinline__ uint64_t gate_desc(uint32_t tile, int ks, int rows) {
 // hk * G + g.  Ordered so that consecutive tiles share the kv-head.
 struct GateTile {
   int b, hk, g, rt;
-  int c;        // own block of the tile's rows: (q_off + 128 rt) / block
+  int c;        // own block of the tile's first row: (q_off + 128 rt) / block
+  int c_hi;     // own block of the tile's last row (c or c + 1)
   int chunk;    // query chunk of the tile's rows: 128 rt / chunk_rows
 };
+__device__ __forceinline__ void gate_tile_last(const GateParams &p, GateTile &r) {
+  const int last = p.q_off + min(r.rt * 128 + 127, p.N - 1);
+  r.c_hi = r.c + (last >= (r.c + 1) * p.block ? 1 : 0);
+}
 __device__ __forceinline__ GateTile gate_tile(const GateParams &p, int t) {
   GateTile r;
   r.g = t % p.G;
   t /= p.G;
-  const int nrt = p.N / 128;
+  const int nrt = (p.N + 127) / 128;
   r.rt = t % nrt;
   t /= nrt;
   r.hk = t % p.hkv;
   r.b = t / p.hkv;
   r.c = (p.q_off + r.rt * 128) / p.block;
   r.chunk = (r.rt * 128) / p.chunk_rows;
+  gate_tile_last(p, r);
   return r;
 }
 
-// The next tile in that order, without divisions (one decode per range, then steps).
+// The next tile in that order, without divisions (one decode per range, then steps;
+// the first row moves by 128 <= block positions, so its block grows by at most one).
 __device__ __forceinline__ void gate_tile_next(const GateParams &p, GateTile &r) {
   if (++r.g < p.G) return;
   r.g = 0;
   ++r.rt;
-  if (p.q_off + r.rt * 128 == (r.c + 1) * p.block) ++r.c;
+  if (p.q_off + r.rt * 128 >= (r.c + 1) * p.block) ++r.c;
   if (r.rt * 128 == (r.chunk + 1) * p.chunk_rows) ++r.chunk;
-  if (r.rt < p.N / 128) return;
+  if (r.rt < (p.N + 127) / 128) {
+    gate_tile_last(p, r);
+    return;
+  }
   r.rt = 0;
   r.c = p.q_off / p.block;
   r.chunk = 0;
+  gate_tile_last(p, r);
   if (++r.hk < p.hkv) return;
   r.hk = 0;
   ++r.b;
@@ -164,16 +177,17 @@ __device__ __forceinline__ void topk_insert(float (&val)[KM], int (&idx)[KM], fl
 }
 
 // The k-1 best (score, block) pairs of one row over blocks [0, c), from the TMEM
-// accumulator row at `acc`, in the float list above.
+// accumulator row at `acc`, in the float list above.  cw (>= c, the same on every
+// lane of the warp) bounds the warp-collective TMEM loads.
 template <int KM>
-__device__ __forceinline__ void topk_scan(uint32_t acc, int c, int npick, float (&val)[KM],
+__device__ __forceinline__ void topk_scan(uint32_t acc, int c, int cw, int npick, float (&val)[KM],
                                           int (&idx)[KM]) {
 #pragma unroll
   for (int e = 0; e < KM; ++e) {
     val[e] = (e < npick) ? -INFINITY : INFINITY;
     idx[e] = -1;
   }
-  for (int j0 = 0; j0 < c; j0 += 32) {
+  for (int j0 = 0; j0 < cw; j0 += 32) {
     uint32_t sc[32];
     tmem_ld32(acc + j0, sc);
     tmem_wait_ld();
@@ -302,7 +316,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // Tiles are handed out in chunks of p.chunk_tiles consecutive tiles from a global
   // counter: the producer takes a chunk and passes its first tile through the sched
   // ring to the MMA issuer and the top-k warps, which walk the same tiles in order.
-  const int ntiles = p.batch * p.hkv * (p.N / 128) * p.G;
+  const int ntiles = p.batch * p.hkv * ((p.N + 127) / 128) * p.G;
 
   if (tid == 0) {
     for (int s = 0; s < qst; ++s) {
@@ -401,9 +415,9 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // Let issued loads land before the CTA can retire.
         const unsigned long long t0 = global_timer_ns();
         for (uint32_t u = (quse > (uint32_t)qst ? quse - qst : 0u); u < quse; ++u)
-          while (!mbar_try_wait(&bar.q_full[u % qst], (u / qst) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+          while (!mbar_try_wait(&bar.q_full[u % qst], (u / qst) & 1) && global_timer_ns() - t0 < wait_limit_ns(p.status)) {}
         for (uint32_t u = (kuse > (uint32_t)ks ? kuse - ks : 0u); u < kuse; ++u)
-          while (!mbar_try_wait(&bar.k_full[u % ks], (u / ks) & 1) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+          while (!mbar_try_wait(&bar.k_full[u % ks], (u / ks) & 1) && global_timer_ns() - t0 < wait_limit_ns(p.status)) {}
       }
     }
   } else if (warp == 1) {
@@ -435,8 +449,8 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!(ok = mbar_wait(&bar.acc_empty[a], ((ause / nacc) & 1) ^ 1, abort, p.status, site0 + 5)))
           break;
         tc_fence_after();
-        const int c = gt.c;                                 // own block of every row
-        // Score columns needed (none when every past block is kept anyway).
+        const int c = gt.c_hi;                              // own block of the last row
+        // Score columns needed (none when every row keeps all its past blocks).
         const int nn = (c > p.topk - 1) ? min((c + 15) & ~15, kc16) : 0;
         if (nn > 0) {
           const uint32_t idesc = idesc_bf16(128, nn, 0, 0);
@@ -459,7 +473,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       umma_commit(&bar.mma_done);
       const unsigned long long t0 = global_timer_ns();
-      while (!mbar_try_wait(&bar.mma_done, 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {}
+      while (!mbar_try_wait(&bar.mma_done, 0) && global_timer_ns() - t0 < wait_limit_ns(p.status)) {}
     }
   } else {
     // ------------------------------------------------------------ top-k
@@ -505,7 +519,9 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int t = start; ok && t < end; ++t, ++u, gate_tile_next(p, gt)) {
       if ((int)(u & 1) != gi) continue;                    // the other group's tile
       const int i = gt.rt * 128 + r;
-      const int c = gt.c;
+      const bool valid = i < p.N;                         // the last tile may be partial
+      // The row's own block: the tile's first row's, or the next one past a boundary.
+      const int c = gt.c + ((p.q_off + i >= (gt.c + 1) * p.block) ? 1 : 0);
       const int h = gt.hk * p.G + gt.g;
       const int a = u % nacc;
       const int list = (gt.chunk * p.batch + gt.b) * p.hkv + gt.hk;
@@ -516,24 +532,28 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       ok = mbar_wait(&bar.acc_full[a], (u / nacc) & 1, abort, p.status, site0 + 6);
       if (!(ok = __all_sync(FULL, ok))) break;
       tc_fence_after();
-      int32_t *gout = p.idx + (((int64_t)gt.b * p.hq + h) * p.N + (i - lane)) * p.topk;
-      if (c <= npast || npast == 0) {
-        // Every past block is kept (or none is asked for): no scores needed.
+      const int i0w = i - lane;                            // the warp's first row
+      int32_t *gout = p.idx + (((int64_t)gt.b * p.hq + h) * p.N + i0w) * p.topk;
+      // Rows that keep every past block (c <= npast) need no scores; the warp scans the
+      // accumulator when any of its rows needs one, up to its largest own block.
+      const bool scored = valid && npast > 0 && c > npast;
+      const int cw = __reduce_max_sync(FULL, scored ? c : 0);
+      if (cw == 0) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar.acc_empty[a]);
         const int nk = min(c, npast);
         for (int s = 0; s < p.topk; ++s) orow[s] = (s < nk) ? s : (s == nk ? c : -1);
-        if (lane == 0)
-          for (int j = 0; j < nk; ++j) whist[j] += 32;
+        if (valid)
+          for (int j = 0; j < nk; ++j) atomicAdd(&whist[j], 1);
       } else {
-        const int npick = npast;                            // c > npast here
+        const int npick = npast;
         const uint32_t acc = tmem + lane_off + accw * a;
         int pk[KM];                                         // the row's picks, any order
         if constexpr (KM <= kGateMaxPicks) {
           float val[KM];
           int idx[KM];
-          topk_scan<KM>(acc, c, npick, val, idx);
+          topk_scan<KM>(acc, c, cw, npick, val, idx);
 #pragma unroll
           for (int e = 0; e < KM; ++e) pk[e] = idx[e];
         } else {
@@ -549,12 +569,12 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             uint32_t s0[16], s1[16];
             tmem_ld16(acc, s0);
             tmem_wait_ld();
-            for (int j0 = 0; j0 < c; j0 += 32) {
-              if (j0 + 16 < c) tmem_ld16(acc + j0 + 16, s1);
+            for (int j0 = 0; j0 < cw; j0 += 32) {
+              if (j0 + 16 < cw) tmem_ld16(acc + j0 + 16, s1);
               net_batches<KM>(L, s0, j0, c, imask);
               tmem_wait_ld();
-              if (j0 + 16 < c) {
-                if (j0 + 32 < c) tmem_ld16(acc + j0 + 32, s0);
+              if (j0 + 16 < cw) {
+                if (j0 + 32 < cw) tmem_ld16(acc + j0 + 32, s0);
                 net_batches<KM>(L, s1, j0 + 16, c, imask);
                 tmem_wait_ld();
               }
@@ -562,7 +582,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           } else {
 #pragma unroll
             for (int e = 0; e < KM; ++e) L[e] = (e <= npick) ? 0u : 0xFFFFFFFFu;
-            for (int j0 = 0; j0 < c; j0 += 32) {
+            for (int j0 = 0; j0 < cw; j0 += 32) {
               uint32_t sc[32];
               tmem_ld32(acc + j0, sc);
               tmem_wait_ld();
@@ -585,6 +605,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
           for (int e = 0; e + 1 < KM; ++e)
             near_tie |= (e + 1 == npick) & (((L[e] ^ L[e + 1]) & ~imask) == 0u);
+          near_tie &= scored;
 #pragma unroll
           for (int e = 0; e < KM; ++e) pk[e] = (int)(imask - (L[e] & imask));
           if (__any_sync(FULL, near_tie)) {
@@ -593,7 +614,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             unsigned long long X[KM];
 #pragma unroll
             for (int e = 0; e < KM; ++e) X[e] = (e < npick) ? 0ull : ~0ull;
-            for (int j0 = 0; j0 < c; j0 += 32) {
+            for (int j0 = 0; j0 < cw; j0 += 32) {
               uint32_t sc[32];
               tmem_ld32(acc + j0, sc);
               tmem_wait_ld();
@@ -615,39 +636,49 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar.acc_empty[a]);
-        // Ascending block order.
-        if (c <= 64) {
-          unsigned long long m = 0;
-#pragma unroll
-          for (int e = 0; e < KM; ++e)
-            if (e < npick) m |= 1ull << pk[e];
-          for (int s = 0; s < npick; ++s) {
-            orow[s] = __ffsll((long long)m) - 1;
-            m &= m - 1;
-          }
+        if (!scored) {
+          // A row of a scoring warp that keeps all of its past blocks.
+          const int nk = min(c, npast);
+          for (int s = 0; s < p.topk; ++s) orow[s] = (s < nk) ? s : (s == nk ? c : -1);
+          if (valid)
+            for (int j = 0; j < nk; ++j) atomicAdd(&whist[j], 1);
         } else {
+          // Ascending block order.
+          if (c <= 64) {
+            unsigned long long m = 0;
 #pragma unroll
-          for (int e = 0; e < KM; ++e) {
-            if (e < npick) {
-              int rank = 0;
+            for (int e = 0; e < KM; ++e)
+              if (e < npick) m |= 1ull << pk[e];
+            for (int s = 0; s < npick; ++s) {
+              orow[s] = __ffsll((long long)m) - 1;
+              m &= m - 1;
+            }
+          } else {
 #pragma unroll
-              for (int f = 0; f < KM; ++f)
-                if (f < npick) rank += pk[f] < pk[e];
-              orow[rank] = pk[e];
+            for (int e = 0; e < KM; ++e) {
+              if (e < npick) {
+                int rank = 0;
+#pragma unroll
+                for (int f = 0; f < KM; ++f)
+                  if (f < npick) rank += pk[f] < pk[e];
+                orow[rank] = pk[e];
+              }
             }
           }
-        }
 #pragma unroll
-        for (int e = 0; e < KM; ++e)
-          if (e < npick && pk[e] >= 0) atomicAdd(&whist[pk[e]], 1);  // < 0 only for NaN scores
-        orow[npick] = c;
-        for (int s = npick + 1; s < p.topk; ++s) orow[s] = -1;
+          for (int e = 0; e < KM; ++e)
+            if (e < npick && pk[e] >= 0) atomicAdd(&whist[pk[e]], 1);  // < 0 only for NaN scores
+          orow[npick] = c;
+          for (int s = npick + 1; s < p.topk; ++s) orow[s] = -1;
+        }
       }
-      // Staged rows -> idx: word w = 32 m + lane of the run is entry (r, s) of the warp.
+      // Staged rows -> idx: word w = 32 m + lane of the run is entry (r, s) of the warp;
+      // only the warp's rows below N are written.
       __syncwarp();
       {
+        const int nw = max(0, min(32, p.N - i0w)) * p.topk;
         int rr = r0, ss = s0;
-        for (int w = lane; w < 32 * p.topk; w += 32) {
+        for (int w = lane; w < nw; w += 32) {
           gout[w] = stg[rr * str + ss];
           rr += dq;
           ss += dr;
@@ -683,7 +714,7 @@ static cudaError_t launch_gate_tc_dk(const CUtensorMap *maps, GateParams p, int 
                                      cudaStream_t st) {
   using C = GateCfg<D>;
   // About eight chunks per CTA.
-  const long long ntiles = (long long)p.batch * p.hkv * (p.N / 128) * p.G;
+  const long long ntiles = (long long)p.batch * p.hkv * ((p.N + 127) / 128) * p.G;
   p.chunk_tiles = (int)std::max(1LL, std::min(32LL, ntiles / (8LL * grid)));
   auto kern = gate_tc_kernel<D, KM>;
   const int kc16 = (min(p.nblk, kGateMaxBlocks) + 15) & ~15;

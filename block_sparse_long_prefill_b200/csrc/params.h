@@ -96,7 +96,7 @@ struct GateParams {
   int32_t *idx;          // [batch, hq, N, topk]
   int *counts;           // workspace list counts
   int batch, hq, hkv, N, d, block, topk, nblk, G, chunk_rows;
-  int q_off;             // position of query row 0 among the keys (a multiple of 128)
+  int q_off;             // position of query row 0 among the keys
   int qstages;           // query tile ring depth (set by the launcher)
   int kslots;            // pooled-key staging slots, 1 or 2 (set by the launcher)
   int *sched;            // tile counter, zero at launch (the word after the list counts)
@@ -139,7 +139,7 @@ struct AttnParams {
   float *lse;              // [batch, hq, N]
   const int32_t *idx;      // [batch, hq, N, topk] (MoBA) or null (SWA)
   // Problem: N query rows; keys and values run over q_off + N positions, query row i
-  // sits at position q_off + i (q_off a multiple of 128).
+  // sits at position q_off + i.
   int batch, hq, hkv, N, d, block, topk, window, G;
   int q_off;
   float scale_log2;        // scale * log2(e)
@@ -149,7 +149,7 @@ struct AttnParams {
   // single row stride, or the row count exceeds int32).
   int q_gather_tma;
   // Query-major pass: row range of this pass.
-  int row_begin, row_end;  // multiples of 128 except row_end == N
+  int row_begin, row_end;  // multiples of 128 except row_end == N (any N)
   int ntiles;              // query-major work units in this pass
   // Block-major lists and partials (MoBA).
   const int *listoff;
@@ -172,5 +172,31 @@ struct MergeParams {
   int batch, hq, N, d, block, topk, chunk_rows, row_begin, row_end;
   int q_off;               // position of query row 0 among the keys
 };
+
+// Parameters of the backward kernels (bwd.cu).
+struct BwdParams {
+  int *status;             // device status words
+  const uint16_t *q, *out, *dout;
+  int64_t q_sb, q_sh, q_sn, o_sb, o_sh, o_sn, do_sb, do_sh, do_sn;
+  const float *lse;        // [batch, hq, N] (natural log)
+  uint16_t *dq, *dk, *dv;
+  int64_t dq_sb, dq_sh, dq_sn, dk_sb, dk_sh, dk_sn, dv_sb, dv_sh, dv_sn;
+  float2 *rowstat;         // [batch, hq, N]: lse * log2(e), D = dO . o
+  float *dqp;              // [batch, hq, N, topk, d] fp32 partial dQ per block slot
+  int batch, hq, hkv, N, d, block, topk, npast, nblk, G, nchunks, nlists;
+  float scale, scale_log2;
+  // Dispatch lists of the forward's selection step (its workspace).
+  const uint32_t *entries;
+  const int4 *tiles;
+  const int *tileoff, *listoff;
+};
+
+// Bytes of the backward's own workspace: the row statistics, then the dQ partials.
+inline size_t bwd_workspace_bytes(int batch, int hq, int N, int d, int topk, size_t *off_dqp) {
+  const size_t rows = size_t(batch) * hq * size_t(N);
+  const size_t a = align_up(rows * 8, 256);
+  if (off_dqp) *off_dqp = a;
+  return a + align_up(rows * size_t(topk) * size_t(d) * 4, 256);
+}
 
 }  // namespace moba

@@ -457,10 +457,21 @@ scatter_kernel(const ScatterParams p) {
 // picks the most recent blocks; an attention sink is MoBA whose gate picks the first
 // block together with the most recent ones.  Row i (own block c) keeps block c, the
 // first `sink` blocks and the k-1-sink most recent blocks before c (all past blocks
-// when c <= k-1).  The choice depends on c alone, so one CTA = one 128-row tile (one
-// c) of one (batch, kv-head): it writes the tile's G * 128 idx rows and adds G * 128 per
-// past pick to the list counts.
+// when c <= k-1).  The choice depends on c alone.  One CTA = one 128-row tile of one
+// (batch, kv-head): the tile's rows have own block c0 = (q_off + i0) / block, or c0 + 1
+// past a block boundary inside the tile (block >= 128); it writes the tile's G * 128
+// idx rows and adds, per own block, its rows times G to the list count of every past
+// pick.
 constexpr int kStaticThreads = 256;
+
+// Entry s of the choice list of a row whose own block is c.
+__device__ __forceinline__ int static_pick(int c, int s, int npast, int sink) {
+  const int recent = npast - sink;
+  if (c <= npast) return s < c ? s : (s == c ? c : -1);
+  if (s < sink) return s;
+  if (s < npast) return c - recent + (s - sink);
+  return s == npast ? c : -1;
+}
 
 __global__ void __launch_bounds__(kStaticThreads)
 static_select_kernel(int32_t *__restrict__ idx, int *__restrict__ counts, int batch, int hq,
@@ -470,28 +481,27 @@ static_select_kernel(int32_t *__restrict__ idx, int *__restrict__ counts, int ba
   const int hk = blockIdx.y, b = blockIdx.z;
   const int G = hq / hkv;
   const int rows = min(kTileRows, N - i0);
-  const int c = (q_off + i0) / block;
+  const int c0 = (q_off + i0) / block;
+  // Rows [0, rows0) of the tile sit in block c0, the rest in c0 + 1.
+  const int rows0 = min(rows, (c0 + 1) * block - (q_off + i0));
   const int npast = topk - 1;
-  const int recent = npast - sink;
-  // Entry s of the tile's (shared) choice list.
-  auto pick = [&](int s) -> int {
-    if (c <= npast) return s < c ? s : (s == c ? c : -1);
-    if (s < sink) return s;
-    if (s < npast) return c - recent + (s - sink);
-    return s == npast ? c : -1;
-  };
   // Each head's rows i0 .. i0 + rows - 1 are one contiguous run of rows * topk words.
   const int run = rows * topk;
   for (int g = 0; g < G; ++g) {
     int32_t *dst = idx + (((int64_t)b * hq + (int64_t)hk * G + g) * N + i0) * topk;
-    for (int e = threadIdx.x; e < run; e += kStaticThreads) dst[e] = pick(e % topk);
-  }
-  if (threadIdx.x < npast) {
-    const int j = pick(threadIdx.x);
-    if (j >= 0 && j < c) {
-      const int chunk = i0 / chunk_rows;
-      atomicAdd(&counts[(((int64_t)chunk * batch + b) * hkv + hk) * nblk + j], rows * G);
+    for (int e = threadIdx.x; e < run; e += kStaticThreads) {
+      const int r = e / topk;
+      dst[e] = static_pick(r < rows0 ? c0 : c0 + 1, e - r * topk, npast, sink);
     }
+  }
+  const int chunk = i0 / chunk_rows;
+  int *cnt = counts + (((int64_t)chunk * batch + b) * hkv + hk) * nblk;
+  for (int part = 0; part < 2; ++part) {
+    const int c = c0 + part;
+    const int nr = part ? rows - rows0 : rows0;
+    if (nr <= 0 || (int)threadIdx.x >= npast) continue;
+    const int j = static_pick(c, threadIdx.x, npast, sink);
+    if (j >= 0 && j < c) atomicAdd(&cnt[j], nr * G);
   }
 }
 

@@ -24,8 +24,9 @@
  *   - Block j covers key positions [j*block, min((j+1)*block, N)) (0-based; the MoBA
  *     page numbers blocks from 1); there are n = ceil(N / block) blocks.  When block
  *     does not divide N the last block is partial: it holds the N mod block remaining
- *     positions and is pooled over those keys.  block and N must be multiples of 128
- *     (moba_pool_keys alone takes any N and block >= 1).
+ *     positions and is pooled over those keys.  block must be a multiple of 128 (the
+ *     attention kernels walk keys in chunks of 128, and a chunk must not hold keys of
+ *     two blocks); N is free (moba_pool_keys alone takes any block >= 1).
  *   - d must be 64, 80 or 128 (moba_pool_keys alone takes any multiple of 8 up to
  *     256).
  *   - Ownership: the caller allocates every buffer (inputs, outputs, workspace); the
@@ -49,7 +50,7 @@ extern "C" {
 #endif
 
 #define MOBA_OK 0
-#define MOBA_ERR_SHAPE -1     /* N % 128, hq % hkv, block % 128, sizes out of range */
+#define MOBA_ERR_SHAPE -1     /* hq % hkv, block % 128, sizes out of range */
 #define MOBA_ERR_DIM -2       /* unsupported head dimension */
 #define MOBA_ERR_ALIGN -3     /* pointer or stride not 16-byte aligned */
 #define MOBA_ERR_ARG -4       /* topk < 1, window < 0, null pointer, ... */
@@ -139,10 +140,10 @@ int swa_attn_fwd(moba_tensor q, moba_tensor k, moba_tensor v, int batch, int hq,
  * sees only keys at or before its own position, so it does not depend on the other
  * rows).  k and v hold the Nk positions ([batch, hkv, Nk, d]); pool them with
  * moba_pool_keys(k, ..., Nk, ...).  q, idx, out and lse hold the N query rows.
- * Nk - N must be a multiple of 128 (and N, block as for the whole prefill); Nk = N is
- * the whole prefill, and the calls without _chunk are exactly that.  The workspace is
- * sized by moba_workspace_size_chunk for the same (N, Nk).  swa_attn_fwd_chunk takes
- * any N and window with Nk - N a multiple of 128.
+ * Any N and Nk >= N (block as for the whole prefill); Nk = N is the whole prefill, and
+ * the calls without _chunk are exactly that.  The workspace is sized by
+ * moba_workspace_size_chunk for the same (N, Nk).  swa_attn_fwd_chunk takes any N,
+ * Nk >= N and window >= 1.
  */
 int moba_workspace_size_chunk(int batch, int hq, int hkv, int N, int Nk, int d, int block,
                               int topk, size_t *bytes);
@@ -213,10 +214,56 @@ int moba_prefill_static(moba_tensor q, moba_tensor k, moba_tensor v, int batch, 
                         moba_tensor out, float *lse, void *stream);
 
 /*
+ * Backward of MoBA attention (training: [MoBA] §"MoBA와 전체 어텐션의 하이브리드" trains
+ * models whose layers are MoBA attention).  The gate is a parameter-free top-k and passes
+ * no gradient, so for the block choice idx of the forward the layer is softmax attention
+ * over each row's key set J_i, and with z_ij = scale q_i.k_j, p_ij = exp(z_ij - lse_i):
+ *     D_i = dO_i . o_i,  dz_ij = p_ij (dO_i . v_j - D_i),
+ *     dQ_i = scale sum_j dz_ij k_j,  dK_j = scale sum_i dz_ij q_i,  dV_j = sum_i p_ij dO_i
+ * (a KV head's dK and dV sum over the q-heads that read it).  Whole prefills (Nk = N)
+ * without a window; d in {64, 128}; any N (block a multiple of 128).
+ *   q, k, v, out, lse, idx : as given to / returned by moba_attn_fwd (out bf16, lse the
+ *                            natural-log row statistic)
+ *   workspace   : the buffer moba_select_topk filled for this idx (its dispatch lists
+ *                 are read; moba_attn_fwd leaves them intact)
+ *   dout        : bf16 upstream gradient [batch, hq, N, d]
+ *   dq          : bf16 out [batch, hq, N, d];  dk, dv : bf16 out [batch, hkv, N, d]
+ *   bwd_workspace : device buffer of at least moba_bwd_workspace_size() bytes (row
+ *                 statistics and fp32 dQ partials, one per row and block slot)
+ * Errors: MOBA_ERR_ARG for window != 0, MOBA_ERR_DIM for d = 80, MOBA_ERR_WORKSPACE for a
+ * missing or short buffer; the rest as for moba_attn_fwd.  Four kernels, no atomics:
+ * results are deterministic.
+ */
+int moba_bwd_workspace_size(int batch, int hq, int hkv, int N, int d, int block, int topk,
+                            size_t *bytes);
+int moba_attn_bwd(moba_tensor q, moba_tensor k, moba_tensor v, moba_tensor out, moba_tensor dout,
+                  const float *lse, const int32_t *idx, const void *workspace,
+                  size_t workspace_bytes, int batch, int hq, int hkv, int N, int d, int block,
+                  int topk, int window, float scale, moba_tensor dq, moba_tensor dk,
+                  moba_tensor dv, void *bwd_workspace, size_t bwd_workspace_bytes, void *stream);
+
+/*
  * Reads and clears the device-side status word that bounded kernel waits write
  * (MOBA_OK or MOBA_ERR_DEVICE) on the current device.  Synchronises the device.
  */
 int moba_device_status(void);
+
+/*
+ * Test hooks for the bounded waits (they change nothing unless called; both
+ * synchronise the current device first).
+ * moba_debug_set_wait_limit_us: every kernel wait that has not completed after this
+ *   many microseconds gives up (MOBA_ERR_DEVICE); 0 restores the default of 2 s.
+ * moba_debug_fault_next_launch(1): the next attention launch (moba_attn_fwd's passes or
+ *   swa_attn_fwd) leaves the first V chunk of its first CTA unloaded, so that a wait
+ *   runs out on purpose: the launch ends through the bounded-wait path (its roles stop,
+ *   copies in flight are drained, TMEM is freed) and moba_device_status() then reports
+ *   MOBA_ERR_DEVICE.  One shot: the launch that takes the flag clears it; 0 clears it.
+ *   Nothing faults or traps, and the context stays usable.
+ * Return MOBA_OK, MOBA_ERR_ARG for a value out of range, MOBA_ERR_LAUNCH when a CUDA call
+ * fails.  The paper has no counterpart; these exist to test failure handling.
+ */
+int moba_debug_set_wait_limit_us(int microseconds);
+int moba_debug_fault_next_launch(int kind);
 
 /* Static description of a status code. */
 const char *moba_status_string(int status);

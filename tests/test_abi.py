@@ -46,7 +46,6 @@ def test_workspace_size_is_host_only_and_grows_with_topk():
 
 @pytest.mark.parametrize("args,code", [
     ((1, 32, 8, 32768, 128, 500, 3), -1),   # block not a multiple of 128
-    ((1, 32, 8, 32064, 128, 512, 3), -1),   # N not a multiple of 128
     ((1, 30, 8, 32768, 128, 512, 3), -1),   # hq not a multiple of hkv
     ((1, 32, 8, 32768, 96, 512, 3), -2),    # unsupported d
     ((1, 32, 8, 32768, 128, 512, 0), -4),   # topk < 1
@@ -77,8 +76,8 @@ def test_bad_arguments_are_rejected_before_any_launch():
     assert lib.moba_pool_keys(odd, 1, 1, 1024, 128, 128, 1 << 20, 1 << 20, None) == -3
     assert lib.moba_pool_keys(ok, 1, 1, 0, 128, 128, 1 << 20, 1 << 20, None) == -1
     assert lib.moba_pool_keys(ok, 1, 1, 1000, 128, 0, 1 << 20, 1 << 20, None) == -1
-    # select: N not a multiple of 128
-    assert lib.moba_select_topk(ok, 1 << 20, 1, 1, 1, 1000, 128, 128, 3, 1 << 20, 1 << 20,
+    # select: a block that is not a multiple of 128 (any N is taken)
+    assert lib.moba_select_topk(ok, 1 << 20, 1, 1, 1, 1000, 128, 100, 3, 1 << 20, 1 << 20,
                                 1 << 30, None) == -1
     # select: workspace too small
     assert lib.moba_select_topk(ok, 1 << 20, 1, 1, 1, 1024, 128, 128, 3, 1 << 20, 1 << 20, 16,
@@ -100,18 +99,17 @@ def test_valid_call_without_a_device_reports_no_device():
 
 def test_chunk_workspace_and_offset_checks():
     """Chunked prefill (N query rows, the last N of Nk positions): the workspace of the
-    last 8K rows of a 32K context is smaller than the whole prefill's, and the query
-    offset Nk - N must be a non-negative multiple of 128."""
+    last 8K rows of a 32K context is smaller than the whole prefill's; the query offset
+    Nk - N may be any non-negative number."""
     whole = moba.workspace_size(1, 32, 8, 32768, 128, 512, 3)
     chunk = moba.workspace_size_chunk(1, 32, 8, 8192, 32768, 128, 512, 3)
     assert 0 < chunk < whole
     assert moba.workspace_size_chunk(1, 32, 8, 32768, 32768, 128, 512, 3) == whole
     lib = moba.library()
     out = ctypes.c_size_t(0)
-    assert lib.moba_workspace_size_chunk(1, 32, 8, 8192, 8192 + 64, 128, 512, 3, ctypes.byref(out)) == -1
+    assert lib.moba_workspace_size_chunk(1, 32, 8, 8192, 8192 + 64, 128, 512, 3, ctypes.byref(out)) == 0
     assert lib.moba_workspace_size_chunk(1, 32, 8, 8192, 4096, 128, 512, 3, ctypes.byref(out)) == -1
     ok = moba.MobaTensor(1 << 20, 8 * 1024, 8 * 1024, 128)
-    assert lib.swa_attn_fwd_chunk(ok, ok, ok, 1, 1, 1, 1000, 1064, 128, 64, 0.0, ok, 1 << 20, None) == -1
     assert lib.swa_attn_fwd_chunk(ok, ok, ok, 1, 1, 1, 1000, 900, 128, 64, 0.0, ok, 1 << 20, None) == -1
 
 
@@ -128,8 +126,8 @@ def test_minmax_entries_check_arguments():
     ok = moba.MobaTensor(1 << 20, 8 * 1024, 8 * 1024, 128)
     assert lib.moba_pool_keys_minmax(ok, 1, 1, 1024, 128, 0, 1 << 20, None) == -1
     assert lib.moba_pool_keys_minmax(ok, 1, 1, 1024, 128, 128, None, None) == -4
-    assert lib.moba_select_topk_minmax(ok, 1 << 20, 1, 2, 1, 1024, 1088, 128, 128, 3, 1 << 20,
-                                       1 << 20, 1 << 30, None) == -1  # offset not a multiple of 128
+    assert lib.moba_select_topk_minmax(ok, 1 << 20, 1, 2, 1, 1024, 1000, 128, 128, 3, 1 << 20,
+                                       1 << 20, 1 << 30, None) == -1  # fewer keys than queries
 
 
 @pytest.mark.parametrize("cu", [[1, 256], [0, 128, 64], [0, 100], []])
@@ -143,3 +141,17 @@ def test_varlen_rejects_bad_offsets_before_any_launch(cu):
 def test_host_pipeline_needs_groups_that_divide_the_kv_heads():
     with pytest.raises(ValueError):
         moba.MobaPrefillHost(1, 8, 4, 1024, 128, 512, 3, groups=3)
+
+
+def test_backward_checks_arguments_on_the_host():
+    lib = moba.library()
+    ok = moba.MobaTensor(1 << 20, 8 * 1024, 8 * 1024, 128)
+    out = ctypes.c_size_t(0)
+    assert lib.moba_bwd_workspace_size(1, 2, 1, 1024, 128, 128, 3, ctypes.byref(out)) == 0
+    assert out.value > 0
+    assert lib.moba_bwd_workspace_size(1, 2, 1, 1024, 80, 128, 3, ctypes.byref(out)) == -2
+    args = lambda window, d, ws: (ok, ok, ok, ok, ok, 1 << 20, 1 << 20, 1 << 20, 1 << 30, 1, 2, 1,
+                                 1024, d, 128, 3, window, 0.0, ok, ok, ok, 1 << 20, ws, None)
+    assert lib.moba_attn_bwd(*args(5, 128, 1 << 30)) == -4     # a window: not supported
+    assert lib.moba_attn_bwd(*args(0, 80, 1 << 30)) == -2      # d = 80: not supported
+    assert lib.moba_attn_bwd(*args(0, 128, 16)) == -5          # backward workspace too small

@@ -30,6 +30,12 @@ def _moba():
     ("chunk_partial_block", dict(batch=1, hq=4, hkv=1, seqlen=2176, d=64, block=256, topk=3), 896),
     # one row tile
     ("chunk_one_tile", dict(batch=1, hq=2, hkv=1, seqlen=2048, d=128, block=128, topk=4), 128),
+    # offsets that are not multiples of 128: query tiles span two blocks
+    ("chunk_offset_2500", dict(batch=1, hq=4, hkv=2, seqlen=6000, d=128, block=512, topk=3), 3500),
+    ("chunk_offset_window", dict(batch=1, hq=2, hkv=1, seqlen=3333, d=64, block=256, topk=4,
+                                 window=300), 1111),
+    ("chunk_offset_long_list_d80", dict(batch=1, hq=2, hkv=2, seqlen=5000, d=80, block=128,
+                                        topk=10), 2345),
 ])
 def test_moba_chunk_matches_whole_sequence_rows(name, kw, N):
     moba = _moba()
@@ -66,7 +72,8 @@ def test_moba_chunk_of_the_whole_sequence_equals_the_whole_prefill():
 
 
 @pytest.mark.parametrize("Nk,N,window,d", [(3000, 1080, 500, 80), (4096, 1024, 4096, 128),
-                                           (2304, 256, 64, 64)])
+                                           (2304, 256, 64, 64), (3000, 1100, 700, 80),
+                                           (2049, 1000, 300, 64)])
 def test_swa_chunk_matches_whole_sequence_rows(Nk, N, window, d):
     moba = _moba()
     w = workloads.small_swa(batch=1, hq=4, hkv=2, seqlen=Nk, d=d, window=window)

@@ -17,6 +17,7 @@ pytestmark = pytest.mark.gpu
     ("small_blocks", dict(batch=1, hq=4, hkv=2, seqlen=2048, d=128, block=128, topk=4), None),
     ("d64_window", dict(batch=2, hq=2, hkv=1, seqlen=1536, d=64, block=128, topk=3, window=200), None),
     ("d80_chunk_partial", dict(batch=1, hq=2, hkv=1, seqlen=2176, d=80, block=256, topk=3), 1024),
+    ("chunk_offset_any_n", dict(batch=1, hq=2, hkv=1, seqlen=2500, d=128, block=256, topk=3), 1003),
 ])
 def test_minmax_selection_matches_oracle(name, kw, N):
     import block_sparse_long_prefill_b200 as moba

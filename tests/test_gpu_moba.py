@@ -64,6 +64,13 @@ def run_and_check(w: workloads.Workload, seed=0, rows=None, check_pool=True):
     ("partial_window", dict(batch=1, hq=2, hkv=1, seqlen=2432, d=64, block=512, topk=2, window=300)),
     ("partial_long_list", dict(batch=1, hq=2, hkv=2, seqlen=4224, d=128, block=256, topk=12)),
     ("partial_k_all", dict(batch=2, hq=2, hkv=1, seqlen=1152, d=64, block=256, topk=8)),
+    # N not a multiple of 128: a partial last query tile (and a partial last block)
+    ("any_n_1000", dict(batch=1, hq=4, hkv=2, seqlen=1000, d=128, block=256, topk=3)),
+    ("any_n_4097_window", dict(batch=1, hq=2, hkv=1, seqlen=4097, d=64, block=512, topk=4,
+                               window=300)),
+    ("any_n_d80_long_list", dict(batch=1, hq=2, hkv=2, seqlen=3001, d=80, block=128, topk=12)),
+    ("any_n_below_one_tile", dict(batch=2, hq=2, hkv=1, seqlen=77, d=64, block=128, topk=2)),
+    ("any_n_k1", dict(batch=1, hq=2, hkv=1, seqlen=700, d=128, block=128, topk=1)),
 ])
 def test_moba_small_full_rows(name, kw):
     w = workloads.WORKLOADS["tiny"] if name == "tiny" else workloads.small_moba(name=name, **kw)
@@ -112,6 +119,9 @@ def test_moba_strided_inputs():
     # packed-key lists of 8 (k - 1 = 5) and 24 (k - 1 = 19) entries
     ("k6_blocks64", dict(batch=1, hq=2, hkv=1, seqlen=8192, d=64, block=128, topk=6)),
     ("k20_blocks64", dict(batch=1, hq=2, hkv=1, seqlen=8192, d=128, block=128, topk=20)),
+    # N not a multiple of 128 at 65 and 129 blocks (tensor-core gate, float and packed lists)
+    ("any_n_33000", dict(batch=1, hq=4, hkv=1, seqlen=33000, d=128, block=512, topk=3)),
+    ("any_n_33000_k13", dict(batch=1, hq=2, hkv=1, seqlen=33000, d=128, block=256, topk=13)),
 ])
 def test_moba_block_count_limits_sampled_rows(name, kw):
     w = workloads.small_moba(name=name, **kw)

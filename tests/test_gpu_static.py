@@ -19,6 +19,8 @@ pytestmark = pytest.mark.gpu
     ("sink2_chunk", dict(batch=1, hq=2, hkv=2, seqlen=4096, d=64, block=128, topk=5), 2, 1024),
     ("own_block_only", dict(batch=1, hq=2, hkv=1, seqlen=1024, d=128, block=128, topk=1), 0, None),
     ("sink_partial_block", dict(batch=1, hq=2, hkv=1, seqlen=1664, d=128, block=256, topk=3), 1, None),
+    # a chunk at offset 1223: query tiles span two blocks
+    ("sink_chunk_offset", dict(batch=1, hq=2, hkv=1, seqlen=3000, d=128, block=256, topk=4), 1, 1777),
 ])
 def test_static_gate_matches_oracle(name, kw, sink, N):
     import block_sparse_long_prefill_b200 as moba

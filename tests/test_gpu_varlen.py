@@ -16,6 +16,9 @@ pytestmark = pytest.mark.gpu
     ([1024, 384, 2176], 4, 2, 128, 256, 3, 0),     # 2176: a partial last block
     ([640, 128, 1536, 896], 2, 1, 64, 128, 4, 200),
     ([1280], 2, 2, 80, 512, 2, 0),
+    # lengths that are not multiples of 128, a one-token sequence among them
+    ([1000, 1, 2049], 4, 2, 128, 256, 3, 0),
+    ([333, 1500, 77], 2, 1, 64, 128, 4, 100),
 ])
 def test_varlen_equals_each_sequence_alone(lens, hq, hkv, d, block, topk, window):
     import block_sparse_long_prefill_b200 as moba
@@ -23,8 +26,9 @@ def test_varlen_equals_each_sequence_alone(lens, hq, hkv, d, block, topk, window
     T = offs[-1]
     g = torch.Generator().manual_seed(5)
     q = torch.randn(T, hq, d, generator=g).to(torch.bfloat16)
+    nb = -(-T // 128)
     k = (torch.randn(T, hkv, d, generator=g)
-         + 0.5 * torch.randn(T // 128, 1, d, generator=g).repeat_interleave(128, 0)).to(torch.bfloat16)
+         + 0.5 * torch.randn(nb, 1, d, generator=g).repeat_interleave(128, 0)[:T]).to(torch.bfloat16)
     v = torch.randn(T, hkv, d, generator=g).to(torch.bfloat16)
     out, lse = moba.moba_prefill_varlen(q.cuda(), k.cuda(), v.cuda(), offs, block, topk, window)
     torch.cuda.synchronize()
