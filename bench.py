@@ -482,7 +482,7 @@ def measure(w, steps, warmup, rank, world, device, seed, full=True, cpu_leg=True
         traffic = stored_traffic(w.name, kname)
         roofline = {"bound": "tensor", "achieved": passes[dom]["tflops"], "peak": tc_peak,
                     "unit": "TFLOP/s", "frac": passes[dom]["frac"],
-                    "traffic": None if traffic is None else traffic / nchunks,
+                    "traffic": traffic,
                     "kernel": f"{kname} ({dom.replace('_', ' ')}; {nchunks} launches per step, "
                               "one per query chunk)",
                     "work": "4*d FLOPs per attended (query, key) pair of the pass, all launches",
