@@ -32,7 +32,9 @@
 //   bwd_dq_merge_kernel  dQ_i = scale * (sum of the row's slots)
 // Roles in both tile kernels: warp 0 TMA loads of K/V, warp 1 the tcgen05 issuer and
 // TMEM owner, warps 2-3 the cp.async gather of the query-side rows (Q, dO, row
-// statistics) into the 128-byte-swizzled tile layout, warps 4-7 the elementwise work.
+// statistics) into the 128-byte-swizzled tile layout, warps 4-11 the elementwise work
+// (two warp groups over the same TMEM lanes, one per half of the 128 columns: the
+// backward needs no reduction along a row, so the columns split freely).
 // Every wait is bounded (2 s), as in the forward.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -44,7 +46,7 @@
 
 namespace moba {
 
-constexpr int kBwdThreads = 256;
+constexpr int kBwdThreads = 384;
 
 // Tile geometry: a 128-row bf16 tile of D columns is stored as 64-column regions of
 // 128-byte rows with the 128-byte swizzle (the TMA layout the forward uses).
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
 struct BwdBars {
   uint64_t q_full[2], q_empty[2];   // query-side tile (Q, dO, row statistics) per stage
   uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
-  uint64_t s_full, ds_full;         // S / dP ready; dS (and P) written back
+  uint64_t s_full[2], ds_full[2];   // per half: S / dP ready; dS (and P) written back
   uint64_t acc_full, acc_empty;     // accumulators final / read out
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -158,25 +160,54 @@ __device__ __forceinline__ void tile_row(const BwdParams &p, const BwdRows &t, i
   }
 }
 
-// Gathers a query tile: Q and dO rows into the swizzled tiles and the row statistics
-// (rows past the tile's end: zero rows and lse = +inf, so that p = 0 there).  Run by the
-// 64 threads of warps 2-3; each arrives once on `full` when its copies have landed.
-template <int D>
-__device__ __forceinline__ void gather_tile(const BwdParams &p, const BwdRows &t, int b, int hk,
-                                            uint32_t qt, uint32_t dot, float2 *stats,
-                                            uint64_t *full, int gt) {
-  for (int r = gt; r < 128; r += 64) {
-    const bool valid = r < t.rows;
+// The two rows (gt and gt + 64) that gather thread gt copies for a query tile: their
+// source rows and statistics, decoded ahead of the copies (the list entries of a
+// gathered tile are global loads, so the next tile's are read while the current tile's
+// copies are in flight).
+struct GatherRows {
+  const uint16_t *q[2], *g[2];
+  const float2 *st[2];
+  bool valid[2];
+};
+
+__device__ __forceinline__ void decode_rows(const BwdParams &p, const BwdRows &t, int b, int hk,
+                                            int gt, GatherRows &gr) {
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int r = gt + 64 * x;
+    gr.valid[x] = r < t.rows;
     int h = 0, i = 0, slot = 0;
-    if (valid) tile_row(p, t, hk, r, h, i, slot);
+    if (gr.valid[x]) tile_row(p, t, hk, r, h, i, slot);
     const int bb = t.gathered ? b : t.b;
-    const uint16_t *qrow = p.q + bb * p.q_sb + (int64_t)h * p.q_sh + (int64_t)i * p.q_sn;
-    const uint16_t *grow = p.dout + bb * p.do_sb + (int64_t)h * p.do_sh + (int64_t)i * p.do_sn;
-    gather_row<D>(qt, r, qrow, valid, p.q);
-    gather_row<D>(dot, r, grow, valid, p.dout);
-    stats[r] = valid ? p.rowstat[((int64_t)bb * p.hq + h) * p.N + i] : make_float2(INFINITY, 0.f);
+    gr.q[x] = p.q + bb * p.q_sb + (int64_t)h * p.q_sh + (int64_t)i * p.q_sn;
+    gr.g[x] = p.dout + bb * p.do_sb + (int64_t)h * p.do_sh + (int64_t)i * p.do_sn;
+    gr.st[x] = p.rowstat + ((int64_t)bb * p.hq + h) * p.N + i;
+  }
+}
+
+__device__ __forceinline__ void cp_async_8(uint32_t dst_smem, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+
+// Issues the copies of a decoded pair of rows into a query tile: Q and dO rows into the
+// swizzled tiles, the row statistics into `stats` (rows past the tile's end: zero rows
+// and lse = +inf, so that p = 0 there), as one cp.async group.  Run by the 64 threads of
+// warps 2-3; land_tile then waits for the group and arrives once on `full`.
+template <int D>
+__device__ __forceinline__ void issue_rows(const BwdParams &p, const GatherRows &gr, uint32_t qt,
+                                           uint32_t dot, float2 *stats, int gt) {
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int r = gt + 64 * x;
+    gather_row<D>(qt, r, gr.q[x], gr.valid[x], p.q);
+    gather_row<D>(dot, r, gr.g[x], gr.valid[x], p.dout);
+    if (gr.valid[x]) cp_async_8(smem_u32(stats + r), gr.st[x]);
+    else stats[r] = make_float2(INFINITY, 0.f);
   }
   cp_async_commit();
+}
+
+__device__ __forceinline__ void land_tile(uint64_t *full) {
   cp_async_wait_all();
   fence_proxy_async_smem();
   mbar_arrive(full);
@@ -271,10 +302,12 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
       mbar_init(&bar.v_full[s], 1);
       mbar_init(&bar.v_empty[s], 1);
     }
-    mbar_init(&bar.s_full, 1);
-    mbar_init(&bar.ds_full, 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bar.s_full[x], 1);
+      mbar_init(&bar.ds_full[x], 128);
+    }
     mbar_init(&bar.acc_full, 1);
-    mbar_init(&bar.acc_empty, 128);
+    mbar_init(&bar.acc_empty, 256);
     mbar_init(&bar.mma_done, 1);
     bar.abort = 0;
     fence_barrier_init();
@@ -327,11 +360,15 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+      // Each 128-key chunk is taken as two 64-key halves x, one per elementwise warp
+      // group, each with its own TMEM buffer: S_x at 128 x, dP_x at 128 x + 64; dQ at
+      // 256.  While one group works on its half, the tensor core computes the other's.
+      constexpr uint32_t idS = idesc_bf16(128, 64, 0, 0);
       constexpr uint32_t idQ = idesc_bf16(128, D, 0, 1);
-      const uint32_t tS = tmem, tP = tmem + 128, tQ = tmem + 256;
+      const uint32_t tQ = tmem + 256;
       const uint32_t qt = base + C::Q_OFF, dot = base + C::DO_OFF;
-      uint32_t kvc = 0, qn = 0, sc = 0, an = 0;
+      uint32_t kvc = 0, qn = 0, an = 0;
+      uint32_t sc[2] = {0u, 0u};
       bool ok = true;
       for (int u = blockIdx.x; ok && u < nitems; u += gridDim.x) {
         DqItem it;
@@ -344,32 +381,39 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         tc_fence_after();
         for (int m2 = 0; m2 <= it.nc && ok; ++m2) {
           const uint32_t sm = kvc + m2, sp = kvc + m2 - 1;
-          if (m2 > 0) {
-            // dQ += dS(m-1) K(m-1), once the elementwise warps wrote dS back.
-            if (!(ok = mbar_wait(&bar.ds_full, sc & 1, abort, p.status, site0 + 4))) break;
-            ++sc;
-            tc_fence_after();
-            const uint32_t kt = base + C::K_OFF + (sp % C::ST) * T::TILE;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              umma_ts(tQ, tS + kk * 8, bwd_mn_desc<D>(kt, kk), idQ, (m2 == 1 && kk == 0) ? 0u : 1u);
-            umma_commit(&bar.k_empty[sp % C::ST]);
-          }
+          const int st = sm % C::ST;
           if (m2 < it.nc) {
-            const int st = sm % C::ST;
             if (!(ok = mbar_wait(&bar.k_full[st], (sm / C::ST) & 1, abort, p.status, site0 + 5))) break;
             if (!(ok = mbar_wait(&bar.v_full[st], (sm / C::ST) & 1, abort, p.status, site0 + 6))) break;
             tc_fence_after();
-            const uint32_t kt = base + C::K_OFF + st * T::TILE;
-            const uint32_t vt = base + C::V_OFF + st * T::TILE;
+          }
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks)
-              umma_ss(tS, bwd_kmajor_desc<D>(qt, ks), bwd_kmajor_desc<D>(kt, ks), idS, ks > 0 ? 1u : 0u);
+          for (int x = 0; x < 2; ++x) {
+            const uint32_t tS = tmem + 128 * x, tP = tmem + 128 * x + 64;
+            if (m2 > 0) {
+              // dQ += dS_x(m-1) K_x(m-1), once group x wrote dS back.
+              if (!(ok = mbar_wait(&bar.ds_full[x], sc[x] & 1, abort, p.status, site0 + 4))) break;
+              ++sc[x];
+              tc_fence_after();
+              const uint32_t kt = base + C::K_OFF + (sp % C::ST) * T::TILE;
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks)
-              umma_ss(tP, bwd_kmajor_desc<D>(dot, ks), bwd_kmajor_desc<D>(vt, ks), idS, ks > 0 ? 1u : 0u);
-            umma_commit(&bar.s_full);
-            umma_commit(&bar.v_empty[st]);
+              for (int kk = 0; kk < 4; ++kk)
+                umma_ts(tQ, tS + kk * 8, bwd_mn_desc<D>(kt, 4 * x + kk), idQ,
+                        (m2 == 1 && x == 0 && kk == 0) ? 0u : 1u);
+              if (x == 1) umma_commit(&bar.k_empty[sp % C::ST]);
+            }
+            if (m2 < it.nc) {
+              const uint32_t kt = base + C::K_OFF + st * T::TILE + x * 8192;
+              const uint32_t vt = base + C::V_OFF + st * T::TILE + x * 8192;
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                umma_ss(tS, bwd_kmajor_desc<D>(qt, ks), bwd_kmajor_desc<D>(kt, ks), idS, ks > 0 ? 1u : 0u);
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                umma_ss(tP, bwd_kmajor_desc<D>(dot, ks), bwd_kmajor_desc<D>(vt, ks), idS, ks > 0 ? 1u : 0u);
+              umma_commit(&bar.s_full[x]);
+              if (x == 1) umma_commit(&bar.v_empty[st]);
+            }
           }
         }
         if (!ok) break;
@@ -386,18 +430,34 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     const int gt = tid - 64;
     uint32_t qn = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < nitems; u += gridDim.x) {
-      DqItem it;
-      if (!dq_item(p, u, ngath, it)) continue;
+    // The next item's rows are decoded while the current item's copies are in flight.
+    auto next_item = [&](int u, DqItem &it) -> int {
+      for (; u < nitems; u += gridDim.x)
+        if (dq_item(p, u, ngath, it)) return u;
+      return nitems;
+    };
+    DqItem it;
+    GatherRows gr;
+    int u = next_item(blockIdx.x, it);
+    if (u < nitems) decode_rows(p, it.t, it.b, it.hk, gt, gr);
+    while (ok && u < nitems) {
       if (!(ok = mbar_wait(&bar.q_empty[0], (qn & 1) ^ 1, abort, p.status, site0 + 7))) break;
       ++qn;
-      gather_tile<D>(p, it.t, it.b, it.hk, base + C::Q_OFF, base + C::DO_OFF, stats, &bar.q_full[0], gt);
+      issue_rows<D>(p, gr, base + C::Q_OFF, base + C::DO_OFF, stats, gt);
+      u = next_item(u + gridDim.x, it);
+      if (u < nitems) decode_rows(p, it.t, it.b, it.hk, gt, gr);
+      land_tile(&bar.q_full[0]);
     }
+    cp_async_wait_all();
   } else {
     // ------------------------------------------------------------ dS and dQ out
-    const int r = tid - 128;                       // row == TMEM lane
+    // Two warp groups share the rows: group grp (warps 4-7 or 8-11) takes the columns
+    // [64 grp, 64 grp + 64) of S and dP and half of dQ's columns, so that two warps per
+    // sub-partition hide each other's TMEM and exponential latencies.
+    const int r = (tid - 128) & 127;               // row == TMEM lane
+    const int grp = (warp - 4) >> 2;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t tS = tmem + lane_off, tP = tmem + lane_off + 128, tQ = tmem + lane_off + 256;
+    const uint32_t tS = tmem + lane_off + 128 * grp, tP = tS + 64, tQ = tmem + lane_off + 256;
     const float sl2 = p.scale_log2;
     uint32_t sc = 0, an = 0;
     bool ok = true;
@@ -415,15 +475,14 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         Dr = st2.y;
       }
       for (int m2 = 0; m2 < it.nc; ++m2, ++sc) {
-        ok = mbar_wait(&bar.s_full, sc & 1, abort, p.status, site0 + 8);
+        ok = mbar_wait(&bar.s_full[grp], sc & 1, abort, p.status, site0 + 8);
         if (!(ok = __all_sync(FULL, ok))) break;
         tc_fence_after();
-        const int key0 = it.key0 + m2 * kTileKeys;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        const int key0 = it.key0 + m2 * kTileKeys + 64 * grp;
+        {
           uint32_t sv[64], pv[64];
-          tmem_ld64(tS + half * 64, sv);
-          tmem_ld64(tP + half * 64, pv);
+          tmem_ld64(tS, sv);
+          tmem_ld64(tP, pv);
           tmem_wait_ld();
           uint32_t ds[32];
 #pragma unroll
@@ -431,18 +490,18 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             float d2[2];
 #pragma unroll
             for (int f = 0; f < 2; ++f) {
-              const int key = key0 + half * 64 + e + f;
+              const int key = key0 + e + f;
               float pr = ex2_approx(fmaf(__uint_as_float(sv[e + f]), sl2, -lse2));
               if (it.causal && key > i) pr = 0.f;
               d2[f] = pr * (__uint_as_float(pv[e + f]) - Dr);
             }
             ds[e / 2] = pack_bf16x2(d2[0], d2[1]);
           }
-          tmem_st32(tS + half * 32, ds);
+          tmem_st32(tS, ds);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bar.ds_full);
+        mbar_arrive(&bar.ds_full[grp]);
       }
       if (!ok) break;
       ok = mbar_wait(&bar.acc_full, an & 1, abort, p.status, site0 + 9);
@@ -451,7 +510,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
       tc_fence_after();
       float *dst = p.dqp + ((((int64_t)it.b * p.hq + h) * p.N + i) * p.topk + slot) * D;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = grp * (D / 2); c0 < (grp + 1) * (D / 2); c0 += 32) {
         uint32_t o[32];
         tmem_ld32(tQ + c0, o);
         tmem_wait_ld();
@@ -500,14 +559,24 @@ struct DkvWalk {
   int phase;            // 0 lists, 1 own rows, 2 done
 };
 
-__device__ __forceinline__ void dkv_walk_begin(const BwdParams &p, int u, DkvWalk &w) {
+// Unit u of CTA blockIdx.x (u = blockIdx.x + k gridDim.x) -> the k-th unit of the CTA
+// in cost order.  Units are ranked with the block index slowest (early blocks are past
+// blocks of the most rows, so their lists are the longest: roughly longest first), and
+// CTA x takes rank x of even stripes of gridDim.x ranks and rank gridDim.x - 1 - x of odd
+// ones (a snake), so that every CTA gets a similar mix of long and short walks.
+// Returns false when the rank is past the last unit.
+__device__ __forceinline__ bool dkv_walk_begin(const BwdParams &p, int u, DkvWalk &w) {
   const int tpb = p.block / kTileKeys;
-  const int t = u % tpb;
-  int rest = u / tpb;
-  w.j = rest % p.nblk;
-  rest /= p.nblk;
+  const int nunits = p.batch * p.hkv * p.nblk * tpb;
+  const int stripe = u / (int)gridDim.x, pos = u - stripe * (int)gridDim.x;
+  const int rank = stripe * (int)gridDim.x + ((stripe & 1) ? (int)gridDim.x - 1 - pos : pos);
+  if (rank >= nunits) return false;
+  const int t = rank % tpb;
+  int rest = rank / tpb;
   w.hk = rest % p.hkv;
-  w.b = rest / p.hkv;
+  rest /= p.hkv;
+  w.b = rest % p.batch;
+  w.j = rest / p.batch;
   w.kt0 = w.j * p.block + t * kTileKeys;
   w.blk_end = min((w.j + 1) * p.block, p.N);
   w.ch = 0;
@@ -520,6 +589,7 @@ __device__ __forceinline__ void dkv_walk_begin(const BwdParams &p, int u, DkvWal
     w.e = __ldg(p.listoff + L);
     w.e_end = __ldg(p.listoff + L + 1);
   }
+  return w.kt0 < p.N;
 }
 
 // The next query tile (returns false when the walk is over).
@@ -581,7 +651,10 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int site0 = (9 * 16 + (D == 64 ? 0 : 2)) * 256;
   constexpr uint32_t FULL = 0xffffffffu;
-  const int nunits = p.batch * p.hkv * p.nblk * (p.block / kTileKeys);
+  // Loop bound over whole stripes of gridDim.x units (the snake order of dkv_walk_begin
+  // maps the last, partial stripe onto ranks in reverse; ranks past the last unit skip).
+  const int nunits0 = p.batch * p.hkv * p.nblk * (p.block / kTileKeys);
+  const int nunits = (nunits0 + (int)gridDim.x - 1) / (int)gridDim.x * (int)gridDim.x;
 
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -590,10 +663,12 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     }
     mbar_init(&bar.k_full[0], 1);
     mbar_init(&bar.k_empty[0], 1);
-    mbar_init(&bar.s_full, 1);
-    mbar_init(&bar.ds_full, 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bar.s_full[x], 1);
+      mbar_init(&bar.ds_full[x], 128);
+    }
     mbar_init(&bar.acc_full, 1);
-    mbar_init(&bar.acc_empty, 128);
+    mbar_init(&bar.acc_empty, 256);
     mbar_init(&bar.mma_done, 1);
     bar.abort = 0;
     fence_barrier_init();
@@ -620,8 +695,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       bool ok = true;
       for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
         DkvWalk w;
-        dkv_walk_begin(p, u, w);
-        if (w.kt0 >= p.N) continue;
+        if (!dkv_walk_begin(p, u, w)) continue;
         if (!(ok = mbar_wait(&bar.k_empty[0], (kn & 1) ^ 1, abort, p.status, site0 + 1))) break;
         ++kn;
         mbar_arrive_expect_tx(&bar.k_full[0], 2 * T::BYTES);
@@ -641,16 +715,20 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+      // Each 128-row query tile is taken as two 64-row halves x, one per elementwise
+      // warp group, each with its own TMEM buffer: S^T_x at 128 x, dP^T_x at 128 x + 64;
+      // dK at 256, dV at 256 + D.  While one group works on its half, the tensor core
+      // computes the other's products.
+      constexpr uint32_t idS = idesc_bf16(128, 64, 0, 0);
       constexpr uint32_t idG = idesc_bf16(128, D, 0, 1);
-      const uint32_t tS = tmem, tP = tmem + 128, tK = tmem + 256, tV = tmem + 256 + D;
+      const uint32_t tK = tmem + 256, tV = tmem + 256 + D;
       const uint32_t kt = base + C::K_OFF, vt = base + C::V_OFF;
-      uint32_t kn = 0, qn = 0, sc = 0, an = 0;
+      uint32_t kn = 0, qn = 0, an = 0;
+      uint32_t sc[2] = {0u, 0u};
       bool ok = true;
       for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
         DkvWalk w;
-        dkv_walk_begin(p, u, w);
-        if (w.kt0 >= p.N) continue;
+        if (!dkv_walk_begin(p, u, w)) continue;
         if (!(ok = mbar_wait(&bar.k_full[0], kn & 1, abort, p.status, site0 + 2))) break;
         ++kn;
         if (!(ok = mbar_wait(&bar.acc_empty, (an & 1) ^ 1, abort, p.status, site0 + 3))) break;
@@ -667,31 +745,37 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             if (!(ok = mbar_wait(&bar.q_full[st], (qn / 2) & 1, abort, p.status, site0 + 4))) break;
             tc_fence_after();
           }
-          if (n > 0) {
-            // dV += P^T dO and dK += dS^T Q of the previous query tile.
-            if (!(ok = mbar_wait(&bar.ds_full, sc & 1, abort, p.status, site0 + 5))) break;
-            ++sc;
-            tc_fence_after();
-            const uint32_t qp = base + C::Q_OFF + prev_stage * T::TILE;
-            const uint32_t dp = base + C::DO_OFF + prev_stage * T::TILE;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t acc = (n == 1 && kk == 0) ? 0u : 1u;
-              umma_ts(tV, tS + kk * 8, bwd_mn_desc<D>(dp, kk), idG, acc);
-              umma_ts(tK, tP + kk * 8, bwd_mn_desc<D>(qp, kk), idG, acc);
+          for (int x = 0; x < 2; ++x) {
+            const uint32_t tS = tmem + 128 * x, tP = tmem + 128 * x + 64;
+            if (n > 0) {
+              // dV += P^T_x dO_x and dK += dS^T_x Q_x of the previous query tile.
+              if (!(ok = mbar_wait(&bar.ds_full[x], sc[x] & 1, abort, p.status, site0 + 5))) break;
+              ++sc[x];
+              tc_fence_after();
+              const uint32_t qp = base + C::Q_OFF + prev_stage * T::TILE;
+              const uint32_t dp = base + C::DO_OFF + prev_stage * T::TILE;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t acc = (n == 1 && x == 0 && kk == 0) ? 0u : 1u;
+                umma_ts(tV, tS + kk * 8, bwd_mn_desc<D>(dp, 4 * x + kk), idG, acc);
+                umma_ts(tK, tP + kk * 8, bwd_mn_desc<D>(qp, 4 * x + kk), idG, acc);
+              }
+              if (x == 1) umma_commit(&bar.q_empty[prev_stage]);
             }
-            umma_commit(&bar.q_empty[prev_stage]);
+            if (more) {
+              const uint32_t qt = base + C::Q_OFF + st * T::TILE + x * 8192;
+              const uint32_t dot = base + C::DO_OFF + st * T::TILE + x * 8192;
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                umma_ss(tS, bwd_kmajor_desc<D>(kt, ks), bwd_kmajor_desc<D>(qt, ks), idS, ks > 0 ? 1u : 0u);
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                umma_ss(tP, bwd_kmajor_desc<D>(vt, ks), bwd_kmajor_desc<D>(dot, ks), idS, ks > 0 ? 1u : 0u);
+              umma_commit(&bar.s_full[x]);
+            }
           }
-          if (!more) break;
-          const uint32_t qt = base + C::Q_OFF + st * T::TILE;
-          const uint32_t dot = base + C::DO_OFF + st * T::TILE;
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            umma_ss(tS, bwd_kmajor_desc<D>(kt, ks), bwd_kmajor_desc<D>(qt, ks), idS, ks > 0 ? 1u : 0u);
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            umma_ss(tP, bwd_kmajor_desc<D>(vt, ks), bwd_kmajor_desc<D>(dot, ks), idS, ks > 0 ? 1u : 0u);
-          umma_commit(&bar.s_full);
+          if (!ok || !more) break;
           prev_stage = st;
           ++qn;
           ++n;
@@ -712,31 +796,40 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     bool ok = true;
     for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
       DkvWalk w;
-      dkv_walk_begin(p, u, w);
-      if (w.kt0 >= p.N) continue;
+      if (!dkv_walk_begin(p, u, w)) continue;
       BwdRows t;
       int diag;
-      while (ok && dkv_walk_next(p, w, t, diag)) {
+      GatherRows gr;
+      // The next tile's rows are decoded while the current tile's copies are in flight.
+      bool have = dkv_walk_next(p, w, t, diag);
+      if (have) decode_rows(p, t, w.b, w.hk, gt, gr);
+      while (ok && have) {
         const uint32_t st = qn % 2;
         if (!(ok = mbar_wait(&bar.q_empty[st], ((qn / 2) & 1) ^ 1, abort, p.status, site0 + 6))) break;
         ++qn;
-        gather_tile<D>(p, t, w.b, w.hk, base + C::Q_OFF + st * T::TILE,
-                       base + C::DO_OFF + st * T::TILE, stats_all + st * 128, &bar.q_full[st], gt);
+        issue_rows<D>(p, gr, base + C::Q_OFF + st * T::TILE, base + C::DO_OFF + st * T::TILE,
+                      stats_all + st * 128, gt);
+        have = dkv_walk_next(p, w, t, diag);
+        if (have) decode_rows(p, t, w.b, w.hk, gt, gr);
+        land_tile(&bar.q_full[st]);
       }
     }
+    cp_async_wait_all();
   } else {
     // ------------------------------------------------------------ P^T, dS^T; dK, dV out
-    const int r = tid - 128;                       // key within the tile == TMEM lane
+    // Two warp groups share the keys: group grp takes the query columns
+    // [64 grp, 64 grp + 64) of S^T and dP^T and half of dK's and dV's columns.
+    const int r = (tid - 128) & 127;               // key within the tile == TMEM lane
+    const int grp = (warp - 4) >> 2;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t tS = tmem + lane_off, tP = tmem + lane_off + 128;
+    const uint32_t tS = tmem + lane_off + 128 * grp, tP = tS + 64;
     const uint32_t tK = tmem + lane_off + 256, tV = tmem + lane_off + 256 + D;
     const float sl2 = p.scale_log2;
     uint32_t sc = 0, an = 0, qn = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
       DkvWalk w;
-      dkv_walk_begin(p, u, w);
-      if (w.kt0 >= p.N) continue;
+      if (!dkv_walk_begin(p, u, w)) continue;
       const int key = w.kt0 + r;
       BwdRows t;
       int diag;
@@ -749,15 +842,15 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         if (!(ok = __all_sync(FULL, ok))) break;
         const float2 *stats = stats_all + st * 128;
         ++qn;
-        ok = mbar_wait(&bar.s_full, sc & 1, abort, p.status, site0 + 7);
+        ok = mbar_wait(&bar.s_full[grp], sc & 1, abort, p.status, site0 + 7);
         if (!(ok = __all_sync(FULL, ok))) break;
         ++sc;
         tc_fence_after();
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        {
+          const int half = grp;
           uint32_t sv[64], pv[64];
-          tmem_ld64(tS + half * 64, sv);
-          tmem_ld64(tP + half * 64, pv);
+          tmem_ld64(tS, sv);
+          tmem_ld64(tP, pv);
           tmem_wait_ld();
           uint32_t pp[32], dd[32];
 #pragma unroll
@@ -774,12 +867,12 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             pp[e / 2] = pack_bf16x2(pr[0], pr[1]);
             dd[e / 2] = pack_bf16x2(d2[0], d2[1]);
           }
-          tmem_st32(tS + half * 32, pp);
-          tmem_st32(tP + half * 32, dd);
+          tmem_st32(tS, pp);
+          tmem_st32(tP, dd);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bar.ds_full);
+        mbar_arrive(&bar.ds_full[grp]);
       }
       if (!ok) break;
       ok = mbar_wait(&bar.acc_full, an & 1, abort, p.status, site0 + 8);
@@ -791,7 +884,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       uint16_t *dvr = p.dv + w.b * p.dv_sb + (int64_t)w.hk * p.dv_sh + (int64_t)key * p.dv_sn;
       const float sc_k = p.scale;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = grp * (D / 2); c0 < (grp + 1) * (D / 2); c0 += 32) {
         uint32_t a[32], bv[32];
         tmem_ld32(tK + c0, a);
         tmem_ld32(tV + c0, bv);

@@ -19,7 +19,8 @@
 namespace moba {
 
 constexpr int kMergeThreads = 256;
-constexpr int kMergeEager = 4;  // past slots whose loads are issued before the weights
+// Past slots whose loads are issued before the weights: 4, or 12 for long lists (all of
+// a row's partial loads in flight at once, for fewer resident warps).
 
 __device__ __forceinline__ void add_scaled(float (&acc)[8], float w, uint4 v) {
   const uint32_t x[4] = {v.x, v.y, v.z, v.w};
@@ -36,7 +37,7 @@ __device__ __forceinline__ void add_scaled(float (&acc)[8], float w, uint4 v) {
 // computes the weight of slot v alone (one exponential), and the sub-group shares the
 // maximum, the sum and the weights with shuffles.  Row indices fit 32 bits: the host
 // bounds batch * hq * N below 2^31 whenever partials exist.
-template <int D>
+template <int D, int kMergeEager>
 __device__ __forceinline__ void merge_row(const MergeParams &p, int row, int nrows, int v,
                                           unsigned gmask, int gbase) {
   constexpr int LPR = D / 8;
@@ -123,7 +124,7 @@ __device__ __forceinline__ void merge_row(const MergeParams &p, int row, int nro
   if (v == 0) p.lse[(int64_t)bh * p.N + i] = lse;
 }
 
-template <int D>
+template <int D, int EAGER>
 __global__ void __launch_bounds__(kMergeThreads)
 merge_partials_kernel(const MergeParams p) {
   constexpr int LPR = D / 8;       // lanes per row
@@ -139,7 +140,7 @@ merge_partials_kernel(const MergeParams p) {
   const int total = p.batch * p.hq * nrows;
   // Rows warp_id * RPW + sub, then a grid-stride walk.
   for (int row = warp_id * RPW + sub; row < total; row += nwarps * RPW)
-    merge_row<D>(p, row, nrows, v, gmask, gbase);
+    merge_row<D, EAGER>(p, row, nrows, v, gmask, gbase);
 }
 
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t st) {
@@ -154,10 +155,20 @@ cudaError_t launch_merge(const MergeParams &p, cudaStream_t st) {
   const int64_t cap = (int64_t)nsm * 8 * 4;
   if (blocks > cap) blocks = cap;
   if (blocks <= 0) return cudaSuccess;
+  const bool long_list = p.topk - 1 > 4;
   switch (p.d) {
-    case 64: merge_partials_kernel<64><<<(unsigned)blocks, kMergeThreads, 0, st>>>(p); break;
-    case 80: merge_partials_kernel<80><<<(unsigned)blocks, kMergeThreads, 0, st>>>(p); break;
-    case 128: merge_partials_kernel<128><<<(unsigned)blocks, kMergeThreads, 0, st>>>(p); break;
+    case 64:
+      if (long_list) merge_partials_kernel<64, 12><<<(unsigned)blocks, kMergeThreads, 0, st>>>(p);
+      else merge_partials_kernel<64, 4><<<(unsigned)blocks, kMergeThreads, 0, st>>>(p);
+      break;
+    case 80:
+      if (long_list) merge_partials_kernel<80, 12><<<(unsigned)blocks, kMergeThreads, 0, st>>>(p);
+      else merge_partials_kernel<80, 4><<<(unsigned)blocks, kMergeThreads, 0, st>>>(p);
+      break;
+    case 128:
+      if (long_list) merge_partials_kernel<128, 12><<<(unsigned)blocks, kMergeThreads, 0, st>>>(p);
+      else merge_partials_kernel<128, 4><<<(unsigned)blocks, kMergeThreads, 0, st>>>(p);
+      break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
