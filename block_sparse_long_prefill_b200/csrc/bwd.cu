@@ -73,18 +73,6 @@ __device__ __forceinline__ uint64_t bwd_mn_desc(uint32_t tile, int kk) {
   return smem_desc(tile + kk * 2048, 16, 1024, kSwizzle128);
 }
 
-// cp.async of one D-column bf16 row into row r of a swizzled tile (zeros when !valid).
-template <int D>
-__device__ __forceinline__ void gather_row(uint32_t tile, int r, const uint16_t *src, bool valid,
-                                           const uint16_t *fallback) {
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c) {
-    const uint32_t dst = (c < 8) ? tile + r * 128 + ((c ^ (r & 7)) << 4)
-                                 : tile + BwdTile<D>::R0 + r * 128 + (((c - 8) ^ (r & 7)) << 4);
-    cp_async_16_zfill(dst, valid ? src + c * 8 : fallback, valid);
-  }
-}
-
 // ------------------------------------------------------------------ prep
 
 // rowstat[(b * hq + h) * N + i] = (lse_i * log2(e), D_i = dO_i . o_i), one warp per row
@@ -160,51 +148,74 @@ __device__ __forceinline__ void tile_row(const BwdParams &p, const BwdRows &t, i
   }
 }
 
-// The two rows (gt and gt + 64) that gather thread gt copies for a query tile: their
-// source rows and statistics, decoded ahead of the copies (the list entries of a
-// gathered tile are global loads, so the next tile's are read while the current tile's
-// copies are in flight).
+// Gather of a query tile by the 64 threads of warps 2-3: warp w (0 or 1) copies tile
+// rows [64 w, 64 w + 64).  Lane l decodes rows 64 w + 2 l and 64 w + 2 l + 1 (the list
+// entries of a gathered tile are global loads, so the next tile's rows are decoded while
+// the gather waits for a free stage) and leaves their source rows in the warp's table in
+// shared memory; the copies then go eight lanes to a row, each lane 16 bytes of a 128-byte
+// row segment, so that one warp instruction moves four whole segments (coalesced).
 struct GatherRows {
-  const uint16_t *q[2], *g[2];
   const float2 *st[2];
   bool valid[2];
 };
 
+struct RowSrc {
+  const uint16_t *q, *g;   // source rows of Q and dO, or null (a row past the tile's end)
+};
+
 __device__ __forceinline__ void decode_rows(const BwdParams &p, const BwdRows &t, int b, int hk,
-                                            int gt, GatherRows &gr) {
+                                            int gt, RowSrc *tab, GatherRows &gr) {
+  const int w = gt >> 5, l = gt & 31;
 #pragma unroll
   for (int x = 0; x < 2; ++x) {
-    const int r = gt + 64 * x;
+    const int r = 64 * w + 2 * l + x;
     gr.valid[x] = r < t.rows;
     int h = 0, i = 0, slot = 0;
     if (gr.valid[x]) tile_row(p, t, hk, r, h, i, slot);
     const int bb = t.gathered ? b : t.b;
-    gr.q[x] = p.q + bb * p.q_sb + (int64_t)h * p.q_sh + (int64_t)i * p.q_sn;
-    gr.g[x] = p.dout + bb * p.do_sb + (int64_t)h * p.do_sh + (int64_t)i * p.do_sn;
+    RowSrc src;
+    src.q = gr.valid[x] ? p.q + bb * p.q_sb + (int64_t)h * p.q_sh + (int64_t)i * p.q_sn : nullptr;
+    src.g = gr.valid[x] ? p.dout + bb * p.do_sb + (int64_t)h * p.do_sh + (int64_t)i * p.do_sn : nullptr;
+    tab[r] = src;
     gr.st[x] = p.rowstat + ((int64_t)bb * p.hq + h) * p.N + i;
   }
+  __syncwarp();
 }
 
 __device__ __forceinline__ void cp_async_8(uint32_t dst_smem, const void *src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst_smem), "l"(src) : "memory");
 }
 
-// Issues the copies of a decoded pair of rows into a query tile: Q and dO rows into the
-// swizzled tiles, the row statistics into `stats` (rows past the tile's end: zero rows
-// and lse = +inf, so that p = 0 there), as one cp.async group.  Run by the 64 threads of
-// warps 2-3; land_tile then waits for the group and arrives once on `full`.
+// Issues the copies of the warp's 64 decoded rows into a query tile: Q and dO rows into
+// the swizzled tiles, the row statistics into `stats` (rows past the tile's end: zero
+// rows and lse = +inf, so that p = 0 there), as one cp.async group; land_tile then waits
+// for the group and arrives once on `full` (64 arrivals complete it).
 template <int D>
-__device__ __forceinline__ void issue_rows(const BwdParams &p, const GatherRows &gr, uint32_t qt,
-                                           uint32_t dot, float2 *stats, int gt) {
+__device__ __forceinline__ void issue_rows(const BwdParams &p, const GatherRows &gr,
+                                           const RowSrc *tab, uint32_t qt, uint32_t dot,
+                                           float2 *stats, int gt) {
+  const int w = gt >> 5, l = gt & 31;
+  const int cc = l & 7;                      // 16-byte chunk of a 128-byte row segment
+#pragma unroll 4
+  for (int s4 = 0; s4 < 16; ++s4) {
+    const int r = 64 * w + 4 * s4 + (l >> 3);
+    const RowSrc src = tab[r];
+    const bool valid = src.q != nullptr;
+#pragma unroll
+    for (int rg = 0; rg < D / 64; ++rg) {
+      const uint32_t off = rg * BwdTile<D>::R0 + r * 128 + ((cc ^ (r & 7)) << 4);
+      cp_async_16_zfill(qt + off, valid ? src.q + rg * 64 + cc * 8 : p.q, valid);
+      cp_async_16_zfill(dot + off, valid ? src.g + rg * 64 + cc * 8 : p.dout, valid);
+    }
+  }
 #pragma unroll
   for (int x = 0; x < 2; ++x) {
-    const int r = gt + 64 * x;
-    gather_row<D>(qt, r, gr.q[x], gr.valid[x], p.q);
-    gather_row<D>(dot, r, gr.g[x], gr.valid[x], p.dout);
+    const int r = 64 * w + 2 * l + x;
     if (gr.valid[x]) cp_async_8(smem_u32(stats + r), gr.st[x]);
     else stats[r] = make_float2(INFINITY, 0.f);
   }
   cp_async_commit();
+  __syncwarp();   // the table is read; the next decode may overwrite it
 }
 
 __device__ __forceinline__ void land_tile(uint64_t *full) {
@@ -271,7 +282,8 @@ struct DqCfg {
   static constexpr int K_OFF = 2 * BwdTile<D>::TILE;
   static constexpr int V_OFF = K_OFF + ST * BwdTile<D>::TILE;
   static constexpr int ST_OFF = V_OFF + ST * BwdTile<D>::TILE;   // float2 stats [128]
-  static constexpr int BAR_OFF = ST_OFF + 128 * 8;
+  static constexpr int TAB_OFF = ST_OFF + 128 * 8;                 // RowSrc [128]
+  static constexpr int BAR_OFF = TAB_OFF + 128 * 16;
   static constexpr int SMEM = BAR_OFF + 1024 + 1024;
 };
 
@@ -430,7 +442,9 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     const int gt = tid - 64;
     uint32_t qn = 0;
     bool ok = true;
-    // The next item's rows are decoded while the current item's copies are in flight.
+    // The next item's rows are decoded after the current item's copies have landed and
+    // been handed on (their arrive is what the MMA issuer waits for), while the gather
+    // waits for the buffer to come free again.
     auto next_item = [&](int u, DqItem &it) -> int {
       for (; u < nitems; u += gridDim.x)
         if (dq_item(p, u, ngath, it)) return u;
@@ -438,15 +452,17 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     };
     DqItem it;
     GatherRows gr;
+    RowSrc *tab = reinterpret_cast<RowSrc *>(sbase + C::TAB_OFF);
     int u = next_item(blockIdx.x, it);
-    if (u < nitems) decode_rows(p, it.t, it.b, it.hk, gt, gr);
+    if (u < nitems) decode_rows(p, it.t, it.b, it.hk, gt, tab, gr);
     while (ok && u < nitems) {
-      if (!(ok = mbar_wait(&bar.q_empty[0], (qn & 1) ^ 1, abort, p.status, site0 + 7))) break;
+      ok = mbar_wait(&bar.q_empty[0], (qn & 1) ^ 1, abort, p.status, site0 + 7);
+      if (!(ok = __all_sync(FULL, ok))) break;
       ++qn;
-      issue_rows<D>(p, gr, base + C::Q_OFF, base + C::DO_OFF, stats, gt);
-      u = next_item(u + gridDim.x, it);
-      if (u < nitems) decode_rows(p, it.t, it.b, it.hk, gt, gr);
+      issue_rows<D>(p, gr, tab, base + C::Q_OFF, base + C::DO_OFF, stats, gt);
       land_tile(&bar.q_full[0]);
+      u = next_item(u + gridDim.x, it);
+      if (u < nitems) decode_rows(p, it.t, it.b, it.hk, gt, tab, gr);
     }
     cp_async_wait_all();
   } else {
@@ -543,7 +559,8 @@ struct DkvCfg {
   static constexpr int Q_OFF = 2 * BwdTile<D>::TILE;                  // 2 stages of Q
   static constexpr int DO_OFF = Q_OFF + 2 * BwdTile<D>::TILE;         // 2 stages of dO
   static constexpr int ST_OFF = DO_OFF + 2 * BwdTile<D>::TILE;        // 2 x float2 [128]
-  static constexpr int BAR_OFF = ST_OFF + 2 * 128 * 8;
+  static constexpr int TAB_OFF = ST_OFF + 2 * 128 * 8;                 // RowSrc [128]
+  static constexpr int BAR_OFF = TAB_OFF + 128 * 16;
   static constexpr int SMEM = BAR_OFF + 1024 + 1024;
 };
 
@@ -800,18 +817,21 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       BwdRows t;
       int diag;
       GatherRows gr;
-      // The next tile's rows are decoded while the current tile's copies are in flight.
+      RowSrc *tab = reinterpret_cast<RowSrc *>(sbase + C::TAB_OFF);
+      // The next tile's rows are decoded after the current tile's copies have landed and
+      // been handed on, while the gather waits for the next stage to come free.
       bool have = dkv_walk_next(p, w, t, diag);
-      if (have) decode_rows(p, t, w.b, w.hk, gt, gr);
+      if (have) decode_rows(p, t, w.b, w.hk, gt, tab, gr);
       while (ok && have) {
         const uint32_t st = qn % 2;
-        if (!(ok = mbar_wait(&bar.q_empty[st], ((qn / 2) & 1) ^ 1, abort, p.status, site0 + 6))) break;
+        ok = mbar_wait(&bar.q_empty[st], ((qn / 2) & 1) ^ 1, abort, p.status, site0 + 6);
+        if (!(ok = __all_sync(FULL, ok))) break;
         ++qn;
-        issue_rows<D>(p, gr, base + C::Q_OFF + st * T::TILE, base + C::DO_OFF + st * T::TILE,
+        issue_rows<D>(p, gr, tab, base + C::Q_OFF + st * T::TILE, base + C::DO_OFF + st * T::TILE,
                       stats_all + st * 128, gt);
-        have = dkv_walk_next(p, w, t, diag);
-        if (have) decode_rows(p, t, w.b, w.hk, gt, gr);
         land_tile(&bar.q_full[st]);
+        have = dkv_walk_next(p, w, t, diag);
+        if (have) decode_rows(p, t, w.b, w.hk, gt, tab, gr);
       }
     }
     cp_async_wait_all();
