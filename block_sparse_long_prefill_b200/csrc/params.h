@@ -101,7 +101,6 @@ struct GateParams {
   int kslots;            // pooled-key staging slots, 1 or 2 (set by the launcher)
   int *sched;            // tile counter, zero at launch (the word after the list counts)
   int chunk_tiles;       // tiles per chunk taken from it (set by the launcher)
-  int tmem_cols;         // TMEM columns a CTA allocates: 512, or 256 with two CTAs per SM
   // When done is set (zero at launch, the second word after the counts), the last
   // CTA to finish writes the list offsets (cursor, listoff, tileoff over nlists).
   int *done;
