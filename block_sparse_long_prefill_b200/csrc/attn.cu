@@ -44,6 +44,24 @@
 namespace moba {
 
 constexpr int kAttnThreads = 384;
+
+// Packed f32x2 arithmetic (two lanes of fp32 per instruction, each rounded as the
+// scalar instruction would be): d = a * b + c and d += a on pairs.
+__device__ __forceinline__ void fma_f32x2(float &d0, float &d1, float a0, float a1, float b,
+                                          float c) {
+  asm("{.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+__device__ __forceinline__ void add_f32x2(float &d0, float &d1, float a0, float a1) {
+  asm("{.reg .b64 ra, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rd, {%0, %1};\n\t"
+      "add.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
+}
 constexpr int kRescaleThreshold = 8;  // log2 units
 // Of every 16 probabilities, this many take the FMA-pipe 2^x (exp2_fma) instead of
 // the MUFU unit.
@@ -447,7 +465,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // (and the 16-column tail for D = 80) per instruction, into the swizzled tile
         // layout; rows past the unit's end repeat a valid row and are never stored.
         // While a unit's copies are in flight the warp decodes the next unit's rows.
-        auto rows_of = [&](const Tile &t, int (&rr)[4]) {
+        auto rows_of = [&](const Tile &t, int (&rr)[4], bool pf) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int r = 4 * lane + e;
@@ -456,6 +474,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const int g = (int)(ig % (uint32_t)p.G);
             const int i = (int)(ig / (uint32_t)p.G);
             rr[e] = ((t.b * p.hq + t.hk * p.G + g) * p.N) + i;
+            // The next unit's rows go into L2 while the current unit runs, so that its
+            // gather reads L2 instead of DRAM.
+            if (pf && r < t.rows)
+              prefetch_l2_bulk(p.q + t.b * p.q_sb + (int64_t)(t.hk * p.G + g) * p.q_sh + (int64_t)i * p.q_sn, D * 2);
           }
         };
         int u = u_begin + (int)blockIdx.x;
@@ -466,7 +488,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (u < u_end) {
           gathered_unit(p, __ldg(p.tiles + u), w);
           tx = x ? w.t[1] : w.t[0];
-          if (tx.rows > 0) rows_of(tx, rr);
+          if (tx.rows > 0) rows_of(tx, rr, false);
         }
         for (; ok && u < u_end; u += gridDim.x) {
           if (tx.rows > 0) {
@@ -485,7 +507,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (un < u_end) {
             gathered_unit(p, __ldg(p.tiles + un), w);
             tx = x ? w.t[1] : w.t[0];
-            if (tx.rows > 0) rows_of(tx, rr);
+            if (tx.rows > 0) rows_of(tx, rr, true);
           }
         }
         // After an abort, let the last gather land before the CTA can retire.
@@ -673,15 +695,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         ++tcnt;
         if (!(ok = __all_sync(FULL, ok))) break;
         const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+        // Scale and row sums in packed pairs (eight running sums: four pairs).
         float ls[8];
 #pragma unroll
         for (int u2 = 0; u2 < 8; ++u2) ls[u2] = 0.f;
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
-          const float x0 = fmaf(s[2 * e], sl2, -mu), x1 = fmaf(s[2 * e + 1], sl2, -mu);
+          float x0, x1;
+          fma_f32x2(x0, x1, s[2 * e], s[2 * e + 1], sl2, -mu);
           const float p0 = ((2 * e) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x0) : ex2_approx(x0);
           const float p1 = ((2 * e + 1) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x1) : ex2_approx(x1);
-          ls[e & 7] += p0 + p1;
+          add_f32x2(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], p0, p1);
           sv[e] = pack_bf16x2(p0, p1);
         }
         __syncwarp();
