@@ -32,7 +32,10 @@
 // chunk m is issued after its P V of chunk m-1, so when the softmax sees S(m) complete
 // (commit semantics: every earlier MMA is complete) it may rescale O at once.  The
 // running maximum is raised lazily: O and l are rescaled only when it grows by more
-// than 2^8.
+// than 2^8.  The gathered pass skips the row maximum once a row has one: a chunk is
+// computed against the running maximum and redone with its exact maximum only when its
+// row sum exceeds 2^60.  MoBA launches let the two streams' exponentials overlap;
+// sliding-window launches alternate them per sub-partition.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -73,6 +76,10 @@ __device__ __forceinline__ void add_f32x2(float &d0, float &d1, float a0, float 
       : "f"(a0), "f"(a1));
 }
 constexpr int kRescaleThreshold = 8;  // log2 units
+// A gathered chunk computed against a stale running maximum is kept while its row sum is
+// at most 2^60: every probability is then below 2^60, so P (bf16), l and O (fp32) stay
+// finite.
+constexpr float kSumBound = 1.152921504606846976e18f;
 // Of every 16 probabilities, this many take the FMA-pipe 2^x (exp2_fma) instead of
 // the MUFU unit.
 #ifndef MOBA_EXP_EMU_PER16
@@ -640,97 +647,133 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (!(ok = __all_sync(FULL, ok))) break;
         tc_fence_after();
         uint32_t sv[128];
-        tmem_ld64(tS, *reinterpret_cast<uint32_t(*)[64]>(&sv[0]));
-        tmem_ld64(tS + 64, *reinterpret_cast<uint32_t(*)[64]>(&sv[64]));
-        tmem_wait_ld();
         float *s = reinterpret_cast<float *>(sv);
-        // Masks.
         const int key0 = w.key0 + m * kTileKeys;
-        if (MODE == kQueryMajor) {
-          if (p.is_moba) {
-            if (key0 < cBr) {
-              // Window tail into an earlier block: keys i - j < window that the row's
-              // own selection does not already cover.  (block is a multiple of 128, so
-              // the chunk's keys all lie in one block.)
-              bool covered = false;
-              if (irow) {
-                const int blk = key0 / p.block;
-                for (int u2 = 0; u2 < p.topk; ++u2) covered |= (__ldg(irow + u2) == blk);
+        // S of the chunk into registers, masked.
+        auto load_s = [&]() {
+          tmem_ld64(tS, *reinterpret_cast<uint32_t(*)[64]>(&sv[0]));
+          tmem_ld64(tS + 64, *reinterpret_cast<uint32_t(*)[64]>(&sv[64]));
+          tmem_wait_ld();
+          if (MODE == kQueryMajor) {
+            if (p.is_moba) {
+              if (key0 < cBr) {
+                // Window tail into an earlier block: keys i - j < window that the row's
+                // own selection does not already cover.  (block is a multiple of 128,
+                // so the chunk's keys all lie in one block.)
+                bool covered = false;
+                if (irow) {
+                  const int blk = key0 / p.block;
+                  for (int u2 = 0; u2 < p.topk; ++u2) covered |= (__ldg(irow + u2) == blk);
+                }
+                const bool none = covered || !live || p.window <= 0;
+#pragma unroll
+                for (int e = 0; e < 128; ++e)
+                  if (none || pos - (key0 + e) >= p.window) s[e] = -INFINITY;
+              } else if (key0 + kTileKeys - 1 > pos) {
+#pragma unroll
+                for (int e = 0; e < 128; ++e)
+                  if (key0 + e > pos) s[e] = -INFINITY;
               }
-              const bool none = covered || !live || p.window <= 0;
+            } else {
+              const bool full = (key0 + kTileKeys - 1 <= a0) &&
+                                (key0 >= a0 + t.rows - 1 - p.window + 1);
+              if (!full) {
 #pragma unroll
-              for (int e = 0; e < 128; ++e)
-                if (none || pos - (key0 + e) >= p.window) s[e] = -INFINITY;
-            } else if (key0 + kTileKeys - 1 > pos) {
-#pragma unroll
-              for (int e = 0; e < 128; ++e)
-                if (key0 + e > pos) s[e] = -INFINITY;
-            }
-          } else {
-            const bool full = (key0 + kTileKeys - 1 <= a0) &&
-                              (key0 >= a0 + t.rows - 1 - p.window + 1);
-            if (!full) {
-#pragma unroll
-              for (int e = 0; e < 128; ++e) {
-                const int j = key0 + e;
-                if (j > pos || pos - j >= p.window) s[e] = -INFINITY;
+                for (int e = 0; e < 128; ++e) {
+                  const int j = key0 + e;
+                  if (j > pos || pos - j >= p.window) s[e] = -INFINITY;
+                }
               }
             }
           }
-        }
-        float mx8[8];
+        };
+        // The chunk's exact row maximum raises the running maximum when it grows by
+        // more than thr (always from -inf); l and O are rescaled by the same factor.
+        // S(m) complete implies P V of chunk m-1 complete: O is final for now.
+        auto raise_max = [&](float thr) {
+          float mx8[8];
 #pragma unroll
-        for (int u2 = 0; u2 < 8; ++u2) mx8[u2] = s[u2];
+          for (int u2 = 0; u2 < 8; ++u2) mx8[u2] = s[u2];
 #pragma unroll
-        for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[e]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        const float m_new = fmaxf(m_run, mx * sl2);
-        // Raise the running maximum only when it grows by more than 2^8 (or from
-        // -inf); rows that keep theirs multiply O by 1 when the warp rescales.
-        const bool raise = (m == 0) || (m_new > m_run + (float)kRescaleThreshold);
-        const bool scale_o = raise && m > 0 && m_run != -INFINITY;
-        const float alpha = scale_o ? ex2_approx(m_run - m_new) : 1.f;
-        if (raise) {
-          l_run *= alpha;
-          m_run = m_new;
-        }
-        if (__any_sync(FULL, scale_o)) {
-          // S(m) complete implies P V of chunk m-1 complete: O is final for now.
-#pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 16) {
-            uint32_t o[16];
-            tmem_ld16(tO + c0, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st16(tO + c0, o);
+          for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[e]);
+          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          const float m_new = fmaxf(m_run, mx * sl2);
+          const bool raise = (m_run == -INFINITY) || (m_new > m_run + thr);
+          const bool scale_o = raise && m_run != -INFINITY;
+          const float alpha = scale_o ? ex2_approx(m_run - m_new) : 1.f;
+          if (raise) {
+            l_run *= alpha;
+            m_run = m_new;
           }
-        }
-        if (turns) {
-          ok = mbar_wait(my_turn, tcnt & 1, abort, p.status, site0 + 15);
-          ++tcnt;
-          if (!(ok = __all_sync(FULL, ok))) break;
-        }
-        const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-        // Scale and row sums in packed pairs (eight running sums: four pairs).
-        float ls[8];
+          if (__any_sync(FULL, scale_o)) {
 #pragma unroll
-        for (int u2 = 0; u2 < 8; ++u2) ls[u2] = 0.f;
+            for (int c0 = 0; c0 < D; c0 += 16) {
+              uint32_t o[16];
+              tmem_ld16(tO + c0, o);
+              tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          float x0, x1;
-          fma_f32x2(x0, x1, s[2 * e], s[2 * e + 1], sl2, -mu);
-          const float p0 = ((2 * e) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x0) : ex2_in_order(x0);
-          const float p1 = ((2 * e + 1) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x1) : ex2_in_order(x1);
-          add_f32x2(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], p0, p1);
-          sv[e] = pack_bf16x2(p0, p1);
+              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st16(tO + c0, o);
+            }
+          }
+        };
+        // P = 2^(s * scale * log2 e - mu) packed to bf16 over the first 64 words of sv;
+        // returns the chunk's row sum.  Scale and sums in packed pairs (eight running
+        // sums: four pairs).
+        auto exps = [&]() -> float {
+          const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+          float ls[8];
+#pragma unroll
+          for (int u2 = 0; u2 < 8; ++u2) ls[u2] = 0.f;
+#pragma unroll
+          for (int e = 0; e < 64; ++e) {
+            float x0, x1;
+            fma_f32x2(x0, x1, s[2 * e], s[2 * e + 1], sl2, -mu);
+            const float p0 = ((2 * e) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x0) : ex2_in_order(x0);
+            const float p1 = ((2 * e + 1) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x1) : ex2_in_order(x1);
+            add_f32x2(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], p0, p1);
+            sv[e] = pack_bf16x2(p0, p1);
+          }
+          return ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        };
+        load_s();
+        float lsum;
+        if (MODE == kGathered) {
+          // The exact maximum is taken while some row of the warp has none yet; after
+          // that a chunk reuses the running maximum.  Its probabilities are then bounded
+          // by their sum, and the chunk is redone with its exact maximum only when that
+          // sum leaves the range that keeps P, l and O finite in fp32 and bf16 (S is
+          // still in TMEM: P is not stored yet).  This takes the row maximum off the
+          // chunk's critical path (measured 4-5% on the 1M-token pass).
+          if (__any_sync(FULL, m_run == -INFINITY)) raise_max((float)kRescaleThreshold);
+          if (turns) {
+            ok = mbar_wait(my_turn, tcnt & 1, abort, p.status, site0 + 15);
+            ++tcnt;
+            if (!(ok = __all_sync(FULL, ok))) break;
+          }
+          lsum = exps();
+          if (__any_sync(FULL, !(lsum <= kSumBound))) {
+            load_s();
+            raise_max(0.f);
+            lsum = exps();
+          }
+        } else {
+          // Query-major passes (own block, sliding window): the exact maximum of every
+          // chunk, raised lazily.
+          raise_max((float)kRescaleThreshold);
+          if (turns) {
+            ok = mbar_wait(my_turn, tcnt & 1, abort, p.status, site0 + 15);
+            ++tcnt;
+            if (!(ok = __all_sync(FULL, ok))) break;
+          }
+          lsum = exps();
         }
         __syncwarp();
         if (turns && lane == 0) mbar_arrive(other_turn);
         tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
         tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        l_run += lsum;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bar.p_full[x]);
