@@ -213,6 +213,36 @@ def test_moba_tied_blocks_keep_the_lower_block(name, kw):
     print(name, "checked", checked, "split pairs", split)
 
 
+def test_moba_score_jump_after_the_first_chunk():
+    """Past block 0's first 128 keys score about 0 against every later query row and its
+    other keys about 600 (raw dot product): in the gathered pass the first chunk sets the
+    row's running maximum, and the next chunk's probabilities against it would be about
+    2^76.  That chunk must be redone with its exact maximum (its row sum leaves the bound
+    the pass accepts), so the output and lse still match the fp64 oracle."""
+    moba = _moba()
+    w = workloads.small_moba(name="score_jump", batch=1, hq=2, hkv=1, seqlen=2048, d=128,
+                             block=512, topk=2)
+    q, k, v = workloads.make_inputs(w, 11)
+    u = torch.ones(w.d) / w.d ** 0.5
+    kf = 0.05 * k.float()
+    kf[0, 0, 128:512] += 24.0 * u
+    qf = 0.05 * q.float()
+    qf[0, :, 512:] += 25.0 * u
+    q, k = qf.to(torch.bfloat16), kf.to(torch.bfloat16)
+    runner = moba.MobaPrefill(w.batch, w.hq, w.hkv, w.seqlen, w.d, w.block, w.topk, w.window)
+    out, lse = runner(q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    assert moba.device_status() == 0
+    rows = np.arange(w.seqlen, dtype=np.int32)
+    idx_g = rows_of(runner.idx, rows)
+    assert np.all(idx_g[0, :, 512:, 0] == 0)   # every later row picks block 0
+    out_o, lse_o = oracle.attention(q, k, v, mode=oracle.MODE_MOBA, block=w.block, topk=w.topk,
+                                    idx=idx_g, window=w.window, rows=rows)
+    assert lse_o[0, :, 512:].min() > 40.0     # the jump really dominates those rows
+    stats = check_out(rows_of(out, rows), rows_of(lse, rows), out_o, lse_o)
+    print("score jump", stats)
+
+
 @pytest.mark.parametrize("batch,hq,hkv,groups", [(1, 8, 4, 4), (2, 4, 2, 2), (1, 2, 1, 1)])
 def test_host_pipeline_equals_device_path(batch, hq, hkv, groups):
     """MobaPrefillHost (pinned host buffers, KV-head groups pipelined over three streams)
