@@ -649,97 +649,97 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         uint32_t sv[128];
         float *s = reinterpret_cast<float *>(sv);
         const int key0 = w.key0 + m * kTileKeys;
-        // S of the chunk into registers, masked.
-        auto load_s = [&]() {
-          tmem_ld64(tS, *reinterpret_cast<uint32_t(*)[64]>(&sv[0]));
-          tmem_ld64(tS + 64, *reinterpret_cast<uint32_t(*)[64]>(&sv[64]));
-          tmem_wait_ld();
-          if (MODE == kQueryMajor) {
-            if (p.is_moba) {
-              if (key0 < cBr) {
-                // Window tail into an earlier block: keys i - j < window that the row's
-                // own selection does not already cover.  (block is a multiple of 128,
-                // so the chunk's keys all lie in one block.)
-                bool covered = false;
-                if (irow) {
-                  const int blk = key0 / p.block;
-                  for (int u2 = 0; u2 < p.topk; ++u2) covered |= (__ldg(irow + u2) == blk);
-                }
-                const bool none = covered || !live || p.window <= 0;
-#pragma unroll
-                for (int e = 0; e < 128; ++e)
-                  if (none || pos - (key0 + e) >= p.window) s[e] = -INFINITY;
-              } else if (key0 + kTileKeys - 1 > pos) {
-#pragma unroll
-                for (int e = 0; e < 128; ++e)
-                  if (key0 + e > pos) s[e] = -INFINITY;
-              }
-            } else {
-              const bool full = (key0 + kTileKeys - 1 <= a0) &&
-                                (key0 >= a0 + t.rows - 1 - p.window + 1);
-              if (!full) {
-#pragma unroll
-                for (int e = 0; e < 128; ++e) {
-                  const int j = key0 + e;
-                  if (j > pos || pos - j >= p.window) s[e] = -INFINITY;
-                }
-              }
-            }
-          }
-        };
-        // The chunk's exact row maximum raises the running maximum when it grows by
-        // more than thr (always from -inf); l and O are rescaled by the same factor.
-        // S(m) complete implies P V of chunk m-1 complete: O is final for now.
-        auto raise_max = [&](float thr) {
-          float mx8[8];
-#pragma unroll
-          for (int u2 = 0; u2 < 8; ++u2) mx8[u2] = s[u2];
-#pragma unroll
-          for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[e]);
-          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-          const float m_new = fmaxf(m_run, mx * sl2);
-          const bool raise = (m_run == -INFINITY) || (m_new > m_run + thr);
-          const bool scale_o = raise && m_run != -INFINITY;
-          const float alpha = scale_o ? ex2_approx(m_run - m_new) : 1.f;
-          if (raise) {
-            l_run *= alpha;
-            m_run = m_new;
-          }
-          if (__any_sync(FULL, scale_o)) {
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 16) {
-              uint32_t o[16];
-              tmem_ld16(tO + c0, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st16(tO + c0, o);
-            }
-          }
-        };
-        // P = 2^(s * scale * log2 e - mu) packed to bf16 over the first 64 words of sv;
-        // returns the chunk's row sum.  Scale and sums in packed pairs (eight running
-        // sums: four pairs).
-        auto exps = [&]() -> float {
-          const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-          float ls[8];
-#pragma unroll
-          for (int u2 = 0; u2 < 8; ++u2) ls[u2] = 0.f;
-#pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            float x0, x1;
-            fma_f32x2(x0, x1, s[2 * e], s[2 * e + 1], sl2, -mu);
-            const float p0 = ((2 * e) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x0) : ex2_in_order(x0);
-            const float p1 = ((2 * e + 1) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x1) : ex2_in_order(x1);
-            add_f32x2(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], p0, p1);
-            sv[e] = pack_bf16x2(p0, p1);
-          }
-          return ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-        };
-        load_s();
         float lsum;
-        if (MODE == kGathered) {
+        if constexpr (MODE == kGathered) {
+          // S of the chunk into registers, masked.
+          auto load_s = [&]() {
+            tmem_ld64(tS, *reinterpret_cast<uint32_t(*)[64]>(&sv[0]));
+            tmem_ld64(tS + 64, *reinterpret_cast<uint32_t(*)[64]>(&sv[64]));
+            tmem_wait_ld();
+            if (MODE == kQueryMajor) {
+              if (p.is_moba) {
+                if (key0 < cBr) {
+                  // Window tail into an earlier block: keys i - j < window that the row's
+                  // own selection does not already cover.  (block is a multiple of 128,
+                  // so the chunk's keys all lie in one block.)
+                  bool covered = false;
+                  if (irow) {
+                    const int blk = key0 / p.block;
+                    for (int u2 = 0; u2 < p.topk; ++u2) covered |= (__ldg(irow + u2) == blk);
+                  }
+                  const bool none = covered || !live || p.window <= 0;
+  #pragma unroll
+                  for (int e = 0; e < 128; ++e)
+                    if (none || pos - (key0 + e) >= p.window) s[e] = -INFINITY;
+                } else if (key0 + kTileKeys - 1 > pos) {
+  #pragma unroll
+                  for (int e = 0; e < 128; ++e)
+                    if (key0 + e > pos) s[e] = -INFINITY;
+                }
+              } else {
+                const bool full = (key0 + kTileKeys - 1 <= a0) &&
+                                  (key0 >= a0 + t.rows - 1 - p.window + 1);
+                if (!full) {
+  #pragma unroll
+                  for (int e = 0; e < 128; ++e) {
+                    const int j = key0 + e;
+                    if (j > pos || pos - j >= p.window) s[e] = -INFINITY;
+                  }
+                }
+              }
+            }
+          };
+          // The chunk's exact row maximum raises the running maximum when it grows by
+          // more than thr (always from -inf); l and O are rescaled by the same factor.
+          // S(m) complete implies P V of chunk m-1 complete: O is final for now.
+          auto raise_max = [&](float thr) {
+            float mx8[8];
+  #pragma unroll
+            for (int u2 = 0; u2 < 8; ++u2) mx8[u2] = s[u2];
+  #pragma unroll
+            for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[e]);
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            const float m_new = fmaxf(m_run, mx * sl2);
+            const bool raise = (m_run == -INFINITY) || (m_new > m_run + thr);
+            const bool scale_o = raise && m_run != -INFINITY;
+            const float alpha = scale_o ? ex2_approx(m_run - m_new) : 1.f;
+            if (raise) {
+              l_run *= alpha;
+              m_run = m_new;
+            }
+            if (__any_sync(FULL, scale_o)) {
+  #pragma unroll
+              for (int c0 = 0; c0 < D; c0 += 16) {
+                uint32_t o[16];
+                tmem_ld16(tO + c0, o);
+                tmem_wait_ld();
+  #pragma unroll
+                for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                tmem_st16(tO + c0, o);
+              }
+            }
+          };
+          // P = 2^(s * scale * log2 e - mu) packed to bf16 over the first 64 words of sv;
+          // returns the chunk's row sum.  Scale and sums in packed pairs (eight running
+          // sums: four pairs).
+          auto exps = [&]() -> float {
+            const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+            float ls[8];
+  #pragma unroll
+            for (int u2 = 0; u2 < 8; ++u2) ls[u2] = 0.f;
+  #pragma unroll
+            for (int e = 0; e < 64; ++e) {
+              float x0, x1;
+              fma_f32x2(x0, x1, s[2 * e], s[2 * e + 1], sl2, -mu);
+              const float p0 = ((2 * e) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x0) : ex2_in_order(x0);
+              const float p1 = ((2 * e + 1) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x1) : ex2_in_order(x1);
+              add_f32x2(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], p0, p1);
+              sv[e] = pack_bf16x2(p0, p1);
+            }
+            return ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+          };
+          load_s();
           // The exact maximum is taken while some row of the warp has none yet; after
           // that a chunk reuses the running maximum.  Its probabilities are then bounded
           // by their sum, and the chunk is redone with its exact maximum only when that
@@ -761,13 +761,91 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         } else {
           // Query-major passes (own block, sliding window): the exact maximum of every
           // chunk, raised lazily.
-          raise_max((float)kRescaleThreshold);
+          tmem_ld64(tS, *reinterpret_cast<uint32_t(*)[64]>(&sv[0]));
+          tmem_ld64(tS + 64, *reinterpret_cast<uint32_t(*)[64]>(&sv[64]));
+          tmem_wait_ld();
+          // Masks.
+          if (MODE == kQueryMajor) {
+            if (p.is_moba) {
+              if (key0 < cBr) {
+                // Window tail into an earlier block: keys i - j < window that the row's
+                // own selection does not already cover.  (block is a multiple of 128, so
+                // the chunk's keys all lie in one block.)
+                bool covered = false;
+                if (irow) {
+                  const int blk = key0 / p.block;
+                  for (int u2 = 0; u2 < p.topk; ++u2) covered |= (__ldg(irow + u2) == blk);
+                }
+                const bool none = covered || !live || p.window <= 0;
+  #pragma unroll
+                for (int e = 0; e < 128; ++e)
+                  if (none || pos - (key0 + e) >= p.window) s[e] = -INFINITY;
+              } else if (key0 + kTileKeys - 1 > pos) {
+  #pragma unroll
+                for (int e = 0; e < 128; ++e)
+                  if (key0 + e > pos) s[e] = -INFINITY;
+              }
+            } else {
+              const bool full = (key0 + kTileKeys - 1 <= a0) &&
+                                (key0 >= a0 + t.rows - 1 - p.window + 1);
+              if (!full) {
+  #pragma unroll
+                for (int e = 0; e < 128; ++e) {
+                  const int j = key0 + e;
+                  if (j > pos || pos - j >= p.window) s[e] = -INFINITY;
+                }
+              }
+            }
+          }
+          float mx8[8];
+  #pragma unroll
+          for (int u2 = 0; u2 < 8; ++u2) mx8[u2] = s[u2];
+  #pragma unroll
+          for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[e]);
+          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          const float m_new = fmaxf(m_run, mx * sl2);
+          // Raise the running maximum only when it grows by more than 2^8 (or from
+          // -inf); rows that keep theirs multiply O by 1 when the warp rescales.
+          const bool raise = (m == 0) || (m_new > m_run + (float)kRescaleThreshold);
+          const bool scale_o = raise && m > 0 && m_run != -INFINITY;
+          const float alpha = scale_o ? ex2_approx(m_run - m_new) : 1.f;
+          if (raise) {
+            l_run *= alpha;
+            m_run = m_new;
+          }
+          if (__any_sync(FULL, scale_o)) {
+            // S(m) complete implies P V of chunk m-1 complete: O is final for now.
+  #pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 16) {
+              uint32_t o[16];
+              tmem_ld16(tO + c0, o);
+              tmem_wait_ld();
+  #pragma unroll
+              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st16(tO + c0, o);
+            }
+          }
           if (turns) {
             ok = mbar_wait(my_turn, tcnt & 1, abort, p.status, site0 + 15);
             ++tcnt;
             if (!(ok = __all_sync(FULL, ok))) break;
           }
-          lsum = exps();
+          const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+          // Scale and row sums in packed pairs (eight running sums: four pairs).
+          float ls[8];
+  #pragma unroll
+          for (int u2 = 0; u2 < 8; ++u2) ls[u2] = 0.f;
+  #pragma unroll
+          for (int e = 0; e < 64; ++e) {
+            float x0, x1;
+            fma_f32x2(x0, x1, s[2 * e], s[2 * e + 1], sl2, -mu);
+            const float p0 = ((2 * e) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x0) : ex2_in_order(x0);
+            const float p1 = ((2 * e + 1) % 16 >= 16 - kExpEmuPer16) ? exp2_fma(x1) : ex2_in_order(x1);
+            add_f32x2(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], p0, p1);
+            sv[e] = pack_bf16x2(p0, p1);
+          }
+          lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         }
         __syncwarp();
         if (turns && lane == 0) mbar_arrive(other_turn);
