@@ -164,7 +164,7 @@ struct RowSrc {
 };
 
 __device__ __forceinline__ void decode_rows(const BwdParams &p, const BwdRows &t, int b, int hk,
-                                            int gt, RowSrc *tab, GatherRows &gr) {
+                                            int gt, RowSrc *tab, GatherRows &gr, bool prefetch = false) {
   const int w = gt >> 5, l = gt & 31;
 #pragma unroll
   for (int x = 0; x < 2; ++x) {
@@ -176,6 +176,12 @@ __device__ __forceinline__ void decode_rows(const BwdParams &p, const BwdRows &t
     RowSrc src;
     src.q = gr.valid[x] ? p.q + bb * p.q_sb + (int64_t)h * p.q_sh + (int64_t)i * p.q_sn : nullptr;
     src.g = gr.valid[x] ? p.dout + bb * p.do_sb + (int64_t)h * p.do_sh + (int64_t)i * p.do_sn : nullptr;
+    // (dQ pass) The rows go into L2 now: their copies wait for the current tile to
+    // release the buffer, and then read L2 instead of DRAM.
+    if (prefetch && gr.valid[x]) {
+      prefetch_l2_bulk(src.q, (uint32_t)p.d * 2u);
+      prefetch_l2_bulk(src.g, (uint32_t)p.d * 2u);
+    }
     tab[r] = src;
     gr.st[x] = p.rowstat + ((int64_t)bb * p.hq + h) * p.N + i;
   }
@@ -283,7 +289,8 @@ struct DqCfg {
   static constexpr int V_OFF = K_OFF + ST * BwdTile<D>::TILE;
   static constexpr int ST_OFF = V_OFF + ST * BwdTile<D>::TILE;   // float2 stats [128]
   static constexpr int TAB_OFF = ST_OFF + 128 * 8;                 // RowSrc [128]
-  static constexpr int BAR_OFF = TAB_OFF + 128 * 16;
+  static constexpr int STG_OFF = TAB_OFF + 128 * 16;              // 8 warps x 32 rows x 64 B
+  static constexpr int BAR_OFF = STG_OFF + 8 * 2048;
   static constexpr int SMEM = BAR_OFF + 1024 + 1024;
 };
 
@@ -462,7 +469,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
       issue_rows<D>(p, gr, tab, base + C::Q_OFF, base + C::DO_OFF, stats, gt);
       land_tile(&bar.q_full[0]);
       u = next_item(u + gridDim.x, it);
-      if (u < nitems) decode_rows(p, it.t, it.b, it.hk, gt, tab, gr);
+      if (u < nitems) decode_rows(p, it.t, it.b, it.hk, gt, tab, gr, true);
     }
     cp_async_wait_all();
   } else {
@@ -525,18 +532,37 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
       ++an;
       tc_fence_after();
       float *dst = p.dqp + ((((int64_t)it.b * p.hq + h) * p.N + i) * p.topk + slot) * D;
+      // The fp32 partials go out through a per-warp staging buffer (32 rows x 16 columns,
+      // 16-byte chunks XOR-swizzled by row pair): lane r writes its row's 64 bytes, then
+      // each store instruction writes eight whole 64-byte row segments (coalesced).
+      unsigned char *stg = sbase + C::STG_OFF + (warp - 4) * 2048;
+      float *rdst[4];
+      bool rlive[4];
 #pragma unroll
-      for (int c0 = grp * (D / 2); c0 < (grp + 1) * (D / 2); c0 += 32) {
-        uint32_t o[32];
-        tmem_ld32(tQ + c0, o);
+      for (int jj = 0; jj < 4; ++jj) {
+        const int src = jj * 8 + (lane >> 2);
+        rdst[jj] = reinterpret_cast<float *>(__shfl_sync(FULL, reinterpret_cast<uintptr_t>(dst), src));
+        rlive[jj] = __shfl_sync(FULL, live ? 1 : 0, src) != 0;
+      }
+#pragma unroll
+      for (int c0 = grp * (D / 2); c0 < (grp + 1) * (D / 2); c0 += 16) {
+        uint32_t o[16];
+        tmem_ld16(tQ + c0, o);
         tmem_wait_ld();
-        if (live) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4 *>(dst + c0 + e) =
-                make_float4(__uint_as_float(o[e]), __uint_as_float(o[e + 1]),
-                            __uint_as_float(o[e + 2]), __uint_as_float(o[e + 3]));
+        for (int v4 = 0; v4 < 4; ++v4)
+          *reinterpret_cast<uint4 *>(stg + lane * 64 + ((v4 ^ ((lane >> 1) & 3)) << 4)) =
+              make_uint4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int row = jj * 8 + (lane >> 2), ch = lane & 3;
+          if (rlive[jj]) {
+            const uint4 q = *reinterpret_cast<const uint4 *>(stg + row * 64 + ((ch ^ ((row >> 1) & 3)) << 4));
+            *reinterpret_cast<uint4 *>(rdst[jj] + c0 + ch * 4) = q;
+          }
         }
+        __syncwarp();
       }
       tc_fence_before();
       mbar_arrive(&bar.acc_empty);
