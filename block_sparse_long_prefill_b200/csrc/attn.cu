@@ -651,43 +651,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int key0 = w.key0 + m * kTileKeys;
         float lsum;
         if constexpr (MODE == kGathered) {
-          // S of the chunk into registers, masked.
+          // S of the chunk into registers (the gathered pass has no masks).
           auto load_s = [&]() {
             tmem_ld64(tS, *reinterpret_cast<uint32_t(*)[64]>(&sv[0]));
             tmem_ld64(tS + 64, *reinterpret_cast<uint32_t(*)[64]>(&sv[64]));
             tmem_wait_ld();
-            if (MODE == kQueryMajor) {
-              if (p.is_moba) {
-                if (key0 < cBr) {
-                  // Window tail into an earlier block: keys i - j < window that the row's
-                  // own selection does not already cover.  (block is a multiple of 128,
-                  // so the chunk's keys all lie in one block.)
-                  bool covered = false;
-                  if (irow) {
-                    const int blk = key0 / p.block;
-                    for (int u2 = 0; u2 < p.topk; ++u2) covered |= (__ldg(irow + u2) == blk);
-                  }
-                  const bool none = covered || !live || p.window <= 0;
-  #pragma unroll
-                  for (int e = 0; e < 128; ++e)
-                    if (none || pos - (key0 + e) >= p.window) s[e] = -INFINITY;
-                } else if (key0 + kTileKeys - 1 > pos) {
-  #pragma unroll
-                  for (int e = 0; e < 128; ++e)
-                    if (key0 + e > pos) s[e] = -INFINITY;
-                }
-              } else {
-                const bool full = (key0 + kTileKeys - 1 <= a0) &&
-                                  (key0 >= a0 + t.rows - 1 - p.window + 1);
-                if (!full) {
-  #pragma unroll
-                  for (int e = 0; e < 128; ++e) {
-                    const int j = key0 + e;
-                    if (j > pos || pos - j >= p.window) s[e] = -INFINITY;
-                  }
-                }
-              }
-            }
           };
           // The chunk's exact row maximum raises the running maximum when it grows by
           // more than thr (always from -inf); l and O are rescaled by the same factor.
